@@ -1,0 +1,7 @@
+"""fp64 CPU oracle of the recurrent-depth block (test infrastructure only; see rdt_oracle)."""
+from .rdt_oracle import *  # noqa: F401,F403
+from .rdt_oracle import (rmsnorm, rope_angles, apply_rope, silu, swiglu_ffn, causal_attention,
+                         gqa_attention, router_topk, moe_combine, attention_sublayer,
+                         moe_sublayer, loop_forward, loop_step_rows, input_injection,
+                         spectral_radius, mla_attention_explicit, mla_attention_absorbed,
+                         LoopTrace, Routing, NEAR_TIE)
