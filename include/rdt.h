@@ -1,0 +1,218 @@
+/*
+ * rdt.h - C ABI of the B200 (sm_100a) recurrent-depth block library, librdt.so.
+ *
+ * The library runs the looped recurrent block of a recurrent-depth transformer:
+ *
+ *     h_{t+1} = A (.) h_t + B.e + Block(h_t, e),      t = 0 .. T-1,
+ *
+ * (update equation of the techbriefly article on the OpenMythos project:
+ * "h_{t+1} = A.h_t + B.e + Transformer(h_t, e)", with e the prelude encoding
+ * re-injected every loop and rho(A) < 1). Block is a pre-RMSNorm causal
+ * attention sublayer (GQA, or MLA with a latent KV) followed by a top-k sparse
+ * mixture of SwiGLU experts, with optional per-loop (depth-wise) LoRA on the Q
+ * and O projections (getting-started page "Introducao ao OpenMythos",
+ * Passo 2 and Passo 5; techbriefly article, MoE and LoRA paragraphs).
+ *
+ * Readings fixed by this library where the pages are silent:
+ *   x = h + e (inject_e = 1) or x = h;  a = Attn(RMSNorm1(x));  y = x + a;
+ *   f = MoE(RMSNorm2(y));  Block(h, e) = a + f  (the residual increment).
+ *   A is diagonal (fp32 [dim]); B is diagonal [dim] or dense [dim, dim] (fp32).
+ *
+ * Conventions for every call:
+ *   - Pointers named *device* are CUDA device pointers on the current device;
+ *     *host* pointers are ordinary host memory. Tensors are row-major and
+ *     token-major: a [N, dim] tensor holds token n = b * seq + s in row n.
+ *     Every device tensor must be 16-byte aligned (RDT_ERR_MISALIGNED).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls enqueue work and return without synchronising, except where noted;
+ *     caller buffers must stay valid until that work has completed.
+ *   - Arguments are validated before anything is enqueued; a non-OK status
+ *     means nothing was launched (except RDT_ERR_CUDA, raised by a failing
+ *     CUDA call). rdt_last_error() gives the message of the calling thread's
+ *     last failure.
+ *   - A handle must not be used from two host threads or two streams at once:
+ *     its workspace is shared by all its calls.
+ */
+#ifndef RDT_H
+#define RDT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RDT_OK = 0,
+    RDT_ERR_INVALID_ARG = 1,    /* null pointer, size or loop count out of range      */
+    RDT_ERR_UNSUPPORTED = 2,    /* no sm_100 device, or a shape the kernels do not tile */
+    RDT_ERR_MISALIGNED = 3,     /* a tensor pointer not 16-byte aligned                 */
+    RDT_ERR_UNSTABLE_A = 4,     /* rho(A) = max |A_i| >= 1 at create                    */
+    RDT_ERR_OOM = 5,            /* device allocation failed                             */
+    RDT_ERR_CUDA = 6,           /* a CUDA runtime or driver call failed                 */
+    RDT_ERR_DEVICE_TIMEOUT = 7, /* a bounded device-side wait gave up (diagnostics)     */
+    RDT_ERR_NONFINITE = 8       /* a NaN or Inf reached the state (diagnostics)          */
+} rdt_status;
+
+enum { RDT_F32 = 0, RDT_BF16 = 1 };        /* rdt_config.dtype        */
+enum { RDT_GQA = 0, RDT_MLA = 1 };         /* rdt_config.attn_type    */
+enum { RDT_B_DIAG = 0, RDT_B_DENSE = 1 };  /* rdt_config.b_kind       */
+
+/* Block hyper-parameters (the block-level fields of MythosConfig, getting-started
+ * page Passo 2 and Passo 5). `batch` and `seq` are the sizes every forward call
+ * uses; the workspace is allocated for them at create.
+ * Tiling limits checked at create (RDT_ERR_UNSUPPORTED otherwise): dim = 128 * 2^k
+ * <= 4096; GQA head_dim 64 (bf16) or 32 / 64 (fp32), n_heads % n_kv_heads == 0,
+ * n_heads * head_dim % 128 == 0; expert_hidden % 64 == 0 (fp32: % 128);
+ * n_experts + n_shared <= 256; top_k <= min(n_experts, 16); LoRA on GQA only with
+ * lora_rank <= 64 (bf16) / 32 (fp32); MLA in bf16 only with kv_lora_rank 128,
+ * qk_rope_dim 32, q_lora_rank % 64 == 0, v_head_dim % 32 == 0. */
+typedef struct {
+    int32_t dtype;                  /* RDT_F32 or RDT_BF16: storage of h0, e, weights   */
+    int32_t batch, seq, dim;
+    int32_t attn_type;              /* RDT_GQA or RDT_MLA                               */
+    int32_t n_heads, n_kv_heads, head_dim;                            /* GQA           */
+    int32_t q_lora_rank, kv_lora_rank, qk_nope_dim, qk_rope_dim, v_head_dim; /* MLA    */
+    float rope_base;                /* RoPE base (1e4)                                  */
+    float norm_eps;                 /* RMSNorm epsilon (1e-6)                           */
+    int32_t n_experts, top_k, n_shared, expert_hidden;
+    int32_t lora_rank, n_lora;      /* depth-wise LoRA on Q and O; n_lora = 0: none     */
+    int32_t b_kind;                 /* RDT_B_DIAG or RDT_B_DENSE                        */
+    int32_t inject_e;               /* 1: block input x = h + e; 0: x = h               */
+    int32_t max_loops;              /* largest T accepted (<= 64; the pages loop <= 16) */
+} rdt_config;
+
+/* Weights, all DEVICE pointers, row-major [out, in]; element type = cfg.dtype
+ * unless marked fp32. rdt_create copies and repacks them into library-owned
+ * memory, so the caller may free them once rdt_create has returned.
+ * Fields a configuration does not use must be NULL. */
+typedef struct {
+    const float* A;            /* [dim] fp32, diagonal of A; rho(A) < 1 required         */
+    const float* B;            /* [dim] (RDT_B_DIAG) or [dim, dim] (RDT_B_DENSE), fp32   */
+    const float* norm1;        /* [dim] fp32 RMSNorm gain before attention               */
+    const float* norm2;        /* [dim] fp32 RMSNorm gain before the MoE                 */
+    /* GQA */
+    const void* wq;            /* [n_heads * head_dim, dim]                              */
+    const void* wk;            /* [n_kv_heads * head_dim, dim]                           */
+    const void* wv;            /* [n_kv_heads * head_dim, dim]                           */
+    const void* wo;            /* [dim, n_heads * head_dim] (MLA: [dim, n_heads * v_head_dim]) */
+    /* MLA */
+    const void* w_dq;          /* [q_lora_rank, dim]                                     */
+    const float* q_norm;       /* [q_lora_rank] fp32                                     */
+    const void* w_uq;          /* [n_heads * (qk_nope_dim + qk_rope_dim), q_lora_rank]   */
+    const void* w_dkv;         /* [kv_lora_rank, dim]                                    */
+    const float* kv_norm;      /* [kv_lora_rank] fp32                                    */
+    const void* w_kr;          /* [qk_rope_dim, dim]                                     */
+    const void* w_uk;          /* [n_heads * qk_nope_dim, kv_lora_rank]                  */
+    const void* w_uv;          /* [n_heads * v_head_dim, kv_lora_rank]                   */
+    /* MoE */
+    const void* w_router;      /* [n_experts, dim]                                       */
+    const float* router_bias;  /* [n_experts] fp32 or NULL: added for selection only     */
+    const void* w1;            /* [n_experts, expert_hidden, dim] (gate)                 */
+    const void* w3;            /* [n_experts, expert_hidden, dim] (up)                   */
+    const void* w2;            /* [n_experts, dim, expert_hidden] (down)                 */
+    const void* ws1;           /* [n_shared, expert_hidden, dim] or NULL                 */
+    const void* ws3;           /* [n_shared, expert_hidden, dim] or NULL                 */
+    const void* ws2;           /* [n_shared, dim, expert_hidden] or NULL                 */
+    /* depth-wise LoRA (GQA): W_t = W + B_t A_t, adapter min(t, n_lora - 1) at loop t */
+    const void* lq_a;          /* [n_lora, lora_rank, dim]                               */
+    const void* lq_b;          /* [n_lora, n_heads * head_dim, lora_rank]                */
+    const void* lo_a;          /* [n_lora, lora_rank, n_heads * head_dim]                */
+    const void* lo_b;          /* [n_lora, dim, lora_rank]                               */
+} rdt_weights;
+
+typedef struct rdt_handle rdt_handle;
+
+typedef struct {
+    float rho_A;                   /* max |A_i| of the weights given at create             */
+    int32_t nonfinite;             /* 1 if a non-finite value reached the state            */
+    int32_t timeout;               /* 1 if a bounded device wait gave up                   */
+    int32_t last_routed_rows;      /* sum of the per-expert counts of the last MoE         */
+    int32_t expert_counts[256];    /* tokens per expert in the last MoE (routed, then shared) */
+} rdt_diag;
+
+/* Validates cfg and weights, allocates the workspace for cfg.batch * cfg.seq
+ * tokens, copies and repacks the weights (on `stream`, then synchronises it) and
+ * returns a handle in *out. Errors: INVALID_ARG (bad sizes or NULL weights),
+ * UNSUPPORTED (not an sm_100 device, or a shape outside the tiling limits),
+ * UNSTABLE_A (max |A_i| >= 1: the parameterisation, not a clip, must keep
+ * rho(A) < 1 - getting-started page, Passo 6 and troubleshooting item 3), OOM, CUDA. */
+rdt_status rdt_create(const rdt_config* cfg, const rdt_weights* w, void* stream,
+                      rdt_handle** out);
+
+/* Attention sublayer alone: a = Attn(RMSNorm1(x)) including the output
+ * projection and the LoRA adapter of loop `loop` (ignored without LoRA).
+ *   x     : device fp32 [N, dim] block input (N = batch * seq)
+ *   a_out : device fp32 [N, dim]                                              */
+rdt_status rdt_attn_forward(rdt_handle* h, const float* x, int loop, float* a_out,
+                            void* stream);
+
+/* MoE sublayer alone: f = MoE(RMSNorm2(y)), routed top-k experts weighted by the
+ * softmax of their logits renormalised over the k chosen, plus every shared
+ * expert with weight 1.
+ *   y        : device fp32 [N, dim]
+ *   f_out    : device fp32 [N, dim]
+ *   topk_idx : device int32 [N, top_k] or NULL: chosen experts, by (logit + bias)
+ *              descending, ties to the lower index
+ *   topk_w   : device fp32 [N, top_k] or NULL: their gate weights             */
+rdt_status rdt_moe_forward(rdt_handle* h, const float* y, float* f_out, int32_t* topk_idx,
+                           float* topk_w, void* stream);
+
+/* The looped block: out = h_T after T loops of the update equation.
+ *   h0, e : device [N, dim] in cfg.dtype (h0 may alias e)
+ *   T     : 1 .. cfg.max_loops (INVALID_ARG otherwise)
+ *   out   : device fp32 [N, dim]; the state is kept in fp32 throughout        */
+rdt_status rdt_loop_forward(rdt_handle* h, const void* h0, const void* e, int T, float* out,
+                            void* stream);
+
+/* The same call for callers holding HOST buffers: copies h0 and e (cfg.dtype,
+ * [N, dim]) to the device, runs rdt_loop_forward, copies h_T (fp32 [N, dim])
+ * back to `out_host` and synchronises `stream` before returning. Page-locked
+ * host memory gives asynchronous copies; pageable memory also works. */
+rdt_status rdt_loop_forward_host(rdt_handle* h, const void* h0_host, const void* e_host, int T,
+                                 float* out_host, void* stream);
+
+/* Per-loop trace for parity checks (all device pointers, or NULL to disable):
+ *   idx    : int32 [max_loops, N, top_k] routing of every loop
+ *   w      : fp32  [max_loops, N, top_k] gate weights of every loop
+ *   h_traj : fp32  [max_loops + 1, N, dim] the state h_0 .. h_T
+ * Later rdt_loop_forward calls write loop t at offset t. Pass all NULL to stop. */
+rdt_status rdt_set_trace(rdt_handle* h, int32_t* idx, float* w, float* h_traj);
+
+/* Synchronises the handle's last stream and fills *out (see rdt_diag). */
+rdt_status rdt_get_diagnostics(rdt_handle* h, rdt_diag* out);
+
+/* Bytes of device memory the handle owns (weights + workspace). */
+rdt_status rdt_memory_bytes(const rdt_handle* h, size_t* bytes);
+
+/* ---- kernel-level calls: the tensor-core GEMM and the attention kernel alone, on
+ * caller buffers (unit parity and per-kernel measurement). */
+
+/* C = A B^T on the 5th-generation tensor cores (bf16 operands, or fp32 operands read as
+ * tf32), fp32 accumulation and output.
+ *   dtype : RDT_BF16 or RDT_F32, element type of A and B
+ *   A     : device [M, K] row-major;  B : device [N, K] row-major;  C : device fp32 [M, N]
+ * Limits: K * element size a multiple of 128 bytes; N a multiple of 32; M >= 1. */
+rdt_status rdt_matmul(int32_t dtype, const void* A, const void* B, float* C, int M, int N, int K,
+                      void* stream);
+
+/* Causal attention o = softmax(q k^T * scale, keys after the query masked) v per sequence
+ * and query head; query head h reads KV head floor(h * n_kv_heads / n_heads).
+ *   q : device [batch * seq, n_heads * dqk]    k : device [batch * seq, n_kv_heads * dqk]
+ *   v : device [batch * seq, n_kv_heads * dv]  o : device [batch * seq, n_heads * dv]
+ * bf16: (dqk, dv) = (64, 64) or (160, 128); fp32: (32, 32) or (64, 64). */
+rdt_status rdt_attention(int32_t dtype, const void* q, const void* k, const void* v, void* o,
+                         int batch, int seq, int n_heads, int n_kv_heads, int dqk, int dv,
+                         float scale, void* stream);
+
+const char* rdt_status_string(rdt_status s);
+const char* rdt_last_error(void);
+
+/* Frees everything the handle owns (after synchronising the device). NULL is a no-op. */
+void rdt_destroy(rdt_handle* h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RDT_H */

@@ -1,0 +1,266 @@
+"""Python binding of librdt, the B200 (sm_100a) recurrent-depth block library.
+
+Argument marshalling only: every step of the forward pass runs in the CUDA kernels of
+``librdt.so`` behind the C ABI of ``include/rdt.h``. PyTorch provides device memory and
+streams. There is no CPU path: without the built library (or a CUDA device) the calls
+raise.
+
+    from recurrent_depth_transformer_b200 import RDT
+    m = RDT(config, weights)             # weights: dict name -> CUDA tensor
+    out = m.loop_forward(h0, e, T)       # fp32 [batch, seq, dim] = h_T
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import numpy as np
+
+__all__ = ["RDT", "RdtError", "library_path", "load_library", "make_config", "device_weights",
+           "EXPORTED"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG, "librdt.so")
+
+RDT_F32, RDT_BF16 = 0, 1
+RDT_GQA, RDT_MLA = 0, 1
+RDT_B_DIAG, RDT_B_DENSE = 0, 1
+
+STATUS = {0: "RDT_OK", 1: "RDT_ERR_INVALID_ARG", 2: "RDT_ERR_UNSUPPORTED", 3: "RDT_ERR_MISALIGNED",
+          4: "RDT_ERR_UNSTABLE_A", 5: "RDT_ERR_OOM", 6: "RDT_ERR_CUDA", 7: "RDT_ERR_DEVICE_TIMEOUT",
+          8: "RDT_ERR_NONFINITE"}
+
+EXPORTED = ("rdt_create", "rdt_attn_forward", "rdt_moe_forward", "rdt_loop_forward",
+            "rdt_loop_forward_host", "rdt_set_trace", "rdt_get_diagnostics", "rdt_memory_bytes",
+            "rdt_status_string", "rdt_last_error", "rdt_destroy", "rdt_matmul", "rdt_attention")
+
+
+class RdtError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class RdtConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "dtype", "batch", "seq", "dim", "attn_type", "n_heads", "n_kv_heads", "head_dim",
+        "q_lora_rank", "kv_lora_rank", "qk_nope_dim", "qk_rope_dim", "v_head_dim")] + [
+        ("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float)] + [
+        (n, ctypes.c_int32) for n in ("n_experts", "top_k", "n_shared", "expert_hidden",
+                                      "lora_rank", "n_lora", "b_kind", "inject_e", "max_loops")]
+
+
+WEIGHT_FIELDS = ("A", "B", "norm1", "norm2", "wq", "wk", "wv", "wo", "w_dq", "q_norm", "w_uq",
+                 "w_dkv", "kv_norm", "w_kr", "w_uk", "w_uv", "w_router", "router_bias", "w1",
+                 "w3", "w2", "ws1", "ws3", "ws2", "lq_a", "lq_b", "lo_a", "lo_b")
+FP32_FIELDS = ("A", "B", "norm1", "norm2", "q_norm", "kv_norm", "router_bias")
+
+
+class RdtWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS]
+
+
+class RdtDiag(ctypes.Structure):
+    _fields_ = [("rho_A", ctypes.c_float), ("nonfinite", ctypes.c_int32), ("timeout", ctypes.c_int32),
+                ("last_routed_rows", ctypes.c_int32), ("expert_counts", ctypes.c_int32 * 256)]
+
+
+_LIB = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load the in-tree librdt.so (build it with ``python -m recurrent_depth_transformer_b200.build``)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(library_path):
+        raise RuntimeError(f"{library_path} is missing: build it with "
+                           "`python -m recurrent_depth_transformer_b200.build`")
+    lib = ctypes.CDLL(library_path)
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    lib.rdt_create.argtypes = [ctypes.POINTER(RdtConfig), ctypes.POINTER(RdtWeights), vp,
+                               ctypes.POINTER(vp)]
+    lib.rdt_attn_forward.argtypes = [vp, vp, i32, vp, vp]
+    lib.rdt_moe_forward.argtypes = [vp, vp, vp, vp, vp, vp]
+    lib.rdt_loop_forward.argtypes = [vp, vp, vp, i32, vp, vp]
+    lib.rdt_loop_forward_host.argtypes = [vp, vp, vp, i32, vp, vp]
+    lib.rdt_set_trace.argtypes = [vp, vp, vp, vp]
+    lib.rdt_get_diagnostics.argtypes = [vp, ctypes.POINTER(RdtDiag)]
+    lib.rdt_memory_bytes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t)]
+    lib.rdt_status_string.argtypes = [i32]
+    lib.rdt_status_string.restype = ctypes.c_char_p
+    lib.rdt_last_error.argtypes = []
+    lib.rdt_last_error.restype = ctypes.c_char_p
+    lib.rdt_destroy.argtypes = [vp]
+    lib.rdt_destroy.restype = None
+    lib.rdt_matmul.argtypes = [i32, vp, vp, vp, i32, i32, i32, vp]
+    lib.rdt_attention.argtypes = [i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                  ctypes.c_float, vp]
+    for f in ("rdt_create", "rdt_attn_forward", "rdt_moe_forward", "rdt_loop_forward",
+              "rdt_loop_forward_host", "rdt_set_trace", "rdt_get_diagnostics", "rdt_memory_bytes",
+              "rdt_matmul", "rdt_attention"):
+        getattr(lib, f).restype = i32
+    _LIB = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        lib = load_library()
+        raise RdtError(status, lib.rdt_last_error().decode(errors="replace"))
+
+
+def make_config(wl, max_loops: int = 16, batch: Optional[int] = None, seq: Optional[int] = None) -> RdtConfig:
+    """Fill the C config from any object with the block's hyper-parameters as attributes."""
+    c = RdtConfig()
+    c.dtype = RDT_BF16 if wl.dtype == "bf16" else RDT_F32
+    c.batch = wl.batch if batch is None else batch
+    c.seq = wl.seq if seq is None else seq
+    c.dim = wl.dim
+    c.attn_type = RDT_GQA if wl.attn == "gqa" else RDT_MLA
+    c.n_heads = wl.n_heads
+    c.n_kv_heads = wl.n_kv_heads
+    c.head_dim = wl.head_dim
+    c.q_lora_rank = wl.q_lora_rank
+    c.kv_lora_rank = wl.kv_lora_rank
+    c.qk_nope_dim = wl.qk_nope_dim
+    c.qk_rope_dim = wl.qk_rope_dim
+    c.v_head_dim = wl.v_head_dim
+    c.rope_base = wl.rope_base
+    c.norm_eps = wl.norm_eps
+    c.n_experts = wl.n_experts
+    c.top_k = wl.top_k
+    c.n_shared = wl.n_shared
+    c.expert_hidden = wl.expert_hidden
+    c.lora_rank = wl.lora_rank
+    c.n_lora = wl.n_lora
+    c.b_kind = RDT_B_DIAG if wl.b_kind == "diag" else RDT_B_DENSE
+    c.inject_e = 1 if wl.inject_e else 0
+    c.max_loops = max_loops
+    return c
+
+
+def device_weights(arrays: Dict[str, np.ndarray], bf16: bool, device="cuda"):
+    """Upload host weight arrays (float32 holding element-type values) as CUDA tensors:
+    fp32 for A, B, norm gains and the router bias; bf16 or fp32 for the matrices."""
+    import torch
+    out = {}
+    for k in WEIGHT_FIELDS:
+        if k not in arrays or arrays[k] is None:
+            continue
+        t = torch.from_numpy(np.ascontiguousarray(arrays[k], dtype=np.float32))
+        if bf16 and k not in FP32_FIELDS:
+            t = t.to(torch.bfloat16)
+        out[k] = t.to(device)
+    return out
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else int(t.data_ptr())
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def matmul(A, B, C=None, stream=None):
+    """C = A B^T (fp32) on the tensor-core GEMM; A [M, K], B [N, K] bf16 or fp32 CUDA tensors."""
+    import torch
+    lib = load_library()
+    M, K = A.shape
+    N = B.shape[0]
+    C = torch.empty((M, N), dtype=torch.float32, device=A.device) if C is None else C
+    dt = RDT_BF16 if A.dtype == torch.bfloat16 else RDT_F32
+    _check(lib.rdt_matmul(dt, _ptr(A), _ptr(B), _ptr(C), M, N, K, _stream(stream)))
+    return C
+
+
+def attention(q, k, v, batch, seq, n_heads, n_kv_heads, dqk, dv, scale, o=None, stream=None):
+    """Causal GQA attention on [batch*seq, heads*dim] CUDA tensors (see rdt_attention)."""
+    import torch
+    lib = load_library()
+    o = torch.empty((batch * seq, n_heads * dv), dtype=q.dtype, device=q.device) if o is None else o
+    dt = RDT_BF16 if q.dtype == torch.bfloat16 else RDT_F32
+    _check(lib.rdt_attention(dt, _ptr(q), _ptr(k), _ptr(v), _ptr(o), batch, seq, n_heads, n_kv_heads,
+                             dqk, dv, scale, _stream(stream)))
+    return o
+
+
+class RDT:
+    """A created handle: weights copied into library memory, workspace for batch x seq tokens."""
+
+    def __init__(self, config: RdtConfig, weights: Dict[str, "object"], stream=None):
+        import torch
+        self._lib = load_library()
+        if not torch.cuda.is_available():
+            raise RuntimeError("a CUDA device is required")
+        self.cfg = config
+        w = RdtWeights()
+        for k in WEIGHT_FIELDS:
+            setattr(w, k, _ptr(weights.get(k)))
+        h = ctypes.c_void_p()
+        _check(self._lib.rdt_create(ctypes.byref(config), ctypes.byref(w), _stream(stream), ctypes.byref(h)))
+        self._h = h
+        self.ntok = config.batch * config.seq
+        self._trace = None
+
+    # ---------------------------------------------------------------- calls
+    def attn_forward(self, x, loop: int = 0, a_out=None, stream=None):
+        import torch
+        a_out = torch.empty_like(x, dtype=torch.float32) if a_out is None else a_out
+        _check(self._lib.rdt_attn_forward(self._h, _ptr(x), loop, _ptr(a_out), _stream(stream)))
+        return a_out
+
+    def moe_forward(self, y, f_out=None, idx=None, w=None, stream=None):
+        import torch
+        f_out = torch.empty_like(y, dtype=torch.float32) if f_out is None else f_out
+        _check(self._lib.rdt_moe_forward(self._h, _ptr(y), _ptr(f_out), _ptr(idx), _ptr(w), _stream(stream)))
+        return f_out
+
+    def loop_forward(self, h0, e, T: int, out=None, stream=None):
+        import torch
+        if out is None:
+            out = torch.empty(e.shape, dtype=torch.float32, device=e.device)
+        _check(self._lib.rdt_loop_forward(self._h, _ptr(h0), _ptr(e), T, _ptr(out), _stream(stream)))
+        return out
+
+    def loop_forward_host(self, h0, e, T: int, out, stream=None):
+        """Host (CPU, ideally pinned) tensors in, host fp32 tensor out; synchronous."""
+        _check(self._lib.rdt_loop_forward_host(self._h, _ptr(h0), _ptr(e), T, _ptr(out), _stream(stream)))
+        return out
+
+    def set_trace(self, idx=None, w=None, h_traj=None):
+        self._trace = (idx, w, h_traj)       # keep the buffers alive
+        _check(self._lib.rdt_set_trace(self._h, _ptr(idx), _ptr(w), _ptr(h_traj)))
+
+    def diagnostics(self) -> dict:
+        d = RdtDiag()
+        _check(self._lib.rdt_get_diagnostics(self._h, ctypes.byref(d)))
+        E = self.cfg.n_experts + self.cfg.n_shared
+        return {"rho_A": d.rho_A, "nonfinite": d.nonfinite, "timeout": d.timeout,
+                "last_routed_rows": d.last_routed_rows, "expert_counts": list(d.expert_counts[:E])}
+
+    def memory_bytes(self) -> int:
+        n = ctypes.c_size_t()
+        _check(self._lib.rdt_memory_bytes(self._h, ctypes.byref(n)))
+        return n.value
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.rdt_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        self.close()

@@ -1,0 +1,433 @@
+// Dense and grouped GEMM on the sm_100a 5th-generation tensor cores, C = A * B^T.
+//
+// One CTA computes one 128 x BN output tile:
+//   warp 0      one thread issues TMA loads of 128-byte-wide K slices of A and B into a
+//               ring of shared-memory stages (128-byte swizzle, K-major);
+//   warp 1      allocates the TMEM accumulator; one thread issues tcgen05.mma (M = 128,
+//               N = BN, K = 16 bf16 / 8 tf32 per instruction) and frees each stage with
+//               tcgen05.commit when its MMAs have read it;
+//   warps 2-5   the epilogue: each warp reads its 32-lane quadrant of TMEM (one output row
+//               per thread) and applies one of the fused epilogues below.
+//
+// The fused epilogues are where the block's element-wise work lives:
+//   EPI_ROPE        Q/K/V projection + rotary embedding on the rotated heads;
+//   EPI_OPROJ_LOOP  output projection fused with the residual (y = x + a) and the
+//                   recurrent update h_next = A (.) h + B.e + a (the MoE adds f later);
+//   EPI_SWIGLU      expert up-projection (gate and up rows interleaved per tile) -> silu(g)*u;
+//   EPI_SCATTER     expert down-projection, gate weight, and reduction into h_next
+//                   (h_{t+1} = A h + B e + a + sum_j w_j E_j(yn)).
+// Grouped mode reads a device-resident tile list (expert, A row, output row, rows), so
+// the per-expert row counts never travel to the host.
+#include <type_traits>
+
+#include "rdt_internal.cuh"
+
+namespace rdt {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int kThreads = 192;
+
+template <int BN>
+struct TcCfg {
+    static constexpr int STAGES = (BN <= 128) ? 6 : 4;
+    static constexpr int A_BYTES = BM * 128;
+    static constexpr int B_BYTES = BN * 128;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int TMEM_COLS = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+    static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte alignment of stages");
+};
+
+__device__ __forceinline__ void ld_chunk(uint32_t taddr, int c, float (&v)[32]) {
+    uint32_t r[32];
+    tmem_ld32(taddr + static_cast<uint32_t>(c * 32), r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <typename OutT>
+__device__ __forceinline__ void store_row32(OutT* p, const float (&v)[32]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float t[4] = {v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]};
+        store4(p + 4 * j, t);
+    }
+}
+
+// Rotary embedding: the pair (i, i + R/2) turns by angle pos * base^(-2i/R); the table
+// rows hold cos/sin of those angles for one position.
+template <int R>
+__device__ __forceinline__ void rope_rotate(float (&v)[32], const float* cosr, const float* sinr) {
+#pragma unroll
+    for (int i = 0; i < R / 2; ++i) {
+        const float c = cosr[i], s = sinr[i];
+        const float x1 = v[i], x2 = v[i + R / 2];
+        v[i] = x1 * c - x2 * s;
+        v[i + R / 2] = x2 * c + x1 * s;
+    }
+}
+__device__ __forceinline__ void rope_rotate_pair(float (&lo)[32], float (&hi)[32],
+                                                 const float* cosr, const float* sinr) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const float c = cosr[i], s = sinr[i];
+        const float x1 = lo[i], x2 = hi[i];
+        lo[i] = x1 * c - x2 * s;
+        hi[i] = x2 * c + x1 * s;
+    }
+}
+
+// ----------------------------------------------------------------------------- epilogues
+
+template <typename T, int BN, int KIND>
+__device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, bool valid, int crow,
+                                         int n0) {
+    if constexpr (KIND == EPI_STORE || KIND == EPI_STORE_F32 || KIND == EPI_OPROJ_PLAIN) {
+        using OutT = std::conditional_t<KIND == EPI_STORE, T, float>;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            ld_chunk(taddr, c, v);
+            const int col = n0 + c * 32;
+            if (valid && col < p.ncols_valid)
+                store_row32(static_cast<OutT*>(p.out) + static_cast<size_t>(crow) * p.ldo + col, v);
+        }
+    } else if constexpr (KIND == EPI_ROPE) {
+        // Heads of width head_w tile the BN columns exactly (host checks BN % head_w == 0).
+        const int pos = crow % p.seq;
+        const int hw_chunks = p.head_w / 32;
+        const int rc0 = p.rot_off / 32;
+        const int rch = p.rot_dim / 32;
+        const float* cosr = p.rope_cos + static_cast<size_t>(pos) * (p.rot_dim / 2);
+        const float* sinr = p.rope_sin + static_cast<size_t>(pos) * (p.rot_dim / 2);
+        T* out = static_cast<T*>(p.out) + static_cast<size_t>(crow) * p.ldo;
+#pragma unroll 1
+        for (int hc = 0; hc < BN / 32; hc += hw_chunks) {
+            const int head_col0 = n0 + hc * 32;
+            const bool rotate = head_col0 < p.rope_limit;
+#pragma unroll 1
+            for (int c = 0; c < hw_chunks; ++c) {
+                const int col = head_col0 + c * 32;
+                if (rotate && c == rc0) {
+                    if (rch == 2) {
+                        float v0[32], v1[32];
+                        ld_chunk(taddr, hc + c, v0);
+                        ld_chunk(taddr, hc + c + 1, v1);
+                        rope_rotate_pair(v0, v1, cosr, sinr);
+                        if (valid && col < p.ncols_valid) {
+                            store_row32(out + col, v0);
+                            store_row32(out + col + 32, v1);
+                        }
+                        c += 1;
+                    } else {
+                        float v[32];
+                        ld_chunk(taddr, hc + c, v);
+                        rope_rotate<32>(v, cosr, sinr);
+                        if (valid && col < p.ncols_valid) store_row32(out + col, v);
+                    }
+                } else {
+                    float v[32];
+                    ld_chunk(taddr, hc + c, v);
+                    if (valid && col < p.ncols_valid) store_row32(out + col, v);
+                }
+            }
+        }
+    } else if constexpr (KIND == EPI_OPROJ_LOOP) {
+        const size_t rbase = static_cast<size_t>(crow) * p.ld;
+        const T* e = static_cast<const T*>(p.e);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            ld_chunk(taddr, c, v);
+            const int col = n0 + c * 32;
+            if (!valid || col >= p.ncols_valid) continue;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const size_t off = rbase + col + 4 * j;
+                float hh[4], be[4], aa[4], x[4], yv[4], hn[4];
+                load4(p.h + off, hh);
+                load4(p.Be + off, be);
+                load4(p.Adiag + col + 4 * j, aa);
+                if (e) {
+                    float ee[4];
+                    load4(e + off, ee);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) x[i] = hh[i] + ee[i];
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) x[i] = hh[i];
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float a = v[4 * j + i];
+                    yv[i] = x[i] + a;
+                    hn[i] = aa[i] * hh[i] + be[i] + a;
+                }
+                store4(p.y + off, yv);
+                store4(p.h_next + off, hn);
+            }
+        }
+    } else if constexpr (KIND == EPI_SWIGLU) {
+        // Tile columns [0, BN/2) are gate rows (W1), [BN/2, BN) the matching up rows (W3).
+        T* out = static_cast<T*>(p.out) + static_cast<size_t>(crow) * p.ldo + n0 / 2;
+#pragma unroll 1
+        for (int c = 0; c < BN / 64; ++c) {
+            float g[32], u[32];
+            ld_chunk(taddr, c, g);
+            ld_chunk(taddr, c + BN / 64, u);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) g[i] = g[i] / (1.0f + expf(-g[i])) * u[i];
+            if (valid) store_row32(out + c * 32, g);
+        }
+    } else if constexpr (KIND == EPI_SCATTER) {
+        int token = -1;
+        float w = 0.0f;
+        if (valid) {
+            if (crow < p.shared_rows) {
+                token = crow % p.ntok;
+                w = 1.0f;
+            } else {
+                token = p.row_token[crow - p.shared_rows];
+                w = p.row_w[crow - p.shared_rows];
+            }
+        }
+        float* dst = p.dst + static_cast<size_t>(token < 0 ? 0 : token) * p.ld;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            ld_chunk(taddr, c, v);
+            const int col = n0 + c * 32;
+            if (token < 0 || col >= p.ncols_valid) continue;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float4 add = make_float4(w * v[4 * j], w * v[4 * j + 1], w * v[4 * j + 2],
+                                         w * v[4 * j + 3]);
+                atomicAdd(reinterpret_cast<float4*>(dst + col + 4 * j), add);
+            }
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------- the kernel
+
+template <typename T, int BN, int KIND>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
+                   const __grid_constant__ CUtensorMap tA2, const __grid_constant__ CUtensorMap tB2,
+                   const GemmArgs args, const EpiParams epi) {
+    using C = TcCfg<BN>;
+    constexpr bool kBf16 = std::is_same<T, bf16>::value;
+    constexpr int kElemsPerRow = 128 / static_cast<int>(sizeof(T));   // K elements per stage
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+    uint64_t* empty = full + C::STAGES;
+    uint64_t* done = empty + C::STAGES;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    int a_row0, c_row0, nrows, group = 0;
+    if (args.tiles != nullptr) {
+        if (static_cast<int>(blockIdx.y) >= *args.n_tiles) return;   // uniform per CTA
+        const GroupTile t = args.tiles[blockIdx.y];
+        group = t.group;
+        a_row0 = args.a_from_c ? t.c_row0 : t.a_row0;
+        c_row0 = t.c_row0;
+        nrows = t.nrows;
+    } else {
+        a_row0 = blockIdx.y * BM;
+        c_row0 = a_row0;
+        nrows = min(BM, args.M - a_row0);
+    }
+    const int n0 = blockIdx.x * BN;
+    const int b_row0 = group * args.N + n0;
+    const int num_kb = args.kb_main + args.kb_ext;
+
+    if (threadIdx.x == 0) {
+#pragma unroll 1
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(done, 1);
+        mbar_fence_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tA);
+            tma_prefetch_desc(&tB);
+#pragma unroll 1
+            for (int kb = 0; kb < num_kb; ++kb) {
+                const int s = kb % C::STAGES;
+                const uint32_t ph = (kb / C::STAGES) & 1;
+                if (!mbar_wait(&empty[s], ph ^ 1, epi.flags)) break;
+                uint8_t* sa = smem + s * C::STAGE_BYTES;
+                uint8_t* sb = sa + C::A_BYTES;
+                mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+                if (kb < args.kb_main) {
+                    tma_load_2d(sa, &tA, &full[s], kb * kElemsPerRow, a_row0);
+                    tma_load_2d(sb, &tB, &full[s], kb * kElemsPerRow, b_row0);
+                } else {
+                    tma_load_2d(sa, &tA2, &full[s], 0, a_row0);
+                    tma_load_2d(sb, &tB2, &full[s], 0, args.b2_row0 + n0);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = make_idesc(kBf16 ? 1 : 2, BM, BN);
+#pragma unroll 1
+            for (int kb = 0; kb < num_kb; ++kb) {
+                const int s = kb % C::STAGES;
+                const uint32_t ph = (kb / C::STAGES) & 1;
+                if (!mbar_wait(&full[s], ph, epi.flags)) break;
+                tc_fence_after();
+                const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+                const uint64_t da = sw128_kmajor_desc(sa);
+                const uint64_t db = sw128_kmajor_desc(sa + C::A_BYTES);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    // each MMA consumes 32 bytes of K: advance the start address by 32 B (>> 4 = 2)
+                    if constexpr (kBf16)
+                        tc_mma_bf16(tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                    else
+                        tc_mma_tf32(tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                }
+                tc_commit(&empty[s]);
+            }
+            tc_commit(done);
+        }
+    } else {
+        const int q = warp & 3;            // TMEM lane quadrant accessible to this warp
+        const int r = q * 32 + lane;       // row inside the tile
+        const bool ok = mbar_wait(done, 0, epi.flags);
+        tc_fence_after();
+        if (ok)
+            epilogue<T, BN, KIND>(epi, tmem + (static_cast<uint32_t>(q * 32) << 16), r < nrows,
+                                  c_row0 + r, n0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <typename T, int BN, int KIND>
+rdt_status launch(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap* tA2,
+                  const CUtensorMap* tB2, const GemmArgs& args, const EpiParams& epi,
+                  cudaStream_t st) {
+    using C = TcCfg<BN>;
+    auto kern = gemm_tc_kernel<T, BN, KIND>;
+    static bool configured = false;
+    if (!configured) {
+        RDT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          C::SMEM));
+        configured = true;
+    }
+    const int gy = args.tiles ? args.max_tiles : (args.M + BM - 1) / BM;
+    const dim3 grid((args.N + BN - 1) / BN, gy);
+    if (gy <= 0) return RDT_OK;
+    kern<<<grid, kThreads, C::SMEM, st>>>(tA, tB, tA2 ? *tA2 : tA, tB2 ? *tB2 : tB, args, epi);
+    RDT_CUDA_TRY(cudaGetLastError());
+    return RDT_OK;
+}
+
+template <typename T, int BN>
+rdt_status dispatch_kind(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap* tA2,
+                         const CUtensorMap* tB2, const GemmArgs& args, const EpiParams& epi,
+                         cudaStream_t st) {
+    switch (epi.kind) {
+        case EPI_STORE: return launch<T, BN, EPI_STORE>(tA, tB, tA2, tB2, args, epi, st);
+        case EPI_STORE_F32: return launch<T, BN, EPI_STORE_F32>(tA, tB, tA2, tB2, args, epi, st);
+        case EPI_ROPE: return launch<T, BN, EPI_ROPE>(tA, tB, tA2, tB2, args, epi, st);
+        case EPI_OPROJ_LOOP: return launch<T, BN, EPI_OPROJ_LOOP>(tA, tB, tA2, tB2, args, epi, st);
+        case EPI_OPROJ_PLAIN: return launch<T, BN, EPI_OPROJ_PLAIN>(tA, tB, tA2, tB2, args, epi, st);
+        case EPI_SWIGLU: return launch<T, BN, EPI_SWIGLU>(tA, tB, tA2, tB2, args, epi, st);
+        case EPI_SCATTER: return launch<T, BN, EPI_SCATTER>(tA, tB, tA2, tB2, args, epi, st);
+        default: set_error("gemm_tc: unknown epilogue"); return RDT_ERR_INVALID_ARG;
+    }
+}
+
+}  // namespace
+
+rdt_status gemm_tc(bool bf16_elems, int bn, const CUtensorMap& tA, const CUtensorMap& tB,
+                   const CUtensorMap* tA2, const CUtensorMap* tB2, const GemmArgs& args,
+                   const EpiParams& epi, cudaStream_t st) {
+    if (bf16_elems) {
+        if (bn == 128) return dispatch_kind<bf16, 128>(tA, tB, tA2, tB2, args, epi, st);
+        if (bn == 160) return dispatch_kind<bf16, 160>(tA, tB, tA2, tB2, args, epi, st);
+        if (bn == 256) return dispatch_kind<bf16, 256>(tA, tB, tA2, tB2, args, epi, st);
+    } else {
+        if (bn == 128) return dispatch_kind<float, 128>(tA, tB, tA2, tB2, args, epi, st);
+    }
+    set_error("gemm_tc: unsupported tile width");
+    return RDT_ERR_UNSUPPORTED;
+}
+
+// ----------------------------------------------------------------------------- tensor maps
+
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+}  // namespace
+
+rdt_status make_tmap_2d(CUtensorMap* map, const void* base, bool bf16_elems, uint64_t inner,
+                        uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner,
+                        uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) {
+        set_error("cuTensorMapEncodeTiled entry point unavailable");
+        return RDT_ERR_CUDA;
+    }
+    if ((reinterpret_cast<uintptr_t>(base) & 15) || (row_stride_bytes & 15)) {
+        set_error("tensor map: base or row stride not 16-byte aligned");
+        return RDT_ERR_MISALIGNED;
+    }
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {row_stride_bytes};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, bf16_elems ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                    2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed with code " + std::to_string(static_cast<int>(r)));
+        return RDT_ERR_CUDA;
+    }
+    return RDT_OK;
+}
+
+}  // namespace rdt

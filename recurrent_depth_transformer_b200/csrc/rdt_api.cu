@@ -1,0 +1,957 @@
+// The C ABI of librdt (include/rdt.h): argument validation, weight repacking, the
+// library-owned workspace, TMA descriptors, and the per-loop launch sequence of the
+// recurrent block
+//
+//   h_{t+1} = A (.) h_t + B.e + a_t + f_t       (techbriefly article, update equation)
+//
+// per loop t:  norm1 -> QKV(+RoPE, +LoRA) -> attention -> [LoRA-down] -> O-proj fused with
+//              y = x + a and h_next = A h + Be + a -> norm2 + router top-k -> dispatch ->
+//              expert up (SwiGLU) -> expert down fused with gate weight and h_next += w E(yn).
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "rdt_internal.cuh"
+
+namespace rdt {
+
+static thread_local std::string g_last_error;
+void set_error(const std::string& msg) { g_last_error = msg; }
+
+}  // namespace rdt
+
+using namespace rdt;
+
+struct rdt_handle {
+    rdt_config cfg{};
+    bool bf = true;
+    size_t esz = 2;
+    int ntok = 0;
+    int kext = 64;                 // padded LoRA width = one 128-byte K block
+    int G = 0;                     // expert groups = routed + shared
+    float rho = 0.0f;
+    cudaStream_t last_stream = nullptr;
+    std::vector<void*> allocs;
+    size_t bytes = 0;
+
+    // weights (library-owned)
+    float *A = nullptr, *Bw = nullptr, *g1 = nullptr, *g2 = nullptr, *rbias = nullptr;
+    float *q_norm = nullptr, *kv_norm = nullptr;
+    void *wqkv = nullptr, *wo = nullptr, *wr = nullptr, *w13 = nullptr, *w2 = nullptr;
+    void *lqa = nullptr, *lqb = nullptr, *loa = nullptr, *lob = nullptr;
+    void *wlat = nullptr, *wqabs = nullptr;
+    float *rope_cos = nullptr, *rope_sin = nullptr;
+    int rot = 0;
+
+    // geometry
+    int nq = 0, nkv = 0, nqkv = 0;  // GQA projection widths
+    int owidth = 0;                 // width of the attention output o
+    int qt_w = 0;                   // MLA: width of q~ (H * (kv_lat + rope))
+    int lat_w = 0;                  // MLA: q_lat + kv_lat + rope
+
+    // workspace
+    float *hbuf[2] = {nullptr, nullptr}, *Be = nullptr, *y = nullptr, *lat = nullptr;
+    void *xn = nullptr, *tq = nullptr, *to = nullptr, *qkv = nullptr, *o = nullptr;
+    void *cq = nullptr, *kvlat = nullptr, *xperm = nullptr, *U = nullptr;
+    int32_t* idx = nullptr;
+    float* wts = nullptr;
+    int *counts = nullptr, *offsets = nullptr, *fill = nullptr, *ntiles = nullptr, *row_token = nullptr;
+    float* row_w = nullptr;
+    GroupTile* tiles = nullptr;
+    int max_tiles = 0;
+    int* flags = nullptr;
+    void *stage_h0 = nullptr, *stage_e = nullptr;
+    float* stage_out = nullptr;
+
+    // tensor maps
+    CUtensorMap m_xn, m_wqkv, m_tq, m_lqb, m_o, m_wo, m_to, m_lob, m_xperm, m_w13, m_U, m_w2;
+    CUtensorMap m_wlat, m_cq, m_wqabs;
+
+    // trace
+    int32_t* tr_idx = nullptr;
+    float* tr_w = nullptr;
+    float* tr_h = nullptr;
+};
+
+namespace {
+
+template <typename P>
+rdt_status dev_alloc(rdt_handle* h, P** p, size_t bytes, bool zero = false) {
+    void* q = nullptr;
+    if (bytes == 0) bytes = 16;
+    if (cudaMalloc(&q, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        set_error("cudaMalloc of " + std::to_string(bytes) + " bytes failed");
+        return RDT_ERR_OOM;
+    }
+    h->allocs.push_back(q);
+    h->bytes += bytes;
+    if (zero) RDT_CUDA_TRY(cudaMemset(q, 0, bytes));
+    *p = static_cast<P*>(q);
+    return RDT_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+rdt_status validate_config(const rdt_config* c) {
+    auto bad = [](const char* m) { set_error(std::string("config: ") + m); return RDT_ERR_INVALID_ARG; };
+    auto uns = [](const char* m) { set_error(std::string("config: ") + m); return RDT_ERR_UNSUPPORTED; };
+    if (!c) return bad("NULL config");
+    if (c->dtype != RDT_F32 && c->dtype != RDT_BF16) return bad("dtype");
+    if (c->batch < 1 || c->seq < 1 || c->dim < 1) return bad("batch, seq and dim must be >= 1");
+    if (static_cast<long long>(c->batch) * c->seq > (1 << 24)) return uns("too many tokens");
+    const int nv = c->dim / 128;
+    if (c->dim % 128 || (nv & (nv - 1)) || nv > 32) return uns("dim must be 128 * 2^k <= 4096");
+    if (c->n_heads < 1) return bad("n_heads");
+    if (c->n_experts < 1 || c->top_k < 1 || c->top_k > c->n_experts) return bad("n_experts / top_k");
+    if (c->top_k > 16) return uns("top_k > 16");
+    if (c->n_shared < 0 || c->n_experts + c->n_shared > 256) return uns("n_experts + n_shared > 256");
+    if (c->expert_hidden < 64 || c->expert_hidden % 64) return uns("expert_hidden % 64 != 0");
+    if (c->dtype == RDT_F32 && c->expert_hidden % 128) return uns("f32: expert_hidden % 128 != 0");
+    if (c->max_loops < 1 || c->max_loops > 64) return bad("max_loops must be in [1, 64]");
+    if (c->b_kind != RDT_B_DIAG && c->b_kind != RDT_B_DENSE) return bad("b_kind");
+    if (!(c->norm_eps >= 0.0f) || !(c->rope_base > 1.0f)) return bad("norm_eps / rope_base");
+    if (c->lora_rank < 0 || c->n_lora < 0) return bad("lora");
+    if (c->n_lora > 0) {
+        if (c->attn_type != RDT_GQA) return uns("LoRA is provided for the GQA projections");
+        if (c->lora_rank < 1 || c->lora_rank > (c->dtype == RDT_BF16 ? 64 : 32)) return uns("lora_rank");
+    }
+    if (c->attn_type == RDT_GQA) {
+        if (c->n_kv_heads < 1 || c->n_heads % c->n_kv_heads) return bad("n_heads % n_kv_heads");
+        if (c->dtype == RDT_BF16 ? c->head_dim != 64 : (c->head_dim != 32 && c->head_dim != 64))
+            return uns("head_dim (bf16: 64; f32: 32 or 64)");
+        if ((c->n_heads * c->head_dim) % 128) return uns("n_heads * head_dim % 128 != 0");
+    } else if (c->attn_type == RDT_MLA) {
+        if (c->dtype != RDT_BF16) return uns("MLA is provided in bf16");
+        if (c->kv_lora_rank != 128 || c->qk_rope_dim != 32) return uns("MLA: kv_lora_rank 128, qk_rope_dim 32");
+        if (c->q_lora_rank < 64 || c->q_lora_rank % 64) return uns("MLA: q_lora_rank % 64");
+        if (c->qk_nope_dim < 1 || c->v_head_dim < 1 || c->v_head_dim % 32) return uns("MLA head dims");
+    } else {
+        return bad("attn_type");
+    }
+    return RDT_OK;
+}
+
+rdt_status need(const void* p, const char* name) {
+    if (!p) {
+        set_error(std::string("weights: ") + name + " is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (!aligned16(p)) {
+        set_error(std::string("weights: ") + name + " is not 16-byte aligned");
+        return RDT_ERR_MISALIGNED;
+    }
+    return RDT_OK;
+}
+
+rdt_status copy_d2d(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+    RDT_CUDA_TRY(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st));
+    return RDT_OK;
+}
+
+// W1 || W3 interleaved in 64-row blocks: rows [128j, 128j+64) = W1 rows [64j, 64j+64),
+// rows [128j+64, 128j+128) = W3 rows [64j, 64j+64) (one 128-column tile of the up GEMM
+// holds matching gate and up columns).
+rdt_status interleave_w13(void* dst, const void* w1, const void* w3, int hid, int dim, size_t esz,
+                          cudaStream_t st) {
+    const size_t blk = static_cast<size_t>(64) * dim * esz;
+    RDT_CUDA_TRY(cudaMemcpy2DAsync(dst, 2 * blk, w1, blk, blk, hid / 64, cudaMemcpyDeviceToDevice, st));
+    RDT_CUDA_TRY(cudaMemcpy2DAsync(static_cast<char*>(dst) + blk, 2 * blk, w3, blk, blk, hid / 64,
+                                   cudaMemcpyDeviceToDevice, st));
+    return RDT_OK;
+}
+
+rdt_status build_maps(rdt_handle* h) {
+    const rdt_config& c = h->cfg;
+    const bool bf = h->bf;
+    const uint32_t kbox = static_cast<uint32_t>(128 / h->esz);
+    const size_t es = h->esz;
+    const int N = h->ntok, d = c.dim;
+    const int S = c.n_shared, E = c.n_experts, hid = c.expert_hidden;
+    RDT_TRY(make_tmap_2d(&h->m_xn, h->xn, bf, d, N, d * es, kbox, 128));
+    RDT_TRY(make_tmap_2d(&h->m_o, h->o, bf, h->owidth, N, h->owidth * es, kbox, 128));
+    RDT_TRY(make_tmap_2d(&h->m_wo, h->wo, bf, h->owidth, d, h->owidth * es, kbox, 128));
+    if (c.attn_type == RDT_GQA) {
+        RDT_TRY(make_tmap_2d(&h->m_wqkv, h->wqkv, bf, d, h->nqkv, d * es, kbox, 128));
+    } else {
+        RDT_TRY(make_tmap_2d(&h->m_wlat, h->wlat, bf, d, h->lat_w, d * es, kbox, 128));
+        RDT_TRY(make_tmap_2d(&h->m_cq, h->cq, bf, c.q_lora_rank, N, c.q_lora_rank * es, kbox, 128));
+        RDT_TRY(make_tmap_2d(&h->m_wqabs, h->wqabs, bf, c.q_lora_rank, h->qt_w, c.q_lora_rank * es, kbox, 160));
+    }
+    if (c.n_lora) {
+        RDT_TRY(make_tmap_2d(&h->m_tq, h->tq, bf, h->kext, N, h->kext * es, kbox, 128));
+        RDT_TRY(make_tmap_2d(&h->m_to, h->to, bf, h->kext, N, h->kext * es, kbox, 128));
+        RDT_TRY(make_tmap_2d(&h->m_lqb, h->lqb, bf, h->kext, static_cast<uint64_t>(c.n_lora) * h->nqkv,
+                             h->kext * es, kbox, 128));
+        RDT_TRY(make_tmap_2d(&h->m_lob, h->lob, bf, h->kext, static_cast<uint64_t>(c.n_lora) * d,
+                             h->kext * es, kbox, 128));
+    }
+    const uint64_t xrows = static_cast<uint64_t>(N) * (1 + c.top_k);
+    const uint64_t urows = static_cast<uint64_t>(N) * (S + c.top_k);
+    RDT_TRY(make_tmap_2d(&h->m_xperm, h->xperm, bf, d, xrows, d * es, kbox, 128));
+    RDT_TRY(make_tmap_2d(&h->m_w13, h->w13, bf, d, static_cast<uint64_t>(E + S) * 2 * hid, d * es, kbox, 128));
+    RDT_TRY(make_tmap_2d(&h->m_U, h->U, bf, hid, urows, hid * es, kbox, 128));
+    RDT_TRY(make_tmap_2d(&h->m_w2, h->w2, bf, hid, static_cast<uint64_t>(E + S) * d, hid * es, kbox, 128));
+    return RDT_OK;
+}
+
+rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t st, rdt_handle* h) {
+    const rdt_config& c = *cfg;
+    h->cfg = c;
+    h->bf = c.dtype == RDT_BF16;
+    h->esz = h->bf ? 2 : 4;
+    h->kext = static_cast<int>(128 / h->esz);
+    h->ntok = c.batch * c.seq;
+    h->G = c.n_experts + c.n_shared;
+    const size_t es = h->esz;
+    const int N = h->ntok, d = c.dim, E = c.n_experts, S = c.n_shared, hid = c.expert_hidden;
+    const int K = c.top_k;
+
+    // ---- weights present and aligned
+    RDT_TRY(need(w->A, "A"));
+    RDT_TRY(need(w->B, "B"));
+    RDT_TRY(need(w->norm1, "norm1"));
+    RDT_TRY(need(w->norm2, "norm2"));
+    RDT_TRY(need(w->w_router, "w_router"));
+    RDT_TRY(need(w->w1, "w1"));
+    RDT_TRY(need(w->w3, "w3"));
+    RDT_TRY(need(w->w2, "w2"));
+    if (w->router_bias) RDT_TRY(need(w->router_bias, "router_bias"));
+    if (S) {
+        RDT_TRY(need(w->ws1, "ws1"));
+        RDT_TRY(need(w->ws3, "ws3"));
+        RDT_TRY(need(w->ws2, "ws2"));
+    }
+    if (c.attn_type == RDT_GQA) {
+        RDT_TRY(need(w->wq, "wq"));
+        RDT_TRY(need(w->wk, "wk"));
+        RDT_TRY(need(w->wv, "wv"));
+        RDT_TRY(need(w->wo, "wo"));
+    } else {
+        RDT_TRY(need(w->w_dq, "w_dq"));
+        RDT_TRY(need(w->q_norm, "q_norm"));
+        RDT_TRY(need(w->w_uq, "w_uq"));
+        RDT_TRY(need(w->w_dkv, "w_dkv"));
+        RDT_TRY(need(w->kv_norm, "kv_norm"));
+        RDT_TRY(need(w->w_kr, "w_kr"));
+        RDT_TRY(need(w->w_uk, "w_uk"));
+        RDT_TRY(need(w->w_uv, "w_uv"));
+        RDT_TRY(need(w->wo, "wo"));
+    }
+    if (c.n_lora) {
+        RDT_TRY(need(w->lq_a, "lq_a"));
+        RDT_TRY(need(w->lq_b, "lq_b"));
+        RDT_TRY(need(w->lo_a, "lo_a"));
+        RDT_TRY(need(w->lo_b, "lo_b"));
+    }
+
+    // ---- device and stability check (rho(A) = max |A_i| < 1, no clipping)
+    int dev = 0;
+    RDT_CUDA_TRY(cudaGetDevice(&dev));
+    cudaDeviceProp prop;
+    RDT_CUDA_TRY(cudaGetDeviceProperties(&prop, dev));
+    if (prop.major != 10) {
+        set_error("an sm_100 (B200-class) device is required");
+        return RDT_ERR_UNSUPPORTED;
+    }
+    {
+        std::vector<float> a(d);
+        RDT_CUDA_TRY(cudaMemcpy(a.data(), w->A, d * sizeof(float), cudaMemcpyDeviceToHost));
+        float rho = 0.0f;
+        for (float v : a) {
+            if (!std::isfinite(v)) {
+                set_error("A has a non-finite entry");
+                return RDT_ERR_UNSTABLE_A;
+            }
+            rho = std::max(rho, std::fabs(v));
+        }
+        h->rho = rho;
+        if (rho >= 1.0f) {
+            set_error("rho(A) = " + std::to_string(rho) + " >= 1: the loop would not be stable");
+            return RDT_ERR_UNSTABLE_A;
+        }
+    }
+
+    // ---- weights
+    RDT_TRY(dev_alloc(h, &h->A, d * 4));
+    RDT_TRY(copy_d2d(h->A, w->A, d * 4, st));
+    const size_t bsz = c.b_kind == RDT_B_DIAG ? d * 4 : static_cast<size_t>(d) * d * 4;
+    RDT_TRY(dev_alloc(h, &h->Bw, bsz));
+    RDT_TRY(copy_d2d(h->Bw, w->B, bsz, st));
+    RDT_TRY(dev_alloc(h, &h->g1, d * 4));
+    RDT_TRY(copy_d2d(h->g1, w->norm1, d * 4, st));
+    RDT_TRY(dev_alloc(h, &h->g2, d * 4));
+    RDT_TRY(copy_d2d(h->g2, w->norm2, d * 4, st));
+    RDT_TRY(dev_alloc(h, &h->wr, static_cast<size_t>(E) * d * es));
+    RDT_TRY(copy_d2d(h->wr, w->w_router, static_cast<size_t>(E) * d * es, st));
+    if (w->router_bias) {
+        RDT_TRY(dev_alloc(h, &h->rbias, E * 4));
+        RDT_TRY(copy_d2d(h->rbias, w->router_bias, E * 4, st));
+    }
+    const size_t wexp = static_cast<size_t>(hid) * d * es;   // one expert matrix
+    RDT_TRY(dev_alloc(h, &h->w13, 2 * wexp * (E + S)));
+    RDT_TRY(dev_alloc(h, &h->w2, wexp * (E + S)));
+    for (int e = 0; e < E; ++e) {
+        RDT_TRY(interleave_w13(static_cast<char*>(h->w13) + 2 * wexp * e,
+                               static_cast<const char*>(w->w1) + wexp * e,
+                               static_cast<const char*>(w->w3) + wexp * e, hid, d, es, st));
+    }
+    RDT_TRY(copy_d2d(h->w2, w->w2, wexp * E, st));
+    for (int s = 0; s < S; ++s) {
+        RDT_TRY(interleave_w13(static_cast<char*>(h->w13) + 2 * wexp * (E + s),
+                               static_cast<const char*>(w->ws1) + wexp * s,
+                               static_cast<const char*>(w->ws3) + wexp * s, hid, d, es, st));
+    }
+    if (S) RDT_TRY(copy_d2d(static_cast<char*>(h->w2) + wexp * E, w->ws2, wexp * S, st));
+
+    if (c.attn_type == RDT_GQA) {
+        h->nq = c.n_heads * c.head_dim;
+        h->nkv = c.n_kv_heads * c.head_dim;
+        h->nqkv = h->nq + 2 * h->nkv;
+        h->owidth = h->nq;
+        h->rot = c.head_dim;
+        RDT_TRY(dev_alloc(h, &h->wqkv, static_cast<size_t>(h->nqkv) * d * es));
+        char* q = static_cast<char*>(h->wqkv);
+        RDT_TRY(copy_d2d(q, w->wq, static_cast<size_t>(h->nq) * d * es, st));
+        RDT_TRY(copy_d2d(q + static_cast<size_t>(h->nq) * d * es, w->wk, static_cast<size_t>(h->nkv) * d * es, st));
+        RDT_TRY(copy_d2d(q + static_cast<size_t>(h->nq + h->nkv) * d * es, w->wv,
+                         static_cast<size_t>(h->nkv) * d * es, st));
+        RDT_TRY(dev_alloc(h, &h->wo, static_cast<size_t>(d) * h->nq * es));
+        RDT_TRY(copy_d2d(h->wo, w->wo, static_cast<size_t>(d) * h->nq * es, st));
+        if (c.n_lora) {
+            const int L = c.n_lora, r = c.lora_rank, kx = h->kext;
+            RDT_TRY(dev_alloc(h, &h->lqa, static_cast<size_t>(L) * r * d * es));
+            RDT_TRY(copy_d2d(h->lqa, w->lq_a, static_cast<size_t>(L) * r * d * es, st));
+            RDT_TRY(dev_alloc(h, &h->loa, static_cast<size_t>(L) * r * h->nq * es));
+            RDT_TRY(copy_d2d(h->loa, w->lo_a, static_cast<size_t>(L) * r * h->nq * es, st));
+            RDT_TRY(dev_alloc(h, &h->lqb, static_cast<size_t>(L) * h->nqkv * kx * es, true));
+            RDT_TRY(dev_alloc(h, &h->lob, static_cast<size_t>(L) * d * kx * es, true));
+            for (int l = 0; l < L; ++l) {
+                RDT_CUDA_TRY(cudaMemcpy2DAsync(static_cast<char*>(h->lqb) + static_cast<size_t>(l) * h->nqkv * kx * es,
+                                               kx * es,
+                                               static_cast<const char*>(w->lq_b) + static_cast<size_t>(l) * h->nq * r * es,
+                                               r * es, r * es, h->nq, cudaMemcpyDeviceToDevice, st));
+                RDT_CUDA_TRY(cudaMemcpy2DAsync(static_cast<char*>(h->lob) + static_cast<size_t>(l) * d * kx * es,
+                                               kx * es,
+                                               static_cast<const char*>(w->lo_b) + static_cast<size_t>(l) * d * r * es,
+                                               r * es, r * es, d, cudaMemcpyDeviceToDevice, st));
+            }
+        }
+    } else {
+        const int H = c.n_heads, ql = c.q_lora_rank, kvl = c.kv_lora_rank, rp = c.qk_rope_dim;
+        const int nope = c.qk_nope_dim, vd = c.v_head_dim;
+        h->lat_w = ql + kvl + rp;
+        h->qt_w = H * (kvl + rp);
+        h->owidth = H * kvl;
+        h->rot = rp;
+        RDT_TRY(dev_alloc(h, &h->q_norm, ql * 4));
+        RDT_TRY(copy_d2d(h->q_norm, w->q_norm, ql * 4, st));
+        RDT_TRY(dev_alloc(h, &h->kv_norm, kvl * 4));
+        RDT_TRY(copy_d2d(h->kv_norm, w->kv_norm, kvl * 4, st));
+        // [W_dq; W_dkv; W_kr] -> one latent projection
+        RDT_TRY(dev_alloc(h, &h->wlat, static_cast<size_t>(h->lat_w) * d * es));
+        char* wl = static_cast<char*>(h->wlat);
+        RDT_TRY(copy_d2d(wl, w->w_dq, static_cast<size_t>(ql) * d * es, st));
+        RDT_TRY(copy_d2d(wl + static_cast<size_t>(ql) * d * es, w->w_dkv, static_cast<size_t>(kvl) * d * es, st));
+        RDT_TRY(copy_d2d(wl + static_cast<size_t>(ql + kvl) * d * es, w->w_kr, static_cast<size_t>(rp) * d * es, st));
+        // absorbed query projection, per head: rows [0, kvl) = W_uk,h^T W_uq_nope,h;
+        // rows [kvl, kvl + rope) = W_uq_rope,h
+        RDT_TRY(dev_alloc(h, &h->wqabs, static_cast<size_t>(h->qt_w) * ql * es));
+        for (int hh = 0; hh < H; ++hh) {
+            const char* uk = static_cast<const char*>(w->w_uk) + static_cast<size_t>(hh) * nope * kvl * es;
+            const char* uq = static_cast<const char*>(w->w_uq) + static_cast<size_t>(hh) * (nope + rp) * ql * es;
+            char* dst = static_cast<char*>(h->wqabs) + static_cast<size_t>(hh) * (kvl + rp) * ql * es;
+            RDT_TRY(prep_matmul(h->bf, uk, 1, kvl, uq, ql, 1, dst, ql, kvl, ql, nope, st));
+            RDT_TRY(copy_d2d(dst + static_cast<size_t>(kvl) * ql * es, uq + static_cast<size_t>(nope) * ql * es,
+                             static_cast<size_t>(rp) * ql * es, st));
+        }
+        // absorbed output projection: W_o~[:, h*kvl + c] = sum_v W_o[:, h*vd + v] W_uv[h*vd + v, c]
+        RDT_TRY(dev_alloc(h, &h->wo, static_cast<size_t>(d) * h->owidth * es));
+        for (int hh = 0; hh < H; ++hh) {
+            const char* wo = static_cast<const char*>(w->wo) + static_cast<size_t>(hh) * vd * es;
+            const char* uv = static_cast<const char*>(w->w_uv) + static_cast<size_t>(hh) * vd * kvl * es;
+            char* dst = static_cast<char*>(h->wo) + static_cast<size_t>(hh) * kvl * es;
+            RDT_TRY(prep_matmul(h->bf, wo, static_cast<long>(H) * vd, 1, uv, kvl, 1, dst, h->owidth, d, kvl, vd, st));
+        }
+    }
+
+    // RoPE tables [seq, rot/2] from double-precision angles
+    {
+        const int half = h->rot / 2;
+        std::vector<float> cs(static_cast<size_t>(c.seq) * half), sn(cs.size());
+        for (int p = 0; p < c.seq; ++p)
+            for (int i = 0; i < half; ++i) {
+                const double ang = p * std::pow(static_cast<double>(c.rope_base), -2.0 * i / h->rot);
+                cs[static_cast<size_t>(p) * half + i] = static_cast<float>(std::cos(ang));
+                sn[static_cast<size_t>(p) * half + i] = static_cast<float>(std::sin(ang));
+            }
+        RDT_TRY(dev_alloc(h, &h->rope_cos, cs.size() * 4));
+        RDT_TRY(dev_alloc(h, &h->rope_sin, sn.size() * 4));
+        RDT_CUDA_TRY(cudaMemcpy(h->rope_cos, cs.data(), cs.size() * 4, cudaMemcpyHostToDevice));
+        RDT_CUDA_TRY(cudaMemcpy(h->rope_sin, sn.data(), sn.size() * 4, cudaMemcpyHostToDevice));
+    }
+
+    // ---- workspace
+    const size_t nd = static_cast<size_t>(N) * d;
+    RDT_TRY(dev_alloc(h, &h->hbuf[0], nd * 4));
+    RDT_TRY(dev_alloc(h, &h->hbuf[1], nd * 4));
+    RDT_TRY(dev_alloc(h, &h->Be, nd * 4));
+    RDT_TRY(dev_alloc(h, &h->y, nd * 4));
+    RDT_TRY(dev_alloc(h, &h->xn, nd * es));
+    if (c.n_lora) {
+        RDT_TRY(dev_alloc(h, &h->tq, static_cast<size_t>(N) * h->kext * es, true));
+        RDT_TRY(dev_alloc(h, &h->to, static_cast<size_t>(N) * h->kext * es, true));
+    }
+    if (c.attn_type == RDT_GQA) {
+        RDT_TRY(dev_alloc(h, &h->qkv, static_cast<size_t>(N) * h->nqkv * es));
+    } else {
+        RDT_TRY(dev_alloc(h, &h->lat, static_cast<size_t>(N) * h->lat_w * 4));
+        RDT_TRY(dev_alloc(h, &h->cq, static_cast<size_t>(N) * c.q_lora_rank * es));
+        RDT_TRY(dev_alloc(h, &h->kvlat, static_cast<size_t>(N) * (c.kv_lora_rank + c.qk_rope_dim) * es));
+        RDT_TRY(dev_alloc(h, &h->qkv, static_cast<size_t>(N) * h->qt_w * es));
+    }
+    RDT_TRY(dev_alloc(h, &h->o, static_cast<size_t>(N) * h->owidth * es));
+    RDT_TRY(dev_alloc(h, &h->xperm, static_cast<size_t>(N) * (1 + K) * d * es, true));
+    RDT_TRY(dev_alloc(h, &h->U, static_cast<size_t>(N) * (S + K) * hid * es, true));
+    RDT_TRY(dev_alloc(h, &h->idx, static_cast<size_t>(N) * K * 4));
+    RDT_TRY(dev_alloc(h, &h->wts, static_cast<size_t>(N) * K * 4));
+    RDT_TRY(dev_alloc(h, &h->counts, 256 * 4, true));
+    RDT_TRY(dev_alloc(h, &h->offsets, 256 * 4, true));
+    RDT_TRY(dev_alloc(h, &h->fill, 256 * 4, true));
+    RDT_TRY(dev_alloc(h, &h->ntiles, 16, true));
+    RDT_TRY(dev_alloc(h, &h->row_token, static_cast<size_t>(N) * K * 4));
+    RDT_TRY(dev_alloc(h, &h->row_w, static_cast<size_t>(N) * K * 4));
+    h->max_tiles = (N * K + 127) / 128 + E + S * ((N + 127) / 128);
+    RDT_TRY(dev_alloc(h, &h->tiles, static_cast<size_t>(h->max_tiles) * sizeof(GroupTile), true));
+    RDT_TRY(dev_alloc(h, &h->flags, FLAG_COUNT * 4, true));
+    RDT_TRY(dev_alloc(h, &h->stage_h0, nd * es));
+    RDT_TRY(dev_alloc(h, &h->stage_e, nd * es));
+    RDT_TRY(dev_alloc(h, &h->stage_out, nd * 4));
+
+    RDT_TRY(build_maps(h));
+    RDT_CUDA_TRY(cudaStreamSynchronize(st));
+    return RDT_OK;
+}
+
+int lora_index(const rdt_handle* h, int t) { return std::min(t, h->cfg.n_lora - 1); }
+
+// ---- the attention sublayer: norm1 -> projections -> attention -> O projection
+rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t, bool loop_mode,
+                           float* a_out, float* h_next, cudaStream_t st) {
+    const rdt_config& c = h->cfg;
+    const int N = h->ntok, d = c.dim;
+    const bool lora = c.n_lora > 0;
+    const int li = lora ? lora_index(h, t) : 0;
+
+    Norm1Args n1{};
+    n1.h = hin;
+    n1.e = e;
+    n1.gamma = h->g1;
+    n1.xn = h->xn;
+    n1.ntok = N;
+    n1.dim = d;
+    n1.eps = c.norm_eps;
+    if (lora) {
+        n1.lora_a = static_cast<const char*>(h->lqa) + static_cast<size_t>(li) * c.lora_rank * d * h->esz;
+        n1.lora_r = c.lora_rank;
+        n1.lora_t = h->tq;
+    }
+    if (loop_mode) {
+        n1.zero_counts = h->counts;
+        n1.n_zero = h->G;
+    }
+    RDT_TRY(norm1(h->bf, n1, st));
+
+    GemmArgs ga{};
+    ga.M = N;
+    ga.flags = h->flags;
+    EpiParams ep{};
+    ep.flags = h->flags;
+    AttnArgs at{};
+    at.batch = c.batch;
+    at.seq = c.seq;
+    at.hq = c.n_heads;
+    at.o = h->o;
+    at.ldo = h->owidth;
+    if (c.attn_type == RDT_GQA) {
+        ga.N = h->nqkv;
+        ga.kb_main = static_cast<int>(d * h->esz / 128);
+        ga.kb_ext = lora ? 1 : 0;
+        ga.b2_row0 = li * h->nqkv;
+        ep.kind = EPI_ROPE;
+        ep.out = h->qkv;
+        ep.ldo = h->nqkv;
+        ep.ncols_valid = h->nqkv;
+        ep.rope_cos = h->rope_cos;
+        ep.rope_sin = h->rope_sin;
+        ep.seq = c.seq;
+        ep.head_w = c.head_dim;
+        ep.rot_off = 0;
+        ep.rot_dim = c.head_dim;
+        ep.rope_limit = h->nq + h->nkv;
+        RDT_TRY(gemm_tc(h->bf, 128, h->m_xn, h->m_wqkv, lora ? &h->m_tq : nullptr,
+                        lora ? &h->m_lqb : nullptr, ga, ep, st));
+        at.q = h->qkv;
+        at.ldq = h->nqkv;
+        at.q_hstride = c.head_dim;
+        at.k = static_cast<const char*>(h->qkv) + static_cast<size_t>(h->nq) * h->esz;
+        at.ldk = h->nqkv;
+        at.k_hstride = c.head_dim;
+        at.v = static_cast<const char*>(h->qkv) + static_cast<size_t>(h->nq + h->nkv) * h->esz;
+        at.ldv = h->nqkv;
+        at.v_hstride = c.head_dim;
+        at.hkv = c.n_kv_heads;
+        at.dqk = c.head_dim;
+        at.dv = c.head_dim;
+        at.scale = 1.0f / std::sqrt(static_cast<float>(c.head_dim));
+    } else {
+        const int ql = c.q_lora_rank, kvl = c.kv_lora_rank, rp = c.qk_rope_dim;
+        // latent projection -> fp32 [N, ql + kvl + rope]
+        ga.N = h->lat_w;
+        ga.kb_main = static_cast<int>(d * h->esz / 128);
+        ep.kind = EPI_STORE_F32;
+        ep.out = h->lat;
+        ep.ldo = h->lat_w;
+        ep.ncols_valid = h->lat_w;
+        RDT_TRY(gemm_tc(h->bf, 128, h->m_xn, h->m_wlat, nullptr, nullptr, ga, ep, st));
+        MlaNormArgs mn{};
+        mn.lat = h->lat;
+        mn.ld_lat = h->lat_w;
+        mn.q_norm = h->q_norm;
+        mn.kv_norm = h->kv_norm;
+        mn.cq = h->cq;
+        mn.kv = h->kvlat;
+        mn.rope_cos = h->rope_cos;
+        mn.rope_sin = h->rope_sin;
+        mn.ntok = N;
+        mn.seq = c.seq;
+        mn.q_lat = ql;
+        mn.kv_lat = kvl;
+        mn.rope = rp;
+        mn.eps = c.norm_eps;
+        RDT_TRY(mla_latent_norm(h->bf, mn, st));
+        // absorbed query projection with RoPE on the last rope columns of each head
+        GemmArgs gq{};
+        gq.M = N;
+        gq.N = h->qt_w;
+        gq.kb_main = static_cast<int>(ql * h->esz / 128);
+        gq.flags = h->flags;
+        EpiParams eq{};
+        eq.flags = h->flags;
+        eq.kind = EPI_ROPE;
+        eq.out = h->qkv;
+        eq.ldo = h->qt_w;
+        eq.ncols_valid = h->qt_w;
+        eq.rope_cos = h->rope_cos;
+        eq.rope_sin = h->rope_sin;
+        eq.seq = c.seq;
+        eq.head_w = kvl + rp;
+        eq.rot_off = kvl;
+        eq.rot_dim = rp;
+        eq.rope_limit = h->qt_w;
+        RDT_TRY(gemm_tc(h->bf, 160, h->m_cq, h->m_wqabs, nullptr, nullptr, gq, eq, st));
+        at.q = h->qkv;
+        at.ldq = h->qt_w;
+        at.q_hstride = kvl + rp;
+        at.k = h->kvlat;
+        at.ldk = kvl + rp;
+        at.k_hstride = 0;
+        at.v = h->kvlat;
+        at.ldv = kvl + rp;
+        at.v_hstride = 0;
+        at.hkv = 1;
+        at.dqk = kvl + rp;
+        at.dv = kvl;
+        at.scale = 1.0f / std::sqrt(static_cast<float>(c.qk_nope_dim + rp));
+    }
+    RDT_TRY(attention(h->bf, at, st));
+
+    if (lora) {
+        const void* A = static_cast<const char*>(h->loa) + static_cast<size_t>(li) * c.lora_rank * h->nq * h->esz;
+        RDT_TRY(lora_down(h->bf, h->o, h->owidth, N, h->owidth, A, c.lora_rank, h->to, st));
+    }
+    GemmArgs go{};
+    go.M = N;
+    go.N = d;
+    go.kb_main = static_cast<int>(h->owidth * h->esz / 128);
+    go.kb_ext = lora ? 1 : 0;
+    go.b2_row0 = li * d;
+    go.flags = h->flags;
+    EpiParams eo{};
+    eo.flags = h->flags;
+    eo.ncols_valid = d;
+    if (loop_mode) {
+        eo.kind = EPI_OPROJ_LOOP;
+        eo.h = hin;
+        eo.e = c.inject_e ? e : nullptr;
+        eo.Be = h->Be;
+        eo.Adiag = h->A;
+        eo.y = h->y;
+        eo.h_next = h_next;
+        eo.ld = d;
+    } else {
+        eo.kind = EPI_OPROJ_PLAIN;
+        eo.out = a_out;
+        eo.ldo = d;
+    }
+    RDT_TRY(gemm_tc(h->bf, 128, h->m_o, h->m_wo, lora ? &h->m_to : nullptr, lora ? &h->m_lob : nullptr,
+                    go, eo, st));
+    return RDT_OK;
+}
+
+// ---- the MoE sublayer: norm2 + router -> dispatch -> experts; adds into dst
+rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_out, float* w_out,
+                     int32_t* tr_idx, float* tr_w, cudaStream_t st) {
+    const rdt_config& c = h->cfg;
+    const int N = h->ntok, d = c.dim, hid = c.expert_hidden;
+    RouterArgs ra{};
+    ra.y = yin;
+    ra.gamma = h->g2;
+    ra.yn = h->xperm;
+    ra.ntok = N;
+    ra.dim = d;
+    ra.eps = c.norm_eps;
+    ra.w_router = h->wr;
+    ra.bias = h->rbias;
+    ra.n_exp = c.n_experts;
+    ra.top_k = c.top_k;
+    ra.idx = idx_out ? idx_out : h->idx;
+    ra.w = w_out ? w_out : h->wts;
+    ra.counts = h->counts;
+    ra.trace_idx = tr_idx;
+    ra.trace_w = tr_w;
+    RDT_TRY(norm2_router(h->bf, ra, st));
+
+    DispatchArgs da{};
+    da.counts = h->counts;
+    da.n_exp = c.n_experts;
+    da.n_shared = c.n_shared;
+    da.ntok = N;
+    da.top_k = c.top_k;
+    da.dim = d;
+    da.offsets = h->offsets;
+    da.fill = h->fill;
+    da.tiles = h->tiles;
+    da.n_tiles = h->ntiles;
+    da.max_tiles = h->max_tiles;
+    da.idx = ra.idx;
+    da.w = ra.w;
+    da.xperm = h->xperm;
+    da.row_token = h->row_token;
+    da.row_w = h->row_w;
+    RDT_TRY(moe_dispatch(h->bf, da, st));
+
+    GemmArgs gu{};
+    gu.N = 2 * hid;
+    gu.kb_main = static_cast<int>(d * h->esz / 128);
+    gu.tiles = h->tiles;
+    gu.n_tiles = h->ntiles;
+    gu.max_tiles = h->max_tiles;
+    gu.flags = h->flags;
+    EpiParams eu{};
+    eu.kind = EPI_SWIGLU;
+    eu.out = h->U;
+    eu.ldo = hid;
+    eu.ncols_valid = 2 * hid;
+    eu.flags = h->flags;
+    RDT_TRY(gemm_tc(h->bf, 128, h->m_xperm, h->m_w13, nullptr, nullptr, gu, eu, st));
+
+    GemmArgs gd{};
+    gd.N = d;
+    gd.kb_main = static_cast<int>(hid * h->esz / 128);
+    gd.tiles = h->tiles;
+    gd.n_tiles = h->ntiles;
+    gd.max_tiles = h->max_tiles;
+    gd.a_from_c = 1;
+    gd.flags = h->flags;
+    EpiParams ed{};
+    ed.kind = EPI_SCATTER;
+    ed.ncols_valid = d;
+    ed.row_token = h->row_token;
+    ed.row_w = h->row_w;
+    ed.shared_rows = c.n_shared * N;
+    ed.ntok = N;
+    ed.dst = dst;
+    ed.ld = d;
+    ed.flags = h->flags;
+    RDT_TRY(gemm_tc(h->bf, 128, h->m_U, h->m_w2, nullptr, nullptr, gd, ed, st));
+    return RDT_OK;
+}
+
+rdt_status loop_impl(rdt_handle* h, const void* h0, const void* e, int T, float* out, cudaStream_t st) {
+    const rdt_config& c = h->cfg;
+    const int N = h->ntok, d = c.dim;
+    const size_t nd = static_cast<size_t>(N) * d;
+    RDT_TRY(hoist(h->bf, h0, e, c.b_kind == RDT_B_DIAG ? h->Bw : nullptr, h->hbuf[0], h->Be, nd, d, st));
+    if (c.b_kind == RDT_B_DENSE) RDT_TRY(matmul_nt_simt(h->bf, e, h->Bw, h->Be, N, d, d, st));
+    if (h->tr_h) RDT_CUDA_TRY(cudaMemcpyAsync(h->tr_h, h->hbuf[0], nd * 4, cudaMemcpyDeviceToDevice, st));
+    for (int t = 0; t < T; ++t) {
+        float* hcur = h->hbuf[t & 1];
+        float* hnext = (t == T - 1) ? out : h->hbuf[(t + 1) & 1];
+        RDT_TRY(attention_block(h, hcur, c.inject_e ? e : nullptr, t, true, nullptr, hnext, st));
+        const size_t tk = static_cast<size_t>(t) * N * c.top_k;
+        RDT_TRY(moe_block(h, h->y, hnext, nullptr, nullptr, h->tr_idx ? h->tr_idx + tk : nullptr,
+                          h->tr_w ? h->tr_w + tk : nullptr, st));
+        if (h->tr_h)
+            RDT_CUDA_TRY(cudaMemcpyAsync(h->tr_h + (t + 1) * nd, hnext, nd * 4, cudaMemcpyDeviceToDevice, st));
+    }
+    RDT_TRY(check_finite(out, nd, h->flags, st));
+    return RDT_OK;
+}
+
+}  // namespace
+
+// =====================================================================================
+// C ABI
+// =====================================================================================
+
+extern "C" {
+
+const char* rdt_status_string(rdt_status s) {
+    switch (s) {
+        case RDT_OK: return "ok";
+        case RDT_ERR_INVALID_ARG: return "invalid argument";
+        case RDT_ERR_UNSUPPORTED: return "unsupported configuration or device";
+        case RDT_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case RDT_ERR_UNSTABLE_A: return "rho(A) >= 1";
+        case RDT_ERR_OOM: return "out of device memory";
+        case RDT_ERR_CUDA: return "CUDA error";
+        case RDT_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        case RDT_ERR_NONFINITE: return "non-finite value in the state";
+    }
+    return "unknown status";
+}
+
+const char* rdt_last_error(void) { return g_last_error.c_str(); }
+
+rdt_status rdt_create(const rdt_config* cfg, const rdt_weights* w, void* stream, rdt_handle** out) {
+    if (!out) {
+        set_error("out is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    *out = nullptr;
+    RDT_TRY(validate_config(cfg));
+    if (!w) {
+        set_error("weights is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    rdt_handle* h = new rdt_handle();
+    const rdt_status s = create_impl(cfg, w, static_cast<cudaStream_t>(stream), h);
+    if (s != RDT_OK) {
+        rdt_destroy(h);
+        return s;
+    }
+    *out = h;
+    return RDT_OK;
+}
+
+static rdt_status check_ptr(const void* p, const char* name) {
+    if (!p) {
+        set_error(std::string(name) + " is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (!aligned16(p)) {
+        set_error(std::string(name) + " is not 16-byte aligned");
+        return RDT_ERR_MISALIGNED;
+    }
+    return RDT_OK;
+}
+
+rdt_status rdt_attn_forward(rdt_handle* h, const float* x, int loop, float* a_out, void* stream) {
+    if (!h) {
+        set_error("handle is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    RDT_TRY(check_ptr(x, "x"));
+    RDT_TRY(check_ptr(a_out, "a_out"));
+    if (loop < 0) {
+        set_error("loop must be >= 0");
+        return RDT_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    h->last_stream = st;
+    return attention_block(h, x, nullptr, loop, false, a_out, nullptr, st);
+}
+
+rdt_status rdt_moe_forward(rdt_handle* h, const float* y, float* f_out, int32_t* topk_idx, float* topk_w,
+                           void* stream) {
+    if (!h) {
+        set_error("handle is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    RDT_TRY(check_ptr(y, "y"));
+    RDT_TRY(check_ptr(f_out, "f_out"));
+    if (topk_idx) RDT_TRY(check_ptr(topk_idx, "topk_idx"));
+    if (topk_w) RDT_TRY(check_ptr(topk_w, "topk_w"));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    h->last_stream = st;
+    const size_t nd = static_cast<size_t>(h->ntok) * h->cfg.dim;
+    RDT_CUDA_TRY(cudaMemsetAsync(f_out, 0, nd * 4, st));
+    RDT_CUDA_TRY(cudaMemsetAsync(h->counts, 0, 256 * 4, st));
+    return moe_block(h, y, f_out, topk_idx, topk_w, nullptr, nullptr, st);
+}
+
+rdt_status rdt_loop_forward(rdt_handle* h, const void* h0, const void* e, int T, float* out, void* stream) {
+    if (!h) {
+        set_error("handle is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    RDT_TRY(check_ptr(h0, "h0"));
+    RDT_TRY(check_ptr(e, "e"));
+    RDT_TRY(check_ptr(out, "out"));
+    if (T < 1 || T > h->cfg.max_loops) {
+        set_error("T must be in [1, max_loops]");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (out == e) {
+        set_error("out must not alias e (e is read in every loop)");
+        return RDT_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    h->last_stream = st;
+    return loop_impl(h, h0, e, T, out, st);
+}
+
+rdt_status rdt_loop_forward_host(rdt_handle* h, const void* h0_host, const void* e_host, int T, float* out_host,
+                                 void* stream) {
+    if (!h) {
+        set_error("handle is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (!h0_host || !e_host || !out_host) {
+        set_error("host buffers must be non-NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (T < 1 || T > h->cfg.max_loops) {
+        set_error("T must be in [1, max_loops]");
+        return RDT_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    h->last_stream = st;
+    const size_t nd = static_cast<size_t>(h->ntok) * h->cfg.dim;
+    RDT_CUDA_TRY(cudaMemcpyAsync(h->stage_e, e_host, nd * h->esz, cudaMemcpyHostToDevice, st));
+    const void* h0d = h->stage_e;
+    if (h0_host != e_host) {
+        RDT_CUDA_TRY(cudaMemcpyAsync(h->stage_h0, h0_host, nd * h->esz, cudaMemcpyHostToDevice, st));
+        h0d = h->stage_h0;
+    }
+    RDT_TRY(loop_impl(h, h0d, h->stage_e, T, h->stage_out, st));
+    RDT_CUDA_TRY(cudaMemcpyAsync(out_host, h->stage_out, nd * 4, cudaMemcpyDeviceToHost, st));
+    RDT_CUDA_TRY(cudaStreamSynchronize(st));
+    return RDT_OK;
+}
+
+rdt_status rdt_matmul(int32_t dtype, const void* A, const void* B, float* C, int M, int N, int K,
+                      void* stream) {
+    if (dtype != RDT_BF16 && dtype != RDT_F32) {
+        set_error("dtype must be RDT_BF16 or RDT_F32");
+        return RDT_ERR_INVALID_ARG;
+    }
+    RDT_TRY(check_ptr(A, "A"));
+    RDT_TRY(check_ptr(B, "B"));
+    RDT_TRY(check_ptr(C, "C"));
+    const bool bf = dtype == RDT_BF16;
+    const int es = bf ? 2 : 4;
+    if (M < 1 || N < 32 || K < 1 || N % 32 || (static_cast<long>(K) * es) % 128) {
+        set_error("matmul: need M >= 1, N % 32 == 0, K * element size % 128 == 0");
+        return RDT_ERR_UNSUPPORTED;
+    }
+    CUtensorMap ta, tb;
+    const uint32_t kbox = 128 / es;
+    RDT_TRY(make_tmap_2d(&ta, A, bf, K, M, static_cast<uint64_t>(K) * es, kbox, 128));
+    RDT_TRY(make_tmap_2d(&tb, B, bf, K, N, static_cast<uint64_t>(K) * es, kbox, 128));
+    GemmArgs ga{};
+    ga.M = M;
+    ga.N = N;
+    ga.kb_main = static_cast<int>(static_cast<long>(K) * es / 128);
+    EpiParams ep{};
+    ep.kind = EPI_STORE_F32;
+    ep.out = C;
+    ep.ldo = N;
+    ep.ncols_valid = N;
+    return gemm_tc(bf, 128, ta, tb, nullptr, nullptr, ga, ep, static_cast<cudaStream_t>(stream));
+}
+
+rdt_status rdt_attention(int32_t dtype, const void* q, const void* k, const void* v, void* o,
+                         int batch, int seq, int n_heads, int n_kv_heads, int dqk, int dv,
+                         float scale, void* stream) {
+    if (dtype != RDT_BF16 && dtype != RDT_F32) {
+        set_error("dtype must be RDT_BF16 or RDT_F32");
+        return RDT_ERR_INVALID_ARG;
+    }
+    RDT_TRY(check_ptr(q, "q"));
+    RDT_TRY(check_ptr(k, "k"));
+    RDT_TRY(check_ptr(v, "v"));
+    RDT_TRY(check_ptr(o, "o"));
+    if (batch < 1 || seq < 1 || n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads) {
+        set_error("attention: bad sizes");
+        return RDT_ERR_INVALID_ARG;
+    }
+    AttnArgs a{};
+    a.q = q; a.ldq = n_heads * dqk; a.q_hstride = dqk;
+    a.k = k; a.ldk = n_kv_heads * dqk; a.k_hstride = dqk;
+    a.v = v; a.ldv = n_kv_heads * dv; a.v_hstride = dv;
+    a.o = o; a.ldo = n_heads * dv;
+    a.batch = batch; a.seq = seq; a.hq = n_heads; a.hkv = n_kv_heads; a.dqk = dqk; a.dv = dv;
+    a.scale = scale;
+    return attention(dtype == RDT_BF16, a, static_cast<cudaStream_t>(stream));
+}
+
+rdt_status rdt_set_trace(rdt_handle* h, int32_t* idx, float* w, float* h_traj) {
+    if (!h) {
+        set_error("handle is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if ((idx && !aligned16(idx)) || (w && !aligned16(w)) || (h_traj && !aligned16(h_traj))) {
+        set_error("trace buffers must be 16-byte aligned");
+        return RDT_ERR_MISALIGNED;
+    }
+    h->tr_idx = idx;
+    h->tr_w = w;
+    h->tr_h = h_traj;
+    return RDT_OK;
+}
+
+rdt_status rdt_get_diagnostics(rdt_handle* h, rdt_diag* out) {
+    if (!h || !out) {
+        set_error("handle or out is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    RDT_CUDA_TRY(cudaStreamSynchronize(h->last_stream));
+    int flags[FLAG_COUNT];
+    RDT_CUDA_TRY(cudaMemcpy(flags, h->flags, sizeof(flags), cudaMemcpyDeviceToHost));
+    std::memset(out, 0, sizeof(*out));
+    out->rho_A = h->rho;
+    out->nonfinite = flags[FLAG_NONFINITE];
+    out->timeout = flags[FLAG_TIMEOUT];
+    int counts[256];
+    RDT_CUDA_TRY(cudaMemcpy(counts, h->counts, sizeof(counts), cudaMemcpyDeviceToHost));
+    int tot = 0;
+    for (int i = 0; i < h->cfg.n_experts; ++i) {
+        out->expert_counts[i] = counts[i];
+        tot += counts[i];
+    }
+    for (int s = 0; s < h->cfg.n_shared; ++s) out->expert_counts[h->cfg.n_experts + s] = h->ntok;
+    out->last_routed_rows = tot;
+    return RDT_OK;
+}
+
+rdt_status rdt_memory_bytes(const rdt_handle* h, size_t* bytes) {
+    if (!h || !bytes) {
+        set_error("handle or bytes is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    *bytes = h->bytes;
+    return RDT_OK;
+}
+
+void rdt_destroy(rdt_handle* h) {
+    if (!h) return;
+    cudaDeviceSynchronize();
+    for (void* p : h->allocs) cudaFree(p);
+    delete h;
+}
+
+}  // extern "C"

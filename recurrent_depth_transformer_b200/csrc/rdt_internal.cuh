@@ -1,0 +1,378 @@
+// Internal declarations of librdt: device helpers (mbarrier, TMA, tcgen05 wrappers in
+// inline PTX for sm_100a) and the host launchers each .cu file provides.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/rdt.h"
+
+namespace rdt {
+
+using bf16 = __nv_bfloat16;
+
+// ------------------------------------------------------------------ error plumbing (host)
+
+void set_error(const std::string& msg);
+#define RDT_CUDA_TRY(expr)                                                                   \
+    do {                                                                                     \
+        cudaError_t _e = (expr);                                                             \
+        if (_e != cudaSuccess) {                                                             \
+            ::rdt::set_error(std::string(#expr) + ": " + cudaGetErrorString(_e));            \
+            return RDT_ERR_CUDA;                                                             \
+        }                                                                                    \
+    } while (0)
+#define RDT_TRY(expr)                                                                        \
+    do {                                                                                     \
+        rdt_status _s = (expr);                                                              \
+        if (_s != RDT_OK) return _s;                                                         \
+    } while (0)
+
+// Device-side status words (one int each, in a small device buffer).
+enum DevFlag { FLAG_NONFINITE = 0, FLAG_TIMEOUT = 1, FLAG_COUNT = 8 };
+
+// Bound on any single device-side wait before the kernel records a timeout and bails out.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
+
+// ------------------------------------------------------------------ small device helpers
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(bf16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ bf16 from_f<bf16>(float x) { return __float2bfloat16_rn(x); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Load 4 consecutive elements as fp32.
+__device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
+    float4 x = *reinterpret_cast<const float4*>(p);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+__device__ __forceinline__ void load4(const bf16* p, float (&v)[4]) {
+    uint2 x = *reinterpret_cast<const uint2*>(p);
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&x.x);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&x.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    v[0] = fa.x; v[1] = fa.y; v[2] = fb.x; v[3] = fb.y;
+}
+__device__ __forceinline__ void store4(float* p, const float (&v)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void store4(bf16* p, const float (&v)[4]) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+    uint2 x;
+    x.x = *reinterpret_cast<uint32_t*>(&a);
+    x.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = x;
+}
+
+// ------------------------------------------------------------------ mbarrier (sm_90+)
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Wait for the phase of parity `parity` to complete, at most kWaitLimitNs. On timeout
+// sets flags[FLAG_TIMEOUT] and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* flags) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 256; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            if (flags) atomicExch(flags + FLAG_TIMEOUT, 1);
+            return false;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ TMA (bulk tensor copies)
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+// 2-D tiled load global -> this CTA's shared memory, completion counted on `bar`.
+// x is the innermost (contiguous) coordinate in elements; it is always a multiple of the
+// 128-byte box width here, so the 16-byte alignment rule of tiled copies holds.
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m, uint64_t* bar,
+                                            int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+// ------------------------------------------------------------------ tcgen05 (5th-gen tensor cores)
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* smem_slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(smem_slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Arrive on `bar` once every tcgen05 operation this thread issued so far has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T, both K-major; kind::f16 (bf16 inputs, fp32 accumulate).
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+        : "memory");
+}
+// Same with kind::tf32 (fp32 operands read as tf32, fp32 accumulate).
+__device__ __forceinline__ void tc_mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+        : "memory");
+}
+// Warp-collective: lane i reads TMEM lane (base lane + i), 32 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major tile written by TMA with the 128-byte
+// swizzle: rows of 128 bytes, 8-row swizzle atoms 1024 bytes apart (stride byte offset),
+// leading byte offset unused for this layout, descriptor version 1 (sm_100), layout
+// code 2 (128-byte swizzle) in bits 61-63.
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(1) << 16;
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
+// Instruction descriptor: fp32 accumulator, A/B format (1 = bf16, 2 = tf32), both K-major,
+// N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+__host__ __device__ constexpr uint32_t make_idesc(int ab_format, int M, int N) {
+    return (1u << 4) | (static_cast<uint32_t>(ab_format) << 7) |
+           (static_cast<uint32_t>(ab_format) << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ host-side launchers
+
+// Tensor maps (driver entry point resolved once through the runtime).
+rdt_status make_tmap_2d(CUtensorMap* map, const void* base, bool bf16_elems, uint64_t inner,
+                        uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner,
+                        uint32_t box_rows);
+
+// One M-tile of a grouped (per-expert) GEMM.
+struct GroupTile {
+    int group;     // expert (routed 0..E-1, shared E..E+S-1)
+    int a_row0;    // first row of A for this tile
+    int c_row0;    // first output row
+    int nrows;     // valid rows (<= 128)
+};
+
+enum EpiKind {
+    EPI_STORE = 0,      // C[row, col] = acc                     (OutT)
+    EPI_ROPE = 1,       // C = acc with RoPE on the rotary part of rotated heads (OutT)
+    EPI_OPROJ_LOOP = 2, // y = x + acc, h_next = A*h + Be + acc   (fp32)
+    EPI_OPROJ_PLAIN = 3,// a_out = acc                             (fp32)
+    EPI_SWIGLU = 4,     // U[row, j] = silu(acc_gate) * acc_up    (OutT)
+    EPI_SCATTER = 5,    // dst[token, col] += w * acc             (fp32, vector atomics)
+    EPI_STORE_F32 = 6   // C[row, col] = acc                     (fp32)
+};
+
+struct EpiParams {
+    int kind;
+    void* out;             // EPI_STORE / ROPE / SWIGLU: output base; OPROJ_PLAIN: a_out
+    int ldo;               // row stride (elements) of `out`
+    int ncols_valid;       // N (columns beyond are not stored)
+    // RoPE
+    const float* rope_cos; // [seq, rot/2]
+    const float* rope_sin;
+    int seq;
+    int head_w;            // width of one head's columns (64 or 160)
+    int rot_off;           // rotary part starts at this column inside a head
+    int rot_dim;           // rotary width
+    int rope_limit;        // columns >= rope_limit are not rotated (V heads)
+    // O-projection loop epilogue
+    const float* h;        // state h_t
+    const void* e;         // injection input (cfg dtype) or NULL (x = h)
+    const float* Be;
+    const float* Adiag;
+    float* y;              // x + a
+    float* h_next;         // A*h + Be + a (the MoE adds its share later)
+    int ld;                // row stride of h, e, Be, y, h_next (= dim)
+    // scatter
+    const int* row_token;  // routed rows: token of each output row
+    const float* row_w;    // routed rows: gate weight
+    int shared_rows;       // rows [0, shared_rows) are shared-expert rows: token = row % ntok
+    int ntok;
+    float* dst;            // scatter destination [ntok, ld]
+    int* flags;            // device status words
+};
+
+struct GemmArgs {
+    int M;                 // rows of A / C (dense); unused for grouped
+    int N;                 // columns of C (= rows of B per group)
+    int kb_main;           // K blocks (128 bytes each) of A/B
+    int kb_ext;            // 0 or 1 extra K blocks from (A2, B2)
+    int b2_row0;           // row offset into B2 for the extension block
+    const GroupTile* tiles;// grouped: tile list (NULL = dense)
+    const int* n_tiles;    // grouped: number of valid tiles (device)
+    int max_tiles;         // grouped: grid size along M
+    int a_from_c;          // grouped: read A at the tile's output row (down projection)
+    int* flags;
+};
+
+// C = A B^T (+ extension) with the chosen epilogue, on tcgen05 tensor cores.
+// tA: [rows, K] box (128 B x 128 rows); tB: [Nrows, K] box (128 B x BN rows).
+rdt_status gemm_tc(bool bf16_elems, int bn, const CUtensorMap& tA, const CUtensorMap& tB,
+                   const CUtensorMap* tA2, const CUtensorMap* tB2, const GemmArgs& args,
+                   const EpiParams& epi, cudaStream_t st);
+
+// Causal attention. q rows [N, ldq], head h at column h*q_hstride; k/v similarly with
+// Hkv heads; o [N, ldo] head h at column h*dv.
+struct AttnArgs {
+    const void* q; int ldq; int q_hstride;
+    const void* k; int ldk; int k_hstride;
+    const void* v; int ldv; int v_hstride;
+    void* o; int ldo;
+    int batch, seq, hq, hkv, dqk, dv;
+    float scale;
+};
+rdt_status attention(bool bf16_elems, const AttnArgs& a, cudaStream_t st);
+
+// Row kernels (rowops.cu).
+struct Norm1Args {
+    const float* h;    // fp32 state, or the fp32 block input x when e == NULL
+    const void* e;     // cfg-dtype injection (x = h + e) or NULL
+    const float* gamma;
+    void* xn;          // [N, dim] cfg dtype
+    int ntok, dim; float eps;
+    const void* lora_a;   // [r, dim] adapter down-projection or NULL
+    int lora_r;
+    void* lora_t;         // [N, 64] cfg dtype, columns [0, r) written
+    int* zero_counts; int n_zero;   // counts to clear (next MoE), or NULL
+};
+rdt_status norm1(bool bf16_elems, const Norm1Args& a, cudaStream_t st);
+
+struct RouterArgs {
+    const float* y; const float* gamma; void* yn; int ntok, dim; float eps;
+    const void* w_router; const float* bias; int n_exp, top_k;
+    int32_t* idx; float* w; int* counts;
+    int32_t* trace_idx; float* trace_w;
+};
+rdt_status norm2_router(bool bf16_elems, const RouterArgs& a, cudaStream_t st);
+
+struct DispatchArgs {
+    const int* counts; int n_exp, n_shared, ntok, top_k, dim;
+    int* offsets; int* fill; GroupTile* tiles; int* n_tiles; int max_tiles;
+    const int32_t* idx; const float* w; void* xperm; int* row_token; float* row_w;
+};
+rdt_status moe_dispatch(bool bf16_elems, const DispatchArgs& a, cudaStream_t st);
+
+rdt_status lora_down(bool bf16_elems, const void* x, int ldx, int ntok, int width,
+                     const void* lora_a, int r, void* t_out, cudaStream_t st);
+
+rdt_status hoist(bool bf16_elems, const void* h0, const void* e, const float* Bdiag, float* h,
+                 float* Be, size_t n, int dim, cudaStream_t st);
+rdt_status matmul_nt_simt(bool a_bf16, const void* A, const float* B, float* C, int M, int N,
+                          int K, cudaStream_t st);
+
+struct MlaNormArgs {
+    const float* lat; int ld_lat;   // [N, q_lat + kv_lat + rope] fp32
+    const float* q_norm; const float* kv_norm;
+    void* cq;   // [N, q_lat]
+    void* kv;   // [N, kv_lat + rope]
+    const float* rope_cos; const float* rope_sin;
+    int ntok, seq, q_lat, kv_lat, rope; float eps;
+};
+rdt_status mla_latent_norm(bool bf16_elems, const MlaNormArgs& a, cudaStream_t st);
+
+// Weight preparation: C[m, n] = sum_k A(m, k) B(k, n) with A(m, k) = A[m*sam + k*sak] and
+// B(k, n) = B[k*sbk + n*sbn] (element type of the configuration), fp32 sums.
+rdt_status prep_matmul(bool bf16_elems, const void* A, long sam, long sak, const void* B, long sbk,
+                       long sbn, void* C, int ldc, int M, int N, int K, cudaStream_t st);
+rdt_status check_finite(const float* x, size_t n, int* flags, cudaStream_t st);
+
+}  // namespace rdt

@@ -1,0 +1,527 @@
+// Memory-bound row kernels of the recurrent block (one warp per token row, 16-byte
+// vectorised, coalesced across the warp):
+//   hoist          h <- h0 (fp32 state), Be <- B (.) e      (once per call)
+//   norm1          x = h + e, xn = RMSNorm1(x), optional LoRA-down t = xn A_t^T
+//   norm2_router   yn = RMSNorm2(y) (fp32 in registers, stored in the element type for the
+//                  experts), router logits yn W_r^T in fp32, top-k of logits + bias with
+//                  ties to the lower expert index, softmax over the k chosen logits,
+//                  per-expert histogram
+//   moe_dispatch   per-expert offsets and the grouped-GEMM tile list (device side), then
+//                  the scatter of each (token, slot) to its expert's rows
+//   lora_down      t = x A^T for the O-projection adapter
+//   mla_latent_norm  RMSNorm of c_q and c_kv, RoPE of the decoupled key
+// plus the weight-preparation matmul and a finite-value check.
+#include <algorithm>
+
+#include "rdt_internal.cuh"
+
+namespace rdt {
+namespace {
+
+constexpr int kRowThreads = 256;   // 8 rows (warps) per block
+
+template <typename T>
+__device__ __forceinline__ void store_t(T* p, float v) { *p = from_f<T>(v); }
+
+// ----------------------------------------------------------------------------- hoist
+
+template <typename T>
+__global__ void hoist_kernel(const T* h0, const T* e, const float* Bd, float* h, float* Be,
+                             size_t n4, int dim) {
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const size_t off = i * 4;
+        float a[4], b[4];
+        load4(h0 + off, a);
+        store4(h + off, a);
+        if (Bd) {
+            float bd[4];
+            load4(e + off, b);
+            load4(Bd + off % dim, bd);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] *= bd[j];
+            store4(Be + off, b);
+        }
+    }
+}
+
+// C[M,N] = A[M,K] B[N,K]^T, fp32 sums, 16x16 tiles (once-per-call dense B.e only).
+template <typename T>
+__global__ void matmul_nt_kernel(const T* A, const float* B, float* C, int M, int N, int K) {
+    __shared__ float sa[16][17], sb[16][17];
+    const int tx = threadIdx.x, ty = threadIdx.y;
+    const int row = blockIdx.y * 16 + ty, col = blockIdx.x * 16 + tx;
+    float acc = 0.0f;
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        sa[ty][tx] = (row < M && k0 + tx < K) ? to_f(A[static_cast<size_t>(row) * K + k0 + tx]) : 0.0f;
+        const int bn = blockIdx.x * 16 + ty;
+        sb[ty][tx] = (bn < N && k0 + tx < K) ? B[static_cast<size_t>(bn) * K + k0 + tx] : 0.0f;
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) acc = fmaf(sa[ty][k], sb[tx][k], acc);
+        __syncthreads();
+    }
+    if (row < M && col < N) C[static_cast<size_t>(row) * N + col] = acc;
+}
+
+// ----------------------------------------------------------------------------- norm1
+
+template <typename T, int NV>
+__global__ void __launch_bounds__(kRowThreads) norm1_kernel(const Norm1Args a) {
+    if (blockIdx.x == 0 && a.zero_counts)
+        for (int i = threadIdx.x; i < a.n_zero; i += blockDim.x) a.zero_counts[i] = 0;
+    const int row = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= a.ntok) return;
+    const size_t base = static_cast<size_t>(row) * a.dim;
+    const T* e = static_cast<const T*>(a.e);
+    float x[NV][4];
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int col = i * 128 + lane * 4;
+        load4(a.h + base + col, x[i]);
+        if (e) {
+            float ev[4];
+            load4(e + base + col, ev);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) x[i][j] += ev[j];
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ss = fmaf(x[i][j], x[i][j], ss);
+    }
+    ss = warp_sum(ss);
+    const float inv = rsqrtf(ss / a.dim + a.eps);
+    T* xn = static_cast<T*>(a.xn) + base;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int col = i * 128 + lane * 4;
+        float g[4];
+        load4(a.gamma + col, g);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) x[i][j] = to_f(from_f<T>(x[i][j] * inv * g[j]));
+        store4(xn + col, x[i]);
+    }
+    if (a.lora_a) {
+        const T* A = static_cast<const T*>(a.lora_a);
+        T* t = static_cast<T*>(a.lora_t) + static_cast<size_t>(row) * (128 / sizeof(T));
+#pragma unroll 1
+        for (int r = 0; r < a.lora_r; ++r) {
+            float p = 0.0f;
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+                float w[4];
+                load4(A + static_cast<size_t>(r) * a.dim + i * 128 + lane * 4, w);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) p = fmaf(x[i][j], w[j], p);
+            }
+            p = warp_sum(p);
+            if (lane == 0) store_t(t + r, p);
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------- norm2 + router
+
+template <typename T, int NV, int ESLOT>
+__global__ void __launch_bounds__(kRowThreads) norm2_router_kernel(const RouterArgs a) {
+    const int row = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= a.ntok) return;
+    const size_t base = static_cast<size_t>(row) * a.dim;
+    float y[NV][4];
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        load4(a.y + base + i * 128 + lane * 4, y[i]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ss = fmaf(y[i][j], y[i][j], ss);
+    }
+    ss = warp_sum(ss);
+    const float inv = rsqrtf(ss / a.dim + a.eps);
+    T* yn = static_cast<T*>(a.yn) + base;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int col = i * 128 + lane * 4;
+        float g[4];
+        load4(a.gamma + col, g);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) y[i][j] *= inv * g[j];
+        store4(yn + col, y[i]);   // rounded copy for the experts; the router keeps fp32
+    }
+
+    // logits: lane (e % 32) keeps expert e in slot e / 32
+    const T* W = static_cast<const T*>(a.w_router);
+    float lg[ESLOT];
+#pragma unroll
+    for (int s = 0; s < ESLOT; ++s) lg[s] = -INFINITY;
+#pragma unroll 1
+    for (int ex = 0; ex < a.n_exp; ++ex) {
+        float p = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            float w[4];
+            load4(W + static_cast<size_t>(ex) * a.dim + i * 128 + lane * 4, w);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) p = fmaf(y[i][j], w[j], p);
+        }
+        p = warp_sum(p);
+#pragma unroll
+        for (int s = 0; s < ESLOT; ++s)
+            if (lane == (ex & 31) && s == (ex >> 5)) lg[s] = p;
+    }
+    float score[ESLOT];
+    bool taken[ESLOT];
+#pragma unroll
+    for (int s = 0; s < ESLOT; ++s) {
+        const int ex = s * 32 + lane;
+        const float sc = ex < a.n_exp ? lg[s] + (a.bias ? a.bias[ex] : 0.0f) : -INFINITY;
+        score[s] = isnan(sc) ? -INFINITY : sc;   // a NaN never wins; indices stay in range
+        taken[s] = ex >= a.n_exp;
+    }
+    // top-k by (score desc, index asc)
+    int sel_idx = -1;
+    float sel_logit = 0.0f;
+#pragma unroll 1
+    for (int k = 0; k < a.top_k; ++k) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+        float bl = 0.0f;
+#pragma unroll
+        for (int s = 0; s < ESLOT; ++s) {
+            const int ex = s * 32 + lane;
+            if (!taken[s] && (score[s] > bv || (score[s] == bv && ex < bi))) {
+                bv = score[s];
+                bi = ex;
+                bl = lg[s];
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            const float ol = __shfl_xor_sync(0xffffffffu, bl, o);
+            if (ov > bv || (ov == bv && oi < bi)) {
+                bv = ov;
+                bi = oi;
+                bl = ol;
+            }
+        }
+#pragma unroll
+        for (int s = 0; s < ESLOT; ++s)
+            if (s * 32 + lane == bi) taken[s] = true;
+        if (lane == k) {
+            sel_idx = min(max(bi, 0), a.n_exp - 1);
+            sel_logit = bl;
+        }
+    }
+    // softmax over the k selected logits (lanes 0..k-1 hold one each)
+    const bool mine = lane < a.top_k;
+    float mx = mine ? sel_logit : -INFINITY;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float ex = mine ? expf(sel_logit - mx) : 0.0f;
+    const float den = warp_sum(ex);
+    if (mine) {
+        const float wv = ex / den;
+        const size_t o = static_cast<size_t>(row) * a.top_k + lane;
+        a.idx[o] = sel_idx;
+        a.w[o] = wv;
+        if (a.trace_idx) a.trace_idx[o] = sel_idx;
+        if (a.trace_w) a.trace_w[o] = wv;
+        atomicAdd(a.counts + sel_idx, 1);
+    }
+}
+
+// ----------------------------------------------------------------------------- MoE dispatch
+
+// One block: exclusive scans of the routed counts (row offsets inside the routed region)
+// and of the per-group tile counts; writes the grouped-GEMM tile list.
+__global__ void __launch_bounds__(256) moe_scan_kernel(const DispatchArgs a) {
+    __shared__ int s_cnt[256], s_tiles[256], s_off[256], s_toff[256];
+    const int G = a.n_exp + a.n_shared;
+    const int t = threadIdx.x;
+    const int cnt = t < a.n_exp ? a.counts[t] : (t < G ? a.ntok : 0);
+    s_cnt[t] = t < a.n_exp ? cnt : 0;
+    s_tiles[t] = t < G ? (cnt + 127) / 128 : 0;
+    __syncthreads();
+    // Hillis-Steele inclusive scans
+    for (int d = 1; d < 256; d <<= 1) {
+        const int v1 = t >= d ? s_cnt[t - d] : 0;
+        const int v2 = t >= d ? s_tiles[t - d] : 0;
+        __syncthreads();
+        s_cnt[t] += v1;
+        s_tiles[t] += v2;
+        __syncthreads();
+    }
+    s_off[t] = t == 0 ? 0 : s_cnt[t - 1];
+    s_toff[t] = t == 0 ? 0 : s_tiles[t - 1];
+    __syncthreads();
+    if (t < a.n_exp) {
+        a.offsets[t] = s_off[t];
+        a.fill[t] = 0;
+    }
+    if (t == 0) *a.n_tiles = s_tiles[255];
+    if (t < G) {
+        const int ntile = (cnt + 127) / 128;
+        for (int i = 0; i < ntile; ++i) {
+            GroupTile gt;
+            gt.group = t;
+            gt.nrows = min(128, cnt - 128 * i);
+            if (t < a.n_exp) {
+                gt.a_row0 = a.ntok + s_off[t] + 128 * i;                      // routed copies
+                gt.c_row0 = a.n_shared * a.ntok + s_off[t] + 128 * i;
+            } else {
+                const int s = t - a.n_exp;
+                gt.a_row0 = 128 * i;                                          // yn itself
+                gt.c_row0 = s * a.ntok + 128 * i;
+            }
+            const int slot = s_toff[t] + i;
+            if (slot < a.max_tiles) a.tiles[slot] = gt;
+        }
+    }
+}
+
+// One warp per (token, slot): claim a row in the expert's range, record token and gate
+// weight, copy the normalised row yn[token] into it.
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads) moe_scatter_kernel(const DispatchArgs a) {
+    const int ws = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (ws >= a.ntok * a.top_k) return;
+    const int n = ws / a.top_k;
+    const int ex = a.idx[ws];
+    int pos = 0;
+    if (lane == 0) pos = atomicAdd(a.fill + ex, 1);
+    pos = __shfl_sync(0xffffffffu, pos, 0);
+    const int r = a.offsets[ex] + pos;
+    if (lane == 0) {
+        a.row_token[r] = n;
+        a.row_w[r] = a.w[ws];
+    }
+    T* xp = static_cast<T*>(a.xperm);
+    const uint4* src = reinterpret_cast<const uint4*>(xp + static_cast<size_t>(n) * a.dim);
+    uint4* dst = reinterpret_cast<uint4*>(xp + static_cast<size_t>(a.ntok + r) * a.dim);
+    const int nvec = a.dim * static_cast<int>(sizeof(T)) / 16;
+    for (int i = lane; i < nvec; i += 32) dst[i] = src[i];
+}
+
+// ----------------------------------------------------------------------------- LoRA down
+
+template <typename T, int NV>
+__global__ void __launch_bounds__(kRowThreads) lora_down_kernel(const T* x, int ldx, int ntok,
+                                                                const T* A, int r, T* t) {
+    const int row = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= ntok) return;
+    const int width = NV * 128;
+    float v[NV][4];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) load4(x + static_cast<size_t>(row) * ldx + i * 128 + lane * 4, v[i]);
+    T* out = t + static_cast<size_t>(row) * (128 / sizeof(T));
+#pragma unroll 1
+    for (int j = 0; j < r; ++j) {
+        float p = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            float w[4];
+            load4(A + static_cast<size_t>(j) * width + i * 128 + lane * 4, w);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) p = fmaf(v[i][q], w[q], p);
+        }
+        p = warp_sum(p);
+        if (lane == 0) store_t(out + j, p);
+    }
+}
+
+// ----------------------------------------------------------------------------- MLA latents
+
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads) mla_latent_norm_kernel(const MlaNormArgs a) {
+    const int row = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= a.ntok) return;
+    const float* L = a.lat + static_cast<size_t>(row) * a.ld_lat;
+    // c_q
+    float ss = 0.0f;
+    for (int i = lane; i < a.q_lat; i += 32) ss = fmaf(L[i], L[i], ss);
+    ss = warp_sum(ss);
+    float inv = rsqrtf(ss / a.q_lat + a.eps);
+    T* cq = static_cast<T*>(a.cq) + static_cast<size_t>(row) * a.q_lat;
+    for (int i = lane; i < a.q_lat; i += 32) store_t(cq + i, L[i] * inv * a.q_norm[i]);
+    // c_kv
+    const float* C = L + a.q_lat;
+    ss = 0.0f;
+    for (int i = lane; i < a.kv_lat; i += 32) ss = fmaf(C[i], C[i], ss);
+    ss = warp_sum(ss);
+    inv = rsqrtf(ss / a.kv_lat + a.eps);
+    T* kv = static_cast<T*>(a.kv) + static_cast<size_t>(row) * (a.kv_lat + a.rope);
+    for (int i = lane; i < a.kv_lat; i += 32) store_t(kv + i, C[i] * inv * a.kv_norm[i]);
+    // decoupled RoPE key
+    const float* R = C + a.kv_lat;
+    const int half = a.rope / 2;
+    const int pos = row % a.seq;
+    for (int i = lane; i < half; i += 32) {
+        const float c = a.rope_cos[pos * half + i], s = a.rope_sin[pos * half + i];
+        const float x1 = R[i], x2 = R[i + half];
+        store_t(kv + a.kv_lat + i, x1 * c - x2 * s);
+        store_t(kv + a.kv_lat + half + i, x2 * c + x1 * s);
+    }
+}
+
+// ----------------------------------------------------------------------------- weight prep / checks
+
+template <typename T>
+__global__ void prep_matmul_kernel(const T* A, long sam, long sak, const T* B, long sbk, long sbn,
+                                   T* C, int ldc, int M, int N, int K) {
+    const int m = blockIdx.y * blockDim.y + threadIdx.y;
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    if (m >= M || n >= N) return;
+    float acc = 0.0f;
+    for (int k = 0; k < K; ++k) acc = fmaf(to_f(A[m * sam + k * sak]), to_f(B[k * sbk + n * sbn]), acc);
+    C[static_cast<size_t>(m) * ldc + n] = from_f<T>(acc);
+}
+
+__global__ void check_finite_kernel(const float* x, size_t n, int* flags) {
+    bool bad = false;
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x)
+        bad |= !isfinite(x[i]);
+    if (__syncthreads_or(bad) && threadIdx.x == 0) atomicExch(flags + FLAG_NONFINITE, 1);
+}
+
+template <typename T, template <typename, int> class K, typename... Args>
+rdt_status launch_rows(int nv, int rows, cudaStream_t st, Args... args) {
+    const dim3 grid((rows + kRowThreads / 32 - 1) / (kRowThreads / 32));
+    switch (nv) {
+        case 1: K<T, 1>::run(grid, st, args...); break;
+        case 2: K<T, 2>::run(grid, st, args...); break;
+        case 4: K<T, 4>::run(grid, st, args...); break;
+        case 8: K<T, 8>::run(grid, st, args...); break;
+        case 16: K<T, 16>::run(grid, st, args...); break;
+        case 32: K<T, 32>::run(grid, st, args...); break;
+        default: set_error("row kernel: unsupported width"); return RDT_ERR_UNSUPPORTED;
+    }
+    RDT_CUDA_TRY(cudaGetLastError());
+    return RDT_OK;
+}
+
+template <typename T, int NV>
+struct Norm1L {
+    static void run(dim3 g, cudaStream_t st, Norm1Args a) {
+        norm1_kernel<T, NV><<<g, kRowThreads, 0, st>>>(a);
+    }
+};
+template <typename T, int NV>
+struct LoraL {
+    static void run(dim3 g, cudaStream_t st, const void* x, int ldx, int ntok, const void* A,
+                    int r, void* t) {
+        lora_down_kernel<T, NV><<<g, kRowThreads, 0, st>>>(static_cast<const T*>(x), ldx, ntok,
+                                                           static_cast<const T*>(A), r,
+                                                           static_cast<T*>(t));
+    }
+};
+template <typename T, int NV>
+struct RouterL {
+    static void run(dim3 g, cudaStream_t st, RouterArgs a) {
+        if (a.n_exp <= 32)
+            norm2_router_kernel<T, NV, 1><<<g, kRowThreads, 0, st>>>(a);
+        else if (a.n_exp <= 64)
+            norm2_router_kernel<T, NV, 2><<<g, kRowThreads, 0, st>>>(a);
+        else
+            norm2_router_kernel<T, NV, 8><<<g, kRowThreads, 0, st>>>(a);
+    }
+};
+
+}  // namespace
+
+rdt_status hoist(bool bf, const void* h0, const void* e, const float* Bdiag, float* h, float* Be,
+                 size_t n, int dim, cudaStream_t st) {
+    const size_t n4 = n / 4;
+    const int grid = static_cast<int>(std::min<size_t>((n4 + 255) / 256, 148 * 16));
+    if (bf)
+        hoist_kernel<bf16><<<grid, 256, 0, st>>>(static_cast<const bf16*>(h0),
+                                                 static_cast<const bf16*>(e), Bdiag, h, Be, n4, dim);
+    else
+        hoist_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(h0),
+                                                  static_cast<const float*>(e), Bdiag, h, Be, n4, dim);
+    RDT_CUDA_TRY(cudaGetLastError());
+    return RDT_OK;
+}
+
+rdt_status matmul_nt_simt(bool a_bf16, const void* A, const float* B, float* C, int M, int N,
+                          int K, cudaStream_t st) {
+    const dim3 blk(16, 16), grid((N + 15) / 16, (M + 15) / 16);
+    if (a_bf16)
+        matmul_nt_kernel<bf16><<<grid, blk, 0, st>>>(static_cast<const bf16*>(A), B, C, M, N, K);
+    else
+        matmul_nt_kernel<float><<<grid, blk, 0, st>>>(static_cast<const float*>(A), B, C, M, N, K);
+    RDT_CUDA_TRY(cudaGetLastError());
+    return RDT_OK;
+}
+
+rdt_status norm1(bool bf, const Norm1Args& a, cudaStream_t st) {
+    const int nv = a.dim / 128;
+    return bf ? launch_rows<bf16, Norm1L>(nv, a.ntok, st, a)
+              : launch_rows<float, Norm1L>(nv, a.ntok, st, a);
+}
+
+rdt_status lora_down(bool bf, const void* x, int ldx, int ntok, int width, const void* A, int r,
+                     void* t, cudaStream_t st) {
+    const int nv = width / 128;
+    return bf ? launch_rows<bf16, LoraL>(nv, ntok, st, x, ldx, ntok, A, r, t)
+              : launch_rows<float, LoraL>(nv, ntok, st, x, ldx, ntok, A, r, t);
+}
+
+rdt_status norm2_router(bool bf, const RouterArgs& a, cudaStream_t st) {
+    const int nv = a.dim / 128;
+    return bf ? launch_rows<bf16, RouterL>(nv, a.ntok, st, a)
+              : launch_rows<float, RouterL>(nv, a.ntok, st, a);
+}
+
+rdt_status moe_dispatch(bool bf, const DispatchArgs& a, cudaStream_t st) {
+    moe_scan_kernel<<<1, 256, 0, st>>>(a);
+    RDT_CUDA_TRY(cudaGetLastError());
+    const int warps = a.ntok * a.top_k;
+    const dim3 grid((warps + kRowThreads / 32 - 1) / (kRowThreads / 32));
+    if (bf)
+        moe_scatter_kernel<bf16><<<grid, kRowThreads, 0, st>>>(a);
+    else
+        moe_scatter_kernel<float><<<grid, kRowThreads, 0, st>>>(a);
+    RDT_CUDA_TRY(cudaGetLastError());
+    return RDT_OK;
+}
+
+rdt_status mla_latent_norm(bool bf, const MlaNormArgs& a, cudaStream_t st) {
+    const dim3 grid((a.ntok + kRowThreads / 32 - 1) / (kRowThreads / 32));
+    if (bf)
+        mla_latent_norm_kernel<bf16><<<grid, kRowThreads, 0, st>>>(a);
+    else
+        mla_latent_norm_kernel<float><<<grid, kRowThreads, 0, st>>>(a);
+    RDT_CUDA_TRY(cudaGetLastError());
+    return RDT_OK;
+}
+
+rdt_status prep_matmul(bool bf, const void* A, long sam, long sak, const void* B, long sbk,
+                       long sbn, void* C, int ldc, int M, int N, int K, cudaStream_t st) {
+    const dim3 blk(32, 8), grid((N + 31) / 32, (M + 7) / 8);
+    if (bf)
+        prep_matmul_kernel<bf16><<<grid, blk, 0, st>>>(static_cast<const bf16*>(A), sam, sak,
+                                                       static_cast<const bf16*>(B), sbk, sbn,
+                                                       static_cast<bf16*>(C), ldc, M, N, K);
+    else
+        prep_matmul_kernel<float><<<grid, blk, 0, st>>>(static_cast<const float*>(A), sam, sak,
+                                                        static_cast<const float*>(B), sbk, sbn,
+                                                        static_cast<float*>(C), ldc, M, N, K);
+    RDT_CUDA_TRY(cudaGetLastError());
+    return RDT_OK;
+}
+
+rdt_status check_finite(const float* x, size_t n, int* flags, cudaStream_t st) {
+    const int grid = static_cast<int>(std::min<size_t>((n + 255) / 256, 148 * 8));
+    check_finite_kernel<<<grid, 256, 0, st>>>(x, n, flags);
+    RDT_CUDA_TRY(cudaGetLastError());
+    return RDT_OK;
+}
+
+}  // namespace rdt

@@ -1,0 +1,78 @@
+"""The tensor-core GEMM and the attention kernel alone (rdt_matmul, rdt_attention) against
+fp64 references on the same rounded inputs."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+def _torch():
+    import torch
+    return torch
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 64), (300, 256, 1024), (2048, 1536, 1024),
+                                   (77, 96, 128), (1, 32, 64), (4096, 2048, 2048)])
+def test_matmul_bf16(M, N, K):
+    torch = _torch()
+    import recurrent_depth_transformer_b200 as R
+    g = torch.Generator().manual_seed(M * 7 + N)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    B = torch.randn(N, K, generator=g).to(torch.bfloat16)
+    C = R.matmul(A.cuda(), B.cuda())
+    torch.cuda.synchronize()
+    ref = A.double() @ B.double().T
+    err = (C.cpu().double() - ref).abs().max().item()
+    assert err <= 2e-5 * K, err          # fp32 accumulation of exact bf16 products
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 128, 128), (200, 256, 512)])
+def test_matmul_tf32(M, N, K):
+    torch = _torch()
+    import recurrent_depth_transformer_b200 as R
+    g = torch.Generator().manual_seed(M + N)
+    A = torch.randn(M, K, generator=g)
+    B = torch.randn(N, K, generator=g)
+    C = R.matmul(A.cuda(), B.cuda())
+    torch.cuda.synchronize()
+    ref = A.double() @ B.double().T
+    err = (C.cpu().double() - ref).abs().max().item()
+    # tf32 keeps 10 mantissa bits: relative error 2^-11 per operand
+    assert err <= 6 * 2.0 ** -11 * math.sqrt(K) * 4, err
+
+
+@pytest.mark.parametrize("batch,seq,hq,hkv,dqk,dv", [(2, 200, 4, 2, 64, 64), (1, 64, 2, 2, 64, 64),
+                                                     (1, 1, 2, 1, 64, 64), (2, 130, 4, 1, 160, 128),
+                                                     (1, 513, 16, 4, 64, 64)])
+def test_attention_bf16(batch, seq, hq, hkv, dqk, dv):
+    torch = _torch()
+    import recurrent_depth_transformer_b200 as R
+    g = torch.Generator().manual_seed(seq * 3 + dqk)
+    q = torch.randn(batch * seq, hq * dqk, generator=g).to(torch.bfloat16)
+    k = torch.randn(batch * seq, hkv * dqk, generator=g).to(torch.bfloat16)
+    v = torch.randn(batch * seq, hkv * dv, generator=g).to(torch.bfloat16)
+    scale = 1.0 / math.sqrt(dqk)
+    o = R.attention(q.cuda(), k.cuda(), v.cuda(), batch, seq, hq, hkv, dqk, dv, scale)
+    torch.cuda.synchronize()
+    ref = O.gqa_attention(q.float().numpy().reshape(batch, seq, hq, dqk),
+                          k.float().numpy().reshape(batch, seq, hkv, dqk),
+                          v.float().numpy().reshape(batch, seq, hkv, dv), scale)
+    err = np.abs(o.cpu().float().numpy().reshape(ref.shape) - ref).max()
+    assert err < 2e-2, err
+
+
+def test_attention_f32():
+    torch = _torch()
+    import recurrent_depth_transformer_b200 as R
+    batch, seq, hq, hkv, d = 1, 64, 4, 2, 32
+    g = torch.Generator().manual_seed(5)
+    q, k, v = (torch.randn(batch * seq, h * d, generator=g) for h in (hq, hkv, hkv))
+    o = R.attention(q.cuda(), k.cuda(), v.cuda(), batch, seq, hq, hkv, d, d, 0.2)
+    torch.cuda.synchronize()
+    ref = O.gqa_attention(q.numpy().reshape(1, seq, hq, d), k.numpy().reshape(1, seq, hkv, d),
+                          v.numpy().reshape(1, seq, hkv, d), 0.2)
+    assert np.abs(o.cpu().numpy().reshape(ref.shape) - ref).max() < 1e-4

@@ -1,0 +1,211 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerances: hidden states after T loops within max-abs 3e-2 and relative Frobenius 1e-2;
+router indices identical wherever the oracle's k-th/(k+1)-th score gap exceeds 1e-3 (the
+oracle adopts the GPU's choice only on near-ties and counts every other difference).
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+from workloads import WORKLOADS, generate, prefix
+
+from rdt_testlib import (MAX_ABS, REL_FRO, act, assert_close, errors, handle, oracle_follow,
+                         run_loop, torch_mod)
+
+pytestmark = pytest.mark.gpu
+
+C0, C1, C2, C3, C4 = WORKLOADS
+
+# Reduced-size variants: same widths, heads and experts, fewer tokens; sequence lengths
+# that leave ragged GEMM row tiles (not multiples of 128) and ragged attention blocks.
+SMALL = {
+    "tiny-f32": C0,
+    "gqa-s200": C1.replace(batch=2, seq=200),
+    "mla-s136": C2.replace(batch=2, seq=136),
+    "widemoe-s192": C3.replace(batch=1, seq=192),
+    "long-lora-s320": C4.replace(seq=320),
+}
+
+
+def _loops(name):
+    return 4 if name == "tiny-f32" else 3
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_loop_matches_oracle_small(name):
+    wl = SMALL[name]
+    inputs = generate(wl)
+    T = _loops(name)
+    got, idx, w, _, diag = run_loop(wl, inputs, T)
+    assert diag["nonfinite"] == 0 and diag["timeout"] == 0
+    want, mism, ties, _ = oracle_follow(wl, inputs, T, idx)
+    assert mism == 0, f"{mism} routing differences outside near-ties"
+    assert_close(got, want, what=name)
+
+
+def test_zero_block_is_closed_form():
+    # every block weight zero: h_T = A^T h0 + (1 - A^T)/(1 - A) B e exactly (fp32 state)
+    wl = C1.replace(batch=2, seq=64)
+    inputs = generate(wl, zero_block=True, h0_independent=True)
+    for T in (1, 2, 7, 16):
+        got, *_ = run_loop(wl, inputs, T, trace=False)
+        A = inputs["A"].astype(np.float64)
+        Be = inputs["B"].astype(np.float64) * inputs["e"]
+        want = A ** T * inputs["h0"] + (1 - A ** T) / (1 - A) * Be
+        ma, _ = errors(got, want)
+        assert ma < 2e-4 * max(1.0, np.max(np.abs(want))), (T, ma)
+
+
+def test_dense_B_and_h0_independent():
+    wl = C2.replace(batch=1, seq=96, b_kind="dense")
+    inputs = generate(wl, h0_independent=True)
+    got, idx, *_ = run_loop(wl, inputs, 3)
+    want, mism, _, _ = oracle_follow(wl, inputs, 3, idx)
+    assert mism == 0
+    assert_close(got, want, what="mla dense B")
+
+
+def test_lora_depth_extrapolation_uses_last_adapter():
+    wl = C4.replace(seq=128, n_lora=2)
+    inputs = generate(wl)
+    got, idx, *_ = run_loop(wl, inputs, 4)            # loops 2, 3 reuse adapter 1
+    want, mism, _, _ = oracle_follow(wl, inputs, 4, idx)
+    assert mism == 0
+    assert_close(got, want, what="lora T > n_lora")
+
+
+def test_attention_sublayer():
+    torch = torch_mod()
+    for wl in (C0, C1.replace(batch=2, seq=200), C2.replace(batch=2, seq=136), C4.replace(seq=192)):
+        inputs = generate(wl)
+        x = inputs["e"].astype(np.float32) * 1.5 + 0.25
+        with handle(wl, inputs) as h:
+            a = h.attn_forward(torch.from_numpy(x).cuda(), loop=1)
+            torch.cuda.synchronize()
+            got = a.cpu().numpy()
+        want = O.attention_sublayer(x, inputs, wl, 1)
+        assert_close(got, want, max_abs=2e-2, rel_fro=1e-2, what=f"attn {wl.name}")
+
+
+def test_moe_sublayer_and_router_exactness():
+    torch = torch_mod()
+    for wl in (C0, C1.replace(batch=2, seq=200), C3.replace(batch=1, seq=192)):
+        inputs = generate(wl)
+        y = inputs["e"].astype(np.float32) * 3.0
+        N = wl.batch * wl.seq
+        idx = torch.empty((N, wl.top_k), dtype=torch.int32, device="cuda")
+        w = torch.empty((N, wl.top_k), dtype=torch.float32, device="cuda")
+        with handle(wl, inputs) as h:
+            f = h.moe_forward(torch.from_numpy(y).cuda(), idx=idx, w=w)
+            torch.cuda.synchronize()
+            got, gi, gw = f.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy()
+            counts = h.diagnostics()["expert_counts"]
+        fo, r, st = O.moe_sublayer(y, inputs, wl, follow_idx=gi)
+        assert st["mismatch"] == 0
+        np.testing.assert_array_equal(np.bincount(gi.ravel(), minlength=wl.n_experts),
+                                      counts[:wl.n_experts])
+        np.testing.assert_allclose(gw, r.w, atol=1e-5)
+        np.testing.assert_allclose(gw.sum(axis=1), 1.0, atol=1e-5)
+        assert_close(got, fo, max_abs=2e-2, rel_fro=1e-2, what=f"moe {wl.name}")
+
+
+def test_T1_equals_sublayer_composition():
+    torch = torch_mod()
+    wl = C1.replace(batch=1, seq=256)
+    inputs = generate(wl)
+    with handle(wl, inputs) as h:
+        e = act(wl, inputs["e"])
+        hT = h.loop_forward(e, e, 1)
+        x0 = e.float() + e.float()
+        a = h.attn_forward(x0, loop=0)
+        f = h.moe_forward(x0 + a)
+        A = torch.from_numpy(inputs["A"]).cuda()
+        B = torch.from_numpy(inputs["B"]).cuda()
+        comp = A * e.float() + B * e.float() + a + f
+        torch.cuda.synchronize()
+    ma, rf = errors(hT.cpu().numpy(), comp.cpu().numpy())
+    assert ma < 1e-2 and rf < 1e-3, (ma, rf)
+
+
+def test_causality_and_batch_independence():
+    torch = torch_mod()
+    wl = C1.replace(batch=2, seq=256)
+    inputs = generate(wl)
+    with handle(wl, inputs) as h:
+        e = act(wl, inputs["e"])
+        out1 = h.loop_forward(e, e, 2).clone()
+        e2 = e.clone()
+        e2[0, 100:] = e2[0, 100:] * -1.0
+        e2[1] = e2[1] * 0.5
+        out2 = h.loop_forward(e2, e2, 2)
+        torch.cuda.synchronize()
+    d = (out1[0, :100] - out2[0, :100]).abs().max().item()
+    assert d < 1e-4, d      # atomics may reorder the expert sums; values must agree
+
+
+def test_host_entry_matches_device_entry():
+    torch = torch_mod()
+    wl = C1.replace(batch=1, seq=128)
+    inputs = generate(wl)
+    with handle(wl, inputs) as h:
+        e = act(wl, inputs["e"])
+        dev = h.loop_forward(e, e, 3).cpu()
+        eh = e.cpu().pin_memory()
+        out = torch.empty(dev.shape, dtype=torch.float32).pin_memory()
+        h.loop_forward_host(eh, eh, 3, out)
+    ma, _ = errors(out.numpy(), dev.numpy())
+    assert ma < 1e-3
+
+
+@pytest.mark.parametrize("wi", [1, 2, 3, 4])
+def test_full_size_prefix_and_sampled_rows(wi):
+    """The configuration at its full size in the benchmark's launch configuration: the first
+    64 positions of every sequence against the oracle (causality makes them independent of
+    later positions), and the last loop at sampled late positions from the GPU's own h_{T-1}."""
+    wl = WORKLOADS[wi]
+    T = max(wl.loops)
+    inputs = generate(wl)
+    got, idx, _, traj, diag = run_loop(wl, inputs, T, traj=True)
+    assert diag["nonfinite"] == 0 and diag["timeout"] == 0
+    P = 64
+    pin = prefix(inputs, P)
+    pwl = wl.replace(seq=P)
+    pidx = idx.reshape(T, wl.batch, wl.seq, wl.top_k)[:, :, :P]
+    want, mism, _, _ = oracle_follow(pwl, pin, T, pidx)
+    assert mism == 0
+    assert_close(got[:, :P], want, what=f"{wl.name} prefix")
+    rng = np.random.default_rng(wi)
+    rows = [(int(rng.integers(wl.batch)), int(s)) for s in
+            (wl.seq - 1, wl.seq // 2 + 1, int(rng.integers(P, wl.seq)))]
+    hT1 = traj[T - 1].reshape(wl.batch, wl.seq, wl.dim)
+    fidx = np.stack([idx[T - 1].reshape(wl.batch, wl.seq, -1)[b, s] for b, s in rows])
+    hn, r, st = O.loop_step_rows(hT1, inputs["e"], inputs, wl, T - 1, rows, follow_idx=fidx)
+    assert st["mismatch"] == 0
+    gt = np.stack([got[b, s] for b, s in rows])
+    assert_close(gt, hn, what=f"{wl.name} sampled rows")
+
+
+def test_invalid_arguments_return_errors():
+    torch = torch_mod()
+    import recurrent_depth_transformer_b200 as R
+    wl = C1.replace(batch=1, seq=64)
+    inputs = generate(wl)
+    with handle(wl, inputs, max_loops=4) as h:
+        e = act(wl, inputs["e"])
+        with pytest.raises(R.RdtError) as ex:
+            h.loop_forward(e, e, 0)
+        assert ex.value.status == 1
+        with pytest.raises(R.RdtError) as ex:
+            h.loop_forward(e, e, 5)
+        assert ex.value.status == 1
+        bad = torch.empty(e.numel() * 2 + 8, dtype=torch.uint8, device="cuda")[1:]
+        with pytest.raises(R.RdtError) as ex:
+            h.attn_forward(bad, 0)
+        assert ex.value.status == 3
+    unstable = dict(inputs)
+    unstable["A"] = inputs["A"].copy()
+    unstable["A"][3] = 1.0
+    with pytest.raises(R.RdtError) as ex:
+        handle(wl, unstable)
+    assert ex.value.status == 4
