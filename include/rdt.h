@@ -206,6 +206,23 @@ rdt_status rdt_attention(int32_t dtype, const void* q, const void* k, const void
                          int batch, int seq, int n_heads, int n_kv_heads, int dqk, int dv,
                          float scale, void* stream);
 
+/* ---- per-kernel timing (CUDA events recorded around every launch of the handle) */
+typedef struct {
+    char name[32];          /* kernel class, e.g. "gemm_up", "attention", "norm2_router" */
+    int64_t launches;       /* launches timed since profiling was enabled               */
+    double total_ms;        /* summed event time of those launches                      */
+} rdt_kernel_stat;
+
+/* enable = 1 clears the statistics and starts timing; 0 stops it. Timing adds two
+ * event records per launch on the launch stream. */
+rdt_status rdt_profile(rdt_handle* h, int enable);
+
+/* Synchronises the handle's last stream and returns up to max_entries statistics
+ * (*n_entries set to their number) and, in *total_launches, the number of kernels
+ * the handle has launched since create (counted whether or not timing is on). */
+rdt_status rdt_profile_read(rdt_handle* h, rdt_kernel_stat* out, int max_entries, int* n_entries,
+                            int64_t* total_launches);
+
 const char* rdt_status_string(rdt_status s);
 const char* rdt_last_error(void);
 

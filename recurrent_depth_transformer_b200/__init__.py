@@ -33,7 +33,8 @@ STATUS = {0: "RDT_OK", 1: "RDT_ERR_INVALID_ARG", 2: "RDT_ERR_UNSUPPORTED", 3: "R
 
 EXPORTED = ("rdt_create", "rdt_attn_forward", "rdt_moe_forward", "rdt_loop_forward",
             "rdt_loop_forward_host", "rdt_set_trace", "rdt_get_diagnostics", "rdt_memory_bytes",
-            "rdt_status_string", "rdt_last_error", "rdt_destroy", "rdt_matmul", "rdt_attention")
+            "rdt_status_string", "rdt_last_error", "rdt_destroy", "rdt_matmul", "rdt_attention",
+            "rdt_profile", "rdt_profile_read")
 
 
 class RdtError(RuntimeError):
@@ -59,6 +60,10 @@ FP32_FIELDS = ("A", "B", "norm1", "norm2", "q_norm", "kv_norm", "router_bias")
 
 class RdtWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS]
+
+
+class RdtKernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64), ("total_ms", ctypes.c_double)]
 
 
 class RdtDiag(ctypes.Structure):
@@ -95,11 +100,14 @@ def load_library() -> ctypes.CDLL:
     lib.rdt_destroy.argtypes = [vp]
     lib.rdt_destroy.restype = None
     lib.rdt_matmul.argtypes = [i32, vp, vp, vp, i32, i32, i32, vp]
+    lib.rdt_profile.argtypes = [vp, i32]
+    lib.rdt_profile_read.argtypes = [vp, ctypes.POINTER(RdtKernelStat), i32, ctypes.POINTER(i32),
+                                     ctypes.POINTER(ctypes.c_int64)]
     lib.rdt_attention.argtypes = [i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                   ctypes.c_float, vp]
     for f in ("rdt_create", "rdt_attn_forward", "rdt_moe_forward", "rdt_loop_forward",
               "rdt_loop_forward_host", "rdt_set_trace", "rdt_get_diagnostics", "rdt_memory_bytes",
-              "rdt_matmul", "rdt_attention"):
+              "rdt_matmul", "rdt_attention", "rdt_profile", "rdt_profile_read"):
         getattr(lib, f).restype = i32
     _LIB = lib
     return lib
@@ -242,6 +250,22 @@ class RDT:
         E = self.cfg.n_experts + self.cfg.n_shared
         return {"rho_A": d.rho_A, "nonfinite": d.nonfinite, "timeout": d.timeout,
                 "last_routed_rows": d.last_routed_rows, "expert_counts": list(d.expert_counts[:E])}
+
+    def profile(self, enable: bool = True):
+        _check(self._lib.rdt_profile(self._h, 1 if enable else 0))
+
+    def profile_read(self):
+        """(per-kernel {name: (launches, total_ms)}, kernels launched since create)."""
+        arr = (RdtKernelStat * 64)()
+        n = ctypes.c_int()
+        tot = ctypes.c_int64()
+        _check(self._lib.rdt_profile_read(self._h, arr, 64, ctypes.byref(n), ctypes.byref(tot)))
+        return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(n.value)}, tot.value
+
+    def launch_count(self) -> int:
+        tot = ctypes.c_int64()
+        _check(self._lib.rdt_profile_read(self._h, None, 0, None, ctypes.byref(tot)))
+        return tot.value
 
     def memory_bytes(self) -> int:
         n = ctypes.c_size_t()

@@ -73,9 +73,66 @@ struct rdt_handle {
     int32_t* tr_idx = nullptr;
     float* tr_w = nullptr;
     float* tr_h = nullptr;
+
+    // launch accounting and optional per-kernel event timing
+    int64_t launches = 0;
+    bool prof_on = false;
+    std::vector<cudaEvent_t> ev_pool;
+    size_t ev_used = 0;
+    struct Pending { int kind; cudaEvent_t a, b; int n; };
+    std::vector<Pending> pending;
+    std::vector<double> prof_ms;
+    std::vector<int64_t> prof_n;
 };
 
 namespace {
+
+// kernel classes reported by rdt_profile_read
+enum Kind { K_HOIST, K_NORM1, K_GEMM_QKV, K_GEMM_LAT, K_MLA_NORM, K_GEMM_Q, K_ATTENTION, K_LORA_DOWN,
+            K_GEMM_O, K_NORM2_ROUTER, K_DISPATCH, K_GEMM_UP, K_GEMM_DOWN, K_CHECK, K_DENSE_B, K_COUNT };
+const char* const kKindName[K_COUNT] = {"hoist", "norm1", "gemm_qkv", "gemm_latent", "mla_latent_norm",
+                                         "gemm_q_absorbed", "attention", "lora_down", "gemm_o",
+                                         "norm2_router", "moe_dispatch", "gemm_up", "gemm_down",
+                                         "check_finite", "dense_injection"};
+
+rdt_status prof_begin(rdt_handle* h, int kind, int nlaunch, cudaStream_t st) {
+    h->launches += nlaunch;
+    if (!h->prof_on) return RDT_OK;
+    while (h->ev_pool.size() < h->ev_used + 2) {
+        cudaEvent_t ev;
+        RDT_CUDA_TRY(cudaEventCreate(&ev));
+        h->ev_pool.push_back(ev);
+    }
+    rdt_handle::Pending p{kind, h->ev_pool[h->ev_used], h->ev_pool[h->ev_used + 1], nlaunch};
+    h->ev_used += 2;
+    RDT_CUDA_TRY(cudaEventRecord(p.a, st));
+    h->pending.push_back(p);
+    return RDT_OK;
+}
+rdt_status prof_end(rdt_handle* h, cudaStream_t st) {
+    if (!h->prof_on) return RDT_OK;
+    RDT_CUDA_TRY(cudaEventRecord(h->pending.back().b, st));
+    return RDT_OK;
+}
+// Resolve recorded event pairs into the per-kind sums (the stream must have completed).
+rdt_status prof_flush(rdt_handle* h) {
+    for (const auto& p : h->pending) {
+        float ms = 0.0f;
+        RDT_CUDA_TRY(cudaEventElapsedTime(&ms, p.a, p.b));
+        h->prof_ms[p.kind] += ms;
+        h->prof_n[p.kind] += p.n;
+    }
+    h->pending.clear();
+    h->ev_used = 0;
+    return RDT_OK;
+}
+
+#define TIMED(h, kind, n, st, expr)                \
+    do {                                           \
+        RDT_TRY(prof_begin((h), (kind), (n), (st))); \
+        RDT_TRY(expr);                             \
+        RDT_TRY(prof_end((h), (st)));              \
+    } while (0)
 
 template <typename P>
 rdt_status dev_alloc(rdt_handle* h, P** p, size_t bytes, bool zero = false) {
@@ -205,6 +262,8 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
     h->kext = static_cast<int>(128 / h->esz);
     h->ntok = c.batch * c.seq;
     h->G = c.n_experts + c.n_shared;
+    h->prof_ms.assign(K_COUNT, 0.0);
+    h->prof_n.assign(K_COUNT, 0);
     const size_t es = h->esz;
     const int N = h->ntok, d = c.dim, E = c.n_experts, S = c.n_shared, hid = c.expert_hidden;
     const int K = c.top_k;
@@ -462,7 +521,7 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         n1.zero_counts = h->counts;
         n1.n_zero = h->G;
     }
-    RDT_TRY(norm1(h->bf, n1, st));
+    TIMED(h, K_NORM1, 1, st, norm1(h->bf, n1, st));
 
     GemmArgs ga{};
     ga.M = N;
@@ -491,8 +550,8 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         ep.rot_off = 0;
         ep.rot_dim = c.head_dim;
         ep.rope_limit = h->nq + h->nkv;
-        RDT_TRY(gemm_tc(h->bf, 128, h->m_xn, h->m_wqkv, lora ? &h->m_tq : nullptr,
-                        lora ? &h->m_lqb : nullptr, ga, ep, st));
+        TIMED(h, K_GEMM_QKV, 1, st, gemm_tc(h->bf, 128, h->m_xn, h->m_wqkv, lora ? &h->m_tq : nullptr,
+                                           lora ? &h->m_lqb : nullptr, ga, ep, st));
         at.q = h->qkv;
         at.ldq = h->nqkv;
         at.q_hstride = c.head_dim;
@@ -515,7 +574,7 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         ep.out = h->lat;
         ep.ldo = h->lat_w;
         ep.ncols_valid = h->lat_w;
-        RDT_TRY(gemm_tc(h->bf, 128, h->m_xn, h->m_wlat, nullptr, nullptr, ga, ep, st));
+        TIMED(h, K_GEMM_LAT, 1, st, gemm_tc(h->bf, 128, h->m_xn, h->m_wlat, nullptr, nullptr, ga, ep, st));
         MlaNormArgs mn{};
         mn.lat = h->lat;
         mn.ld_lat = h->lat_w;
@@ -531,7 +590,7 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         mn.kv_lat = kvl;
         mn.rope = rp;
         mn.eps = c.norm_eps;
-        RDT_TRY(mla_latent_norm(h->bf, mn, st));
+        TIMED(h, K_MLA_NORM, 1, st, mla_latent_norm(h->bf, mn, st));
         // absorbed query projection with RoPE on the last rope columns of each head
         GemmArgs gq{};
         gq.M = N;
@@ -551,7 +610,7 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         eq.rot_off = kvl;
         eq.rot_dim = rp;
         eq.rope_limit = h->qt_w;
-        RDT_TRY(gemm_tc(h->bf, 160, h->m_cq, h->m_wqabs, nullptr, nullptr, gq, eq, st));
+        TIMED(h, K_GEMM_Q, 1, st, gemm_tc(h->bf, 160, h->m_cq, h->m_wqabs, nullptr, nullptr, gq, eq, st));
         at.q = h->qkv;
         at.ldq = h->qt_w;
         at.q_hstride = kvl + rp;
@@ -566,11 +625,11 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         at.dv = kvl;
         at.scale = 1.0f / std::sqrt(static_cast<float>(c.qk_nope_dim + rp));
     }
-    RDT_TRY(attention(h->bf, at, st));
+    TIMED(h, K_ATTENTION, 1, st, attention(h->bf, at, st));
 
     if (lora) {
         const void* A = static_cast<const char*>(h->loa) + static_cast<size_t>(li) * c.lora_rank * h->nq * h->esz;
-        RDT_TRY(lora_down(h->bf, h->o, h->owidth, N, h->owidth, A, c.lora_rank, h->to, st));
+        TIMED(h, K_LORA_DOWN, 1, st, lora_down(h->bf, h->o, h->owidth, N, h->owidth, A, c.lora_rank, h->to, st));
     }
     GemmArgs go{};
     go.M = N;
@@ -596,8 +655,8 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         eo.out = a_out;
         eo.ldo = d;
     }
-    RDT_TRY(gemm_tc(h->bf, 128, h->m_o, h->m_wo, lora ? &h->m_to : nullptr, lora ? &h->m_lob : nullptr,
-                    go, eo, st));
+    TIMED(h, K_GEMM_O, 1, st, gemm_tc(h->bf, 128, h->m_o, h->m_wo, lora ? &h->m_to : nullptr,
+                                      lora ? &h->m_lob : nullptr, go, eo, st));
     return RDT_OK;
 }
 
@@ -622,7 +681,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     ra.counts = h->counts;
     ra.trace_idx = tr_idx;
     ra.trace_w = tr_w;
-    RDT_TRY(norm2_router(h->bf, ra, st));
+    TIMED(h, K_NORM2_ROUTER, 1, st, norm2_router(h->bf, ra, st));
 
     DispatchArgs da{};
     da.counts = h->counts;
@@ -641,7 +700,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     da.xperm = h->xperm;
     da.row_token = h->row_token;
     da.row_w = h->row_w;
-    RDT_TRY(moe_dispatch(h->bf, da, st));
+    TIMED(h, K_DISPATCH, 2, st, moe_dispatch(h->bf, da, st));
 
     GemmArgs gu{};
     gu.N = 2 * hid;
@@ -656,7 +715,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     eu.ldo = hid;
     eu.ncols_valid = 2 * hid;
     eu.flags = h->flags;
-    RDT_TRY(gemm_tc(h->bf, 128, h->m_xperm, h->m_w13, nullptr, nullptr, gu, eu, st));
+    TIMED(h, K_GEMM_UP, 1, st, gemm_tc(h->bf, 128, h->m_xperm, h->m_w13, nullptr, nullptr, gu, eu, st));
 
     GemmArgs gd{};
     gd.N = d;
@@ -676,7 +735,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     ed.dst = dst;
     ed.ld = d;
     ed.flags = h->flags;
-    RDT_TRY(gemm_tc(h->bf, 128, h->m_U, h->m_w2, nullptr, nullptr, gd, ed, st));
+    TIMED(h, K_GEMM_DOWN, 1, st, gemm_tc(h->bf, 128, h->m_U, h->m_w2, nullptr, nullptr, gd, ed, st));
     return RDT_OK;
 }
 
@@ -684,8 +743,8 @@ rdt_status loop_impl(rdt_handle* h, const void* h0, const void* e, int T, float*
     const rdt_config& c = h->cfg;
     const int N = h->ntok, d = c.dim;
     const size_t nd = static_cast<size_t>(N) * d;
-    RDT_TRY(hoist(h->bf, h0, e, c.b_kind == RDT_B_DIAG ? h->Bw : nullptr, h->hbuf[0], h->Be, nd, d, st));
-    if (c.b_kind == RDT_B_DENSE) RDT_TRY(matmul_nt_simt(h->bf, e, h->Bw, h->Be, N, d, d, st));
+    TIMED(h, K_HOIST, 1, st, hoist(h->bf, h0, e, c.b_kind == RDT_B_DIAG ? h->Bw : nullptr, h->hbuf[0], h->Be, nd, d, st));
+    if (c.b_kind == RDT_B_DENSE) TIMED(h, K_DENSE_B, 1, st, matmul_nt_simt(h->bf, e, h->Bw, h->Be, N, d, d, st));
     if (h->tr_h) RDT_CUDA_TRY(cudaMemcpyAsync(h->tr_h, h->hbuf[0], nd * 4, cudaMemcpyDeviceToDevice, st));
     for (int t = 0; t < T; ++t) {
         float* hcur = h->hbuf[t & 1];
@@ -697,7 +756,7 @@ rdt_status loop_impl(rdt_handle* h, const void* h0, const void* e, int T, float*
         if (h->tr_h)
             RDT_CUDA_TRY(cudaMemcpyAsync(h->tr_h + (t + 1) * nd, hnext, nd * 4, cudaMemcpyDeviceToDevice, st));
     }
-    RDT_TRY(check_finite(out, nd, h->flags, st));
+    TIMED(h, K_CHECK, 1, st, check_finite(out, nd, h->flags, st));
     return RDT_OK;
 }
 
@@ -938,6 +997,46 @@ rdt_status rdt_get_diagnostics(rdt_handle* h, rdt_diag* out) {
     return RDT_OK;
 }
 
+rdt_status rdt_profile(rdt_handle* h, int enable) {
+    if (!h) {
+        set_error("handle is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (enable) {
+        RDT_CUDA_TRY(cudaStreamSynchronize(h->last_stream));
+        h->pending.clear();
+        h->ev_used = 0;
+        std::fill(h->prof_ms.begin(), h->prof_ms.end(), 0.0);
+        std::fill(h->prof_n.begin(), h->prof_n.end(), 0);
+    }
+    h->prof_on = enable != 0;
+    return RDT_OK;
+}
+
+rdt_status rdt_profile_read(rdt_handle* h, rdt_kernel_stat* out, int max_entries, int* n_entries,
+                            int64_t* total_launches) {
+    if (!h) {
+        set_error("handle is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    RDT_CUDA_TRY(cudaStreamSynchronize(h->last_stream));
+    RDT_TRY(prof_flush(h));
+    int n = 0;
+    for (int k = 0; k < K_COUNT; ++k) {
+        if (h->prof_n[k] == 0) continue;
+        if (out && n < max_entries) {
+            std::memset(out[n].name, 0, sizeof(out[n].name));
+            std::strncpy(out[n].name, kKindName[k], sizeof(out[n].name) - 1);
+            out[n].launches = h->prof_n[k];
+            out[n].total_ms = h->prof_ms[k];
+        }
+        ++n;
+    }
+    if (n_entries) *n_entries = std::min(n, max_entries);
+    if (total_launches) *total_launches = h->launches;
+    return RDT_OK;
+}
+
 rdt_status rdt_memory_bytes(const rdt_handle* h, size_t* bytes) {
     if (!h || !bytes) {
         set_error("handle or bytes is NULL");
@@ -950,6 +1049,7 @@ rdt_status rdt_memory_bytes(const rdt_handle* h, size_t* bytes) {
 void rdt_destroy(rdt_handle* h) {
     if (!h) return;
     cudaDeviceSynchronize();
+    for (cudaEvent_t ev : h->ev_pool) cudaEventDestroy(ev);
     for (void* p : h->allocs) cudaFree(p);
     delete h;
 }

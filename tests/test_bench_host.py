@@ -1,0 +1,83 @@
+"""Host-side logic of bench.py: algorithmic work, clock parsing, the multi-rank reduction
+(two gloo ranks on CPU) and the reference arm's JSON line."""
+import json
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from workloads import WORKLOADS, by_name
+
+
+def test_algorithmic_flops_of_the_bench_workload():
+    wl = by_name(bench.WORKLOAD)
+    assert wl is WORKLOADS[1]
+    per_loop = bench.step_flops(wl, 1)
+    # 2N d (Hq+2Hkv) dh + 2N Hq dh d + 4 B Hq dh S(S+1)/2 + 2N d E + 6 d hid N k
+    N, d = 2048, 1024
+    want = (2 * N * d * 1536 + 2 * N * 1024 * d + 4 * 4 * 16 * 64 * 512 * 513 / 2
+            + 2 * N * d * 16 + 6 * d * 1024 * N * 2)
+    assert per_loop == pytest.approx(want)
+    assert per_loop == pytest.approx(38.7e9, rel=0.01)
+
+
+def test_parse_clocks():
+    txt = ("0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n"
+           "0, 1800, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n"
+           "0, 1700, 1965, 999.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n")
+    c = bench.parse_clocks(txt)
+    assert c["sm_mhz"] == 1800 and c["sm_max_mhz"] == 1965 and c["reasons"] == ["sw_power_cap"]
+    assert bench.parse_clocks("") is None
+
+
+def test_aggregate_is_whole_job_over_slowest_rank():
+    v, ms = bench.aggregate([2.0, 4.0], 2048, 8, 2)
+    assert ms == 4.0 and v == pytest.approx(2 * 2048 * 8 / 0.004)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    assert bench.dist_env() == (rank, rank, world)
+    m = bench.reduce_max(1.5 + rank, device="cpu")
+    v, ms = bench.aggregate([m], 1000, 4, world)
+    q.put((rank, m, v))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_ranks_take_the_max_over_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    assert [r[1] for r in res] == [2.5, 2.5]
+    assert res[0][2] == pytest.approx(2 * 1000 * 4 / 0.0025)
+
+
+def test_reference_arm_prints_one_json_line(capsys):
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"]) == 0
+    out = capsys.readouterr().out.strip().splitlines()
+    assert len(out) == 1
+    line = json.loads(out[0])
+    assert line["impl"] == "reference" and line["unit"] == bench.UNIT and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
