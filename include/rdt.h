@@ -206,6 +206,31 @@ rdt_status rdt_attention(int32_t dtype, const void* q, const void* k, const void
                          int batch, int seq, int n_heads, int n_kv_heads, int dqk, int dv,
                          float scale, void* stream);
 
+/* ---- MoE router without allocation (the pages have no counterpart: this is a library
+ * convenience). For callers that cannot call cudaMalloc - code running inside another
+ * framework's memory pool that owns all device memory, serving loops that forbid
+ * allocation after start-up, or hosts that capture the work into their own CUDA graphs -
+ * and so cannot create a handle. Runs the router kernel of rdt_moe_forward: RMSNorm2 of y
+ * with gain norm2, fp32 logits against w_router, top-k of logits + bias (ties to the lower
+ * expert index), softmax over the k chosen logits, per-expert token counts.
+ *   dtype         : RDT_BF16 or RDT_F32, element type of w_router
+ *   y             : device fp32 [ntok, dim];  norm2 : device fp32 [dim]
+ *   w_router      : device [n_experts, dim];  router_bias : device fp32 [n_experts] or NULL
+ *   topk_idx      : device int32 [ntok, top_k];  topk_w : device fp32 [ntok, top_k]
+ *   expert_counts : device int32 [n_experts] or NULL
+ * No allocation: the kernel's scratch (normalised rows and counters) is one static device
+ * array of 8 MiB that every process loading librdt holds on every GPU it uses until exit.
+ * ntok * dim * element size must not exceed 8 MiB - 4 KiB (RDT_ERR_UNSUPPORTED otherwise);
+ * dim = 128 * 2^k <= 4096, n_experts <= 256, top_k <= min(n_experts, 16).
+ * The first call on a device looks up the array's device address (a runtime call, no
+ * allocation); make that first call before any stream capture. All calls share the array
+ * and the counters are cleared at the start of each call, so calls that overlap on the GPU
+ * (other streams, other threads) race: serialise them. */
+rdt_status rdt_moe_route_noalloc(int32_t dtype, const float* y, const float* norm2,
+                                 const void* w_router, const float* router_bias, int ntok, int dim,
+                                 int n_experts, int top_k, float eps, int32_t* topk_idx,
+                                 float* topk_w, int32_t* expert_counts, void* stream);
+
 /* ---- per-kernel timing (CUDA events recorded around every launch of the handle) */
 typedef struct {
     char name[32];          /* kernel class, e.g. "gemm_up", "attention", "norm2_router" */

@@ -34,7 +34,7 @@ STATUS = {0: "RDT_OK", 1: "RDT_ERR_INVALID_ARG", 2: "RDT_ERR_UNSUPPORTED", 3: "R
 EXPORTED = ("rdt_create", "rdt_attn_forward", "rdt_moe_forward", "rdt_loop_forward",
             "rdt_loop_forward_host", "rdt_set_trace", "rdt_get_diagnostics", "rdt_memory_bytes",
             "rdt_status_string", "rdt_last_error", "rdt_destroy", "rdt_matmul", "rdt_attention",
-            "rdt_profile", "rdt_profile_read")
+            "rdt_profile", "rdt_profile_read", "rdt_moe_route_noalloc")
 
 
 class RdtError(RuntimeError):
@@ -100,6 +100,8 @@ def load_library() -> ctypes.CDLL:
     lib.rdt_destroy.argtypes = [vp]
     lib.rdt_destroy.restype = None
     lib.rdt_matmul.argtypes = [i32, vp, vp, vp, i32, i32, i32, vp]
+    lib.rdt_moe_route_noalloc.argtypes = [i32, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
+                                          vp, vp, vp, vp]
     lib.rdt_profile.argtypes = [vp, i32]
     lib.rdt_profile_read.argtypes = [vp, ctypes.POINTER(RdtKernelStat), i32, ctypes.POINTER(i32),
                                      ctypes.POINTER(ctypes.c_int64)]
@@ -107,7 +109,7 @@ def load_library() -> ctypes.CDLL:
                                   ctypes.c_float, vp]
     for f in ("rdt_create", "rdt_attn_forward", "rdt_moe_forward", "rdt_loop_forward",
               "rdt_loop_forward_host", "rdt_set_trace", "rdt_get_diagnostics", "rdt_memory_bytes",
-              "rdt_matmul", "rdt_attention", "rdt_profile", "rdt_profile_read"):
+              "rdt_matmul", "rdt_attention", "rdt_profile", "rdt_profile_read", "rdt_moe_route_noalloc"):
         getattr(lib, f).restype = i32
     _LIB = lib
     return lib
