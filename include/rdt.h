@@ -218,9 +218,10 @@ rdt_status rdt_attention(int32_t dtype, const void* q, const void* k, const void
  *   w_router      : device [n_experts, dim];  router_bias : device fp32 [n_experts] or NULL
  *   topk_idx      : device int32 [ntok, top_k];  topk_w : device fp32 [ntok, top_k]
  *   expert_counts : device int32 [n_experts] or NULL
- * No allocation: the kernel's scratch (normalised rows and counters) is one static device
- * array of 8 MiB that every process loading librdt holds on every GPU it uses until exit.
- * ntok * dim * element size must not exceed 8 MiB - 4 KiB (RDT_ERR_UNSUPPORTED otherwise);
+ * No allocation: the kernels' scratch (normalised rows, for bf16 also their residuals, and
+ * counters) is one static device array of 8 MiB that every process loading librdt holds
+ * on every GPU it uses until exit. 2 * ntok * dim * 2 bytes (bf16) or ntok * dim * 4 bytes
+ * (fp32) must not exceed 8 MiB - 4 KiB (RDT_ERR_UNSUPPORTED otherwise);
  * dim = 128 * 2^k <= 4096, n_experts <= 256, top_k <= min(n_experts, 16).
  * The first call on a device looks up the array's device address (a runtime call, no
  * allocation); make that first call before any stream capture. All calls share the array

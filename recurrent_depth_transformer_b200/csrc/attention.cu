@@ -74,6 +74,8 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const AttnArgs a) {
     bf16* sK = sQ + kBM * SQ;
     bf16* sV = sK + 2 * kBN * SQ;
 
+    pdl_trigger();
+    pdl_wait();
     const int qb = gridDim.x - 1 - blockIdx.x;
     const int h = blockIdx.y;
     const int b = blockIdx.z;
@@ -217,6 +219,8 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const AttnArgs a) {
 
 template <int DQK, int DV>
 __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnArgs a) {
+    pdl_trigger();
+    pdl_wait();
     const int tid = blockIdx.x * blockDim.x + threadIdx.x;
     if (tid >= a.batch * a.hq * a.seq) return;
     const int s = tid % a.seq;
@@ -263,16 +267,14 @@ rdt_status launch_bf16(const AttnArgs& a, cudaStream_t st) {
         configured = true;
     }
     const dim3 grid((a.seq + kBM - 1) / kBM, a.hq, a.batch);
-    attn_bf16_kernel<DQK, DV><<<grid, 128, smem, st>>>(a);
-    RDT_CUDA_TRY(cudaGetLastError());
+    RDT_CUDA_TRY(launch_pdl(attn_bf16_kernel<DQK, DV>, grid, dim3(128), smem, st, a));
     return RDT_OK;
 }
 
 template <int DQK, int DV>
 rdt_status launch_f32(const AttnArgs& a, cudaStream_t st) {
     const int n = a.batch * a.hq * a.seq;
-    attn_f32_kernel<DQK, DV><<<(n + 127) / 128, 128, 0, st>>>(a);
-    RDT_CUDA_TRY(cudaGetLastError());
+    RDT_CUDA_TRY(launch_pdl(attn_f32_kernel<DQK, DV>, dim3((n + 127) / 128), dim3(128), 0, st, a));
     return RDT_OK;
 }
 

@@ -18,6 +18,7 @@
 //                   (h_{t+1} = A h + B e + a + sum_j w_j E_j(yn)).
 // Grouped mode reads a device-resident tile list (expert, A row, output row, rows), so
 // the per-expert row counts never travel to the host.
+#include <algorithm>
 #include <type_traits>
 
 #include "rdt_internal.cuh"
@@ -31,11 +32,12 @@ constexpr int kThreads = 192;
 
 template <int BN>
 struct TcCfg {
-    static constexpr int STAGES = (BN <= 128) ? 6 : 4;
+    static constexpr int STAGES = (BN <= 64) ? 8 : (BN <= 128) ? 6 : 4;
     static constexpr int A_BYTES = BM * 128;
     static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int TMEM_COLS = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+    // two accumulators of BN fp32 columns, rounded up to a power of two
+    static constexpr int TMEM_COLS = 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
     static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
     static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte alignment of stages");
 };
@@ -57,30 +59,68 @@ __device__ __forceinline__ void store_row32(OutT* p, const float (&v)[32]) {
     }
 }
 
-// Rotary embedding: the pair (i, i + R/2) turns by angle pos * base^(-2i/R); the table
-// rows hold cos/sin of those angles for one position.
-template <int R>
-__device__ __forceinline__ void rope_rotate(float (&v)[32], const float* cosr, const float* sinr) {
-#pragma unroll
-    for (int i = 0; i < R / 2; ++i) {
-        const float c = cosr[i], s = sinr[i];
-        const float x1 = v[i], x2 = v[i + R / 2];
-        v[i] = x1 * c - x2 * s;
-        v[i + R / 2] = x2 * c + x1 * s;
-    }
-}
-__device__ __forceinline__ void rope_rotate_pair(float (&lo)[32], float (&hi)[32],
-                                                 const float* cosr, const float* sinr) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const float c = cosr[i], s = sinr[i];
-        const float x1 = lo[i], x2 = hi[i];
-        lo[i] = x1 * c - x2 * s;
-        hi[i] = x2 * c + x1 * s;
-    }
-}
-
 // ----------------------------------------------------------------------------- epilogues
+
+// Router epilogue: the thread's row holds the logits of all experts (BN >= n_exp). Keeps the
+// KMAX best (score = logit + bias) in registers, visiting experts in ascending index so that
+// strict comparisons leave ties to the lower index; gate weights are the softmax of the
+// chosen logits.
+template <int BN, int KMAX>
+__device__ __forceinline__ void epilogue_topk(const EpiParams& p, uint32_t taddr, bool valid, int crow) {
+    float bs[KMAX], bl[KMAX];
+    int bi[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+        bs[j] = -INFINITY;
+        bl[j] = 0.0f;
+        bi[j] = -1;
+    }
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        ld_chunk(taddr, c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int ex = c * 32 + i;
+            if (ex >= p.n_exp) break;
+            float cs = v[i] + (p.bias ? p.bias[ex] : 0.0f);
+            float cl = v[i];
+            int ci = ex;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                if (j < p.top_k && cs > bs[j]) {
+                    const float ts = bs[j], tl = bl[j];
+                    const int ti = bi[j];
+                    bs[j] = cs; bl[j] = cl; bi[j] = ci;
+                    cs = ts; cl = tl; ci = ti;
+                }
+            }
+        }
+    }
+    if (!valid) return;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+        if (j < p.top_k && bi[j] >= 0) mx = fmaxf(mx, bl[j]);
+    float ex[KMAX], den = 0.0f;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+        ex[j] = (j < p.top_k && bi[j] >= 0) ? expf(bl[j] - mx) : 0.0f;
+        den += ex[j];
+    }
+    const size_t o = static_cast<size_t>(crow) * p.top_k;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+        if (j >= p.top_k) break;
+        const int e = bi[j] < 0 ? 0 : bi[j];      // only when every score was NaN
+        const float w = den > 0.0f ? ex[j] / den : 0.0f;
+        p.idx_out[o + j] = e;
+        p.w_out[o + j] = w;
+        if (p.trace_idx) p.trace_idx[o + j] = e;
+        if (p.trace_w) p.trace_w[o + j] = w;
+        atomicAdd(p.counts + e, 1);
+    }
+}
 
 template <typename T, int BN, int KIND>
 __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, bool valid, int crow,
@@ -97,12 +137,15 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, boo
         }
     } else if constexpr (KIND == EPI_ROPE) {
         // Heads of width head_w tile the BN columns exactly (host checks BN % head_w == 0).
+        // The angle tables are [rot/2][seq]: for a fixed frequency the lanes (consecutive
+        // positions) read consecutive floats.
         const int pos = crow % p.seq;
         const int hw_chunks = p.head_w / 32;
         const int rc0 = p.rot_off / 32;
         const int rch = p.rot_dim / 32;
-        const float* cosr = p.rope_cos + static_cast<size_t>(pos) * (p.rot_dim / 2);
-        const float* sinr = p.rope_sin + static_cast<size_t>(pos) * (p.rot_dim / 2);
+        const float* cosr = p.rope_cos + pos;
+        const float* sinr = p.rope_sin + pos;
+        const int ts = p.seq;
         T* out = static_cast<T*>(p.out) + static_cast<size_t>(crow) * p.ldo;
 #pragma unroll 1
         for (int hc = 0; hc < BN / 32; hc += hw_chunks) {
@@ -116,7 +159,13 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, boo
                         float v0[32], v1[32];
                         ld_chunk(taddr, hc + c, v0);
                         ld_chunk(taddr, hc + c + 1, v1);
-                        rope_rotate_pair(v0, v1, cosr, sinr);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float cs = cosr[i * ts], sn = sinr[i * ts];
+                            const float x1 = v0[i], x2 = v1[i];
+                            v0[i] = x1 * cs - x2 * sn;
+                            v1[i] = x2 * cs + x1 * sn;
+                        }
                         if (valid && col < p.ncols_valid) {
                             store_row32(out + col, v0);
                             store_row32(out + col + 32, v1);
@@ -125,7 +174,13 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, boo
                     } else {
                         float v[32];
                         ld_chunk(taddr, hc + c, v);
-                        rope_rotate<32>(v, cosr, sinr);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float cs = cosr[i * ts], sn = sinr[i * ts];
+                            const float x1 = v[i], x2 = v[i + 16];
+                            v[i] = x1 * cs - x2 * sn;
+                            v[i + 16] = x2 * cs + x1 * sn;
+                        }
                         if (valid && col < p.ncols_valid) store_row32(out + col, v);
                     }
                 } else {
@@ -208,11 +263,46 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, boo
                 atomicAdd(reinterpret_cast<float4*>(dst + col + 4 * j), add);
             }
         }
+    } else if constexpr (KIND == EPI_TOPK) {
+        if (p.top_k <= 2)
+            epilogue_topk<BN, 2>(p, taddr, valid, crow);
+        else if (p.top_k <= 4)
+            epilogue_topk<BN, 4>(p, taddr, valid, crow);
+        else if (p.top_k <= 8)
+            epilogue_topk<BN, 8>(p, taddr, valid, crow);
+        else
+            epilogue_topk<BN, 16>(p, taddr, valid, crow);
     }
 }
 
 // ----------------------------------------------------------------------------- the kernel
 
+struct TileCoord {
+    int a_row0, c_row0, nrows, group, n0;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const GemmArgs& args, int tile, int n_ntiles, int bn) {
+    TileCoord t;
+    const int mt = tile / n_ntiles;
+    t.n0 = (tile - mt * n_ntiles) * bn;
+    if (args.tiles != nullptr) {
+        const GroupTile g = args.tiles[mt];
+        t.group = g.group;
+        t.a_row0 = args.a_from_c ? g.c_row0 : g.a_row0;
+        t.c_row0 = g.c_row0;
+        t.nrows = g.nrows;
+    } else {
+        t.group = 0;
+        t.a_row0 = mt * BM;
+        t.c_row0 = t.a_row0;
+        t.nrows = min(BM, args.M - t.a_row0);
+    }
+    return t;
+}
+
+// Persistent: each CTA walks tiles blockIdx.x, blockIdx.x + gridDim.x, ... The TMA warp
+// and the MMA warp run ahead through a ring of shared-memory stages; the accumulator is
+// double-buffered in TMEM so the epilogue of one tile overlaps the MMAs of the next.
 template <typename T, int BN, int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
@@ -227,28 +317,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
     uint64_t* empty = full + C::STAGES;
-    uint64_t* done = empty + C::STAGES;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* tfull = empty + C::STAGES;      // accumulator b ready for the epilogue
+    uint64_t* tempty = tfull + 2;             // accumulator b drained by the epilogue
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    int a_row0, c_row0, nrows, group = 0;
-    if (args.tiles != nullptr) {
-        if (static_cast<int>(blockIdx.y) >= *args.n_tiles) return;   // uniform per CTA
-        const GroupTile t = args.tiles[blockIdx.y];
-        group = t.group;
-        a_row0 = args.a_from_c ? t.c_row0 : t.a_row0;
-        c_row0 = t.c_row0;
-        nrows = t.nrows;
-    } else {
-        a_row0 = blockIdx.y * BM;
-        c_row0 = a_row0;
-        nrows = min(BM, args.M - a_row0);
-    }
-    const int n0 = blockIdx.x * BN;
-    const int b_row0 = group * args.N + n0;
-    const int num_kb = args.kb_main + args.kb_ext;
 
     if (threadIdx.x == 0) {
 #pragma unroll 1
@@ -256,8 +330,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(done, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);         // one arrival per epilogue warp
+        }
         mbar_fence_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tA);
+        tma_prefetch_desc(&tB);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -267,60 +348,99 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_trigger();
+    pdl_wait();
+
+    const int n_ntiles = (args.N + BN - 1) / BN;
+    const int n_mtiles = args.tiles != nullptr ? min(*args.n_tiles, args.max_tiles)
+                                               : (args.M + BM - 1) / BM;
+    const int total = n_mtiles * n_ntiles;
+    const int num_kb = args.kb_main + args.kb_ext;
 
     if (warp == 0) {
         if (lane == 0) {
-            tma_prefetch_desc(&tA);
-            tma_prefetch_desc(&tB);
+            int it = 0;
+            bool ok = true;
 #pragma unroll 1
-            for (int kb = 0; kb < num_kb; ++kb) {
-                const int s = kb % C::STAGES;
-                const uint32_t ph = (kb / C::STAGES) & 1;
-                if (!mbar_wait(&empty[s], ph ^ 1, epi.flags)) break;
-                uint8_t* sa = smem + s * C::STAGE_BYTES;
-                uint8_t* sb = sa + C::A_BYTES;
-                mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-                if (kb < args.kb_main) {
-                    tma_load_2d(sa, &tA, &full[s], kb * kElemsPerRow, a_row0);
-                    tma_load_2d(sb, &tB, &full[s], kb * kElemsPerRow, b_row0);
-                } else {
-                    tma_load_2d(sa, &tA2, &full[s], 0, a_row0);
-                    tma_load_2d(sb, &tB2, &full[s], 0, args.b2_row0 + n0);
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const TileCoord tc = tile_coord(args, tile, n_ntiles, BN);
+                const int b_row0 = tc.group * args.N + tc.n0;
+#pragma unroll 1
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t ph = (it / C::STAGES) & 1;
+                    if (!mbar_wait(&empty[s], ph ^ 1, epi.flags)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + s * C::STAGE_BYTES;
+                    uint8_t* sb = sa + C::A_BYTES;
+                    mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+                    if (kb < args.kb_main) {
+                        tma_load_2d(sa, &tA, &full[s], kb * kElemsPerRow, tc.a_row0);
+                        tma_load_2d(sb, &tB, &full[s], kb * kElemsPerRow, b_row0);
+                    } else {
+                        const int kx = (kb - args.kb_main) * kElemsPerRow;
+                        tma_load_2d(sa, &tA2, &full[s], kx, tc.a_row0);
+                        tma_load_2d(sb, &tB2, &full[s], kx, args.b2_row0 + b_row0);
+                    }
                 }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = make_idesc(kBf16 ? 1 : 2, BM, BN);
+            int it = 0, local = 0;
+            bool ok = true;
 #pragma unroll 1
-            for (int kb = 0; kb < num_kb; ++kb) {
-                const int s = kb % C::STAGES;
-                const uint32_t ph = (kb / C::STAGES) & 1;
-                if (!mbar_wait(&full[s], ph, epi.flags)) break;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
+                const int b = local & 1;
+                const uint32_t use = static_cast<uint32_t>(local >> 1);
+                if (!mbar_wait(&tempty[b], (use & 1) ^ 1, epi.flags)) break;
                 tc_fence_after();
-                const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
-                const uint64_t da = sw128_kmajor_desc(sa);
-                const uint64_t db = sw128_kmajor_desc(sa + C::A_BYTES);
+                const uint32_t dt = tmem + static_cast<uint32_t>(b * BN);
+#pragma unroll 1
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t ph = (it / C::STAGES) & 1;
+                    if (!mbar_wait(&full[s], ph, epi.flags)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+                    const uint64_t da = sw128_kmajor_desc(sa);
+                    const uint64_t db = sw128_kmajor_desc(sa + C::A_BYTES);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    // each MMA consumes 32 bytes of K: advance the start address by 32 B (>> 4 = 2)
-                    if constexpr (kBf16)
-                        tc_mma_bf16(tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
-                    else
-                        tc_mma_tf32(tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                    for (int k = 0; k < 4; ++k) {
+                        // each MMA consumes 32 bytes of K: advance the start address by 32 B (>> 4 = 2)
+                        if constexpr (kBf16)
+                            tc_mma_bf16(dt, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                        else
+                            tc_mma_tf32(dt, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                    }
+                    tc_commit(&empty[s]);
                 }
-                tc_commit(&empty[s]);
+                tc_commit(&tfull[b]);
             }
-            tc_commit(done);
         }
     } else {
         const int q = warp & 3;            // TMEM lane quadrant accessible to this warp
         const int r = q * 32 + lane;       // row inside the tile
-        const bool ok = mbar_wait(done, 0, epi.flags);
-        tc_fence_after();
-        if (ok)
-            epilogue<T, BN, KIND>(epi, tmem + (static_cast<uint32_t>(q * 32) << 16), r < nrows,
-                                  c_row0 + r, n0);
+        int local = 0;
+#pragma unroll 1
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+            const int b = local & 1;
+            const uint32_t use = static_cast<uint32_t>(local >> 1);
+            if (!mbar_wait(&tfull[b], use & 1, epi.flags)) break;
+            tc_fence_after();
+            const TileCoord tc = tile_coord(args, tile, n_ntiles, BN);
+            epilogue<T, BN, KIND>(epi, tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN,
+                                  r < tc.nrows, tc.c_row0 + r, tc.n0);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[b]);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -342,11 +462,13 @@ rdt_status launch(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMa
                                           C::SMEM));
         configured = true;
     }
-    const int gy = args.tiles ? args.max_tiles : (args.M + BM - 1) / BM;
-    const dim3 grid((args.N + BN - 1) / BN, gy);
-    if (gy <= 0) return RDT_OK;
-    kern<<<grid, kThreads, C::SMEM, st>>>(tA, tB, tA2 ? *tA2 : tA, tB2 ? *tB2 : tB, args, epi);
-    RDT_CUDA_TRY(cudaGetLastError());
+    const int n_ntiles = (args.N + BN - 1) / BN;
+    const long mt = args.tiles ? args.max_tiles : (args.M + BM - 1) / BM;
+    const long total = mt * n_ntiles;
+    if (total <= 0) return RDT_OK;
+    const int grid = static_cast<int>(std::min<long>(total, num_sms()));
+    RDT_CUDA_TRY(launch_pdl(kern, dim3(grid), dim3(kThreads), C::SMEM, st, tA, tB, tA2 ? *tA2 : tA,
+                            tB2 ? *tB2 : tB, args, epi));
     return RDT_OK;
 }
 
@@ -366,11 +488,29 @@ rdt_status dispatch_kind(const CUtensorMap& tA, const CUtensorMap& tB, const CUt
     }
 }
 
+template <typename T, int BN>
+rdt_status dispatch_router(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap* tA2,
+                           const CUtensorMap* tB2, const GemmArgs& args, const EpiParams& epi,
+                           cudaStream_t st) {
+    return launch<T, BN, EPI_TOPK>(tA, tB, tA2, tB2, args, epi, st);
+}
+
 }  // namespace
 
 rdt_status gemm_tc(bool bf16_elems, int bn, const CUtensorMap& tA, const CUtensorMap& tB,
                    const CUtensorMap* tA2, const CUtensorMap* tB2, const GemmArgs& args,
                    const EpiParams& epi, cudaStream_t st) {
+    if (epi.kind == EPI_TOPK) {
+        if (bf16_elems) {
+            if (bn == 64) return dispatch_router<bf16, 64>(tA, tB, tA2, tB2, args, epi, st);
+            if (bn == 128) return dispatch_router<bf16, 128>(tA, tB, tA2, tB2, args, epi, st);
+            if (bn == 256) return dispatch_router<bf16, 256>(tA, tB, tA2, tB2, args, epi, st);
+        } else {
+            if (bn == 64) return dispatch_router<float, 64>(tA, tB, tA2, tB2, args, epi, st);
+        }
+        set_error("router: unsupported expert count");
+        return RDT_ERR_UNSUPPORTED;
+    }
     if (bf16_elems) {
         if (bn == 128) return dispatch_kind<bf16, 128>(tA, tB, tA2, tB2, args, epi, st);
         if (bn == 160) return dispatch_kind<bf16, 160>(tA, tB, tA2, tB2, args, epi, st);
@@ -380,6 +520,19 @@ rdt_status gemm_tc(bool bf16_elems, int bn, const CUtensorMap& tA, const CUtenso
     }
     set_error("gemm_tc: unsupported tile width");
     return RDT_ERR_UNSUPPORTED;
+}
+
+int num_sms() {
+    static int n[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (!n[dev]) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        n[dev] = v > 0 ? v : 148;
+    }
+    return n[dev];
 }
 
 // ----------------------------------------------------------------------------- tensor maps

@@ -1,10 +1,12 @@
 // MoE router for callers that cannot allocate device memory.
 //
-// rdt_moe_route_noalloc runs the same router kernel as rdt_moe_forward (RMSNorm2 of y,
-// fp32 logits, top-k, softmax over the chosen logits, per-expert histogram) without a
-// handle and without any allocation. The kernel's scratch - the normalised rows it writes
-// for the experts and the per-expert counters - lives in the file-scope array below,
-// which every process that loads librdt holds on every GPU it uses until exit.
+// rdt_moe_route_noalloc runs the router of rdt_moe_forward (RMSNorm2 of y, logits of the
+// fp32 normalised row, top-k, softmax over the chosen logits, per-expert histogram) without
+// a handle and without any allocation: bf16 routers use the same RMSNorm2 split kernel and
+// tensor-core router GEMM as the handle, fp32 routers the same fp32 FMA kernel. Their
+// scratch - the normalised rows (and, for bf16, their residuals) and the per-expert
+// counters - lives in the file-scope array below, which every process that loads librdt
+// holds on every GPU it uses until exit.
 #include <mutex>
 
 #include "rdt_internal.cuh"
@@ -78,12 +80,14 @@ extern "C" rdt_status rdt_moe_route_noalloc(int32_t dtype, const float* y, const
         set_error("need 1 <= top_k <= min(n_experts, 16) and n_experts <= 256");
         return RDT_ERR_UNSUPPORTED;
     }
-    const size_t esz = dtype == RDT_BF16 ? 2 : 4;
-    const size_t rows_bytes = static_cast<size_t>(ntok) * dim * esz;
-    if (rows_bytes > kScratchBytes - kCountsBytes) {
-        set_error("ntok * dim * element size = " + std::to_string(rows_bytes) +
-                  " bytes exceeds the router scratch of " +
-                  std::to_string(kScratchBytes - kCountsBytes) + " bytes");
+    const bool bf = dtype == RDT_BF16;
+    const size_t esz = bf ? 2 : 4;
+    const size_t row_bytes = static_cast<size_t>(ntok) * dim * esz;
+    const size_t need = bf ? 2 * row_bytes : row_bytes;   // bf16: yn and its residual yn_lo
+    if (need > kScratchBytes - kCountsBytes) {
+        set_error("the router needs " + std::to_string(need) + " bytes of scratch for ntok = " +
+                  std::to_string(ntok) + ", dim = " + std::to_string(dim) + "; the array holds " +
+                  std::to_string(kScratchBytes - kCountsBytes));
         return RDT_ERR_UNSUPPORTED;
     }
     void* base = nullptr;
@@ -91,23 +95,57 @@ extern "C" rdt_status rdt_moe_route_noalloc(int32_t dtype, const float* y, const
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int* counts = static_cast<int*>(base);
     void* yn = static_cast<unsigned char*>(base) + kCountsBytes;
+    void* yn_lo = static_cast<unsigned char*>(yn) + row_bytes;
     RDT_CUDA_TRY(cudaMemsetAsync(counts, 0, kCountsBytes, st));   // the counters start at zero
 
-    RouterArgs ra{};
-    ra.y = y;
-    ra.gamma = norm2;
-    ra.yn = yn;
-    ra.ntok = ntok;
-    ra.dim = dim;
-    ra.eps = eps;
-    ra.w_router = w_router;
-    ra.bias = router_bias;
-    ra.n_exp = n_experts;
-    ra.top_k = top_k;
-    ra.idx = topk_idx;
-    ra.w = topk_w;
-    ra.counts = counts;
-    RDT_TRY(norm2_router(dtype == RDT_BF16, ra, st));
+    if (bf) {
+        // the same two steps as rdt_moe_forward: RMSNorm2 split into yn + yn_lo, then the
+        // tensor-core router GEMM [yn | yn_lo] . [W_r | W_r]^T with the top-k epilogue
+        Norm2Args n2{};
+        n2.y = y;
+        n2.gamma = norm2;
+        n2.yn = yn;
+        n2.yn_lo = yn_lo;
+        n2.ntok = ntok;
+        n2.dim = dim;
+        n2.eps = eps;
+        RDT_TRY(norm2_split(true, n2, st));
+        const int bn = n_experts <= 64 ? 64 : n_experts <= 128 ? 128 : 256;
+        CUtensorMap m_yn, m_lo, m_wr;   // host-side descriptors: encoding allocates nothing
+        RDT_TRY(make_tmap_2d(&m_yn, yn, true, dim, ntok, static_cast<uint64_t>(dim) * 2, 64, 128));
+        RDT_TRY(make_tmap_2d(&m_lo, yn_lo, true, dim, ntok, static_cast<uint64_t>(dim) * 2, 64, 128));
+        RDT_TRY(make_tmap_2d(&m_wr, w_router, true, dim, n_experts, static_cast<uint64_t>(dim) * 2, 64, bn));
+        GemmArgs gr{};
+        gr.M = ntok;
+        gr.N = n_experts;
+        gr.kb_main = dim * 2 / 128;
+        gr.kb_ext = gr.kb_main;
+        EpiParams er{};
+        er.kind = EPI_TOPK;
+        er.n_exp = n_experts;
+        er.top_k = top_k;
+        er.bias = router_bias;
+        er.idx_out = topk_idx;
+        er.w_out = topk_w;
+        er.counts = counts;
+        RDT_TRY(gemm_tc(true, bn, m_yn, m_wr, &m_lo, &m_wr, gr, er, st));
+    } else {
+        RouterArgs ra{};
+        ra.y = y;
+        ra.gamma = norm2;
+        ra.yn = yn;
+        ra.ntok = ntok;
+        ra.dim = dim;
+        ra.eps = eps;
+        ra.w_router = w_router;
+        ra.bias = router_bias;
+        ra.n_exp = n_experts;
+        ra.top_k = top_k;
+        ra.idx = topk_idx;
+        ra.w = topk_w;
+        ra.counts = counts;
+        RDT_TRY(norm2_router(false, ra, st));
+    }
     if (expert_counts)
         RDT_CUDA_TRY(cudaMemcpyAsync(expert_counts, counts, static_cast<size_t>(n_experts) * 4,
                                      cudaMemcpyDeviceToDevice, st));

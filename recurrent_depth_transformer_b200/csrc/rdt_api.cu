@@ -54,7 +54,8 @@ struct rdt_handle {
     // workspace
     float *hbuf[2] = {nullptr, nullptr}, *Be = nullptr, *y = nullptr, *lat = nullptr;
     void *xn = nullptr, *tq = nullptr, *to = nullptr, *qkv = nullptr, *o = nullptr;
-    void *cq = nullptr, *kvlat = nullptr, *xperm = nullptr, *U = nullptr;
+    void *cq = nullptr, *kvlat = nullptr, *xperm = nullptr, *U = nullptr, *yn_lo = nullptr;
+    int bn_router = 64;
     int32_t* idx = nullptr;
     float* wts = nullptr;
     int *counts = nullptr, *offsets = nullptr, *fill = nullptr, *ntiles = nullptr, *row_token = nullptr;
@@ -67,7 +68,7 @@ struct rdt_handle {
 
     // tensor maps
     CUtensorMap m_xn, m_wqkv, m_tq, m_lqb, m_o, m_wo, m_to, m_lob, m_xperm, m_w13, m_U, m_w2;
-    CUtensorMap m_wlat, m_cq, m_wqabs;
+    CUtensorMap m_wlat, m_cq, m_wqabs, m_ynlo, m_wr;
 
     // trace
     int32_t* tr_idx = nullptr;
@@ -79,6 +80,18 @@ struct rdt_handle {
     bool prof_on = false;
     std::vector<cudaEvent_t> ev_pool;
     size_t ev_used = 0;
+    // CUDA graph of the whole T-loop launch sequence, keyed by the call's pointers and T
+    struct GraphKey {
+        const void* h0 = nullptr;
+        const void* e = nullptr;
+        const float* out = nullptr;
+        int T = 0;
+        bool operator==(const GraphKey& o) const { return h0 == o.h0 && e == o.e && out == o.out && T == o.T; }
+    };
+    cudaStream_t cap_stream = nullptr;
+    cudaGraphExec_t gexec = nullptr;
+    GraphKey gkey, seen_key;
+    int64_t g_launches = 0;
     struct Pending { int kind; cudaEvent_t a, b; int n; };
     std::vector<Pending> pending;
     std::vector<double> prof_ms;
@@ -89,10 +102,10 @@ namespace {
 
 // kernel classes reported by rdt_profile_read
 enum Kind { K_HOIST, K_NORM1, K_GEMM_QKV, K_GEMM_LAT, K_MLA_NORM, K_GEMM_Q, K_ATTENTION, K_LORA_DOWN,
-            K_GEMM_O, K_NORM2_ROUTER, K_DISPATCH, K_GEMM_UP, K_GEMM_DOWN, K_CHECK, K_DENSE_B, K_COUNT };
+            K_GEMM_O, K_NORM2, K_ROUTER, K_DISPATCH, K_GEMM_UP, K_GEMM_DOWN, K_CHECK, K_DENSE_B, K_COUNT };
 const char* const kKindName[K_COUNT] = {"hoist", "norm1", "gemm_qkv", "gemm_latent", "mla_latent_norm",
                                          "gemm_q_absorbed", "attention", "lora_down", "gemm_o",
-                                         "norm2_router", "moe_dispatch", "gemm_up", "gemm_down",
+                                         "norm2", "router_topk", "moe_dispatch", "gemm_up", "gemm_down",
                                          "check_finite", "dense_injection"};
 
 rdt_status prof_begin(rdt_handle* h, int kind, int nlaunch, cudaStream_t st) {
@@ -165,6 +178,7 @@ rdt_status validate_config(const rdt_config* c) {
     if (c->n_experts < 1 || c->top_k < 1 || c->top_k > c->n_experts) return bad("n_experts / top_k");
     if (c->top_k > 16) return uns("top_k > 16");
     if (c->n_shared < 0 || c->n_experts + c->n_shared > 256) return uns("n_experts + n_shared > 256");
+    if (c->dtype == RDT_F32 && c->n_experts > 64) return uns("f32: n_experts > 64");
     if (c->expert_hidden < 64 || c->expert_hidden % 64) return uns("expert_hidden % 64 != 0");
     if (c->dtype == RDT_F32 && c->expert_hidden % 128) return uns("f32: expert_hidden % 128 != 0");
     if (c->max_loops < 1 || c->max_loops > 64) return bad("max_loops must be in [1, 64]");
@@ -251,6 +265,8 @@ rdt_status build_maps(rdt_handle* h) {
     RDT_TRY(make_tmap_2d(&h->m_w13, h->w13, bf, d, static_cast<uint64_t>(E + S) * 2 * hid, d * es, kbox, 128));
     RDT_TRY(make_tmap_2d(&h->m_U, h->U, bf, hid, urows, hid * es, kbox, 128));
     RDT_TRY(make_tmap_2d(&h->m_w2, h->w2, bf, hid, static_cast<uint64_t>(E + S) * d, hid * es, kbox, 128));
+    RDT_TRY(make_tmap_2d(&h->m_ynlo, h->yn_lo, bf, d, N, d * es, kbox, 128));
+    RDT_TRY(make_tmap_2d(&h->m_wr, h->wr, bf, d, E, d * es, kbox, h->bn_router));
     return RDT_OK;
 }
 
@@ -436,15 +452,16 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         }
     }
 
-    // RoPE tables [seq, rot/2] from double-precision angles
+    // RoPE tables [rot/2][seq] (frequency-major, so that consecutive positions are adjacent)
+    // from double-precision angles
     {
         const int half = h->rot / 2;
         std::vector<float> cs(static_cast<size_t>(c.seq) * half), sn(cs.size());
-        for (int p = 0; p < c.seq; ++p)
-            for (int i = 0; i < half; ++i) {
+        for (int i = 0; i < half; ++i)
+            for (int p = 0; p < c.seq; ++p) {
                 const double ang = p * std::pow(static_cast<double>(c.rope_base), -2.0 * i / h->rot);
-                cs[static_cast<size_t>(p) * half + i] = static_cast<float>(std::cos(ang));
-                sn[static_cast<size_t>(p) * half + i] = static_cast<float>(std::sin(ang));
+                cs[static_cast<size_t>(i) * c.seq + p] = static_cast<float>(std::cos(ang));
+                sn[static_cast<size_t>(i) * c.seq + p] = static_cast<float>(std::sin(ang));
             }
         RDT_TRY(dev_alloc(h, &h->rope_cos, cs.size() * 4));
         RDT_TRY(dev_alloc(h, &h->rope_sin, sn.size() * 4));
@@ -474,6 +491,8 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
     RDT_TRY(dev_alloc(h, &h->o, static_cast<size_t>(N) * h->owidth * es));
     RDT_TRY(dev_alloc(h, &h->xperm, static_cast<size_t>(N) * (1 + K) * d * es, true));
     RDT_TRY(dev_alloc(h, &h->U, static_cast<size_t>(N) * (S + K) * hid * es, true));
+    RDT_TRY(dev_alloc(h, &h->yn_lo, nd * es, true));
+    h->bn_router = E <= 64 ? 64 : E <= 128 ? 128 : 256;
     RDT_TRY(dev_alloc(h, &h->idx, static_cast<size_t>(N) * K * 4));
     RDT_TRY(dev_alloc(h, &h->wts, static_cast<size_t>(N) * K * 4));
     RDT_TRY(dev_alloc(h, &h->counts, 256 * 4, true));
@@ -660,28 +679,64 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
     return RDT_OK;
 }
 
-// ---- the MoE sublayer: norm2 + router -> dispatch -> experts; adds into dst
+// ---- the MoE sublayer: norm2 -> router (tensor cores, top-k epilogue) -> dispatch -> experts;
+// adds into dst
 rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_out, float* w_out,
                      int32_t* tr_idx, float* tr_w, cudaStream_t st) {
     const rdt_config& c = h->cfg;
     const int N = h->ntok, d = c.dim, hid = c.expert_hidden;
-    RouterArgs ra{};
-    ra.y = yin;
-    ra.gamma = h->g2;
-    ra.yn = h->xperm;
-    ra.ntok = N;
-    ra.dim = d;
-    ra.eps = c.norm_eps;
-    ra.w_router = h->wr;
-    ra.bias = h->rbias;
-    ra.n_exp = c.n_experts;
-    ra.top_k = c.top_k;
-    ra.idx = idx_out ? idx_out : h->idx;
-    ra.w = w_out ? w_out : h->wts;
-    ra.counts = h->counts;
-    ra.trace_idx = tr_idx;
-    ra.trace_w = tr_w;
-    TIMED(h, K_NORM2_ROUTER, 1, st, norm2_router(h->bf, ra, st));
+    int32_t* idx = idx_out ? idx_out : h->idx;
+    float* wts = w_out ? w_out : h->wts;
+    if (!h->bf) {
+        // fp32: the tensor cores would read W_r as tf32, so the router stays in fp32 FMA
+        RouterArgs ra{};
+        ra.y = yin;
+        ra.gamma = h->g2;
+        ra.yn = h->xperm;
+        ra.ntok = N;
+        ra.dim = d;
+        ra.eps = c.norm_eps;
+        ra.w_router = h->wr;
+        ra.bias = h->rbias;
+        ra.n_exp = c.n_experts;
+        ra.top_k = c.top_k;
+        ra.idx = idx;
+        ra.w = wts;
+        ra.counts = h->counts;
+        ra.trace_idx = tr_idx;
+        ra.trace_w = tr_w;
+        TIMED(h, K_ROUTER, 1, st, norm2_router(false, ra, st));
+    } else {
+    Norm2Args n2{};
+    n2.y = yin;
+    n2.gamma = h->g2;
+    n2.yn = h->xperm;
+    n2.yn_lo = h->yn_lo;
+    n2.ntok = N;
+    n2.dim = d;
+    n2.eps = c.norm_eps;
+    TIMED(h, K_NORM2, 1, st, norm2_split(h->bf, n2, st));
+
+    GemmArgs gr{};
+    gr.M = N;
+    gr.N = c.n_experts;
+    gr.kb_main = static_cast<int>(d * h->esz / 128);
+    gr.kb_ext = gr.kb_main;
+    gr.b2_row0 = 0;
+    gr.flags = h->flags;
+    EpiParams er{};
+    er.kind = EPI_TOPK;
+    er.n_exp = c.n_experts;
+    er.top_k = c.top_k;
+    er.bias = h->rbias;
+    er.idx_out = idx;
+    er.w_out = wts;
+    er.counts = h->counts;
+    er.trace_idx = tr_idx;
+    er.trace_w = tr_w;
+    er.flags = h->flags;
+    TIMED(h, K_ROUTER, 1, st, gemm_tc(h->bf, h->bn_router, h->m_xperm, h->m_wr, &h->m_ynlo, &h->m_wr, gr, er, st));
+    }
 
     DispatchArgs da{};
     da.counts = h->counts;
@@ -695,8 +750,8 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     da.tiles = h->tiles;
     da.n_tiles = h->ntiles;
     da.max_tiles = h->max_tiles;
-    da.idx = ra.idx;
-    da.w = ra.w;
+    da.idx = idx;
+    da.w = wts;
     da.xperm = h->xperm;
     da.row_token = h->row_token;
     da.row_w = h->row_w;
@@ -757,6 +812,67 @@ rdt_status loop_impl(rdt_handle* h, const void* h0, const void* e, int T, float*
             RDT_CUDA_TRY(cudaMemcpyAsync(h->tr_h + (t + 1) * nd, hnext, nd * 4, cudaMemcpyDeviceToDevice, st));
     }
     TIMED(h, K_CHECK, 1, st, check_finite(out, nd, h->flags, st));
+    return RDT_OK;
+}
+
+void drop_graph(rdt_handle* h) {
+    if (h->gexec) cudaGraphExecDestroy(h->gexec);
+    h->gexec = nullptr;
+    h->gkey = rdt_handle::GraphKey{};
+    h->seen_key = rdt_handle::GraphKey{};
+}
+
+// Runs the loop, replaying a captured CUDA graph when the same pointers and T come back:
+// the first call with a key runs eagerly, the second captures (on the handle's own stream)
+// and launches the graph, later ones only launch it. Tracing or profiling runs eagerly.
+rdt_status run_loop(rdt_handle* h, const void* h0, const void* e, int T, float* out, cudaStream_t st) {
+    const bool graphable = !h->prof_on && !h->tr_idx && !h->tr_w && !h->tr_h;
+    if (!graphable) return loop_impl(h, h0, e, T, out, st);
+    rdt_handle::GraphKey key;
+    key.h0 = h0;
+    key.e = e;
+    key.out = out;
+    key.T = T;
+    if (h->gexec && h->gkey == key) {
+        RDT_CUDA_TRY(cudaGraphLaunch(h->gexec, st));
+        h->launches += h->g_launches;
+        return RDT_OK;
+    }
+    if (!(h->seen_key == key)) {
+        h->seen_key = key;
+        return loop_impl(h, h0, e, T, out, st);
+    }
+    if (h->gexec) {
+        cudaGraphExecDestroy(h->gexec);
+        h->gexec = nullptr;
+    }
+    if (!h->cap_stream) RDT_CUDA_TRY(cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking));
+    const int64_t l0 = h->launches;
+    RDT_CUDA_TRY(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal));
+    const rdt_status s = loop_impl(h, h0, e, T, out, h->cap_stream);
+    cudaGraph_t g = nullptr;
+    const cudaError_t ce = cudaStreamEndCapture(h->cap_stream, &g);
+    if (s != RDT_OK) {
+        if (g) cudaGraphDestroy(g);
+        h->launches = l0;
+        return s;
+    }
+    if (ce != cudaSuccess) {
+        set_error(std::string("stream capture failed: ") + cudaGetErrorString(ce));
+        return RDT_ERR_CUDA;
+    }
+    const cudaError_t ie = cudaGraphInstantiate(&h->gexec, g, 0);
+    cudaGraphDestroy(g);
+    if (ie != cudaSuccess) {
+        h->gexec = nullptr;
+        set_error(std::string("graph instantiation failed: ") + cudaGetErrorString(ie));
+        return RDT_ERR_CUDA;
+    }
+    h->g_launches = h->launches - l0;
+    h->launches = l0;
+    h->gkey = key;
+    RDT_CUDA_TRY(cudaGraphLaunch(h->gexec, st));
+    h->launches += h->g_launches;
     return RDT_OK;
 }
 
@@ -870,7 +986,7 @@ rdt_status rdt_loop_forward(rdt_handle* h, const void* h0, const void* e, int T,
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     h->last_stream = st;
-    return loop_impl(h, h0, e, T, out, st);
+    return run_loop(h, h0, e, T, out, st);
 }
 
 rdt_status rdt_loop_forward_host(rdt_handle* h, const void* h0_host, const void* e_host, int T, float* out_host,
@@ -896,7 +1012,7 @@ rdt_status rdt_loop_forward_host(rdt_handle* h, const void* h0_host, const void*
         RDT_CUDA_TRY(cudaMemcpyAsync(h->stage_h0, h0_host, nd * h->esz, cudaMemcpyHostToDevice, st));
         h0d = h->stage_h0;
     }
-    RDT_TRY(loop_impl(h, h0d, h->stage_e, T, h->stage_out, st));
+    RDT_TRY(run_loop(h, h0d, h->stage_e, T, h->stage_out, st));
     RDT_CUDA_TRY(cudaMemcpyAsync(out_host, h->stage_out, nd * 4, cudaMemcpyDeviceToHost, st));
     RDT_CUDA_TRY(cudaStreamSynchronize(st));
     return RDT_OK;
@@ -970,6 +1086,7 @@ rdt_status rdt_set_trace(rdt_handle* h, int32_t* idx, float* w, float* h_traj) {
     h->tr_idx = idx;
     h->tr_w = w;
     h->tr_h = h_traj;
+    drop_graph(h);
     return RDT_OK;
 }
 
@@ -1010,6 +1127,7 @@ rdt_status rdt_profile(rdt_handle* h, int enable) {
         std::fill(h->prof_n.begin(), h->prof_n.end(), 0);
     }
     h->prof_on = enable != 0;
+    drop_graph(h);
     return RDT_OK;
 }
 
@@ -1050,6 +1168,8 @@ void rdt_destroy(rdt_handle* h) {
     if (!h) return;
     cudaDeviceSynchronize();
     for (cudaEvent_t ev : h->ev_pool) cudaEventDestroy(ev);
+    if (h->gexec) cudaGraphExecDestroy(h->gexec);
+    if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
     for (void* p : h->allocs) cudaFree(p);
     delete h;
 }

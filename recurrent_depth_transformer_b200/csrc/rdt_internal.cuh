@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include <string>
+#include <utility>
 
 #include "../../include/rdt.h"
 
@@ -85,6 +86,34 @@ __device__ __forceinline__ void store4(bf16* p, const float (&v)[4]) {
     x.y = *reinterpret_cast<uint32_t*>(&b);
     *reinterpret_cast<uint2*>(p) = x;
 }
+
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Every kernel of the library is launched with programmatic stream serialisation: it may
+// start while its predecessor finishes, runs only its prologue (shared memory, barriers,
+// TMEM, descriptor prefetch) before pdl_wait(), and touches global memory only after it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+int num_sms();   // SM count of the current device (cached)
 
 // ------------------------------------------------------------------ mbarrier (sm_90+)
 
@@ -258,7 +287,8 @@ enum EpiKind {
     EPI_OPROJ_PLAIN = 3,// a_out = acc                             (fp32)
     EPI_SWIGLU = 4,     // U[row, j] = silu(acc_gate) * acc_up    (OutT)
     EPI_SCATTER = 5,    // dst[token, col] += w * acc             (fp32, vector atomics)
-    EPI_STORE_F32 = 6   // C[row, col] = acc                     (fp32)
+    EPI_STORE_F32 = 6,  // C[row, col] = acc                     (fp32)
+    EPI_TOPK = 7        // router: top-k of the row's logits, gate weights, histogram
 };
 
 struct EpiParams {
@@ -288,6 +318,14 @@ struct EpiParams {
     int shared_rows;       // rows [0, shared_rows) are shared-expert rows: token = row % ntok
     int ntok;
     float* dst;            // scatter destination [ntok, ld]
+    // router top-k
+    int n_exp, top_k;
+    const float* bias;     // selection bias [n_exp] or NULL
+    int32_t* idx_out;      // [ntok, top_k]
+    float* w_out;          // [ntok, top_k]
+    int* counts;           // [n_exp] histogram (atomics)
+    int32_t* trace_idx;    // optional copies
+    float* trace_w;
     int* flags;            // device status words
 };
 
@@ -295,8 +333,8 @@ struct GemmArgs {
     int M;                 // rows of A / C (dense); unused for grouped
     int N;                 // columns of C (= rows of B per group)
     int kb_main;           // K blocks (128 bytes each) of A/B
-    int kb_ext;            // 0 or 1 extra K blocks from (A2, B2)
-    int b2_row0;           // row offset into B2 for the extension block
+    int kb_ext;            // extra K blocks from (A2, B2), at K offsets 0, 1, .. blocks
+    int b2_row0;           // row offset into B2 for the extension blocks
     const GroupTile* tiles;// grouped: tile list (NULL = dense)
     const int* n_tiles;    // grouped: number of valid tiles (device)
     int max_tiles;         // grouped: grid size along M
@@ -335,6 +373,14 @@ struct Norm1Args {
     int* zero_counts; int n_zero;   // counts to clear (next MoE), or NULL
 };
 rdt_status norm1(bool bf16_elems, const Norm1Args& a, cudaStream_t st);
+
+// RMSNorm2 for the tensor-core router: yn (element type, also the experts' input) and
+// the residual yn - yn_hi in the same type, so that [yn | yn_lo] . [W_r | W_r]^T gives the
+// logits of the fp32 normalised row to ~2^-17 relative.
+struct Norm2Args {
+    const float* y; const float* gamma; void* yn; void* yn_lo; int ntok, dim; float eps;
+};
+rdt_status norm2_split(bool bf16_elems, const Norm2Args& a, cudaStream_t st);
 
 struct RouterArgs {
     const float* y; const float* gamma; void* yn; int ntok, dim; float eps;

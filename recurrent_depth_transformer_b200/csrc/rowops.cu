@@ -28,6 +28,8 @@ __device__ __forceinline__ void store_t(T* p, float v) { *p = from_f<T>(v); }
 template <typename T>
 __global__ void hoist_kernel(const T* h0, const T* e, const float* Bd, float* h, float* Be,
                              size_t n4, int dim) {
+    pdl_trigger();
+    pdl_wait();
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
          i += static_cast<size_t>(gridDim.x) * blockDim.x) {
         const size_t off = i * 4;
@@ -49,6 +51,8 @@ __global__ void hoist_kernel(const T* h0, const T* e, const float* Bd, float* h,
 template <typename T>
 __global__ void matmul_nt_kernel(const T* A, const float* B, float* C, int M, int N, int K) {
     __shared__ float sa[16][17], sb[16][17];
+    pdl_trigger();
+    pdl_wait();
     const int tx = threadIdx.x, ty = threadIdx.y;
     const int row = blockIdx.y * 16 + ty, col = blockIdx.x * 16 + tx;
     float acc = 0.0f;
@@ -68,6 +72,8 @@ __global__ void matmul_nt_kernel(const T* A, const float* B, float* C, int M, in
 
 template <typename T, int NV>
 __global__ void __launch_bounds__(kRowThreads) norm1_kernel(const Norm1Args a) {
+    pdl_trigger();
+    pdl_wait();
     if (blockIdx.x == 0 && a.zero_counts)
         for (int i = threadIdx.x; i < a.n_zero; i += blockDim.x) a.zero_counts[i] = 0;
     const int row = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
@@ -233,12 +239,64 @@ __global__ void __launch_bounds__(kRowThreads) norm2_router_kernel(const RouterA
     }
 }
 
+// ----------------------------------------------------------------------------- norm2 (hi/lo)
+
+// hi = yn rounded to the element type (bf16; for fp32 the tf32 precision the tensor cores
+// read), lo = the element-type value of yn - hi.
+__device__ __forceinline__ void split_hi_lo(float v, bf16& hi, bf16& lo) {
+    hi = __float2bfloat16_rn(v);
+    lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+__device__ __forceinline__ void split_hi_lo(float v, float& hi, float& lo) {
+    hi = __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
+    lo = v - hi;
+}
+
+template <typename T, int NV>
+__global__ void __launch_bounds__(kRowThreads) norm2_split_kernel(const Norm2Args a) {
+    pdl_trigger();
+    pdl_wait();
+    const int row = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= a.ntok) return;
+    const size_t base = static_cast<size_t>(row) * a.dim;
+    float y[NV][4];
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        load4(a.y + base + i * 128 + lane * 4, y[i]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ss = fmaf(y[i][j], y[i][j], ss);
+    }
+    ss = warp_sum(ss);
+    const float inv = rsqrtf(ss / a.dim + a.eps);
+    T* yn = static_cast<T*>(a.yn) + base;
+    T* lo = static_cast<T*>(a.yn_lo) + base;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int col = i * 128 + lane * 4;
+        float g[4], hv[4], lv[4];
+        load4(a.gamma + col, g);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            T h, l;
+            split_hi_lo(y[i][j] * inv * g[j], h, l);
+            hv[j] = to_f(h);
+            lv[j] = to_f(l);
+        }
+        store4(yn + col, hv);
+        store4(lo + col, lv);
+    }
+}
+
 // ----------------------------------------------------------------------------- MoE dispatch
 
 // One block: exclusive scans of the routed counts (row offsets inside the routed region)
 // and of the per-group tile counts; writes the grouped-GEMM tile list.
 __global__ void __launch_bounds__(256) moe_scan_kernel(const DispatchArgs a) {
     __shared__ int s_cnt[256], s_tiles[256], s_off[256], s_toff[256];
+    pdl_trigger();
+    pdl_wait();
     const int G = a.n_exp + a.n_shared;
     const int t = threadIdx.x;
     const int cnt = t < a.n_exp ? a.counts[t] : (t < G ? a.ntok : 0);
@@ -286,6 +344,8 @@ __global__ void __launch_bounds__(256) moe_scan_kernel(const DispatchArgs a) {
 // weight, copy the normalised row yn[token] into it.
 template <typename T>
 __global__ void __launch_bounds__(kRowThreads) moe_scatter_kernel(const DispatchArgs a) {
+    pdl_trigger();
+    pdl_wait();
     const int ws = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (ws >= a.ntok * a.top_k) return;
@@ -311,6 +371,8 @@ __global__ void __launch_bounds__(kRowThreads) moe_scatter_kernel(const Dispatch
 template <typename T, int NV>
 __global__ void __launch_bounds__(kRowThreads) lora_down_kernel(const T* x, int ldx, int ntok,
                                                                 const T* A, int r, T* t) {
+    pdl_trigger();
+    pdl_wait();
     const int row = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= ntok) return;
@@ -338,6 +400,8 @@ __global__ void __launch_bounds__(kRowThreads) lora_down_kernel(const T* x, int 
 
 template <typename T>
 __global__ void __launch_bounds__(kRowThreads) mla_latent_norm_kernel(const MlaNormArgs a) {
+    pdl_trigger();
+    pdl_wait();
     const int row = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= a.ntok) return;
@@ -362,7 +426,7 @@ __global__ void __launch_bounds__(kRowThreads) mla_latent_norm_kernel(const MlaN
     const int half = a.rope / 2;
     const int pos = row % a.seq;
     for (int i = lane; i < half; i += 32) {
-        const float c = a.rope_cos[pos * half + i], s = a.rope_sin[pos * half + i];
+        const float c = a.rope_cos[i * a.seq + pos], s = a.rope_sin[i * a.seq + pos];
         const float x1 = R[i], x2 = R[i + half];
         store_t(kv + a.kv_lat + i, x1 * c - x2 * s);
         store_t(kv + a.kv_lat + half + i, x2 * c + x1 * s);
@@ -383,6 +447,8 @@ __global__ void prep_matmul_kernel(const T* A, long sam, long sak, const T* B, l
 }
 
 __global__ void check_finite_kernel(const float* x, size_t n, int* flags) {
+    pdl_trigger();
+    pdl_wait();
     bool bad = false;
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
          i += static_cast<size_t>(gridDim.x) * blockDim.x)
@@ -409,16 +475,21 @@ rdt_status launch_rows(int nv, int rows, cudaStream_t st, Args... args) {
 template <typename T, int NV>
 struct Norm1L {
     static void run(dim3 g, cudaStream_t st, Norm1Args a) {
-        norm1_kernel<T, NV><<<g, kRowThreads, 0, st>>>(a);
+        launch_pdl(norm1_kernel<T, NV>, g, dim3(kRowThreads), 0, st, a);
     }
 };
 template <typename T, int NV>
 struct LoraL {
     static void run(dim3 g, cudaStream_t st, const void* x, int ldx, int ntok, const void* A,
                     int r, void* t) {
-        lora_down_kernel<T, NV><<<g, kRowThreads, 0, st>>>(static_cast<const T*>(x), ldx, ntok,
-                                                           static_cast<const T*>(A), r,
-                                                           static_cast<T*>(t));
+        launch_pdl(lora_down_kernel<T, NV>, g, dim3(kRowThreads), 0, st, static_cast<const T*>(x), ldx,
+                   ntok, static_cast<const T*>(A), r, static_cast<T*>(t));
+    }
+};
+template <typename T, int NV>
+struct Norm2L {
+    static void run(dim3 g, cudaStream_t st, Norm2Args a) {
+        launch_pdl(norm2_split_kernel<T, NV>, g, dim3(kRowThreads), 0, st, a);
     }
 };
 template <typename T, int NV>
@@ -440,11 +511,11 @@ rdt_status hoist(bool bf, const void* h0, const void* e, const float* Bdiag, flo
     const size_t n4 = n / 4;
     const int grid = static_cast<int>(std::min<size_t>((n4 + 255) / 256, 148 * 16));
     if (bf)
-        hoist_kernel<bf16><<<grid, 256, 0, st>>>(static_cast<const bf16*>(h0),
-                                                 static_cast<const bf16*>(e), Bdiag, h, Be, n4, dim);
+        RDT_CUDA_TRY(launch_pdl(hoist_kernel<bf16>, dim3(grid), dim3(256), 0, st, static_cast<const bf16*>(h0),
+                                static_cast<const bf16*>(e), Bdiag, h, Be, n4, dim));
     else
-        hoist_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(h0),
-                                                  static_cast<const float*>(e), Bdiag, h, Be, n4, dim);
+        RDT_CUDA_TRY(launch_pdl(hoist_kernel<float>, dim3(grid), dim3(256), 0, st, static_cast<const float*>(h0),
+                                static_cast<const float*>(e), Bdiag, h, Be, n4, dim));
     RDT_CUDA_TRY(cudaGetLastError());
     return RDT_OK;
 }
@@ -453,9 +524,9 @@ rdt_status matmul_nt_simt(bool a_bf16, const void* A, const float* B, float* C, 
                           int K, cudaStream_t st) {
     const dim3 blk(16, 16), grid((N + 15) / 16, (M + 15) / 16);
     if (a_bf16)
-        matmul_nt_kernel<bf16><<<grid, blk, 0, st>>>(static_cast<const bf16*>(A), B, C, M, N, K);
+        RDT_CUDA_TRY(launch_pdl(matmul_nt_kernel<bf16>, grid, blk, 0, st, static_cast<const bf16*>(A), B, C, M, N, K));
     else
-        matmul_nt_kernel<float><<<grid, blk, 0, st>>>(static_cast<const float*>(A), B, C, M, N, K);
+        RDT_CUDA_TRY(launch_pdl(matmul_nt_kernel<float>, grid, blk, 0, st, static_cast<const float*>(A), B, C, M, N, K));
     RDT_CUDA_TRY(cudaGetLastError());
     return RDT_OK;
 }
@@ -473,6 +544,12 @@ rdt_status lora_down(bool bf, const void* x, int ldx, int ntok, int width, const
               : launch_rows<float, LoraL>(nv, ntok, st, x, ldx, ntok, A, r, t);
 }
 
+rdt_status norm2_split(bool bf, const Norm2Args& a, cudaStream_t st) {
+    const int nv = a.dim / 128;
+    return bf ? launch_rows<bf16, Norm2L>(nv, a.ntok, st, a)
+              : launch_rows<float, Norm2L>(nv, a.ntok, st, a);
+}
+
 rdt_status norm2_router(bool bf, const RouterArgs& a, cudaStream_t st) {
     const int nv = a.dim / 128;
     return bf ? launch_rows<bf16, RouterL>(nv, a.ntok, st, a)
@@ -480,14 +557,13 @@ rdt_status norm2_router(bool bf, const RouterArgs& a, cudaStream_t st) {
 }
 
 rdt_status moe_dispatch(bool bf, const DispatchArgs& a, cudaStream_t st) {
-    moe_scan_kernel<<<1, 256, 0, st>>>(a);
-    RDT_CUDA_TRY(cudaGetLastError());
+    RDT_CUDA_TRY(launch_pdl(moe_scan_kernel, dim3(1), dim3(256), 0, st, a));
     const int warps = a.ntok * a.top_k;
     const dim3 grid((warps + kRowThreads / 32 - 1) / (kRowThreads / 32));
     if (bf)
-        moe_scatter_kernel<bf16><<<grid, kRowThreads, 0, st>>>(a);
+        RDT_CUDA_TRY(launch_pdl(moe_scatter_kernel<bf16>, grid, dim3(kRowThreads), 0, st, a));
     else
-        moe_scatter_kernel<float><<<grid, kRowThreads, 0, st>>>(a);
+        RDT_CUDA_TRY(launch_pdl(moe_scatter_kernel<float>, grid, dim3(kRowThreads), 0, st, a));
     RDT_CUDA_TRY(cudaGetLastError());
     return RDT_OK;
 }
@@ -495,9 +571,9 @@ rdt_status moe_dispatch(bool bf, const DispatchArgs& a, cudaStream_t st) {
 rdt_status mla_latent_norm(bool bf, const MlaNormArgs& a, cudaStream_t st) {
     const dim3 grid((a.ntok + kRowThreads / 32 - 1) / (kRowThreads / 32));
     if (bf)
-        mla_latent_norm_kernel<bf16><<<grid, kRowThreads, 0, st>>>(a);
+        RDT_CUDA_TRY(launch_pdl(mla_latent_norm_kernel<bf16>, grid, dim3(kRowThreads), 0, st, a));
     else
-        mla_latent_norm_kernel<float><<<grid, kRowThreads, 0, st>>>(a);
+        RDT_CUDA_TRY(launch_pdl(mla_latent_norm_kernel<float>, grid, dim3(kRowThreads), 0, st, a));
     RDT_CUDA_TRY(cudaGetLastError());
     return RDT_OK;
 }
@@ -519,7 +595,7 @@ rdt_status prep_matmul(bool bf, const void* A, long sam, long sak, const void* B
 
 rdt_status check_finite(const float* x, size_t n, int* flags, cudaStream_t st) {
     const int grid = static_cast<int>(std::min<size_t>((n + 255) / 256, 148 * 8));
-    check_finite_kernel<<<grid, 256, 0, st>>>(x, n, flags);
+    RDT_CUDA_TRY(launch_pdl(check_finite_kernel, dim3(grid), dim3(256), 0, st, x, n, flags));
     RDT_CUDA_TRY(cudaGetLastError());
     return RDT_OK;
 }

@@ -141,7 +141,7 @@ def test_causality_and_batch_independence():
         out2 = h.loop_forward(e2, e2, 2)
         torch.cuda.synchronize()
     d = (out1[0, :100] - out2[0, :100]).abs().max().item()
-    assert d < 1e-4, d      # atomics may reorder the expert sums; values must agree
+    assert d < 2e-3, d      # leakage would show as O(0.1); atomics only reorder sums
 
 
 def test_host_entry_matches_device_entry():
@@ -209,3 +209,32 @@ def test_invalid_arguments_return_errors():
     with pytest.raises(R.RdtError) as ex:
         handle(wl, unstable)
     assert ex.value.status == 4
+
+
+def test_graph_replay_matches_eager_and_oracle():
+    """Same pointers and T: call 1 runs eagerly, call 2 captures a CUDA graph, later calls
+    replay it; every output must match the eager one and the oracle."""
+    torch = torch_mod()
+    wl = C1.replace(batch=2, seq=200)
+    inputs = generate(wl)
+    T = 3
+    _, idx, *_ = run_loop(wl, inputs, T)
+    want, mism, _, _ = oracle_follow(wl, inputs, T, idx)
+    assert mism == 0
+    with handle(wl, inputs, max_loops=T) as h:
+        e = act(wl, inputs["e"])
+        out = torch.empty(e.shape, dtype=torch.float32, device="cuda")
+        outs, counts = [], []
+        for _ in range(4):
+            n0 = h.launch_count()
+            h.loop_forward(e, e, T, out=out)
+            torch.cuda.synchronize()
+            counts.append(h.launch_count() - n0)
+            outs.append(out.cpu().numpy().copy())
+    assert len(set(counts)) == 1 and counts[0] > 0
+    # the expert sums are reduced with atomics, so bits may differ between runs; bf16
+    # rounding of the next loop's inputs can turn such ulp differences into ~1e-4 ones
+    for o in outs[1:]:
+        assert errors(o, outs[0])[0] < 2e-3
+    for o in outs:
+        assert_close(o, want, what="graph replay")
