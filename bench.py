@@ -60,8 +60,8 @@ def kernel_work(wl, T):
     w["gemm_down"] = dict(flops=2.0 * rows * hid * d, bytes=b2 * (rows * hid + (E + S) * d * hid) + 4 * N * d * 2,
                           bound="tensor")
     w["norm1"] = dict(flops=0.0, bytes=N * d * (4 + b2 + b2), bound="hbm")
-    w["norm2"] = dict(flops=0.0, bytes=N * d * (4 + b2 + b2), bound="hbm")
-    w["router_topk"] = dict(flops=2.0 * N * 2 * d * E, bytes=2 * N * d * b2 + E * d * b2 + N * k * 8, bound="hbm")
+    # RMSNorm2 fused with the fp32 router (W_r staged in shared memory): y in, yn and routing out
+    w["router_topk"] = dict(flops=2.0 * N * d * E, bytes=N * d * (4 + b2) + E * d * b2 + N * k * 8, bound="hbm")
     w["moe_dispatch"] = dict(flops=0.0, bytes=N * k * (d * b2 * 2 + 16), bound="hbm")
     w["hoist"] = dict(flops=0.0, bytes=N * d * (b2 + b2 + 4 + 4), bound="hbm")
     w["check_finite"] = dict(flops=0.0, bytes=N * d * 4, bound="hbm")

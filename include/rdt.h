@@ -201,7 +201,9 @@ rdt_status rdt_matmul(int32_t dtype, const void* A, const void* B, float* C, int
  * and query head; query head h reads KV head floor(h * n_kv_heads / n_heads).
  *   q : device [batch * seq, n_heads * dqk]    k : device [batch * seq, n_kv_heads * dqk]
  *   v : device [batch * seq, n_kv_heads * dv]  o : device [batch * seq, n_heads * dv]
- * bf16: (dqk, dv) = (64, 64) or (160, 128); fp32: (32, 32) or (64, 64). */
+ * bf16: (dqk, dv) = (64, 64) or (160, 128); fp32: (32, 32) or (64, 64). v may equal k
+ * with dv <= dqk: the values are then the first dv columns of each key row (absorbed MLA's
+ * shared latent), read with the keys' row stride. */
 rdt_status rdt_attention(int32_t dtype, const void* q, const void* k, const void* v, void* o,
                          int batch, int seq, int n_heads, int n_kv_heads, int dqk, int dv,
                          float scale, void* stream);

@@ -281,6 +281,8 @@ rdt_status launch_f32(const AttnArgs& a, cudaStream_t st) {
 }  // namespace
 
 rdt_status attention(bool bf16_elems, const AttnArgs& a, cudaStream_t st) {
+    if (bf16_elems && ((a.dqk == 64 && a.dv == 64) || (a.dqk == 160 && a.dv == 128 && a.v == a.k)))
+        return attention_tc(a, st);
     if (bf16_elems) {
         if (a.dqk == 64 && a.dv == 64) return launch_bf16<64, 64>(a, st);
         if (a.dqk == 160 && a.dv == 128) return launch_bf16<160, 128>(a, st);

@@ -1,0 +1,391 @@
+// Causal attention forward on the sm_100a tensor cores (tcgen05), one CTA per
+// (128 queries, query head, sequence), two CTAs per SM:
+//
+//   o = softmax(q k^T * scale, key > query masked) v
+//
+// For each block j of 128 keys:  S_j = Q K_j^T  (tcgen05.mma, M = 128 queries, N = 128 keys,
+// fp32 in TMEM)  ->  four softmax warps, one query row per thread: row maximum, then
+// P_j = 2^(S_j * scale * log2 e - m_ref) in bf16, written to shared memory in the
+// 128-byte-swizzled K-major layout, and the row sum l  ->  O += P_j V_j  (tcgen05.mma into a
+// TMEM accumulator, N = dv; V read as an MN-major operand straight from its [key][dv] layout).
+// m_ref is raised only when a row maximum exceeds it by more than 2^8; O (in TMEM) and l are
+// then rescaled once. The division by l happens when o is written.
+//
+// Grouped-query heads read KV head floor(h * Hkv / Hq) ("Introducao ao OpenMythos" Passo 5).
+// Absorbed MLA attends over the shared latent key [c_kv ; k_rope] (160 wide) with the value
+// c_kv = the key's first 128 columns, so its V operand is the K tile itself.
+//
+// Roles: warp 0 issues TMA loads (Q once, K two stages ahead, V one stage); warp 1 owns TMEM
+// and issues the MMAs (S_{j+1} before P_j V_j); warps 2-5 do the softmax and write o.
+// Every wait is bounded.
+#include <algorithm>
+
+#include "rdt_internal.cuh"
+
+namespace rdt {
+namespace {
+
+constexpr int kBQ = 128;     // queries per CTA
+constexpr int kBK = 128;     // keys per block
+constexpr int kAtom = 16384; // one 128-row x 128-byte swizzled region
+
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// K-major (a_major = b_major = 0) or K-major A with MN-major B (b_major = 1).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(b_mn_major) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// MN-major operand with the 128-byte swizzle: 8 K-rows of 128 bytes per atom (stride byte
+// offset 1024), consecutive 64-element MN atoms `lbo` bytes apart.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr, uint32_t lbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
+template <int DQK, int DV, bool SHARE_KV>
+struct AttnCfg {
+    static constexpr int QA = (DQK + 63) / 64;     // 64-wide atoms of the query/key width
+    static constexpr int VA = DV / 64;             // 64-wide atoms of the value width
+    static constexpr int Q_BYTES = QA * kAtom;
+    static constexpr int K_BYTES = QA * kAtom;     // one stage of K (128 keys)
+    static constexpr int KSTAGES = 2;
+    static constexpr int V_BYTES = SHARE_KV ? 0 : VA * kAtom;
+    static constexpr int P_BYTES = 2 * kAtom;      // 128 x 128 bf16 probabilities
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_V = OFF_K + KSTAGES * K_BYTES;
+    static constexpr int OFF_P = OFF_V + V_BYTES;
+    static constexpr int OFF_BAR = OFF_P + P_BYTES;
+    static constexpr int SMEM = OFF_BAR + 128 + 1024;
+    static constexpr int S_COL = 0;                 // S: columns [0, 128)
+    static constexpr int O_COL = 128;               // O: columns [128, 128 + DV)
+    static constexpr int TMEM_COLS = 128 + DV <= 256 ? 256 : 512;
+};
+
+struct AttnTcArgs {
+    int seq, hq, hkv, q_hstride, k_hstride, v_hstride, ldo, dv_out;
+    float scale_log2;
+    void* o;
+    int* flags;
+};
+
+// O is accumulated in TMEM by the P.V MMAs. P_j is taken relative to a reference maximum
+// m_ref that is raised only when a row's maximum exceeds it by more than 8 (in log2 units),
+// so P <= 2^8; then O and l are rescaled once by 2^(m_ref_old - m_ref_new).
+constexpr float kRescaleThreshold = 8.0f;
+
+template <int DQK, int DV, bool SHARE_KV>
+__global__ void __launch_bounds__(192, 2)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                   const __grid_constant__ CUtensorMap tv, const AttnTcArgs a) {
+    using C = AttnCfg<DQK, DV, SHARE_KV>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* bar_q = bars + 0;
+    uint64_t* kfull = bars + 1;    // [2]
+    uint64_t* kempty = bars + 3;   // [2]
+    uint64_t* vfull = bars + 5;
+    uint64_t* vempty = bars + 6;
+    uint64_t* sfull = bars + 7;    // S_j in TMEM
+    uint64_t* sfree = bars + 8;    // S_j read by the softmax warps
+    uint64_t* pfull = bars + 9;    // P_j in shared memory (and O rescaled if needed)
+    uint64_t* ofull = bars + 10;   // P_j . V_j accumulated (P buffer and V stage free)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int qb = gridDim.x - 1 - blockIdx.x;        // longest rows first
+    const int h = blockIdx.y;
+    const int b = blockIdx.z;
+    const int g = (h * a.hkv) / a.hq;
+    const int q0 = qb * kBQ;
+    const int row0 = b * a.seq;                        // first token row of this sequence
+    const int n_kb = min(qb + 1, (a.seq + kBK - 1) / kBK);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&kfull[i], 1);
+            mbar_init(&kempty[i], 1);
+        }
+        mbar_init(vfull, 1);
+        mbar_init(vempty, 1);
+        mbar_init(sfull, 1);
+        mbar_init(sfree, 4);
+        mbar_init(pfull, 4);
+        mbar_init(ofull, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tq);
+        tma_prefetch_desc(&tk);
+        if (!SHARE_KV) tma_prefetch_desc(&tv);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_trigger();
+    pdl_wait();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
+            for (int t = 0; t < C::QA; ++t)
+                tma_load_2d(smem + C::OFF_Q + t * kAtom, &tq, bar_q, h * a.q_hstride + 64 * t, row0 + q0);
+            // K runs one block ahead of V so that S_{j+1} never waits behind the V buffer
+            auto load_k = [&](int j) -> bool {
+                const int s = j & 1;
+                if (!mbar_wait(&kempty[s], ((j >> 1) & 1) ^ 1, a.flags)) return false;
+                mbar_arrive_expect_tx(&kfull[s], C::K_BYTES);
+                for (int t = 0; t < C::QA; ++t)
+                    tma_load_2d(smem + C::OFF_K + s * C::K_BYTES + t * kAtom, &tk, &kfull[s],
+                                g * a.k_hstride + 64 * t, row0 + j * kBK);
+                return true;
+            };
+            bool ok = load_k(0);
+#pragma unroll 1
+            for (int j = 0; j < n_kb && ok; ++j) {
+                if (j + 1 < n_kb) ok = load_k(j + 1);
+                if (ok && !SHARE_KV) {
+                    if (!mbar_wait(vempty, (j & 1) ^ 1, a.flags)) break;
+                    mbar_arrive_expect_tx(vfull, C::V_BYTES);
+                    for (int t = 0; t < C::VA; ++t)
+                        tma_load_2d(smem + C::OFF_V + t * kAtom, &tv, vfull, g * a.v_hstride + 64 * t,
+                                    row0 + j * kBK);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t id_s = idesc_bf16(kBQ, kBK, 0);
+            constexpr uint32_t id_o = idesc_bf16(kBQ, DV, 1);
+            const uint32_t sq = smem_u32(smem + C::OFF_Q);
+            const uint32_t sp = smem_u32(smem + C::OFF_P);
+            bool ok = mbar_wait(bar_q, 0, a.flags);
+            auto issue_s = [&](int j) -> bool {
+                const int s = j & 1;
+                if (!mbar_wait(&kfull[s], (j >> 1) & 1, a.flags)) return false;
+                if (!mbar_wait(sfree, (j & 1) ^ 1, a.flags)) return false;
+                tc_fence_after();
+                const uint32_t sk = smem_u32(smem + C::OFF_K + s * C::K_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < DQK / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+                    tc_mma_bf16(tmem + C::S_COL, sw128_kmajor_desc(sq + off), sw128_kmajor_desc(sk + off),
+                                id_s, kk > 0);
+                }
+                tc_commit(sfull);
+                if (!SHARE_KV) tc_commit(&kempty[s]);     // K stage consumed
+                return true;
+            };
+            auto issue_o = [&](int j) -> bool {
+                const int s = j & 1;
+                if (!mbar_wait(pfull, j & 1, a.flags)) return false;
+                if (!SHARE_KV && !mbar_wait(vfull, j & 1, a.flags)) return false;
+                tc_fence_after();
+                const uint32_t sv = SHARE_KV ? smem_u32(smem + C::OFF_K + s * C::K_BYTES)
+                                             : smem_u32(smem + C::OFF_V);
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk) {
+                    const uint32_t offp = (kk >> 2) * kAtom + (kk & 3) * 32;
+                    tc_mma_bf16(tmem + C::O_COL, sw128_kmajor_desc(sp + offp),
+                                sw128_mnmajor_desc(sv + kk * 16 * 128, kAtom), id_o, (j > 0) || kk);
+                }
+                tc_commit(ofull);
+                if (SHARE_KV)
+                    tc_commit(&kempty[s]);
+                else
+                    tc_commit(vempty);
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+#pragma unroll 1
+            for (int j = 1; j < n_kb && ok; ++j) {
+                ok = issue_s(j);
+                if (ok) ok = issue_o(j - 1);
+            }
+            if (ok) issue_o(n_kb - 1);
+        }
+    } else {
+        // softmax warps: thread = query row
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const int qpos = q0 + r;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+        const float sl = a.scale_log2;
+        float m_ref = -INFINITY, l = 0.0f;
+        uint8_t* arow0 = smem + C::OFF_P + r * 128;
+        bool ok = true;
+#pragma unroll 1
+        for (int j = 0; j < n_kb && ok; ++j) {
+            if (!mbar_wait(sfull, j & 1, a.flags)) { ok = false; break; }
+            tc_fence_after();
+            const int key0 = j * kBK;
+            const bool need_mask = (j == qb) || (key0 + kBK > a.seq);
+            const int kmax = need_mask ? min(qpos, a.seq - 1) - key0 : kBK - 1;  // last allowed key
+            // pass 1: row maximum (scaled to log2 units)
+            float mx = -INFINITY;
+#pragma unroll 1
+            for (int c = 0; c < kBK / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(lane_base + C::S_COL + c * 32, v);
+                tmem_wait_ld();
+                if (!need_mask) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(v[i]));
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (c * 32 + i <= kmax) mx = fmaxf(mx, __uint_as_float(v[i]));
+                }
+            }
+            mx *= sl;
+            // O (accumulated by P_{j-1} V_{j-1}) is stable once that MMA has completed
+            if (j > 0 && !mbar_wait(ofull, (j - 1) & 1, a.flags)) { ok = false; break; }
+            tc_fence_after();
+            if (mx > m_ref + kRescaleThreshold) {
+                const float corr = exp2f(m_ref - mx);
+                if (j > 0) {
+#pragma unroll
+                    for (int c = 0; c < DV / 32; ++c) {
+                        uint32_t v[32];
+                        tmem_ld32(lane_base + C::O_COL + c * 32, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * corr);
+                        tmem_st32(lane_base + C::O_COL + c * 32, v);
+                    }
+                    tmem_wait_st();
+                }
+                l *= corr;
+                m_ref = mx;
+            }
+            // pass 2: P = 2^(S*sl - m_ref) in bf16 into the swizzled K-major P buffer
+            float rs = 0.0f;
+#pragma unroll 1
+            for (int c = 0; c < kBK / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(lane_base + C::S_COL + c * 32, v);
+                tmem_wait_ld();
+                uint32_t packed[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float p0 = exp2f(__uint_as_float(v[2 * i]) * sl - m_ref);
+                    float p1 = exp2f(__uint_as_float(v[2 * i + 1]) * sl - m_ref);
+                    if (need_mask) {
+                        if (c * 32 + 2 * i > kmax) p0 = 0.0f;
+                        if (c * 32 + 2 * i + 1 > kmax) p1 = 0.0f;
+                    }
+                    rs += p0 + p1;
+                    __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                    packed[i] = *reinterpret_cast<uint32_t*>(&pb);
+                }
+                uint8_t* arow = arow0 + (c >> 1) * kAtom;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int phys = ((c & 1) * 4 + q) ^ (r & 7);
+                    *reinterpret_cast<uint4*>(arow + phys * 16) =
+                        make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                }
+            }
+            l += rs;
+            fence_proxy_async();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(sfree);
+                mbar_arrive(pfull);
+            }
+        }
+        if (ok) ok = mbar_wait(ofull, (n_kb - 1) & 1, a.flags);
+        tc_fence_after();
+        const float inv = 1.0f / l;
+        bf16* out = static_cast<bf16*>(a.o) + static_cast<size_t>(row0 + qpos) * a.ldo + h * a.dv_out;
+#pragma unroll 1
+        for (int c = 0; c < DV / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(lane_base + C::O_COL + c * 32, v);
+            tmem_wait_ld();
+            if (!ok || qpos >= a.seq) continue;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t w[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * u]) * inv,
+                                                              __uint_as_float(v[8 * q + 2 * u + 1]) * inv);
+                    w[u] = *reinterpret_cast<uint32_t*>(&pb);
+                }
+                *reinterpret_cast<uint4*>(out + c * 32 + 8 * q) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <int DQK, int DV, bool SHARE_KV>
+rdt_status launch_tc(const AttnArgs& a, cudaStream_t st) {
+    using C = AttnCfg<DQK, DV, SHARE_KV>;
+    auto kern = attn_tc_kernel<DQK, DV, SHARE_KV>;
+    static bool configured = false;
+    if (!configured) {
+        RDT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+        RDT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
+        configured = true;
+    }
+    const long rows = static_cast<long>(a.batch) * a.seq;
+    CUtensorMap tq, tk, tv;
+    RDT_TRY(make_tmap_2d(&tq, a.q, true, a.ldq, rows, static_cast<uint64_t>(a.ldq) * 2, 64, 128));
+    RDT_TRY(make_tmap_2d(&tk, a.k, true, a.ldk, rows, static_cast<uint64_t>(a.ldk) * 2, 64, 128));
+    if (!SHARE_KV)
+        RDT_TRY(make_tmap_2d(&tv, a.v, true, a.ldv, rows, static_cast<uint64_t>(a.ldv) * 2, 64, 128));
+    else
+        tv = tk;
+    AttnTcArgs ta{};
+    ta.seq = a.seq;
+    ta.hq = a.hq;
+    ta.hkv = a.hkv;
+    ta.q_hstride = a.q_hstride;
+    ta.k_hstride = a.k_hstride;
+    ta.v_hstride = a.v_hstride;
+    ta.ldo = a.ldo;
+    ta.dv_out = a.dv;
+    ta.scale_log2 = a.scale * 1.4426950408889634f;
+    ta.o = a.o;
+    ta.flags = a.flags;
+    const dim3 grid((a.seq + kBQ - 1) / kBQ, a.hq, a.batch);
+    RDT_CUDA_TRY(launch_pdl(kern, grid, dim3(192), C::SMEM, st, tq, tk, tv, ta));
+    return RDT_OK;
+}
+
+}  // namespace
+
+rdt_status attention_tc(const AttnArgs& a, cudaStream_t st) {
+    if (a.dqk == 64 && a.dv == 64) return launch_tc<64, 64, false>(a, st);
+    if (a.dqk == 160 && a.dv == 128 && a.v == a.k) return launch_tc<160, 128, true>(a, st);
+    set_error("tensor-core attention: unsupported head dimensions");
+    return RDT_ERR_UNSUPPORTED;
+}
+
+}  // namespace rdt

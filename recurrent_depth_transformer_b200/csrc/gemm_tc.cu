@@ -16,8 +16,8 @@
 //   EPI_SWIGLU      expert up-projection (gate and up rows interleaved per tile) -> silu(g)*u;
 //   EPI_SCATTER     expert down-projection, gate weight, and reduction into h_next
 //                   (h_{t+1} = A h + B e + a + sum_j w_j E_j(yn)).
-// Grouped mode reads a device-resident tile list (expert, A row, output row, rows), so
-// the per-expert row counts never travel to the host.
+// Grouped mode decodes its tiles from the per-expert row counters on the device (capacity
+// layout: expert e's rows start at e * tokens), so the counts never travel to the host.
 #include <algorithm>
 #include <type_traits>
 
@@ -61,70 +61,122 @@ __device__ __forceinline__ void store_row32(OutT* p, const float (&v)[32]) {
 
 // ----------------------------------------------------------------------------- epilogues
 
-// Router epilogue: the thread's row holds the logits of all experts (BN >= n_exp). Keeps the
-// KMAX best (score = logit + bias) in registers, visiting experts in ascending index so that
-// strict comparisons leave ties to the lower index; gate weights are the softmax of the
-// chosen logits.
-template <int BN, int KMAX>
-__device__ __forceinline__ void epilogue_topk(const EpiParams& p, uint32_t taddr, bool valid, int crow) {
+// Router top-k: keep the KMAX best (score = logit + bias) in registers, visiting experts in
+// ascending index so that strict comparisons leave ties to the lower index; gate weights
+// are the softmax of the chosen logits.
+template <int KMAX>
+struct TopK {
     float bs[KMAX], bl[KMAX];
     int bi[KMAX];
+    __device__ __forceinline__ TopK() {
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-        bs[j] = -INFINITY;
-        bl[j] = 0.0f;
-        bi[j] = -1;
+        for (int j = 0; j < KMAX; ++j) {
+            bs[j] = -INFINITY;
+            bl[j] = 0.0f;
+            bi[j] = -1;
+        }
     }
+    __device__ __forceinline__ void insert(float logit, float bias, int ex, int k) {
+        float cs = logit + bias, cl = logit;
+        int ci = ex;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j < k && cs > bs[j]) {
+                const float ts = bs[j], tl = bl[j];
+                const int ti = bi[j];
+                bs[j] = cs; bl[j] = cl; bi[j] = ci;
+                cs = ts; cl = tl; ci = ti;
+            }
+        }
+    }
+    __device__ __forceinline__ void write(const EpiParams& p, int row) const {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+            if (j < p.top_k && bi[j] >= 0) mx = fmaxf(mx, bl[j]);
+        float ex[KMAX], den = 0.0f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            ex[j] = (j < p.top_k && bi[j] >= 0) ? expf(bl[j] - mx) : 0.0f;
+            den += ex[j];
+        }
+        const size_t o = static_cast<size_t>(row) * p.top_k;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j >= p.top_k) break;
+            const int e = bi[j] < 0 ? 0 : bi[j];      // only when every score was NaN
+            const float w = den > 0.0f ? ex[j] / den : 0.0f;
+            p.idx_out[o + j] = e;
+            p.w_out[o + j] = w;
+            if (p.trace_idx) p.trace_idx[o + j] = e;
+            if (p.trace_w) p.trace_w[o + j] = w;
+            const int pos = atomicAdd(p.counts + e, 1);          // histogram and row claim
+            if (p.route_token) {
+                const int rr = e * p.cap + pos;
+                p.route_token[rr] = row;
+                p.route_w[rr] = w;
+                p.slot_row[o + j] = rr;
+            }
+        }
+    }
+};
+
+// Router epilogue. Unsplit: the thread's row holds all logits (BN >= n_exp) in TMEM.
+// Split over K: every CTA adds its partial logits into p.logits; the CTA that arrives last
+// on the row tile's counter (threadfence-reduction order: adds, fence, count) reads the
+// complete rows back and selects.
+template <int BN, int KMAX>
+__device__ __forceinline__ void epilogue_topk(const EpiParams& p, uint32_t taddr, bool valid, int crow,
+                                              int split, int mtile) {
+    if (split <= 1) {
+        TopK<KMAX> tk;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            ld_chunk(taddr, c, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int ex = c * 32 + i;
+                if (ex < p.n_exp) tk.insert(v[i], p.bias ? p.bias[ex] : 0.0f, ex, p.top_k);
+            }
+        }
+        if (valid) tk.write(p, crow);
+        return;
+    }
+    __shared__ int s_last;
+    float* lrow = p.logits + static_cast<size_t>(crow) * p.n_exp;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
         float v[32];
         ld_chunk(taddr, c, v);
+        if (!valid) continue;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const int ex = c * 32 + i;
-            if (ex >= p.n_exp) break;
-            float cs = v[i] + (p.bias ? p.bias[ex] : 0.0f);
-            float cl = v[i];
-            int ci = ex;
-#pragma unroll
-            for (int j = 0; j < KMAX; ++j) {
-                if (j < p.top_k && cs > bs[j]) {
-                    const float ts = bs[j], tl = bl[j];
-                    const int ti = bi[j];
-                    bs[j] = cs; bl[j] = cl; bi[j] = ci;
-                    cs = ts; cl = tl; ci = ti;
-                }
-            }
+            if (ex < p.n_exp) atomicAdd(lrow + ex, v[i]);
         }
     }
+    __threadfence();
+    asm volatile("bar.sync 1, 128;" ::: "memory");     // the four epilogue warps
+    if (threadIdx.x == 64) {
+        const int old = atomicAdd(p.tile_count + mtile, 1);
+        s_last = old == split - 1;
+        if (s_last) p.tile_count[mtile] = 0;             // ready for the next launch
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (!s_last) return;
+    __threadfence();
     if (!valid) return;
-    float mx = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j)
-        if (j < p.top_k && bi[j] >= 0) mx = fmaxf(mx, bl[j]);
-    float ex[KMAX], den = 0.0f;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-        ex[j] = (j < p.top_k && bi[j] >= 0) ? expf(bl[j] - mx) : 0.0f;
-        den += ex[j];
-    }
-    const size_t o = static_cast<size_t>(crow) * p.top_k;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-        if (j >= p.top_k) break;
-        const int e = bi[j] < 0 ? 0 : bi[j];      // only when every score was NaN
-        const float w = den > 0.0f ? ex[j] / den : 0.0f;
-        p.idx_out[o + j] = e;
-        p.w_out[o + j] = w;
-        if (p.trace_idx) p.trace_idx[o + j] = e;
-        if (p.trace_w) p.trace_w[o + j] = w;
-        atomicAdd(p.counts + e, 1);
-    }
+    TopK<KMAX> tk;
+#pragma unroll 1
+    for (int ex = 0; ex < p.n_exp; ++ex)
+        tk.insert(__ldcg(lrow + ex), p.bias ? p.bias[ex] : 0.0f, ex, p.top_k);
+    tk.write(p, crow);
 }
 
 template <typename T, int BN, int KIND>
 __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, bool valid, int crow,
-                                         int n0) {
+                                         int n0, int split = 1, int mtile = 0) {
     if constexpr (KIND == EPI_STORE || KIND == EPI_STORE_F32 || KIND == EPI_OPROJ_PLAIN) {
         using OutT = std::conditional_t<KIND == EPI_STORE, T, float>;
 #pragma unroll 1
@@ -138,14 +190,18 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, boo
     } else if constexpr (KIND == EPI_ROPE) {
         // Heads of width head_w tile the BN columns exactly (host checks BN % head_w == 0).
         // The angle tables are [rot/2][seq]: for a fixed frequency the lanes (consecutive
-        // positions) read consecutive floats.
+        // positions) read consecutive floats. One position per row: load its angles once.
         const int pos = crow % p.seq;
         const int hw_chunks = p.head_w / 32;
         const int rc0 = p.rot_off / 32;
         const int rch = p.rot_dim / 32;
-        const float* cosr = p.rope_cos + pos;
-        const float* sinr = p.rope_sin + pos;
-        const int ts = p.seq;
+        const int half = p.rot_dim / 2;
+        float cs[32], sn[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            cs[i] = i < half ? p.rope_cos[static_cast<size_t>(i) * p.seq + pos] : 0.0f;
+            sn[i] = i < half ? p.rope_sin[static_cast<size_t>(i) * p.seq + pos] : 0.0f;
+        }
         T* out = static_cast<T*>(p.out) + static_cast<size_t>(crow) * p.ldo;
 #pragma unroll 1
         for (int hc = 0; hc < BN / 32; hc += hw_chunks) {
@@ -161,10 +217,9 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, boo
                         ld_chunk(taddr, hc + c + 1, v1);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
-                            const float cs = cosr[i * ts], sn = sinr[i * ts];
                             const float x1 = v0[i], x2 = v1[i];
-                            v0[i] = x1 * cs - x2 * sn;
-                            v1[i] = x2 * cs + x1 * sn;
+                            v0[i] = x1 * cs[i] - x2 * sn[i];
+                            v1[i] = x2 * cs[i] + x1 * sn[i];
                         }
                         if (valid && col < p.ncols_valid) {
                             store_row32(out + col, v0);
@@ -176,10 +231,9 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, boo
                         ld_chunk(taddr, hc + c, v);
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            const float cs = cosr[i * ts], sn = sinr[i * ts];
                             const float x1 = v[i], x2 = v[i + 16];
-                            v[i] = x1 * cs - x2 * sn;
-                            v[i + 16] = x2 * cs + x1 * sn;
+                            v[i] = x1 * cs[i] - x2 * sn[i];
+                            v[i + 16] = x2 * cs[i] + x1 * sn[i];
                         }
                         if (valid && col < p.ncols_valid) store_row32(out + col, v);
                     }
@@ -191,6 +245,8 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, boo
             }
         }
     } else if constexpr (KIND == EPI_OPROJ_LOOP) {
+        // All loads of a 32-column chunk are issued before any store (the stores could alias
+        // them as far as the compiler knows, which would serialise every load behind them).
         const size_t rbase = static_cast<size_t>(crow) * p.ld;
         const T* e = static_cast<const T*>(p.e);
 #pragma unroll 1
@@ -199,27 +255,34 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, boo
             ld_chunk(taddr, c, v);
             const int col = n0 + c * 32;
             if (!valid || col >= p.ncols_valid) continue;
+            float hh[32], be[32], aa[32], ee[32];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const size_t off = rbase + col + 4 * j;
-                float hh[4], be[4], aa[4], x[4], yv[4], hn[4];
-                load4(p.h + off, hh);
-                load4(p.Be + off, be);
-                load4(p.Adiag + col + 4 * j, aa);
+                float t[4];
+                load4(p.h + off, t);
+                hh[4 * j] = t[0]; hh[4 * j + 1] = t[1]; hh[4 * j + 2] = t[2]; hh[4 * j + 3] = t[3];
+                load4(p.Be + off, t);
+                be[4 * j] = t[0]; be[4 * j + 1] = t[1]; be[4 * j + 2] = t[2]; be[4 * j + 3] = t[3];
+                load4(p.Adiag + col + 4 * j, t);
+                aa[4 * j] = t[0]; aa[4 * j + 1] = t[1]; aa[4 * j + 2] = t[2]; aa[4 * j + 3] = t[3];
                 if (e) {
-                    float ee[4];
-                    load4(e + off, ee);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) x[i] = hh[i] + ee[i];
+                    load4(e + off, t);
                 } else {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) x[i] = hh[i];
+                    t[0] = t[1] = t[2] = t[3] = 0.0f;
                 }
+                ee[4 * j] = t[0]; ee[4 * j + 1] = t[1]; ee[4 * j + 2] = t[2]; ee[4 * j + 3] = t[3];
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const size_t off = rbase + col + 4 * j;
+                float yv[4], hn[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const float a = v[4 * j + i];
-                    yv[i] = x[i] + a;
-                    hn[i] = aa[i] * hh[i] + be[i] + a;
+                    const int q = 4 * j + i;
+                    const float a = v[q];
+                    yv[i] = hh[q] + ee[q] + a;
+                    hn[i] = aa[q] * hh[q] + be[q] + a;
                 }
                 store4(p.y + off, yv);
                 store4(p.h_next + off, hn);
@@ -265,32 +328,85 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, boo
         }
     } else if constexpr (KIND == EPI_TOPK) {
         if (p.top_k <= 2)
-            epilogue_topk<BN, 2>(p, taddr, valid, crow);
+            epilogue_topk<BN, 2>(p, taddr, valid, crow, split, mtile);
         else if (p.top_k <= 4)
-            epilogue_topk<BN, 4>(p, taddr, valid, crow);
+            epilogue_topk<BN, 4>(p, taddr, valid, crow, split, mtile);
         else if (p.top_k <= 8)
-            epilogue_topk<BN, 8>(p, taddr, valid, crow);
+            epilogue_topk<BN, 8>(p, taddr, valid, crow, split, mtile);
         else
-            epilogue_topk<BN, 16>(p, taddr, valid, crow);
+            epilogue_topk<BN, 16>(p, taddr, valid, crow, split, mtile);
     }
 }
 
 // ----------------------------------------------------------------------------- the kernel
 
 struct TileCoord {
-    int a_row0, c_row0, nrows, group, n0;
+    int a_row0, c_row0, nrows, group, n0, mt, kb0, kb1;
 };
 
-__device__ __forceinline__ TileCoord tile_coord(const GemmArgs& args, int tile, int n_ntiles, int bn) {
+// Grouped mode: s_pref[g] = first 128-row tile of group g (routed groups, then shared ones),
+// s_pref[256] = tile count; s_cnt[g] = rows of group g.
+struct GroupTables {
+    int pref[257];
+    int cnt[256];
+};
+
+__device__ __forceinline__ void build_group_tables(const GemmArgs& args, GroupTables& t, int lane) {
+    const int G = args.n_routed + args.n_shared;
+    int tiles[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int g = lane * 8 + i;
+        const int c = g < args.n_routed ? args.counts[g] : (g < G ? args.M : 0);   // shared: all tokens
+        t.cnt[g] = c;
+        tiles[i] = (c + BM - 1) / BM;
+        sum += tiles[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        t.pref[lane * 8 + i] = run;
+        run += tiles[i];
+    }
+    if (lane == 31) t.pref[256] = incl;
+}
+
+// tile = (mt * n_ntiles + nt) * split + ks; split > 1 divides the K blocks evenly
+__device__ __forceinline__ TileCoord tile_coord(const GemmArgs& args, const GroupTables* gt, int tile,
+                                                int n_ntiles, int bn, int split, int num_kb) {
     TileCoord t;
+    const int ks = tile % split;
+    tile /= split;
     const int mt = tile / n_ntiles;
+    t.mt = mt;
     t.n0 = (tile - mt * n_ntiles) * bn;
-    if (args.tiles != nullptr) {
-        const GroupTile g = args.tiles[mt];
-        t.group = g.group;
-        t.a_row0 = args.a_from_c ? g.c_row0 : g.a_row0;
-        t.c_row0 = g.c_row0;
-        t.nrows = g.nrows;
+    const int per = (num_kb + split - 1) / split;
+    t.kb0 = ks * per;
+    t.kb1 = min(num_kb, t.kb0 + per);
+    if (gt != nullptr) {
+        const int G = args.n_routed + args.n_shared;
+        int lo = 0, hi = G - 1;                      // last group whose first tile <= mt
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (gt->pref[mid] <= mt) lo = mid; else hi = mid - 1;
+        }
+        const int local = (mt - gt->pref[lo]) * BM;
+        t.group = lo;
+        t.nrows = min(BM, gt->cnt[lo] - local);
+        if (lo < args.n_routed) {
+            t.a_row0 = args.a_routed_base + lo * args.cap + local;
+            t.c_row0 = (args.n_shared + lo) * args.cap + local;
+        } else {
+            t.a_row0 = local;
+            t.c_row0 = (lo - args.n_routed) * args.cap + local;
+        }
+        if (args.a_from_c) t.a_row0 = t.c_row0;
     } else {
         t.group = 0;
         t.a_row0 = mt * BM;
@@ -323,6 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    __shared__ GroupTables s_groups;
 
     if (threadIdx.x == 0) {
 #pragma unroll 1
@@ -351,10 +468,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_trigger();
     pdl_wait();
 
+    const GroupTables* gt = nullptr;
+    if (args.counts != nullptr) {          // grouped: per-group tile offsets from the counters
+        if (warp == 0) build_group_tables(args, s_groups, lane);
+        __syncthreads();
+        gt = &s_groups;
+    }
     const int n_ntiles = (args.N + BN - 1) / BN;
-    const int n_mtiles = args.tiles != nullptr ? min(*args.n_tiles, args.max_tiles)
-                                               : (args.M + BM - 1) / BM;
-    const int total = n_mtiles * n_ntiles;
+    const int n_mtiles = gt != nullptr ? gt->pref[256] : (args.M + BM - 1) / BM;
+    const int split = args.split_k > 1 ? args.split_k : 1;
+    const int total = n_mtiles * n_ntiles * split;
     const int num_kb = args.kb_main + args.kb_ext;
 
     if (warp == 0) {
@@ -363,10 +486,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
 #pragma unroll 1
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const TileCoord tc = tile_coord(args, tile, n_ntiles, BN);
+                const TileCoord tc = tile_coord(args, gt, tile, n_ntiles, BN, split, num_kb);
                 const int b_row0 = tc.group * args.N + tc.n0;
 #pragma unroll 1
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = tc.kb0; kb < tc.kb1; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1;
                     if (!mbar_wait(&empty[s], ph ^ 1, epi.flags)) {
@@ -399,8 +522,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(&tempty[b], (use & 1) ^ 1, epi.flags)) break;
                 tc_fence_after();
                 const uint32_t dt = tmem + static_cast<uint32_t>(b * BN);
+                const TileCoord tc = tile_coord(args, gt, tile, n_ntiles, BN, split, num_kb);
 #pragma unroll 1
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = tc.kb0; kb < tc.kb1; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1;
                     if (!mbar_wait(&full[s], ph, epi.flags)) {
@@ -415,9 +539,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int k = 0; k < 4; ++k) {
                         // each MMA consumes 32 bytes of K: advance the start address by 32 B (>> 4 = 2)
                         if constexpr (kBf16)
-                            tc_mma_bf16(dt, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                            tc_mma_bf16(dt, da + 2 * k, db + 2 * k, idesc, (kb > tc.kb0) || k);
                         else
-                            tc_mma_tf32(dt, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                            tc_mma_tf32(dt, da + 2 * k, db + 2 * k, idesc, (kb > tc.kb0) || k);
                     }
                     tc_commit(&empty[s]);
                 }
@@ -434,9 +558,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t use = static_cast<uint32_t>(local >> 1);
             if (!mbar_wait(&tfull[b], use & 1, epi.flags)) break;
             tc_fence_after();
-            const TileCoord tc = tile_coord(args, tile, n_ntiles, BN);
+            const TileCoord tc = tile_coord(args, gt, tile, n_ntiles, BN, split, num_kb);
             epilogue<T, BN, KIND>(epi, tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN,
-                                  r < tc.nrows, tc.c_row0 + r, tc.n0);
+                                  r < tc.nrows, tc.c_row0 + r, tc.n0, split, tc.mt);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[b]);
@@ -463,8 +587,8 @@ rdt_status launch(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMa
         configured = true;
     }
     const int n_ntiles = (args.N + BN - 1) / BN;
-    const long mt = args.tiles ? args.max_tiles : (args.M + BM - 1) / BM;
-    const long total = mt * n_ntiles;
+    const long mt = args.counts ? args.max_tiles : (args.M + BM - 1) / BM;
+    const long total = mt * n_ntiles * (args.split_k > 1 ? args.split_k : 1);
     if (total <= 0) return RDT_OK;
     const int grid = static_cast<int>(std::min<long>(total, num_sms()));
     RDT_CUDA_TRY(launch_pdl(kern, dim3(grid), dim3(kThreads), C::SMEM, st, tA, tB, tA2 ? *tA2 : tA,

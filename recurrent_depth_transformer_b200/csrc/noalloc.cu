@@ -2,8 +2,10 @@
 //
 // rdt_moe_route_noalloc runs the router of rdt_moe_forward (RMSNorm2 of y, logits of the
 // fp32 normalised row, top-k, softmax over the chosen logits, per-expert histogram) without
-// a handle and without any allocation: bf16 routers use the same RMSNorm2 split kernel and
-// tensor-core router GEMM as the handle, fp32 routers the same fp32 FMA kernel. Their
+// a handle and without any allocation, choosing its kernels exactly as the handle does:
+// routers whose weight fits in shared memory run the fused RMSNorm2 + fp32-logit kernel,
+// larger bf16 routers the RMSNorm2 split kernel and the tensor-core router GEMM, larger fp32
+// routers the fp32 FMA kernel. Their
 // scratch - the normalised rows (and, for bf16, their residuals) and the per-expert
 // counters - lives in the file-scope array below, which every process that loads librdt
 // holds on every GPU it uses until exit.
@@ -98,7 +100,25 @@ extern "C" rdt_status rdt_moe_route_noalloc(int32_t dtype, const float* y, const
     void* yn_lo = static_cast<unsigned char*>(yn) + row_bytes;
     RDT_CUDA_TRY(cudaMemsetAsync(counts, 0, kCountsBytes, st));   // the counters start at zero
 
-    if (bf) {
+    if (router_fits_smem(bf, n_experts, top_k, dim)) {
+        // the same kernel as rdt_moe_forward for routers whose weight fits in shared memory
+        RouterArgs ra{};
+        ra.y = y;
+        ra.gamma = norm2;
+        ra.yn = yn;
+        ra.ntok = ntok;
+        ra.dim = dim;
+        ra.eps = eps;
+        ra.w_router = w_router;
+        ra.bias = router_bias;
+        ra.n_exp = n_experts;
+        ra.top_k = top_k;
+        ra.idx = topk_idx;
+        ra.w = topk_w;
+        ra.counts = counts;
+        ra.store_yn = 1;
+        RDT_TRY(norm2_router_smem(bf, ra, st));
+    } else if (bf) {
         // the same two steps as rdt_moe_forward: RMSNorm2 split into yn + yn_lo, then the
         // tensor-core router GEMM [yn | yn_lo] . [W_r | W_r]^T with the top-k epilogue
         Norm2Args n2{};

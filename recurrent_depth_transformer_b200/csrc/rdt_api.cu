@@ -56,11 +56,16 @@ struct rdt_handle {
     void *xn = nullptr, *tq = nullptr, *to = nullptr, *qkv = nullptr, *o = nullptr;
     void *cq = nullptr, *kvlat = nullptr, *xperm = nullptr, *U = nullptr, *yn_lo = nullptr;
     int bn_router = 64;
+    int router_split = 1;          // K split of the router GEMM over CTAs
+    float* logits = nullptr;       // [N, E] partial-logit accumulator of the split router
+    int* tile_count = nullptr;     // per row-tile arrival counters of the split router
+    // output tile widths of the projection and expert GEMMs (128 or 256)
+    int bn_qkv = 128, bn_o = 128, bn_up = 128, bn_down = 128;
     int32_t* idx = nullptr;
     float* wts = nullptr;
-    int *counts = nullptr, *offsets = nullptr, *fill = nullptr, *ntiles = nullptr, *row_token = nullptr;
+    int cap = 0;                   // rows reserved per expert group (tokens + padding)
+    int *counts = nullptr, *row_token = nullptr, *slot_row = nullptr;
     float* row_w = nullptr;
-    GroupTile* tiles = nullptr;
     int max_tiles = 0;
     int* flags = nullptr;
     void *stage_h0 = nullptr, *stage_e = nullptr;
@@ -222,16 +227,37 @@ rdt_status copy_d2d(void* dst, const void* src, size_t bytes, cudaStream_t st) {
     return RDT_OK;
 }
 
-// W1 || W3 interleaved in 64-row blocks: rows [128j, 128j+64) = W1 rows [64j, 64j+64),
-// rows [128j+64, 128j+128) = W3 rows [64j, 64j+64) (one 128-column tile of the up GEMM
-// holds matching gate and up columns).
-rdt_status interleave_w13(void* dst, const void* w1, const void* w3, int hid, int dim, size_t esz,
+// W1 || W3 interleaved in blocks of g rows (g = half the up-projection tile width):
+// rows [2gj, 2gj+g) = W1 rows [gj, gj+g), rows [2gj+g, 2gj+2g) = W3 rows [gj, gj+g), so one
+// output tile of the up GEMM holds matching gate and up columns.
+rdt_status interleave_w13(void* dst, const void* w1, const void* w3, int hid, int dim, size_t esz, int g,
                           cudaStream_t st) {
-    const size_t blk = static_cast<size_t>(64) * dim * esz;
-    RDT_CUDA_TRY(cudaMemcpy2DAsync(dst, 2 * blk, w1, blk, blk, hid / 64, cudaMemcpyDeviceToDevice, st));
-    RDT_CUDA_TRY(cudaMemcpy2DAsync(static_cast<char*>(dst) + blk, 2 * blk, w3, blk, blk, hid / 64,
+    const size_t blk = static_cast<size_t>(g) * dim * esz;
+    RDT_CUDA_TRY(cudaMemcpy2DAsync(dst, 2 * blk, w1, blk, blk, hid / g, cudaMemcpyDeviceToDevice, st));
+    RDT_CUDA_TRY(cudaMemcpy2DAsync(static_cast<char*>(dst) + blk, 2 * blk, w3, blk, blk, hid / g,
                                    cudaMemcpyDeviceToDevice, st));
     return RDT_OK;
+}
+
+// Output tile width for a GEMM with about m_tiles row tiles and N columns. The persistent
+// grid's time is that of its busiest CTA: (tiles per CTA) x (tile time), a tile's time
+// taken as proportional to BN plus a fixed share for its pipeline fill and epilogue.
+int choose_bn(long m_tiles, int N, bool allow256) {
+    const long sms = num_sms();
+    long best_cost = -1;
+    int best = 128;
+    for (int bn : {256, 128}) {
+        if (bn == 256 && (!allow256 || N % 256)) continue;
+        if (N % bn) continue;
+        const long tiles = m_tiles * (N / bn);
+        const long per_cta = (tiles + sms - 1) / sms;
+        const long cost = per_cta * (32 + bn);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    return best;
 }
 
 rdt_status build_maps(rdt_handle* h) {
@@ -243,9 +269,9 @@ rdt_status build_maps(rdt_handle* h) {
     const int S = c.n_shared, E = c.n_experts, hid = c.expert_hidden;
     RDT_TRY(make_tmap_2d(&h->m_xn, h->xn, bf, d, N, d * es, kbox, 128));
     RDT_TRY(make_tmap_2d(&h->m_o, h->o, bf, h->owidth, N, h->owidth * es, kbox, 128));
-    RDT_TRY(make_tmap_2d(&h->m_wo, h->wo, bf, h->owidth, d, h->owidth * es, kbox, 128));
+    RDT_TRY(make_tmap_2d(&h->m_wo, h->wo, bf, h->owidth, d, h->owidth * es, kbox, h->bn_o));
     if (c.attn_type == RDT_GQA) {
-        RDT_TRY(make_tmap_2d(&h->m_wqkv, h->wqkv, bf, d, h->nqkv, d * es, kbox, 128));
+        RDT_TRY(make_tmap_2d(&h->m_wqkv, h->wqkv, bf, d, h->nqkv, d * es, kbox, h->bn_qkv));
     } else {
         RDT_TRY(make_tmap_2d(&h->m_wlat, h->wlat, bf, d, h->lat_w, d * es, kbox, 128));
         RDT_TRY(make_tmap_2d(&h->m_cq, h->cq, bf, c.q_lora_rank, N, c.q_lora_rank * es, kbox, 128));
@@ -255,16 +281,18 @@ rdt_status build_maps(rdt_handle* h) {
         RDT_TRY(make_tmap_2d(&h->m_tq, h->tq, bf, h->kext, N, h->kext * es, kbox, 128));
         RDT_TRY(make_tmap_2d(&h->m_to, h->to, bf, h->kext, N, h->kext * es, kbox, 128));
         RDT_TRY(make_tmap_2d(&h->m_lqb, h->lqb, bf, h->kext, static_cast<uint64_t>(c.n_lora) * h->nqkv,
-                             h->kext * es, kbox, 128));
+                             h->kext * es, kbox, h->bn_qkv));
         RDT_TRY(make_tmap_2d(&h->m_lob, h->lob, bf, h->kext, static_cast<uint64_t>(c.n_lora) * d,
-                             h->kext * es, kbox, 128));
+                             h->kext * es, kbox, h->bn_o));
     }
-    const uint64_t xrows = static_cast<uint64_t>(N) * (1 + c.top_k);
-    const uint64_t urows = static_cast<uint64_t>(N) * (S + c.top_k);
+    // capacity layout: xperm = [yn (N rows) | expert e: rows N + e N .. N + e N + N),
+    // U = [shared expert s: rows s N .. | expert e: rows (S + e) N ..]
+    const uint64_t xrows = static_cast<uint64_t>(N) + static_cast<uint64_t>(h->cap) * E;
+    const uint64_t urows = static_cast<uint64_t>(h->cap) * (S + E);
     RDT_TRY(make_tmap_2d(&h->m_xperm, h->xperm, bf, d, xrows, d * es, kbox, 128));
-    RDT_TRY(make_tmap_2d(&h->m_w13, h->w13, bf, d, static_cast<uint64_t>(E + S) * 2 * hid, d * es, kbox, 128));
+    RDT_TRY(make_tmap_2d(&h->m_w13, h->w13, bf, d, static_cast<uint64_t>(E + S) * 2 * hid, d * es, kbox, h->bn_up));
     RDT_TRY(make_tmap_2d(&h->m_U, h->U, bf, hid, urows, hid * es, kbox, 128));
-    RDT_TRY(make_tmap_2d(&h->m_w2, h->w2, bf, hid, static_cast<uint64_t>(E + S) * d, hid * es, kbox, 128));
+    RDT_TRY(make_tmap_2d(&h->m_w2, h->w2, bf, hid, static_cast<uint64_t>(E + S) * d, hid * es, kbox, h->bn_down));
     RDT_TRY(make_tmap_2d(&h->m_ynlo, h->yn_lo, bf, d, N, d * es, kbox, 128));
     RDT_TRY(make_tmap_2d(&h->m_wr, h->wr, bf, d, E, d * es, kbox, h->bn_router));
     return RDT_OK;
@@ -365,19 +393,30 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         RDT_TRY(dev_alloc(h, &h->rbias, E * 4));
         RDT_TRY(copy_d2d(h->rbias, w->router_bias, E * 4, st));
     }
+    if (h->bf) {
+        const long mt_dense = (N + 127) / 128;
+        const long mt_group = (static_cast<long>(N) * (K + S) + 127) / 128 + (E + S + 1) / 2;
+        h->bn_up = choose_bn(mt_group, 2 * hid, hid % 128 == 0);
+        h->bn_down = choose_bn(mt_group, d, true);
+        h->bn_o = choose_bn(mt_dense, d, true);
+        if (c.attn_type == RDT_GQA) {
+            const int nqkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
+            h->bn_qkv = choose_bn(mt_dense, nqkv, nqkv % 256 == 0);
+        }
+    }
     const size_t wexp = static_cast<size_t>(hid) * d * es;   // one expert matrix
     RDT_TRY(dev_alloc(h, &h->w13, 2 * wexp * (E + S)));
     RDT_TRY(dev_alloc(h, &h->w2, wexp * (E + S)));
     for (int e = 0; e < E; ++e) {
         RDT_TRY(interleave_w13(static_cast<char*>(h->w13) + 2 * wexp * e,
                                static_cast<const char*>(w->w1) + wexp * e,
-                               static_cast<const char*>(w->w3) + wexp * e, hid, d, es, st));
+                               static_cast<const char*>(w->w3) + wexp * e, hid, d, es, h->bn_up / 2, st));
     }
     RDT_TRY(copy_d2d(h->w2, w->w2, wexp * E, st));
     for (int s = 0; s < S; ++s) {
         RDT_TRY(interleave_w13(static_cast<char*>(h->w13) + 2 * wexp * (E + s),
                                static_cast<const char*>(w->ws1) + wexp * s,
-                               static_cast<const char*>(w->ws3) + wexp * s, hid, d, es, st));
+                               static_cast<const char*>(w->ws3) + wexp * s, hid, d, es, h->bn_up / 2, st));
     }
     if (S) RDT_TRY(copy_d2d(static_cast<char*>(h->w2) + wexp * E, w->ws2, wexp * S, st));
 
@@ -489,20 +528,31 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         RDT_TRY(dev_alloc(h, &h->qkv, static_cast<size_t>(N) * h->qt_w * es));
     }
     RDT_TRY(dev_alloc(h, &h->o, static_cast<size_t>(N) * h->owidth * es));
-    RDT_TRY(dev_alloc(h, &h->xperm, static_cast<size_t>(N) * (1 + K) * d * es, true));
-    RDT_TRY(dev_alloc(h, &h->U, static_cast<size_t>(N) * (S + K) * hid * es, true));
+    // groups are `cap` rows apart: the token count rounded up plus 64 rows, so that group
+    // bases do not all fall on the same large power-of-two stride
+    h->cap = (N + 63) / 64 * 64 + 64;
+    RDT_TRY(dev_alloc(h, &h->xperm, (static_cast<size_t>(N) + static_cast<size_t>(h->cap) * E) * d * es, true));
+    RDT_TRY(dev_alloc(h, &h->U, static_cast<size_t>(h->cap) * (S + E) * hid * es, true));
     RDT_TRY(dev_alloc(h, &h->yn_lo, nd * es, true));
     h->bn_router = E <= 64 ? 64 : E <= 128 ? 128 : 256;
+    if (h->bf) {
+        // split the router's K blocks (2 d * 2 B / 128 B) so that the row tiles fill the GPU
+        const int mt = (N + 127) / 128;
+        const int kb = 2 * d * 2 / 128;
+        int split = 1;
+        for (int sp = 1; sp <= kb; ++sp)
+            if (kb % sp == 0 && static_cast<long>(mt) * sp <= num_sms()) split = sp;
+        h->router_split = split;
+        RDT_TRY(dev_alloc(h, &h->logits, static_cast<size_t>(N) * E * 4, true));
+        RDT_TRY(dev_alloc(h, &h->tile_count, static_cast<size_t>(mt) * 4, true));
+    }
     RDT_TRY(dev_alloc(h, &h->idx, static_cast<size_t>(N) * K * 4));
     RDT_TRY(dev_alloc(h, &h->wts, static_cast<size_t>(N) * K * 4));
     RDT_TRY(dev_alloc(h, &h->counts, 256 * 4, true));
-    RDT_TRY(dev_alloc(h, &h->offsets, 256 * 4, true));
-    RDT_TRY(dev_alloc(h, &h->fill, 256 * 4, true));
-    RDT_TRY(dev_alloc(h, &h->ntiles, 16, true));
-    RDT_TRY(dev_alloc(h, &h->row_token, static_cast<size_t>(N) * K * 4));
-    RDT_TRY(dev_alloc(h, &h->row_w, static_cast<size_t>(N) * K * 4));
+    RDT_TRY(dev_alloc(h, &h->row_token, static_cast<size_t>(h->cap) * E * 4, true));
+    RDT_TRY(dev_alloc(h, &h->row_w, static_cast<size_t>(h->cap) * E * 4, true));
+    RDT_TRY(dev_alloc(h, &h->slot_row, static_cast<size_t>(N) * K * 4, true));
     h->max_tiles = (N * K + 127) / 128 + E + S * ((N + 127) / 128);
-    RDT_TRY(dev_alloc(h, &h->tiles, static_cast<size_t>(h->max_tiles) * sizeof(GroupTile), true));
     RDT_TRY(dev_alloc(h, &h->flags, FLAG_COUNT * 4, true));
     RDT_TRY(dev_alloc(h, &h->stage_h0, nd * es));
     RDT_TRY(dev_alloc(h, &h->stage_e, nd * es));
@@ -569,7 +619,7 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         ep.rot_off = 0;
         ep.rot_dim = c.head_dim;
         ep.rope_limit = h->nq + h->nkv;
-        TIMED(h, K_GEMM_QKV, 1, st, gemm_tc(h->bf, 128, h->m_xn, h->m_wqkv, lora ? &h->m_tq : nullptr,
+        TIMED(h, K_GEMM_QKV, 1, st, gemm_tc(h->bf, h->bn_qkv, h->m_xn, h->m_wqkv, lora ? &h->m_tq : nullptr,
                                            lora ? &h->m_lqb : nullptr, ga, ep, st));
         at.q = h->qkv;
         at.ldq = h->nqkv;
@@ -644,6 +694,7 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         at.dv = kvl;
         at.scale = 1.0f / std::sqrt(static_cast<float>(c.qk_nope_dim + rp));
     }
+    at.flags = h->flags;
     TIMED(h, K_ATTENTION, 1, st, attention(h->bf, at, st));
 
     if (lora) {
@@ -674,7 +725,7 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         eo.out = a_out;
         eo.ldo = d;
     }
-    TIMED(h, K_GEMM_O, 1, st, gemm_tc(h->bf, 128, h->m_o, h->m_wo, lora ? &h->m_to : nullptr,
+    TIMED(h, K_GEMM_O, 1, st, gemm_tc(h->bf, h->bn_o, h->m_o, h->m_wo, lora ? &h->m_to : nullptr,
                                       lora ? &h->m_lob : nullptr, go, eo, st));
     return RDT_OK;
 }
@@ -687,7 +738,35 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     const int N = h->ntok, d = c.dim, hid = c.expert_hidden;
     int32_t* idx = idx_out ? idx_out : h->idx;
     float* wts = w_out ? w_out : h->wts;
-    if (!h->bf) {
+    bool copies_written = false;
+    if (router_fits_smem(h->bf, c.n_experts, c.top_k, d)) {
+        // small router: RMSNorm2, fp32 logits, top-k and the experts' row copies in one
+        // kernel, W_r staged in shared memory
+        RouterArgs ra{};
+        ra.y = yin;
+        ra.gamma = h->g2;
+        ra.yn = h->xperm;
+        ra.ntok = N;
+        ra.dim = d;
+        ra.eps = c.norm_eps;
+        ra.w_router = h->wr;
+        ra.bias = h->rbias;
+        ra.n_exp = c.n_experts;
+        ra.top_k = c.top_k;
+        ra.idx = idx;
+        ra.w = wts;
+        ra.counts = h->counts;
+        ra.trace_idx = tr_idx;
+        ra.trace_w = tr_w;
+        ra.row_token = h->row_token;
+        ra.row_w = h->row_w;
+        ra.cap = h->cap;
+        ra.xperm = h->xperm;
+        ra.a_routed_base = N;
+        ra.store_yn = c.n_shared > 0;          // shared experts read yn itself
+        TIMED(h, K_ROUTER, 1, st, norm2_router_smem(h->bf, ra, st));
+        copies_written = true;
+    } else if (!h->bf) {
         // fp32: the tensor cores would read W_r as tf32, so the router stays in fp32 FMA
         RouterArgs ra{};
         ra.y = yin;
@@ -705,63 +784,65 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
         ra.counts = h->counts;
         ra.trace_idx = tr_idx;
         ra.trace_w = tr_w;
+        ra.row_token = h->row_token;
+        ra.row_w = h->row_w;
+        ra.slot_row = h->slot_row;
+        ra.cap = h->cap;
         TIMED(h, K_ROUTER, 1, st, norm2_router(false, ra, st));
     } else {
-    Norm2Args n2{};
-    n2.y = yin;
-    n2.gamma = h->g2;
-    n2.yn = h->xperm;
-    n2.yn_lo = h->yn_lo;
-    n2.ntok = N;
-    n2.dim = d;
-    n2.eps = c.norm_eps;
-    TIMED(h, K_NORM2, 1, st, norm2_split(h->bf, n2, st));
+        Norm2Args n2{};
+        n2.y = yin;
+        n2.gamma = h->g2;
+        n2.yn = h->xperm;
+        n2.yn_lo = h->yn_lo;
+        n2.ntok = N;
+        n2.dim = d;
+        n2.eps = c.norm_eps;
+        if (h->router_split > 1) {
+            n2.zero_rows = h->logits;
+            n2.zero_width = c.n_experts;
+        }
+        TIMED(h, K_NORM2, 1, st, norm2_split(h->bf, n2, st));
 
-    GemmArgs gr{};
-    gr.M = N;
-    gr.N = c.n_experts;
-    gr.kb_main = static_cast<int>(d * h->esz / 128);
-    gr.kb_ext = gr.kb_main;
-    gr.b2_row0 = 0;
-    gr.flags = h->flags;
-    EpiParams er{};
-    er.kind = EPI_TOPK;
-    er.n_exp = c.n_experts;
-    er.top_k = c.top_k;
-    er.bias = h->rbias;
-    er.idx_out = idx;
-    er.w_out = wts;
-    er.counts = h->counts;
-    er.trace_idx = tr_idx;
-    er.trace_w = tr_w;
-    er.flags = h->flags;
-    TIMED(h, K_ROUTER, 1, st, gemm_tc(h->bf, h->bn_router, h->m_xperm, h->m_wr, &h->m_ynlo, &h->m_wr, gr, er, st));
+        GemmArgs gr{};
+        gr.M = N;
+        gr.N = c.n_experts;
+        gr.kb_main = static_cast<int>(d * h->esz / 128);
+        gr.kb_ext = gr.kb_main;
+        gr.b2_row0 = 0;
+        gr.split_k = h->router_split;
+        gr.flags = h->flags;
+        EpiParams er{};
+        er.kind = EPI_TOPK;
+        er.n_exp = c.n_experts;
+        er.top_k = c.top_k;
+        er.bias = h->rbias;
+        er.idx_out = idx;
+        er.w_out = wts;
+        er.counts = h->counts;
+        er.trace_idx = tr_idx;
+        er.trace_w = tr_w;
+        er.logits = h->logits;
+        er.tile_count = h->tile_count;
+        er.route_token = h->row_token;
+        er.route_w = h->row_w;
+        er.slot_row = h->slot_row;
+        er.cap = h->cap;
+        er.flags = h->flags;
+        TIMED(h, K_ROUTER, 1, st, gemm_tc(h->bf, h->bn_router, h->m_xperm, h->m_wr, &h->m_ynlo, &h->m_wr, gr, er, st));
     }
-
-    DispatchArgs da{};
-    da.counts = h->counts;
-    da.n_exp = c.n_experts;
-    da.n_shared = c.n_shared;
-    da.ntok = N;
-    da.top_k = c.top_k;
-    da.dim = d;
-    da.offsets = h->offsets;
-    da.fill = h->fill;
-    da.tiles = h->tiles;
-    da.n_tiles = h->ntiles;
-    da.max_tiles = h->max_tiles;
-    da.idx = idx;
-    da.w = wts;
-    da.xperm = h->xperm;
-    da.row_token = h->row_token;
-    da.row_w = h->row_w;
-    TIMED(h, K_DISPATCH, 2, st, moe_dispatch(h->bf, da, st));
+    if (!copies_written)
+        TIMED(h, K_DISPATCH, 1, st, moe_copy(h->bf, h->xperm, h->slot_row, N, c.top_k, d, N, st));
 
     GemmArgs gu{};
+    gu.M = N;
     gu.N = 2 * hid;
     gu.kb_main = static_cast<int>(d * h->esz / 128);
-    gu.tiles = h->tiles;
-    gu.n_tiles = h->ntiles;
+    gu.counts = h->counts;
+    gu.n_routed = c.n_experts;
+    gu.n_shared = c.n_shared;
+    gu.cap = h->cap;
+    gu.a_routed_base = N;
     gu.max_tiles = h->max_tiles;
     gu.flags = h->flags;
     EpiParams eu{};
@@ -770,13 +851,17 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     eu.ldo = hid;
     eu.ncols_valid = 2 * hid;
     eu.flags = h->flags;
-    TIMED(h, K_GEMM_UP, 1, st, gemm_tc(h->bf, 128, h->m_xperm, h->m_w13, nullptr, nullptr, gu, eu, st));
+    TIMED(h, K_GEMM_UP, 1, st, gemm_tc(h->bf, h->bn_up, h->m_xperm, h->m_w13, nullptr, nullptr, gu, eu, st));
 
     GemmArgs gd{};
+    gd.M = N;
     gd.N = d;
     gd.kb_main = static_cast<int>(hid * h->esz / 128);
-    gd.tiles = h->tiles;
-    gd.n_tiles = h->ntiles;
+    gd.counts = h->counts;
+    gd.n_routed = c.n_experts;
+    gd.n_shared = c.n_shared;
+    gd.cap = h->cap;
+    gd.a_routed_base = N;
     gd.max_tiles = h->max_tiles;
     gd.a_from_c = 1;
     gd.flags = h->flags;
@@ -785,12 +870,12 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     ed.ncols_valid = d;
     ed.row_token = h->row_token;
     ed.row_w = h->row_w;
-    ed.shared_rows = c.n_shared * N;
-    ed.ntok = N;
+    ed.shared_rows = c.n_shared * h->cap;
+    ed.ntok = h->cap;
     ed.dst = dst;
     ed.ld = d;
     ed.flags = h->flags;
-    TIMED(h, K_GEMM_DOWN, 1, st, gemm_tc(h->bf, 128, h->m_U, h->m_w2, nullptr, nullptr, gd, ed, st));
+    TIMED(h, K_GEMM_DOWN, 1, st, gemm_tc(h->bf, h->bn_down, h->m_U, h->m_w2, nullptr, nullptr, gd, ed, st));
     return RDT_OK;
 }
 
@@ -1068,6 +1153,10 @@ rdt_status rdt_attention(int32_t dtype, const void* q, const void* k, const void
     a.q = q; a.ldq = n_heads * dqk; a.q_hstride = dqk;
     a.k = k; a.ldk = n_kv_heads * dqk; a.k_hstride = dqk;
     a.v = v; a.ldv = n_kv_heads * dv; a.v_hstride = dv;
+    if (v == k && dv <= dqk) {          // values are the first dv columns of the keys
+        a.ldv = a.ldk;
+        a.v_hstride = a.k_hstride;
+    }
     a.o = o; a.ldo = n_heads * dv;
     a.batch = batch; a.seq = seq; a.hq = n_heads; a.hkv = n_kv_heads; a.dqk = dqk; a.dv = dv;
     a.scale = scale;

@@ -242,6 +242,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// Warp-collective: lane i writes TMEM lane (base lane + i), 32 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 
 // Shared-memory matrix descriptor for a K-major tile written by TMA with the 128-byte
 // swizzle: rows of 128 bytes, 8-row swizzle atoms 1024 bytes apart (stride byte offset),
@@ -272,14 +287,11 @@ rdt_status make_tmap_2d(CUtensorMap* map, const void* base, bool bf16_elems, uin
                         uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner,
                         uint32_t box_rows);
 
-// One M-tile of a grouped (per-expert) GEMM.
-struct GroupTile {
-    int group;     // expert (routed 0..E-1, shared E..E+S-1)
-    int a_row0;    // first row of A for this tile
-    int c_row0;    // first output row
-    int nrows;     // valid rows (<= 128)
-};
-
+// Grouped (per-expert) operands use a capacity layout: group g's rows start at a fixed
+// offset (routed expert e: e * cap, cap = tokens, since a token picks an expert at most once;
+// shared expert s: all tokens), and a row inside a group is claimed with one atomic on the
+// group's counter. The grouped GEMM decodes its 128-row tiles from those counters on the
+// device; the host never sees them.
 enum EpiKind {
     EPI_STORE = 0,      // C[row, col] = acc                     (OutT)
     EPI_ROPE = 1,       // C = acc with RoPE on the rotary part of rotated heads (OutT)
@@ -316,29 +328,38 @@ struct EpiParams {
     const int* row_token;  // routed rows: token of each output row
     const float* row_w;    // routed rows: gate weight
     int shared_rows;       // rows [0, shared_rows) are shared-expert rows: token = row % ntok
-    int ntok;
+    int ntok;              // scatter: row stride of the shared groups in U
     float* dst;            // scatter destination [ntok, ld]
-    // router top-k
+    // router top-k (and dispatch: claim a row of each chosen expert)
     int n_exp, top_k;
+    int* route_token;      // [n_exp * cap] token of each claimed row (or NULL: no dispatch)
+    float* route_w;        // [n_exp * cap] gate weight of each claimed row
+    int* slot_row;         // [ntok, top_k] claimed row of each (token, slot)
+    int cap;
     const float* bias;     // selection bias [n_exp] or NULL
     int32_t* idx_out;      // [ntok, top_k]
     float* w_out;          // [ntok, top_k]
     int* counts;           // [n_exp] histogram (atomics)
     int32_t* trace_idx;    // optional copies
     float* trace_w;
+    float* logits;         // split-K router: [ntok, n_exp] fp32 partial sums (zeroed beforehand)
+    int* tile_count;       // split-K router: per row-tile arrival counters (zero, reset after use)
     int* flags;            // device status words
 };
 
 struct GemmArgs {
-    int M;                 // rows of A / C (dense); unused for grouped
+    int M;                 // rows of A / C (dense); grouped: rows of each shared group (tokens)
     int N;                 // columns of C (= rows of B per group)
     int kb_main;           // K blocks (128 bytes each) of A/B
     int kb_ext;            // extra K blocks from (A2, B2), at K offsets 0, 1, .. blocks
     int b2_row0;           // row offset into B2 for the extension blocks
-    const GroupTile* tiles;// grouped: tile list (NULL = dense)
-    const int* n_tiles;    // grouped: number of valid tiles (device)
-    int max_tiles;         // grouped: grid size along M
+    const int* counts;     // grouped: rows of each routed group [n_routed] (NULL = dense)
+    int n_routed, n_shared;// grouped: routed groups, then shared groups (n_rows = cap each)
+    int cap;               // grouped: rows reserved per group (>= tokens; the group stride)
+    int a_routed_base;     // grouped: first A row of routed group 0 (shared groups read rows 0..cap)
+    int max_tiles;         // grouped: upper bound on the 128-row tiles (grid sizing)
     int a_from_c;          // grouped: read A at the tile's output row (down projection)
+    int split_k;           // > 1: K blocks split over that many CTAs per output tile (router)
     int* flags;
 };
 
@@ -357,8 +378,11 @@ struct AttnArgs {
     void* o; int ldo;
     int batch, seq, hq, hkv, dqk, dv;
     float scale;
+    int* flags;
 };
 rdt_status attention(bool bf16_elems, const AttnArgs& a, cudaStream_t st);
+// tcgen05 kernel: (dqk, dv) = (64, 64), or (160, 128) with v == k (absorbed MLA)
+rdt_status attention_tc(const AttnArgs& a, cudaStream_t st);
 
 // Row kernels (rowops.cu).
 struct Norm1Args {
@@ -379,6 +403,7 @@ rdt_status norm1(bool bf16_elems, const Norm1Args& a, cudaStream_t st);
 // logits of the fp32 normalised row to ~2^-17 relative.
 struct Norm2Args {
     const float* y; const float* gamma; void* yn; void* yn_lo; int ntok, dim; float eps;
+    float* zero_rows; int zero_width;   // optional: rows of a [ntok, zero_width] fp32 buffer to clear
 };
 rdt_status norm2_split(bool bf16_elems, const Norm2Args& a, cudaStream_t st);
 
@@ -387,15 +412,21 @@ struct RouterArgs {
     const void* w_router; const float* bias; int n_exp, top_k;
     int32_t* idx; float* w; int* counts;
     int32_t* trace_idx; float* trace_w;
+    // dispatch (optional): counts double as the claim counters of the capacity layout
+    int* row_token; float* row_w; int* slot_row; int cap;
+    void* xperm; int a_routed_base;   // fused router: write yn into the claimed rows here
+    int store_yn;                      // fused router: also write yn at row `row` of yn
 };
 rdt_status norm2_router(bool bf16_elems, const RouterArgs& a, cudaStream_t st);
+// RMSNorm2 fused with the fp32 router when W_r (n_exp x dim) fits in 64 KB of shared memory,
+// n_exp <= 64, top_k <= 8 and dim is 128, 1024 or 2048
+bool router_fits_smem(bool bf16_elems, int n_exp, int top_k, int dim);
+rdt_status norm2_router_smem(bool bf16_elems, const RouterArgs& a, cudaStream_t st);
 
-struct DispatchArgs {
-    const int* counts; int n_exp, n_shared, ntok, top_k, dim;
-    int* offsets; int* fill; GroupTile* tiles; int* n_tiles; int max_tiles;
-    const int32_t* idx; const float* w; void* xperm; int* row_token; float* row_w;
-};
-rdt_status moe_dispatch(bool bf16_elems, const DispatchArgs& a, cudaStream_t st);
+// Copy yn[token] into the claimed row of every (token, slot) (routers that do not write
+// the copies themselves): xperm[a_routed_base + slot_row[token * k + j]] = xperm[token].
+rdt_status moe_copy(bool bf16_elems, void* xperm, const int* slot_row, int ntok, int top_k, int dim,
+                    int a_routed_base, cudaStream_t st);
 
 rdt_status lora_down(bool bf16_elems, const void* x, int ldx, int ntok, int width,
                      const void* lora_a, int r, void* t_out, cudaStream_t st);

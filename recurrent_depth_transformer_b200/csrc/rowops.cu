@@ -6,8 +6,8 @@
 //                  experts), router logits yn W_r^T in fp32, top-k of logits + bias with
 //                  ties to the lower expert index, softmax over the k chosen logits,
 //                  per-expert histogram
-//   moe_dispatch   per-expert offsets and the grouped-GEMM tile list (device side), then
-//                  the scatter of each (token, slot) to its expert's rows
+//   moe_copy       the copy of each token's normalised row into the expert rows its
+//                  router claimed (capacity layout), for routers that do not write them
 //   lora_down      t = x A^T for the O-projection adapter
 //   mla_latent_norm  RMSNorm of c_q and c_kv, RoPE of the decoupled key
 // plus the weight-preparation matmul and a finite-value check.
@@ -235,7 +235,13 @@ __global__ void __launch_bounds__(kRowThreads) norm2_router_kernel(const RouterA
         a.w[o] = wv;
         if (a.trace_idx) a.trace_idx[o] = sel_idx;
         if (a.trace_w) a.trace_w[o] = wv;
-        atomicAdd(a.counts + sel_idx, 1);
+        const int pos = atomicAdd(a.counts + sel_idx, 1);     // histogram and row claim
+        if (a.row_token) {
+            const int rr = sel_idx * a.cap + pos;
+            a.row_token[rr] = row;
+            a.row_w[rr] = wv;
+            a.slot_row[o] = rr;
+        }
     }
 }
 
@@ -270,6 +276,8 @@ __global__ void __launch_bounds__(kRowThreads) norm2_split_kernel(const Norm2Arg
     }
     ss = warp_sum(ss);
     const float inv = rsqrtf(ss / a.dim + a.eps);
+    if (a.zero_rows)
+        for (int i = lane; i < a.zero_width; i += 32) a.zero_rows[static_cast<size_t>(row) * a.zero_width + i] = 0.0f;
     T* yn = static_cast<T*>(a.yn) + base;
     T* lo = static_cast<T*>(a.yn_lo) + base;
 #pragma unroll
@@ -289,80 +297,23 @@ __global__ void __launch_bounds__(kRowThreads) norm2_split_kernel(const Norm2Arg
     }
 }
 
-// ----------------------------------------------------------------------------- MoE dispatch
+// ----------------------------------------------------------------------------- MoE dispatch copy
 
-// One block: exclusive scans of the routed counts (row offsets inside the routed region)
-// and of the per-group tile counts; writes the grouped-GEMM tile list.
-__global__ void __launch_bounds__(256) moe_scan_kernel(const DispatchArgs a) {
-    __shared__ int s_cnt[256], s_tiles[256], s_off[256], s_toff[256];
-    pdl_trigger();
-    pdl_wait();
-    const int G = a.n_exp + a.n_shared;
-    const int t = threadIdx.x;
-    const int cnt = t < a.n_exp ? a.counts[t] : (t < G ? a.ntok : 0);
-    s_cnt[t] = t < a.n_exp ? cnt : 0;
-    s_tiles[t] = t < G ? (cnt + 127) / 128 : 0;
-    __syncthreads();
-    // Hillis-Steele inclusive scans
-    for (int d = 1; d < 256; d <<= 1) {
-        const int v1 = t >= d ? s_cnt[t - d] : 0;
-        const int v2 = t >= d ? s_tiles[t - d] : 0;
-        __syncthreads();
-        s_cnt[t] += v1;
-        s_tiles[t] += v2;
-        __syncthreads();
-    }
-    s_off[t] = t == 0 ? 0 : s_cnt[t - 1];
-    s_toff[t] = t == 0 ? 0 : s_tiles[t - 1];
-    __syncthreads();
-    if (t < a.n_exp) {
-        a.offsets[t] = s_off[t];
-        a.fill[t] = 0;
-    }
-    if (t == 0) *a.n_tiles = s_tiles[255];
-    if (t < G) {
-        const int ntile = (cnt + 127) / 128;
-        for (int i = 0; i < ntile; ++i) {
-            GroupTile gt;
-            gt.group = t;
-            gt.nrows = min(128, cnt - 128 * i);
-            if (t < a.n_exp) {
-                gt.a_row0 = a.ntok + s_off[t] + 128 * i;                      // routed copies
-                gt.c_row0 = a.n_shared * a.ntok + s_off[t] + 128 * i;
-            } else {
-                const int s = t - a.n_exp;
-                gt.a_row0 = 128 * i;                                          // yn itself
-                gt.c_row0 = s * a.ntok + 128 * i;
-            }
-            const int slot = s_toff[t] + i;
-            if (slot < a.max_tiles) a.tiles[slot] = gt;
-        }
-    }
-}
-
-// One warp per (token, slot): claim a row in the expert's range, record token and gate
-// weight, copy the normalised row yn[token] into it.
+// One warp per (token, slot): copy the normalised row yn[token] into the row the router
+// claimed for it (capacity layout).
 template <typename T>
-__global__ void __launch_bounds__(kRowThreads) moe_scatter_kernel(const DispatchArgs a) {
+__global__ void __launch_bounds__(kRowThreads) moe_copy_kernel(T* xperm, const int* slot_row, int ntok,
+                                                               int top_k, int dim, int a_routed_base) {
     pdl_trigger();
     pdl_wait();
     const int ws = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (ws >= a.ntok * a.top_k) return;
-    const int n = ws / a.top_k;
-    const int ex = a.idx[ws];
-    int pos = 0;
-    if (lane == 0) pos = atomicAdd(a.fill + ex, 1);
-    pos = __shfl_sync(0xffffffffu, pos, 0);
-    const int r = a.offsets[ex] + pos;
-    if (lane == 0) {
-        a.row_token[r] = n;
-        a.row_w[r] = a.w[ws];
-    }
-    T* xp = static_cast<T*>(a.xperm);
-    const uint4* src = reinterpret_cast<const uint4*>(xp + static_cast<size_t>(n) * a.dim);
-    uint4* dst = reinterpret_cast<uint4*>(xp + static_cast<size_t>(a.ntok + r) * a.dim);
-    const int nvec = a.dim * static_cast<int>(sizeof(T)) / 16;
+    if (ws >= ntok * top_k) return;
+    const int n = ws / top_k;
+    const int r = a_routed_base + slot_row[ws];
+    const uint4* src = reinterpret_cast<const uint4*>(xperm + static_cast<size_t>(n) * dim);
+    uint4* dst = reinterpret_cast<uint4*>(xperm + static_cast<size_t>(r) * dim);
+    const int nvec = dim * static_cast<int>(sizeof(T)) / 16;
     for (int i = lane; i < nvec; i += 32) dst[i] = src[i];
 }
 
@@ -556,14 +507,16 @@ rdt_status norm2_router(bool bf, const RouterArgs& a, cudaStream_t st) {
               : launch_rows<float, RouterL>(nv, a.ntok, st, a);
 }
 
-rdt_status moe_dispatch(bool bf, const DispatchArgs& a, cudaStream_t st) {
-    RDT_CUDA_TRY(launch_pdl(moe_scan_kernel, dim3(1), dim3(256), 0, st, a));
-    const int warps = a.ntok * a.top_k;
+rdt_status moe_copy(bool bf, void* xperm, const int* slot_row, int ntok, int top_k, int dim,
+                    int a_routed_base, cudaStream_t st) {
+    const int warps = ntok * top_k;
     const dim3 grid((warps + kRowThreads / 32 - 1) / (kRowThreads / 32));
     if (bf)
-        RDT_CUDA_TRY(launch_pdl(moe_scatter_kernel<bf16>, grid, dim3(kRowThreads), 0, st, a));
+        RDT_CUDA_TRY(launch_pdl(moe_copy_kernel<bf16>, grid, dim3(kRowThreads), 0, st, static_cast<bf16*>(xperm),
+                                slot_row, ntok, top_k, dim, a_routed_base));
     else
-        RDT_CUDA_TRY(launch_pdl(moe_scatter_kernel<float>, grid, dim3(kRowThreads), 0, st, a));
+        RDT_CUDA_TRY(launch_pdl(moe_copy_kernel<float>, grid, dim3(kRowThreads), 0, st, static_cast<float*>(xperm),
+                                slot_row, ntok, top_k, dim, a_routed_base));
     RDT_CUDA_TRY(cudaGetLastError());
     return RDT_OK;
 }

@@ -76,3 +76,22 @@ def test_attention_f32():
     ref = O.gqa_attention(q.numpy().reshape(1, seq, hq, d), k.numpy().reshape(1, seq, hkv, d),
                           v.numpy().reshape(1, seq, hkv, d), 0.2)
     assert np.abs(o.cpu().numpy().reshape(ref.shape) - ref).max() < 1e-4
+
+
+@pytest.mark.parametrize("batch,seq,hq", [(2, 130, 4), (1, 300, 16)])
+def test_attention_shared_latent_kv(batch, seq, hq):
+    """Absorbed MLA: every head attends over the shared 160-wide key [c_kv ; k_rope] with the
+    value c_kv = the key's first 128 columns (v passed as the key tensor itself)."""
+    torch = _torch()
+    import recurrent_depth_transformer_b200 as R
+    g = torch.Generator().manual_seed(seq + hq)
+    q = torch.randn(batch * seq, hq * 160, generator=g).to(torch.bfloat16)
+    k = torch.randn(batch * seq, 160, generator=g).to(torch.bfloat16)
+    scale = 1.0 / math.sqrt(96)
+    kc = k.cuda()
+    o = R.attention(q.cuda(), kc, kc, batch, seq, hq, 1, 160, 128, scale)
+    torch.cuda.synchronize()
+    kf = k.float().numpy().reshape(batch, seq, 1, 160)
+    ref = O.gqa_attention(q.float().numpy().reshape(batch, seq, hq, 160), kf, kf[..., :128], scale)
+    err = np.abs(o.cpu().float().numpy().reshape(ref.shape) - ref).max()
+    assert err < 2e-2, err
