@@ -38,7 +38,12 @@ struct TcCfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     // two accumulators of BN fp32 columns, rounded up to a power of two
     static constexpr int TMEM_COLS = 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
-    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+    // [stages][barriers][group tables]: all dynamic, so that the kernel (with the 1 KB the
+    // driver reserves per CTA) stays within the 196 KB shared-memory carveout and keeps
+    // 60 KB of L1 for the epilogue's loads
+    static constexpr int BAR_BYTES = 192;
+    static constexpr int GROUP_BYTES = 2064;
+    static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + GROUP_BYTES;
     static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte alignment of stages");
 };
 
@@ -428,18 +433,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr bool kBf16 = std::is_same<T, bf16>::value;
     constexpr int kElemsPerRow = 128 / static_cast<int>(sizeof(T));   // K elements per stage
 
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // The dynamic shared memory of a CTA without static shared memory starts 1024-aligned,
+    // as the 128-byte swizzle atoms need; checked below rather than padded for.
+    extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
     uint64_t* empty = full + C::STAGES;
     uint64_t* tfull = empty + C::STAGES;      // accumulator b ready for the epilogue
     uint64_t* tempty = tfull + 2;             // accumulator b drained by the epilogue
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    GroupTables& s_groups = *reinterpret_cast<GroupTables*>(smem + C::STAGES * C::STAGE_BYTES + C::BAR_BYTES);
+    static_assert(2 * C::STAGES * 8 + 4 * 8 + 4 <= C::BAR_BYTES, "barrier area");
+    static_assert(sizeof(GroupTables) <= C::GROUP_BYTES, "group tables");
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    __shared__ GroupTables s_groups;
+    if (smem_u32(smem) & 1023) {              // uniform per CTA: misaligned base, do nothing
+        if (threadIdx.x == 0 && epi.flags) atomicExch(epi.flags + FLAG_TIMEOUT, 1);
+        return;
+    }
 
     if (threadIdx.x == 0) {
 #pragma unroll 1
