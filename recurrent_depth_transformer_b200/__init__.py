@@ -49,7 +49,8 @@ class RdtConfig(ctypes.Structure):
         "q_lora_rank", "kv_lora_rank", "qk_nope_dim", "qk_rope_dim", "v_head_dim")] + [
         ("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float)] + [
         (n, ctypes.c_int32) for n in ("n_experts", "top_k", "n_shared", "expert_hidden",
-                                      "lora_rank", "n_lora", "b_kind", "inject_e", "max_loops")]
+                                      "lora_rank", "n_lora", "b_kind", "inject_e", "max_loops",
+                                      "gemm_tiles")]
 
 
 WEIGHT_FIELDS = ("A", "B", "norm1", "norm2", "wq", "wk", "wv", "wo", "w_dq", "q_norm", "w_uq",
@@ -121,7 +122,8 @@ def _check(status: int) -> None:
         raise RdtError(status, lib.rdt_last_error().decode(errors="replace"))
 
 
-def make_config(wl, max_loops: int = 16, batch: Optional[int] = None, seq: Optional[int] = None) -> RdtConfig:
+def make_config(wl, max_loops: int = 16, batch: Optional[int] = None, seq: Optional[int] = None,
+                gemm_tiles: int = 0) -> RdtConfig:
     """Fill the C config from any object with the block's hyper-parameters as attributes."""
     c = RdtConfig()
     c.dtype = RDT_BF16 if wl.dtype == "bf16" else RDT_F32
@@ -148,6 +150,7 @@ def make_config(wl, max_loops: int = 16, batch: Optional[int] = None, seq: Optio
     c.b_kind = RDT_B_DIAG if wl.b_kind == "diag" else RDT_B_DENSE
     c.inject_e = 1 if wl.inject_e else 0
     c.max_loops = max_loops
+    c.gemm_tiles = gemm_tiles
     return c
 
 

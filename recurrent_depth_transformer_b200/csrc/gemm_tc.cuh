@@ -1,0 +1,773 @@
+// Dense and grouped GEMM on the sm_100a 5th-generation tensor cores, C = A * B^T.
+//
+// Kernel template shared by the single-CTA and the CTA-pair instantiations. A single CTA
+// computes 128 x BN output tiles; a CTA pair (cluster of two, cta_group::2) computes
+// 256 x BN tiles, each CTA loading its 128 rows of A and half of the tile's B rows, the even
+// CTA issuing the M = 256 MMAs that read both halves, each CTA holding its 128 accumulator
+// rows in its own TMEM. The pair loads half as many bytes per multiply-add as one CTA,
+// which is what bounds these GEMMs (per-SM ingest from L2), not the tensor pipe.
+//
+// Roles inside a CTA:
+//   warp 0      one thread issues TMA loads of 128-byte-wide K slices of A and B into a
+//               ring of shared-memory stages (128-byte swizzle, K-major);
+//   warp 1      allocates the TMEM accumulator; one thread issues tcgen05.mma (M = 128,
+//               N = BN, K = 16 bf16 / 8 tf32 per instruction) and frees each stage with
+//               tcgen05.commit when its MMAs have read it;
+//   warps 2-5   the epilogue: each warp reads its 32-lane quadrant of TMEM (one output row
+//               per thread, 32 columns at a time), transposes the 32 x 32 chunk through a
+//               private shared-memory buffer so that each global access of the warp covers
+//               four whole row segments, and applies one of the fused epilogues below.
+//
+// The fused epilogues are where the block's element-wise work lives:
+//   EPI_ROPE        Q/K/V projection + rotary embedding on the rotated heads;
+//   EPI_OPROJ_LOOP  output projection fused with the residual (y = x + a) and the
+//                   recurrent update h_next = A (.) h + B.e + a (the MoE adds f later);
+//   EPI_SWIGLU      expert up-projection (gate and up rows interleaved per tile) -> silu(g)*u;
+//   EPI_SCATTER     expert down-projection, gate weight, and reduction into h_next
+//                   (h_{t+1} = A h + B e + a + sum_j w_j E_j(yn)).
+// Grouped mode decodes its tiles from the per-expert row counters on the device (capacity
+// layout: expert e's rows start at e * tokens), so the counts never travel to the host.
+#pragma once
+#include <algorithm>
+#include <type_traits>
+
+#include "rdt_internal.cuh"
+
+namespace rdt {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int kThreads = 192;
+
+template <int BN, int CG>
+struct TcCfg {
+    static constexpr int B_ROWS = BN / CG;               // B rows this CTA loads per stage
+    static constexpr int A_BYTES = BM * 128;
+    static constexpr int B_BYTES = B_ROWS * 128;
+    static constexpr int STAGES = (A_BYTES + B_BYTES <= 24 * 1024) ? 8 : (A_BYTES + B_BYTES <= 32 * 1024) ? 6 : 4;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    // two accumulators of BN fp32 columns, rounded up to a power of two
+    static constexpr int TMEM_COLS = 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
+    // [stages][barriers][group tables][epilogue staging], all dynamic (no static shared
+    // memory, so that the dynamic block starts 1024-byte aligned)
+    static constexpr int BAR_BYTES = 192;
+    static constexpr int GROUP_BYTES = 2064;
+    static constexpr int STG_BYTES = 4 * 32 * 32 * 4;     // one 32 x 32 fp32 chunk per epilogue warp
+    static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + GROUP_BYTES + STG_BYTES;
+    static_assert((BAR_BYTES + GROUP_BYTES) % 16 == 0, "staging buffers must be 16-byte aligned");
+    static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte alignment of stages");
+    static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
+};
+
+__device__ __forceinline__ void ld_chunk(uint32_t taddr, int c, float (&v)[32]) {
+    uint32_t r[32];
+    tmem_ld32(taddr + static_cast<uint32_t>(c * 32), r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Transpose of one warp's 32 x 32 fp32 chunk through its private staging buffer. Before:
+// lane l holds row l (as TMEM hands it out). After: pass it = 0..7 gives lane l row
+// 4 * it + l / 8, columns 4 * (l % 8) .. + 3, so a warp-wide 16-byte access covers four
+// contiguous row segments rather than 32 rows. The 16-byte slots of a row are XOR-swizzled
+// by the row index: eight lanes of a quarter-warp always hit eight different bank groups,
+// in both directions.
+__device__ __forceinline__ void stage_put(float* stg, int lane, const float (&v)[32]) {
+    __syncwarp();                                   // the previous chunk has been read
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        *reinterpret_cast<float4*>(stg + lane * 32 + ((k ^ (lane & 7)) << 2)) =
+            make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+    __syncwarp();
+}
+
+__device__ __forceinline__ void stage_get(const float* stg, int lane, int it, float (&o)[4]) {
+    const int row = it * 4 + (lane >> 3);
+    const float4 x = *reinterpret_cast<const float4*>(stg + row * 32 + (((lane & 7) ^ (row & 7)) << 2));
+    o[0] = x.x; o[1] = x.y; o[2] = x.z; o[3] = x.w;
+}
+
+// Store a 32-column chunk of the warp's 32 rows (row-per-lane in v) to base[r * ld + c],
+// r < nvalid.
+template <typename OutT>
+__device__ __forceinline__ void store_chunk(float* stg, int lane, const float (&v)[32], OutT* base,
+                                            size_t ld, int nvalid) {
+    stage_put(stg, lane, v);
+    const int cc = (lane & 7) * 4;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+        const int rr = it * 4 + (lane >> 3);
+        float o[4];
+        stage_get(stg, lane, it, o);
+        if (rr < nvalid) store4(base + rr * ld + cc, o);
+    }
+}
+
+// ----------------------------------------------------------------------------- epilogues
+
+// Router top-k: keep the KMAX best (score = logit + bias) in registers, visiting experts in
+// ascending index so that strict comparisons leave ties to the lower index; gate weights
+// are the softmax of the chosen logits.
+template <int KMAX>
+struct TopK {
+    float bs[KMAX], bl[KMAX];
+    int bi[KMAX];
+    __device__ __forceinline__ TopK() {
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            bs[j] = -INFINITY;
+            bl[j] = 0.0f;
+            bi[j] = -1;
+        }
+    }
+    __device__ __forceinline__ void insert(float logit, float bias, int ex, int k) {
+        float cs = logit + bias, cl = logit;
+        int ci = ex;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j < k && cs > bs[j]) {
+                const float ts = bs[j], tl = bl[j];
+                const int ti = bi[j];
+                bs[j] = cs; bl[j] = cl; bi[j] = ci;
+                cs = ts; cl = tl; ci = ti;
+            }
+        }
+    }
+    __device__ __forceinline__ void write(const EpiParams& p, int row) const {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+            if (j < p.top_k && bi[j] >= 0) mx = fmaxf(mx, bl[j]);
+        float ex[KMAX], den = 0.0f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            ex[j] = (j < p.top_k && bi[j] >= 0) ? expf(bl[j] - mx) : 0.0f;
+            den += ex[j];
+        }
+        const size_t o = static_cast<size_t>(row) * p.top_k;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j >= p.top_k) break;
+            const int e = bi[j] < 0 ? 0 : bi[j];      // only when every score was NaN
+            const float w = den > 0.0f ? ex[j] / den : 0.0f;
+            p.idx_out[o + j] = e;
+            p.w_out[o + j] = w;
+            if (p.trace_idx) p.trace_idx[o + j] = e;
+            if (p.trace_w) p.trace_w[o + j] = w;
+            const int pos = atomicAdd(p.counts + e, 1);          // histogram and row claim
+            if (p.route_token) {
+                const int rr = e * p.cap + pos;
+                p.route_token[rr] = row;
+                p.route_w[rr] = w;
+                p.slot_row[o + j] = rr;
+            }
+        }
+    }
+};
+
+// Router epilogue. Unsplit: the thread's row holds all logits (BN >= n_exp) in TMEM.
+// Split over K: every CTA adds its partial logits into p.logits; the CTA that arrives last
+// on the row tile's counter (threadfence-reduction order: adds, fence, count) reads the
+// complete rows back and selects.
+template <int BN, int KMAX>
+__device__ __forceinline__ void epilogue_topk(const EpiParams& p, uint32_t taddr, bool valid, int crow,
+                                              int split, int mtile) {
+    if (split <= 1) {
+        TopK<KMAX> tk;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            ld_chunk(taddr, c, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int ex = c * 32 + i;
+                if (ex < p.n_exp) tk.insert(v[i], p.bias ? p.bias[ex] : 0.0f, ex, p.top_k);
+            }
+        }
+        if (valid) tk.write(p, crow);
+        return;
+    }
+    __shared__ int s_last;
+    float* lrow = p.logits + static_cast<size_t>(crow) * p.n_exp;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        ld_chunk(taddr, c, v);
+        if (!valid) continue;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int ex = c * 32 + i;
+            if (ex < p.n_exp) atomicAdd(lrow + ex, v[i]);
+        }
+    }
+    __threadfence();
+    asm volatile("bar.sync 1, 128;" ::: "memory");     // the four epilogue warps
+    if (threadIdx.x == 64) {
+        const int old = atomicAdd(p.tile_count + mtile, 1);
+        s_last = old == split - 1;
+        if (s_last) p.tile_count[mtile] = 0;             // ready for the next launch
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (!s_last) return;
+    __threadfence();
+    if (!valid) return;
+    TopK<KMAX> tk;
+#pragma unroll 1
+    for (int ex = 0; ex < p.n_exp; ++ex)
+        tk.insert(__ldcg(lrow + ex), p.bias ? p.bias[ex] : 0.0f, ex, p.top_k);
+    tk.write(p, crow);
+}
+
+// One epilogue warp's share of a tile: rows row0 .. row0 + 31 of C (lane l owns row
+// row0 + l in TMEM, the first nvalid of them are real), columns n0 .. n0 + BN - 1.
+template <typename T, int BN, int KIND>
+__device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, float* stg, int lane,
+                                         int nvalid, int row0, int n0, int split = 1, int mtile = 0) {
+    const int cc = (lane & 7) * 4;                 // this lane's columns after the transpose
+    if constexpr (KIND == EPI_STORE || KIND == EPI_STORE_F32 || KIND == EPI_OPROJ_PLAIN) {
+        using OutT = std::conditional_t<KIND == EPI_STORE, T, float>;
+        OutT* out = static_cast<OutT*>(p.out) + static_cast<size_t>(row0) * p.ldo;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            ld_chunk(taddr, c, v);
+            const int col = n0 + c * 32;
+            if (col < p.ncols_valid) store_chunk(stg, lane, v, out + col, p.ldo, nvalid);
+        }
+    } else if constexpr (KIND == EPI_ROPE) {
+        // Heads of width head_w tile the BN columns exactly (host checks BN % head_w == 0).
+        // The rotation pairs columns i and i + rot/2 of a head, so it runs row-per-lane
+        // (before the transpose). The angle tables are [rot/2][seq]: for a fixed frequency
+        // the lanes (consecutive positions) read consecutive floats.
+        const int pos = (row0 + lane) % p.seq;
+        const int hw_chunks = p.head_w / 32;
+        const int rc0 = p.rot_off / 32;
+        const int rch = p.rot_dim / 32;
+        const int half = p.rot_dim / 2;
+        float cs[32], sn[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            cs[i] = i < half ? p.rope_cos[static_cast<size_t>(i) * p.seq + pos] : 0.0f;
+            sn[i] = i < half ? p.rope_sin[static_cast<size_t>(i) * p.seq + pos] : 0.0f;
+        }
+        T* out = static_cast<T*>(p.out) + static_cast<size_t>(row0) * p.ldo;
+#pragma unroll 1
+        for (int hc = 0; hc < BN / 32; hc += hw_chunks) {
+            const int head_col0 = n0 + hc * 32;
+            const bool rotate = head_col0 < p.rope_limit;
+#pragma unroll 1
+            for (int c = 0; c < hw_chunks; ++c) {
+                const int col = head_col0 + c * 32;
+                const bool keep = col < p.ncols_valid;
+                if (rotate && c == rc0) {
+                    if (rch == 2) {
+                        float v0[32], v1[32];
+                        ld_chunk(taddr, hc + c, v0);
+                        ld_chunk(taddr, hc + c + 1, v1);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float x1 = v0[i], x2 = v1[i];
+                            v0[i] = x1 * cs[i] - x2 * sn[i];
+                            v1[i] = x2 * cs[i] + x1 * sn[i];
+                        }
+                        if (keep) {
+                            store_chunk(stg, lane, v0, out + col, p.ldo, nvalid);
+                            store_chunk(stg, lane, v1, out + col + 32, p.ldo, nvalid);
+                        }
+                        c += 1;
+                    } else {
+                        float v[32];
+                        ld_chunk(taddr, hc + c, v);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float x1 = v[i], x2 = v[i + 16];
+                            v[i] = x1 * cs[i] - x2 * sn[i];
+                            v[i + 16] = x2 * cs[i] + x1 * sn[i];
+                        }
+                        if (keep) store_chunk(stg, lane, v, out + col, p.ldo, nvalid);
+                    }
+                } else {
+                    float v[32];
+                    ld_chunk(taddr, hc + c, v);
+                    if (keep) store_chunk(stg, lane, v, out + col, p.ldo, nvalid);
+                }
+            }
+        }
+    } else if constexpr (KIND == EPI_OPROJ_LOOP) {
+        // y = h + e + a and h_next = A (.) h + B.e + a. Every load of a chunk is issued before
+        // its stores (the stores could alias the loads as far as the compiler knows).
+        const T* e = static_cast<const T*>(p.e);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            ld_chunk(taddr, c, v);
+            const int col = n0 + c * 32 + cc;
+            if (n0 + c * 32 >= p.ncols_valid) continue;
+            stage_put(stg, lane, v);
+            float aa[4];
+            load4(p.Adiag + col, aa);
+            float hh[8][4], be[8][4], ee[8][4];
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+                const int rr = it * 4 + (lane >> 3);
+                const size_t off = static_cast<size_t>(row0 + rr) * p.ld + col;
+                if (rr < nvalid) {
+                    load4(p.h + off, hh[it]);
+                    load4(p.Be + off, be[it]);
+                    if (e) load4(e + off, ee[it]);
+                    else ee[it][0] = ee[it][1] = ee[it][2] = ee[it][3] = 0.0f;
+                }
+            }
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+                const int rr = it * 4 + (lane >> 3);
+                float av[4];
+                stage_get(stg, lane, it, av);
+                if (rr >= nvalid) continue;
+                const size_t off = static_cast<size_t>(row0 + rr) * p.ld + col;
+                float yv[4], hn[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    yv[i] = hh[it][i] + ee[it][i] + av[i];
+                    hn[i] = aa[i] * hh[it][i] + be[it][i] + av[i];
+                }
+                store4(p.y + off, yv);
+                store4(p.h_next + off, hn);
+            }
+        }
+    } else if constexpr (KIND == EPI_SWIGLU) {
+        // Tile columns [0, BN/2) are gate rows (W1), [BN/2, BN) the matching up rows (W3).
+        T* out = static_cast<T*>(p.out) + static_cast<size_t>(row0) * p.ldo + n0 / 2;
+#pragma unroll 1
+        for (int c = 0; c < BN / 64; ++c) {
+            float g[32], u[32];
+            ld_chunk(taddr, c, g);
+            ld_chunk(taddr, c + BN / 64, u);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) g[i] = g[i] / (1.0f + expf(-g[i])) * u[i];
+            store_chunk(stg, lane, g, out + c * 32, p.ldo, nvalid);
+        }
+    } else if constexpr (KIND == EPI_SCATTER) {
+        // Row r of the tile is expert output for token row_token[r] with gate weight row_w[r]
+        // (shared experts: every token, weight 1); it is added into h_next with vector atomics.
+        int token = -1;
+        float w = 0.0f;
+        if (lane < nvalid) {
+            const int crow = row0 + lane;
+            if (crow < p.shared_rows) {
+                token = crow % p.ntok;
+                w = 1.0f;
+            } else {
+                token = p.row_token[crow - p.shared_rows];
+                w = p.row_w[crow - p.shared_rows];
+            }
+        }
+        int tok[8];
+        float wt[8];
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+            tok[it] = __shfl_sync(0xffffffffu, token, it * 4 + (lane >> 3));
+            wt[it] = __shfl_sync(0xffffffffu, w, it * 4 + (lane >> 3));
+        }
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            ld_chunk(taddr, c, v);
+            const int col = n0 + c * 32;
+            if (col >= p.ncols_valid) continue;
+            stage_put(stg, lane, v);
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+                float o[4];
+                stage_get(stg, lane, it, o);
+                if (tok[it] < 0) continue;
+                const float4 add = make_float4(wt[it] * o[0], wt[it] * o[1], wt[it] * o[2], wt[it] * o[3]);
+                atomicAdd(reinterpret_cast<float4*>(p.dst + static_cast<size_t>(tok[it]) * p.ld + col + cc), add);
+            }
+        }
+    } else if constexpr (KIND == EPI_TOPK) {
+        const bool valid = lane < nvalid;
+        const int crow = row0 + lane;
+        if (p.top_k <= 2)
+            epilogue_topk<BN, 2>(p, taddr, valid, crow, split, mtile);
+        else if (p.top_k <= 4)
+            epilogue_topk<BN, 4>(p, taddr, valid, crow, split, mtile);
+        else if (p.top_k <= 8)
+            epilogue_topk<BN, 8>(p, taddr, valid, crow, split, mtile);
+        else
+            epilogue_topk<BN, 16>(p, taddr, valid, crow, split, mtile);
+    }
+}
+
+// ----------------------------------------------------------------------------- the kernel
+
+struct TileCoord {
+    int a_row0, c_row0, nrows, group, n0, mt, kb0, kb1;
+};
+
+// Grouped mode: pref[g] = first row tile of group g (routed groups, then shared ones),
+// pref[256] = tile count; cnt[g] = rows of group g.
+struct GroupTables {
+    int pref[257];
+    int cnt[256];
+};
+
+__device__ __forceinline__ void build_group_tables(const GemmArgs& args, GroupTables& t, int lane,
+                                                   int tile_rows) {
+    const int G = args.n_routed + args.n_shared;
+    int tiles[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int g = lane * 8 + i;
+        const int c = g < args.n_routed ? args.counts[g] : (g < G ? args.M : 0);   // shared: all tokens
+        t.cnt[g] = c;
+        tiles[i] = (c + tile_rows - 1) / tile_rows;
+        sum += tiles[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        t.pref[lane * 8 + i] = run;
+        run += tiles[i];
+    }
+    if (lane == 31) t.pref[256] = incl;
+}
+
+// tile = (mt * n_ntiles + nt) * split + ks; split > 1 divides the K blocks evenly.
+// Rows are those of the whole (pair) tile: tile_rows = 128 or 256.
+__device__ __forceinline__ TileCoord tile_coord(const GemmArgs& args, const GroupTables* gt, int tile,
+                                                int n_ntiles, int bn, int split, int num_kb,
+                                                int tile_rows) {
+    TileCoord t;
+    const int ks = tile % split;
+    tile /= split;
+    const int mt = tile / n_ntiles;
+    t.mt = mt;
+    t.n0 = (tile - mt * n_ntiles) * bn;
+    const int per = (num_kb + split - 1) / split;
+    t.kb0 = ks * per;
+    t.kb1 = min(num_kb, t.kb0 + per);
+    if (gt != nullptr) {
+        const int G = args.n_routed + args.n_shared;
+        int lo = 0, hi = G - 1;                      // last group whose first tile <= mt
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (gt->pref[mid] <= mt) lo = mid; else hi = mid - 1;
+        }
+        const int local = (mt - gt->pref[lo]) * tile_rows;
+        t.group = lo;
+        t.nrows = min(tile_rows, gt->cnt[lo] - local);
+        if (lo < args.n_routed) {
+            t.a_row0 = args.a_routed_base + lo * args.cap + local;
+            t.c_row0 = (args.n_shared + lo) * args.cap + local;
+        } else {
+            t.a_row0 = local;
+            t.c_row0 = (lo - args.n_routed) * args.cap + local;
+        }
+        if (args.a_from_c) t.a_row0 = t.c_row0;
+    } else {
+        t.group = 0;
+        t.a_row0 = mt * tile_rows;
+        t.c_row0 = t.a_row0;
+        t.nrows = min(tile_rows, args.M - t.a_row0);
+    }
+    return t;
+}
+
+// Persistent: each CTA (pair) walks tiles cid, cid + n_clusters, ... The TMA warp and the
+// MMA warp run ahead through a ring of shared-memory stages; the accumulator is
+// double-buffered in TMEM so the epilogue of one tile overlaps the MMAs of the next.
+//
+// Pair protocol (CG = 2; "leader" = the even CTA):
+//   full[s]   leader only: one arrival, the leader producer's expect_tx for the bytes of
+//             both CTAs; both CTAs' TMA loads complete on it (the peer's bytes may land
+//             before that arrival: the phase cannot complete while it is pending).
+//   empty[s]  each CTA: the leader's commit arrives on both CTAs' barriers when the MMAs
+//             that read stage s (in both CTAs) are done.
+//   tfull[b]  each CTA: the leader's commit arrives on both when accumulator b is complete.
+//   tempty[b] leader only: eight arrivals, the epilogue warps of both CTAs.
+// Every wait is bounded; on a timeout the roles stop and the kernel still passes its
+// closing barriers.
+template <typename T, int BN, int KIND, int CG>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
+                   const __grid_constant__ CUtensorMap tA2, const __grid_constant__ CUtensorMap tB2,
+                   const GemmArgs args, const EpiParams epi) {
+    using C = TcCfg<BN, CG>;
+    constexpr bool kBf16 = std::is_same<T, bf16>::value;
+    constexpr int kElemsPerRow = 128 / static_cast<int>(sizeof(T));   // K elements per stage
+    constexpr int kTileRows = BM * CG;
+    static_assert(CG == 1 || kBf16, "pair tiles are bf16 only");
+
+    // The dynamic shared memory of a CTA without static shared memory starts 1024-aligned,
+    // as the 128-byte swizzle atoms need; checked below rather than padded for (the result
+    // is the same in both CTAs of a pair).
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+    uint64_t* empty = full + C::STAGES;
+    uint64_t* tfull = empty + C::STAGES;      // accumulator b ready for the epilogue
+    uint64_t* tempty = tfull + 2;             // accumulator b drained by the epilogue
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    GroupTables& s_groups = *reinterpret_cast<GroupTables*>(smem + C::STAGES * C::STAGE_BYTES + C::BAR_BYTES);
+    static_assert(2 * C::STAGES * 8 + 4 * 8 + 4 <= C::BAR_BYTES, "barrier area");
+    static_assert(sizeof(GroupTables) <= C::GROUP_BYTES, "group tables");
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    // A misaligned base (never expected) skips every tile but still passes the barriers
+    // below, so that a CTA pair cannot be left waiting on one of its CTAs.
+    const bool misaligned = (smem_u32(smem) & 1023) != 0;
+    if (misaligned && threadIdx.x == 0 && epi.flags) atomicExch(epi.flags + FLAG_TIMEOUT, 1);
+    const uint32_t rank = CG == 2 ? cluster_ctarank() : 0;
+    const bool leader = rank == 0;
+
+    if (threadIdx.x == 0) {
+#pragma unroll 1
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4 * CG);    // one arrival per epilogue warp of the pair
+        }
+        mbar_fence_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tA);
+        tma_prefetch_desc(&tB);
+    }
+    if (warp == 1) {
+        if constexpr (CG == 2) {
+            tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, C::TMEM_COLS);
+            tmem_relinquish();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if constexpr (CG == 2) cluster_sync();    // the peer's barriers exist before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_trigger();
+    pdl_wait();
+
+    const GroupTables* gt = nullptr;
+    if (args.counts != nullptr && !misaligned) {   // grouped: per-group tile offsets from the counters
+        if (warp == 0) build_group_tables(args, s_groups, lane, kTileRows);
+        __syncthreads();
+        gt = &s_groups;
+    }
+    const int n_ntiles = (args.N + BN - 1) / BN;
+    const int n_mtiles = gt != nullptr ? gt->pref[256]
+                       : args.counts != nullptr ? 0 : (args.M + kTileRows - 1) / kTileRows;
+    const int split = args.split_k > 1 ? args.split_k : 1;
+    const int total = misaligned ? 0 : n_mtiles * n_ntiles * split;
+    const int num_kb = args.kb_main + args.kb_ext;
+    const int cid = static_cast<int>(blockIdx.x) / CG;
+    const int ncl = static_cast<int>(gridDim.x) / CG;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // the leader's full barriers, by cluster address (own address when CG == 1)
+            const uint32_t full0 = CG == 2 ? mapa_shared(smem_u32(full), 0) : smem_u32(full);
+            int it = 0;
+            bool ok = true;
+#pragma unroll 1
+            for (int tile = cid; tile < total && ok; tile += ncl) {
+                const TileCoord tc = tile_coord(args, gt, tile, n_ntiles, BN, split, num_kb, kTileRows);
+                const int a_row = tc.a_row0 + static_cast<int>(rank) * BM;
+                const int b_row = tc.group * args.N + tc.n0 + static_cast<int>(rank) * C::B_ROWS;
+#pragma unroll 1
+                for (int kb = tc.kb0; kb < tc.kb1; ++kb, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t ph = (it / C::STAGES) & 1;
+                    if (!mbar_wait(&empty[s], ph ^ 1, epi.flags)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + s * C::STAGE_BYTES;
+                    uint8_t* sb = sa + C::A_BYTES;
+                    const bool ext = kb >= args.kb_main;
+                    const CUtensorMap* ma = ext ? &tA2 : &tA;
+                    const CUtensorMap* mb = ext ? &tB2 : &tB;
+                    const int kx = (ext ? kb - args.kb_main : kb) * kElemsPerRow;
+                    const int brow = ext ? args.b2_row0 + b_row : b_row;
+                    if constexpr (CG == 2) {
+                        const uint32_t fb = full0 + static_cast<uint32_t>(s) * 8;
+                        if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::STAGE_BYTES);
+                        tma_load_2d_pair(sa, ma, fb, kx, a_row);
+                        tma_load_2d_pair(sb, mb, fb, kx, brow);
+                    } else {
+                        mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+                        tma_load_2d(sa, ma, &full[s], kx, a_row);
+                        tma_load_2d(sb, mb, &full[s], kx, brow);
+                    }
+                }
+            }
+            // Tail: wait until the MMAs have released every stage this CTA filled, so that no
+            // commit to this CTA's barriers, and no MMA read of its stages, is still in flight
+            // when it leaves.
+            // (fill i of stage i % STAGES is released by phase i / STAGES of its barrier).
+#pragma unroll 1
+            for (int i = it > C::STAGES ? it - C::STAGES : 0; ok && i < it; ++i)
+                if (!mbar_wait(&empty[i % C::STAGES], (i / C::STAGES) & 1, epi.flags)) ok = false;
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            constexpr uint32_t idesc = make_idesc(kBf16 ? 1 : 2, kTileRows, BN);
+            int it = 0, local = 0;
+            bool ok = true;
+#pragma unroll 1
+            for (int tile = cid; tile < total && ok; tile += ncl, ++local) {
+                const int b = local & 1;
+                const uint32_t use = static_cast<uint32_t>(local >> 1);
+                if (!mbar_wait(&tempty[b], (use & 1) ^ 1, epi.flags)) break;
+                tc_fence_after();
+                const uint32_t dt = tmem + static_cast<uint32_t>(b * BN);
+                const TileCoord tc = tile_coord(args, gt, tile, n_ntiles, BN, split, num_kb, kTileRows);
+#pragma unroll 1
+                for (int kb = tc.kb0; kb < tc.kb1; ++kb, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t ph = (it / C::STAGES) & 1;
+                    if (!mbar_wait(&full[s], ph, epi.flags)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+                    const uint64_t da = sw128_kmajor_desc(sa);
+                    const uint64_t db = sw128_kmajor_desc(sa + C::A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        // each MMA consumes 32 bytes of K: advance the start address by 32 B (>> 4 = 2)
+                        const uint32_t acc = (kb > tc.kb0) || k;
+                        if constexpr (CG == 2)
+                            tc_mma_bf16_pair(dt, da + 2 * k, db + 2 * k, idesc, acc);
+                        else if constexpr (kBf16)
+                            tc_mma_bf16(dt, da + 2 * k, db + 2 * k, idesc, acc);
+                        else
+                            tc_mma_tf32(dt, da + 2 * k, db + 2 * k, idesc, acc);
+                    }
+                    if constexpr (CG == 2) tc_commit_pair(&empty[s], 0x3);
+                    else tc_commit(&empty[s]);
+                }
+                if (!ok) break;
+                if constexpr (CG == 2) tc_commit_pair(&tfull[b], 0x3);
+                else tc_commit(&tfull[b]);
+            }
+        }
+    } else {
+        const int q = warp & 3;            // TMEM lane quadrant accessible to this warp
+        float* stg = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES + C::BAR_BYTES +
+                                              C::GROUP_BYTES) + (warp - 2) * 32 * 32;
+        const uint32_t tempty0 = CG == 2 ? mapa_shared(smem_u32(tempty), 0) : smem_u32(tempty);
+        const int row_off = static_cast<int>(rank) * BM + q * 32;   // first row of this warp in the tile
+        int local = 0;
+#pragma unroll 1
+        for (int tile = cid; tile < total; tile += ncl, ++local) {
+            const int b = local & 1;
+            const uint32_t use = static_cast<uint32_t>(local >> 1);
+            const TileCoord tc = tile_coord(args, gt, tile, n_ntiles, BN, split, num_kb, kTileRows);
+            const int nvalid = min(32, max(0, tc.nrows - row_off));
+            if (!mbar_wait(&tfull[b], use & 1, epi.flags)) break;
+            tc_fence_after();
+            epilogue<T, BN, KIND>(epi, tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN, stg, lane,
+                                  nvalid, tc.c_row0 + row_off, tc.n0, split, tc.mt);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if constexpr (CG == 2) mbar_arrive_cluster(tempty0 + static_cast<uint32_t>(b) * 8);
+                else mbar_arrive(&tempty[b]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if constexpr (CG == 2) cluster_sync();    // neither CTA leaves while the other may touch it
+    if (warp == 1) {
+        tc_fence_after();
+        if constexpr (CG == 2) tmem_dealloc_pair(tmem, C::TMEM_COLS);
+        else tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <typename T, int BN, int KIND, int CG>
+rdt_status launch(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap* tA2,
+                  const CUtensorMap* tB2, const GemmArgs& args, const EpiParams& epi,
+                  cudaStream_t st) {
+    using C = TcCfg<BN, CG>;
+    auto kern = gemm_tc_kernel<T, BN, KIND, CG>;
+    constexpr int kTileRows = BM * CG;
+    static int dev_ready[64] = {};         // per device: attributes set, co-resident clusters
+    static int max_clusters[64] = {};
+    int dev = 0;
+    RDT_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) {
+        set_error("gemm_tc: device index out of range");
+        return RDT_ERR_UNSUPPORTED;
+    }
+    if (!dev_ready[dev]) {
+        RDT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+        int mc = num_sms() / CG;
+        if (CG > 1) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(2 * mc);
+            cfg.blockDim = dim3(kThreads);
+            cfg.dynamicSmemBytes = C::SMEM;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = CG;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            RDT_CUDA_TRY(cudaOccupancyMaxActiveClusters(&n, kern, &cfg));
+            if (n < 1) {
+                set_error("gemm_tc: a CTA pair with this shared memory cannot be resident");
+                return RDT_ERR_UNSUPPORTED;
+            }
+            mc = std::min(mc, n);
+        }
+        max_clusters[dev] = mc;
+        dev_ready[dev] = 1;
+    }
+    const int n_ntiles = (args.N + BN - 1) / BN;
+    const long mt = args.counts ? args.max_tiles : (args.M + kTileRows - 1) / kTileRows;
+    const long total = mt * n_ntiles * (args.split_k > 1 ? args.split_k : 1);
+    if (total <= 0) return RDT_OK;
+    const int clusters = static_cast<int>(std::min<long>(total, max_clusters[dev]));
+    RDT_CUDA_TRY(launch_pdl_cluster(kern, dim3(clusters * CG), dim3(kThreads), C::SMEM, st, CG, tA, tB,
+                                    tA2 ? *tA2 : tA, tB2 ? *tB2 : tB, args, epi));
+    return RDT_OK;
+}
+
+template <typename T, int BN, int CG>
+rdt_status dispatch_kind(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap* tA2,
+                         const CUtensorMap* tB2, const GemmArgs& args, const EpiParams& epi,
+                         cudaStream_t st) {
+    switch (epi.kind) {
+        case EPI_STORE: return launch<T, BN, EPI_STORE, CG>(tA, tB, tA2, tB2, args, epi, st);
+        case EPI_STORE_F32: return launch<T, BN, EPI_STORE_F32, CG>(tA, tB, tA2, tB2, args, epi, st);
+        case EPI_ROPE: return launch<T, BN, EPI_ROPE, CG>(tA, tB, tA2, tB2, args, epi, st);
+        case EPI_OPROJ_LOOP: return launch<T, BN, EPI_OPROJ_LOOP, CG>(tA, tB, tA2, tB2, args, epi, st);
+        case EPI_OPROJ_PLAIN: return launch<T, BN, EPI_OPROJ_PLAIN, CG>(tA, tB, tA2, tB2, args, epi, st);
+        case EPI_SWIGLU: return launch<T, BN, EPI_SWIGLU, CG>(tA, tB, tA2, tB2, args, epi, st);
+        case EPI_SCATTER: return launch<T, BN, EPI_SCATTER, CG>(tA, tB, tA2, tB2, args, epi, st);
+        default: set_error("gemm_tc: unknown epilogue"); return RDT_ERR_INVALID_ARG;
+    }
+}
+
+}  // namespace
+}  // namespace rdt

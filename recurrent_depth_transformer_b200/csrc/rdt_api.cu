@@ -59,14 +59,17 @@ struct rdt_handle {
     int router_split = 1;          // K split of the router GEMM over CTAs
     float* logits = nullptr;       // [N, E] partial-logit accumulator of the split router
     int* tile_count = nullptr;     // per row-tile arrival counters of the split router
-    // output tile widths of the projection and expert GEMMs (128 or 256)
+    // output tile widths of the projection and expert GEMMs (128 or 256), and whether each
+    // runs on CTA pairs (256-row tiles) or single CTAs (128-row tiles)
     int bn_qkv = 128, bn_o = 128, bn_up = 128, bn_down = 128;
+    int pair_qkv = 0, pair_o = 0, pair_up = 0, pair_down = 0;
     int32_t* idx = nullptr;
     float* wts = nullptr;
     int cap = 0;                   // rows reserved per expert group (tokens + padding)
     int *counts = nullptr, *row_token = nullptr, *slot_row = nullptr;
     float* row_w = nullptr;
-    int max_tiles = 0;
+    int max_tiles = 0;             // grouped GEMMs: bound on 128-row tiles
+    int max_tiles_pair = 0;        // ... and on 256-row tiles
     int* flags = nullptr;
     void *stage_h0 = nullptr, *stage_e = nullptr;
     float* stage_out = nullptr;
@@ -104,6 +107,9 @@ struct rdt_handle {
 };
 
 namespace {
+
+// rows of filler after the grouped GEMMs' operand buffers (one pair tile)
+constexpr int kFillerRows = 256;
 
 // kernel classes reported by rdt_profile_read
 enum Kind { K_HOIST, K_NORM1, K_GEMM_QKV, K_GEMM_LAT, K_MLA_NORM, K_GEMM_Q, K_ATTENTION, K_LORA_DOWN,
@@ -187,6 +193,7 @@ rdt_status validate_config(const rdt_config* c) {
     if (c->expert_hidden < 64 || c->expert_hidden % 64) return uns("expert_hidden % 64 != 0");
     if (c->dtype == RDT_F32 && c->expert_hidden % 128) return uns("f32: expert_hidden % 128 != 0");
     if (c->max_loops < 1 || c->max_loops > 64) return bad("max_loops must be in [1, 64]");
+    if (c->gemm_tiles < 0 || c->gemm_tiles > 2) return bad("gemm_tiles must be 0, 1 or 2");
     if (c->b_kind != RDT_B_DIAG && c->b_kind != RDT_B_DENSE) return bad("b_kind");
     if (!(c->norm_eps >= 0.0f) || !(c->rope_base > 1.0f)) return bad("norm_eps / rope_base");
     if (c->lora_rank < 0 || c->n_lora < 0) return bad("lora");
@@ -239,23 +246,44 @@ rdt_status interleave_w13(void* dst, const void* w1, const void* w3, int hid, in
     return RDT_OK;
 }
 
-// Output tile width for a GEMM with about m_tiles row tiles and N columns. The persistent
-// grid's time is that of its busiest CTA: (tiles per CTA) x (tile time), a tile's time
-// taken as proportional to BN plus a fixed share for its pipeline fill and epilogue.
-int choose_bn(long m_tiles, int N, bool allow256) {
+// Tile shape for a GEMM with `rows` output rows (grouped: plus the partial last tile of each
+// of `groups` groups, estimated as half a tile) and N columns; mode 0 chooses, 1 forces single
+// CTAs, 2 forces CTA pairs where the shape allows them.
+//
+// Single CTAs: the persistent grid's time is that of its busiest CTA, (tiles per CTA) x (tile
+// time), a tile's time taken as proportional to BN plus a fixed share for its pipeline fill
+// and epilogue. Measured on B200 this favours 128-wide tiles whenever the grid runs more
+// than one wave. CTA pairs (256 x 256 tiles, each CTA loading half of B) load fewer bytes per
+// CTA for the same output; measured, that pays only when the whole GEMM fits in one wave of
+// pairs and its best single-CTA shape would load more per CTA, so that is when they are
+// chosen.
+struct TileChoice {
+    int bn;
+    int pair;
+};
+TileChoice choose_tiles(long rows, long groups, int N, bool allow256, bool allow_pair, int mode) {
     const long sms = num_sms();
+    const bool n256 = allow256 && N % 256 == 0;
+    if (mode == 2 && allow_pair) return {n256 ? 256 : 128, 1};
     long best_cost = -1;
-    int best = 128;
+    TileChoice best{128, 0};
+    long best_tiles = 0;
     for (int bn : {256, 128}) {
-        if (bn == 256 && (!allow256 || N % 256)) continue;
+        if (bn == 256 && !n256) continue;
         if (N % bn) continue;
-        const long tiles = m_tiles * (N / bn);
-        const long per_cta = (tiles + sms - 1) / sms;
-        const long cost = per_cta * (32 + bn);
+        const long tiles = ((rows + 127) / 128 + (groups + 1) / 2) * (N / bn);
+        const long per = (tiles + sms - 1) / sms;
+        const long cost = per * (32 + bn);
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
-            best = bn;
+            best = {bn, 0};
+            best_tiles = tiles;
         }
+    }
+    if (mode == 0 && allow_pair && n256) {
+        const long pairs = ((rows + 255) / 256 + (groups + 1) / 2) * (N / 256);
+        const bool one_wave = best_tiles <= sms && pairs <= sms / 2;
+        if (one_wave && 128 + best.bn > 128 + 128) best = {256, 1};   // bytes per CTA per K block
     }
     return best;
 }
@@ -269,9 +297,9 @@ rdt_status build_maps(rdt_handle* h) {
     const int S = c.n_shared, E = c.n_experts, hid = c.expert_hidden;
     RDT_TRY(make_tmap_2d(&h->m_xn, h->xn, bf, d, N, d * es, kbox, 128));
     RDT_TRY(make_tmap_2d(&h->m_o, h->o, bf, h->owidth, N, h->owidth * es, kbox, 128));
-    RDT_TRY(make_tmap_2d(&h->m_wo, h->wo, bf, h->owidth, d, h->owidth * es, kbox, h->bn_o));
+    RDT_TRY(make_tmap_2d(&h->m_wo, h->wo, bf, h->owidth, d, h->owidth * es, kbox, h->bn_o >> h->pair_o));
     if (c.attn_type == RDT_GQA) {
-        RDT_TRY(make_tmap_2d(&h->m_wqkv, h->wqkv, bf, d, h->nqkv, d * es, kbox, h->bn_qkv));
+        RDT_TRY(make_tmap_2d(&h->m_wqkv, h->wqkv, bf, d, h->nqkv, d * es, kbox, h->bn_qkv >> h->pair_qkv));
     } else {
         RDT_TRY(make_tmap_2d(&h->m_wlat, h->wlat, bf, d, h->lat_w, d * es, kbox, 128));
         RDT_TRY(make_tmap_2d(&h->m_cq, h->cq, bf, c.q_lora_rank, N, c.q_lora_rank * es, kbox, 128));
@@ -281,18 +309,18 @@ rdt_status build_maps(rdt_handle* h) {
         RDT_TRY(make_tmap_2d(&h->m_tq, h->tq, bf, h->kext, N, h->kext * es, kbox, 128));
         RDT_TRY(make_tmap_2d(&h->m_to, h->to, bf, h->kext, N, h->kext * es, kbox, 128));
         RDT_TRY(make_tmap_2d(&h->m_lqb, h->lqb, bf, h->kext, static_cast<uint64_t>(c.n_lora) * h->nqkv,
-                             h->kext * es, kbox, h->bn_qkv));
+                             h->kext * es, kbox, h->bn_qkv >> h->pair_qkv));
         RDT_TRY(make_tmap_2d(&h->m_lob, h->lob, bf, h->kext, static_cast<uint64_t>(c.n_lora) * d,
-                             h->kext * es, kbox, h->bn_o));
+                             h->kext * es, kbox, h->bn_o >> h->pair_o));
     }
     // capacity layout: xperm = [yn (N rows) | expert e: rows N + e N .. N + e N + N),
     // U = [shared expert s: rows s N .. | expert e: rows (S + e) N ..]
-    const uint64_t xrows = static_cast<uint64_t>(N) + static_cast<uint64_t>(h->cap) * E;
-    const uint64_t urows = static_cast<uint64_t>(h->cap) * (S + E);
+    const uint64_t xrows = static_cast<uint64_t>(N) + static_cast<uint64_t>(h->cap) * E + kFillerRows;
+    const uint64_t urows = static_cast<uint64_t>(h->cap) * (S + E) + kFillerRows;
     RDT_TRY(make_tmap_2d(&h->m_xperm, h->xperm, bf, d, xrows, d * es, kbox, 128));
-    RDT_TRY(make_tmap_2d(&h->m_w13, h->w13, bf, d, static_cast<uint64_t>(E + S) * 2 * hid, d * es, kbox, h->bn_up));
+    RDT_TRY(make_tmap_2d(&h->m_w13, h->w13, bf, d, static_cast<uint64_t>(E + S) * 2 * hid, d * es, kbox, h->bn_up >> h->pair_up));
     RDT_TRY(make_tmap_2d(&h->m_U, h->U, bf, hid, urows, hid * es, kbox, 128));
-    RDT_TRY(make_tmap_2d(&h->m_w2, h->w2, bf, hid, static_cast<uint64_t>(E + S) * d, hid * es, kbox, h->bn_down));
+    RDT_TRY(make_tmap_2d(&h->m_w2, h->w2, bf, hid, static_cast<uint64_t>(E + S) * d, hid * es, kbox, h->bn_down >> h->pair_down));
     RDT_TRY(make_tmap_2d(&h->m_ynlo, h->yn_lo, bf, d, N, d * es, kbox, 128));
     RDT_TRY(make_tmap_2d(&h->m_wr, h->wr, bf, d, E, d * es, kbox, h->bn_router));
     return RDT_OK;
@@ -394,14 +422,24 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         RDT_TRY(copy_d2d(h->rbias, w->router_bias, E * 4, st));
     }
     if (h->bf) {
-        const long mt_dense = (N + 127) / 128;
-        const long mt_group = (static_cast<long>(N) * (K + S) + 127) / 128 + (E + S + 1) / 2;
-        h->bn_up = choose_bn(mt_group, 2 * hid, hid % 128 == 0);
-        h->bn_down = choose_bn(mt_group, d, true);
-        h->bn_o = choose_bn(mt_dense, d, true);
+        const long grows = static_cast<long>(N) * (K + S);
+        const int mode = c.gemm_tiles;
+        // SwiGLU tiles hold BN/2 gate and BN/2 up columns; W1/W3 are interleaved in blocks
+        // of BN/2 rows, which must divide the hidden width
+        TileChoice t = choose_tiles(grows, E + S, 2 * hid, hid % 128 == 0, hid % 64 == 0, mode);
+        h->bn_up = t.bn;
+        h->pair_up = t.pair;
+        t = choose_tiles(grows, E + S, d, true, true, mode);
+        h->bn_down = t.bn;
+        h->pair_down = t.pair;
+        t = choose_tiles(N, 0, d, true, true, mode);
+        h->bn_o = t.bn;
+        h->pair_o = t.pair;
         if (c.attn_type == RDT_GQA) {
             const int nqkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
-            h->bn_qkv = choose_bn(mt_dense, nqkv, nqkv % 256 == 0);
+            t = choose_tiles(N, 0, nqkv, nqkv % 256 == 0, true, mode);
+            h->bn_qkv = t.bn;
+            h->pair_qkv = t.pair;
         }
     }
     const size_t wexp = static_cast<size_t>(hid) * d * es;   // one expert matrix
@@ -535,8 +573,11 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
     // and masked in its epilogue. They hold a non-zero filler (bytes 0x3F: 0.746 in bf16):
     // measured on B200, tiles whose padding rows are exact zeros run the grouped GEMMs
     // 1.6-1.8x slower than tiles padded with any non-zero value.
-    RDT_TRY(dev_alloc(h, &h->xperm, (static_cast<size_t>(N) + static_cast<size_t>(h->cap) * E) * d * es, true, 0x3F));
-    RDT_TRY(dev_alloc(h, &h->U, static_cast<size_t>(h->cap) * (S + E) * hid * es, true, 0x3F));
+    // The last group's last tile may reach up to 255 rows past its group: kFillerRows more
+    // rows of filler keep those reads inside the buffers (no zero fill from out-of-range TMA).
+    RDT_TRY(dev_alloc(h, &h->xperm, (static_cast<size_t>(N) + static_cast<size_t>(h->cap) * E + kFillerRows) * d * es,
+                      true, 0x3F));
+    RDT_TRY(dev_alloc(h, &h->U, (static_cast<size_t>(h->cap) * (S + E) + kFillerRows) * hid * es, true, 0x3F));
     RDT_TRY(dev_alloc(h, &h->yn_lo, nd * es, true));
     h->bn_router = E <= 64 ? 64 : E <= 128 ? 128 : 256;
     if (h->bf) {
@@ -557,6 +598,7 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
     RDT_TRY(dev_alloc(h, &h->row_w, static_cast<size_t>(h->cap) * E * 4, true));
     RDT_TRY(dev_alloc(h, &h->slot_row, static_cast<size_t>(N) * K * 4, true));
     h->max_tiles = (N * K + 127) / 128 + E + S * ((N + 127) / 128);
+    h->max_tiles_pair = (N * K + 255) / 256 + E + S * ((N + 255) / 256);
     RDT_TRY(dev_alloc(h, &h->flags, FLAG_COUNT * 4, true));
     RDT_TRY(dev_alloc(h, &h->stage_h0, nd * es));
     RDT_TRY(dev_alloc(h, &h->stage_e, nd * es));
@@ -612,6 +654,7 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         ga.kb_main = static_cast<int>(d * h->esz / 128);
         ga.kb_ext = lora ? 1 : 0;
         ga.b2_row0 = li * h->nqkv;
+        ga.pair = h->pair_qkv;
         ep.kind = EPI_ROPE;
         ep.out = h->qkv;
         ep.ldo = h->nqkv;
@@ -711,6 +754,7 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
     go.kb_main = static_cast<int>(h->owidth * h->esz / 128);
     go.kb_ext = lora ? 1 : 0;
     go.b2_row0 = li * d;
+    go.pair = h->pair_o;
     go.flags = h->flags;
     EpiParams eo{};
     eo.flags = h->flags;
@@ -768,6 +812,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
         ra.xperm = h->xperm;
         ra.a_routed_base = N;
         ra.store_yn = c.n_shared > 0;          // shared experts read yn itself
+        ra.weights_static = 1;                 // the library's own copy, written at create
         TIMED(h, K_ROUTER, 1, st, norm2_router_smem(h->bf, ra, st));
         copies_written = true;
     } else if (!h->bf) {
@@ -847,7 +892,8 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     gu.n_shared = c.n_shared;
     gu.cap = h->cap;
     gu.a_routed_base = N;
-    gu.max_tiles = h->max_tiles;
+    gu.pair = h->pair_up;
+    gu.max_tiles = h->pair_up ? h->max_tiles_pair : h->max_tiles;
     gu.flags = h->flags;
     EpiParams eu{};
     eu.kind = EPI_SWIGLU;
@@ -866,7 +912,8 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     gd.n_shared = c.n_shared;
     gd.cap = h->cap;
     gd.a_routed_base = N;
-    gd.max_tiles = h->max_tiles;
+    gd.pair = h->pair_down;
+    gd.max_tiles = h->pair_down ? h->max_tiles_pair : h->max_tiles;
     gd.a_from_c = 1;
     gd.flags = h->flags;
     EpiParams ed{};

@@ -97,20 +97,34 @@ __device__ __forceinline__ void pdl_trigger() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// cluster_x > 1 launches clusters of that many consecutive CTAs.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                       Args&&... args) {
+cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                               cudaStream_t st, int cluster_x, Args&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    int n = 1;
+    if (cluster_x > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        n = 2;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = n;
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+    return launch_pdl_cluster(kern, grid, block, smem, st, 1, std::forward<Args>(args)...);
 }
 
 int num_sms();   // SM count of the current device (cached)
@@ -175,6 +189,40 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
+// ------------------------------------------------------------------ clusters (CTA pairs)
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Shared-window address of the same variable in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+// All threads of every CTA in the cluster; release/acquire orders shared-memory traffic.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+// Arrive on a barrier given by its cluster address (default semantics: release, CTA scope;
+// the arrivals here only order tcgen05 reads already waited for, not memory traffic).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// 2-D tiled load into this CTA's shared memory whose completion is counted on a barrier of
+// either CTA of the pair (given by its cluster address). Not a multicast: one destination.
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* m, uint32_t bar,
+                                                 int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05 (5th-gen tensor cores)
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_slot, uint32_t ncols) {
@@ -203,6 +251,43 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
             smem_u32(bar))
         : "memory");
 }
+// CTA-pair forms (cta_group::2): allocation and release are issued by the same warp of both
+// CTAs of the pair; the MMA by one thread of the even CTA, reading A and B from both CTAs'
+// shared memory at the same offsets and accumulating into both CTAs' TMEM.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(smem_slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+// Arrive on the barrier at this shared offset in every CTA of `cta_mask` once the pair's
+// prior tcgen05 operations issued by this thread have completed.
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8, %9, %10, %11, %12}, p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0), "r"(0),
+        "r"(0), "r"(0), "r"(0)
+        : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, both K-major; kind::f16 (bf16 inputs, fp32 accumulate).
 __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                             uint32_t idesc, uint32_t accumulate) {
@@ -357,17 +442,23 @@ struct GemmArgs {
     int n_routed, n_shared;// grouped: routed groups, then shared groups (n_rows = cap each)
     int cap;               // grouped: rows reserved per group (>= tokens; the group stride)
     int a_routed_base;     // grouped: first A row of routed group 0 (shared groups read rows 0..cap)
-    int max_tiles;         // grouped: upper bound on the 128-row tiles (grid sizing)
+    int max_tiles;         // grouped: upper bound on the row tiles (128 or 256 rows; grid sizing)
     int a_from_c;          // grouped: read A at the tile's output row (down projection)
     int split_k;           // > 1: K blocks split over that many CTAs per output tile (router)
+    int pair;              // 1: CTA-pair tiles of 256 rows (cta_group::2); 0: one CTA, 128 rows
     int* flags;
 };
 
 // C = A B^T (+ extension) with the chosen epilogue, on tcgen05 tensor cores.
-// tA: [rows, K] box (128 B x 128 rows); tB: [Nrows, K] box (128 B x BN rows).
+// tA: [rows, K] box (128 B x 128 rows); tB: [Nrows, K] box (128 B x BN rows, or BN/2 rows
+// for pair tiles, where each CTA of the pair loads half of the tile's B rows).
 rdt_status gemm_tc(bool bf16_elems, int bn, const CUtensorMap& tA, const CUtensorMap& tB,
                    const CUtensorMap* tA2, const CUtensorMap* tB2, const GemmArgs& args,
                    const EpiParams& epi, cudaStream_t st);
+// The pair-tile instantiations (bf16, BN 128 or 256, every epilogue but the router's).
+rdt_status gemm_tc_pair(int bn, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap* tA2,
+                        const CUtensorMap* tB2, const GemmArgs& args, const EpiParams& epi,
+                        cudaStream_t st);
 
 // Causal attention. q rows [N, ldq], head h at column h*q_hstride; k/v similarly with
 // Hkv heads; o [N, ldo] head h at column h*dv.
@@ -416,10 +507,13 @@ struct RouterArgs {
     int* row_token; float* row_w; int* slot_row; int cap;
     void* xperm; int a_routed_base;   // fused router: write yn into the claimed rows here
     int store_yn;                      // fused router: also write yn at row `row` of yn
+    int weights_static;                // fused router: w_router is not written by the previous
+                                       // kernel in the stream (staged before waiting on it)
 };
 rdt_status norm2_router(bool bf16_elems, const RouterArgs& a, cudaStream_t st);
-// RMSNorm2 fused with the fp32 router when W_r (n_exp x dim) fits in 64 KB of shared memory,
-// n_exp <= 64, top_k <= 8 and dim is 128, 1024 or 2048
+// RMSNorm2 fused with the fp32 router when W_r (n_exp x dim, element type) takes at most
+// 64 KB (staged as fp32 in up to 128 KB of shared memory), n_exp <= 64, top_k <= 8 and dim is
+// 128, 1024 or 2048
 bool router_fits_smem(bool bf16_elems, int n_exp, int top_k, int dim);
 rdt_status norm2_router_smem(bool bf16_elems, const RouterArgs& a, cudaStream_t st);
 

@@ -1,9 +1,10 @@
 // RMSNorm2 fused with the MoE router for routers whose weight fits in shared memory:
-// each block stages W_r (n_experts x dim) once, then every warp takes one row: RMSNorm2 in
-// fp32 (stored in the element type as the experts' input), the n_experts logits of the fp32
-// normalised row, top-k of logits + bias with ties to the lower expert index, softmax over
-// the k chosen logits, per-expert histogram.
+// each block stages W_r (n_experts x dim) once as fp32, then every warp takes rows in turn:
+// RMSNorm2 in fp32 (stored in the element type as the experts' input), the n_experts logits
+// of the fp32 normalised row, top-k of logits + bias with ties to the lower expert index,
+// softmax over the k chosen logits, per-expert histogram.
 #include <algorithm>
+#include <type_traits>
 
 #include "rdt_internal.cuh"
 
@@ -12,107 +13,215 @@ namespace {
 
 // ----------------------------------------------------------------------------- norm2 + router (W_r in shared memory)
 
-// For routers whose weight fits in shared memory: each block stages W_r once, then every
-// warp takes rows in turn: RMSNorm2 (fp32, stored in the element type for the experts), the
-// n_exp logits of the fp32 row against W_r, top-k of logits + bias (ties to the lower expert
-// index), softmax over the k chosen logits, histogram.
-constexpr int kRouterThreads = 512;   // 16 rows in flight per staged copy of W_r
+// For routers whose weight fits in shared memory: each block stages W_r once, as fp32, then
+// every warp takes rows in turn: RMSNorm2 (fp32, stored in the element type for the experts),
+// the n_exp logits of the fp32 row against W_r, top-k of logits + bias (ties to the lower
+// expert index), softmax over the k chosen logits, histogram, and the row's copies for the
+// chosen experts.
+//
+// The work per row is a few hundred instructions, so the kernel is bound by instruction
+// issue and latency, not bytes: each lane owns 4 * NV columns of the row, forms its partial
+// logits with packed fp32 FMAs from 16-byte shared loads, and the warp reduces the EMAX
+// partials with a transposing butterfly (EMAX - 1 + 1 shuffles instead of 5 per logit) that
+// leaves lane l holding whole logits (expert l / 2 for 16 experts, experts 2l, 2l + 1 for 64).
+// Top-k is then k warp-wide argmax rounds over (score desc, index asc).
+constexpr int kRouterMaxThreads = 512;
+
+// Butterfly transpose-reduce of v[0..E) over the warp. On return v[0 .. max(E/32, 1)) hold
+// full sums; router_expert() gives their expert indices.
+template <int E>
+__device__ __forceinline__ void transpose_reduce(float (&v)[E], int lane) {
+    int n = E;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        if (n > 1) {
+            const int half = n / 2;
+            const bool up = (lane & off) != 0;
+#pragma unroll
+            for (int j = 0; j < E / 2; ++j) {
+                if (j < half) {
+                    const float send = up ? v[j] : v[j + half];
+                    const float keep = up ? v[j + half] : v[j];
+                    v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                }
+            }
+            n = half;
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+        }
+    }
+}
+// Expert index of v[j] after transpose_reduce<E>.
+template <int E>
+__device__ __forceinline__ int router_expert(int lane, int j) {
+    int e = j, n = E;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        if (n > 1) {
+            n /= 2;
+            if (lane & off) e += n;
+        }
+    }
+    return e;
+}
+
+// (score, index) order: higher score first, then lower index; invalid entries last.
+__device__ __forceinline__ bool router_better(float s, int e, float so, int eo) {
+    return s > so || (s == so && e < eo);
+}
 
 template <typename T, int NV, int EMAX, int KMAX>
-__global__ void __launch_bounds__(kRouterThreads) norm2_router_smem_kernel(const RouterArgs a) {
-    extern __shared__ __align__(16) uint8_t smem_w[];
-    T* Ws = reinterpret_cast<T*>(smem_w);
-    pdl_trigger();
-    pdl_wait();
-    {
-        const int nvec = a.n_exp * a.dim * static_cast<int>(sizeof(T)) / 16;
-        const uint4* src = static_cast<const uint4*>(a.w_router);
-        uint4* dst = reinterpret_cast<uint4*>(smem_w);
-        for (int i = threadIdx.x; i < nvec; i += blockDim.x) dst[i] = src[i];
-    }
-    __syncthreads();
+__global__ void __launch_bounds__(kRouterMaxThreads) norm2_router_smem_kernel(const RouterArgs a) {
+    extern __shared__ __align__(16) float Ws[];     // [n_exp][dim] fp32
+    constexpr int NL = EMAX >= 32 ? EMAX / 32 : 1;  // logits held per lane after the reduce
     const int lane = threadIdx.x & 31;
-    const int warps_total = gridDim.x * (kRouterThreads / 32);
+    const int nthreads = blockDim.x;
+    auto stage = [&]() {
+        const int n8 = a.n_exp * a.dim / 8;
+        for (int i = threadIdx.x; i < n8; i += nthreads) {
+            float f[8];
+            if constexpr (std::is_same<T, bf16>::value) {
+                const uint4 x = static_cast<const uint4*>(a.w_router)[i];
+                const uint32_t u[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[j]));
+                    f[2 * j] = t.x;
+                    f[2 * j + 1] = t.y;
+                }
+            } else {
+                const float4 x0 = static_cast<const float4*>(a.w_router)[2 * i];
+                const float4 x1 = static_cast<const float4*>(a.w_router)[2 * i + 1];
+                f[0] = x0.x; f[1] = x0.y; f[2] = x0.z; f[3] = x0.w;
+                f[4] = x1.x; f[5] = x1.y; f[6] = x1.z; f[7] = x1.w;
+            }
+            reinterpret_cast<float4*>(Ws)[2 * i] = make_float4(f[0], f[1], f[2], f[3]);
+            reinterpret_cast<float4*>(Ws)[2 * i + 1] = make_float4(f[4], f[5], f[6], f[7]);
+        }
+    };
+    pdl_trigger();
+    if (a.weights_static) stage();      // overlaps the tail of the previous kernel
+    pdl_wait();
+    if (!a.weights_static) stage();
+    __syncthreads();
+    const int warps_total = gridDim.x * (nthreads / 32);
+    float bias_l[NL];
+    int ex_l[NL];
+#pragma unroll
+    for (int j = 0; j < NL; ++j) {
+        ex_l[j] = router_expert<EMAX>(lane, j);
+        bias_l[j] = (a.bias && ex_l[j] < a.n_exp) ? a.bias[ex_l[j]] : 0.0f;
+    }
+    // gamma stays in registers when they allow it (128 per thread at 512 threads)
+    constexpr bool kHoistGamma = NV * 4 + EMAX <= 64;
+    float g[kHoistGamma ? NV : 1][4];
+    if constexpr (kHoistGamma) {
+#pragma unroll
+        for (int i = 0; i < NV; ++i) load4(a.gamma + i * 128 + lane * 4, g[i]);
+    }
 #pragma unroll 1
-    for (int row = blockIdx.x * (kRouterThreads / 32) + (threadIdx.x >> 5); row < a.ntok; row += warps_total) {
+    for (int row = blockIdx.x * (nthreads / 32) + (threadIdx.x >> 5); row < a.ntok; row += warps_total) {
         const size_t base = static_cast<size_t>(row) * a.dim;
         float y[NV][4];
         float ss = 0.0f;
 #pragma unroll
-        for (int i = 0; i < NV; ++i) {
-            load4(a.y + base + i * 128 + lane * 4, y[i]);
+        for (int i = 0; i < NV; ++i) load4(a.y + base + i * 128 + lane * 4, y[i]);
+#pragma unroll
+        for (int i = 0; i < NV; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j) ss = fmaf(y[i][j], y[i][j], ss);
-        }
         ss = warp_sum(ss);
         const float inv = rsqrtf(ss / a.dim + a.eps);
         T* yn = static_cast<T*>(a.yn) + base;
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
-            const int col = i * 128 + lane * 4;
-            float g[4];
-            load4(a.gamma + col, g);
+            float gi[4];
+            if constexpr (kHoistGamma) {
+                gi[0] = g[i][0]; gi[1] = g[i][1]; gi[2] = g[i][2]; gi[3] = g[i][3];
+            } else {
+                load4(a.gamma + i * 128 + lane * 4, gi);
+            }
 #pragma unroll
-            for (int j = 0; j < 4; ++j) y[i][j] *= inv * g[j];
-            if (a.store_yn) store4(yn + col, y[i]);   // element-type copy; the router keeps fp32
+            for (int j = 0; j < 4; ++j) y[i][j] *= inv * gi[j];
+            if (a.store_yn) store4(yn + i * 128 + lane * 4, y[i]);   // element-type copy; logits use fp32
         }
         float lg[EMAX];
 #pragma unroll
         for (int e = 0; e < EMAX; ++e) {
-            float p = 0.0f;
+            float2 acc = make_float2(0.0f, 0.0f);
             if (e < a.n_exp) {
+                const float4* wrow = reinterpret_cast<const float4*>(Ws + static_cast<size_t>(e) * a.dim) + lane;
 #pragma unroll
                 for (int i = 0; i < NV; ++i) {
-                    float w[4];
-                    load4(Ws + static_cast<size_t>(e) * a.dim + i * 128 + lane * 4, w);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) p = fmaf(y[i][j], w[j], p);
+                    const float4 w = wrow[i * 32];
+                    acc = __ffma2_rn(make_float2(y[i][0], y[i][1]), make_float2(w.x, w.y), acc);
+                    acc = __ffma2_rn(make_float2(y[i][2], y[i][3]), make_float2(w.z, w.w), acc);
                 }
             }
-            lg[e] = p;
+            lg[e] = acc.x + acc.y;
         }
+        transpose_reduce<EMAX>(lg, lane);
+        // this lane's candidates: score = logit + bias, NaN scores rank below every number
+        float sc[NL];
+        bool taken[NL];
 #pragma unroll
-        for (int e = 0; e < EMAX; ++e) lg[e] = warp_sum(lg[e]);   // every lane holds every logit
-        // top-k by (score desc, index asc), kept sorted in registers (lane-redundant)
-        float bs[KMAX], bl[KMAX];
-        int bi[KMAX];
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            bs[j] = -INFINITY;
-            bl[j] = 0.0f;
-            bi[j] = -1;
+        for (int j = 0; j < NL; ++j) {
+            const float s = lg[j] + bias_l[j];
+            sc[j] = (ex_l[j] < a.n_exp && !isnan(s)) ? s : -INFINITY;
+            taken[j] = ex_l[j] >= a.n_exp;
         }
+        int ci[KMAX];
+        float cl[KMAX];
 #pragma unroll
-        for (int e = 0; e < EMAX; ++e) {
-            if (e >= a.n_exp) break;
-            float cs = lg[e] + (a.bias ? a.bias[e] : 0.0f), cl = lg[e];
-            int ci = e;
+        for (int r = 0; r < KMAX; ++r) {
+            if (r >= a.top_k) break;
+            // lane-local best untaken candidate, then the warp's best
+            float bs = -INFINITY;
+            int be = 0x7fffffff;
 #pragma unroll
-            for (int j = 0; j < KMAX; ++j) {
-                if (j < a.top_k && cs > bs[j]) {
-                    const float ts = bs[j], tl = bl[j];
-                    const int ti = bi[j];
-                    bs[j] = cs; bl[j] = cl; bi[j] = ci;
-                    cs = ts; cl = tl; ci = ti;
+            for (int j = 0; j < NL; ++j)
+                if (!taken[j] && router_better(sc[j], ex_l[j], bs, be)) {
+                    bs = sc[j];
+                    be = ex_l[j];
+                }
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) {
+                const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                if (router_better(os, oe, bs, be)) {
+                    bs = os;
+                    be = oe;
                 }
             }
+            if (be >= a.n_exp) be = 0;                 // only if every expert was taken (k > E)
+            float l = 0.0f;
+#pragma unroll
+            for (int j = 0; j < NL; ++j)
+                if (ex_l[j] == be) {
+                    taken[j] = true;
+                    l = lg[j];
+                }
+            // the logit of the winner from a lane that holds it
+            const int owner = EMAX >= 32 ? be / NL : 2 * be;
+            ci[r] = be;
+            cl[r] = __shfl_sync(0xffffffffu, l, owner & 31);
         }
         float mx = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j)
-            if (j < a.top_k && bi[j] >= 0) mx = fmaxf(mx, bl[j]);
+        for (int r = 0; r < KMAX; ++r)
+            if (r < a.top_k) mx = fmaxf(mx, cl[r]);
         float den = 0.0f;
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j)
-            if (j < a.top_k && bi[j] >= 0) den += expf(bl[j] - mx);
+        for (int r = 0; r < KMAX; ++r)
+            if (r < a.top_k) den += expf(cl[r] - mx);
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            if (j >= a.top_k) break;
+        for (int r = 0; r < KMAX; ++r) {
+            if (r >= a.top_k) break;
             int rr = 0;
-            if (lane == j) {
-                const int e = bi[j] < 0 ? 0 : bi[j];
-                const float wv = bi[j] < 0 ? 0.0f : expf(bl[j] - mx) / den;
-                const size_t o = static_cast<size_t>(row) * a.top_k + j;
+            if (lane == r) {
+                const int e = ci[r];
+                const float wv = expf(cl[r] - mx) / den;
+                const size_t o = static_cast<size_t>(row) * a.top_k + r;
                 a.idx[o] = e;
                 a.w[o] = wv;
                 if (a.trace_idx) a.trace_idx[o] = e;
@@ -125,7 +234,7 @@ __global__ void __launch_bounds__(kRouterThreads) norm2_router_smem_kernel(const
                 }
             }
             if (a.xperm) {                                       // the expert's copy of yn
-                rr = __shfl_sync(0xffffffffu, rr, j);
+                rr = __shfl_sync(0xffffffffu, rr, r);
                 T* dst = static_cast<T*>(a.xperm) + static_cast<size_t>(a.a_routed_base + rr) * a.dim;
 #pragma unroll
                 for (int i = 0; i < NV; ++i) store4(dst + i * 128 + lane * 4, y[i]);
@@ -143,14 +252,17 @@ bool router_fits_smem(bool bf, int n_exp, int top_k, int dim) {
 
 namespace {
 
+// One block per SM at most (each stages W_r), with enough warps that every SM gets a block
+// and every warp about one row per pass: 4..16 warps per block, rows strided over the grid.
 template <typename T, int NV, int EMAX, int KMAX>
 rdt_status launch_router_smem_k(const RouterArgs& a, cudaStream_t st) {
-    const size_t smem = static_cast<size_t>(a.n_exp) * a.dim * sizeof(T);
-    const int rows_per_block = kRouterThreads / 32;
-    const int grid = (a.ntok + rows_per_block - 1) / rows_per_block;
+    const size_t smem = static_cast<size_t>(a.n_exp) * a.dim * 4;
+    const int sms = num_sms();
+    const int warps = std::min(16, std::max(4, (a.ntok + sms - 1) / sms));
+    const int grid = std::min(sms, (a.ntok + warps - 1) / warps);
     auto k = norm2_router_smem_kernel<T, NV, EMAX, KMAX>;
-    RDT_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
-    RDT_CUDA_TRY(launch_pdl(k, dim3(grid), dim3(kRouterThreads), smem, st, a));
+    RDT_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024));
+    RDT_CUDA_TRY(launch_pdl(k, dim3(grid), dim3(warps * 32), smem, st, a));
     return RDT_OK;
 }
 
@@ -160,10 +272,19 @@ rdt_status launch_router_smem_e(const RouterArgs& a, cudaStream_t st) {
     return launch_router_smem_k<T, NV, EMAX, 8>(a, st);
 }
 
+// Only the expert-count classes that router_fits_smem admits at this width are built.
 template <typename T, int NV>
 rdt_status launch_router_smem(const RouterArgs& a, cudaStream_t st) {
+    constexpr long kRow = 128L * NV * static_cast<long>(sizeof(T));   // bytes of one W_r row
     if (a.n_exp <= 16) return launch_router_smem_e<T, NV, 16>(a, st);
-    return launch_router_smem_e<T, NV, 64>(a, st);
+    if constexpr (17 * kRow <= 64 * 1024) {
+        if (a.n_exp <= 32) return launch_router_smem_e<T, NV, 32>(a, st);
+    }
+    if constexpr (33 * kRow <= 64 * 1024) {
+        if (a.n_exp <= 64) return launch_router_smem_e<T, NV, 64>(a, st);
+    }
+    set_error("router: expert count does not fit the shared-memory router");
+    return RDT_ERR_UNSUPPORTED;
 }
 
 }  // namespace

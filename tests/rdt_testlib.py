@@ -16,10 +16,10 @@ def torch_mod():
     return torch
 
 
-def handle(wl: Workload, inputs, max_loops: int = 16):
+def handle(wl: Workload, inputs, max_loops: int = 16, gemm_tiles: int = 0):
     import recurrent_depth_transformer_b200 as R
     w = R.device_weights(inputs, wl.dtype == "bf16")
-    return R.RDT(R.make_config(wl, max_loops=max_loops), w)
+    return R.RDT(R.make_config(wl, max_loops=max_loops, gemm_tiles=gemm_tiles), w)
 
 
 def act(wl: Workload, arr):
@@ -31,12 +31,13 @@ def act(wl: Workload, arr):
     return t.cuda()
 
 
-def run_loop(wl: Workload, inputs, T: int, trace: bool = True, traj: bool = False, h=None):
+def run_loop(wl: Workload, inputs, T: int, trace: bool = True, traj: bool = False, h=None,
+             gemm_tiles: int = 0):
     """Run rdt_loop_forward; returns (h_T [B,S,d] fp32, idx [T,N,k], w [T,N,k], traj or None)."""
     torch = torch_mod()
     own = h is None
     if own:
-        h = handle(wl, inputs, max_loops=max(T, 1))
+        h = handle(wl, inputs, max_loops=max(T, 1), gemm_tiles=gemm_tiles)
     N = wl.batch * wl.seq
     idx = torch.full((max(T, 1), N, wl.top_k), -1, dtype=torch.int32, device="cuda") if trace else None
     wts = torch.zeros((max(T, 1), N, wl.top_k), dtype=torch.float32, device="cuda") if trace else None

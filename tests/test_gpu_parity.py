@@ -44,6 +44,21 @@ def test_loop_matches_oracle_small(name):
     assert_close(got, want, what=name)
 
 
+@pytest.mark.parametrize("tiles", [1, 2])
+@pytest.mark.parametrize("name", ["gqa-s200", "mla-s136", "widemoe-s192", "long-lora-s320"])
+def test_gemm_tile_modes_match_oracle(name, tiles):
+    """The projection and expert GEMMs forced onto single-CTA 128-row tiles (1) or CTA-pair
+    256-row tiles (2): both must match the oracle; the ragged sizes leave partial pair tiles
+    in the dense GEMMs and in every expert group."""
+    wl = SMALL[name]
+    inputs = generate(wl)
+    got, idx, _, _, diag = run_loop(wl, inputs, 2, gemm_tiles=tiles)
+    assert diag["nonfinite"] == 0 and diag["timeout"] == 0
+    want, mism, _, _ = oracle_follow(wl, inputs, 2, idx)
+    assert mism == 0, f"{mism} routing differences outside near-ties"
+    assert_close(got, want, what=f"{name} tiles={tiles}")
+
+
 def test_zero_block_is_closed_form():
     # every block weight zero: h_T = A^T h0 + (1 - A^T)/(1 - A) B e exactly (fp32 state)
     wl = C1.replace(batch=2, seq=64)
