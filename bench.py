@@ -53,15 +53,21 @@ def kernel_work(wl, T):
     w["gemm_qkv"] = dict(flops=2.0 * N * d * nqkv, bytes=b2 * (N * d + nqkv * d + N * nqkv), bound="tensor")
     pairs = wl.batch * wl.seq * (wl.seq + 1) / 2
     w["attention"] = dict(flops=4.0 * hq * dh * pairs, bytes=b2 * N * (nqkv + hq * dh), bound="tensor")
-    w["gemm_o"] = dict(flops=2.0 * N * hq * dh * d, bytes=b2 * (N * hq * dh + d * hq * dh) + 4 * 5 * N * d,
+    # the O projection completes y = x + a and h_next = A h + B e + a with two fp32 reductions
+    w["gemm_o"] = dict(flops=2.0 * N * hq * dh * d, bytes=b2 * (N * hq * dh + d * hq * dh) + 4 * 2 * N * d,
                        bound="tensor")
     w["gemm_up"] = dict(flops=2.0 * rows * d * 2 * hid, bytes=b2 * (rows * d + (E + S) * 2 * hid * d + rows * hid),
                         bound="tensor")
     w["gemm_down"] = dict(flops=2.0 * rows * hid * d, bytes=b2 * (rows * hid + (E + S) * d * hid) + 4 * N * d * 2,
                           bound="tensor")
-    w["norm1"] = dict(flops=0.0, bytes=N * d * (4 + b2 + b2), bound="hbm")
-    # RMSNorm2 fused with the fp32 router (W_r staged in shared memory): y in, yn and routing out
-    w["router_topk"] = dict(flops=2.0 * N * d * E, bytes=N * d * (4 + b2) + E * d * b2 + N * k * 8, bound="hbm")
+    # RMSNorm1 reads h, e, B e and writes xn, y = x and h_next = A h + B e
+    w["norm1"] = dict(flops=0.0, bytes=N * d * (4 + b2 + 4 + b2 + 4 + 4), bound="hbm")
+    # RMSNorm2 fused with the fp32 router and the dispatch (W_r staged in shared memory): y in;
+    # per (token, slot) the routing (index, weight, row token, row weight) and the yn copy in
+    # the expert's rows; yn itself only when shared experts read it
+    w["router_topk"] = dict(flops=2.0 * N * d * E,
+                            bytes=N * d * 4 + (N * d * b2 if S else 0) + E * d * b2 + N * k * (d * b2 + 16),
+                            bound="hbm")
     w["moe_dispatch"] = dict(flops=0.0, bytes=N * k * (d * b2 * 2 + 16), bound="hbm")
     w["hoist"] = dict(flops=0.0, bytes=N * d * (b2 + b2 + 4 + 4), bound="hbm")
     w["check_finite"] = dict(flops=0.0, bytes=N * d * 4, bound="hbm")
@@ -87,7 +93,7 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- clocks
 
-CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+CLOCK_FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
@@ -104,12 +110,12 @@ class ClockSampler:
             os.close(fd)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, window=None):
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -118,27 +124,46 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.f.close()
-        return parse_clocks(open(self.path).read())
+        return parse_clocks(open(self.path).read(), window)
 
 
-def parse_clocks(text):
-    sm, mx, reasons = [], [], set()
+def _stamp(text):
+    """nvidia-smi timestamp ('2026/12/02 19:04:21.123', host local time) -> epoch seconds."""
+    import datetime
+    for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+        try:
+            return datetime.datetime.strptime(text, fmt).timestamp()
+        except ValueError:
+            pass
+    return None
+
+
+def parse_clocks(text, window=None):
+    """Median SM clock and the throttle reasons seen. With window = (t0, t1) (host epoch
+    seconds of the timed region) only the samples taken inside it count, unless none was."""
+    rows = []
     for line in text.strip().splitlines():
         parts = [p.strip() for p in line.split(",")]
-        if len(parts) < 9:
+        if len(parts) < 10:
             continue
         try:
-            sm.append(float(parts[1]))
-            mx.append(float(parts[2]))
+            rows.append((_stamp(parts[0]), float(parts[2]), float(parts[3]), parts[6:10]))
         except ValueError:
             continue
-        for name, val in zip(REASONS, parts[5:9]):
+    if window is not None:
+        inside = [r for r in rows if r[0] is not None and window[0] <= r[0] <= window[1]]
+        if inside:
+            rows = inside
+    if not rows:
+        return None
+    reasons = set()
+    for r in rows:
+        for name, val in zip(REASONS, r[3]):
             if val.lower() == "active":
                 reasons.add(name)
-    if not sm:
-        return None
-    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-            "samples": len(sm)}
+    return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": max(r[2] for r in rows),
+            "reasons": sorted(reasons), "samples": len(rows), "in_timed_region": window is not None and
+            any(window[0] <= (r[0] or 0) <= window[1] for r in rows)}
 
 
 # ----------------------------------------------------------------------------- distributed plumbing
@@ -279,16 +304,18 @@ def run_gpu(args):
     torch.cuda.synchronize()
     launches0 = h.launch_count()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_wall0 = time.time()
     for a, b in evs:
         flush.zero_()
         a.record(stream)
         step()
         b.record(stream)
     torch.cuda.synchronize()
+    t_wall1 = time.time()
     if world > 1:
         dist.barrier()
     launches = h.launch_count() - launches0
-    clocks = sampler.stop() if sampler else None
+    clocks = sampler.stop((t_wall0, t_wall1)) if sampler else None
     ms_rank = sum(a.elapsed_time(b) for a, b in evs) / args.steps
     ms_all = reduce_max(ms_rank, dev)
     value, ms = aggregate([ms_all], N, LOOPS, world)
@@ -387,7 +414,7 @@ def run_gpu(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

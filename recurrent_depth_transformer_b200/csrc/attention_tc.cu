@@ -73,6 +73,7 @@ struct AttnCfg {
 
 struct AttnTcArgs {
     int seq, hq, hkv, q_hstride, k_hstride, v_hstride, ldo, dv_out;
+    int nqb, batch, sms;   // query blocks per sequence; sequences; SMs (first-round CTA slots)
     float scale_log2;
     void* o;
     int* flags;
@@ -105,9 +106,17 @@ __global__ void __launch_bounds__(192, 2)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int qb = gridDim.x - 1 - blockIdx.x;        // longest rows first
-    const int h = blockIdx.y;
-    const int b = blockIdx.z;
+    // Work items ranked by cost, heaviest (last query block: most keys) first. CTAs start in
+    // launch order, one per SM and then a second one per SM; when the grid needs more than
+    // one CTA per SM but fits two, the CTA in position S + i takes the lightest item left,
+    // so that an SM pairs a long query block with a short one instead of two long ones.
+    const int W = a.nqb * a.hq * a.batch;
+    const int L = blockIdx.x;
+    const int rank = (W > a.sms && W <= 2 * a.sms && L >= a.sms) ? W - 1 - (L - a.sms) : L;
+    const int per_qb = a.hq * a.batch;
+    const int qb = a.nqb - 1 - rank / per_qb;
+    const int h = (rank % per_qb) % a.hq;
+    const int b = (rank % per_qb) / a.hq;
     const int g = (h * a.hkv) / a.hq;
     const int q0 = qb * kBQ;
     const int row0 = b * a.seq;                        // first token row of this sequence
@@ -374,7 +383,10 @@ rdt_status launch_tc(const AttnArgs& a, cudaStream_t st) {
     ta.scale_log2 = a.scale * 1.4426950408889634f;
     ta.o = a.o;
     ta.flags = a.flags;
-    const dim3 grid((a.seq + kBQ - 1) / kBQ, a.hq, a.batch);
+    ta.nqb = (a.seq + kBQ - 1) / kBQ;
+    ta.batch = a.batch;
+    ta.sms = num_sms();
+    const dim3 grid(static_cast<unsigned>(ta.nqb) * a.hq * a.batch);
     RDT_CUDA_TRY(launch_pdl(kern, grid, dim3(192), C::SMEM, st, tq, tk, tv, ta));
     return RDT_OK;
 }

@@ -20,8 +20,9 @@
 //
 // The fused epilogues are where the block's element-wise work lives:
 //   EPI_ROPE        Q/K/V projection + rotary embedding on the rotated heads;
-//   EPI_OPROJ_LOOP  output projection fused with the residual (y = x + a) and the
-//                   recurrent update h_next = A (.) h + B.e + a (the MoE adds f later);
+//   EPI_OPROJ_LOOP  output projection completing the residual y = x + a and the recurrent
+//                   update h_next = A (.) h + B.e + a (RMSNorm1 wrote x and A h + B.e; the
+//                   MoE adds f later);
 //   EPI_SWIGLU      expert up-projection (gate and up rows interleaved per tile) -> silu(g)*u;
 //   EPI_SCATTER     expert down-projection, gate weight, and reduction into h_next
 //                   (h_{t+1} = A h + B e + a + sum_j w_j E_j(yn)).
@@ -45,19 +46,24 @@ struct TcCfg {
     static constexpr int B_ROWS = BN / CG;               // B rows this CTA loads per stage
     static constexpr int A_BYTES = BM * 128;
     static constexpr int B_BYTES = B_ROWS * 128;
-    static constexpr int STAGES = (A_BYTES + B_BYTES <= 24 * 1024) ? 8 : (A_BYTES + B_BYTES <= 32 * 1024) ? 6 : 4;
+    static constexpr int BAR_BYTES = 192;
+    static constexpr int GROUP_BYTES = 2064;
+    static constexpr int STG_BYTES = 4 * 32 * 32 * 4;     // one 32 x 32 fp32 chunk per epilogue warp
+    // As many stages as keep the block (plus the 1 KB reserved per CTA) within the 196 KB
+    // shared-memory carveout, at most 8: beyond it the driver takes the 228 KB carveout and
+    // L1 shrinks from 60 to 28 KB, which measurably slows the epilogues' global traffic.
+    static constexpr int STAGES_FIT = (195 * 1024 - BAR_BYTES - GROUP_BYTES - STG_BYTES) / (A_BYTES + B_BYTES);
+    static constexpr int STAGES = STAGES_FIT < 8 ? STAGES_FIT : 8;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     // two accumulators of BN fp32 columns, rounded up to a power of two
     static constexpr int TMEM_COLS = 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
     // [stages][barriers][group tables][epilogue staging], all dynamic (no static shared
     // memory, so that the dynamic block starts 1024-byte aligned)
-    static constexpr int BAR_BYTES = 192;
-    static constexpr int GROUP_BYTES = 2064;
-    static constexpr int STG_BYTES = 4 * 32 * 32 * 4;     // one 32 x 32 fp32 chunk per epilogue warp
     static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + GROUP_BYTES + STG_BYTES;
     static_assert((BAR_BYTES + GROUP_BYTES) % 16 == 0, "staging buffers must be 16-byte aligned");
     static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte alignment of stages");
     static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
+    static_assert(STAGES >= 3, "too few pipeline stages");
 };
 
 __device__ __forceinline__ void ld_chunk(uint32_t taddr, int c, float (&v)[32]) {
@@ -296,45 +302,26 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, flo
             }
         }
     } else if constexpr (KIND == EPI_OPROJ_LOOP) {
-        // y = h + e + a and h_next = A (.) h + B.e + a. Every load of a chunk is issued before
-        // its stores (the stores could alias the loads as far as the compiler knows).
-        const T* e = static_cast<const T*>(p.e);
+        // y (= x) and h_next (= A (.) h + B.e) were written by RMSNorm1; the attention output
+        // completes both: y = x + a, h_next = A (.) h + B.e + a. Vector atomics need no reads
+        // here, so the epilogue never waits on memory.
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
             float v[32];
             ld_chunk(taddr, c, v);
-            const int col = n0 + c * 32 + cc;
-            if (n0 + c * 32 >= p.ncols_valid) continue;
+            const int col = n0 + c * 32;
+            if (col >= p.ncols_valid) continue;
             stage_put(stg, lane, v);
-            float aa[4];
-            load4(p.Adiag + col, aa);
-            float hh[8][4], be[8][4], ee[8][4];
 #pragma unroll
             for (int it = 0; it < 8; ++it) {
                 const int rr = it * 4 + (lane >> 3);
-                const size_t off = static_cast<size_t>(row0 + rr) * p.ld + col;
-                if (rr < nvalid) {
-                    load4(p.h + off, hh[it]);
-                    load4(p.Be + off, be[it]);
-                    if (e) load4(e + off, ee[it]);
-                    else ee[it][0] = ee[it][1] = ee[it][2] = ee[it][3] = 0.0f;
-                }
-            }
-#pragma unroll
-            for (int it = 0; it < 8; ++it) {
-                const int rr = it * 4 + (lane >> 3);
-                float av[4];
-                stage_get(stg, lane, it, av);
+                float o[4];
+                stage_get(stg, lane, it, o);
                 if (rr >= nvalid) continue;
-                const size_t off = static_cast<size_t>(row0 + rr) * p.ld + col;
-                float yv[4], hn[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    yv[i] = hh[it][i] + ee[it][i] + av[i];
-                    hn[i] = aa[i] * hh[it][i] + be[it][i] + av[i];
-                }
-                store4(p.y + off, yv);
-                store4(p.h_next + off, hn);
+                const size_t off = static_cast<size_t>(row0 + rr) * p.ld + col + cc;
+                const float4 add = make_float4(o[0], o[1], o[2], o[3]);
+                atomicAdd(reinterpret_cast<float4*>(p.y + off), add);
+                atomicAdd(reinterpret_cast<float4*>(p.h_next + off), add);
             }
         }
     } else if constexpr (KIND == EPI_SWIGLU) {

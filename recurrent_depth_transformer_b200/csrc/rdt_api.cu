@@ -63,6 +63,7 @@ struct rdt_handle {
     // runs on CTA pairs (256-row tiles) or single CTAs (128-row tiles)
     int bn_qkv = 128, bn_o = 128, bn_up = 128, bn_down = 128;
     int pair_qkv = 0, pair_o = 0, pair_up = 0, pair_down = 0;
+    int split_down = 1;            // K split of the expert down-projection (linear epilogue)
     int32_t* idx = nullptr;
     float* wts = nullptr;
     int cap = 0;                   // rows reserved per expert group (tokens + padding)
@@ -288,6 +289,26 @@ TileChoice choose_tiles(long rows, long groups, int N, bool allow256, bool allow
     return best;
 }
 
+// K split for a GEMM whose epilogue is a reduction (the expert down-projection): splitting
+// K trades a fuller last wave for one more pipeline fill per tile. Busiest CTA's cost:
+// (tiles per CTA) x (K blocks per tile + a fill share of 3 K blocks); only splits that
+// divide the K blocks, so no tile has an empty K range.
+int choose_split(long tiles, int num_kb, int max_split) {
+    const long sms = num_sms();
+    int best = 1;
+    long best_cost = -1;
+    for (int sp = 1; sp <= max_split; ++sp) {
+        if (num_kb % sp) continue;
+        const long per = (tiles * sp + sms - 1) / sms;
+        const long cost = per * (num_kb / sp + 3);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = sp;
+        }
+    }
+    return best;
+}
+
 rdt_status build_maps(rdt_handle* h) {
     const rdt_config& c = h->cfg;
     const bool bf = h->bf;
@@ -432,6 +453,10 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         t = choose_tiles(grows, E + S, d, true, true, mode);
         h->bn_down = t.bn;
         h->pair_down = t.pair;
+        if (!t.pair) {
+            const long dtiles = ((grows + 127) / 128 + (E + S + 1) / 2) * (d / t.bn);
+            h->split_down = choose_split(dtiles, static_cast<int>(hid * es / 128), 4);
+        }
         t = choose_tiles(N, 0, d, true, true, mode);
         h->bn_o = t.bn;
         h->pair_o = t.pair;
@@ -636,6 +661,12 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         n1.zero_counts = h->counts;
         n1.n_zero = h->G;
     }
+    if (loop_mode) {
+        n1.y0 = h->y;
+        n1.hn0 = h_next;
+        n1.Be = h->Be;
+        n1.Adiag = h->A;
+    }
     TIMED(h, K_NORM1, 1, st, norm1(h->bf, n1, st));
 
     GemmArgs ga{};
@@ -761,10 +792,6 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
     eo.ncols_valid = d;
     if (loop_mode) {
         eo.kind = EPI_OPROJ_LOOP;
-        eo.h = hin;
-        eo.e = c.inject_e ? e : nullptr;
-        eo.Be = h->Be;
-        eo.Adiag = h->A;
         eo.y = h->y;
         eo.h_next = h_next;
         eo.ld = d;
@@ -913,6 +940,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     gd.cap = h->cap;
     gd.a_routed_base = N;
     gd.pair = h->pair_down;
+    gd.split_k = h->split_down;
     gd.max_tiles = h->pair_down ? h->max_tiles_pair : h->max_tiles;
     gd.a_from_c = 1;
     gd.flags = h->flags;

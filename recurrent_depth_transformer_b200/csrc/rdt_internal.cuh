@@ -380,7 +380,7 @@ rdt_status make_tmap_2d(CUtensorMap* map, const void* base, bool bf16_elems, uin
 enum EpiKind {
     EPI_STORE = 0,      // C[row, col] = acc                     (OutT)
     EPI_ROPE = 1,       // C = acc with RoPE on the rotary part of rotated heads (OutT)
-    EPI_OPROJ_LOOP = 2, // y = x + acc, h_next = A*h + Be + acc   (fp32)
+    EPI_OPROJ_LOOP = 2, // y += acc, h_next += acc (fp32 vector atomics; both preset by RMSNorm1)
     EPI_OPROJ_PLAIN = 3,// a_out = acc                             (fp32)
     EPI_SWIGLU = 4,     // U[row, j] = silu(acc_gate) * acc_up    (OutT)
     EPI_SCATTER = 5,    // dst[token, col] += w * acc             (fp32, vector atomics)
@@ -401,14 +401,10 @@ struct EpiParams {
     int rot_off;           // rotary part starts at this column inside a head
     int rot_dim;           // rotary width
     int rope_limit;        // columns >= rope_limit are not rotated (V heads)
-    // O-projection loop epilogue
-    const float* h;        // state h_t
-    const void* e;         // injection input (cfg dtype) or NULL (x = h)
-    const float* Be;
-    const float* Adiag;
-    float* y;              // x + a
-    float* h_next;         // A*h + Be + a (the MoE adds its share later)
-    int ld;                // row stride of h, e, Be, y, h_next (= dim)
+    // O-projection loop epilogue: y and h_next hold x and A (.) h + B.e (RMSNorm1 wrote them)
+    float* y;              // += a   ->  x + a
+    float* h_next;         // += a   ->  A*h + Be + a (the MoE adds its share later)
+    int ld;                // row stride of y and h_next (= dim)
     // scatter
     const int* row_token;  // routed rows: token of each output row
     const float* row_w;    // routed rows: gate weight
@@ -486,6 +482,9 @@ struct Norm1Args {
     int lora_r;
     void* lora_t;         // [N, 64] cfg dtype, columns [0, r) written
     int* zero_counts; int n_zero;   // counts to clear (next MoE), or NULL
+    // loop mode: also write the fp32 block input x into y0 and A (.) h + Be into hn0, which
+    // the O projection then completes with its output a (NULL: not written)
+    float* y0; float* hn0; const float* Be; const float* Adiag;
 };
 rdt_status norm1(bool bf16_elems, const Norm1Args& a, cudaStream_t st);
 

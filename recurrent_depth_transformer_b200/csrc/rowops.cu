@@ -71,7 +71,7 @@ __global__ void matmul_nt_kernel(const T* A, const float* B, float* C, int M, in
 // ----------------------------------------------------------------------------- norm1
 
 template <typename T, int NV>
-__global__ void __launch_bounds__(kRowThreads) norm1_kernel(const Norm1Args a) {
+__global__ void __launch_bounds__(kRowThreads, NV <= 8 ? 2 : 1) norm1_kernel(const Norm1Args a) {
     pdl_trigger();
     pdl_wait();
     if (blockIdx.x == 0 && a.zero_counts)
@@ -81,20 +81,46 @@ __global__ void __launch_bounds__(kRowThreads) norm1_kernel(const Norm1Args a) {
     if (row >= a.ntok) return;
     const size_t base = static_cast<size_t>(row) * a.dim;
     const T* e = static_cast<const T*>(a.e);
-    float x[NV][4];
+    constexpr bool kHoistG = NV <= 8;          // gamma in flight with the row, registers allowing
+    float x[NV][4], g[kHoistG ? NV : 1][4];
     float ss = 0.0f;
+    if constexpr (kHoistG) {
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        const int col = i * 128 + lane * 4;
-        load4(a.h + base + col, x[i]);
-        if (e) {
-            float ev[4];
-            load4(e + base + col, ev);
+        for (int i = 0; i < NV; ++i) load4(a.gamma + i * 128 + lane * 4, g[i]);
+    }
+    // Groups of up to 4 vectors: every load of a group is issued before its stores (which
+    // could alias the loads as far as the compiler knows, and would serialise them).
+    constexpr int GV = NV < 4 ? NV : 4;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) x[i][j] += ev[j];
+    for (int i0 = 0; i0 < NV; i0 += GV) {
+        float ev[GV][4], be[GV][4], ad[GV][4];
+#pragma unroll
+        for (int i = 0; i < GV; ++i) {
+            const int col = (i0 + i) * 128 + lane * 4;
+            load4(a.h + base + col, x[i0 + i]);
+            if (e) load4(e + base + col, ev[i]);
+            if (a.hn0) {
+                load4(a.Be + base + col, be[i]);
+                load4(a.Adiag + col, ad[i]);
+            }
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) ss = fmaf(x[i][j], x[i][j], ss);
+        for (int i = 0; i < GV; ++i) {
+            const int col = (i0 + i) * 128 + lane * 4;
+            if (a.hn0) {   // A (.) h + B.e, the part of h_next the O projection and the MoE complete
+                float hn[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) hn[j] = fmaf(ad[i][j], x[i0 + i][j], be[i][j]);
+                store4(a.hn0 + base + col, hn);
+            }
+            if (e) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) x[i0 + i][j] += ev[i][j];
+            }
+            if (a.y0) store4(a.y0 + base + col, x[i0 + i]);   // the block input x, completed to x + a
+#pragma unroll
+            for (int j = 0; j < 4; ++j) ss = fmaf(x[i0 + i][j], x[i0 + i][j], ss);
+        }
     }
     ss = warp_sum(ss);
     const float inv = rsqrtf(ss / a.dim + a.eps);
@@ -102,10 +128,14 @@ __global__ void __launch_bounds__(kRowThreads) norm1_kernel(const Norm1Args a) {
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
         const int col = i * 128 + lane * 4;
-        float g[4];
-        load4(a.gamma + col, g);
+        float gi[4];
+        if constexpr (kHoistG) {
+            gi[0] = g[i][0]; gi[1] = g[i][1]; gi[2] = g[i][2]; gi[3] = g[i][3];
+        } else {
+            load4(a.gamma + col, gi);
+        }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) x[i][j] = to_f(from_f<T>(x[i][j] * inv * g[j]));
+        for (int j = 0; j < 4; ++j) x[i][j] = to_f(from_f<T>(x[i][j] * inv * gi[j]));
         store4(xn + col, x[i]);
     }
     if (a.lora_a) {

@@ -26,11 +26,18 @@ def test_algorithmic_flops_of_the_bench_workload():
 
 
 def test_parse_clocks():
-    txt = ("0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n"
-           "0, 1800, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n"
-           "0, 1700, 1965, 999.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n")
+    txt = ("2026/12/02 19:04:21.000, 0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n"
+           "2026/12/02 19:04:21.050, 0, 1800, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n"
+           "2026/12/02 19:04:21.100, 0, 1700, 1965, 999.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n")
     c = bench.parse_clocks(txt)
     assert c["sm_mhz"] == 1800 and c["sm_max_mhz"] == 1965 and c["reasons"] == ["sw_power_cap"]
+    assert c["samples"] == 3 and not c["in_timed_region"]
+    # only the samples inside the timed region count when some fall in it
+    t0 = bench._stamp("2026/12/02 19:04:21.040")
+    c = bench.parse_clocks(txt, (t0, t0 + 0.02))
+    assert c["samples"] == 1 and c["sm_mhz"] == 1800 and c["in_timed_region"]
+    c = bench.parse_clocks(txt, (t0 + 10, t0 + 11))       # none inside: all samples, flagged
+    assert c["samples"] == 3 and not c["in_timed_region"]
     assert bench.parse_clocks("") is None
 
 
