@@ -88,3 +88,13 @@ def test_reference_arm_prints_one_json_line(capsys):
     line = json.loads(out[0])
     assert line["impl"] == "reference" and line["unit"] == bench.UNIT and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_measured_traffic_only_for_unchanged_sources(monkeypatch):
+    files = bench.KERNEL_SOURCES["gemm_up"]
+    fp = bench.source_fingerprint(files)
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, "gemm_up", (123.0, fp))
+    assert bench.measured_traffic("gemm_up") == 123.0
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, "gemm_up", (123.0, "0" * 16))
+    assert bench.measured_traffic("gemm_up") is None          # sources changed since the capture
+    assert bench.measured_traffic("attention") is None        # never captured
