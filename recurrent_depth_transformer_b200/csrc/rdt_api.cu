@@ -249,20 +249,23 @@ rdt_status interleave_w13(void* dst, const void* w1, const void* w3, int hid, in
 
 // Tile shape for a GEMM with `rows` output rows (grouped: plus the partial last tile of each
 // of `groups` groups, estimated as half a tile) and N columns; mode 0 chooses, 1 forces single
-// CTAs, 2 forces CTA pairs where the shape allows them.
+// CTAs, 2 forces CTA pairs where the shape allows them. allow192: 192-wide pair tiles fit the
+// epilogue (whole RoPE heads, no SwiGLU interleave).
 //
 // Single CTAs: the persistent grid's time is that of its busiest CTA, (tiles per CTA) x (tile
 // time), a tile's time taken as proportional to BN plus a fixed share for its pipeline fill
 // and epilogue. Measured on B200 this favours 128-wide tiles whenever the grid runs more
-// than one wave. CTA pairs (256 x 256 tiles, each CTA loading half of B) load fewer bytes per
-// CTA for the same output; measured, that pays only when the whole GEMM fits in one wave of
-// pairs and its best single-CTA shape would load more per CTA, so that is when they are
-// chosen.
+// than one wave. CTA pairs (256-row tiles, each CTA loading half of the B rows) load fewer
+// bytes per CTA for the same output, but a pair's CTA ingests about a quarter less per
+// second than a single CTA (measured, one-wave grids); so a pair shape is chosen only when
+// the whole GEMM fits one wave of pairs and each CTA then loads under 3/4 of what the best
+// single-CTA shape loads per K block (128 + BN rows single, 128 + BN/2 per CTA of a pair).
 struct TileChoice {
     int bn;
     int pair;
 };
-TileChoice choose_tiles(long rows, long groups, int N, bool allow256, bool allow_pair, int mode) {
+TileChoice choose_tiles(long rows, long groups, int N, bool allow256, bool allow_pair, int mode,
+                        bool allow192 = false) {
     const long sms = num_sms();
     const bool n256 = allow256 && N % 256 == 0;
     if (mode == 2 && allow_pair) return {n256 ? 256 : 128, 1};
@@ -281,10 +284,18 @@ TileChoice choose_tiles(long rows, long groups, int N, bool allow256, bool allow
             best_tiles = tiles;
         }
     }
-    if (mode == 0 && allow_pair && n256) {
-        const long pairs = ((rows + 255) / 256 + (groups + 1) / 2) * (N / 256);
-        const bool one_wave = best_tiles <= sms && pairs <= sms / 2;
-        if (one_wave && 128 + best.bn > 128 + 128) best = {256, 1};   // bytes per CTA per K block
+    if (mode == 0 && allow_pair && best_tiles <= sms) {
+        const long single_rows = 128 + best.bn;          // rows one CTA loads per K block
+        long pair_rows = -1;
+        for (int bn : {256, 192, 128}) {
+            if ((bn == 256 && !n256) || (bn == 192 && !(allow192 && N % 192 == 0)) || N % bn) continue;
+            const long pairs = ((rows + 255) / 256 + (groups + 1) / 2) * (N / bn);
+            const long r = 128 + bn / 2;
+            if (pairs <= sms / 2 && 4 * r < 3 * single_rows && (pair_rows < 0 || r < pair_rows)) {
+                pair_rows = r;
+                best = {bn, 1};
+            }
+        }
     }
     return best;
 }
@@ -462,7 +473,7 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         h->pair_o = t.pair;
         if (c.attn_type == RDT_GQA) {
             const int nqkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
-            t = choose_tiles(N, 0, nqkv, nqkv % 256 == 0, true, mode);
+            t = choose_tiles(N, 0, nqkv, nqkv % 256 == 0, true, mode, 192 % c.head_dim == 0);
             h->bn_qkv = t.bn;
             h->pair_qkv = t.pair;
         }
