@@ -29,6 +29,14 @@ constexpr int kBQ = 128;     // queries per CTA
 constexpr int kBK = 128;     // keys per block
 constexpr int kAtom = 16384; // one 128-row x 128-byte swizzled region
 
+// 2^x by the hardware approximation (ex2.approx, flush-to-zero): the probabilities are
+// rounded to bf16 for the P.V product, and P below 2^-126 contributes nothing there.
+__device__ __forceinline__ float exp2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -269,7 +277,7 @@ __global__ void __launch_bounds__(192, 2)
             if (j > 0 && !mbar_wait(ofull, (j - 1) & 1, a.flags)) { ok = false; break; }
             tc_fence_after();
             if (mx > m_ref + kRescaleThreshold) {
-                const float corr = exp2f(m_ref - mx);
+                const float corr = exp2_ftz(m_ref - mx);
                 if (j > 0) {
 #pragma unroll
                     for (int c = 0; c < DV / 32; ++c) {
@@ -295,8 +303,8 @@ __global__ void __launch_bounds__(192, 2)
                 uint32_t packed[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    float p0 = exp2f(__uint_as_float(v[2 * i]) * sl - m_ref);
-                    float p1 = exp2f(__uint_as_float(v[2 * i + 1]) * sl - m_ref);
+                    float p0 = exp2_ftz(__uint_as_float(v[2 * i]) * sl - m_ref);
+                    float p1 = exp2_ftz(__uint_as_float(v[2 * i + 1]) * sl - m_ref);
                     if (need_mask) {
                         if (c * 32 + 2 * i > kmax) p0 = 0.0f;
                         if (c * 32 + 2 * i + 1 > kmax) p1 = 0.0f;

@@ -332,8 +332,12 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, flo
             float g[32], u[32];
             ld_chunk(taddr, c, g);
             ld_chunk(taddr, c + BN / 64, u);
+            // silu(g) * u with the fast exponential and division intrinsics: the result is
+            // stored in bf16, whose rounding (2^-8 relative) dwarfs their few-ulp fp32 error;
+            // IEEE expf and division made this epilogue longer than a tile's MMAs on pairs
+            // (for g -> -inf: exp -> inf, 1 / inf = 0, silu -> 0 as it should)
 #pragma unroll
-            for (int i = 0; i < 32; ++i) g[i] = g[i] / (1.0f + expf(-g[i])) * u[i];
+            for (int i = 0; i < 32; ++i) g[i] = g[i] * __fdividef(1.0f, 1.0f + __expf(-g[i])) * u[i];
             store_chunk(stg, lane, g, out + c * 32, p.ldo, nvalid);
         }
     } else if constexpr (KIND == EPI_SCATTER) {
