@@ -41,7 +41,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (fingerprint: first 16 hex digits of the SHA-256 of the listed files, concatenated).
 KERNEL_SOURCES = {"gemm_up": ("recurrent_depth_transformer_b200/csrc/gemm_tc.cuh",
                               "recurrent_depth_transformer_b200/csrc/gemm_tc.cu",
-                              "recurrent_depth_transformer_b200/csrc/rdt_internal.cuh")}
+                              "recurrent_depth_transformer_b200/csrc/gemm_tc_pair.cu",
+                              "recurrent_depth_transformer_b200/csrc/rdt_internal.cuh",
+                              "recurrent_depth_transformer_b200/csrc/rdt_api.cu")}
 MEASURED_TRAFFIC = {"gemm_up": (77.635328e6 + 3.635456e6, "142fa22d4475c880")}
 
 

@@ -82,7 +82,8 @@ typedef struct {
     int32_t inject_e;               /* 1: block input x = h + e; 0: x = h               */
     int32_t max_loops;              /* largest T accepted (<= 64; the pages loop <= 16) */
     int32_t gemm_tiles;             /* projection / expert GEMM tiles: 0 chosen per GEMM
-                                     * from its shape, 1 one CTA per 128-row tile, 2 CTA
+                                     * from its shape (and a K split for the expert
+                                     * down-projection), 1 one CTA per 128-row tile, 2 CTA
                                      * pairs per 256-row tile (bf16 only; fp32 uses 1).
                                      * Results agree up to fp32 summation order.        */
 } rdt_config;

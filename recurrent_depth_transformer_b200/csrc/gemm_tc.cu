@@ -18,6 +18,12 @@ rdt_status dispatch_router(const CUtensorMap& tA, const CUtensorMap& tB, const C
 rdt_status gemm_tc(bool bf16_elems, int bn, const CUtensorMap& tA, const CUtensorMap& tB,
                    const CUtensorMap* tA2, const CUtensorMap* tB2, const GemmArgs& args,
                    const EpiParams& epi, cudaStream_t st) {
+    // a K split leaves partial sums to combine: only epilogues that reduce into their output
+    // (and the router's, which combines its partial logits itself) may split
+    if (args.split_k > 1 && epi.kind != EPI_SCATTER && epi.kind != EPI_OPROJ_LOOP && epi.kind != EPI_TOPK) {
+        set_error("gemm_tc: a K split needs an epilogue that reduces into its output");
+        return RDT_ERR_INVALID_ARG;
+    }
     if (epi.kind == EPI_TOPK) {
         if (bf16_elems) {
             if (bn == 64) return dispatch_router<bf16, 64>(tA, tB, tA2, tB2, args, epi, st);

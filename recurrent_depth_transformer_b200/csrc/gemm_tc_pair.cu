@@ -11,10 +11,6 @@ rdt_status gemm_tc_pair(int bn, const CUtensorMap& tA, const CUtensorMap& tB, co
         set_error("gemm_tc: the router runs on single-CTA tiles");
         return RDT_ERR_UNSUPPORTED;
     }
-    if (args.split_k > 1) {
-        set_error("gemm_tc: pair tiles do not split K");
-        return RDT_ERR_UNSUPPORTED;
-    }
     if (bn == 128) return dispatch_kind<bf16, 128, 2>(tA, tB, tA2, tB2, args, epi, st);
     if (bn == 192) return dispatch_kind<bf16, 192, 2>(tA, tB, tA2, tB2, args, epi, st);
     if (bn == 256) return dispatch_kind<bf16, 256, 2>(tA, tB, tA2, tB2, args, epi, st);

@@ -247,74 +247,48 @@ rdt_status interleave_w13(void* dst, const void* w1, const void* w3, int hid, in
     return RDT_OK;
 }
 
-// Tile shape for a GEMM with `rows` output rows (grouped: plus the partial last tile of each
-// of `groups` groups, estimated as half a tile) and N columns; mode 0 chooses, 1 forces single
-// CTAs, 2 forces CTA pairs where the shape allows them. allow192: 192-wide pair tiles fit the
-// epilogue (whole RoPE heads, no SwiGLU interleave).
+// Tile shape of a projection or expert GEMM: `rows` output rows (grouped: plus the partial
+// last tile of each of `groups` groups, counted as half a tile), N columns, num_kb K blocks of
+// 128 bytes. mode 0 chooses, 1 forces single CTAs, 2 forces CTA pairs where allowed.
 //
-// Single CTAs: the persistent grid's time is that of its busiest CTA, (tiles per CTA) x (tile
-// time), a tile's time taken as proportional to BN plus a fixed share for its pipeline fill
-// and epilogue. Measured on B200 this favours 128-wide tiles whenever the grid runs more
-// than one wave. CTA pairs (256-row tiles, each CTA loading half of the B rows) load fewer
-// bytes per CTA for the same output, but a pair's CTA ingests about a quarter less per
-// second than a single CTA (measured, one-wave grids); so a pair shape is chosen only when
-// the whole GEMM fits one wave of pairs and each CTA then loads under 3/4 of what the best
-// single-CTA shape loads per K block (128 + BN rows single, 128 + BN/2 per CTA of a pair).
+// Measured on B200, these GEMMs are bound by what each SM ingests through TMA, so a tile's
+// time is taken as proportional to the rows of A and B one CTA loads per K block (128 + BN
+// single, 128 + BN/2 per CTA of a pair) times (its K blocks + 3 for pipeline fill and
+// epilogue), scaled by the measured ingest of the shape (1 single 128-wide; 1.25 single
+// 256-wide, which fits only 3 stages; 4/3 for a CTA of a pair); the persistent grid's time
+// is that of its busiest CTA (pair). K splits (max_split > 1) are for epilogues that reduce
+// into their output. Measured choices at batch 4 x seq 512 x dim 1024: QKV on 192-wide pairs,
+// O single 128-wide, expert up on 256-wide pairs, expert down single 128-wide split 2.
 struct TileChoice {
     int bn;
     int pair;
+    int split;
 };
-TileChoice choose_tiles(long rows, long groups, int N, bool allow256, bool allow_pair, int mode,
-                        bool allow192 = false) {
+TileChoice choose_tiles(long rows, long groups, int N, int num_kb, bool allow256, bool allow192,
+                        bool allow_pair, int max_split, int mode) {
     const long sms = num_sms();
-    const bool n256 = allow256 && N % 256 == 0;
-    if (mode == 2 && allow_pair) return {n256 ? 256 : 128, 1};
-    long best_cost = -1;
-    TileChoice best{128, 0};
-    long best_tiles = 0;
-    for (int bn : {256, 128}) {
-        if (bn == 256 && !n256) continue;
-        if (N % bn) continue;
-        const long tiles = ((rows + 127) / 128 + (groups + 1) / 2) * (N / bn);
-        const long per = (tiles + sms - 1) / sms;
-        const long cost = per * (32 + bn);
-        if (best_cost < 0 || cost < best_cost) {
-            best_cost = cost;
-            best = {bn, 0};
-            best_tiles = tiles;
-        }
-    }
-    if (mode == 0 && allow_pair && best_tiles <= sms) {
-        const long single_rows = 128 + best.bn;          // rows one CTA loads per K block
-        long pair_rows = -1;
+    TileChoice best{128, 0, 1};
+    double best_cost = -1.0;
+    for (int pair : {0, 1}) {
+        if (pair && !allow_pair) continue;
+        if (mode == 1 && pair) continue;
+        if (mode == 2 && allow_pair && !pair) continue;
+        const long tile_rows = pair ? 256 : 128;
+        const long m_tiles = (rows + tile_rows - 1) / tile_rows + (groups + 1) / 2;
+        const long slots = pair ? sms / 2 : sms;
         for (int bn : {256, 192, 128}) {
-            if ((bn == 256 && !n256) || (bn == 192 && !(allow192 && N % 192 == 0)) || N % bn) continue;
-            const long pairs = ((rows + 255) / 256 + (groups + 1) / 2) * (N / bn);
-            const long r = 128 + bn / 2;
-            if (pairs <= sms / 2 && 4 * r < 3 * single_rows && (pair_rows < 0 || r < pair_rows)) {
-                pair_rows = r;
-                best = {bn, 1};
+            if ((bn == 256 && !allow256) || (bn == 192 && !(allow192 && pair)) || N % bn) continue;
+            const double rate = pair ? 4.0 / 3.0 : (bn == 256 ? 1.25 : 1.0);
+            const double load_rows = 128.0 + (pair ? bn / 2 : bn);
+            for (int sp = 1; sp <= max_split; ++sp) {
+                if (num_kb % sp) continue;
+                const long rounds = (m_tiles * (N / bn) * sp + slots - 1) / slots;
+                const double cost = static_cast<double>(rounds) * (num_kb / sp + 3) * load_rows * rate;
+                if (best_cost < 0 || cost < best_cost) {
+                    best_cost = cost;
+                    best = {bn, pair, sp};
+                }
             }
-        }
-    }
-    return best;
-}
-
-// K split for a GEMM whose epilogue is a reduction (the expert down-projection): splitting
-// K trades a fuller last wave for one more pipeline fill per tile. Busiest CTA's cost:
-// (tiles per CTA) x (K blocks per tile + a fill share of 3 K blocks); only splits that
-// divide the K blocks, so no tile has an empty K range.
-int choose_split(long tiles, int num_kb, int max_split) {
-    const long sms = num_sms();
-    int best = 1;
-    long best_cost = -1;
-    for (int sp = 1; sp <= max_split; ++sp) {
-        if (num_kb % sp) continue;
-        const long per = (tiles * sp + sms - 1) / sms;
-        const long cost = per * (num_kb / sp + 3);
-        if (best_cost < 0 || cost < best_cost) {
-            best_cost = cost;
-            best = sp;
         }
     }
     return best;
@@ -456,24 +430,26 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
     if (h->bf) {
         const long grows = static_cast<long>(N) * (K + S);
         const int mode = c.gemm_tiles;
+        const int kb_d = static_cast<int>(d * es / 128), kb_h = static_cast<int>(hid * es / 128);
+        const int ow = c.attn_type == RDT_GQA ? c.n_heads * c.head_dim : c.n_heads * c.kv_lora_rank;
         // SwiGLU tiles hold BN/2 gate and BN/2 up columns; W1/W3 are interleaved in blocks
         // of BN/2 rows, which must divide the hidden width
-        TileChoice t = choose_tiles(grows, E + S, 2 * hid, hid % 128 == 0, hid % 64 == 0, mode);
+        TileChoice t = choose_tiles(grows, E + S, 2 * hid, kb_d, hid % 128 == 0, false, hid % 64 == 0, 1, mode);
         h->bn_up = t.bn;
         h->pair_up = t.pair;
-        t = choose_tiles(grows, E + S, d, true, true, mode);
+        // the down-projection's epilogue reduces every output into h_next; on pairs a CTA's
+        // share of it doubles and measured slower (24.3 vs 22.7 us), so it runs on pairs only
+        // when they are forced
+        t = choose_tiles(grows, E + S, d, kb_h, true, false, mode == 2, 4, mode);
         h->bn_down = t.bn;
         h->pair_down = t.pair;
-        if (!t.pair) {
-            const long dtiles = ((grows + 127) / 128 + (E + S + 1) / 2) * (d / t.bn);
-            h->split_down = choose_split(dtiles, static_cast<int>(hid * es / 128), 4);
-        }
-        t = choose_tiles(N, 0, d, true, true, mode);
+        h->split_down = t.split;
+        t = choose_tiles(N, 0, d, static_cast<int>(ow * es / 128), true, false, true, 1, mode);
         h->bn_o = t.bn;
         h->pair_o = t.pair;
         if (c.attn_type == RDT_GQA) {
             const int nqkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
-            t = choose_tiles(N, 0, nqkv, nqkv % 256 == 0, true, mode, 192 % c.head_dim == 0);
+            t = choose_tiles(N, 0, nqkv, kb_d, nqkv % 256 == 0, 192 % c.head_dim == 0, true, 1, mode);
             h->bn_qkv = t.bn;
             h->pair_qkv = t.pair;
         }
