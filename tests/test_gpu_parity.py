@@ -59,6 +59,38 @@ def test_gemm_tile_modes_match_oracle(name, tiles):
     assert_close(got, want, what=f"{name} tiles={tiles}")
 
 
+@pytest.mark.parametrize("tiles", [0, 1, 2])
+def test_all_tokens_on_two_experts(tiles):
+    """A router bias of +8 on experts 0 and 1 sends every token there: two groups at full
+    capacity (several row tiles, ragged last one), fourteen empty groups; the oracle applies
+    the same bias in its selection (the gap to the third expert is ~8: no near-ties)."""
+    wl = C1.replace(batch=2, seq=200)
+    inputs = generate(wl)
+    inputs["router_bias"] = np.zeros(wl.n_experts, dtype=np.float32)
+    inputs["router_bias"][:2] = 8.0
+    got, idx, _, _, diag = run_loop(wl, inputs, 2, gemm_tiles=tiles)
+    assert diag["nonfinite"] == 0 and diag["timeout"] == 0
+    assert set(np.unique(idx)) == {0, 1}
+    want, mism, ties, _ = oracle_follow(wl, inputs, 2, idx)
+    assert mism == 0 and ties == 0
+    assert_close(got, want, what=f"two experts, tiles={tiles}")
+
+
+@pytest.mark.parametrize("E,k", [(8, 8), (16, 12)])
+def test_top_k_up_to_all_experts(E, k):
+    """k = E: every token goes to every expert (each group holds all tokens; the fused
+    router); k = 12 > 8: the tensor-core router with its 16-wide top-k epilogue."""
+    wl = C1.replace(batch=1, seq=192, n_experts=E, top_k=k)
+    inputs = generate(wl)
+    got, idx, w, _, diag = run_loop(wl, inputs, 2)
+    assert diag["nonfinite"] == 0 and diag["timeout"] == 0
+    assert all(len(set(r)) == k for r in idx.reshape(-1, k))          # k distinct experts per token
+    np.testing.assert_allclose(w.reshape(-1, k).sum(axis=1), 1.0, atol=1e-5)
+    want, mism, _, _ = oracle_follow(wl, inputs, 2, idx)
+    assert mism == 0
+    assert_close(got, want, what=f"E={E} k={k}")
+
+
 def test_zero_block_is_closed_form():
     # every block weight zero: h_T = A^T h0 + (1 - A^T)/(1 - A) B e exactly (fp32 state)
     wl = C1.replace(batch=2, seq=64)
