@@ -1,5 +1,5 @@
 // RMSNorm2 fused with the MoE router for routers whose weight fits in shared memory:
-// each block stages W_r (n_experts x dim) once as fp32, then every warp takes rows in turn:
+// each block stages W_r (n_experts x dim) once, then every warp takes rows in turn:
 // RMSNorm2 in fp32 (stored in the element type as the experts' input), the n_experts logits
 // of the fp32 normalised row, top-k of logits + bias with ties to the lower expert index,
 // softmax over the k chosen logits, per-expert histogram.
@@ -13,19 +13,19 @@ namespace {
 
 // ----------------------------------------------------------------------------- norm2 + router (W_r in shared memory)
 
-// For routers whose weight fits in shared memory: each block stages W_r once, as fp32, then
-// every warp takes rows in turn: RMSNorm2 (fp32, stored in the element type for the experts),
+// For routers whose weight fits in shared memory: each block stages W_r once, then every warp
+// takes rows in turn: RMSNorm2 (fp32, stored in the element type for the experts),
 // the n_exp logits of the fp32 row against W_r, top-k of logits + bias (ties to the lower
 // expert index), softmax over the k chosen logits, histogram, and the row's copies for the
 // chosen experts.
 //
 // The work per row is a few hundred instructions, so the kernel is bound by instruction
 // issue and latency, not bytes: each lane owns 4 * NV columns of the row, forms its partial
-// logits with packed fp32 FMAs from 16-byte shared loads, and the warp reduces the EMAX
+// logits with packed fp32 FMAs from shared loads of 4 weights, and the warp reduces the EMAX
 // partials with a transposing butterfly (EMAX - 1 + 1 shuffles instead of 5 per logit) that
 // leaves lane l holding whole logits (expert l / 2 for 16 experts, experts 2l, 2l + 1 for 64).
 // Top-k is then k warp-wide argmax rounds over (score desc, index asc).
-constexpr int kRouterMaxThreads = 512;
+constexpr int kRouterMaxThreads = 256;
 
 // Butterfly transpose-reduce of v[0..E) over the warp. On return v[0 .. max(E/32, 1)) hold
 // full sums; router_expert() gives their expert indices.
@@ -71,33 +71,20 @@ __device__ __forceinline__ bool router_better(float s, int e, float so, int eo) 
 }
 
 template <typename T, int NV, int EMAX, int KMAX>
-__global__ void __launch_bounds__(kRouterMaxThreads) norm2_router_smem_kernel(const RouterArgs a) {
-    extern __shared__ __align__(16) float Ws[];     // [n_exp][dim] fp32
+__global__ void __launch_bounds__(kRouterMaxThreads, 2) norm2_router_smem_kernel(const RouterArgs a) {
+    extern __shared__ __align__(16) uint8_t ws_raw[];   // W_r [n_exp][dim] in the element type
+    const T* Ws = reinterpret_cast<const T*>(ws_raw);
     constexpr int NL = EMAX >= 32 ? EMAX / 32 : 1;  // logits held per lane after the reduce
     const int lane = threadIdx.x & 31;
     const int nthreads = blockDim.x;
+    // W_r is copied as is (16-byte chunks) and converted where it is read: the copy is half
+    // the size of an fp32 one, small enough for a block to sit beside the projection GEMM's
+    // CTAs and stage it while they run
     auto stage = [&]() {
-        const int n8 = a.n_exp * a.dim / 8;
-        for (int i = threadIdx.x; i < n8; i += nthreads) {
-            float f[8];
-            if constexpr (std::is_same<T, bf16>::value) {
-                const uint4 x = static_cast<const uint4*>(a.w_router)[i];
-                const uint32_t u[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[j]));
-                    f[2 * j] = t.x;
-                    f[2 * j + 1] = t.y;
-                }
-            } else {
-                const float4 x0 = static_cast<const float4*>(a.w_router)[2 * i];
-                const float4 x1 = static_cast<const float4*>(a.w_router)[2 * i + 1];
-                f[0] = x0.x; f[1] = x0.y; f[2] = x0.z; f[3] = x0.w;
-                f[4] = x1.x; f[5] = x1.y; f[6] = x1.z; f[7] = x1.w;
-            }
-            reinterpret_cast<float4*>(Ws)[2 * i] = make_float4(f[0], f[1], f[2], f[3]);
-            reinterpret_cast<float4*>(Ws)[2 * i + 1] = make_float4(f[4], f[5], f[6], f[7]);
-        }
+        const int n16 = a.n_exp * a.dim * static_cast<int>(sizeof(T)) / 16;
+        const uint4* src = static_cast<const uint4*>(a.w_router);
+        uint4* dst = reinterpret_cast<uint4*>(ws_raw);
+        for (int i = threadIdx.x; i < n16; i += nthreads) dst[i] = src[i];
     };
     pdl_trigger();
     if (a.weights_static) stage();      // overlaps the tail of the previous kernel
@@ -150,10 +137,18 @@ __global__ void __launch_bounds__(kRouterMaxThreads) norm2_router_smem_kernel(co
         for (int e = 0; e < EMAX; ++e) {
             float2 acc = make_float2(0.0f, 0.0f);
             if (e < a.n_exp) {
-                const float4* wrow = reinterpret_cast<const float4*>(Ws + static_cast<size_t>(e) * a.dim) + lane;
+                const T* wrow = Ws + static_cast<size_t>(e) * a.dim + lane * 4;
 #pragma unroll
                 for (int i = 0; i < NV; ++i) {
-                    const float4 w = wrow[i * 32];
+                    float4 w;
+                    if constexpr (std::is_same<T, bf16>::value) {
+                        const uint2 u = *reinterpret_cast<const uint2*>(wrow + i * 128);
+                        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+                        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+                        w = make_float4(lo.x, lo.y, hi.x, hi.y);
+                    } else {
+                        w = *reinterpret_cast<const float4*>(wrow + i * 128);
+                    }
                     acc = __ffma2_rn(make_float2(y[i][0], y[i][1]), make_float2(w.x, w.y), acc);
                     acc = __ffma2_rn(make_float2(y[i][2], y[i][3]), make_float2(w.z, w.w), acc);
                 }
@@ -252,16 +247,16 @@ bool router_fits_smem(bool bf, int n_exp, int top_k, int dim) {
 
 namespace {
 
-// One block per SM at most (each stages W_r), with enough warps that every SM gets a block
-// and every warp about one row per pass: 4..16 warps per block, rows strided over the grid.
+// Blocks of 8 warps, one row per warp: small enough (W_r copy <= 64 KB, 256 threads of at most
+// 128 registers) to run beside a GEMM CTA, so that blocks stage W_r while the previous kernel
+// runs (programmatic dependent launch) and the next kernel's prologue can start beside them.
 template <typename T, int NV, int EMAX, int KMAX>
 rdt_status launch_router_smem_k(const RouterArgs& a, cudaStream_t st) {
-    const size_t smem = static_cast<size_t>(a.n_exp) * a.dim * 4;
-    const int sms = num_sms();
-    const int warps = std::min(16, std::max(4, (a.ntok + sms - 1) / sms));
-    const int grid = std::min(sms, (a.ntok + warps - 1) / warps);
+    const size_t smem = static_cast<size_t>(a.n_exp) * a.dim * sizeof(T);
+    const int warps = kRouterMaxThreads / 32;
+    const int grid = (a.ntok + warps - 1) / warps;
     auto k = norm2_router_smem_kernel<T, NV, EMAX, KMAX>;
-    RDT_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024));
+    RDT_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
     RDT_CUDA_TRY(launch_pdl(k, dim3(grid), dim3(warps * 32), smem, st, a));
     return RDT_OK;
 }
