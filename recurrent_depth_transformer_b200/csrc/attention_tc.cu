@@ -16,7 +16,8 @@
 // c_kv = the key's first 128 columns, so its V operand is the K tile itself.
 //
 // Roles: warp 0 issues TMA loads (Q once, K two stages ahead, V one stage); warp 1 owns TMEM
-// and issues the MMAs (S_{j+1} before P_j V_j); warps 2-5 do the softmax and write o.
+// and issues the MMAs (S_{j+1} before P_j V_j); warps 2-9 do the softmax (two warps per 32
+// query rows, one per half of the key block) and write o.
 // Every wait is bounded.
 #include <algorithm>
 
@@ -73,7 +74,8 @@ struct AttnCfg {
     static constexpr int OFF_V = OFF_K + KSTAGES * K_BYTES;
     static constexpr int OFF_P = OFF_V + V_BYTES;
     static constexpr int OFF_BAR = OFF_P + P_BYTES;
-    static constexpr int SMEM = OFF_BAR + 128 + 1024;
+    static constexpr int OFF_X = OFF_BAR + 256;    // softmax exchange: row maxima [2][2][128], sums [2][128]
+    static constexpr int SMEM = OFF_X + 3 * 2 * 128 * 4 + 1024;
     static constexpr int S_COL = 0;                 // S: columns [0, 128)
     static constexpr int O_COL = 128;               // O: columns [128, 128 + DV)
     static constexpr int TMEM_COLS = 128 + DV <= 256 ? 256 : 512;
@@ -92,8 +94,10 @@ struct AttnTcArgs {
 // so P <= 2^8; then O and l are rescaled once by 2^(m_ref_old - m_ref_new).
 constexpr float kRescaleThreshold = 8.0f;
 
+constexpr int kAttnThreads = 320;   // TMA warp, MMA warp, 8 softmax warps
+
 template <int DQK, int DV, bool SHARE_KV>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(kAttnThreads, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                    const __grid_constant__ CUtensorMap tv, const AttnTcArgs a) {
     using C = AttnCfg<DQK, DV, SHARE_KV>;
@@ -111,6 +115,8 @@ __global__ void __launch_bounds__(192, 2)
     uint64_t* pfull = bars + 9;    // P_j in shared memory (and O rescaled if needed)
     uint64_t* ofull = bars + 10;   // P_j . V_j accumulated (P buffer and V stage free)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+    uint64_t* xchg = bars + 12;    // [4] per lane quadrant: both column halves posted their row maxima
+    uint64_t* lfin = bars + 16;    // [4] per lane quadrant: both halves posted their row sums
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -139,9 +145,13 @@ __global__ void __launch_bounds__(192, 2)
         mbar_init(vfull, 1);
         mbar_init(vempty, 1);
         mbar_init(sfull, 1);
-        mbar_init(sfree, 4);
-        mbar_init(pfull, 4);
+        mbar_init(sfree, 8);
+        mbar_init(pfull, 8);
         mbar_init(ofull, 1);
+        for (int q = 0; q < 4; ++q) {
+            mbar_init(&xchg[q], 2);
+            mbar_init(&lfin[q], 2);
+        }
         mbar_fence_init();
     }
     if (warp == 0 && lane == 0) {
@@ -240,14 +250,23 @@ __global__ void __launch_bounds__(192, 2)
             if (ok) issue_o(n_kb - 1);
         }
     } else {
-        // softmax warps: thread = query row
+        // Softmax warps 2..9: warp w covers TMEM lane quadrant w & 3 (32 query rows, a thread
+        // per row) and column half (w - 2) / 4 of each key block and of O. The two halves of a
+        // row exchange their block maxima (and, at the end, their sums) through shared memory,
+        // paired by a per-quadrant mbarrier with bounded waits; both then take the same
+        // rescaling decisions, and each rescales and finally writes its own half of O.
         const int quad = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int r = quad * 32 + lane;
         const int qpos = q0 + r;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
         const float sl = a.scale_log2;
         float m_ref = -INFINITY, l = 0.0f;
-        uint8_t* arow0 = smem + C::OFF_P + r * 128;
+        uint8_t* arow = smem + C::OFF_P + half * kAtom + r * 128;    // this half's P atom
+        float* mxx = reinterpret_cast<float*>(smem + C::OFF_X);      // [2 parity][2 half][128]
+        float* lxx = mxx + 2 * 2 * 128;                              // [2 half][128]
+        constexpr int HC = kBK / 64;                                 // 32-column chunks per half
+        constexpr int OC = DV / 64;                                  // 32-column O chunks per half
         bool ok = true;
 #pragma unroll 1
         for (int j = 0; j < n_kb && ok; ++j) {
@@ -256,12 +275,13 @@ __global__ void __launch_bounds__(192, 2)
             const int key0 = j * kBK;
             const bool need_mask = (j == qb) || (key0 + kBK > a.seq);
             const int kmax = need_mask ? min(qpos, a.seq - 1) - key0 : kBK - 1;  // last allowed key
-            // pass 1: row maximum (scaled to log2 units)
+            // pass 1: maximum of this half of the row (scaled to log2 units), then of the row
             float mx = -INFINITY;
 #pragma unroll 1
-            for (int c = 0; c < kBK / 32; ++c) {
+            for (int c = 0; c < HC; ++c) {
+                const int col0 = half * 64 + c * 32;
                 uint32_t v[32];
-                tmem_ld32(lane_base + C::S_COL + c * 32, v);
+                tmem_ld32(lane_base + C::S_COL + col0, v);
                 tmem_wait_ld();
                 if (!need_mask) {
 #pragma unroll
@@ -269,10 +289,16 @@ __global__ void __launch_bounds__(192, 2)
                 } else {
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
-                        if (c * 32 + i <= kmax) mx = fmaxf(mx, __uint_as_float(v[i]));
+                        if (col0 + i <= kmax) mx = fmaxf(mx, __uint_as_float(v[i]));
                 }
             }
             mx *= sl;
+            float* slot = mxx + (j & 1) * 256;
+            slot[half * 128 + r] = mx;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xchg[quad]);
+            if (!mbar_wait(&xchg[quad], j & 1, a.flags)) { ok = false; break; }
+            mx = fmaxf(mx, slot[(half ^ 1) * 128 + r]);
             // O (accumulated by P_{j-1} V_{j-1}) is stable once that MMA has completed
             if (j > 0 && !mbar_wait(ofull, (j - 1) & 1, a.flags)) { ok = false; break; }
             tc_fence_after();
@@ -280,25 +306,27 @@ __global__ void __launch_bounds__(192, 2)
                 const float corr = exp2_ftz(m_ref - mx);
                 if (j > 0) {
 #pragma unroll
-                    for (int c = 0; c < DV / 32; ++c) {
+                    for (int c = 0; c < OC; ++c) {
+                        const uint32_t ocol = C::O_COL + half * (DV / 2) + c * 32;
                         uint32_t v[32];
-                        tmem_ld32(lane_base + C::O_COL + c * 32, v);
+                        tmem_ld32(lane_base + ocol, v);
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * corr);
-                        tmem_st32(lane_base + C::O_COL + c * 32, v);
+                        tmem_st32(lane_base + ocol, v);
                     }
                     tmem_wait_st();
                 }
                 l *= corr;
                 m_ref = mx;
             }
-            // pass 2: P = 2^(S*sl - m_ref) in bf16 into the swizzled K-major P buffer
+            // pass 2: P = 2^(S*sl - m_ref) in bf16 into this half's atom of the swizzled P buffer
             float rs = 0.0f;
 #pragma unroll 1
-            for (int c = 0; c < kBK / 32; ++c) {
+            for (int c = 0; c < HC; ++c) {
+                const int col0 = half * 64 + c * 32;
                 uint32_t v[32];
-                tmem_ld32(lane_base + C::S_COL + c * 32, v);
+                tmem_ld32(lane_base + C::S_COL + col0, v);
                 tmem_wait_ld();
                 uint32_t packed[16];
 #pragma unroll
@@ -306,17 +334,16 @@ __global__ void __launch_bounds__(192, 2)
                     float p0 = exp2_ftz(__uint_as_float(v[2 * i]) * sl - m_ref);
                     float p1 = exp2_ftz(__uint_as_float(v[2 * i + 1]) * sl - m_ref);
                     if (need_mask) {
-                        if (c * 32 + 2 * i > kmax) p0 = 0.0f;
-                        if (c * 32 + 2 * i + 1 > kmax) p1 = 0.0f;
+                        if (col0 + 2 * i > kmax) p0 = 0.0f;
+                        if (col0 + 2 * i + 1 > kmax) p1 = 0.0f;
                     }
                     rs += p0 + p1;
                     __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
                     packed[i] = *reinterpret_cast<uint32_t*>(&pb);
                 }
-                uint8_t* arow = arow0 + (c >> 1) * kAtom;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const int phys = ((c & 1) * 4 + q) ^ (r & 7);
+                    const int phys = (c * 4 + q) ^ (r & 7);
                     *reinterpret_cast<uint4*>(arow + phys * 16) =
                         make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
                 }
@@ -332,12 +359,18 @@ __global__ void __launch_bounds__(192, 2)
         }
         if (ok) ok = mbar_wait(ofull, (n_kb - 1) & 1, a.flags);
         tc_fence_after();
-        const float inv = 1.0f / l;
-        bf16* out = static_cast<bf16*>(a.o) + static_cast<size_t>(row0 + qpos) * a.ldo + h * a.dv_out;
+        // the row sum is the two halves' partial sums
+        lxx[half * 128 + r] = l;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&lfin[quad]);
+        if (ok) ok = mbar_wait(&lfin[quad], 0, a.flags);
+        const float inv = ok ? 1.0f / (l + lxx[(half ^ 1) * 128 + r]) : 0.0f;
+        bf16* out = static_cast<bf16*>(a.o) + static_cast<size_t>(row0 + qpos) * a.ldo + h * a.dv_out +
+                    half * (DV / 2);
 #pragma unroll 1
-        for (int c = 0; c < DV / 32; ++c) {
+        for (int c = 0; c < OC; ++c) {
             uint32_t v[32];
-            tmem_ld32(lane_base + C::O_COL + c * 32, v);
+            tmem_ld32(lane_base + C::O_COL + half * (DV / 2) + c * 32, v);
             tmem_wait_ld();
             if (!ok || qpos >= a.seq) continue;
 #pragma unroll
@@ -395,7 +428,7 @@ rdt_status launch_tc(const AttnArgs& a, cudaStream_t st) {
     ta.batch = a.batch;
     ta.sms = num_sms();
     const dim3 grid(static_cast<unsigned>(ta.nqb) * a.hq * a.batch);
-    RDT_CUDA_TRY(launch_pdl(kern, grid, dim3(192), C::SMEM, st, tq, tk, tv, ta));
+    RDT_CUDA_TRY(launch_pdl(kern, grid, dim3(kAttnThreads), C::SMEM, st, tq, tk, tv, ta));
     return RDT_OK;
 }
 
