@@ -15,7 +15,8 @@
 // Absorbed MLA attends over the shared latent key [c_kv ; k_rope] (160 wide) with the value
 // c_kv = the key's first 128 columns, so its V operand is the K tile itself.
 //
-// Roles: warp 0 issues TMA loads (Q once, K two stages ahead, V one stage); warp 1 owns TMEM
+// Roles: warp 0 issues TMA loads (Q once; K one stage and V two, or two stages of the shared
+// latent key for MLA); warp 1 owns TMEM
 // and issues the MMAs (S_{j+1} before P_j V_j); warps 2-9 do the softmax (two warps per 32
 // query rows, one per half of the key block) and write o.
 // Every wait is bounded.
@@ -66,13 +67,16 @@ struct AttnCfg {
     static constexpr int VA = DV / 64;             // 64-wide atoms of the value width
     static constexpr int Q_BYTES = QA * kAtom;
     static constexpr int K_BYTES = QA * kAtom;     // one stage of K (128 keys)
-    static constexpr int KSTAGES = 2;
+    // Separate V: one K stage (K_{j+1} loads once S_j has read K_j, during softmax j) and two
+    // V stages (V_{j+1} loads while P_j V_j runs). Shared latent V (= K): two K stages.
+    static constexpr int KSTAGES = SHARE_KV ? 2 : 1;
+    static constexpr int VSTAGES = SHARE_KV ? 0 : 2;
     static constexpr int V_BYTES = SHARE_KV ? 0 : VA * kAtom;
     static constexpr int P_BYTES = 2 * kAtom;      // 128 x 128 bf16 probabilities
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + KSTAGES * K_BYTES;
-    static constexpr int OFF_P = OFF_V + V_BYTES;
+    static constexpr int OFF_P = OFF_V + VSTAGES * V_BYTES;
     static constexpr int OFF_BAR = OFF_P + P_BYTES;
     static constexpr int OFF_X = OFF_BAR + 256;    // softmax exchange: row maxima [2][2][128], sums [2][128]
     static constexpr int SMEM = OFF_X + 3 * 2 * 128 * 4 + 1024;
@@ -108,8 +112,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     uint64_t* bar_q = bars + 0;
     uint64_t* kfull = bars + 1;    // [2]
     uint64_t* kempty = bars + 3;   // [2]
-    uint64_t* vfull = bars + 5;
-    uint64_t* vempty = bars + 6;
+    auto vfull2 = [bars](int st) { return bars + (st ? 20 : 5); };    // per V stage
+    auto vempty2 = [bars](int st) { return bars + (st ? 21 : 6); };
     uint64_t* sfull = bars + 7;    // S_j in TMEM
     uint64_t* sfree = bars + 8;    // S_j read by the softmax warps
     uint64_t* pfull = bars + 9;    // P_j in shared memory (and O rescaled if needed)
@@ -142,8 +146,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             mbar_init(&kfull[i], 1);
             mbar_init(&kempty[i], 1);
         }
-        mbar_init(vfull, 1);
-        mbar_init(vempty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(vfull2(i), 1);
+            mbar_init(vempty2(i), 1);
+        }
         mbar_init(sfull, 1);
         mbar_init(sfree, 8);
         mbar_init(pfull, 8);
@@ -175,27 +181,32 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
             for (int t = 0; t < C::QA; ++t)
                 tma_load_2d(smem + C::OFF_Q + t * kAtom, &tq, bar_q, h * a.q_hstride + 64 * t, row0 + q0);
-            // K runs one block ahead of V so that S_{j+1} never waits behind the V buffer
+            // K block j goes to stage j % KSTAGES (use j / KSTAGES of it), V block j to stage j & 1
             auto load_k = [&](int j) -> bool {
-                const int s = j & 1;
-                if (!mbar_wait(&kempty[s], ((j >> 1) & 1) ^ 1, a.flags)) return false;
+                const int s = j % C::KSTAGES;
+                if (!mbar_wait(&kempty[s], ((j / C::KSTAGES) & 1) ^ 1, a.flags)) return false;
                 mbar_arrive_expect_tx(&kfull[s], C::K_BYTES);
                 for (int t = 0; t < C::QA; ++t)
                     tma_load_2d(smem + C::OFF_K + s * C::K_BYTES + t * kAtom, &tk, &kfull[s],
                                 g * a.k_hstride + 64 * t, row0 + j * kBK);
                 return true;
             };
+            auto load_v = [&](int j) -> bool {
+                const int s = j & 1;
+                if (!mbar_wait(vempty2(s), ((j >> 1) & 1) ^ 1, a.flags)) return false;
+                mbar_arrive_expect_tx(vfull2(s), C::V_BYTES);
+                for (int t = 0; t < C::VA; ++t)
+                    tma_load_2d(smem + C::OFF_V + s * C::V_BYTES + t * kAtom, &tv, vfull2(s),
+                                g * a.v_hstride + 64 * t, row0 + j * kBK);
+                return true;
+            };
             bool ok = load_k(0);
 #pragma unroll 1
             for (int j = 0; j < n_kb && ok; ++j) {
-                if (j + 1 < n_kb) ok = load_k(j + 1);
-                if (ok && !SHARE_KV) {
-                    if (!mbar_wait(vempty, (j & 1) ^ 1, a.flags)) break;
-                    mbar_arrive_expect_tx(vfull, C::V_BYTES);
-                    for (int t = 0; t < C::VA; ++t)
-                        tma_load_2d(smem + C::OFF_V + t * kAtom, &tv, vfull, g * a.v_hstride + 64 * t,
-                                    row0 + j * kBK);
-                }
+                // V_j first (its stage frees when P_{j-2} V_{j-2} is done, well before S_j),
+                // then K_{j+1} (its stage frees when S_j has read K_j)
+                if (!SHARE_KV) ok = load_v(j);
+                if (ok && j + 1 < n_kb) ok = load_k(j + 1);
             }
         }
     } else if (warp == 1) {
@@ -206,8 +217,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             const uint32_t sp = smem_u32(smem + C::OFF_P);
             bool ok = mbar_wait(bar_q, 0, a.flags);
             auto issue_s = [&](int j) -> bool {
-                const int s = j & 1;
-                if (!mbar_wait(&kfull[s], (j >> 1) & 1, a.flags)) return false;
+                const int s = j % C::KSTAGES;
+                if (!mbar_wait(&kfull[s], (j / C::KSTAGES) & 1, a.flags)) return false;
                 if (!mbar_wait(sfree, (j & 1) ^ 1, a.flags)) return false;
                 tc_fence_after();
                 const uint32_t sk = smem_u32(smem + C::OFF_K + s * C::K_BYTES);
@@ -222,12 +233,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                 return true;
             };
             auto issue_o = [&](int j) -> bool {
-                const int s = j & 1;
+                const int s = SHARE_KV ? j % C::KSTAGES : j & 1;
                 if (!mbar_wait(pfull, j & 1, a.flags)) return false;
-                if (!SHARE_KV && !mbar_wait(vfull, j & 1, a.flags)) return false;
+                if (!SHARE_KV && !mbar_wait(vfull2(s), (j >> 1) & 1, a.flags)) return false;
                 tc_fence_after();
                 const uint32_t sv = SHARE_KV ? smem_u32(smem + C::OFF_K + s * C::K_BYTES)
-                                             : smem_u32(smem + C::OFF_V);
+                                             : smem_u32(smem + C::OFF_V + s * C::V_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk) {
                     const uint32_t offp = (kk >> 2) * kAtom + (kk & 3) * 32;
@@ -238,7 +249,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                 if (SHARE_KV)
                     tc_commit(&kempty[s]);
                 else
-                    tc_commit(vempty);
+                    tc_commit(vempty2(s));
                 return true;
             };
             if (ok) ok = issue_s(0);
