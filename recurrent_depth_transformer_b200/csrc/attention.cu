@@ -260,11 +260,13 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnArgs a) {
 template <int DQK, int DV>
 rdt_status launch_bf16(const AttnArgs& a, cudaStream_t st) {
     constexpr int smem = (kBM * (DQK + 8) + 2 * kBN * (DQK + 8) + 2 * kBN * (DV + 8)) * 2;
-    static bool configured = false;
-    if (!configured) {
+    static int configured[64] = {};        // per device: function attributes are set per device
+    int dev = 0;
+    RDT_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64 || !configured[dev]) {
         RDT_CUDA_TRY(cudaFuncSetAttribute(attn_bf16_kernel<DQK, DV>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-        configured = true;
+        if (dev >= 0 && dev < 64) configured[dev] = 1;
     }
     const dim3 grid((a.seq + kBM - 1) / kBM, a.hq, a.batch);
     RDT_CUDA_TRY(launch_pdl(attn_bf16_kernel<DQK, DV>, grid, dim3(128), smem, st, a));

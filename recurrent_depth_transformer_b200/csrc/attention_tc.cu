@@ -409,11 +409,13 @@ template <int DQK, int DV, bool SHARE_KV>
 rdt_status launch_tc(const AttnArgs& a, cudaStream_t st) {
     using C = AttnCfg<DQK, DV, SHARE_KV>;
     auto kern = attn_tc_kernel<DQK, DV, SHARE_KV>;
-    static bool configured = false;
-    if (!configured) {
+    static int configured[64] = {};        // per device: function attributes are set per device
+    int dev = 0;
+    RDT_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64 || !configured[dev]) {
         RDT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
         RDT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
-        configured = true;
+        if (dev >= 0 && dev < 64) configured[dev] = 1;
     }
     const long rows = static_cast<long>(a.batch) * a.seq;
     CUtensorMap tq, tk, tv;
