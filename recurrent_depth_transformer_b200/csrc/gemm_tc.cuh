@@ -226,11 +226,50 @@ __device__ __forceinline__ void epilogue_topk(const EpiParams& p, uint32_t taddr
     tk.write(p, crow);
 }
 
+// Operands of an epilogue that do not depend on the accumulator: loaded before the epilogue
+// warps wait for it (they are idle during the tile's MMAs), so that their memory round trip
+// is not added to the tile's exposed tail.
+struct EpiPre {
+    float cs[32], sn[32];   // RoPE: cos / sin of the row's position, one per rotary pair
+    int token;              // scatter: the row's token (-1: padding row) and gate weight
+    float w;
+};
+
+template <int KIND>
+__device__ __forceinline__ void epilogue_pre(const EpiParams& p, int lane, int nvalid, int row0, EpiPre& pre) {
+    if constexpr (KIND == EPI_ROPE) {
+        // The angle tables are [rot/2][seq]: for a fixed frequency the lanes (consecutive
+        // positions) read consecutive floats.
+        const int pos = (row0 + lane) % p.seq;
+        const int half = p.rot_dim / 2;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            pre.cs[i] = i < half ? p.rope_cos[static_cast<size_t>(i) * p.seq + pos] : 0.0f;
+            pre.sn[i] = i < half ? p.rope_sin[static_cast<size_t>(i) * p.seq + pos] : 0.0f;
+        }
+    } else if constexpr (KIND == EPI_SCATTER) {
+        // Row r of the tile is expert output for token row_token[r] with gate weight row_w[r]
+        // (shared experts: every token, weight 1)
+        pre.token = -1;
+        pre.w = 0.0f;
+        if (lane < nvalid) {
+            const int crow = row0 + lane;
+            if (crow < p.shared_rows) {
+                pre.token = crow % p.ntok;
+                pre.w = 1.0f;
+            } else {
+                pre.token = p.row_token[crow - p.shared_rows];
+                pre.w = p.row_w[crow - p.shared_rows];
+            }
+        }
+    }
+}
+
 // One epilogue warp's share of a tile: rows row0 .. row0 + 31 of C (lane l owns row
 // row0 + l in TMEM, the first nvalid of them are real), columns n0 .. n0 + BN - 1.
 template <typename T, int BN, int KIND>
-__device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, float* stg, int lane,
-                                         int nvalid, int row0, int n0, int split = 1, int mtile = 0) {
+__device__ __forceinline__ void epilogue(const EpiParams& p, const EpiPre& pre, uint32_t taddr, float* stg,
+                                         int lane, int nvalid, int row0, int n0, int split = 1, int mtile = 0) {
     const int cc = (lane & 7) * 4;                 // this lane's columns after the transpose
     if constexpr (KIND == EPI_STORE || KIND == EPI_STORE_F32 || KIND == EPI_OPROJ_PLAIN) {
         using OutT = std::conditional_t<KIND == EPI_STORE, T, float>;
@@ -245,19 +284,12 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, flo
     } else if constexpr (KIND == EPI_ROPE) {
         // Heads of width head_w tile the BN columns exactly (host checks BN % head_w == 0).
         // The rotation pairs columns i and i + rot/2 of a head, so it runs row-per-lane
-        // (before the transpose). The angle tables are [rot/2][seq]: for a fixed frequency
-        // the lanes (consecutive positions) read consecutive floats.
-        const int pos = (row0 + lane) % p.seq;
+        // (before the transpose), with the row's angles loaded before the accumulator wait.
         const int hw_chunks = p.head_w / 32;
         const int rc0 = p.rot_off / 32;
         const int rch = p.rot_dim / 32;
-        const int half = p.rot_dim / 2;
-        float cs[32], sn[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            cs[i] = i < half ? p.rope_cos[static_cast<size_t>(i) * p.seq + pos] : 0.0f;
-            sn[i] = i < half ? p.rope_sin[static_cast<size_t>(i) * p.seq + pos] : 0.0f;
-        }
+        const float* cs = pre.cs;
+        const float* sn = pre.sn;
         T* out = static_cast<T*>(p.out) + static_cast<size_t>(row0) * p.ldo;
 #pragma unroll 1
         for (int hc = 0; hc < BN / 32; hc += hw_chunks) {
@@ -341,20 +373,10 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, uint32_t taddr, flo
             store_chunk(stg, lane, g, out + c * 32, p.ldo, nvalid);
         }
     } else if constexpr (KIND == EPI_SCATTER) {
-        // Row r of the tile is expert output for token row_token[r] with gate weight row_w[r]
-        // (shared experts: every token, weight 1); it is added into h_next with vector atomics.
-        int token = -1;
-        float w = 0.0f;
-        if (lane < nvalid) {
-            const int crow = row0 + lane;
-            if (crow < p.shared_rows) {
-                token = crow % p.ntok;
-                w = 1.0f;
-            } else {
-                token = p.row_token[crow - p.shared_rows];
-                w = p.row_w[crow - p.shared_rows];
-            }
-        }
+        // Row r of the tile (token and gate weight loaded before the accumulator wait) is added
+        // into h_next with vector atomics.
+        const int token = pre.token;
+        const float w = pre.w;
         int tok[8];
         float wt[8];
 #pragma unroll
@@ -671,9 +693,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t use = static_cast<uint32_t>(local >> 1);
             const TileCoord tc = tile_coord(args, gt, tile, n_ntiles, BN, split, num_kb, kTileRows);
             const int nvalid = min(32, max(0, tc.nrows - row_off));
+            EpiPre pre;
+            epilogue_pre<KIND>(epi, lane, nvalid, tc.c_row0 + row_off, pre);
             if (!mbar_wait(&tfull[b], use & 1, epi.flags)) break;
             tc_fence_after();
-            epilogue<T, BN, KIND>(epi, tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN, stg, lane,
+            epilogue<T, BN, KIND>(epi, pre, tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN, stg, lane,
                                   nvalid, tc.c_row0 + row_off, tc.n0, split, tc.mt);
             tc_fence_before();
             __syncwarp();
