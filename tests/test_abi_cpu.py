@@ -73,3 +73,31 @@ def test_configs_of_all_workloads_validate_shapes():
     for wl in WORKLOADS:
         c = R.make_config(wl, max_loops=max(wl.loops))
         assert c.batch * c.seq == wl.tokens
+
+
+def test_ctypes_structs_match_the_header(tmp_path):
+    """Every field offset and struct size of the ctypes mirrors in the binding equals the C
+    compiler's for include/rdt.h (a field added on one side only would shift the others)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    mirrors = {"rdt_config": R.RdtConfig, "rdt_weights": R.RdtWeights, "rdt_diag": R.RdtDiag,
+               "rdt_kernel_stat": R.RdtKernelStat}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HDR}"', "int main(void) {"]
+    for cname, py in mirrors.items():
+        lines.append(f'    printf("{cname} size %zu\\n", sizeof({cname}));')
+        for field, _ in py._fields_:
+            lines.append(f'    printf("{cname} {field} %zu\\n", offsetof({cname}, {field}));')
+    lines += ["    return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c11", str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {tuple(l.split()[:2]): int(l.split()[2]) for l in out if l.strip()}
+    for cname, py in mirrors.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for field, _ in py._fields_:
+            assert got[(cname, field)] == getattr(py, field).offset, (cname, field)
