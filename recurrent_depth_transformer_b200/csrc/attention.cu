@@ -4,8 +4,10 @@
 // absorbed MLA). The score is never materialised in memory: keys are consumed in blocks
 // with a running row maximum and row sum (online softmax).
 //
-// bf16: 64 query rows per CTA (16 per warp), 64-key blocks double-buffered in shared
-// memory with cp.async, QK^T and PV on mma.sync m16n8k16 (bf16 in, fp32 accumulate).
+// bf16 head widths that the tcgen05 kernel (attention_tc.cu: 64/64, and the shared latent
+// 160/128) does not cover run here: 64 query rows per CTA (16 per warp), 64-key blocks
+// double-buffered in shared memory with cp.async, QK^T and PV on mma.sync m16n8k16 (bf16 in,
+// fp32 accumulate).
 // Causal blocks above the diagonal are skipped; CTAs with the most key blocks start first.
 // fp32: one thread per query row (the tiny fp32 configuration only).
 #include "rdt_internal.cuh"

@@ -59,8 +59,8 @@ struct rdt_handle {
     int router_split = 1;          // K split of the router GEMM over CTAs
     float* logits = nullptr;       // [N, E] partial-logit accumulator of the split router
     int* tile_count = nullptr;     // per row-tile arrival counters of the split router
-    // output tile widths of the projection and expert GEMMs (128 or 256), and whether each
-    // runs on CTA pairs (256-row tiles) or single CTAs (128-row tiles)
+    // output tile widths of the projection and expert GEMMs (128, 192 on pairs, or 256), and
+    // whether each runs on CTA pairs (256-row tiles) or single CTAs (128-row tiles)
     int bn_qkv = 128, bn_o = 128, bn_up = 128, bn_down = 128;
     int pair_qkv = 0, pair_o = 0, pair_up = 0, pair_down = 0;
     int split_down = 1;            // K split of the expert down-projection (linear epilogue)

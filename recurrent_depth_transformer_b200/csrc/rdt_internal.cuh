@@ -451,7 +451,7 @@ struct GemmArgs {
 rdt_status gemm_tc(bool bf16_elems, int bn, const CUtensorMap& tA, const CUtensorMap& tB,
                    const CUtensorMap* tA2, const CUtensorMap* tB2, const GemmArgs& args,
                    const EpiParams& epi, cudaStream_t st);
-// The pair-tile instantiations (bf16, BN 128 or 256, every epilogue but the router's).
+// The pair-tile instantiations (bf16, BN 128, 192 or 256, every epilogue but the router's).
 rdt_status gemm_tc_pair(int bn, const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap* tA2,
                         const CUtensorMap* tB2, const GemmArgs& args, const EpiParams& epi,
                         cudaStream_t st);
