@@ -13,6 +13,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "rdt_internal.cuh"
 
 namespace rdt {
@@ -152,8 +154,18 @@ rdt_status prof_flush(rdt_handle* h) {
     return RDT_OK;
 }
 
+// Every launch of a kernel class is bracketed by an NVTX range named after the class (host
+// side: visible to a timeline tool on eager calls and during graph capture) and, when
+// profiling is on, by CUDA events.
+struct NvtxRange {   // pushed for a scope, popped on every way out of it
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 #define TIMED(h, kind, n, st, expr)                \
     do {                                           \
+        NvtxRange nvtx_range_(kKindName[(kind)]);  \
         RDT_TRY(prof_begin((h), (kind), (n), (st))); \
         RDT_TRY(expr);                             \
         RDT_TRY(prof_end((h), (st)));              \
@@ -953,6 +965,7 @@ rdt_status loop_impl(rdt_handle* h, const void* h0, const void* e, int T, float*
     if (c.b_kind == RDT_B_DENSE) TIMED(h, K_DENSE_B, 1, st, matmul_nt_simt(h->bf, e, h->Bw, h->Be, N, d, d, st));
     if (h->tr_h) RDT_CUDA_TRY(cudaMemcpyAsync(h->tr_h, h->hbuf[0], nd * 4, cudaMemcpyDeviceToDevice, st));
     for (int t = 0; t < T; ++t) {
+        NvtxRange loop_range("rdt loop");
         float* hcur = h->hbuf[t & 1];
         float* hnext = (t == T - 1) ? out : h->hbuf[(t + 1) & 1];
         RDT_TRY(attention_block(h, hcur, c.inject_e ? e : nullptr, t, true, nullptr, hnext, st));

@@ -157,6 +157,21 @@ def test_moe_sublayer_and_router_exactness():
         assert_close(got, fo, max_abs=2e-2, rel_fro=1e-2, what=f"moe {wl.name}")
 
 
+def test_moe_token_permutation_equivariance():
+    """Routing and the expert rows are per token: permuting the tokens permutes the MoE
+    output (only the fp32 order of the k reductions into a row may differ)."""
+    torch = torch_mod()
+    wl = C1.replace(batch=1, seq=256)
+    inputs = generate(wl)
+    y = inputs["e"].astype(np.float32) * 3.0
+    perm = np.random.default_rng(7).permutation(wl.seq)
+    with handle(wl, inputs) as h:
+        f1 = h.moe_forward(torch.from_numpy(y).cuda()).cpu().numpy()
+        f2 = h.moe_forward(torch.from_numpy(np.ascontiguousarray(y[:, perm])).cuda()).cpu().numpy()
+    ma, _ = errors(f2, f1[:, perm])
+    assert ma < 1e-4, ma
+
+
 def test_T1_equals_sublayer_composition():
     torch = torch_mod()
     wl = C1.replace(batch=1, seq=256)
