@@ -174,9 +174,9 @@ struct TopK {
 };
 
 // Router epilogue. Unsplit: the thread's row holds all logits (BN >= n_exp) in TMEM.
-// Split over K: every CTA adds its partial logits into p.logits; the CTA that arrives last
-// on the row tile's counter (threadfence-reduction order: adds, fence, count) reads the
-// complete rows back and selects.
+// Split over K: every CTA adds its partial logits into p.logits; for each 32 rows, the warp
+// that arrives last on their counter (threadfence-reduction order: adds, fence, count) reads
+// the complete rows back and selects.
 template <int BN, int KMAX>
 __device__ __forceinline__ void epilogue_topk(const EpiParams& p, uint32_t taddr, bool valid, int crow,
                                               int split, int mtile) {
@@ -195,7 +195,6 @@ __device__ __forceinline__ void epilogue_topk(const EpiParams& p, uint32_t taddr
         if (valid) tk.write(p, crow);
         return;
     }
-    __shared__ int s_last;
     float* lrow = p.logits + static_cast<size_t>(crow) * p.n_exp;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
@@ -208,15 +207,19 @@ __device__ __forceinline__ void epilogue_topk(const EpiParams& p, uint32_t taddr
             if (ex < p.n_exp) atomicAdd(lrow + ex, v[i]);
         }
     }
+    // Each warp elects alone, on the counter of its 32 rows (no barrier between warps, so a
+    // warp that left on a timeout cannot stall the others): adds, fence, count.
     __threadfence();
-    asm volatile("bar.sync 1, 128;" ::: "memory");     // the four epilogue warps
-    if (threadIdx.x == 64) {
-        const int old = atomicAdd(p.tile_count + mtile, 1);
-        s_last = old == split - 1;
-        if (s_last) p.tile_count[mtile] = 0;             // ready for the next launch
+    __syncwarp();
+    const int lane = threadIdx.x & 31;
+    const int quad = (threadIdx.x >> 5) & 3;
+    int last = 0;
+    if (lane == 0) {
+        int* cnt = p.tile_count + mtile * 4 + quad;
+        last = atomicAdd(cnt, 1) == split - 1;
+        if (last) *cnt = 0;                              // ready for the next launch
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (!s_last) return;
+    if (!__shfl_sync(0xffffffffu, last, 0)) return;
     __threadfence();
     if (!valid) return;
     TopK<KMAX> tk;

@@ -60,7 +60,7 @@ struct rdt_handle {
     int bn_router = 64;
     int router_split = 1;          // K split of the router GEMM over CTAs
     float* logits = nullptr;       // [N, E] partial-logit accumulator of the split router
-    int* tile_count = nullptr;     // per row-tile arrival counters of the split router
+    int* tile_count = nullptr;     // arrival counters of the split router, per 32 rows of a row tile
     // output tile widths of the projection and expert GEMMs (128, 192 on pairs, or 256), and
     // whether each runs on CTA pairs (256-row tiles) or single CTAs (128-row tiles)
     int bn_qkv = 128, bn_o = 128, bn_up = 128, bn_down = 128;
@@ -613,7 +613,7 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
             if (kb % sp == 0 && static_cast<long>(mt) * sp <= num_sms()) split = sp;
         h->router_split = split;
         RDT_TRY(dev_alloc(h, &h->logits, static_cast<size_t>(N) * E * 4, true));
-        RDT_TRY(dev_alloc(h, &h->tile_count, static_cast<size_t>(mt) * 4, true));
+        RDT_TRY(dev_alloc(h, &h->tile_count, static_cast<size_t>(mt) * 4 * 4, true));   // per 32 rows
     }
     RDT_TRY(dev_alloc(h, &h->idx, static_cast<size_t>(N) * K * 4));
     RDT_TRY(dev_alloc(h, &h->wts, static_cast<size_t>(N) * K * 4));

@@ -424,7 +424,8 @@ struct EpiParams {
     int32_t* trace_idx;    // optional copies
     float* trace_w;
     float* logits;         // split-K router: [ntok, n_exp] fp32 partial sums (zeroed beforehand)
-    int* tile_count;       // split-K router: per row-tile arrival counters (zero, reset after use)
+    int* tile_count;       // split-K router: arrival counters per (row tile, 32-row quadrant)
+                           // (zero, reset after use)
     int* flags;            // device status words
 };
 
