@@ -4,4 +4,5 @@ from .rdt_oracle import (rmsnorm, rope_angles, apply_rope, silu, swiglu_ffn, cau
                          gqa_attention, router_topk, moe_combine, attention_sublayer,
                          moe_sublayer, loop_forward, loop_step_rows, input_injection,
                          spectral_radius, mla_attention_explicit, mla_attention_absorbed,
-                         LoopTrace, Routing, NEAR_TIE)
+                         LoopTrace, Routing, NEAR_TIE, NEAR_HALT, halting_probability,
+                         loop_forward_act, ActResult)

@@ -42,7 +42,15 @@ design notes of the repository):
 * depth-wise LoRA: W_t = W + B_t A_t on the Q and O projections, adapter
   min(t, L - 1) at loop t;
 * MLA: latent RMSNorms on c_q and c_kv, decoupled RoPE key shared by all
-  heads, score scale 1/sqrt(nope + rope).
+  heads, score scale 1/sqrt(nope + rope);
+* ACT halting ([TB] names it; [GS] troubleshooting item 4 gives the 0.99
+  threshold and that a position leaves once its accumulated halting probability
+  reaches it): halting head p = sigmoid(w . h_{t+1} + b) on the new state;
+  a position halts at the first loop where its running sum of p reaches the
+  threshold (or at the last loop), taking the remainder 1 - (sum before) as
+  that loop's weight; the output is the weighted sum of its states; a halted
+  position keeps its state and still serves as a key, and is routed to no
+  expert.
 
 Parity status: every function below is pinned by ``tests/test_oracle_pins.py``
 (closed forms, library special cases, hand-computed fixtures, identities).
@@ -56,6 +64,7 @@ import numpy as np
 
 F = np.float64
 NEAR_TIE = 1.0e-3          # logit gap under which the oracle may follow the GPU's routing
+NEAR_HALT = 1.0e-2         # |sum of p - threshold| under which it may follow the GPU's halting
 ATTN_QBLOCK = 1024         # query rows per block when evaluating long sequences
 
 
@@ -412,3 +421,98 @@ def loop_step_rows(h, e, W, cfg, t: int, rows: Sequence[Tuple[int, int]],
     Be = input_injection(e[bidx, sidx], W["B"])
     h_next = A * h[bidx, sidx] + Be + a_rows + f
     return h_next, r, st
+
+
+# --------------------------------------------------------------------------------------
+# ACT halting inside the loop
+# --------------------------------------------------------------------------------------
+
+def halting_probability(h, w_halt, b_halt) -> np.ndarray:
+    """p = sigmoid(h . w_halt + b_halt) over the last axis: the halting head. [TB] names
+    ACT halting and [GS] troubleshooting item 4 its threshold, but neither gives the head;
+    this is the plainest one, a linear map of the state to one logit."""
+    z = _f(h) @ _f(w_halt) + F(b_halt)
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+@dataclass
+class ActResult:
+    out: np.ndarray          # [B, S, d]: sum over t of weights[t] * h_{t+1}
+    n_loops: np.ndarray      # [B, S]: loops each position ran (its halting loop, 1-based)
+    weights: np.ndarray      # [T, B, S]: weight of h_{t+1} in out (sums to 1 over t)
+    stats: Dict[str, int]
+
+
+def loop_forward_act(h0, e, T: int, W, cfg, w_halt, b_halt: float, threshold: float,
+                     follow: Optional[Sequence[np.ndarray]] = None,
+                     follow_loops: Optional[np.ndarray] = None,
+                     trace: Optional[LoopTrace] = None, mla_form: str = "explicit") -> ActResult:
+    """The loop of :func:`loop_forward` with ACT halting per position ([TB] "Dynamic
+    Adaptive Computation Time"; [GS] troubleshooting item 4, act_threshold = 0.99).
+
+    At loop t every position computes attention as usual (a halted position keeps its
+    state, so its keys and values are those of its last state); positions still running
+    are routed through the MoE and update h_{t+1} = A.h_t + B.e + a + f, halted ones keep
+    h_{t+1} = h_t. Then each running position takes p_t = sigmoid(w . h_{t+1} + b); with
+    c the sum of its earlier p, it halts at this loop if c + p_t >= threshold or t = T - 1,
+    and h_{t+1} enters the output with weight 1 - c (the remainder); otherwise with weight
+    p_t, and c grows by p_t.
+
+    ``follow[t]`` ([N, k]) is another implementation's routing, adopted on near-ties as in
+    :func:`moe_sublayer`; ``follow_loops`` ([B, S]) its halting loops, adopted where
+    |c + p_t - threshold| <= NEAR_HALT; every other difference is counted in ``stats``.
+    """
+    A = _f(W["A"])
+    e = _f(e)
+    Be = input_injection(e, W["B"])
+    h = _f(h0)
+    bs = h.shape[:2]
+    cum = np.zeros(bs, dtype=F)
+    halted = np.zeros(bs, dtype=bool)
+    n_loops = np.zeros(bs, dtype=np.int64)
+    out = np.zeros_like(h)
+    weights = np.zeros((T,) + bs, dtype=F)
+    stats = {"near_ties": 0, "mismatch": 0, "near_halts": 0, "halt_mismatch": 0}
+    theirs_loops = None if follow_loops is None else np.asarray(follow_loops).reshape(bs)
+    if trace is not None:
+        trace.h.append(h.copy())
+    for t in range(T):
+        x = h + e if cfg.inject_e else h
+        a = attention_sublayer(x, W, cfg, t, mla_form)
+        y = x + a
+        run = ~halted
+        f = np.zeros_like(y)
+        if run.any():
+            fi = None
+            if follow is not None:
+                fi = np.asarray(follow[t]).reshape(bs + (-1,))[run]
+            f_run, r, st = moe_sublayer(y[run], W, cfg, fi)
+            f[run] = f_run
+            stats["near_ties"] += st["near_ties"]
+            stats["mismatch"] += st["mismatch"]
+        h_new = A * h + Be + a + f
+        h_new[halted] = h[halted]                       # a halted position keeps its state
+        p = halting_probability(h_new, w_halt, b_halt)
+        reach = cum + p
+        if t == T - 1:
+            stop = run.copy()
+        else:
+            stop = run & (reach >= threshold)
+            if theirs_loops is not None:
+                theirs = run & (theirs_loops == t + 1)
+                near = run & (np.abs(reach - threshold) <= NEAR_HALT)
+                stats["near_halts"] += int(np.count_nonzero(near & (theirs != stop)))
+                stats["halt_mismatch"] += int(np.count_nonzero(~near & (theirs != stop)))
+                stop = np.where(near, theirs, stop)
+        w = np.where(stop, 1.0 - cum, np.where(run, p, 0.0))
+        out += w[..., None] * h_new
+        weights[t] = w
+        cum = np.where(run, reach, cum)
+        n_loops[stop] = t + 1
+        halted |= stop
+        h = h_new
+        if trace is not None:
+            trace.h.append(h.copy())
+            trace.attn.append(a)
+            trace.moe.append(f)
+    return ActResult(out=out, n_loops=n_loops, weights=weights, stats=stats)

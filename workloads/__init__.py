@@ -26,6 +26,11 @@ Recipe (fixed draw order, ``numpy.random.Generator(PCG64(seed))``):
 Draws are float32; for bf16 workloads every drawn tensor except ``A`` and
 ``B`` (which stay fp32, as the state arithmetic does) is rounded to the
 nearest bf16 (ties to even) once, here.
+
+The ACT halting head (:func:`act_head`) is drawn from a stream of its own, so
+that adding it changes none of the draws above: ``w_halt`` ~ N(0, scale^2 / dim)
+(fp32, a random direction of length about ``scale``), ``b_halt`` fixed, and the
+threshold 0.99 of the getting-started page (troubleshooting item 4).
 """
 from __future__ import annotations
 
@@ -38,7 +43,7 @@ import numpy as np
 
 __all__ = [
     "Workload", "WORKLOADS", "by_name", "generate", "round_bf16", "bf16_bits",
-    "WEIGHT_ORDER_GQA", "WEIGHT_ORDER_MLA", "weight_shapes",
+    "WEIGHT_ORDER_GQA", "WEIGHT_ORDER_MLA", "weight_shapes", "act_head", "ACT_THRESHOLD",
 ]
 
 # u range that makes A = exp(-exp(u)) <= 0.95 exactly at the upper end.
@@ -252,3 +257,16 @@ def prefix(inputs: Dict[str, np.ndarray], n_tok: int) -> Dict[str, np.ndarray]:
     d["e"] = np.ascontiguousarray(inputs["e"][:, :n_tok])
     d["h0"] = np.ascontiguousarray(inputs["h0"][:, :n_tok])
     return d
+
+
+ACT_THRESHOLD = 0.99
+
+
+def act_head(wl: Workload, *, scale: float = 0.5, bias: float = -1.0,
+             seed: Optional[int] = None) -> Dict[str, object]:
+    """Halting head of the ACT loop: ``w_halt`` [dim] fp32 ~ N(0, scale^2 / dim),
+    ``b_halt`` = bias, ``threshold`` = 0.99. Drawn from the PCG64 stream keyed by
+    (seed, 1), apart from :func:`generate`'s."""
+    rng = np.random.Generator(np.random.PCG64([wl.seed if seed is None else seed, 1]))
+    w = _normal(rng, (wl.dim,), 0.0, scale / math.sqrt(wl.dim))
+    return {"w_halt": w, "b_halt": float(bias), "threshold": ACT_THRESHOLD}
