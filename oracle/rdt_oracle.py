@@ -64,7 +64,7 @@ import numpy as np
 
 F = np.float64
 NEAR_TIE = 1.0e-3          # logit gap under which the oracle may follow the GPU's routing
-NEAR_HALT = 1.0e-2         # |sum of p - threshold| under which it may follow the GPU's halting
+NEAR_HALT = 2.0e-2         # |sum of p - threshold| under which it may follow the GPU's halting
 ATTN_QBLOCK = 1024         # query rows per block when evaluating long sequences
 
 
