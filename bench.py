@@ -6,12 +6,14 @@ dim 1024, 16/4 heads of 64, 16 experts top-2, SwiGLU hidden 1024, bf16 storage, 
 state) on seeded synthetic inputs resident in HBM. The L2 cache is flushed (256 MiB
 write) before every timed step; each step is timed with CUDA events on its stream.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--act]
 
 N > 1 runs under torchrun: every rank runs its own full replica (no data-path
 collective; weak scaling); the timed region is bracketed by a barrier and a device
 synchronise, and the step time is the maximum over ranks. `--impl reference` times the
-fp64 CPU oracle on the host cores instead (rank 0 only).
+fp64 CPU oracle on the host cores instead (rank 0 only). `--act` times the same workload
+through rdt_loop_forward_act (ACT halting, threshold 0.99, the seeded halting head) and
+reports the halting histogram; its tokens·loops count the T = 8 loops asked for.
 """
 from __future__ import annotations
 
@@ -44,7 +46,7 @@ KERNEL_SOURCES = {"gemm_up": ("recurrent_depth_transformer_b200/csrc/gemm_tc.cuh
                               "recurrent_depth_transformer_b200/csrc/gemm_tc_pair.cu",
                               "recurrent_depth_transformer_b200/csrc/rdt_internal.cuh",
                               "recurrent_depth_transformer_b200/csrc/rdt_api.cu")}
-MEASURED_TRAFFIC = {"gemm_up": (79.729408e6 + 3.210752e6, "f3068fc2162c5a13")}
+MEASURED_TRAFFIC = {"gemm_up": (79.72864e6 + 2.450688e6, "fcd18f1020880b27")}
 
 
 def source_fingerprint(files):
@@ -316,8 +318,18 @@ def run_gpu(args):
     stream = torch.cuda.current_stream()
     N = wl.batch * wl.seq
 
-    def step():
-        h.loop_forward(e, e, LOOPS, out=out)
+    nl = None
+    if args.act:
+        from workloads import act_head
+        head = act_head(wl)
+        h.set_act(torch.from_numpy(head["w_halt"]).to(dev), head["b_halt"], head["threshold"])
+        nl = torch.empty((wl.batch, wl.seq), dtype=torch.int32, device=dev)
+
+        def step():
+            h.loop_forward_act(e, e, LOOPS, out=out, n_loops=nl)
+    else:
+        def step():
+            h.loop_forward(e, e, LOOPS, out=out)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -359,6 +371,8 @@ def run_gpu(args):
     h.profile(False)
 
     # ---- end to end through the host-buffer entry point (pinned memory, copies inside)
+    if args.act:
+        return act_line(args, h, wl, nl, value, ms, world, rank, stats, launches, clocks)
     e_host = e.cpu().pin_memory()
     out_host = torch.empty(out.shape, dtype=torch.float32).pin_memory()
     for _ in range(3):                       # eager, graph capture, first replay
@@ -441,6 +455,40 @@ def run_gpu(args):
     return 0
 
 
+def act_line(args, h, wl, nl, value, ms, world, rank, stats, launches, clocks):
+    """The line of the ACT leg: device-timed throughput and the halting histogram."""
+    import numpy as np
+    import torch.distributed as dist
+    loops = nl.cpu().numpy().ravel()
+    diag = h.diagnostics()
+    if rank == 0:
+        tot = max(sum(v[1] for v in stats.values()), 1e-12)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "ours+act",
+            "config": {"workload": WORKLOAD + "+act", "batch": wl.batch, "seq": wl.seq, "dim": wl.dim,
+                       "loops": LOOPS, "tokens_per_step": wl.batch * wl.seq,
+                       "act": {"threshold": 0.99, "head": "w ~ N(0, 0.25/dim), b = -1"},
+                       "l2": "flushed before every timed step (256 MiB write)"},
+            "act": {"mean_loops": float(loops.mean()),
+                    "hist": np.bincount(loops, minlength=LOOPS + 1)[1:].tolist(),
+                    "loops_run_fraction": float(loops.mean() / LOOPS)},
+            "e2e": None,
+            "gpu_launches": int(launches),
+            "clocks": clocks,
+            "kernels": {k: {"launches_per_step": n / args.steps, "ms_per_step": t / args.steps,
+                            "share": t / tot} for k, (n, t) in stats.items()},
+            "finite": diag["nonfinite"] == 0 and diag["timeout"] == 0,
+        }
+        print(json.dumps(line), flush=True)
+    h.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -449,6 +497,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--act", action="store_true", help="time the ACT halting loop instead")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

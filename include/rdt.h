@@ -178,6 +178,37 @@ rdt_status rdt_loop_forward(rdt_handle* h, const void* h0, const void* e, int T,
 rdt_status rdt_loop_forward_host(rdt_handle* h, const void* h0_host, const void* e_host, int T,
                                  float* out_host, void* stream);
 
+/* ACT halting ("Dynamic Adaptive Computation Time" halting, techbriefly article on
+ * the OpenMythos project; act_threshold = 0.99, getting-started page
+ * "Introducao ao OpenMythos", troubleshooting item 4: a position leaves the
+ * loop once its accumulated halting probability reaches the threshold). The
+ * pages give no halting head; this one is a linear map of the state to one
+ * logit: p_t = sigmoid(w_halt . h_{t+1} + b_halt).
+ *
+ * rdt_set_act sets the head of a handle: copies w_halt (device fp32 [dim],
+ * 16-byte aligned; the caller may free it on return), keeps b_halt and the
+ * threshold. Synchronises `stream`. INVALID_ARG for a NULL w_halt, a
+ * non-finite b_halt or a threshold outside (0, 1]; UNSUPPORTED when dim is
+ * not a multiple of 128; OOM if its small workspace (dim + 2 N words) cannot
+ * be allocated. */
+rdt_status rdt_set_act(rdt_handle* h, const float* w_halt, float b_halt, float threshold,
+                       void* stream);
+
+/* The looped block with ACT halting per position. Each loop runs the block for
+ * every position (attention sees every position's current state); positions
+ * still running are routed through the MoE and updated as in rdt_loop_forward,
+ * halted positions keep their state and are routed to no expert. After loop t
+ * a running position with earlier halting probabilities summing to c takes
+ * p_t; it halts at loop t if c + p_t >= threshold or t = T - 1, and h_{t+1}
+ * enters the output with weight 1 - c; otherwise with weight p_t.
+ *   h0, e   : device [N, dim] in cfg.dtype (h0 may alias e)
+ *   T       : 1 .. cfg.max_loops (INVALID_ARG otherwise)
+ *   out     : device fp32 [N, dim] = sum over t of weight_t * h_{t+1}
+ *   n_loops : device int32 [N] (16-byte aligned) or NULL: loops each position ran
+ * INVALID_ARG if rdt_set_act has not been called on the handle. */
+rdt_status rdt_loop_forward_act(rdt_handle* h, const void* h0, const void* e, int T, float* out,
+                                int32_t* n_loops, void* stream);
+
 /* Per-loop trace for parity checks (all device pointers, or NULL to disable):
  *   idx    : int32 [max_loops, N, top_k] routing of every loop
  *   w      : fp32  [max_loops, N, top_k] gate weights of every loop

@@ -34,7 +34,8 @@ STATUS = {0: "RDT_OK", 1: "RDT_ERR_INVALID_ARG", 2: "RDT_ERR_UNSUPPORTED", 3: "R
 EXPORTED = ("rdt_create", "rdt_attn_forward", "rdt_moe_forward", "rdt_loop_forward",
             "rdt_loop_forward_host", "rdt_set_trace", "rdt_get_diagnostics", "rdt_memory_bytes",
             "rdt_status_string", "rdt_last_error", "rdt_destroy", "rdt_matmul", "rdt_attention",
-            "rdt_profile", "rdt_profile_read", "rdt_moe_route_noalloc")
+            "rdt_profile", "rdt_profile_read", "rdt_moe_route_noalloc", "rdt_set_act",
+            "rdt_loop_forward_act")
 
 
 class RdtError(RuntimeError):
@@ -92,6 +93,8 @@ def load_library() -> ctypes.CDLL:
     lib.rdt_loop_forward.argtypes = [vp, vp, vp, i32, vp, vp]
     lib.rdt_loop_forward_host.argtypes = [vp, vp, vp, i32, vp, vp]
     lib.rdt_set_trace.argtypes = [vp, vp, vp, vp]
+    lib.rdt_set_act.argtypes = [vp, vp, ctypes.c_float, ctypes.c_float, vp]
+    lib.rdt_loop_forward_act.argtypes = [vp, vp, vp, i32, vp, vp, vp]
     lib.rdt_get_diagnostics.argtypes = [vp, ctypes.POINTER(RdtDiag)]
     lib.rdt_memory_bytes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t)]
     lib.rdt_status_string.argtypes = [i32]
@@ -110,7 +113,8 @@ def load_library() -> ctypes.CDLL:
                                   ctypes.c_float, vp]
     for f in ("rdt_create", "rdt_attn_forward", "rdt_moe_forward", "rdt_loop_forward",
               "rdt_loop_forward_host", "rdt_set_trace", "rdt_get_diagnostics", "rdt_memory_bytes",
-              "rdt_matmul", "rdt_attention", "rdt_profile", "rdt_profile_read", "rdt_moe_route_noalloc"):
+              "rdt_matmul", "rdt_attention", "rdt_profile", "rdt_profile_read", "rdt_moe_route_noalloc",
+              "rdt_set_act", "rdt_loop_forward_act"):
         getattr(lib, f).restype = i32
     _LIB = lib
     return lib
@@ -239,6 +243,21 @@ class RDT:
             out = torch.empty(e.shape, dtype=torch.float32, device=e.device)
         _check(self._lib.rdt_loop_forward(self._h, _ptr(h0), _ptr(e), T, _ptr(out), _stream(stream)))
         return out
+
+    def set_act(self, w_halt, b_halt: float, threshold: float = 0.99, stream=None):
+        """ACT halting head: w_halt a device fp32 [dim] tensor (copied)."""
+        _check(self._lib.rdt_set_act(self._h, _ptr(w_halt), float(b_halt), float(threshold), _stream(stream)))
+
+    def loop_forward_act(self, h0, e, T: int, out=None, n_loops=None, stream=None):
+        """Looped block with ACT halting; returns (out fp32 [.., dim], n_loops int32 [..])."""
+        import torch
+        if out is None:
+            out = torch.empty(e.shape, dtype=torch.float32, device=e.device)
+        if n_loops is None:
+            n_loops = torch.empty(e.shape[:-1], dtype=torch.int32, device=e.device)
+        _check(self._lib.rdt_loop_forward_act(self._h, _ptr(h0), _ptr(e), T, _ptr(out), _ptr(n_loops),
+                                              _stream(stream)))
+        return out, n_loops
 
     def loop_forward_host(self, h0, e, T: int, out, stream=None):
         """Host (CPU, ideally pinned) tensors in, host fp32 tensor out; synchronous."""

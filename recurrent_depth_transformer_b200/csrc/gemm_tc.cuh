@@ -142,6 +142,17 @@ struct TopK {
         }
     }
     __device__ __forceinline__ void write(const EpiParams& p, int row) const {
+        const size_t o = static_cast<size_t>(row) * p.top_k;
+        if (p.halted && p.halted[row]) {             // ACT: a halted token is routed nowhere
+            for (int j = 0; j < p.top_k; ++j) {
+                p.idx_out[o + j] = -1;
+                p.w_out[o + j] = 0.0f;
+                if (p.trace_idx) p.trace_idx[o + j] = -1;
+                if (p.trace_w) p.trace_w[o + j] = 0.0f;
+                if (p.route_token) p.slot_row[o + j] = -1;
+            }
+            return;
+        }
         float mx = -INFINITY;
 #pragma unroll
         for (int j = 0; j < KMAX; ++j)
@@ -152,7 +163,6 @@ struct TopK {
             ex[j] = (j < p.top_k && bi[j] >= 0) ? expf(bl[j] - mx) : 0.0f;
             den += ex[j];
         }
-        const size_t o = static_cast<size_t>(row) * p.top_k;
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) {
             if (j >= p.top_k) break;

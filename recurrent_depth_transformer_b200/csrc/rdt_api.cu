@@ -77,6 +77,13 @@ struct rdt_handle {
     void *stage_h0 = nullptr, *stage_e = nullptr;
     float* stage_out = nullptr;
 
+    // ACT halting (rdt_set_act): head, and per-token running sum / loops run
+    bool act_set = false;
+    float* act_w = nullptr;
+    float act_b = 0.0f, act_thr = 0.0f;
+    float* act_cum = nullptr;
+    int* act_loops = nullptr;
+
     // tensor maps
     CUtensorMap m_xn, m_wqkv, m_tq, m_lqb, m_o, m_wo, m_to, m_lob, m_xperm, m_w13, m_U, m_w2;
     CUtensorMap m_wlat, m_cq, m_wqabs, m_ynlo, m_wr;
@@ -97,7 +104,11 @@ struct rdt_handle {
         const void* e = nullptr;
         const float* out = nullptr;
         int T = 0;
-        bool operator==(const GraphKey& o) const { return h0 == o.h0 && e == o.e && out == o.out && T == o.T; }
+        bool act = false;
+        const int32_t* n_loops = nullptr;
+        bool operator==(const GraphKey& o) const {
+            return h0 == o.h0 && e == o.e && out == o.out && T == o.T && act == o.act && n_loops == o.n_loops;
+        }
     };
     cudaStream_t cap_stream = nullptr;
     cudaGraphExec_t gexec = nullptr;
@@ -116,11 +127,12 @@ constexpr int kFillerRows = 256;
 
 // kernel classes reported by rdt_profile_read
 enum Kind { K_HOIST, K_NORM1, K_GEMM_QKV, K_GEMM_LAT, K_MLA_NORM, K_GEMM_Q, K_ATTENTION, K_LORA_DOWN,
-            K_GEMM_O, K_NORM2, K_ROUTER, K_DISPATCH, K_GEMM_UP, K_GEMM_DOWN, K_CHECK, K_DENSE_B, K_COUNT };
+            K_GEMM_O, K_NORM2, K_ROUTER, K_DISPATCH, K_GEMM_UP, K_GEMM_DOWN, K_CHECK, K_DENSE_B, K_ACT,
+            K_COUNT };
 const char* const kKindName[K_COUNT] = {"hoist", "norm1", "gemm_qkv", "gemm_latent", "mla_latent_norm",
                                          "gemm_q_absorbed", "attention", "lora_down", "gemm_o",
                                          "norm2", "router_topk", "moe_dispatch", "gemm_up", "gemm_down",
-                                         "check_finite", "dense_injection"};
+                                         "check_finite", "dense_injection", "act_halting"};
 
 rdt_status prof_begin(rdt_handle* h, int kind, int nlaunch, cudaStream_t st) {
     h->launches += nlaunch;
@@ -807,7 +819,7 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
 // ---- the MoE sublayer: norm2 -> router (tensor cores, top-k epilogue) -> dispatch -> experts;
 // adds into dst
 rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_out, float* w_out,
-                     int32_t* tr_idx, float* tr_w, cudaStream_t st) {
+                     int32_t* tr_idx, float* tr_w, const int* halted, cudaStream_t st) {
     const rdt_config& c = h->cfg;
     const int N = h->ntok, d = c.dim, hid = c.expert_hidden;
     int32_t* idx = idx_out ? idx_out : h->idx;
@@ -839,6 +851,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
         ra.a_routed_base = N;
         ra.store_yn = c.n_shared > 0;          // shared experts read yn itself
         ra.weights_static = 1;                 // the library's own copy, written at create
+        ra.halted = halted;
         TIMED(h, K_ROUTER, 1, st, norm2_router_smem(h->bf, ra, st));
         copies_written = true;
     } else if (!h->bf) {
@@ -863,6 +876,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
         ra.row_w = h->row_w;
         ra.slot_row = h->slot_row;
         ra.cap = h->cap;
+        ra.halted = halted;
         TIMED(h, K_ROUTER, 1, st, norm2_router(false, ra, st));
     } else {
         Norm2Args n2{};
@@ -903,6 +917,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
         er.route_w = h->row_w;
         er.slot_row = h->slot_row;
         er.cap = h->cap;
+        er.halted = halted;
         er.flags = h->flags;
         TIMED(h, K_ROUTER, 1, st, gemm_tc(h->bf, h->bn_router, h->m_xperm, h->m_wr, &h->m_ynlo, &h->m_wr, gr, er, st));
     }
@@ -957,7 +972,10 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     return RDT_OK;
 }
 
-rdt_status loop_impl(rdt_handle* h, const void* h0, const void* e, int T, float* out, cudaStream_t st) {
+// With act, every loop ends with the ACT step: h_{t+1} stays in the workspace, `out`
+// collects the weighted states, halted tokens keep their state and are routed nowhere.
+rdt_status loop_impl(rdt_handle* h, const void* h0, const void* e, int T, float* out, bool act,
+                     int32_t* n_loops, cudaStream_t st) {
     const rdt_config& c = h->cfg;
     const int N = h->ntok, d = c.dim;
     const size_t nd = static_cast<size_t>(N) * d;
@@ -967,14 +985,32 @@ rdt_status loop_impl(rdt_handle* h, const void* h0, const void* e, int T, float*
     for (int t = 0; t < T; ++t) {
         NvtxRange loop_range("rdt loop");
         float* hcur = h->hbuf[t & 1];
-        float* hnext = (t == T - 1) ? out : h->hbuf[(t + 1) & 1];
+        float* hnext = (t == T - 1 && !act) ? out : h->hbuf[(t + 1) & 1];
         RDT_TRY(attention_block(h, hcur, c.inject_e ? e : nullptr, t, true, nullptr, hnext, st));
         const size_t tk = static_cast<size_t>(t) * N * c.top_k;
         RDT_TRY(moe_block(h, h->y, hnext, nullptr, nullptr, h->tr_idx ? h->tr_idx + tk : nullptr,
-                          h->tr_w ? h->tr_w + tk : nullptr, st));
+                          h->tr_w ? h->tr_w + tk : nullptr, act && t > 0 ? h->act_loops : nullptr, st));
+        if (act) {
+            ActArgs aa{};
+            aa.h_cur = hcur;
+            aa.h_next = hnext;
+            aa.out = out;
+            aa.w_halt = h->act_w;
+            aa.b_halt = h->act_b;
+            aa.threshold = h->act_thr;
+            aa.cum = h->act_cum;
+            aa.loops = h->act_loops;
+            aa.ntok = N;
+            aa.dim = d;
+            aa.t = t;
+            aa.last = t == T - 1;
+            TIMED(h, K_ACT, 1, st, act_step(aa, st));
+        }
         if (h->tr_h)
             RDT_CUDA_TRY(cudaMemcpyAsync(h->tr_h + (t + 1) * nd, hnext, nd * 4, cudaMemcpyDeviceToDevice, st));
     }
+    if (act && n_loops)
+        RDT_CUDA_TRY(cudaMemcpyAsync(n_loops, h->act_loops, static_cast<size_t>(N) * 4, cudaMemcpyDeviceToDevice, st));
     TIMED(h, K_CHECK, 1, st, check_finite(out, nd, h->flags, st));
     return RDT_OK;
 }
@@ -989,14 +1025,17 @@ void drop_graph(rdt_handle* h) {
 // Runs the loop, replaying a captured CUDA graph when the same pointers and T come back:
 // the first call with a key runs eagerly, the second captures (on the handle's own stream)
 // and launches the graph, later ones only launch it. Tracing or profiling runs eagerly.
-rdt_status run_loop(rdt_handle* h, const void* h0, const void* e, int T, float* out, cudaStream_t st) {
+rdt_status run_loop(rdt_handle* h, const void* h0, const void* e, int T, float* out, cudaStream_t st,
+                    bool act = false, int32_t* n_loops = nullptr) {
     const bool graphable = !h->prof_on && !h->tr_idx && !h->tr_w && !h->tr_h;
-    if (!graphable) return loop_impl(h, h0, e, T, out, st);
+    if (!graphable) return loop_impl(h, h0, e, T, out, act, n_loops, st);
     rdt_handle::GraphKey key;
     key.h0 = h0;
     key.e = e;
     key.out = out;
     key.T = T;
+    key.act = act;
+    key.n_loops = n_loops;
     if (h->gexec && h->gkey == key) {
         RDT_CUDA_TRY(cudaGraphLaunch(h->gexec, st));
         h->launches += h->g_launches;
@@ -1004,7 +1043,7 @@ rdt_status run_loop(rdt_handle* h, const void* h0, const void* e, int T, float* 
     }
     if (!(h->seen_key == key)) {
         h->seen_key = key;
-        return loop_impl(h, h0, e, T, out, st);
+        return loop_impl(h, h0, e, T, out, act, n_loops, st);
     }
     if (h->gexec) {
         cudaGraphExecDestroy(h->gexec);
@@ -1013,7 +1052,7 @@ rdt_status run_loop(rdt_handle* h, const void* h0, const void* e, int T, float* 
     if (!h->cap_stream) RDT_CUDA_TRY(cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking));
     const int64_t l0 = h->launches;
     RDT_CUDA_TRY(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal));
-    const rdt_status s = loop_impl(h, h0, e, T, out, h->cap_stream);
+    const rdt_status s = loop_impl(h, h0, e, T, out, act, n_loops, h->cap_stream);
     cudaGraph_t g = nullptr;
     const cudaError_t ce = cudaStreamEndCapture(h->cap_stream, &g);
     if (s != RDT_OK) {
@@ -1129,7 +1168,7 @@ rdt_status rdt_moe_forward(rdt_handle* h, const float* y, float* f_out, int32_t*
     const size_t nd = static_cast<size_t>(h->ntok) * h->cfg.dim;
     RDT_CUDA_TRY(cudaMemsetAsync(f_out, 0, nd * 4, st));
     RDT_CUDA_TRY(cudaMemsetAsync(h->counts, 0, 256 * 4, st));
-    return moe_block(h, y, f_out, topk_idx, topk_w, nullptr, nullptr, st);
+    return moe_block(h, y, f_out, topk_idx, topk_w, nullptr, nullptr, nullptr, st);
 }
 
 rdt_status rdt_loop_forward(rdt_handle* h, const void* h0, const void* e, int T, float* out, void* stream) {
@@ -1180,6 +1219,63 @@ rdt_status rdt_loop_forward_host(rdt_handle* h, const void* h0_host, const void*
     RDT_CUDA_TRY(cudaMemcpyAsync(out_host, h->stage_out, nd * 4, cudaMemcpyDeviceToHost, st));
     RDT_CUDA_TRY(cudaStreamSynchronize(st));
     return RDT_OK;
+}
+
+rdt_status rdt_set_act(rdt_handle* h, const float* w_halt, float b_halt, float threshold, void* stream) {
+    if (!h) {
+        set_error("handle is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    RDT_TRY(check_ptr(w_halt, "w_halt"));
+    if (!std::isfinite(b_halt) || !(threshold > 0.0f && threshold <= 1.0f)) {
+        set_error("b_halt must be finite and threshold in (0, 1]");
+        return RDT_ERR_INVALID_ARG;
+    }
+    const int N = h->ntok, d = h->cfg.dim;
+    if (d % 128 != 0) {
+        set_error("ACT halting needs dim to be a multiple of 128");
+        return RDT_ERR_UNSUPPORTED;
+    }
+    if (!h->act_w) {
+        RDT_TRY(dev_alloc(h, &h->act_w, static_cast<size_t>(d) * 4));
+        RDT_TRY(dev_alloc(h, &h->act_cum, static_cast<size_t>(N) * 4, true));
+        RDT_TRY(dev_alloc(h, &h->act_loops, static_cast<size_t>(N) * 4, true));
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    RDT_CUDA_TRY(cudaMemcpyAsync(h->act_w, w_halt, static_cast<size_t>(d) * 4, cudaMemcpyDeviceToDevice, st));
+    RDT_CUDA_TRY(cudaStreamSynchronize(st));
+    h->act_b = b_halt;
+    h->act_thr = threshold;
+    h->act_set = true;
+    drop_graph(h);                    // a captured loop holds the old head's scalars
+    return RDT_OK;
+}
+
+rdt_status rdt_loop_forward_act(rdt_handle* h, const void* h0, const void* e, int T, float* out,
+                                int32_t* n_loops, void* stream) {
+    if (!h) {
+        set_error("handle is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (!h->act_set) {
+        set_error("rdt_set_act has not been called on this handle");
+        return RDT_ERR_INVALID_ARG;
+    }
+    RDT_TRY(check_ptr(h0, "h0"));
+    RDT_TRY(check_ptr(e, "e"));
+    RDT_TRY(check_ptr(out, "out"));
+    if (n_loops) RDT_TRY(check_ptr(n_loops, "n_loops"));
+    if (T < 1 || T > h->cfg.max_loops) {
+        set_error("T must be in [1, max_loops]");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (out == e) {
+        set_error("out must not alias e (e is read in every loop)");
+        return RDT_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    h->last_stream = st;
+    return run_loop(h, h0, e, T, out, st, true, n_loops);
 }
 
 rdt_status rdt_matmul(int32_t dtype, const void* A, const void* B, float* C, int M, int N, int K,

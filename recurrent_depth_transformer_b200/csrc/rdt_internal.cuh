@@ -426,6 +426,8 @@ struct EpiParams {
     float* logits;         // split-K router: [ntok, n_exp] fp32 partial sums (zeroed beforehand)
     int* tile_count;       // split-K router: arrival counters per (row tile, 32-row quadrant)
                            // (zero, reset after use)
+    const int* halted;     // ACT: [ntok] loops run by a halted token, 0 while running (or NULL):
+                           // a halted token is routed to no expert (index -1, weight 0)
     int* flags;            // device status words
 };
 
@@ -509,6 +511,8 @@ struct RouterArgs {
     int store_yn;                      // fused router: also write yn at row `row` of yn
     int weights_static;                // fused router: w_router is not written by the previous
                                        // kernel in the stream (staged before waiting on it)
+    const int* halted;                 // ACT: [ntok], nonzero = halted token, routed to no
+                                       // expert (index -1, weight 0); NULL = all route
 };
 rdt_status norm2_router(bool bf16_elems, const RouterArgs& a, cudaStream_t st);
 // RMSNorm2 fused with the fp32 router when W_r (n_exp x dim, element type) takes at most
@@ -518,7 +522,8 @@ bool router_fits_smem(bool bf16_elems, int n_exp, int top_k, int dim);
 rdt_status norm2_router_smem(bool bf16_elems, const RouterArgs& a, cudaStream_t st);
 
 // Copy yn[token] into the claimed row of every (token, slot) (routers that do not write
-// the copies themselves): xperm[a_routed_base + slot_row[token * k + j]] = xperm[token].
+// the copies themselves): xperm[a_routed_base + slot_row[token * k + j]] = xperm[token];
+// a slot whose claimed row is negative (a halted token) is skipped.
 rdt_status moe_copy(bool bf16_elems, void* xperm, const int* slot_row, int ntok, int top_k, int dim,
                     int a_routed_base, cudaStream_t st);
 
@@ -539,6 +544,21 @@ struct MlaNormArgs {
     int ntok, seq, q_lat, kv_lat, rope; float eps;
 };
 rdt_status mla_latent_norm(bool bf16_elems, const MlaNormArgs& a, cudaStream_t st);
+
+// One loop's ACT halting step over the fp32 state (one warp per token):
+//   a token halted in an earlier loop (t > 0 and loops[n] > 0) keeps its state:
+//     h_next[n] <- h_cur[n];
+//   a running token takes p = sigmoid(w_halt . h_next[n] + b_halt); with c = cum[n] (0 at
+//     t = 0) it halts if c + p >= threshold or last: out[n] (+)= (1 - c) h_next[n] and
+//     loops[n] = t + 1; else out[n] (+)= p h_next[n] and loops[n] = 0; cum[n] = c + p.
+//   At t = 0 out, cum and loops are written, not read.
+struct ActArgs {
+    const float* h_cur; float* h_next; float* out;   // [ntok, dim] fp32
+    const float* w_halt; float b_halt, threshold;     // head [dim] fp32
+    float* cum; int* loops;                           // [ntok]
+    int ntok, dim, t, last;
+};
+rdt_status act_step(const ActArgs& a, cudaStream_t st);
 
 // Weight preparation: C[m, n] = sum_k A(m, k) B(k, n) with A(m, k) = A[m*sam + k*sak] and
 // B(k, n) = B[k*sbk + n*sbn] (element type of the configuration), fp32 sums.

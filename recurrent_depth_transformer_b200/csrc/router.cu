@@ -132,6 +132,16 @@ __global__ void __launch_bounds__(kRouterMaxThreads, 2) norm2_router_smem_kernel
             for (int j = 0; j < 4; ++j) y[i][j] *= inv * gi[j];
             if (a.store_yn) store4(yn + i * 128 + lane * 4, y[i]);   // element-type copy; logits use fp32
         }
+        if (a.halted && a.halted[row]) {          // ACT: a halted token is routed nowhere
+            if (lane < a.top_k) {
+                const size_t o = static_cast<size_t>(row) * a.top_k + lane;
+                a.idx[o] = -1;
+                a.w[o] = 0.0f;
+                if (a.trace_idx) a.trace_idx[o] = -1;
+                if (a.trace_w) a.trace_w[o] = 0.0f;
+            }
+            continue;
+        }
         float lg[EMAX];
 #pragma unroll
         for (int e = 0; e < EMAX; ++e) {

@@ -10,6 +10,8 @@
 //                  router claimed (capacity layout), for routers that do not write them
 //   lora_down      t = x A^T for the O-projection adapter
 //   mla_latent_norm  RMSNorm of c_q and c_kv, RoPE of the decoupled key
+//   act_step       ACT halting after a loop: halting probability of the new state,
+//                  the halting decision, the weighted output sum, frozen halted states
 // plus the weight-preparation matmul and a finite-value check.
 #include <algorithm>
 
@@ -185,6 +187,17 @@ __global__ void __launch_bounds__(kRowThreads) norm2_router_kernel(const RouterA
         for (int j = 0; j < 4; ++j) y[i][j] *= inv * g[j];
         store4(yn + col, y[i]);   // rounded copy for the experts; the router keeps fp32
     }
+    if (a.halted && a.halted[row]) {              // ACT: a halted token is routed nowhere
+        if (lane < a.top_k) {
+            const size_t o = static_cast<size_t>(row) * a.top_k + lane;
+            a.idx[o] = -1;
+            a.w[o] = 0.0f;
+            if (a.trace_idx) a.trace_idx[o] = -1;
+            if (a.trace_w) a.trace_w[o] = 0.0f;
+            if (a.row_token) a.slot_row[o] = -1;
+        }
+        return;
+    }
 
     // logits: lane (e % 32) keeps expert e in slot e / 32
     const T* W = static_cast<const T*>(a.w_router);
@@ -340,6 +353,7 @@ __global__ void __launch_bounds__(kRowThreads) moe_copy_kernel(T* xperm, const i
     const int lane = threadIdx.x & 31;
     if (ws >= ntok * top_k) return;
     const int n = ws / top_k;
+    if (slot_row[ws] < 0) return;                 // halted token: no row claimed
     const int r = a_routed_base + slot_row[ws];
     const uint4* src = reinterpret_cast<const uint4*>(xperm + static_cast<size_t>(n) * dim);
     uint4* dst = reinterpret_cast<uint4*>(xperm + static_cast<size_t>(r) * dim);
@@ -427,6 +441,60 @@ __global__ void prep_matmul_kernel(const T* A, long sam, long sak, const T* B, l
     C[static_cast<size_t>(m) * ldc + n] = from_f<T>(acc);
 }
 
+// ----------------------------------------------------------------------------- ACT halting
+
+// ACT (Dynamic Adaptive Computation Time) after loop t, one warp per token: a token halted
+// before this loop copies its state forward; a running one takes its halting probability
+// p = sigmoid(w . h_next + b) from the new state, halts once its summed p reaches the
+// threshold (or at the last loop) with the remainder as weight, and adds its weighted state
+// to the output. Reads and writes 2-3 fp32 rows per token: bound by HBM bandwidth.
+template <int NV>
+__global__ void __launch_bounds__(kRowThreads) act_step_kernel(const ActArgs a) {
+    pdl_trigger();
+    pdl_wait();
+    const int row = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= a.ntok) return;
+    const size_t base = static_cast<size_t>(row) * a.dim;
+    if (a.t > 0 && a.loops[row] > 0) {            // halted earlier: the state stays put
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            float v[4];
+            load4(a.h_cur + base + i * 128 + lane * 4, v);
+            store4(a.h_next + base + i * 128 + lane * 4, v);
+        }
+        return;
+    }
+    float v[NV][4];
+    float z = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        float w[4];
+        load4(a.h_next + base + i * 128 + lane * 4, v[i]);
+        load4(a.w_halt + i * 128 + lane * 4, w);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) z = fmaf(v[i][j], w[j], z);
+    }
+    z = warp_sum(z) + a.b_halt;
+    const float p = 1.0f / (1.0f + expf(-z));
+    const float c = a.t > 0 ? a.cum[row] : 0.0f;
+    const bool halt = a.last || c + p >= a.threshold;
+    const float wgt = halt ? 1.0f - c : p;
+    if (lane == 0) {
+        a.cum[row] = c + p;
+        a.loops[row] = halt ? a.t + 1 : 0;
+    }
+    float* out = a.out + base;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        if (a.t > 0) load4(out + i * 128 + lane * 4, o);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[j] = fmaf(wgt, v[i][j], o[j]);
+        store4(out + i * 128 + lane * 4, o);
+    }
+}
+
 __global__ void check_finite_kernel(const float* x, size_t n, int* flags) {
     pdl_trigger();
     pdl_wait();
@@ -465,6 +533,12 @@ struct LoraL {
                     int r, void* t) {
         launch_pdl(lora_down_kernel<T, NV>, g, dim3(kRowThreads), 0, st, static_cast<const T*>(x), ldx,
                    ntok, static_cast<const T*>(A), r, static_cast<T*>(t));
+    }
+};
+template <typename T, int NV>
+struct ActL {
+    static void run(dim3 g, cudaStream_t st, ActArgs a) {
+        launch_pdl(act_step_kernel<NV>, g, dim3(kRowThreads), 0, st, a);
     }
 };
 template <typename T, int NV>
@@ -574,6 +648,14 @@ rdt_status prep_matmul(bool bf, const void* A, long sam, long sak, const void* B
                                                         static_cast<float*>(C), ldc, M, N, K);
     RDT_CUDA_TRY(cudaGetLastError());
     return RDT_OK;
+}
+
+rdt_status act_step(const ActArgs& a, cudaStream_t st) {
+    if (a.dim % 128 != 0) {
+        set_error("ACT step: dim must be a multiple of 128");
+        return RDT_ERR_UNSUPPORTED;
+    }
+    return launch_rows<float, ActL>(a.dim / 128, a.ntok, st, a);
 }
 
 rdt_status check_finite(const float* x, size_t n, int* flags, cudaStream_t st) {

@@ -66,6 +66,8 @@ def test_create_rejects_bad_config_before_any_device_call(lib):
 def test_calls_reject_null_handle(lib):
     assert lib.rdt_loop_forward(None, None, None, 1, None, None) == 1
     assert lib.rdt_set_trace(None, None, None, None) == 1
+    assert lib.rdt_set_act(None, None, 0.0, 0.99, None) == 1
+    assert lib.rdt_loop_forward_act(None, None, None, 1, None, None, None) == 1
     lib.rdt_destroy(None)
 
 
