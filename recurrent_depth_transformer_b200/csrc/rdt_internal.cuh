@@ -516,7 +516,7 @@ struct RouterArgs {
 };
 rdt_status norm2_router(bool bf16_elems, const RouterArgs& a, cudaStream_t st);
 // RMSNorm2 fused with the fp32 router when W_r (n_exp x dim, element type) takes at most
-// 64 KB (staged as fp32 in up to 128 KB of shared memory), n_exp <= 64, top_k <= 8 and dim is
+// 64 KB (staged in shared memory in its element type), n_exp <= 64, top_k <= 8 and dim is
 // 128, 1024 or 2048
 bool router_fits_smem(bool bf16_elems, int n_exp, int top_k, int dim);
 rdt_status norm2_router_smem(bool bf16_elems, const RouterArgs& a, cudaStream_t st);

@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kRouterMaxThreads, 2) norm2_router_smem_kernel
         ex_l[j] = router_expert<EMAX>(lane, j);
         bias_l[j] = (a.bias && ex_l[j] < a.n_exp) ? a.bias[ex_l[j]] : 0.0f;
     }
-    // gamma stays in registers when they allow it (128 per thread at 512 threads)
+    // gamma stays in registers when they allow it (128 per thread: two 256-thread blocks per SM)
     constexpr bool kHoistGamma = NV * 4 + EMAX <= 64;
     float g[kHoistGamma ? NV : 1][4];
     if constexpr (kHoistGamma) {

@@ -98,3 +98,20 @@ def test_measured_traffic_only_for_unchanged_sources(monkeypatch):
     monkeypatch.setitem(bench.MEASURED_TRAFFIC, "gemm_up", (123.0, "0" * 16))
     assert bench.measured_traffic("gemm_up") is None          # sources changed since the capture
     assert bench.measured_traffic("attention") is None        # never captured
+
+
+def test_fingerprint_ignores_comments_not_code(tmp_path):
+    src = 'int f(int a) {  // doubles a\n    /* note */ return 2 * a;\n}\nconst char* s = "p//q";\n'
+    f = tmp_path / "k.cu"
+
+    def fp(text):
+        f.write_text(text)
+        return bench.source_fingerprint([str(f)])
+
+    base = fp(src)
+    assert fp(src.replace("doubles a", "twice a")) == base              # comment edit
+    assert fp(src.replace("/* note */", "/* longer\n note */")) == base  # block comment
+    assert fp("\n" + src.replace("    ", "\t")) == base                  # indentation, blank line
+    assert fp(src.replace("2 * a", "3 * a")) != base                     # code
+    assert fp(src.replace("p//q", "p//r")) != base                       # '//' inside a string is code
+
