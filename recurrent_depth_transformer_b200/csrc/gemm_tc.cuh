@@ -25,9 +25,13 @@
 //                   MoE adds f later);
 //   EPI_SWIGLU      expert up-projection (gate and up rows interleaved per tile) -> silu(g)*u;
 //   EPI_SCATTER     expert down-projection, gate weight, and reduction into h_next
-//                   (h_{t+1} = A h + B e + a + sum_j w_j E_j(yn)).
+//                   (h_{t+1} = A h + B e + a + sum_j w_j E_j(yn));
+//   EPI_TOPK        router logits -> top-k, gate weights and the claim of each chosen
+//                   expert's row (K split over CTAs: partial logits reduced, the last
+//                   arrival picks); tokens halted by ACT are routed nowhere;
+//   EPI_STORE, EPI_STORE_F32, EPI_OPROJ_PLAIN  plain stores (element type, fp32).
 // Grouped mode decodes its tiles from the per-expert row counters on the device (capacity
-// layout: expert e's rows start at e * tokens), so the counts never travel to the host.
+// layout: group g's rows start at g * cap), so the counts never travel to the host.
 #pragma once
 #include <algorithm>
 #include <type_traits>

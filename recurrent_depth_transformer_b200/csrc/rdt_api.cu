@@ -343,8 +343,9 @@ rdt_status build_maps(rdt_handle* h) {
         RDT_TRY(make_tmap_2d(&h->m_lob, h->lob, bf, h->kext, static_cast<uint64_t>(c.n_lora) * d,
                              h->kext * es, kbox, h->bn_o >> h->pair_o));
     }
-    // capacity layout: xperm = [yn (N rows) | expert e: rows N + e N .. N + e N + N),
-    // U = [shared expert s: rows s N .. | expert e: rows (S + e) N ..]
+    // capacity layout, cap rows per group: xperm = [yn (N rows) | expert e: rows N + e cap ..
+    // N + (e + 1) cap), U = [shared expert s: rows s cap .. | expert e: rows (S + e) cap ..],
+    // and kFillerRows rows of filler after the last group of each
     const uint64_t xrows = static_cast<uint64_t>(N) + static_cast<uint64_t>(h->cap) * E + kFillerRows;
     const uint64_t urows = static_cast<uint64_t>(h->cap) * (S + E) + kFillerRows;
     RDT_TRY(make_tmap_2d(&h->m_xperm, h->xperm, bf, d, xrows, d * es, kbox, 128));
@@ -462,7 +463,7 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         h->bn_up = t.bn;
         h->pair_up = t.pair;
         // the down-projection's epilogue reduces every output into h_next; on pairs a CTA's
-        // share of it doubles and measured slower (24.3 vs 22.7 us), so it runs on pairs only
+        // share of it doubles and measured slower (24.3 vs 23.7 us), so it runs on pairs only
         // when they are forced
         t = choose_tiles(grows, E + S, d, kb_h, true, false, mode == 2, 4, mode);
         h->bn_down = t.bn;
@@ -816,8 +817,9 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
     return RDT_OK;
 }
 
-// ---- the MoE sublayer: norm2 -> router (tensor cores, top-k epilogue) -> dispatch -> experts;
-// adds into dst
+// ---- the MoE sublayer: norm2 + router (the fused shared-memory router, or RMSNorm2 and the
+// tensor-core router with its top-k epilogue, or the fp32 FMA router) -> dispatch -> experts;
+// adds into dst. With `halted` (ACT), tokens whose entry is nonzero are routed nowhere.
 rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_out, float* w_out,
                      int32_t* tr_idx, float* tr_w, const int* halted, cudaStream_t st) {
     const rdt_config& c = h->cfg;
