@@ -5,9 +5,9 @@
  *
  *     h_{t+1} = A (.) h_t + B.e + Block(h_t, e),      t = 0 .. T-1,
  *
- * (update equation of the techbriefly article on the OpenMythos project:
- * "h_{t+1} = A.h_t + B.e + Transformer(h_t, e)", with e the prelude encoding
- * re-injected every loop and rho(A) < 1). Block is a pre-RMSNorm causal
+ * (the update equation of the techbriefly article on the OpenMythos project,
+ * whose transformer term is Block here; e is the prelude encoding, injected
+ * again in every loop, and rho(A) < 1). Block is a pre-RMSNorm causal
  * attention sublayer (GQA, or MLA with a latent KV) followed by a top-k sparse
  * mixture of SwiGLU experts, with optional per-loop (depth-wise) LoRA on the Q
  * and O projections (getting-started page "Introducao ao OpenMythos",
@@ -167,7 +167,8 @@ rdt_status rdt_moe_forward(rdt_handle* h, const float* y, float* f_out, int32_t*
 /* The looped block: out = h_T after T loops of the update equation.
  *   h0, e : device [N, dim] in cfg.dtype (h0 may alias e)
  *   T     : 1 .. cfg.max_loops (INVALID_ARG otherwise)
- *   out   : device fp32 [N, dim]; the state is kept in fp32 throughout        */
+ *   out   : device fp32 [N, dim]; the state is kept in fp32 throughout; must
+ *           not alias e, which every loop reads (INVALID_ARG)                 */
 rdt_status rdt_loop_forward(rdt_handle* h, const void* h0, const void* e, int T, float* out,
                             void* stream);
 
@@ -203,7 +204,8 @@ rdt_status rdt_set_act(rdt_handle* h, const float* w_halt, float b_halt, float t
  * enters the output with weight 1 - c; otherwise with weight p_t.
  *   h0, e   : device [N, dim] in cfg.dtype (h0 may alias e)
  *   T       : 1 .. cfg.max_loops (INVALID_ARG otherwise)
- *   out     : device fp32 [N, dim] = sum over t of weight_t * h_{t+1}
+ *   out     : device fp32 [N, dim] = sum over t of weight_t * h_{t+1}; must not
+ *             alias e (INVALID_ARG)
  *   n_loops : device int32 [N] (16-byte aligned) or NULL: loops each position ran
  * INVALID_ARG if rdt_set_act has not been called on the handle. */
 rdt_status rdt_loop_forward_act(rdt_handle* h, const void* h0, const void* e, int T, float* out,
@@ -213,7 +215,8 @@ rdt_status rdt_loop_forward_act(rdt_handle* h, const void* h0, const void* e, in
  *   idx    : int32 [max_loops, N, top_k] routing of every loop
  *   w      : fp32  [max_loops, N, top_k] gate weights of every loop
  *   h_traj : fp32  [max_loops + 1, N, dim] the state h_0 .. h_T
- * Later rdt_loop_forward calls write loop t at offset t. Pass all NULL to stop. */
+ * Later rdt_loop_forward and rdt_loop_forward_act calls write loop t at offset t (a
+ * token halted by ACT has index -1 and weight 0 there). Pass all NULL to stop. */
 rdt_status rdt_set_trace(rdt_handle* h, int32_t* idx, float* w, float* h_traj);
 
 /* Synchronises the handle's last stream and fills *out (see rdt_diag). */
@@ -272,7 +275,7 @@ rdt_status rdt_moe_route_noalloc(int32_t dtype, const float* y, const float* nor
 
 /* ---- per-kernel timing (CUDA events recorded around every launch of the handle) */
 typedef struct {
-    char name[32];          /* kernel class, e.g. "gemm_up", "attention", "norm2_router" */
+    char name[32];          /* kernel class, e.g. "gemm_up", "attention", "router_topk"  */
     int64_t launches;       /* launches timed since profiling was enabled               */
     double total_ms;        /* summed event time of those launches                      */
 } rdt_kernel_stat;
