@@ -43,6 +43,12 @@ design notes of the repository):
   min(t, L - 1) at loop t;
 * MLA: latent RMSNorms on c_q and c_kv, decoupled RoPE key shared by all
   heads, score scale 1/sqrt(nope + rope);
+* decode with a per-loop KV cache ([GS] Passo 4: the prompt is processed
+  once, then one token per call; troubleshooting item 1: every loop keeps the
+  KV state of all tokens): loop t of a new token attends over the keys and
+  values that loop t produced for the earlier positions; GQA caches its
+  rotated keys and values, MLA its normalised latent and rotated shared key,
+  from which K/V are rebuilt at every step ([GS] Passo 5);
 * ACT halting ([TB] names it; [GS] troubleshooting item 4 gives the 0.99
   threshold and that a position leaves once its accumulated halting probability
   reaches it): halting head p = sigmoid(w . h_{t+1} + b) on the new state;
@@ -516,3 +522,105 @@ def loop_forward_act(h0, e, T: int, W, cfg, w_halt, b_halt: float, threshold: fl
             trace.attn.append(a)
             trace.moe.append(f)
     return ActResult(out=out, n_loops=n_loops, weights=weights, stats=stats)
+
+
+# --------------------------------------------------------------------------------------
+# Decode with a per-loop KV cache
+# --------------------------------------------------------------------------------------
+
+def apply_rope_at(x, pos, base: float) -> np.ndarray:
+    """Rotate-half RoPE of x [B, Sn, H, r] with row j of axis 1 at position pos[j]
+    (:func:`apply_rope` is the case pos = 0..Sn-1)."""
+    x = _f(x)
+    r = x.shape[-1]
+    pos = np.asarray(pos)
+    cos, sin = rope_angles(int(pos.max()) + 1, r, base)
+    cos = cos[pos][None, :, None, :]
+    sin = sin[pos][None, :, None, :]
+    x1, x2 = x[..., : r // 2], x[..., r // 2:]
+    return np.concatenate([x1 * cos - x2 * sin, x2 * cos + x1 * sin], axis=-1)
+
+
+@dataclass
+class LoopKVCache:
+    """What each loop keeps for the positions processed so far ([GS] Passo 4 and
+    troubleshooting item 1). Per loop t: GQA ``k[t]`` (after RoPE) and ``v[t]``
+    [B, length, Hkv, dh]; MLA ``ckv[t]`` [B, length, kv_lat] (after its RMSNorm) and
+    ``kr[t]`` [B, length, rope] (after RoPE), from which K and V are rebuilt ([GS] Passo 5)."""
+    length: int = 0
+    k: Dict[int, np.ndarray] = field(default_factory=dict)
+    v: Dict[int, np.ndarray] = field(default_factory=dict)
+    ckv: Dict[int, np.ndarray] = field(default_factory=dict)
+    kr: Dict[int, np.ndarray] = field(default_factory=dict)
+
+
+def _append(store: Dict[int, np.ndarray], t: int, new: np.ndarray) -> np.ndarray:
+    store[t] = new if t not in store else np.concatenate([store[t], new], axis=1)
+    return store[t]
+
+
+def attention_cached(x, W, cfg, t: int, cache: LoopKVCache) -> np.ndarray:
+    """a = Attn(RMSNorm1(x)) for x [B, Sn, d] at positions cache.length .. + Sn - 1,
+    attending over loop t's cached keys and values of the earlier positions and its own;
+    appends this loop's new keys and values to the cache (the caller advances
+    ``cache.length`` once every loop has run)."""
+    x = _f(x)
+    Bn, Sn, _ = x.shape
+    pos = cache.length + np.arange(Sn)
+    xn = rmsnorm(x, W["norm1"], cfg.norm_eps)
+    if cfg.attn == "gqa":
+        hq, hkv, dh = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+        q = xn @ _f(W["wq"]).T
+        if cfg.n_lora:
+            li = _lora_index(cfg, t)
+            q = q + (xn @ _f(W["lq_a"][li]).T) @ _f(W["lq_b"][li]).T
+        q = apply_rope_at(q.reshape(Bn, Sn, hq, dh), pos, cfg.rope_base)
+        k = apply_rope_at((xn @ _f(W["wk"]).T).reshape(Bn, Sn, hkv, dh), pos, cfg.rope_base)
+        v = (xn @ _f(W["wv"]).T).reshape(Bn, Sn, hkv, dh)
+        k_all = _append(cache.k, t, k)
+        v_all = _append(cache.v, t, v)
+        o = gqa_attention(q, k_all, v_all, 1.0 / np.sqrt(dh), q_pos=pos).reshape(Bn, Sn, -1)
+    else:
+        H, nope, rope, vd = cfg.n_heads, cfg.qk_nope_dim, cfg.qk_rope_dim, cfg.v_head_dim
+        c_q = rmsnorm(xn @ _f(W["w_dq"]).T, W["q_norm"], cfg.norm_eps)
+        c_kv = rmsnorm(xn @ _f(W["w_dkv"]).T, W["kv_norm"], cfg.norm_eps)
+        k_r = apply_rope_at((xn @ _f(W["w_kr"]).T).reshape(Bn, Sn, 1, rope), pos, cfg.rope_base)
+        ckv_all = _append(cache.ckv, t, c_kv)
+        kr_all = _append(cache.kr, t, k_r[:, :, 0])
+        L = ckv_all.shape[1]
+        qf = (c_q @ _f(W["w_uq"]).T).reshape(Bn, Sn, H, nope + rope)
+        q = np.concatenate([qf[..., :nope], apply_rope_at(qf[..., nope:], pos, cfg.rope_base)], axis=-1)
+        k_nope = (ckv_all @ _f(W["w_uk"]).T).reshape(Bn, L, H, nope)      # rebuilt from the latent
+        v = (ckv_all @ _f(W["w_uv"]).T).reshape(Bn, L, H, vd)
+        k = np.concatenate([k_nope, np.broadcast_to(kr_all[:, :, None, :], (Bn, L, H, rope))], axis=-1)
+        o = gqa_attention(q, k, v, 1.0 / np.sqrt(nope + rope), q_pos=pos).reshape(Bn, Sn, -1)
+    return out_proj(o, W, cfg, t)
+
+
+def _loop_cached(h0, e, T: int, W, cfg, cache: LoopKVCache) -> np.ndarray:
+    A = _f(W["A"])
+    e = _f(e)
+    Be = input_injection(e, W["B"])
+    h = _f(h0)
+    for t in range(T):
+        x = h + e if cfg.inject_e else h
+        a = attention_cached(x, W, cfg, t, cache)
+        y = x + a
+        f, _, _ = moe_sublayer(y, W, cfg)
+        h = A * h + Be + a + f
+    cache.length += h.shape[1]
+    return h
+
+
+def loop_prefill(h0, e, T: int, W, cfg) -> Tuple[np.ndarray, LoopKVCache]:
+    """The loop over a whole prompt [B, S, d] ([GS] Passo 4, first call): h_T and the
+    cache of every loop's keys and values for positions 0..S-1."""
+    cache = LoopKVCache()
+    h = _loop_cached(h0, e, T, W, cfg, cache)
+    return h, cache
+
+
+def loop_decode(h0, e, T: int, W, cfg, cache: LoopKVCache) -> np.ndarray:
+    """T loops for new tokens h0, e [B, Sn, d] (Sn = 1 in a decode step) at positions
+    cache.length .., each loop t attending over loop t's cache; extends the cache."""
+    return _loop_cached(h0, e, T, W, cfg, cache)
