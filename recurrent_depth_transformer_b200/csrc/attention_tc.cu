@@ -4,7 +4,8 @@
 //   o = softmax(q k^T * scale, key > query masked) v
 //
 // For each block j of 128 keys:  S_j = Q K_j^T  (tcgen05.mma, M = 128 queries, N = 128 keys,
-// fp32 in TMEM)  ->  four softmax warps, one query row per thread: row maximum, then
+// fp32 in TMEM)  ->  eight softmax warps, two per 32 query rows (one per half of the key
+// block), one query row per thread: row maximum (the two halves exchange theirs), then
 // P_j = 2^(S_j * scale * log2 e - m_ref) in bf16, written to shared memory in the
 // 128-byte-swizzled K-major layout, and the row sum l  ->  O += P_j V_j  (tcgen05.mma into a
 // TMEM accumulator, N = dv; V read as an MN-major operand straight from its [key][dv] layout).
