@@ -8,6 +8,8 @@ raise.
     from recurrent_depth_transformer_b200 import RDT
     m = RDT(config, weights)             # weights: dict name -> CUDA tensor
     out = m.loop_forward(h0, e, T)       # fp32 [batch, seq, dim] = h_T
+    m.set_act(w_halt, b_halt, 0.99)      # ACT halting head: fp32 [dim] CUDA tensor
+    out, n_loops = m.loop_forward_act(h0, e, T)   # weighted states, loops per position
 """
 from __future__ import annotations
 
