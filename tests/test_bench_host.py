@@ -115,3 +115,33 @@ def test_fingerprint_ignores_comments_not_code(tmp_path):
     assert fp(src.replace("2 * a", "3 * a")) != base                     # code
     assert fp(src.replace("p//q", "p//r")) != base                       # '//' inside a string is code
 
+
+
+def test_act_line_reports_halting_histogram(capsys):
+    """The --act leg's JSON line, from a stand-in handle (no GPU): the workload, the
+    halting histogram, the mean loops and the kernel shares."""
+    import argparse
+
+    class FakeHandle:
+        closed = False
+
+        def diagnostics(self):
+            return {"nonfinite": 0, "timeout": 0}
+
+        def close(self):
+            self.closed = True
+
+    wl = by_name(bench.WORKLOAD)
+    nl = torch.tensor([[1, 2, 2, 8], [8, 8, 3, 1]], dtype=torch.int32)
+    args = argparse.Namespace(steps=10, warmup=3)
+    stats = {"gemm_up": (80, 3.0), "act_halting": (80, 1.0)}
+    h = FakeHandle()
+    assert bench.act_line(args, h, wl, nl, 2.0e7, 0.82, 1, 0, stats, 1234, None) == 0
+    line = json.loads(capsys.readouterr().out.strip())
+    assert h.closed
+    assert line["impl"] == "ours+act" and line["config"]["workload"].endswith("+act")
+    assert line["act"]["hist"] == [2, 2, 1, 0, 0, 0, 0, 3]
+    assert line["act"]["mean_loops"] == pytest.approx(33 / 8)
+    assert line["act"]["loops_run_fraction"] == pytest.approx(33 / 64)
+    assert line["kernels"]["gemm_up"]["share"] == pytest.approx(0.75)
+    assert line["gpu_launches"] == 1234 and line["finite"] is True
