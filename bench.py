@@ -95,7 +95,7 @@ def measured_traffic(kernel):
     value, fp = MEASURED_TRAFFIC[kernel]
     try:
         return value if source_fingerprint(KERNEL_SOURCES[kernel]) == fp else None
-    except OSError:
+    except (OSError, ValueError):          # missing or undecodable source: no claim
         return None
 
 
