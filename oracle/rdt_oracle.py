@@ -58,8 +58,10 @@ design notes of the repository):
   position keeps its state and still serves as a key, and is routed to no
   expert.
 
-Parity status: every function below is pinned by ``tests/test_oracle_pins.py``
-(closed forms, library special cases, hand-computed fixtures, identities).
+Parity status: every function below is pinned (closed forms, library special cases,
+hand-computed fixtures, identities, brute force): the block and the loop by
+``tests/test_oracle_pins.py``, ACT halting by ``tests/test_oracle_act_pins.py``, the
+cached decode by ``tests/test_oracle_decode_pins.py``.
 """
 from __future__ import annotations
 
