@@ -42,3 +42,17 @@ def test_recipe_ranges():
     assert g["B"].shape == (w1.dim,) and abs(g["B"].mean() - 1.0) < 0.02
     g0 = generate(WORKLOADS[0])
     assert g0["B"].shape == (128, 128) and g0["e"].dtype == np.float32
+
+
+def test_act_head_recipe():
+    from workloads import ACT_THRESHOLD, act_head
+    wl = WORKLOADS[1]
+    a, b = act_head(wl), act_head(wl)
+    np.testing.assert_array_equal(a["w_halt"], b["w_halt"])                 # reproducible
+    assert a["w_halt"].dtype == np.float32 and a["w_halt"].shape == (wl.dim,)
+    assert a["b_halt"] == -1.0 and a["threshold"] == ACT_THRESHOLD == 0.99
+    assert abs(a["w_halt"].std() * np.sqrt(wl.dim) - 0.5) < 0.05              # N(0, 0.25 / dim)
+    assert not np.array_equal(act_head(wl, seed=wl.seed + 1)["w_halt"], a["w_halt"])
+    # a stream of its own: not a replay of generate()'s first draws
+    e = generate(wl.replace(batch=1, seq=1))["e"].ravel()
+    assert not np.allclose(a["w_halt"] / a["w_halt"].std(), e / e.std())
