@@ -183,6 +183,92 @@ def test_mla_absorbed_equals_explicit():
                                O.mla_attention_explicit(xn, W, cfg), rtol=1e-11, atol=1e-12)
 
 
+def _gqa_torch(x, W, cfg, t):
+    """The GQA attention sublayer written with PyTorch library calls: rms_norm, F.linear for
+    the projections (the loop's LoRA delta on Q and O), RoPE as a complex rotation of the
+    pairs (i, i + dh/2) of q and k only, SDPA with grouped KV heads, the O projection."""
+    hq, hkv, dh = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+    xt = _t(x)
+    Bn, S, d = xt.shape
+    xn = tF.rms_norm(xt, (d,), weight=_t(W["norm1"]), eps=cfg.norm_eps)
+    li = min(t, cfg.n_lora - 1) if cfg.n_lora else None
+    q = tF.linear(xn, _t(W["wq"]))
+    if li is not None:
+        q = q + tF.linear(tF.linear(xn, _t(W["lq_a"][li])), _t(W["lq_b"][li]))
+    k = tF.linear(xn, _t(W["wk"]))
+    v = tF.linear(xn, _t(W["wv"]))
+    # [B, S, H*dh] -> [B, H, S, dh]: head h owns columns h*dh .. h*dh + dh - 1
+    q = q.view(Bn, S, hq, dh).transpose(1, 2)
+    k = k.view(Bn, S, hkv, dh).transpose(1, 2)
+    v = v.view(Bn, S, hkv, dh).transpose(1, 2)
+
+    def rot(u):
+        z = torch.complex(u[..., : dh // 2], u[..., dh // 2:])
+        ang = torch.arange(S, dtype=TD)[:, None] * cfg.rope_base ** (
+            -torch.arange(dh // 2, dtype=TD) * 2.0 / dh)[None, :]
+        z = z * torch.polar(torch.ones_like(ang), ang)
+        return torch.cat([z.real, z.imag], dim=-1)
+
+    o = tF.scaled_dot_product_attention(rot(q), rot(k), v, is_causal=True, scale=1.0 / math.sqrt(dh),
+                                        enable_gqa=True)
+    o = o.transpose(1, 2).reshape(Bn, S, hq * dh)
+    a = tF.linear(o, _t(W["wo"]))
+    if li is not None:
+        a = a + tF.linear(tF.linear(o, _t(W["lo_a"][li])), _t(W["lo_b"][li]))
+    return a.numpy()
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 2), (4, 1)])
+@pytest.mark.parametrize("lora", [False, True])
+def test_gqa_sublayer_matches_torch_composition(hq, hkv, lora):
+    kw = dict(lora_rank=3, n_lora=2) if lora else {}
+    cfg = small_gqa(n_heads=hq, n_kv_heads=hkv, head_dim=8, dim=32, seq=13, **kw)
+    W = generate(cfg)
+    x = W["e"] * 1.3 + 0.2
+    for t in ((0, 1, 3) if lora else (0,)):
+        np.testing.assert_allclose(O.attention_sublayer(x, W, cfg, t), _gqa_torch(x, W, cfg, t),
+                                   rtol=1e-11, atol=1e-12)
+
+
+def _planted_gqa_qkv(kind):
+    """A copy of the oracle's Q/K/V step with one plausible mistake planted."""
+    def qkv(xn, W, cfg, t):
+        Bn, S, _ = xn.shape
+        hq, hkv, dh = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+        q = xn @ np.asarray(W["wq"], np.float64).T
+        if cfg.n_lora:
+            li = min(t, cfg.n_lora - 1)
+            delta = (xn @ np.asarray(W["lq_a"][li], np.float64).T) @ np.asarray(W["lq_b"][li], np.float64).T
+            q = q + (0.0 if kind == "lora_dropped" else delta)
+        wk, wv = ("wv", "wk") if kind == "k_v_swapped" else ("wk", "wv")
+        k = xn @ np.asarray(W[wk], np.float64).T
+        v = xn @ np.asarray(W[wv], np.float64).T
+        if kind == "dim_major_heads":
+            q = q.reshape(Bn, S, dh, hq).swapaxes(2, 3)
+            k = k.reshape(Bn, S, dh, hkv).swapaxes(2, 3)
+            v = v.reshape(Bn, S, dh, hkv).swapaxes(2, 3)
+        else:
+            q, k, v = q.reshape(Bn, S, hq, dh), k.reshape(Bn, S, hkv, dh), v.reshape(Bn, S, hkv, dh)
+        q = O.apply_rope(q, cfg.rope_base)
+        k = k if kind == "rope_on_q_only" else O.apply_rope(k, cfg.rope_base)
+        if kind == "rope_on_v":
+            v = O.apply_rope(v, cfg.rope_base)
+        return q, k, v
+    return qkv
+
+
+@pytest.mark.parametrize("kind", ["dim_major_heads", "rope_on_v", "rope_on_q_only", "k_v_swapped",
+                                  "lora_dropped"])
+def test_gqa_pin_catches_planted_mistakes(kind, monkeypatch):
+    cfg = small_gqa(n_heads=8, n_kv_heads=2, head_dim=8, dim=32, seq=13, lora_rank=3, n_lora=2)
+    W = generate(cfg)
+    x = W["e"] * 1.3 + 0.2
+    ref = _gqa_torch(x, W, cfg, 1)
+    np.testing.assert_allclose(O.attention_sublayer(x, W, cfg, 1), ref, rtol=1e-11, atol=1e-12)
+    monkeypatch.setattr(O.rdt_oracle, "gqa_qkv", _planted_gqa_qkv(kind))
+    assert np.max(np.abs(O.attention_sublayer(x, W, cfg, 1) - ref)) > 1e-6
+
+
 def test_mla_page_example_dims_absorbed_equals_explicit():
     g = json.load(open(os.path.join(GOLDEN, "mythos_config_examples.json")))
     m = g["passo5_mla"]
