@@ -528,9 +528,16 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--act", action="store_true", help="time the ACT halting loop instead")
+    ap.add_argument("--workload", default=None, help="workload name (default: the headline one)")
+    ap.add_argument("--loops", type=int, default=None, help="loops T per step")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    global WORKLOAD, LOOPS
+    if args.workload:
+        WORKLOAD = args.workload
+    if args.loops:
+        LOOPS = args.loops
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)

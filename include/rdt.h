@@ -86,6 +86,14 @@ typedef struct {
                                      * down-projection), 1 one CTA per 128-row tile, 2 CTA
                                      * pairs per 256-row tile (bf16 only; fp32 uses 1).
                                      * Results agree up to fp32 summation order.        */
+    int32_t deterministic;          /* 1: bit-identical results from run to run: each
+                                     * expert row's weighted output is stored in its own
+                                     * row and the rows of a token are added in a fixed
+                                     * order (shared experts, then slots 0 .. top_k - 1)
+                                     * by a combine kernel; no K splits that reduce with
+                                     * atomics. Costs N * top_k * dim * 8 bytes of extra
+                                     * traffic per loop. 0: reductions by fp32 atomics,
+                                     * whose order (and so the last bits) may vary.      */
 } rdt_config;
 
 /* Weights, all DEVICE pointers, row-major [out, in]; element type = cfg.dtype
@@ -148,9 +156,9 @@ rdt_status rdt_create(const rdt_config* cfg, const rdt_weights* w, void* stream,
 
 /* Attention sublayer alone: a = Attn(RMSNorm1(x)) including the output
  * projection and the LoRA adapter of loop `loop` (ignored without LoRA).
- *   x     : device fp32 [N, dim] block input (N = batch * seq)
+ *   x     : device [N, dim] block input in cfg.dtype (N = batch * seq)
  *   a_out : device fp32 [N, dim]                                              */
-rdt_status rdt_attn_forward(rdt_handle* h, const float* x, int loop, float* a_out,
+rdt_status rdt_attn_forward(rdt_handle* h, const void* x, int loop, float* a_out,
                             void* stream);
 
 /* MoE sublayer alone: f = MoE(RMSNorm2(y)), routed top-k experts weighted by the
@@ -251,7 +259,7 @@ rdt_status rdt_attention(int32_t dtype, const void* q, const void* k, const void
  * convenience). For callers that cannot call cudaMalloc - code running inside another
  * framework's memory pool that owns all device memory, serving loops that forbid
  * allocation after start-up, or hosts that capture the work into their own CUDA graphs -
- * and so cannot create a handle. Runs the router kernel of rdt_moe_forward: RMSNorm2 of y
+ * and so cannot create a handle. Runs the router kernels of rdt_moe_forward: RMSNorm2 of y
  * with gain norm2, fp32 logits against w_router, top-k of logits + bias (ties to the lower
  * expert index), softmax over the k chosen logits, per-expert token counts.
  *   dtype         : RDT_BF16 or RDT_F32, element type of w_router
@@ -259,19 +267,28 @@ rdt_status rdt_attention(int32_t dtype, const void* q, const void* k, const void
  *   w_router      : device [n_experts, dim];  router_bias : device fp32 [n_experts] or NULL
  *   topk_idx      : device int32 [ntok, top_k];  topk_w : device fp32 [ntok, top_k]
  *   expert_counts : device int32 [n_experts] or NULL
- * No allocation: the kernels' scratch (normalised rows, for bf16 also their residuals, and
- * counters) is one static device array of 8 MiB that every process loading librdt holds
- * on every GPU it uses until exit. 2 * ntok * dim * 2 bytes (bf16) or ntok * dim * 4 bytes
- * (fp32) must not exceed 8 MiB - 4 KiB (RDT_ERR_UNSUPPORTED otherwise);
- * dim = 128 * 2^k <= 4096, n_experts <= 256, top_k <= min(n_experts, 16).
- * The first call on a device looks up the array's device address (a runtime call, no
- * allocation); make that first call before any stream capture. All calls share the array
- * and the counters are cleared at the start of each call, so calls that overlap on the GPU
- * (other streams, other threads) race: serialise them. */
+ * No allocation: the kernels' scratch (counters, status words and, where the path needs
+ * them, normalised rows) is one static device array of 8 MiB that every process loading
+ * librdt holds on every GPU it uses until exit. Row scratch by path: none when w_router
+ * takes at most 64 KB with n_experts <= 64, top_k <= 8 and dim 128, 1024 or 2048 (the fused
+ * router); otherwise 2 * ntok * dim * 2 bytes (bf16: rows and their residuals) or
+ * ntok * dim * 4 bytes (fp32), which must not exceed 8 MiB - 4 KiB (RDT_ERR_UNSUPPORTED
+ * otherwise); dim = 128 * 2^k <= 4096, n_experts <= 256, top_k <= min(n_experts, 16).
+ * The first call on a device (and the first after its context was re-created) looks up
+ * the array's device address (a runtime call, no allocation); make that first call before
+ * any stream capture. All calls share the array, and the counters and status words are
+ * cleared at the start of each call, so calls that overlap on the GPU (other streams,
+ * other threads) race: serialise them. */
 rdt_status rdt_moe_route_noalloc(int32_t dtype, const float* y, const float* norm2,
                                  const void* w_router, const float* router_bias, int ntok, int dim,
                                  int n_experts, int top_k, float eps, int32_t* topk_idx,
                                  float* topk_w, int32_t* expert_counts, void* stream);
+
+/* Status of the last rdt_moe_route_noalloc call on the current device: synchronises
+ * `stream` (the one that call used) and reads the router's device status word from the
+ * static array (no allocation). RDT_ERR_DEVICE_TIMEOUT if a bounded device-side wait of
+ * the tensor-core router gave up (its top-k outputs are then incomplete), else RDT_OK. */
+rdt_status rdt_moe_route_noalloc_status(void* stream);
 
 /* ---- per-kernel timing (CUDA events recorded around every launch of the handle) */
 typedef struct {
@@ -289,6 +306,14 @@ rdt_status rdt_profile(rdt_handle* h, int enable);
  * the handle has launched since create (counted whether or not timing is on). */
 rdt_status rdt_profile_read(rdt_handle* h, rdt_kernel_stat* out, int max_entries, int* n_entries,
                             int64_t* total_launches);
+
+/* Failure-detection probe of the bounded device-side waits (library diagnostics; the pages
+ * have no counterpart). Launches one kernel that waits, with the same bounded mbarrier wait
+ * every pipeline kernel uses but a limit of limit_ns (1 .. 2e9), on a barrier that nothing
+ * arrives on; the wait gives up, the kernel records the timeout in its status word and
+ * returns. Synchronises `stream`. Returns RDT_ERR_DEVICE_TIMEOUT, the expected outcome
+ * (the device context stays usable); INVALID_ARG for a limit out of range. */
+rdt_status rdt_wait_probe(int64_t limit_ns, void* stream);
 
 const char* rdt_status_string(rdt_status s);
 const char* rdt_last_error(void);

@@ -36,8 +36,8 @@ STATUS = {0: "RDT_OK", 1: "RDT_ERR_INVALID_ARG", 2: "RDT_ERR_UNSUPPORTED", 3: "R
 EXPORTED = ("rdt_create", "rdt_attn_forward", "rdt_moe_forward", "rdt_loop_forward",
             "rdt_loop_forward_host", "rdt_set_trace", "rdt_get_diagnostics", "rdt_memory_bytes",
             "rdt_status_string", "rdt_last_error", "rdt_destroy", "rdt_matmul", "rdt_attention",
-            "rdt_profile", "rdt_profile_read", "rdt_moe_route_noalloc", "rdt_set_act",
-            "rdt_loop_forward_act")
+            "rdt_profile", "rdt_profile_read", "rdt_moe_route_noalloc", "rdt_moe_route_noalloc_status",
+            "rdt_set_act", "rdt_loop_forward_act", "rdt_wait_probe")
 
 
 class RdtError(RuntimeError):
@@ -53,7 +53,7 @@ class RdtConfig(ctypes.Structure):
         ("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float)] + [
         (n, ctypes.c_int32) for n in ("n_experts", "top_k", "n_shared", "expert_hidden",
                                       "lora_rank", "n_lora", "b_kind", "inject_e", "max_loops",
-                                      "gemm_tiles")]
+                                      "gemm_tiles", "deterministic")]
 
 
 WEIGHT_FIELDS = ("A", "B", "norm1", "norm2", "wq", "wk", "wv", "wo", "w_dq", "q_norm", "w_uq",
@@ -108,6 +108,8 @@ def load_library() -> ctypes.CDLL:
     lib.rdt_matmul.argtypes = [i32, vp, vp, vp, i32, i32, i32, vp]
     lib.rdt_moe_route_noalloc.argtypes = [i32, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
                                           vp, vp, vp, vp]
+    lib.rdt_moe_route_noalloc_status.argtypes = [vp]
+    lib.rdt_wait_probe.argtypes = [ctypes.c_int64, vp]
     lib.rdt_profile.argtypes = [vp, i32]
     lib.rdt_profile_read.argtypes = [vp, ctypes.POINTER(RdtKernelStat), i32, ctypes.POINTER(i32),
                                      ctypes.POINTER(ctypes.c_int64)]
@@ -116,7 +118,7 @@ def load_library() -> ctypes.CDLL:
     for f in ("rdt_create", "rdt_attn_forward", "rdt_moe_forward", "rdt_loop_forward",
               "rdt_loop_forward_host", "rdt_set_trace", "rdt_get_diagnostics", "rdt_memory_bytes",
               "rdt_matmul", "rdt_attention", "rdt_profile", "rdt_profile_read", "rdt_moe_route_noalloc",
-              "rdt_set_act", "rdt_loop_forward_act"):
+              "rdt_set_act", "rdt_loop_forward_act", "rdt_moe_route_noalloc_status", "rdt_wait_probe"):
         getattr(lib, f).restype = i32
     _LIB = lib
     return lib
@@ -129,7 +131,7 @@ def _check(status: int) -> None:
 
 
 def make_config(wl, max_loops: int = 16, batch: Optional[int] = None, seq: Optional[int] = None,
-                gemm_tiles: int = 0) -> RdtConfig:
+                gemm_tiles: int = 0, deterministic: bool = False) -> RdtConfig:
     """Fill the C config from any object with the block's hyper-parameters as attributes."""
     c = RdtConfig()
     c.dtype = RDT_BF16 if wl.dtype == "bf16" else RDT_F32
@@ -157,6 +159,7 @@ def make_config(wl, max_loops: int = 16, batch: Optional[int] = None, seq: Optio
     c.inject_e = 1 if wl.inject_e else 0
     c.max_loops = max_loops
     c.gemm_tiles = gemm_tiles
+    c.deterministic = 1 if deterministic else 0
     return c
 
 

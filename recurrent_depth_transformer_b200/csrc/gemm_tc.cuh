@@ -414,7 +414,12 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, const EpiPre& pre, 
                 stage_get(stg, lane, it, o);
                 if (tok[it] < 0) continue;
                 const float4 add = make_float4(wt[it] * o[0], wt[it] * o[1], wt[it] * o[2], wt[it] * o[3]);
-                atomicAdd(reinterpret_cast<float4*>(p.dst + static_cast<size_t>(tok[it]) * p.ld + col + cc), add);
+                if (p.rows_out) {          // deterministic mode: the row's own slot, combined later
+                    const size_t r = static_cast<size_t>(row0 + it * 4 + (lane >> 3));
+                    *reinterpret_cast<float4*>(p.rows_out + r * p.ld + col + cc) = add;
+                } else {
+                    atomicAdd(reinterpret_cast<float4*>(p.dst + static_cast<size_t>(tok[it]) * p.ld + col + cc), add);
+                }
             }
         }
     } else if constexpr (KIND == EPI_TOPK) {

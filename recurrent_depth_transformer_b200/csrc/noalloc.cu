@@ -5,10 +5,10 @@
 // a handle and without any allocation, choosing its kernels exactly as the handle does:
 // routers whose weight fits in shared memory run the fused RMSNorm2 + fp32-logit kernel,
 // larger bf16 routers the RMSNorm2 split kernel and the tensor-core router GEMM, larger fp32
-// routers the fp32 FMA kernel. Their
-// scratch - the normalised rows (and, for bf16, their residuals) and the per-expert
-// counters - lives in the file-scope array below, which every process that loads librdt
-// holds on every GPU it uses until exit.
+// routers the fp32 FMA kernel. Their scratch - the per-expert counters, a status word and,
+// for the two larger-router paths, the normalised rows (bf16: also their residuals) - lives
+// in the file-scope array below, which every process that loads librdt holds on every GPU
+// it uses until exit.
 #include <mutex>
 
 #include "rdt_internal.cuh"
@@ -17,14 +17,31 @@ namespace rdt {
 namespace {
 
 constexpr size_t kScratchBytes = size_t(8) << 20;   // 8 MiB per device
-constexpr size_t kCountsBytes = 4096;               // 256 int32 counters, padded
+constexpr size_t kCountsBytes = 4096;               // 256 int32 counters, then the status words
+constexpr size_t kFlagsOffset = 1024;               // FLAG_COUNT int32 device status words
 static __device__ __align__(256) unsigned char g_route_scratch[kScratchBytes];
 
-// Device address of g_route_scratch, resolved once per device (host code cannot use the
-// symbol's name as a device address).
+// Device address of g_route_scratch, resolved once per (device, context): host code cannot
+// use the symbol's name as a device address, and a context created anew (after a device
+// reset) may load the module at another address, so the cached address is keyed on the
+// context current when it was looked up.
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_addr[kMaxDevices] = {};
+CUcontext g_ctx[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    }
+    return fn;
+}
 
 rdt_status scratch_address(void** out) {
     int dev = 0;
@@ -33,8 +50,21 @@ rdt_status scratch_address(void** out) {
         set_error("device index out of range for the router scratch table");
         return RDT_ERR_UNSUPPORTED;
     }
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    CUcontext ctx = nullptr;
+    if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS) {
+        set_error("cuCtxGetCurrent is unavailable");
+        return RDT_ERR_CUDA;
+    }
+    if (!ctx) {                                 // nothing initialised yet on this thread:
+        RDT_CUDA_TRY(cudaSetDevice(dev));       // make the device's primary context current
+        if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) {
+            set_error("no CUDA context is current");
+            return RDT_ERR_CUDA;
+        }
+    }
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_addr[dev]) {
+    if (!g_addr[dev] || g_ctx[dev] != ctx) {
         void* p = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
         if (e != cudaSuccess || p == nullptr) {
@@ -42,6 +72,7 @@ rdt_status scratch_address(void** out) {
             return RDT_ERR_CUDA;
         }
         g_addr[dev] = p;
+        g_ctx[dev] = ctx;
     }
     *out = g_addr[dev];
     return RDT_OK;
@@ -85,7 +116,11 @@ extern "C" rdt_status rdt_moe_route_noalloc(int32_t dtype, const float* y, const
     const bool bf = dtype == RDT_BF16;
     const size_t esz = bf ? 2 : 4;
     const size_t row_bytes = static_cast<size_t>(ntok) * dim * esz;
-    const size_t need = bf ? 2 * row_bytes : row_bytes;   // bf16: yn and its residual yn_lo
+    // Row scratch per path: the fused shared-memory router keeps its normalised rows in
+    // registers (none); the bf16 tensor-core router needs yn and its residual yn_lo; the
+    // fp32 FMA router writes yn.
+    const bool fused = router_fits_smem(bf, n_experts, top_k, dim);
+    const size_t need = fused ? 0 : bf ? 2 * row_bytes : row_bytes;
     if (need > kScratchBytes - kCountsBytes) {
         set_error("the router needs " + std::to_string(need) + " bytes of scratch for ntok = " +
                   std::to_string(ntok) + ", dim = " + std::to_string(dim) + "; the array holds " +
@@ -96,16 +131,18 @@ extern "C" rdt_status rdt_moe_route_noalloc(int32_t dtype, const float* y, const
     RDT_TRY(scratch_address(&base));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int* counts = static_cast<int*>(base);
+    int* flags = reinterpret_cast<int*>(static_cast<unsigned char*>(base) + kFlagsOffset);
     void* yn = static_cast<unsigned char*>(base) + kCountsBytes;
     void* yn_lo = static_cast<unsigned char*>(yn) + row_bytes;
-    RDT_CUDA_TRY(cudaMemsetAsync(counts, 0, kCountsBytes, st));   // the counters start at zero
+    // the counters and the status words start at zero
+    RDT_CUDA_TRY(cudaMemsetAsync(counts, 0, kCountsBytes, st));
 
-    if (router_fits_smem(bf, n_experts, top_k, dim)) {
+    if (fused) {
         // the same kernel as rdt_moe_forward for routers whose weight fits in shared memory
         RouterArgs ra{};
         ra.y = y;
         ra.gamma = norm2;
-        ra.yn = yn;
+        ra.yn = nullptr;             // no normalised copy: nothing here reads one
         ra.ntok = ntok;
         ra.dim = dim;
         ra.eps = eps;
@@ -116,7 +153,7 @@ extern "C" rdt_status rdt_moe_route_noalloc(int32_t dtype, const float* y, const
         ra.idx = topk_idx;
         ra.w = topk_w;
         ra.counts = counts;
-        ra.store_yn = 1;
+        ra.store_yn = 0;
         RDT_TRY(norm2_router_smem(bf, ra, st));
     } else if (bf) {
         // the same two steps as rdt_moe_forward: RMSNorm2 split into yn + yn_lo, then the
@@ -140,7 +177,9 @@ extern "C" rdt_status rdt_moe_route_noalloc(int32_t dtype, const float* y, const
         gr.N = n_experts;
         gr.kb_main = dim * 2 / 128;
         gr.kb_ext = gr.kb_main;
+        gr.flags = flags;           // a bounded wait that gives up is recorded here
         EpiParams er{};
+        er.flags = flags;
         er.kind = EPI_TOPK;
         er.n_exp = n_experts;
         er.top_k = top_k;
@@ -169,5 +208,20 @@ extern "C" rdt_status rdt_moe_route_noalloc(int32_t dtype, const float* y, const
     if (expert_counts)
         RDT_CUDA_TRY(cudaMemcpyAsync(expert_counts, counts, static_cast<size_t>(n_experts) * 4,
                                      cudaMemcpyDeviceToDevice, st));
+    return RDT_OK;
+}
+
+extern "C" rdt_status rdt_moe_route_noalloc_status(void* stream) {
+    void* base = nullptr;
+    RDT_TRY(scratch_address(&base));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    RDT_CUDA_TRY(cudaStreamSynchronize(st));
+    int flags[FLAG_COUNT];
+    RDT_CUDA_TRY(cudaMemcpy(flags, static_cast<unsigned char*>(base) + kFlagsOffset, sizeof(flags),
+                            cudaMemcpyDeviceToHost));
+    if (flags[FLAG_TIMEOUT]) {
+        set_error("a bounded device-side wait of the router gave up: its outputs are incomplete");
+        return RDT_ERR_DEVICE_TIMEOUT;
+    }
     return RDT_OK;
 }

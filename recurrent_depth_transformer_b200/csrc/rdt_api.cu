@@ -10,6 +10,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <new>
 #include <string>
 #include <vector>
 
@@ -74,6 +75,7 @@ struct rdt_handle {
     int max_tiles = 0;             // grouped GEMMs: bound on 128-row tiles
     int max_tiles_pair = 0;        // ... and on 256-row tiles
     int* flags = nullptr;
+    float* det_rows = nullptr;     // deterministic mode: [cap * (S + E), dim] expert row outputs
     void *stage_h0 = nullptr, *stage_e = nullptr;
     float* stage_out = nullptr;
 
@@ -128,11 +130,11 @@ constexpr int kFillerRows = 256;
 // kernel classes reported by rdt_profile_read
 enum Kind { K_HOIST, K_NORM1, K_GEMM_QKV, K_GEMM_LAT, K_MLA_NORM, K_GEMM_Q, K_ATTENTION, K_LORA_DOWN,
             K_GEMM_O, K_NORM2, K_ROUTER, K_DISPATCH, K_GEMM_UP, K_GEMM_DOWN, K_CHECK, K_DENSE_B, K_ACT,
-            K_COUNT };
+            K_COMBINE, K_COUNT };
 const char* const kKindName[K_COUNT] = {"hoist", "norm1", "gemm_qkv", "gemm_latent", "mla_latent_norm",
                                          "gemm_q_absorbed", "attention", "lora_down", "gemm_o",
                                          "norm2", "router_topk", "moe_dispatch", "gemm_up", "gemm_down",
-                                         "check_finite", "dense_injection", "act_halting"};
+                                         "check_finite", "dense_injection", "act_halting", "moe_combine"};
 
 rdt_status prof_begin(rdt_handle* h, int kind, int nlaunch, cudaStream_t st) {
     h->launches += nlaunch;
@@ -219,6 +221,7 @@ rdt_status validate_config(const rdt_config* c) {
     if (c->dtype == RDT_F32 && c->expert_hidden % 128) return uns("f32: expert_hidden % 128 != 0");
     if (c->max_loops < 1 || c->max_loops > 64) return bad("max_loops must be in [1, 64]");
     if (c->gemm_tiles < 0 || c->gemm_tiles > 2) return bad("gemm_tiles must be 0, 1 or 2");
+    if (c->deterministic != 0 && c->deterministic != 1) return bad("deterministic must be 0 or 1");
     if (c->b_kind != RDT_B_DIAG && c->b_kind != RDT_B_DENSE) return bad("b_kind");
     if (!(c->norm_eps >= 0.0f) || !(c->rope_base > 1.0f)) return bad("norm_eps / rope_base");
     if (c->lora_rank < 0 || c->n_lora < 0) return bad("lora");
@@ -465,7 +468,8 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         // the down-projection's epilogue reduces every output into h_next; on pairs a CTA's
         // share of it doubles and measured slower (24.3 vs 23.7 us), so it runs on pairs only
         // when they are forced
-        t = choose_tiles(grows, E + S, d, kb_h, true, false, mode == 2, 4, mode);
+        // deterministic mode: no K split (its partial sums would meet in atomics)
+        t = choose_tiles(grows, E + S, d, kb_h, true, false, mode == 2, c.deterministic ? 1 : 4, mode);
         h->bn_down = t.bn;
         h->pair_down = t.pair;
         h->split_down = t.split;
@@ -622,7 +626,7 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         const int mt = (N + 127) / 128;
         const int kb = 2 * d * 2 / 128;
         int split = 1;
-        for (int sp = 1; sp <= kb; ++sp)
+        for (int sp = 1; sp <= kb && !c.deterministic; ++sp)   // deterministic: logits in one CTA
             if (kb % sp == 0 && static_cast<long>(mt) * sp <= num_sms()) split = sp;
         h->router_split = split;
         RDT_TRY(dev_alloc(h, &h->logits, static_cast<size_t>(N) * E * 4, true));
@@ -637,6 +641,8 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
     h->max_tiles = (N * K + 127) / 128 + E + S * ((N + 127) / 128);
     h->max_tiles_pair = (N * K + 255) / 256 + E + S * ((N + 255) / 256);
     RDT_TRY(dev_alloc(h, &h->flags, FLAG_COUNT * 4, true));
+    if (c.deterministic)
+        RDT_TRY(dev_alloc(h, &h->det_rows, static_cast<size_t>(h->cap) * (S + E) * d * 4));
     RDT_TRY(dev_alloc(h, &h->stage_h0, nd * es));
     RDT_TRY(dev_alloc(h, &h->stage_e, nd * es));
     RDT_TRY(dev_alloc(h, &h->stage_out, nd * 4));
@@ -852,6 +858,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
         ra.xperm = h->xperm;
         ra.a_routed_base = N;
         ra.store_yn = c.n_shared > 0;          // shared experts read yn itself
+        if (h->det_rows) ra.slot_row = h->slot_row;   // the combine finds each slot's row
         ra.weights_static = 1;                 // the library's own copy, written at create
         ra.halted = halted;
         TIMED(h, K_ROUTER, 1, st, norm2_router_smem(h->bf, ra, st));
@@ -969,8 +976,11 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     ed.ntok = h->cap;
     ed.dst = dst;
     ed.ld = d;
+    ed.rows_out = h->det_rows;
     ed.flags = h->flags;
     TIMED(h, K_GEMM_DOWN, 1, st, gemm_tc(h->bf, h->bn_down, h->m_U, h->m_w2, nullptr, nullptr, gd, ed, st));
+    if (h->det_rows)
+        TIMED(h, K_COMBINE, 1, st, moe_combine(h->det_rows, h->slot_row, N, c.top_k, c.n_shared, h->cap, dst, d, st));
     return RDT_OK;
 }
 
@@ -1117,8 +1127,21 @@ rdt_status rdt_create(const rdt_config* cfg, const rdt_weights* w, void* stream,
         set_error("weights is NULL");
         return RDT_ERR_INVALID_ARG;
     }
-    rdt_handle* h = new rdt_handle();
-    const rdt_status s = create_impl(cfg, w, static_cast<cudaStream_t>(stream), h);
+    rdt_handle* h = new (std::nothrow) rdt_handle();
+    if (!h) {
+        set_error("host allocation of the handle failed");
+        return RDT_ERR_OOM;
+    }
+    rdt_status s = RDT_ERR_OOM;
+    try {          // std::vector growth inside may throw: no exception crosses the C ABI
+        s = create_impl(cfg, w, static_cast<cudaStream_t>(stream), h);
+    } catch (const std::bad_alloc&) {
+        set_error("host allocation failed during create");
+        s = RDT_ERR_OOM;
+    } catch (...) {
+        set_error("unexpected host exception during create");
+        s = RDT_ERR_CUDA;
+    }
     if (s != RDT_OK) {
         rdt_destroy(h);
         return s;
@@ -1139,7 +1162,7 @@ static rdt_status check_ptr(const void* p, const char* name) {
     return RDT_OK;
 }
 
-rdt_status rdt_attn_forward(rdt_handle* h, const float* x, int loop, float* a_out, void* stream) {
+rdt_status rdt_attn_forward(rdt_handle* h, const void* x, int loop, float* a_out, void* stream) {
     if (!h) {
         set_error("handle is NULL");
         return RDT_ERR_INVALID_ARG;
@@ -1152,7 +1175,9 @@ rdt_status rdt_attn_forward(rdt_handle* h, const float* x, int loop, float* a_ou
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     h->last_stream = st;
-    return attention_block(h, x, nullptr, loop, false, a_out, nullptr, st);
+    // x in the configuration's element type enters RMSNorm1 through its injection operand
+    // (block input = e alone when the state operand is absent)
+    return attention_block(h, nullptr, x, loop, false, a_out, nullptr, st);
 }
 
 rdt_status rdt_moe_forward(rdt_handle* h, const float* y, float* f_out, int32_t* topk_idx, float* topk_w,
@@ -1239,9 +1264,16 @@ rdt_status rdt_set_act(rdt_handle* h, const float* w_halt, float b_halt, float t
         return RDT_ERR_UNSUPPORTED;
     }
     if (!h->act_w) {
-        RDT_TRY(dev_alloc(h, &h->act_w, static_cast<size_t>(d) * 4));
-        RDT_TRY(dev_alloc(h, &h->act_cum, static_cast<size_t>(N) * 4, true));
-        RDT_TRY(dev_alloc(h, &h->act_loops, static_cast<size_t>(N) * 4, true));
+        // all three or none: the handle keeps them only once every allocation succeeded
+        // (a failed one leaves the others in the handle's list, freed by rdt_destroy)
+        float *w = nullptr, *cum = nullptr;
+        int* loops = nullptr;
+        RDT_TRY(dev_alloc(h, &w, static_cast<size_t>(d) * 4));
+        RDT_TRY(dev_alloc(h, &cum, static_cast<size_t>(N) * 4, true));
+        RDT_TRY(dev_alloc(h, &loops, static_cast<size_t>(N) * 4, true));
+        h->act_w = w;
+        h->act_cum = cum;
+        h->act_loops = loops;
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     RDT_CUDA_TRY(cudaMemcpyAsync(h->act_w, w_halt, static_cast<size_t>(d) * 4, cudaMemcpyDeviceToDevice, st));

@@ -156,16 +156,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Wait for the phase of parity `parity` to complete, at most kWaitLimitNs. On timeout
-// sets flags[FLAG_TIMEOUT] and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* flags) {
+// Wait for the phase of parity `parity` to complete, at most limit_ns (kWaitLimitNs in
+// every pipeline kernel). On timeout sets flags[FLAG_TIMEOUT] and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* flags,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
 #pragma unroll 1
         for (int i = 0; i < 256; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             if (flags) atomicExch(flags + FLAG_TIMEOUT, 1);
             return false;
         }
@@ -411,6 +412,8 @@ struct EpiParams {
     int shared_rows;       // rows [0, shared_rows) are shared-expert rows: token = row % ntok
     int ntok;              // scatter: row stride of the shared groups in U
     float* dst;            // scatter destination [ntok, ld]
+    float* rows_out;       // scatter, deterministic mode: w * acc stored at its own row
+                           // ([rows, ld], the tile's output row index) instead of reduced
     // router top-k (and dispatch: claim a row of each chosen expert)
     int n_exp, top_k;
     int* route_token;      // [n_exp * cap] token of each claimed row (or NULL: no dispatch)
@@ -476,7 +479,7 @@ rdt_status attention_tc(const AttnArgs& a, cudaStream_t st);
 
 // Row kernels (rowops.cu).
 struct Norm1Args {
-    const float* h;    // fp32 state, or the fp32 block input x when e == NULL
+    const float* h;    // fp32 state (NULL: none, the block input x is e alone)
     const void* e;     // cfg-dtype injection (x = h + e) or NULL
     const float* gamma;
     void* xn;          // [N, dim] cfg dtype
@@ -526,6 +529,12 @@ rdt_status norm2_router_smem(bool bf16_elems, const RouterArgs& a, cudaStream_t 
 // a slot whose claimed row is negative (a halted token) is skipped.
 rdt_status moe_copy(bool bf16_elems, void* xperm, const int* slot_row, int ntok, int top_k, int dim,
                     int a_routed_base, cudaStream_t st);
+
+// Deterministic combine of the expert outputs: for each token n, in this order,
+// dst[n] += rows[s * cap + n] for every shared expert s, then dst[n] += rows[n_shared * cap
+// + slot_row[n * top_k + j]] for j = 0 .. top_k - 1 (slots with a negative row are skipped).
+rdt_status moe_combine(const float* rows, const int* slot_row, int ntok, int top_k, int n_shared, int cap,
+                       float* dst, int dim, cudaStream_t st);
 
 rdt_status lora_down(bool bf16_elems, const void* x, int ldx, int ntok, int width,
                      const void* lora_a, int r, void* t_out, cudaStream_t st);

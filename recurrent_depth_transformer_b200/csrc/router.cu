@@ -139,6 +139,7 @@ __global__ void __launch_bounds__(kRouterMaxThreads, 2) norm2_router_smem_kernel
                 a.w[o] = 0.0f;
                 if (a.trace_idx) a.trace_idx[o] = -1;
                 if (a.trace_w) a.trace_w[o] = 0.0f;
+                if (a.slot_row) a.slot_row[o] = -1;
             }
             continue;
         }
@@ -237,6 +238,7 @@ __global__ void __launch_bounds__(kRouterMaxThreads, 2) norm2_router_smem_kernel
                     a.row_token[rr] = row;
                     a.row_w[rr] = wv;
                 }
+                if (a.slot_row) a.slot_row[o] = rr;
             }
             if (a.xperm) {                                       // the expert's copy of yn
                 rr = __shfl_sync(0xffffffffu, rr, r);

@@ -99,7 +99,12 @@ __global__ void __launch_bounds__(kRowThreads, NV <= 8 ? 2 : 1) norm1_kernel(con
 #pragma unroll
         for (int i = 0; i < GV; ++i) {
             const int col = (i0 + i) * 128 + lane * 4;
-            load4(a.h + base + col, x[i0 + i]);
+            if (a.h) {
+                load4(a.h + base + col, x[i0 + i]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) x[i0 + i][j] = 0.0f;
+            }
             if (e) load4(e + base + col, ev[i]);
             if (a.hn0) {
                 load4(a.Be + base + col, be[i]);
@@ -361,6 +366,44 @@ __global__ void __launch_bounds__(kRowThreads) moe_copy_kernel(T* xperm, const i
     for (int i = lane; i < nvec; i += 32) dst[i] = src[i];
 }
 
+// ----------------------------------------------------------------------------- deterministic combine
+
+// One warp per token: the token's expert outputs (each stored in its own row by the
+// down-projection) are added into dst in a fixed order - shared experts first, then the
+// routed slots 0 .. top_k - 1 - so that the fp32 sums do not depend on scheduling.
+template <int NV>
+__global__ void __launch_bounds__(kRowThreads) moe_combine_kernel(const float* rows, const int* slot_row,
+                                                                  int ntok, int top_k, int n_shared, int cap,
+                                                                  float* dst) {
+    pdl_trigger();
+    pdl_wait();
+    const int n = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (n >= ntok) return;
+    constexpr int dim = NV * 128;
+    float acc[NV][4];
+    float* d = dst + static_cast<size_t>(n) * dim;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) load4(d + i * 128 + lane * 4, acc[i]);
+    auto add_row = [&](size_t r) {
+        const float* src = rows + r * dim;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            float v[4];
+            load4(src + i * 128 + lane * 4, v);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] += v[j];
+        }
+    };
+    for (int s = 0; s < n_shared; ++s) add_row(static_cast<size_t>(s) * cap + n);
+    for (int j = 0; j < top_k; ++j) {
+        const int r = slot_row[static_cast<size_t>(n) * top_k + j];
+        if (r >= 0) add_row(static_cast<size_t>(n_shared) * cap + r);
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) store4(d + i * 128 + lane * 4, acc[i]);
+}
+
 // ----------------------------------------------------------------------------- LoRA down
 
 template <typename T, int NV>
@@ -542,6 +585,14 @@ struct ActL {
     }
 };
 template <typename T, int NV>
+struct CombineL {
+    static void run(dim3 g, cudaStream_t st, const float* rows, const int* slot_row, int ntok, int top_k,
+                    int n_shared, int cap, float* dst) {
+        launch_pdl(moe_combine_kernel<NV>, g, dim3(kRowThreads), 0, st, rows, slot_row, ntok, top_k, n_shared,
+                   cap, dst);
+    }
+};
+template <typename T, int NV>
 struct Norm2L {
     static void run(dim3 g, cudaStream_t st, Norm2Args a) {
         launch_pdl(norm2_split_kernel<T, NV>, g, dim3(kRowThreads), 0, st, a);
@@ -633,6 +684,11 @@ rdt_status mla_latent_norm(bool bf, const MlaNormArgs& a, cudaStream_t st) {
         RDT_CUDA_TRY(launch_pdl(mla_latent_norm_kernel<float>, grid, dim3(kRowThreads), 0, st, a));
     RDT_CUDA_TRY(cudaGetLastError());
     return RDT_OK;
+}
+
+rdt_status moe_combine(const float* rows, const int* slot_row, int ntok, int top_k, int n_shared, int cap,
+                       float* dst, int dim, cudaStream_t st) {
+    return launch_rows<float, CombineL>(dim / 128, ntok, st, rows, slot_row, ntok, top_k, n_shared, cap, dst);
 }
 
 rdt_status prep_matmul(bool bf, const void* A, long sam, long sak, const void* B, long sbk,

@@ -60,11 +60,28 @@ def run_act(wl, inputs, T, head, traj=True, h=None):
     return res
 
 
-def oracle_act(wl, inputs, T, head, idx, n_loops):
+def oracle_act(wl, inputs, T, head, idx, n_loops, trace=None):
     N = wl.batch * wl.seq
     follow = [idx[t].reshape(N, wl.top_k) for t in range(T)]
     return O.loop_forward_act(inputs["h0"], inputs["e"], T, inputs, wl, head["w_halt"], head["b_halt"],
-                              head["threshold"], follow=follow, follow_loops=n_loops)
+                              head["threshold"], follow=follow, follow_loops=n_loops, trace=trace)
+
+
+def running_sums(states, head, n_loops, T):
+    """c + p_t of every position still running at loop t (NaN once halted), from the states
+    h_1 .. h_T of one implementation, in fp64."""
+    N = n_loops.size
+    nl = n_loops.reshape(N)
+    w = np.asarray(head["w_halt"], dtype=np.float64)
+    c = np.zeros(N)
+    out = np.full((T, N), np.nan)
+    for t in range(T):
+        run = nl > t
+        h = np.asarray(states[t + 1], dtype=np.float64).reshape(N, -1)
+        reach = c + 1.0 / (1.0 + np.exp(-(h @ w + head["b_halt"])))
+        out[t, run] = reach[run]
+        c = np.where(run, reach, c)
+    return out
 
 
 def check_self_consistent(wl, head, T, out, nl, idx, traj, band=1e-4):
@@ -104,11 +121,23 @@ def test_act_matches_oracle_small(name):
     assert diag["nonfinite"] == 0 and diag["timeout"] == 0
     assert len(np.unique(nl)) >= 2, "the head must halt tokens at different loops"
     check_self_consistent(wl, head, T, out, nl, idx, traj)
-    r = oracle_act(wl, inputs, T, head, idx, nl)
+    tr = O.LoopTrace()
+    r = oracle_act(wl, inputs, T, head, idx, nl, trace=tr)
     assert r.stats["mismatch"] == 0, f"{r.stats['mismatch']} routing differences outside near-ties"
     assert r.stats["halt_mismatch"] == 0, f"{r.stats['halt_mismatch']} halting differences outside the band"
     np.testing.assert_array_equal(r.n_loops, nl)
     assert_close(out, r.out, what=f"{name} ACT")
+    # Evidence for the follow band: how far the GPU's running sums c + p_t (from its fp32
+    # states) are from the oracle's (fp64 states), and how many decisions the oracle adopted.
+    gpu = running_sums(traj, head, nl, T)
+    ora = running_sums(tr.h, head, nl, T)
+    diff = np.nanmax(np.abs(gpu - ora))
+    n = wl.batch * wl.seq
+    print(f"ACT band {name}: max|sum_p gpu - oracle| = {diff:.3e} over {np.count_nonzero(~np.isnan(gpu))} "
+          f"running (token, loop) pairs; {r.stats['near_halts']} of {n} decisions adopted in the "
+          f"{O.NEAR_HALT:g} band")
+    assert diff < O.NEAR_HALT / 2, "the band must cover the measured difference with margin"
+    assert r.stats["near_halts"] <= max(2, n // 100)
 
 
 def test_act_certain_halt_is_one_loop():

@@ -95,3 +95,41 @@ def test_attention_shared_latent_kv(batch, seq, hq):
     ref = O.gqa_attention(q.float().numpy().reshape(batch, seq, hq, 160), kf, kf[..., :128], scale)
     err = np.abs(o.cpu().float().numpy().reshape(ref.shape) - ref).max()
     assert err < 2e-2, err
+
+
+@pytest.mark.parametrize("kind", ["gqa", "mla"])
+def test_attention_long_sequence_rows_from_every_tile(kind):
+    """Causal attention at the long configuration's length (8192 positions): about 256 query
+    rows drawn from every 128-row query tile, for two heads, element by element against the
+    oracle's attention at those positions (keys 0 .. position)."""
+    torch = _torch()
+    import recurrent_depth_transformer_b200 as R
+    S = 8192
+    if kind == "gqa":
+        hq, hkv, dqk, dv = 32, 8, 64, 64
+    else:
+        hq, hkv, dqk, dv = 16, 1, 160, 128
+    g = torch.Generator().manual_seed(S + dqk)
+    q = torch.randn(S, hq * dqk, generator=g).to(torch.bfloat16)
+    k = torch.randn(S, hkv * dqk, generator=g).to(torch.bfloat16)
+    scale = 1.0 / math.sqrt(64 if kind == "gqa" else 96)
+    kc = k.cuda()
+    if kind == "gqa":
+        v = torch.randn(S, hkv * dv, generator=g).to(torch.bfloat16)
+        o = R.attention(q.cuda(), kc, v.cuda(), 1, S, hq, hkv, dqk, dv, scale)
+    else:
+        v = k[:, :dv]
+        o = R.attention(q.cuda(), kc, kc, 1, S, hq, 1, dqk, dv, scale)
+    torch.cuda.synchronize()
+    got = o.cpu().float().numpy().reshape(S, hq, dv)
+    rng = np.random.default_rng(11)
+    pos = np.sort(np.concatenate([np.arange(0, S, 128) + rng.integers(0, 128, S // 128),
+                                  rng.integers(0, S, 192), [0, 127, 128, S - 1]]))
+    qf = q.float().numpy().reshape(S, hq, dqk)
+    kf = k.float().numpy().reshape(S, hkv, dqk)
+    vf = v.float().numpy().reshape(S, hkv, dv)
+    for h in (0, hq - 1):
+        kv = (h * hkv) // hq
+        ref = O.causal_attention(qf[pos, h], kf[:, kv], vf[:, kv], scale, q_pos=pos)
+        err = np.abs(got[pos, h] - ref).max()
+        assert err < 2e-2, (h, err)

@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 
 import oracle as O
-from workloads import WORKLOADS, generate, prefix
+from workloads import WORKLOADS, generate, prefix, round_bf16
 
 from rdt_testlib import (MAX_ABS, REL_FRO, act, assert_close, errors, handle, oracle_follow,
                          run_loop, torch_mod)
@@ -127,8 +127,10 @@ def test_attention_sublayer():
     for wl in (C0, C1.replace(batch=2, seq=200), C2.replace(batch=2, seq=136), C4.replace(seq=192)):
         inputs = generate(wl)
         x = inputs["e"].astype(np.float32) * 1.5 + 0.25
+        if wl.dtype == "bf16":
+            x = round_bf16(x)                    # x is passed in the configuration's type
         with handle(wl, inputs) as h:
-            a = h.attn_forward(torch.from_numpy(x).cuda(), loop=1)
+            a = h.attn_forward(act(wl, x), loop=1)
             torch.cuda.synchronize()
             got = a.cpu().numpy()
         want = O.attention_sublayer(x, inputs, wl, 1)
@@ -179,9 +181,9 @@ def test_T1_equals_sublayer_composition():
     with handle(wl, inputs) as h:
         e = act(wl, inputs["e"])
         hT = h.loop_forward(e, e, 1)
-        x0 = e.float() + e.float()
+        x0 = e + e                          # exact in bf16: the block input h0 + e
         a = h.attn_forward(x0, loop=0)
-        f = h.moe_forward(x0 + a)
+        f = h.moe_forward(x0.float() + a)
         A = torch.from_numpy(inputs["A"]).cuda()
         B = torch.from_numpy(inputs["B"]).cuda()
         comp = A * e.float() + B * e.float() + a + f
@@ -220,11 +222,30 @@ def test_host_entry_matches_device_entry():
     assert ma < 1e-3
 
 
+def sampled_rows(wl, seed, per_batch_min=8, total_min=32):
+    """(batch, position) pairs covering every 128-row query tile of every sequence (one
+    random row per tile band, plus each sequence's last row), topped up with random rows
+    until there are at least total_min."""
+    rng = np.random.default_rng(seed)
+    rows = set()
+    for b in range(wl.batch):
+        for t0 in range(0, wl.seq, 128):
+            rows.add((b, int(t0 + rng.integers(0, min(128, wl.seq - t0)))))
+        rows.add((b, wl.seq - 1))
+        while sum(1 for bb, _ in rows if bb == b) < per_batch_min:
+            rows.add((b, int(rng.integers(0, wl.seq))))
+    while len(rows) < total_min:
+        rows.add((int(rng.integers(wl.batch)), int(rng.integers(0, wl.seq))))
+    return sorted(rows)
+
+
 @pytest.mark.parametrize("wi", [1, 2, 3, 4])
 def test_full_size_prefix_and_sampled_rows(wi):
     """The configuration at its full size in the benchmark's launch configuration: the first
-    64 positions of every sequence against the oracle (causality makes them independent of
-    later positions), and the last loop at sampled late positions from the GPU's own h_{T-1}."""
+    64 positions of every sequence through all loops against the oracle (causality makes
+    them independent of later positions); and at the first and the last loop, rows from
+    every 128-row query tile of every sequence, each computed by the oracle's single-step
+    evaluation from the GPU's own state before that loop."""
     wl = WORKLOADS[wi]
     T = max(wl.loops)
     inputs = generate(wl)
@@ -237,15 +258,15 @@ def test_full_size_prefix_and_sampled_rows(wi):
     want, mism, _, _ = oracle_follow(pwl, pin, T, pidx)
     assert mism == 0
     assert_close(got[:, :P], want, what=f"{wl.name} prefix")
-    rng = np.random.default_rng(wi)
-    rows = [(int(rng.integers(wl.batch)), int(s)) for s in
-            (wl.seq - 1, wl.seq // 2 + 1, int(rng.integers(P, wl.seq)))]
-    hT1 = traj[T - 1].reshape(wl.batch, wl.seq, wl.dim)
-    fidx = np.stack([idx[T - 1].reshape(wl.batch, wl.seq, -1)[b, s] for b, s in rows])
-    hn, r, st = O.loop_step_rows(hT1, inputs["e"], inputs, wl, T - 1, rows, follow_idx=fidx)
-    assert st["mismatch"] == 0
-    gt = np.stack([got[b, s] for b, s in rows])
-    assert_close(gt, hn, what=f"{wl.name} sampled rows")
+    rows = sampled_rows(wl, wi)
+    H = traj.reshape(T + 1, wl.batch, wl.seq, wl.dim)
+    for t in (0, T - 1):
+        fidx = np.stack([idx[t].reshape(wl.batch, wl.seq, -1)[b, s] for b, s in rows])
+        hn, r, st = O.loop_step_rows(H[t], inputs["e"], inputs, wl, t, rows, follow_idx=fidx)
+        assert st["mismatch"] == 0
+        gt = np.stack([H[t + 1][b, s] for b, s in rows])
+        assert_close(gt, hn, what=f"{wl.name} loop {t}, {len(rows)} sampled rows")
+    np.testing.assert_array_equal(H[T], got)
 
 
 def test_invalid_arguments_return_errors():
