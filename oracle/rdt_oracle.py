@@ -309,10 +309,12 @@ def attention_sublayer(x, W, cfg, t: int, mla_form: str = "explicit") -> np.ndar
     return out_proj(o, W, cfg, t)
 
 
-def moe_sublayer(y, W, cfg, follow_idx=None) -> Tuple[np.ndarray, Routing, Dict[str, int]]:
+def moe_sublayer(y, W, cfg, follow_idx=None, tie_band: float = NEAR_TIE) -> Tuple[np.ndarray, Routing, Dict[str, int]]:
     """f = MoE(RMSNorm2(y)). With ``follow_idx`` (another implementation's selection),
-    tokens whose k-th/(k+1)-th score gap is at most NEAR_TIE adopt that selection;
-    every other token keeps its own and is counted if the two sets differ."""
+    tokens whose k-th/(k+1)-th score gap is at most ``tie_band`` (NEAR_TIE by default)
+    adopt that selection; every other token keeps its own and is counted if the two sets
+    differ. ``tie_band = inf`` adopts the other selection everywhere (gate weights still
+    from this oracle's logits)."""
     y = _f(y)
     shp = y.shape
     yn = rmsnorm(y, W["norm2"], cfg.norm_eps).reshape(-1, shp[-1])
@@ -321,7 +323,7 @@ def moe_sublayer(y, W, cfg, follow_idx=None) -> Tuple[np.ndarray, Routing, Dict[
     idx = r.idx
     if follow_idx is not None:
         fi = np.asarray(follow_idx).reshape(idx.shape)
-        near = r.gap <= NEAR_TIE
+        near = r.gap <= tie_band
         same = np.all(np.sort(fi, axis=1) == np.sort(idx, axis=1), axis=1)
         stats["near_ties"] = int(np.count_nonzero(near & ~same))
         stats["mismatch"] = int(np.count_nonzero(~near & ~same))
@@ -360,13 +362,14 @@ class LoopTrace:
 
 
 def loop_forward(h0, e, T: int, W, cfg, follow: Optional[Sequence[np.ndarray]] = None,
-                 trace: Optional[LoopTrace] = None, mla_form: str = "explicit") -> np.ndarray:
+                 trace: Optional[LoopTrace] = None, mla_form: str = "explicit",
+                 tie_band: float = NEAR_TIE) -> np.ndarray:
     """h_{t+1} = A.h_t + B.e + Transformer(h_t, e) for t = 0..T-1 ([TB] update equation;
     [GS] Passo 3: the same block repeated n_loops times).
 
     Transformer(h, e) = a + f with x = h + e (or x = h), a = Attn(RMSNorm1(x)),
     y = x + a, f = MoE(RMSNorm2(y)). ``follow[t]`` is an optional [N, k] selection to
-    adopt on near-ties at loop t (see :func:`moe_sublayer`).
+    adopt on near-ties at loop t, those within ``tie_band`` (see :func:`moe_sublayer`).
     """
     A = _f(W["A"])
     e = _f(e)
@@ -378,7 +381,7 @@ def loop_forward(h0, e, T: int, W, cfg, follow: Optional[Sequence[np.ndarray]] =
         x = h + e if cfg.inject_e else h
         a = attention_sublayer(x, W, cfg, t, mla_form)
         y = x + a
-        f, r, st = moe_sublayer(y, W, cfg, None if follow is None else follow[t])
+        f, r, st = moe_sublayer(y, W, cfg, None if follow is None else follow[t], tie_band)
         delta = a + f
         h = A * h + Be + delta
         if trace is not None:

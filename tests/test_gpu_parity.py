@@ -251,15 +251,26 @@ def test_full_size_prefix_and_sampled_rows(wi):
     inputs = generate(wl)
     got, idx, _, traj, diag = run_loop(wl, inputs, T, traj=True)
     assert diag["nonfinite"] == 0 and diag["timeout"] == 0
+    H = traj.reshape(T + 1, wl.batch, wl.seq, wl.dim)
     P = 64
     pin = prefix(inputs, P)
     pwl = wl.replace(seq=P)
     pidx = idx.reshape(T, wl.batch, wl.seq, wl.top_k)[:, :, :P]
-    want, mism, _, _ = oracle_follow(pwl, pin, T, pidx)
-    assert mism == 0
+    # every loop from the GPU's own state: routing identical outside near-ties (one loop of
+    # rounding between the two), the next state within the bounds
+    prows = [(b, s) for b in range(wl.batch) for s in range(P)]
+    for t in range(T):
+        fidx = pidx[t].reshape(-1, wl.top_k)
+        want1, _, st = O.loop_step_rows(H[t][:, :P], pin["e"], pin, pwl, t, prows, follow_idx=fidx)
+        assert st["mismatch"] == 0, f"loop {t}: {st['mismatch']} routing differences outside near-ties"
+        assert_close(H[t + 1][:, :P].reshape(-1, wl.dim), want1, what=f"{wl.name} prefix, loop {t} from the GPU's state")
+    # all T loops from h0: over many loops the two trajectories drift apart (within the
+    # bounds), enough to move logits by more than the near-tie gap, so the oracle adopts the
+    # GPU's routing everywhere here and the states are compared
+    want = O.loop_forward(pin["h0"], pin["e"], T, pin, pwl,
+                          follow=[pidx[t].reshape(-1, wl.top_k) for t in range(T)], tie_band=np.inf)
     assert_close(got[:, :P], want, what=f"{wl.name} prefix")
     rows = sampled_rows(wl, wi)
-    H = traj.reshape(T + 1, wl.batch, wl.seq, wl.dim)
     for t in (0, T - 1):
         fidx = np.stack([idx[t].reshape(wl.batch, wl.seq, -1)[b, s] for b, s in rows])
         hn, r, st = O.loop_step_rows(H[t], inputs["e"], inputs, wl, t, rows, follow_idx=fidx)
