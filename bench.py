@@ -1,25 +1,30 @@
 #!/usr/bin/env python
 """Throughput of the looped recurrent block on B200 through the librdt C ABI.
 
-One step = one rdt_loop_forward call: T = 8 loops of the GQA block (batch 4 x seq 512,
-dim 1024, 16/4 heads of 64, 16 experts top-2, SwiGLU hidden 1024, bf16 storage, fp32
-state) on seeded synthetic inputs resident in HBM. The L2 cache is flushed (256 MiB
-write) before every timed step; each step is timed with CUDA events on its stream.
+One step = one rdt_loop_forward call: T loops of the block over one batch of seeded
+synthetic inputs resident in HBM. The headline workload is the largest single-GPU
+configuration: the long-context GQA block with depth-wise LoRA (batch 1 x seq 8192, dim
+2048, 32/8 heads of 64, 64 experts top-8 with SwiGLU hidden 512, LoRA rank 16 on Q and O),
+T = 16 loops, bf16 storage and an fp32 state. The L2 cache is flushed (256 MiB write)
+before every timed step; each step is timed with CUDA events on its stream and the median
+step is reported.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--act]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload NAME] [--loops T] [--act] [--all]
 
-N > 1 runs under torchrun: every rank runs its own full replica (no data-path
-collective; weak scaling); the timed region is bracketed by a barrier and a device
-synchronise, and the step time is the maximum over ranks. `--impl reference` times the
-fp64 CPU oracle on the host cores instead (rank 0 only). `--act` times the same workload
-through rdt_loop_forward_act (ACT halting, threshold 0.99, the seeded halting head) and
-reports the halting histogram; its tokens·loops count the T = 8 loops asked for.
+--gpus N > 1 runs one process per GPU (re-launched under torch.distributed.run when not
+started by it): every rank runs a replica of the workload on inputs of its own (no
+data-path collective; weak scaling); the timed region is bracketed by a barrier and a
+device synchronise and the step time is the maximum over ranks. `--impl reference` times
+the fp64 CPU oracle on the host cores instead (rank 0 only). `--act` times the same
+workload through rdt_loop_forward_act (ACT halting, threshold 0.99, the seeded halting
+head). `--all` prints one line for every configuration and loop count of the workload
+list instead of the headline line.
 """
 from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -31,24 +36,31 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-WORKLOAD = "gqa-bf16-b4s512-d1024-h16x4-e16k2"
-LOOPS = 8
+WORKLOAD = "long-bf16-b1s8192-d2048-h32x8-e64k8-lora16"
+LOOPS = 16
 METRIC = "recurrent-block tokens·loops/sec (bf16 fwd, 1 B200) and % of roofline"
 UNIT = "tokens*loops/s"
 FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# CPU-baseline sample: at most this many seconds of oracle work per timed sample
+CPU_SECONDS = 30.0
 
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of a kernel, from one
-# ncu capture of this workload, valid only while the kernel's code is the one captured
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of a kernel on a
+# workload, from one ncu capture, valid only while the kernel's code is the one captured
 # (fingerprint: first 16 hex digits of the SHA-256 of the listed files' code, concatenated:
 # comments removed, each line stripped, blank lines dropped, so that an edit of a comment
 # or of indentation keeps the capture while any change to a code token voids it).
-KERNEL_SOURCES = {"gemm_up": ("recurrent_depth_transformer_b200/csrc/gemm_tc.cuh",
-                              "recurrent_depth_transformer_b200/csrc/gemm_tc.cu",
-                              "recurrent_depth_transformer_b200/csrc/gemm_tc_pair.cu",
-                              "recurrent_depth_transformer_b200/csrc/rdt_internal.cuh",
-                              "recurrent_depth_transformer_b200/csrc/rdt_api.cu")}
-MEASURED_TRAFFIC = {"gemm_up": (79.72864e6 + 2.450688e6, "77aada7e305fe0e8")}
+KERNEL_SOURCES = {
+    "attention": ("recurrent_depth_transformer_b200/csrc/attention_tc.cu",
+                  "recurrent_depth_transformer_b200/csrc/rdt_internal.cuh"),
+    "gemm_up": ("recurrent_depth_transformer_b200/csrc/gemm_tc.cuh",
+                "recurrent_depth_transformer_b200/csrc/gemm_tc.cu",
+                "recurrent_depth_transformer_b200/csrc/gemm_tc_pair.cu",
+                "recurrent_depth_transformer_b200/csrc/rdt_internal.cuh",
+                "recurrent_depth_transformer_b200/csrc/rdt_api.cu"),
+}
+# (workload, kernel) -> (bytes per launch, source fingerprint)
+MEASURED_TRAFFIC = {}
 
 
 def code_text(src: str) -> str:
@@ -88,11 +100,12 @@ def source_fingerprint(files):
     return h.hexdigest()[:16]
 
 
-def measured_traffic(kernel):
-    """The captured traffic of `kernel`, or None once its sources differ from the captured."""
-    if kernel not in MEASURED_TRAFFIC or kernel not in KERNEL_SOURCES:
+def measured_traffic(workload, kernel):
+    """The captured traffic of `kernel` on `workload`, or None once its sources differ."""
+    key = (workload, kernel)
+    if key not in MEASURED_TRAFFIC or kernel not in KERNEL_SOURCES:
         return None
-    value, fp = MEASURED_TRAFFIC[kernel]
+    value, fp = MEASURED_TRAFFIC[key]
     try:
         return value if source_fingerprint(KERNEL_SOURCES[kernel]) == fp else None
     except (OSError, ValueError):          # missing or undecodable source: no claim
@@ -101,44 +114,67 @@ def measured_traffic(kernel):
 
 # ----------------------------------------------------------------------------- algorithmic work
 
-def kernel_work(wl, T):
-    """Algorithmic FLOPs and DRAM bytes per launch of each kernel class (counts of what the
-    block must compute and move, not of what a kernel happens to do: causal attention
-    counts the S(S+1)/2 unmasked pairs, the expert GEMMs the N*k routed rows)."""
+def kernel_work(wl):
+    """Algorithmic FLOPs and DRAM bytes per launch of each kernel class: counts of what the
+    block must compute and move, not of what a kernel happens to do (causal attention counts
+    the S(S+1)/2 unmasked pairs, the expert GEMMs the N*k routed rows plus shared rows, the
+    depth-wise LoRA its rank-r products; weights are read once, activations once in and
+    once out)."""
     N, d = wl.batch * wl.seq, wl.dim
-    hq, hkv, dh = wl.n_heads, wl.n_kv_heads, wl.head_dim
     E, k, hid, S = wl.n_experts, wl.top_k, wl.expert_hidden, wl.n_shared
     rows = N * (k + S)
-    nqkv = (hq + 2 * hkv) * dh
-    b2 = 2
-    w = {}
-    w["gemm_qkv"] = dict(flops=2.0 * N * d * nqkv, bytes=b2 * (N * d + nqkv * d + N * nqkv), bound="tensor")
+    b2 = 2 if wl.dtype == "bf16" else 4
     pairs = wl.batch * wl.seq * (wl.seq + 1) / 2
-    w["attention"] = dict(flops=4.0 * hq * dh * pairs, bytes=b2 * N * (nqkv + hq * dh), bound="tensor")
-    # the O projection completes y = x + a and h_next = A h + B e + a with two fp32 reductions
-    w["gemm_o"] = dict(flops=2.0 * N * hq * dh * d, bytes=b2 * (N * hq * dh + d * hq * dh) + 4 * 2 * N * d,
-                       bound="tensor")
+    w = {}
+    if wl.attn == "gqa":
+        hq, hkv, dh = wl.n_heads, wl.n_kv_heads, wl.head_dim
+        nq, nqkv = hq * dh, (hq + 2 * hkv) * dh
+        r = wl.lora_rank if wl.n_lora else 0
+        w["gemm_qkv"] = dict(flops=2.0 * N * d * nqkv + 2.0 * N * r * (d + nq),
+                             bytes=b2 * (N * d + nqkv * d + N * nqkv), bound="tensor")
+        w["attention"] = dict(flops=4.0 * hq * dh * pairs, bytes=b2 * N * (nqkv + nq), bound="tensor")
+        ow = nq
+        w["gemm_o"] = dict(flops=2.0 * N * nq * d + 2.0 * N * r * (nq + d),
+                           bytes=b2 * (N * nq + d * nq) + 4 * 2 * N * d, bound="tensor")
+    else:
+        H, ql, kvl, rp = wl.n_heads, wl.q_lora_rank, wl.kv_lora_rank, wl.qk_rope_dim
+        lat = ql + kvl + rp
+        w["gemm_latent"] = dict(flops=2.0 * N * d * lat, bytes=b2 * (N * d + lat * d) + 4 * N * lat, bound="tensor")
+        w["gemm_q_absorbed"] = dict(flops=2.0 * N * ql * H * (kvl + rp),
+                                    bytes=b2 * (N * ql + ql * H * (kvl + rp) + N * H * (kvl + rp)), bound="tensor")
+        # absorbed attention: every head over the shared (kvl + rope)-wide key, kvl-wide value
+        w["attention"] = dict(flops=2.0 * H * (kvl + rp + kvl) * pairs,
+                              bytes=b2 * N * (H * (kvl + rp) + kvl + rp + H * kvl), bound="tensor")
+        ow = H * kvl
+        w["gemm_o"] = dict(flops=2.0 * N * ow * d, bytes=b2 * (N * ow + d * ow) + 4 * 2 * N * d, bound="tensor")
+        w["mla_latent_norm"] = dict(flops=0.0, bytes=N * (4 * lat + b2 * (ql + kvl + rp)), bound="hbm")
     w["gemm_up"] = dict(flops=2.0 * rows * d * 2 * hid, bytes=b2 * (rows * d + (E + S) * 2 * hid * d + rows * hid),
                         bound="tensor")
     w["gemm_down"] = dict(flops=2.0 * rows * hid * d, bytes=b2 * (rows * hid + (E + S) * d * hid) + 4 * N * d * 2,
                           bound="tensor")
     # RMSNorm1 reads h, e, B e and writes xn, y = x and h_next = A h + B e
     w["norm1"] = dict(flops=0.0, bytes=N * d * (4 + b2 + 4 + b2 + 4 + 4), bound="hbm")
-    # RMSNorm2 fused with the fp32 router and the dispatch (W_r staged in shared memory): y in;
-    # per (token, slot) the routing (index, weight, row token, row weight) and the yn copy in
-    # the expert's rows; yn itself only when shared experts read it
+    # the router: y in, W_r once, per (token, slot) the routing words and the yn copy in the
+    # expert's rows; yn itself where shared experts read it
     w["router_topk"] = dict(flops=2.0 * N * d * E,
                             bytes=N * d * 4 + (N * d * b2 if S else 0) + E * d * b2 + N * k * (d * b2 + 16),
                             bound="hbm")
-    w["moe_dispatch"] = dict(flops=0.0, bytes=N * k * (d * b2 * 2 + 16), bound="hbm")
+    w["norm2"] = dict(flops=0.0, bytes=N * d * (4 + b2), bound="hbm")
+    w["moe_dispatch"] = dict(flops=0.0, bytes=N * k * (d * b2 * 2 + 4), bound="hbm")
+    w["moe_combine"] = dict(flops=0.0, bytes=N * d * 4 * (2 + k + S), bound="hbm")
     w["hoist"] = dict(flops=0.0, bytes=N * d * (b2 + b2 + 4 + 4), bound="hbm")
     w["check_finite"] = dict(flops=0.0, bytes=N * d * 4, bound="hbm")
+    w["act_halting"] = dict(flops=0.0, bytes=N * d * 12, bound="hbm")
     return w
 
 
+PATH_KERNELS = ("gemm_qkv", "gemm_latent", "gemm_q_absorbed", "attention", "gemm_o", "gemm_up", "gemm_down")
+
+
 def step_flops(wl, T):
-    w = kernel_work(wl, T)
-    per_loop = sum(w[k]["flops"] for k in ("gemm_qkv", "attention", "gemm_o", "gemm_up", "gemm_down"))
+    """Algorithmic FLOPs of T loops: the dense contractions plus the router logits."""
+    w = kernel_work(wl)
+    per_loop = sum(w[k]["flops"] for k in PATH_KERNELS if k in w)
     per_loop += 2.0 * wl.batch * wl.seq * wl.dim * wl.n_experts      # router logits
     return per_loop * T
 
@@ -153,6 +189,25 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def roofline_of(name, n_launches, total_ms, work, peaks, peak_src, workload):
+    """The roofline object of one kernel class from its event-timed launches."""
+    wk = work[name]
+    avg_s = total_ms / n_launches / 1e3
+    if wk["bound"] == "tensor":
+        achieved = wk["flops"] / avg_s / 1e12
+        peak = peaks["bf16_tflops"]
+        return {"kernel": name, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": measured_traffic(workload, name),
+                "peak_source": f"{peak_src} bf16 dense (burst)", "avg_launch_us": avg_s * 1e6,
+                "algorithmic_per_launch": wk["flops"]}
+    achieved = wk["bytes"] / avg_s / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"kernel": name, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "traffic": measured_traffic(workload, name),
+            "peak_source": f"{peak_src} HBM copy", "avg_launch_us": avg_s * 1e6,
+            "algorithmic_per_launch": wk["bytes"]}
+
+
 # ----------------------------------------------------------------------------- clocks
 
 CLOCK_FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -162,16 +217,17 @@ REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_powe
 
 
 class ClockSampler:
-    def __init__(self):
+    def __init__(self, gpu_index=0):
         self.proc = None
         self.path = None
+        self.gpu = gpu_index
 
     def start(self):
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}",
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={CLOCK_FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
@@ -228,7 +284,7 @@ def parse_clocks(text, window=None):
             any(window[0] <= (r[0] or 0) <= window[1] for r in rows)}
 
 
-# ----------------------------------------------------------------------------- distributed plumbing
+# ----------------------------------------------------------------------------- ranks
 
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
@@ -253,6 +309,45 @@ def aggregate(per_rank_ms, tokens_per_step, loops, world):
     return world * tokens_per_step * loops / (ms / 1e3), ms
 
 
+def replica_plan(wl, rank, world):
+    """Weak scaling by replicas: the sequences of different ranks never interact, so every
+    rank runs the whole configuration on inputs of its own (the configuration's seed plus the
+    rank: independent sequences, same weights). Returns the rank's input seed and the tokens
+    it processes per step."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    return wl.seed + 1000 * rank, wl.batch * wl.seq
+
+
+def launch_ranks(argv, n):
+    """Re-run this script under torch.distributed.run with one process per GPU."""
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + list(argv)
+    return subprocess.call(cmd)
+
+
+def init_ranks(device=None, backend="nccl", timeout_s=120):
+    """Join the process group of a multi-rank run (nothing for one rank)."""
+    import datetime
+    import torch.distributed as dist
+    rank, local, world = dist_env()
+    if world > 1 and not dist.is_initialized():
+        kw = {"device_id": device} if device is not None else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+    return rank, local, world
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.barrier()
+
+
 # ----------------------------------------------------------------------------- CPU baseline
 
 def cpu_cores():
@@ -266,23 +361,40 @@ def cpu_cores():
     return len(os.sched_getaffinity(0))
 
 
+def oracle_sample_plan(wl, budget_s=CPU_SECONDS):
+    """A bounded sample of the workload for the fp64 oracle: one loop over the whole batch
+    when that fits the budget (every position at its full context, so the per-token cost is
+    the workload's), else one loop over a prefix of every sequence. The estimate scales a
+    loop's FLOPs by an fp64 rate of 50 GFLOP/s."""
+    per_loop = step_flops(wl, 1)
+    if per_loop / 50e9 <= budget_s:
+        return wl.seq
+    seq = wl.seq
+    while seq > 128 and step_flops(wl.replace(seq=seq), 1) / 50e9 > budget_s:
+        seq //= 2
+    return seq
+
+
 def oracle_sample(wl, inputs, seconds=10.0):
-    """Time the fp64 oracle on one sequence (512 tokens) through all loops, repeated until
-    `seconds` of CPU work; returns (tokens*loops/s, description)."""
+    """Time the fp64 oracle on the sample of oracle_sample_plan, repeated until `seconds`
+    of work; returns (tokens*loops/s, description)."""
     import oracle as O
+    seq = oracle_sample_plan(wl)
     sub = dict(inputs)
-    sub["e"] = inputs["e"][:1]
-    sub["h0"] = sub["e"]
-    w1 = wl.replace(batch=1)
+    sub["e"] = inputs["e"][:, :seq]
+    sub["h0"] = sub["e"] if inputs["h0"] is inputs["e"] else inputs["h0"][:, :seq]
+    w1 = wl.replace(seq=seq)
     t0 = time.perf_counter()
     runs = 0
     while True:
-        O.loop_forward(sub["h0"], sub["e"], LOOPS, sub, w1)
+        O.loop_forward(sub["h0"], sub["e"], 1, sub, w1)
         runs += 1
         el = time.perf_counter() - t0
         if el >= seconds:
             break
-    return runs * wl.seq * LOOPS / el, f"{runs} x (1 of {wl.batch} sequences, {wl.seq} tokens, {LOOPS} loops), {el:.1f} s"
+    what = "the whole batch" if seq == wl.seq else f"the first {seq} of {wl.seq} positions of every sequence"
+    return (runs * wl.batch * seq / el,
+            f"{runs} x (1 loop over {what}: {wl.batch * seq} tokens), {el:.1f} s")
 
 
 # ----------------------------------------------------------------------------- arms
@@ -293,27 +405,30 @@ def run_reference(args):
         return 0
     from workloads import by_name, generate
     import oracle as O
-    wl = by_name(WORKLOAD)
+    wl = by_name(args.workload)
     inputs = generate(wl)
+    # per step: one loop of a prefix short enough that the whole run takes minutes
+    seq = oracle_sample_plan(wl, budget_s=4.0)
     sub = dict(inputs)
-    sub["e"] = inputs["e"][:1]
+    sub["e"] = inputs["e"][:, :seq]
     sub["h0"] = sub["e"]
-    w1 = wl.replace(batch=1)
+    w1 = wl.replace(seq=seq)
     for _ in range(args.warmup):
-        O.loop_forward(sub["h0"], sub["e"], 1, sub, w1)
+        O.loop_forward(sub["h0"], sub["e"], 1, sub, w1.replace(seq=min(seq, 64)))
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        O.loop_forward(sub["h0"], sub["e"], LOOPS, sub, w1)
+        O.loop_forward(sub["h0"], sub["e"], 1, sub, w1)
         times.append(time.perf_counter() - t0)
-    ms = 1e3 * statistics.mean(times)
-    value = wl.seq * LOOPS / (ms / 1e3)
-    sample = f"1 of {wl.batch} sequences ({wl.seq} tokens) through all {LOOPS} loops per step"
+    ms = 1e3 * statistics.median(times)
+    value = wl.batch * seq / (ms / 1e3)
+    what = "the whole batch" if seq == wl.seq else f"the first {seq} of {wl.seq} positions"
+    sample = f"1 of {args.loops} loops over {what} per step (fp64 NumPy oracle)"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "batch": wl.batch, "seq": wl.seq, "dim": wl.dim, "loops": LOOPS,
+        "config": {"workload": args.workload, "batch": wl.batch, "seq": wl.seq, "dim": wl.dim, "loops": args.loops,
                    "parallelism": "host cores (fp64 NumPy oracle)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -322,31 +437,24 @@ def run_reference(args):
     return 0
 
 
-def run_gpu(args):
+def bench_one(args, wl_name, T, dev, rank, world, with_cpu):
+    """Time one workload; returns the JSON line (rank 0) or None."""
     import numpy as np
     import torch
-    import torch.distributed as dist
 
     import recurrent_depth_transformer_b200 as R
     from workloads import by_name, generate
 
-    rank, local, world = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
-
-    wl = by_name(WORKLOAD)
-    inputs = generate(wl)
-    weights = R.device_weights(inputs, True, device=dev)
-    h = R.RDT(R.make_config(wl, max_loops=LOOPS), weights)
+    wl = by_name(wl_name)
+    seed, tokens = replica_plan(wl, rank, world)
+    inputs = generate(wl) if seed == wl.seed else generate(wl.replace(seed=seed))
+    weights = R.device_weights(generate(wl) if seed != wl.seed else inputs, wl.dtype == "bf16", device=dev)
+    h = R.RDT(R.make_config(wl, max_loops=T), weights)
     del weights
-    e = torch.from_numpy(inputs["e"]).to(torch.bfloat16).to(dev)
+    e = torch.from_numpy(inputs["e"]).to(torch.bfloat16 if wl.dtype == "bf16" else torch.float32).to(dev)
     out = torch.empty(e.shape, dtype=torch.float32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    N = wl.batch * wl.seq
 
     nl = None
     if args.act:
@@ -356,10 +464,10 @@ def run_gpu(args):
         nl = torch.empty((wl.batch, wl.seq), dtype=torch.int32, device=dev)
 
         def step():
-            h.loop_forward_act(e, e, LOOPS, out=out, n_loops=nl)
+            h.loop_forward_act(e, e, T, out=out, n_loops=nl)
     else:
         def step():
-            h.loop_forward(e, e, LOOPS, out=out)
+            h.loop_forward(e, e, T, out=out)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -367,12 +475,11 @@ def run_gpu(args):
     torch.cuda.synchronize()
 
     # ---- timed region (device time, CUDA events on the launch stream)
-    sampler = ClockSampler() if rank == 0 else None
+    sampler = ClockSampler(dev.index) if rank == 0 else None
     if sampler:
         sampler.start()
         time.sleep(0.3)
-    if world > 1:
-        dist.barrier()
+    barrier()
     torch.cuda.synchronize()
     launches0 = h.launch_count()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -384,160 +491,154 @@ def run_gpu(args):
         b.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
-    if world > 1:
-        dist.barrier()
-    launches = h.launch_count() - launches0
+    barrier()
+    launches = (h.launch_count() - launches0) / args.steps
     clocks = sampler.stop((t_wall0, t_wall1)) if sampler else None
-    ms_rank = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    ms_rank = statistics.median(step_ms)
     ms_all = reduce_max(ms_rank, dev)
-    value, ms = aggregate([ms_all], N, LOOPS, world)
+    value, ms = aggregate([ms_all], tokens, T, world)
 
-    # ---- per-kernel event timing over the same number of steps
-    h.profile(True)
+    # ---- per-kernel event timing inside graph replay (events are nodes of the loop's graph)
+    h.profile(2)
+    for _ in range(2):                    # eager call, then capture with the event nodes
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    h.profile(2)                          # restart the statistics, keep the graph
     for _ in range(args.steps):
         flush.zero_()
         step()
+        h.profile_read()                  # each replay records the graph's events anew
     stats, _ = h.profile_read()
-    h.profile(False)
+    h.profile(0)
 
-    # ---- end to end through the host-buffer entry point (pinned memory, copies inside)
-    if args.act:
-        return act_line(args, h, wl, nl, value, ms, world, rank, stats, launches, clocks)
-    e_host = e.cpu().pin_memory()
-    out_host = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-    for _ in range(3):                       # eager, graph capture, first replay
-        h.loop_forward_host(e_host, e_host, LOOPS, out_host)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e2e_ms = []
-    for _ in range(args.steps):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        h.loop_forward_host(e_host, e_host, LOOPS, out_host)
-        b.record(stream)
-        b.synchronize()
-        e2e_ms.append(a.elapsed_time(b))
-    e2e_rank = statistics.mean(e2e_ms)
-    e2e_all = reduce_max(e2e_rank, dev)
-    e2e_value, _ = aggregate([e2e_all], N, LOOPS, world)
-    ok = bool(np.isfinite(out_host.numpy()).all())
     diag = h.diagnostics()
+    e2e = None
+    if not args.act:
+        # ---- end to end through the host-buffer entry point (pinned memory, copies inside)
+        e_host = e.cpu().pin_memory()
+        out_host = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        for _ in range(3):                   # eager, graph capture, first replay
+            h.loop_forward_host(e_host, e_host, T, out_host)
+        barrier()
+        torch.cuda.synchronize()
+        e2e_ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            h.loop_forward_host(e_host, e_host, T, out_host)
+            b.record(stream)
+            b.synchronize()
+            e2e_ms.append(a.elapsed_time(b))
+        e2e_all = reduce_max(statistics.median(e2e_ms), dev)
+        e2e_value, _ = aggregate([e2e_all], tokens, T, world)
+        finite = bool(np.isfinite(out_host.numpy()).all())
+        e2e = {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(e_host.numel() * e_host.element_size()),
+               "d2h_bytes_per_step": int(out_host.numel() * 4), "ms_per_step": e2e_all}
+    else:
+        finite = bool(torch.isfinite(out).all().item())
 
     peaks, peak_src = load_peaks()
-    work = kernel_work(wl, LOOPS)
-    top = max(stats.items(), key=lambda kv: kv[1][1]) if stats else None
-    roof = None
-    kernels = {}
-    for name, (n, tot) in stats.items():
-        kernels[name] = {"launches_per_step": n / args.steps, "ms_per_step": tot / args.steps,
-                         "share": tot / max(sum(v[1] for v in stats.values()), 1e-12)}
-    if top is not None and top[0] in work:
-        name, (n, tot) = top
-        wk = work[name]
-        avg_s = tot / n / 1e3
-        if wk["bound"] == "tensor":
-            achieved = wk["flops"] / avg_s / 1e12
-            peak = peaks["bf16_tflops"]
-            roof = {"kernel": name, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": measured_traffic(name),
-                    "peak_source": f"{peak_src} bf16 dense (burst)", "avg_launch_us": avg_s * 1e6,
-                    "algorithmic_per_launch": wk["flops"]}
-        else:
-            achieved = wk["bytes"] / avg_s / 1e9
-            peak = peaks["hbm_gbs"]
-            roof = {"kernel": name, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                    "frac": achieved / peak, "traffic": measured_traffic(name), "peak_source": f"{peak_src} HBM copy",
-                    "avg_launch_us": avg_s * 1e6, "algorithmic_per_launch": wk["bytes"]}
-    flops = step_flops(wl, LOOPS)
-    path_roof = {"step_flops": flops, "achieved_tflops": flops / (ms / 1e3) / 1e12 / world,
-                 "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / world / peaks["bf16_tflops"]}
+    work = kernel_work(wl)
+    tot = max(sum(v[1] for v in stats.values()), 1e-12)
+    kernels = {name: {"launches_per_step": n / args.steps, "ms_per_step": t / args.steps, "share": t / tot}
+               for name, (n, t) in stats.items()}
+    ranked = sorted(((t, name, n) for name, (n, t) in stats.items() if name in work), reverse=True)
+    roof = roofline_of(ranked[0][1], ranked[0][2], ranked[0][0], work, peaks, peak_src, wl_name) if ranked else None
+    flops = step_flops(wl, T)
+    # per GPU: every rank runs the whole workload in the step time
+    path_roof = {"step_flops": flops, "achieved_tflops": flops / (ms / 1e3) / 1e12,
+                 "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"]}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if with_cpu and rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, sample = oracle_sample(wl, inputs, seconds=args.cpu_seconds)
         cpu = {"value": v, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": sample}
 
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "batch": wl.batch, "seq": wl.seq, "dim": wl.dim, "loops": LOOPS,
-                       "tokens_per_step": N, "parallelism": f"replicas x{world} (no data-path collective)",
-                       "l2": "flushed before every timed step (256 MiB write)"},
-            "roofline": roof,
-            "path_roofline": path_roof,
-            "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(e_host.numel() * 2),
-                    "d2h_bytes_per_step": int(out_host.numel() * 4), "ms_per_step": e2e_all},
-            "gpu_launches": int(launches),
-            "clocks": clocks,
-            "kernels": kernels,
-            "finite": ok and diag["nonfinite"] == 0 and diag["timeout"] == 0,
-        }
-        print(json.dumps(line), flush=True)
     h.close()
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    return 0
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": wl_name, "batch": wl.batch, "seq": wl.seq, "dim": wl.dim, "loops": T,
+                   "tokens_per_step": tokens, "parallelism": f"replicas x{world} (no data-path collective)",
+                   "l2": "flushed before every timed step (256 MiB write)", "step_time": "median of the timed steps"},
+        "roofline": roof,
+        "path_roofline": path_roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(round(launches)),
+        "clocks": clocks,
+        "kernels": kernels,
+        "kernel_timing": "CUDA events recorded by nodes of the replayed loop graph",
+        "finite": finite and diag["nonfinite"] == 0 and diag["timeout"] == 0,
+    }
+    if args.act:
+        line["impl"] = "ours+act"
+        line["config"]["workload"] = wl_name + "+act"
+        line["config"]["act"] = {"threshold": 0.99, "head": "w ~ N(0, 0.25/dim), b = -1"}
+        line["act"] = act_summary(nl.cpu().numpy(), T)
+    return line
 
 
-def act_line(args, h, wl, nl, value, ms, world, rank, stats, launches, clocks):
-    """The line of the ACT leg: device-timed throughput and the halting histogram."""
+def act_summary(n_loops, T):
+    """Halting histogram of an ACT run: how many positions ran 1 .. T loops, the mean, and
+    the fraction of the T loops asked for that positions ran."""
     import numpy as np
+    loops = np.asarray(n_loops).ravel()
+    return {"mean_loops": float(loops.mean()), "hist": np.bincount(loops, minlength=T + 1)[1:].tolist(),
+            "loops_run_fraction": float(loops.mean() / T)}
+
+
+ALL_RUNS = (("tiny-f32-b1s64-d128-gqa4x2-e4k2", 4), ("gqa-bf16-b4s512-d1024-h16x4-e16k2", 8),
+            ("mla-bf16-b4s512-d1024-h16-lat128-e16k2", 3), ("mla-bf16-b4s512-d1024-h16-lat128-e16k2", 8),
+            ("widemoe-bf16-b2s2048-d2048-h32x8-e64k8s1", 1), ("widemoe-bf16-b2s2048-d2048-h32x8-e64k8s1", 4),
+            ("widemoe-bf16-b2s2048-d2048-h32x8-e64k8s1", 8), ("widemoe-bf16-b2s2048-d2048-h32x8-e64k8s1", 16),
+            ("long-bf16-b1s8192-d2048-h32x8-e64k8-lora16", 16))
+
+
+def run_gpu(args):
+    import torch
     import torch.distributed as dist
-    loops = nl.cpu().numpy().ravel()
-    diag = h.diagnostics()
-    if rank == 0:
-        tot = max(sum(v[1] for v in stats.values()), 1e-12)
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "ours+act",
-            "config": {"workload": WORKLOAD + "+act", "batch": wl.batch, "seq": wl.seq, "dim": wl.dim,
-                       "loops": LOOPS, "tokens_per_step": wl.batch * wl.seq,
-                       "act": {"threshold": 0.99, "head": "w ~ N(0, 0.25/dim), b = -1"},
-                       "l2": "flushed before every timed step (256 MiB write)"},
-            "act": {"mean_loops": float(loops.mean()),
-                    "hist": np.bincount(loops, minlength=LOOPS + 1)[1:].tolist(),
-                    "loops_run_fraction": float(loops.mean() / LOOPS)},
-            "e2e": None,
-            "gpu_launches": int(launches),
-            "clocks": clocks,
-            "kernels": {k: {"launches_per_step": n / args.steps, "ms_per_step": t / args.steps,
-                            "share": t / tot} for k, (n, t) in stats.items()},
-            "finite": diag["nonfinite"] == 0 and diag["timeout"] == 0,
-        }
-        print(json.dumps(line), flush=True)
-    h.close()
+
+    rank, local, world = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_ranks(dev)
+    runs = ALL_RUNS if args.all else ((args.workload, args.loops),)
+    for name, T in runs:
+        line = bench_one(args, name, T, dev, rank, world, with_cpu=not args.all or name == args.workload)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    barrier()
     if world > 1:
-        dist.barrier()
         dist.destroy_process_group()
     return 0
 
 
 def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--act", action="store_true", help="time the ACT halting loop instead")
-    ap.add_argument("--workload", default=None, help="workload name (default: the headline one)")
-    ap.add_argument("--loops", type=int, default=None, help="loops T per step")
+    ap.add_argument("--workload", default=WORKLOAD, help="workload name (default: the headline one)")
+    ap.add_argument("--loops", type=int, default=LOOPS, help="loops T per step")
+    ap.add_argument("--all", action="store_true", help="one line per configuration and loop count")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    global WORKLOAD, LOOPS
-    if args.workload:
-        WORKLOAD = args.workload
-    if args.loops:
-        LOOPS = args.loops
+    _, _, world = dist_env()
+    if args.gpus > 1 and world == 1 and "LOCAL_RANK" not in os.environ:
+        return launch_ranks(argv, args.gpus)
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)

@@ -297,8 +297,14 @@ typedef struct {
     double total_ms;        /* summed event time of those launches                      */
 } rdt_kernel_stat;
 
-/* enable = 1 clears the statistics and starts timing; 0 stops it. Timing adds two
- * event records per launch on the launch stream. */
+/* enable = 1 times eager launches (the loop is not replayed from its CUDA graph while on);
+ * enable = 2 times inside graph replay: the events become event-record nodes of the loop's
+ * captured graph, so the timing describes the replayed sequence (the records sit between the
+ * kernels, so each launch waits for its predecessor to finish); 0 stops timing. Switching
+ * mode clears the statistics and drops a captured graph; enabling the current mode again
+ * only clears the statistics. Timing adds two event records per launch on the launch
+ * stream. In mode 2 a replay records the graph's events anew: rdt_profile_read counts the
+ * last replay before it, so read after every replayed call. */
 rdt_status rdt_profile(rdt_handle* h, int enable);
 
 /* Synchronises the handle's last stream and returns up to max_entries statistics

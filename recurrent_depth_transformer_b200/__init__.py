@@ -280,8 +280,9 @@ class RDT:
         return {"rho_A": d.rho_A, "nonfinite": d.nonfinite, "timeout": d.timeout,
                 "last_routed_rows": d.last_routed_rows, "expert_counts": list(d.expert_counts[:E])}
 
-    def profile(self, enable: bool = True):
-        _check(self._lib.rdt_profile(self._h, 1 if enable else 0))
+    def profile(self, mode=True):
+        """Per-kernel event timing: True or 1 eager launches, 2 inside graph replay, 0 off."""
+        _check(self._lib.rdt_profile(self._h, int(mode)))
 
     def profile_read(self):
         """(per-kernel {name: (launches, total_ms)}, kernels launched since create)."""

@@ -1,26 +1,38 @@
-// Causal attention forward on the sm_100a tensor cores (tcgen05), one CTA per
-// (128 queries, query head, sequence), two CTAs per SM:
+// Causal attention forward on the sm_100a tensor cores (tcgen05):
 //
 //   o = softmax(q k^T * scale, key > query masked) v
 //
-// For each block j of 128 keys:  S_j = Q K_j^T  (tcgen05.mma, M = 128 queries, N = 128 keys,
-// fp32 in TMEM)  ->  eight softmax warps, two per 32 query rows (one per half of the key
-// block), one query row per thread: row maximum (the two halves exchange theirs), then
-// P_j = 2^(S_j * scale * log2 e - m_ref) in bf16, written to shared memory in the
-// 128-byte-swizzled K-major layout, and the row sum l  ->  O += P_j V_j  (tcgen05.mma into a
-// TMEM accumulator, N = dv; V read as an MN-major operand straight from its [key][dv] layout).
-// m_ref is raised only when a row maximum exceeds it by more than 2^8; O (in TMEM) and l are
-// then rescaled once. The division by l happens when o is written.
+// A CTA owns QT tiles of 128 consecutive query rows (QT = 2 for long sequences, 1 for short
+// ones) of one query head and walks the key blocks of 128 keys that the causal mask leaves
+// open. Per tile t and key block j:
+//
+//   S_t(j) = Q_t K_j^T            tcgen05.mma, M = 128 queries, N = 128 keys, fp32 in TMEM
+//   P_t(j) = 2^(S * scale * log2 e - m_ref)   one thread per query row (a warpgroup per
+//            tile), written back into TMEM over S_t(j) as bf16 pairs
+//   O_t   += P_t(j) V_j           tcgen05.mma with A = P read from TMEM, B = V from shared
+//                                 memory (MN-major), fp32 accumulator in TMEM
+//
+// The scores rotate through NSBUF TMEM buffers in the order S_0(0), S_1(0), S_0(1), ...:
+// score n = QT j + t lives in buffer n mod NSBUF. The MMA thread issues PV_t(j) and then,
+// into the buffer that PV_t(j) has just read (tcgen05 MMAs of one thread execute in issue
+// order), the score NSBUF places later. With NSBUF = QT (every shape whose TMEM holds no
+// more) a tile's next S waits for its own PV; with three buffers for two tiles (head width
+// 64: 3 x 128 + 2 x 64 = 512 columns) each tile's next S is computed while its softmax still
+// runs, so the softmax warpgroups never wait for a round trip through the tensor cores.
+// O_t is rescaled (only when a row maximum grows by more than 2^8 over the reference m_ref,
+// so that P <= 2^8) once PV_t(j - 1) is complete; the division by the row sum l happens when
+// o is written.
 //
 // Grouped-query heads read KV head floor(h * Hkv / Hq) ("Introducao ao OpenMythos" Passo 5).
 // Absorbed MLA attends over the shared latent key [c_kv ; k_rope] (160 wide) with the value
 // c_kv = the key's first 128 columns, so its V operand is the K tile itself.
 //
-// Roles: warp 0 issues TMA loads (Q once; K one stage and V two, or two stages of the shared
-// latent key for MLA); warp 1 owns TMEM
-// and issues the MMAs (S_{j+1} before P_j V_j); warps 2-9 do the softmax (two warps per 32
-// query rows, one per half of the key block) and write o.
-// Every wait is bounded.
+// Roles: warpgroup 0 is control: warp 0 issues TMA loads (Q once; K and V in rings of
+// stages), warp 1 owns TMEM and issues the MMAs, warps 2 and 3 only take part in set-up.
+// Warpgroups 1 .. QT are the softmax warpgroups (warpgroup 1 + t: tile t, one query row per
+// thread, its 128 scores held in registers) and write o. Registers are moved from the
+// control warpgroup to the softmax warpgroups with setmaxnreg (the split adds up to the
+// block's launch allocation). Every wait is bounded.
 #include <algorithm>
 
 #include "rdt_internal.cuh"
@@ -28,7 +40,7 @@
 namespace rdt {
 namespace {
 
-constexpr int kBQ = 128;     // queries per CTA
+constexpr int kBQ = 128;     // queries per tile
 constexpr int kBK = 128;     // keys per block
 constexpr int kAtom = 16384; // one 128-row x 128-byte swizzled region
 
@@ -38,10 +50,6 @@ __device__ __forceinline__ float exp2_ftz(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // K-major (a_major = b_major = 0) or K-major A with MN-major B (b_major = 1).
@@ -62,102 +70,128 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr, uint32_t 
     return d;
 }
 
-template <int DQK, int DV, bool SHARE_KV>
+// D[tmem] (+)= A[tmem] * B[smem]: A (M x K, bf16 pairs per 32-bit TMEM cell, lower K in the
+// low half) read from TMEM, B from a shared-memory descriptor; kind::f16, fp32 accumulate.
+__device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&p);
+}
+
+template <int DQK, int DV, bool SHARE_KV, int QT>
 struct AttnCfg {
     static constexpr int QA = (DQK + 63) / 64;     // 64-wide atoms of the query/key width
     static constexpr int VA = DV / 64;             // 64-wide atoms of the value width
-    static constexpr int Q_BYTES = QA * kAtom;
+    static constexpr int Q_BYTES = QA * kAtom;     // one query tile
     static constexpr int K_BYTES = QA * kAtom;     // one stage of K (128 keys)
-    // Separate V: one K stage (K_{j+1} loads once S_j has read K_j, during softmax j) and two
-    // V stages (V_{j+1} loads while P_j V_j runs). Shared latent V (= K): two K stages.
-    static constexpr int KSTAGES = SHARE_KV ? 2 : 1;
-    static constexpr int VSTAGES = SHARE_KV ? 0 : 2;
+    static constexpr int KSTAGES = (QT == 2 && !SHARE_KV) ? 3 : 2;
+    static constexpr int VSTAGES = SHARE_KV ? 0 : KSTAGES;
     static constexpr int V_BYTES = SHARE_KV ? 0 : VA * kAtom;
-    static constexpr int P_BYTES = 2 * kAtom;      // 128 x 128 bf16 probabilities
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_K = OFF_Q + QT * Q_BYTES;
     static constexpr int OFF_V = OFF_K + KSTAGES * K_BYTES;
-    static constexpr int OFF_P = OFF_V + VSTAGES * V_BYTES;
-    static constexpr int OFF_BAR = OFF_P + P_BYTES;
-    static constexpr int OFF_X = OFF_BAR + 256;    // softmax exchange: row maxima [2][2][128], sums [2][128]
-    static constexpr int SMEM = OFF_X + 3 * 2 * 128 * 4 + 1024;
-    static constexpr int S_COL = 0;                 // S: columns [0, 128)
-    static constexpr int O_COL = 128;               // O: columns [128, 128 + DV)
-    static constexpr int TMEM_COLS = 128 + DV <= 256 ? 256 : 512;
+    static constexpr int OFF_BAR = OFF_V + VSTAGES * V_BYTES;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;   // + alignment slack
+    // TMEM: score buffers at columns [128 b, 128 b + 128) (P over the first 64 of its score),
+    // then O_t for every tile
+    static constexpr int NSBUF = (QT == 2 && DV == 64) ? 3 : QT;
+    static constexpr int S_COL = 0;
+    static constexpr int O_COL = 128 * NSBUF;
+    static constexpr int COLS_USED = 128 * NSBUF + QT * DV;
+    static constexpr int TMEM_COLS = COLS_USED <= 256 ? 256 : 512;
+    static constexpr int THREADS = 128 + 128 * QT;
+    static constexpr int BLOCKS_PER_SM = QT == 1 ? 2 : 1;
+    // registers per thread at launch (65536 per SM over the resident threads, in units of 8)
+    static constexpr int REGS_LAUNCH = (65536 / (THREADS * BLOCKS_PER_SM)) / 8 * 8;
+    static constexpr int REGS_CONTROL = QT == 1 ? 40 : 64;
+    // the softmax warpgroups take what the control warpgroup gives up
+    static constexpr int REGS_SOFTMAX = ((REGS_LAUNCH * THREADS - 128 * REGS_CONTROL) / (128 * QT)) / 8 * 8;
+    static_assert(128 * REGS_CONTROL + 128 * QT * REGS_SOFTMAX <= REGS_LAUNCH * THREADS, "register split");
+    static_assert(REGS_SOFTMAX <= 256, "setmaxnreg limit");
+    static_assert(COLS_USED <= 512, "TMEM budget");
+    static_assert(NSBUF >= QT, "one score buffer per tile at least");
+    static_assert(SMEM <= 227 * 1024, "shared-memory budget");
 };
 
 struct AttnTcArgs {
     int seq, hq, hkv, q_hstride, k_hstride, v_hstride, ldo, dv_out;
-    int nqb, batch, sms;   // query blocks per sequence; sequences; SMs (first-round CTA slots)
+    int nqb, npairs, batch, sms;   // query blocks and CTA work items (of QT blocks) per sequence
     float scale_log2;
     void* o;
     int* flags;
 };
 
-// O is accumulated in TMEM by the P.V MMAs. P_j is taken relative to a reference maximum
-// m_ref that is raised only when a row's maximum exceeds it by more than 8 (in log2 units),
-// so P <= 2^8; then O and l are rescaled once by 2^(m_ref_old - m_ref_new).
+// O rows are rescaled only when the running maximum exceeds the reference by more than this
+// (log2 units), so P <= 2^8 and the bf16 probabilities keep their relative precision.
 constexpr float kRescaleThreshold = 8.0f;
 
-constexpr int kAttnThreads = 320;   // TMA warp, MMA warp, 8 softmax warps
-
-template <int DQK, int DV, bool SHARE_KV>
-__global__ void __launch_bounds__(kAttnThreads, 2)
+template <int DQK, int DV, bool SHARE_KV, int QT>
+__global__ void __launch_bounds__(AttnCfg<DQK, DV, SHARE_KV, QT>::THREADS,
+                                  AttnCfg<DQK, DV, SHARE_KV, QT>::BLOCKS_PER_SM)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                    const __grid_constant__ CUtensorMap tv, const AttnTcArgs a) {
-    using C = AttnCfg<DQK, DV, SHARE_KV>;
+    using C = AttnCfg<DQK, DV, SHARE_KV, QT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* bar_q = bars + 0;
-    uint64_t* kfull = bars + 1;    // [2]
-    uint64_t* kempty = bars + 3;   // [2]
-    auto vfull2 = [bars](int st) { return bars + (st ? 20 : 5); };    // per V stage
-    auto vempty2 = [bars](int st) { return bars + (st ? 21 : 6); };
-    uint64_t* sfull = bars + 7;    // S_j in TMEM
-    uint64_t* sfree = bars + 8;    // S_j read by the softmax warps
-    uint64_t* pfull = bars + 9;    // P_j in shared memory (and O rescaled if needed)
-    uint64_t* ofull = bars + 10;   // P_j . V_j accumulated (P buffer and V stage free)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
-    uint64_t* xchg = bars + 12;    // [4] per lane quadrant: both column halves posted their row maxima
-    uint64_t* lfin = bars + 16;    // [4] per lane quadrant: both halves posted their row sums
+    uint64_t* kfull = bars + 1;    // [3] per K stage
+    uint64_t* kempty = bars + 4;   // [3]
+    uint64_t* vfull = bars + 7;    // [3] per V stage
+    uint64_t* vempty = bars + 10;  // [3]
+    uint64_t* sfull = bars + 13;   // [QT] S_t(j) in TMEM
+    uint64_t* pfull = bars + 15;   // [QT] P_t(j) in TMEM (and O_t rescaled if needed)
+    uint64_t* oready = bars + 17;  // [QT] PV_t(j) complete
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+    constexpr int KS = C::KSTAGES;
+    constexpr int VS = C::VSTAGES > 0 ? C::VSTAGES : 1;   // V stages (unused when V is the shared latent K)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // Work items ranked by cost, heaviest (last query block: most keys) first. CTAs start in
-    // launch order, one per SM and then a second one per SM; when the grid needs more than
-    // one CTA per SM but fits two, the CTA in position S + i takes the lightest item left,
-    // so that an SM pairs a long query block with a short one instead of two long ones.
-    const int W = a.nqb * a.hq * a.batch;
+    // Work items ranked by cost, heaviest (last query blocks: most keys) first. With one
+    // tile per CTA and two CTAs per SM, when the grid needs more than one CTA per SM but fits
+    // two, the CTA in position S + i takes the lightest item left, so that an SM pairs a long
+    // query block with a short one.
+    const int W = a.npairs * a.hq * a.batch;
     const int L = blockIdx.x;
-    const int rank = (W > a.sms && W <= 2 * a.sms && L >= a.sms) ? W - 1 - (L - a.sms) : L;
-    const int per_qb = a.hq * a.batch;
-    const int qb = a.nqb - 1 - rank / per_qb;
-    const int h = (rank % per_qb) % a.hq;
-    const int b = (rank % per_qb) / a.hq;
+    const int rank = (QT == 1 && W > a.sms && W <= 2 * a.sms && L >= a.sms) ? W - 1 - (L - a.sms) : L;
+    const int per_p = a.hq * a.batch;
+    const int pr = a.npairs - 1 - rank / per_p;
+    const int h = (rank % per_p) % a.hq;
+    const int b = (rank % per_p) / a.hq;
     const int g = (h * a.hkv) / a.hq;
-    const int q0 = qb * kBQ;
-    const int row0 = b * a.seq;                        // first token row of this sequence
-    const int n_kb = min(qb + 1, (a.seq + kBK - 1) / kBK);
+    const int row0 = b * a.seq;                          // first token row of this sequence
+    // tile t covers query block qb0 + t; a tile past the last block does nothing
+    const int qb0 = pr * QT;
+    int nkb_t[QT];
+#pragma unroll
+    for (int t = 0; t < QT; ++t) nkb_t[t] = qb0 + t < a.nqb ? qb0 + t + 1 : 0;
+    int n_kb = 0;
+#pragma unroll
+    for (int t = 0; t < QT; ++t) n_kb = max(n_kb, nkb_t[t]);
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 3; ++i) {
             mbar_init(&kfull[i], 1);
             mbar_init(&kempty[i], 1);
+            mbar_init(&vfull[i], 1);
+            mbar_init(&vempty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(vfull2(i), 1);
-            mbar_init(vempty2(i), 1);
-        }
-        mbar_init(sfull, 1);
-        mbar_init(sfree, 8);
-        mbar_init(pfull, 8);
-        mbar_init(ofull, 1);
-        for (int q = 0; q < 4; ++q) {
-            mbar_init(&xchg[q], 2);
-            mbar_init(&lfin[q], 2);
+        for (int t = 0; t < QT; ++t) {
+            mbar_init(&sfull[t], 1);
+            mbar_init(&pfull[t], 4);
+            mbar_init(&oready[t], 1);
         }
         mbar_fence_init();
     }
@@ -177,224 +211,216 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     pdl_trigger();
     pdl_wait();
 
-    if (warp == 0) {
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_CONTROL));
+      if (warp == 0) {
         if (lane == 0) {
-            mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
-            for (int t = 0; t < C::QA; ++t)
-                tma_load_2d(smem + C::OFF_Q + t * kAtom, &tq, bar_q, h * a.q_hstride + 64 * t, row0 + q0);
-            // K block j goes to stage j % KSTAGES (use j / KSTAGES of it), V block j to stage j & 1
-            auto load_k = [&](int j) -> bool {
-                const int s = j % C::KSTAGES;
-                if (!mbar_wait(&kempty[s], ((j / C::KSTAGES) & 1) ^ 1, a.flags)) return false;
-                mbar_arrive_expect_tx(&kfull[s], C::K_BYTES);
-                for (int t = 0; t < C::QA; ++t)
-                    tma_load_2d(smem + C::OFF_K + s * C::K_BYTES + t * kAtom, &tk, &kfull[s],
-                                g * a.k_hstride + 64 * t, row0 + j * kBK);
-                return true;
-            };
-            auto load_v = [&](int j) -> bool {
-                const int s = j & 1;
-                if (!mbar_wait(vempty2(s), ((j >> 1) & 1) ^ 1, a.flags)) return false;
-                mbar_arrive_expect_tx(vfull2(s), C::V_BYTES);
-                for (int t = 0; t < C::VA; ++t)
-                    tma_load_2d(smem + C::OFF_V + s * C::V_BYTES + t * kAtom, &tv, vfull2(s),
-                                g * a.v_hstride + 64 * t, row0 + j * kBK);
-                return true;
-            };
-            bool ok = load_k(0);
+            int ntiles = 0;
+#pragma unroll
+            for (int t = 0; t < QT; ++t) ntiles += nkb_t[t] > 0;
+            mbar_arrive_expect_tx(bar_q, ntiles * C::Q_BYTES);
+#pragma unroll
+            for (int t = 0; t < QT; ++t) {
+                if (nkb_t[t] == 0) continue;
+                for (int at = 0; at < C::QA; ++at)
+                    tma_load_2d(smem + C::OFF_Q + t * C::Q_BYTES + at * kAtom, &tq, bar_q,
+                                h * a.q_hstride + 64 * at, row0 + (qb0 + t) * kBQ);
+            }
+            // block j: K into stage j % KS, V into stage j % VS; a stage is refilled once the
+            // MMAs that read its previous block have completed
 #pragma unroll 1
-            for (int j = 0; j < n_kb && ok; ++j) {
-                // V_j first (its stage frees when P_{j-2} V_{j-2} is done, well before S_j),
-                // then K_{j+1} (its stage frees when S_j has read K_j)
-                if (!SHARE_KV) ok = load_v(j);
-                if (ok && j + 1 < n_kb) ok = load_k(j + 1);
+            for (int j = 0; j < n_kb; ++j) {
+                const int sk = j % KS;
+                if (!mbar_wait(&kempty[sk], ((j / KS) & 1) ^ 1, a.flags)) break;
+                mbar_arrive_expect_tx(&kfull[sk], C::K_BYTES);
+                for (int at = 0; at < C::QA; ++at)
+                    tma_load_2d(smem + C::OFF_K + sk * C::K_BYTES + at * kAtom, &tk, &kfull[sk],
+                                g * a.k_hstride + 64 * at, row0 + j * kBK);
+                if (!SHARE_KV) {
+                    const int sv = j % VS;
+                    if (!mbar_wait(&vempty[sv], ((j / VS) & 1) ^ 1, a.flags)) break;
+                    mbar_arrive_expect_tx(&vfull[sv], C::V_BYTES);
+                    for (int at = 0; at < C::VA; ++at)
+                        tma_load_2d(smem + C::OFF_V + sv * C::V_BYTES + at * kAtom, &tv, &vfull[sv],
+                                    g * a.v_hstride + 64 * at, row0 + j * kBK);
+                }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t id_s = idesc_bf16(kBQ, kBK, 0);
             constexpr uint32_t id_o = idesc_bf16(kBQ, DV, 1);
-            const uint32_t sq = smem_u32(smem + C::OFF_Q);
-            const uint32_t sp = smem_u32(smem + C::OFF_P);
             bool ok = mbar_wait(bar_q, 0, a.flags);
-            auto issue_s = [&](int j) -> bool {
-                const int s = j % C::KSTAGES;
-                if (!mbar_wait(&kfull[s], (j / C::KSTAGES) & 1, a.flags)) return false;
-                if (!mbar_wait(sfree, (j & 1) ^ 1, a.flags)) return false;
+            int k_ready = -1;                 // K blocks 0 .. k_ready are known to be loaded
+            // S_t(j) = Q_t K_j^T into score buffer `buf`; after the last tile that reads K_j,
+            // K_j's stage is released (only if it is loaded again, so that no arrival is
+            // pending when the CTA leaves; the shared latent K is released after its PVs)
+            auto issue_s = [&](int t, int j, int buf) -> bool {
+                for (; k_ready < j; ++k_ready)
+                    if (!mbar_wait(&kfull[(k_ready + 1) % KS], ((k_ready + 1) / KS) & 1, a.flags)) return false;
                 tc_fence_after();
-                const uint32_t sk = smem_u32(smem + C::OFF_K + s * C::K_BYTES);
+                const uint32_t sk = smem_u32(smem + C::OFF_K + (j % KS) * C::K_BYTES);
+                const uint32_t sq = smem_u32(smem + C::OFF_Q + t * C::Q_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < DQK / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-                    tc_mma_bf16(tmem + C::S_COL, sw128_kmajor_desc(sq + off), sw128_kmajor_desc(sk + off),
-                                id_s, kk > 0);
+                    tc_mma_bf16(tmem + C::S_COL + buf * 128, sw128_kmajor_desc(sq + off),
+                                sw128_kmajor_desc(sk + off), id_s, kk > 0);
                 }
-                tc_commit(sfull);
-                if (!SHARE_KV) tc_commit(&kempty[s]);     // K stage consumed
-                return true;
-            };
-            auto issue_o = [&](int j) -> bool {
-                const int s = SHARE_KV ? j % C::KSTAGES : j & 1;
-                if (!mbar_wait(pfull, j & 1, a.flags)) return false;
-                if (!SHARE_KV && !mbar_wait(vfull2(s), (j >> 1) & 1, a.flags)) return false;
-                tc_fence_after();
-                const uint32_t sv = SHARE_KV ? smem_u32(smem + C::OFF_K + s * C::K_BYTES)
-                                             : smem_u32(smem + C::OFF_V + s * C::V_BYTES);
+                tc_commit(&sfull[t]);
+                if (!SHARE_KV) {
+                    int last = 0;
 #pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk) {
-                    const uint32_t offp = (kk >> 2) * kAtom + (kk & 3) * 32;
-                    tc_mma_bf16(tmem + C::O_COL, sw128_kmajor_desc(sp + offp),
-                                sw128_mnmajor_desc(sv + kk * 16 * 128, kAtom), id_o, (j > 0) || kk);
+                    for (int u = 0; u < QT; ++u)
+                        if (j < nkb_t[u]) last = u;
+                    if (t == last && j + KS < n_kb) tc_commit(&kempty[j % KS]);
                 }
-                tc_commit(ofull);
-                if (SHARE_KV)
-                    tc_commit(&kempty[s]);
-                else
-                    tc_commit(vempty2(s));
                 return true;
             };
-            if (ok) ok = issue_s(0);
+            // the first NSBUF scores, in order n = QT j + t
 #pragma unroll 1
-            for (int j = 1; j < n_kb && ok; ++j) {
-                ok = issue_s(j);
-                if (ok) ok = issue_o(j - 1);
+            for (int n = 0; n < C::NSBUF && ok; ++n) {
+                const int t = n % QT, j = n / QT;
+                if (j < nkb_t[t]) ok = issue_s(t, j, n);
             }
-            if (ok) issue_o(n_kb - 1);
+#pragma unroll 1
+            for (int j = 0; j < n_kb && ok; ++j) {
+                const int sv = SHARE_KV ? j % KS : j % VS;
+                if (!SHARE_KV && !mbar_wait(&vfull[sv], (j / VS) & 1, a.flags)) { ok = false; break; }
+                const uint32_t vaddr = SHARE_KV ? smem_u32(smem + C::OFF_K + sv * C::K_BYTES)
+                                                : smem_u32(smem + C::OFF_V + sv * C::V_BYTES);
+#pragma unroll 1
+                for (int t = 0; t < QT && ok; ++t) {
+                    if (j >= nkb_t[t]) continue;
+                    if (!mbar_wait(&pfull[t], j & 1, a.flags)) { ok = false; break; }
+                    tc_fence_after();
+                    const int buf = (QT * j + t) % C::NSBUF;
+                    // O_t += P_t(j) V_j: A = P (bf16 pairs in the first 64 columns of the buffer)
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        tc_mma_bf16_ts(tmem + C::O_COL + t * DV, tmem + C::S_COL + buf * 128 + kk * 8,
+                                       sw128_mnmajor_desc(vaddr + kk * 16 * 128, kAtom), id_o, (j > 0) || kk);
+                    tc_commit(&oready[t]);
+                    // the score NSBUF places later goes into the buffer PV_t(j) has just read
+                    const int n2 = QT * j + t + C::NSBUF;
+                    const int t2 = n2 % QT, j2 = n2 / QT;
+                    if (j2 < nkb_t[t2]) ok = issue_s(t2, j2, buf);
+                }
+                if (!ok) break;
+                // V_j (or the shared latent K_j, also the keys of block j) read by every PV of
+                // block j: release its stage if it is loaded again
+                if (SHARE_KV) {
+                    if (j + KS < n_kb) tc_commit(&kempty[sv]);
+                } else {
+                    if (j + VS < n_kb) tc_commit(&vempty[sv]);
+                }
+            }
         }
+      }
     } else {
-        // Softmax warps 2..9: warp w covers TMEM lane quadrant w & 3 (32 query rows, a thread
-        // per row) and column half (w - 2) / 4 of each key block and of O. The two halves of a
-        // row exchange their block maxima (and, at the end, their sums) through shared memory,
-        // paired by a per-quadrant mbarrier with bounded waits; both then take the same
-        // rescaling decisions, and each rescales and finally writes its own half of O.
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_SOFTMAX));
+        // Softmax warpgroup 1 + t (warps 4 + 4t .. 7 + 4t): TMEM lane quadrant warp & 3, one
+        // query row per thread.
+        const int t = (warp - 4) >> 2;
         const int quad = warp & 3;
-        const int half = (warp - 2) >> 2;
         const int r = quad * 32 + lane;
-        const int qpos = q0 + r;
+        const int qb = qb0 + t;
+        const int qpos = qb * kBQ + r;
+        const int nkb = nkb_t[t];
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+        const uint32_t o_col = C::O_COL + t * DV;
         const float sl = a.scale_log2;
         float m_ref = -INFINITY, l = 0.0f;
-        uint8_t* arow = smem + C::OFF_P + half * kAtom + r * 128;    // this half's P atom
-        float* mxx = reinterpret_cast<float*>(smem + C::OFF_X);      // [2 parity][2 half][128]
-        float* lxx = mxx + 2 * 2 * 128;                              // [2 half][128]
-        constexpr int HC = kBK / 64;                                 // 32-column chunks per half
-        constexpr int OC = DV / 64;                                  // 32-column O chunks per half
         bool ok = true;
 #pragma unroll 1
-        for (int j = 0; j < n_kb && ok; ++j) {
-            if (!mbar_wait(sfull, j & 1, a.flags)) { ok = false; break; }
+        for (int j = 0; j < nkb && ok; ++j) {
+            if (!mbar_wait(&sfull[t], j & 1, a.flags)) { ok = false; break; }
             tc_fence_after();
+            const uint32_t s_col = C::S_COL + ((QT * j + t) % C::NSBUF) * 128;
+            uint32_t v[128];
+            tmem_ld32(lane_base + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(v + 0));
+            tmem_ld32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+            tmem_ld32(lane_base + s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
+            tmem_ld32(lane_base + s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
+            tmem_wait_ld();
             const int key0 = j * kBK;
             const bool need_mask = (j == qb) || (key0 + kBK > a.seq);
-            const int kmax = need_mask ? min(qpos, a.seq - 1) - key0 : kBK - 1;  // last allowed key
-            // pass 1: maximum of this half of the row (scaled to log2 units), then of the row
-            float mx = -INFINITY;
-#pragma unroll 1
-            for (int c = 0; c < HC; ++c) {
-                const int col0 = half * 64 + c * 32;
-                uint32_t v[32];
-                tmem_ld32(lane_base + C::S_COL + col0, v);
-                tmem_wait_ld();
-                if (!need_mask) {
+            if (need_mask) {
+                const int kmax = min(qpos, a.seq - 1) - key0;      // last allowed key column
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(v[i]));
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (col0 + i <= kmax) mx = fmaxf(mx, __uint_as_float(v[i]));
-                }
+                for (int i = 0; i < 128; ++i)
+                    if (i > kmax) v[i] = __float_as_uint(-INFINITY);
             }
-            mx *= sl;
-            float* slot = mxx + (j & 1) * 256;
-            slot[half * 128 + r] = mx;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&xchg[quad]);
-            if (!mbar_wait(&xchg[quad], j & 1, a.flags)) { ok = false; break; }
-            mx = fmaxf(mx, slot[(half ^ 1) * 128 + r]);
-            // O (accumulated by P_{j-1} V_{j-1}) is stable once that MMA has completed
-            if (j > 0 && !mbar_wait(ofull, (j - 1) & 1, a.flags)) { ok = false; break; }
-            tc_fence_after();
+            // row maximum, in four independent chains
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int i = 0; i < 128; i += 4) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) m4[u] = fmaxf(m4[u], __uint_as_float(v[i + u]));
+            }
+            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl;
             if (mx > m_ref + kRescaleThreshold) {
                 const float corr = exp2_ftz(m_ref - mx);
                 if (j > 0) {
+                    // O_t holds blocks 0 .. j - 1 once PV_t(j - 1) has completed (PV_t(j - 2)
+                    // has, since S_t(j) was issued after it: the phase is unambiguous)
+                    if (!mbar_wait(&oready[t], (j - 1) & 1, a.flags)) { ok = false; break; }
+                    tc_fence_after();
 #pragma unroll
-                    for (int c = 0; c < OC; ++c) {
-                        const uint32_t ocol = C::O_COL + half * (DV / 2) + c * 32;
-                        uint32_t v[32];
-                        tmem_ld32(lane_base + ocol, v);
+                    for (int c = 0; c < DV / 32; ++c) {
+                        uint32_t ov[32];
+                        tmem_ld32(lane_base + o_col + c * 32, ov);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * corr);
-                        tmem_st32(lane_base + ocol, v);
+                        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
+                        tmem_st32(lane_base + o_col + c * 32, ov);
                     }
-                    tmem_wait_st();
                 }
                 l *= corr;
                 m_ref = mx;
             }
-            // pass 2: P = 2^(S*sl - m_ref) in bf16 into this half's atom of the swizzled P buffer
-            float rs = 0.0f;
-#pragma unroll 1
-            for (int c = 0; c < HC; ++c) {
-                const int col0 = half * 64 + c * 32;
-                uint32_t v[32];
-                tmem_ld32(lane_base + C::S_COL + col0, v);
-                tmem_wait_ld();
-                uint32_t packed[16];
+            // P = 2^(S sl - m_ref) as bf16 pairs (key 2c in the low half of column c)
+            const float2 slv = make_float2(sl, sl);
+            const float2 mneg = make_float2(-m_ref, -m_ref);
+            float2 rs2 = make_float2(0.0f, 0.0f);
+            uint32_t pk[64];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float p0 = exp2_ftz(__uint_as_float(v[2 * i]) * sl - m_ref);
-                    float p1 = exp2_ftz(__uint_as_float(v[2 * i + 1]) * sl - m_ref);
-                    if (need_mask) {
-                        if (col0 + 2 * i > kmax) p0 = 0.0f;
-                        if (col0 + 2 * i + 1 > kmax) p1 = 0.0f;
-                    }
-                    rs += p0 + p1;
-                    __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                    packed[i] = *reinterpret_cast<uint32_t*>(&pb);
-                }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int phys = (c * 4 + q) ^ (r & 7);
-                    *reinterpret_cast<uint4*>(arow + phys * 16) =
-                        make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
-                }
+            for (int c = 0; c < 64; ++c) {
+                const float2 x = __ffma2_rn(make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])),
+                                            slv, mneg);
+                const float p0 = exp2_ftz(x.x);
+                const float p1 = exp2_ftz(x.y);
+                rs2 = __fadd2_rn(rs2, make_float2(p0, p1));
+                pk[c] = pack_bf16(p0, p1);
             }
-            l += rs;
-            fence_proxy_async();
+            l += rs2.x + rs2.y;
+            tmem_st32(lane_base + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(pk + 0));
+            tmem_st32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(sfree);
-                mbar_arrive(pfull);
-            }
+            if (lane == 0) mbar_arrive(&pfull[t]);
         }
-        if (ok) ok = mbar_wait(ofull, (n_kb - 1) & 1, a.flags);
-        tc_fence_after();
-        // the row sum is the two halves' partial sums
-        lxx[half * 128 + r] = l;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&lfin[quad]);
-        if (ok) ok = mbar_wait(&lfin[quad], 0, a.flags);
-        const float inv = ok ? 1.0f / (l + lxx[(half ^ 1) * 128 + r]) : 0.0f;
-        bf16* out = static_cast<bf16*>(a.o) + static_cast<size_t>(row0 + qpos) * a.ldo + h * a.dv_out +
-                    half * (DV / 2);
+        if (nkb > 0) {
+            if (ok) ok = mbar_wait(&oready[t], (nkb - 1) & 1, a.flags);   // the last PV_t
+            tc_fence_after();
+            const float inv = ok ? 1.0f / l : 0.0f;
+            bf16* out = static_cast<bf16*>(a.o) + static_cast<size_t>(row0 + qpos) * a.ldo + h * a.dv_out;
 #pragma unroll 1
-        for (int c = 0; c < OC; ++c) {
-            uint32_t v[32];
-            tmem_ld32(lane_base + C::O_COL + half * (DV / 2) + c * 32, v);
-            tmem_wait_ld();
-            if (!ok || qpos >= a.seq) continue;
+            for (int c = 0; c < DV / 32; ++c) {
+                uint32_t ov[32];
+                tmem_ld32(lane_base + o_col + c * 32, ov);
+                tmem_wait_ld();
+                if (!ok || qpos >= a.seq) continue;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t w[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * u]) * inv,
-                                                              __uint_as_float(v[8 * q + 2 * u + 1]) * inv);
-                    w[u] = *reinterpret_cast<uint32_t*>(&pb);
+                for (int q = 0; q < 4; ++q) {
+                    uint4 w;
+                    w.x = pack_bf16(__uint_as_float(ov[8 * q + 0]) * inv, __uint_as_float(ov[8 * q + 1]) * inv);
+                    w.y = pack_bf16(__uint_as_float(ov[8 * q + 2]) * inv, __uint_as_float(ov[8 * q + 3]) * inv);
+                    w.z = pack_bf16(__uint_as_float(ov[8 * q + 4]) * inv, __uint_as_float(ov[8 * q + 5]) * inv);
+                    w.w = pack_bf16(__uint_as_float(ov[8 * q + 6]) * inv, __uint_as_float(ov[8 * q + 7]) * inv);
+                    *reinterpret_cast<uint4*>(out + c * 32 + 8 * q) = w;
                 }
-                *reinterpret_cast<uint4*>(out + c * 32 + 8 * q) = make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
     }
@@ -406,14 +432,23 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     }
 }
 
-template <int DQK, int DV, bool SHARE_KV>
+template <int DQK, int DV, bool SHARE_KV, int QT>
 rdt_status launch_tc(const AttnArgs& a, cudaStream_t st) {
-    using C = AttnCfg<DQK, DV, SHARE_KV>;
-    auto kern = attn_tc_kernel<DQK, DV, SHARE_KV>;
+    using C = AttnCfg<DQK, DV, SHARE_KV, QT>;
+    auto kern = attn_tc_kernel<DQK, DV, SHARE_KV, QT>;
     static int configured[64] = {};        // per device: function attributes are set per device
     int dev = 0;
     RDT_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= 64 || !configured[dev]) {
+        // setmaxnreg moves registers within the block's launch allocation: the split is
+        // computed for REGS_LAUNCH registers per thread and would wait forever on fewer
+        cudaFuncAttributes fa;
+        RDT_CUDA_TRY(cudaFuncGetAttributes(&fa, kern));
+        if (fa.numRegs != C::REGS_LAUNCH) {
+            set_error("attention kernel: launch register count " + std::to_string(fa.numRegs) +
+                      " differs from the " + std::to_string(C::REGS_LAUNCH) + " its register split assumes");
+            return RDT_ERR_UNSUPPORTED;
+        }
         RDT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
         RDT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
         if (dev >= 0 && dev < 64) configured[dev] = 1;
@@ -439,18 +474,29 @@ rdt_status launch_tc(const AttnArgs& a, cudaStream_t st) {
     ta.o = a.o;
     ta.flags = a.flags;
     ta.nqb = (a.seq + kBQ - 1) / kBQ;
+    ta.npairs = (ta.nqb + QT - 1) / QT;
     ta.batch = a.batch;
     ta.sms = num_sms();
-    const dim3 grid(static_cast<unsigned>(ta.nqb) * a.hq * a.batch);
-    RDT_CUDA_TRY(launch_pdl(kern, grid, dim3(kAttnThreads), C::SMEM, st, tq, tk, tv, ta));
+    const dim3 grid(static_cast<unsigned>(ta.npairs) * a.hq * a.batch);
+    RDT_CUDA_TRY(launch_pdl(kern, grid, dim3(C::THREADS), C::SMEM, st, tq, tk, tv, ta));
     return RDT_OK;
+}
+
+// Two query tiles per CTA (one CTA per SM) once the work items of two tiles still give every
+// SM at least two; otherwise one tile per CTA, two CTAs per SM.
+template <int DQK, int DV, bool SHARE_KV>
+rdt_status launch_choose(const AttnArgs& a, cudaStream_t st) {
+    const long nqb = (a.seq + kBQ - 1) / kBQ;
+    const long items2 = (nqb + 1) / 2 * a.hq * a.batch;
+    if (nqb >= 2 && items2 >= 2L * num_sms()) return launch_tc<DQK, DV, SHARE_KV, 2>(a, st);
+    return launch_tc<DQK, DV, SHARE_KV, 1>(a, st);
 }
 
 }  // namespace
 
 rdt_status attention_tc(const AttnArgs& a, cudaStream_t st) {
-    if (a.dqk == 64 && a.dv == 64) return launch_tc<64, 64, false>(a, st);
-    if (a.dqk == 160 && a.dv == 128 && a.v == a.k) return launch_tc<160, 128, true>(a, st);
+    if (a.dqk == 64 && a.dv == 64) return launch_choose<64, 64, false>(a, st);
+    if (a.dqk == 160 && a.dv == 128 && a.v == a.k) return launch_choose<160, 128, true>(a, st);
     set_error("tensor-core attention: unsupported head dimensions");
     return RDT_ERR_UNSUPPORTED;
 }

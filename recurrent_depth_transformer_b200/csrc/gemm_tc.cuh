@@ -236,10 +236,24 @@ __device__ __forceinline__ void epilogue_topk(const EpiParams& p, uint32_t taddr
     if (!__shfl_sync(0xffffffffu, last, 0)) return;
     __threadfence();
     if (!valid) return;
+    // the complete row, 32 logits at a time: eight 16-byte L2 loads in flight per chunk
+    // (n_exp is a multiple of 8: rows are 32-byte aligned), then the insertions
     TopK<KMAX> tk;
 #pragma unroll 1
-    for (int ex = 0; ex < p.n_exp; ++ex)
-        tk.insert(__ldcg(lrow + ex), p.bias ? p.bias[ex] : 0.0f, ex, p.top_k);
+    for (int c0 = 0; c0 < p.n_exp; c0 += 32) {
+        float v[32];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float4 x = c0 + 4 * q < p.n_exp ? __ldcg(reinterpret_cast<const float4*>(lrow + c0 + 4 * q))
+                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int ex = c0 + i;
+            if (ex < p.n_exp) tk.insert(v[i], p.bias ? p.bias[ex] : 0.0f, ex, p.top_k);
+        }
+    }
     tk.write(p, crow);
 }
 

@@ -32,7 +32,6 @@ struct rdt_handle {
     bool bf = true;
     size_t esz = 2;
     int ntok = 0;
-    int kext = 64;                 // padded LoRA width = one 128-byte K block
     int G = 0;                     // expert groups = routed + shared
     float rho = 0.0f;
     cudaStream_t last_stream = nullptr;
@@ -43,7 +42,10 @@ struct rdt_handle {
     float *A = nullptr, *Bw = nullptr, *g1 = nullptr, *g2 = nullptr, *rbias = nullptr;
     float *q_norm = nullptr, *kv_norm = nullptr;
     void *wqkv = nullptr, *wo = nullptr, *wr = nullptr, *w13 = nullptr, *w2 = nullptr;
-    void *lqa = nullptr, *lqb = nullptr, *loa = nullptr, *lob = nullptr;
+    // depth-wise LoRA: loop t uses W_t = W + B_t A_t, merged at create for every adapter:
+    // wqkv holds [W_q,l ; W_k ; W_v] for l = 0 .. n_lora - 1 (one block of nqkv rows each) and
+    // wo holds W_o,l ([d, nq] each); without LoRA both hold the single base matrix
+    int n_wsets = 1;
     void *wlat = nullptr, *wqabs = nullptr;
     float *rope_cos = nullptr, *rope_sin = nullptr;
     int rot = 0;
@@ -56,7 +58,7 @@ struct rdt_handle {
 
     // workspace
     float *hbuf[2] = {nullptr, nullptr}, *Be = nullptr, *y = nullptr, *lat = nullptr;
-    void *xn = nullptr, *tq = nullptr, *to = nullptr, *qkv = nullptr, *o = nullptr;
+    void *xn = nullptr, *qkv = nullptr, *o = nullptr;
     void *cq = nullptr, *kvlat = nullptr, *xperm = nullptr, *U = nullptr, *yn_lo = nullptr;
     int bn_router = 64;
     int router_split = 1;          // K split of the router GEMM over CTAs
@@ -87,7 +89,8 @@ struct rdt_handle {
     int* act_loops = nullptr;
 
     // tensor maps
-    CUtensorMap m_xn, m_wqkv, m_tq, m_lqb, m_o, m_wo, m_to, m_lob, m_xperm, m_w13, m_U, m_w2;
+    CUtensorMap m_xn, m_o, m_xperm, m_w13, m_U, m_w2;
+    std::vector<CUtensorMap> m_wqkv, m_wo;   // one per weight set (adapter)
     CUtensorMap m_wlat, m_cq, m_wqabs, m_ynlo, m_wr;
 
     // trace
@@ -98,8 +101,11 @@ struct rdt_handle {
     // launch accounting and optional per-kernel event timing
     int64_t launches = 0;
     bool prof_on = false;
-    std::vector<cudaEvent_t> ev_pool;
+    bool prof_graph = false;       // profiling inside graph replay (event-record nodes)
+    bool capturing = false;        // the launch sequence is being captured into the graph
+    std::vector<cudaEvent_t> ev_pool;       // events of eager calls, reused after every read
     size_t ev_used = 0;
+    std::vector<cudaEvent_t> graph_events;  // events recorded by nodes of captured graphs
     // CUDA graph of the whole T-loop launch sequence, keyed by the call's pointers and T
     struct GraphKey {
         const void* h0 = nullptr;
@@ -118,6 +124,8 @@ struct rdt_handle {
     int64_t g_launches = 0;
     struct Pending { int kind; cudaEvent_t a, b; int n; };
     std::vector<Pending> pending;
+    std::vector<Pending> graph_pending;   // event pairs recorded by every replay of the graph
+    bool graph_ran = false;               // the graph ran since its events were last read
     std::vector<double> prof_ms;
     std::vector<int64_t> prof_n;
 };
@@ -128,34 +136,54 @@ namespace {
 constexpr int kFillerRows = 256;
 
 // kernel classes reported by rdt_profile_read
-enum Kind { K_HOIST, K_NORM1, K_GEMM_QKV, K_GEMM_LAT, K_MLA_NORM, K_GEMM_Q, K_ATTENTION, K_LORA_DOWN,
+enum Kind { K_HOIST, K_NORM1, K_GEMM_QKV, K_GEMM_LAT, K_MLA_NORM, K_GEMM_Q, K_ATTENTION,
             K_GEMM_O, K_NORM2, K_ROUTER, K_DISPATCH, K_GEMM_UP, K_GEMM_DOWN, K_CHECK, K_DENSE_B, K_ACT,
             K_COMBINE, K_COUNT };
 const char* const kKindName[K_COUNT] = {"hoist", "norm1", "gemm_qkv", "gemm_latent", "mla_latent_norm",
-                                         "gemm_q_absorbed", "attention", "lora_down", "gemm_o",
+                                         "gemm_q_absorbed", "attention", "gemm_o",
                                          "norm2", "router_topk", "moe_dispatch", "gemm_up", "gemm_down",
                                          "check_finite", "dense_injection", "act_halting", "moe_combine"};
 
+// During graph capture the events become event-record nodes of the graph (external
+// records), so that every replay records them again; they are then kept apart from the
+// events of eager calls, which are reused after every read.
 rdt_status prof_begin(rdt_handle* h, int kind, int nlaunch, cudaStream_t st) {
     h->launches += nlaunch;
     if (!h->prof_on) return RDT_OK;
-    while (h->ev_pool.size() < h->ev_used + 2) {
-        cudaEvent_t ev;
-        RDT_CUDA_TRY(cudaEventCreate(&ev));
-        h->ev_pool.push_back(ev);
+    cudaEvent_t ev[2];
+    for (cudaEvent_t& e : ev) {
+        if (h->capturing) {
+            RDT_CUDA_TRY(cudaEventCreate(&e));
+            h->graph_events.push_back(e);  // destroyed with the handle
+            continue;
+        }
+        while (h->ev_pool.size() <= h->ev_used) {
+            cudaEvent_t x;
+            RDT_CUDA_TRY(cudaEventCreate(&x));
+            h->ev_pool.push_back(x);
+        }
+        e = h->ev_pool[h->ev_used++];
     }
-    rdt_handle::Pending p{kind, h->ev_pool[h->ev_used], h->ev_pool[h->ev_used + 1], nlaunch};
-    h->ev_used += 2;
-    RDT_CUDA_TRY(cudaEventRecord(p.a, st));
-    h->pending.push_back(p);
+    rdt_handle::Pending p{kind, ev[0], ev[1], nlaunch};
+    if (h->capturing) {
+        RDT_CUDA_TRY(cudaEventRecordWithFlags(p.a, st, cudaEventRecordExternal));
+        h->graph_pending.push_back(p);
+    } else {
+        RDT_CUDA_TRY(cudaEventRecord(p.a, st));
+        h->pending.push_back(p);
+    }
     return RDT_OK;
 }
 rdt_status prof_end(rdt_handle* h, cudaStream_t st) {
     if (!h->prof_on) return RDT_OK;
-    RDT_CUDA_TRY(cudaEventRecord(h->pending.back().b, st));
+    if (h->capturing)
+        RDT_CUDA_TRY(cudaEventRecordWithFlags(h->graph_pending.back().b, st, cudaEventRecordExternal));
+    else
+        RDT_CUDA_TRY(cudaEventRecord(h->pending.back().b, st));
     return RDT_OK;
 }
-// Resolve recorded event pairs into the per-kind sums (the stream must have completed).
+// Resolve recorded event pairs into the per-kind sums (the stream must have completed). The
+// graph's pairs describe its last replay only: each replay records them anew.
 rdt_status prof_flush(rdt_handle* h) {
     for (const auto& p : h->pending) {
         float ms = 0.0f;
@@ -164,6 +192,16 @@ rdt_status prof_flush(rdt_handle* h) {
         h->prof_n[p.kind] += p.n;
     }
     h->pending.clear();
+    if (h->graph_ran) {
+        for (const auto& p : h->graph_pending) {
+            float ms = 0.0f;
+            RDT_CUDA_TRY(cudaEventElapsedTime(&ms, p.a, p.b));
+            h->prof_ms[p.kind] += ms;
+            h->prof_n[p.kind] += p.n;
+        }
+        h->graph_ran = false;
+    }
+    // eager events are reused; the graph's belong to it (its nodes record them)
     h->ev_used = 0;
     return RDT_OK;
 }
@@ -330,21 +368,19 @@ rdt_status build_maps(rdt_handle* h) {
     const int S = c.n_shared, E = c.n_experts, hid = c.expert_hidden;
     RDT_TRY(make_tmap_2d(&h->m_xn, h->xn, bf, d, N, d * es, kbox, 128));
     RDT_TRY(make_tmap_2d(&h->m_o, h->o, bf, h->owidth, N, h->owidth * es, kbox, 128));
-    RDT_TRY(make_tmap_2d(&h->m_wo, h->wo, bf, h->owidth, d, h->owidth * es, kbox, h->bn_o >> h->pair_o));
+    h->m_wo.resize(h->n_wsets);
+    for (int l = 0; l < h->n_wsets; ++l)
+        RDT_TRY(make_tmap_2d(&h->m_wo[l], static_cast<const char*>(h->wo) + static_cast<size_t>(l) * d * h->owidth * es,
+                             bf, h->owidth, d, h->owidth * es, kbox, h->bn_o >> h->pair_o));
     if (c.attn_type == RDT_GQA) {
-        RDT_TRY(make_tmap_2d(&h->m_wqkv, h->wqkv, bf, d, h->nqkv, d * es, kbox, h->bn_qkv >> h->pair_qkv));
+        h->m_wqkv.resize(h->n_wsets);
+        for (int l = 0; l < h->n_wsets; ++l)
+            RDT_TRY(make_tmap_2d(&h->m_wqkv[l], static_cast<const char*>(h->wqkv) + static_cast<size_t>(l) * h->nqkv * d * es,
+                                 bf, d, h->nqkv, d * es, kbox, h->bn_qkv >> h->pair_qkv));
     } else {
         RDT_TRY(make_tmap_2d(&h->m_wlat, h->wlat, bf, d, h->lat_w, d * es, kbox, 128));
         RDT_TRY(make_tmap_2d(&h->m_cq, h->cq, bf, c.q_lora_rank, N, c.q_lora_rank * es, kbox, 128));
         RDT_TRY(make_tmap_2d(&h->m_wqabs, h->wqabs, bf, c.q_lora_rank, h->qt_w, c.q_lora_rank * es, kbox, 160));
-    }
-    if (c.n_lora) {
-        RDT_TRY(make_tmap_2d(&h->m_tq, h->tq, bf, h->kext, N, h->kext * es, kbox, 128));
-        RDT_TRY(make_tmap_2d(&h->m_to, h->to, bf, h->kext, N, h->kext * es, kbox, 128));
-        RDT_TRY(make_tmap_2d(&h->m_lqb, h->lqb, bf, h->kext, static_cast<uint64_t>(c.n_lora) * h->nqkv,
-                             h->kext * es, kbox, h->bn_qkv >> h->pair_qkv));
-        RDT_TRY(make_tmap_2d(&h->m_lob, h->lob, bf, h->kext, static_cast<uint64_t>(c.n_lora) * d,
-                             h->kext * es, kbox, h->bn_o >> h->pair_o));
     }
     // capacity layout, cap rows per group: xperm = [yn (N rows) | expert e: rows N + e cap ..
     // N + (e + 1) cap), U = [shared expert s: rows s cap .. | expert e: rows (S + e) cap ..],
@@ -365,7 +401,6 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
     h->cfg = c;
     h->bf = c.dtype == RDT_BF16;
     h->esz = h->bf ? 2 : 4;
-    h->kext = static_cast<int>(128 / h->esz);
     h->ntok = c.batch * c.seq;
     h->G = c.n_experts + c.n_shared;
     h->prof_ms.assign(K_COUNT, 0.0);
@@ -505,32 +540,31 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         h->nqkv = h->nq + 2 * h->nkv;
         h->owidth = h->nq;
         h->rot = c.head_dim;
-        RDT_TRY(dev_alloc(h, &h->wqkv, static_cast<size_t>(h->nqkv) * d * es));
-        char* q = static_cast<char*>(h->wqkv);
-        RDT_TRY(copy_d2d(q, w->wq, static_cast<size_t>(h->nq) * d * es, st));
-        RDT_TRY(copy_d2d(q + static_cast<size_t>(h->nq) * d * es, w->wk, static_cast<size_t>(h->nkv) * d * es, st));
-        RDT_TRY(copy_d2d(q + static_cast<size_t>(h->nq + h->nkv) * d * es, w->wv,
-                         static_cast<size_t>(h->nkv) * d * es, st));
-        RDT_TRY(dev_alloc(h, &h->wo, static_cast<size_t>(d) * h->nq * es));
-        RDT_TRY(copy_d2d(h->wo, w->wo, static_cast<size_t>(d) * h->nq * es, st));
-        if (c.n_lora) {
-            const int L = c.n_lora, r = c.lora_rank, kx = h->kext;
-            RDT_TRY(dev_alloc(h, &h->lqa, static_cast<size_t>(L) * r * d * es));
-            RDT_TRY(copy_d2d(h->lqa, w->lq_a, static_cast<size_t>(L) * r * d * es, st));
-            RDT_TRY(dev_alloc(h, &h->loa, static_cast<size_t>(L) * r * h->nq * es));
-            RDT_TRY(copy_d2d(h->loa, w->lo_a, static_cast<size_t>(L) * r * h->nq * es, st));
-            RDT_TRY(dev_alloc(h, &h->lqb, static_cast<size_t>(L) * h->nqkv * kx * es, true));
-            RDT_TRY(dev_alloc(h, &h->lob, static_cast<size_t>(L) * d * kx * es, true));
-            for (int l = 0; l < L; ++l) {
-                RDT_CUDA_TRY(cudaMemcpy2DAsync(static_cast<char*>(h->lqb) + static_cast<size_t>(l) * h->nqkv * kx * es,
-                                               kx * es,
-                                               static_cast<const char*>(w->lq_b) + static_cast<size_t>(l) * h->nq * r * es,
-                                               r * es, r * es, h->nq, cudaMemcpyDeviceToDevice, st));
-                RDT_CUDA_TRY(cudaMemcpy2DAsync(static_cast<char*>(h->lob) + static_cast<size_t>(l) * d * kx * es,
-                                               kx * es,
-                                               static_cast<const char*>(w->lo_b) + static_cast<size_t>(l) * d * r * es,
-                                               r * es, r * es, d, cudaMemcpyDeviceToDevice, st));
+        // one weight set per adapter: W_q,l = W_q + B_l A_l and W_o,l = W_o + B'_l A'_l, summed
+        // in fp32 and rounded once to the element type
+        const int L = c.n_lora ? c.n_lora : 1, r = c.lora_rank;
+        h->n_wsets = L;
+        const size_t qkv_set = static_cast<size_t>(h->nqkv) * d * es, o_set = static_cast<size_t>(d) * h->nq * es;
+        RDT_TRY(dev_alloc(h, &h->wqkv, qkv_set * L));
+        RDT_TRY(dev_alloc(h, &h->wo, o_set * L));
+        for (int l = 0; l < L; ++l) {
+            char* q = static_cast<char*>(h->wqkv) + qkv_set * l;
+            char* o = static_cast<char*>(h->wo) + o_set * l;
+            if (c.n_lora) {
+                const char* qa = static_cast<const char*>(w->lq_a) + static_cast<size_t>(l) * r * d * es;
+                const char* qb = static_cast<const char*>(w->lq_b) + static_cast<size_t>(l) * h->nq * r * es;
+                const char* oa = static_cast<const char*>(w->lo_a) + static_cast<size_t>(l) * r * h->nq * es;
+                const char* ob = static_cast<const char*>(w->lo_b) + static_cast<size_t>(l) * d * r * es;
+                // C[m, n] = W[m, n] + sum_k B[m, k] A[k, n]
+                RDT_TRY(prep_matmul(h->bf, qb, r, 1, qa, d, 1, q, d, h->nq, d, r, st, w->wq, d));
+                RDT_TRY(prep_matmul(h->bf, ob, r, 1, oa, h->nq, 1, o, h->nq, d, h->nq, r, st, w->wo, h->nq));
+            } else {
+                RDT_TRY(copy_d2d(q, w->wq, static_cast<size_t>(h->nq) * d * es, st));
+                RDT_TRY(copy_d2d(o, w->wo, o_set, st));
             }
+            RDT_TRY(copy_d2d(q + static_cast<size_t>(h->nq) * d * es, w->wk, static_cast<size_t>(h->nkv) * d * es, st));
+            RDT_TRY(copy_d2d(q + static_cast<size_t>(h->nq + h->nkv) * d * es, w->wv,
+                             static_cast<size_t>(h->nkv) * d * es, st));
         }
     } else {
         const int H = c.n_heads, ql = c.q_lora_rank, kvl = c.kv_lora_rank, rp = c.qk_rope_dim;
@@ -594,10 +628,6 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
     RDT_TRY(dev_alloc(h, &h->Be, nd * 4));
     RDT_TRY(dev_alloc(h, &h->y, nd * 4));
     RDT_TRY(dev_alloc(h, &h->xn, nd * es));
-    if (c.n_lora) {
-        RDT_TRY(dev_alloc(h, &h->tq, static_cast<size_t>(N) * h->kext * es, true));
-        RDT_TRY(dev_alloc(h, &h->to, static_cast<size_t>(N) * h->kext * es, true));
-    }
     if (c.attn_type == RDT_GQA) {
         RDT_TRY(dev_alloc(h, &h->qkv, static_cast<size_t>(N) * h->nqkv * es));
     } else {
@@ -626,7 +656,9 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         const int mt = (N + 127) / 128;
         const int kb = 2 * d * 2 / 128;
         int split = 1;
-        for (int sp = 1; sp <= kb && !c.deterministic; ++sp)   // deterministic: logits in one CTA
+        // deterministic: logits in one CTA; the split's final read takes 16-byte row pieces,
+        // so the expert count must be a multiple of 4
+        for (int sp = 1; sp <= kb && !c.deterministic && E % 4 == 0; ++sp)
             if (kb % sp == 0 && static_cast<long>(mt) * sp <= num_sms()) split = sp;
         h->router_split = split;
         RDT_TRY(dev_alloc(h, &h->logits, static_cast<size_t>(N) * E * 4, true));
@@ -670,11 +702,6 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
     n1.ntok = N;
     n1.dim = d;
     n1.eps = c.norm_eps;
-    if (lora) {
-        n1.lora_a = static_cast<const char*>(h->lqa) + static_cast<size_t>(li) * c.lora_rank * d * h->esz;
-        n1.lora_r = c.lora_rank;
-        n1.lora_t = h->tq;
-    }
     if (loop_mode) {
         n1.zero_counts = h->counts;
         n1.n_zero = h->G;
@@ -701,8 +728,6 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
     if (c.attn_type == RDT_GQA) {
         ga.N = h->nqkv;
         ga.kb_main = static_cast<int>(d * h->esz / 128);
-        ga.kb_ext = lora ? 1 : 0;
-        ga.b2_row0 = li * h->nqkv;
         ga.pair = h->pair_qkv;
         ep.kind = EPI_ROPE;
         ep.out = h->qkv;
@@ -715,8 +740,7 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         ep.rot_off = 0;
         ep.rot_dim = c.head_dim;
         ep.rope_limit = h->nq + h->nkv;
-        TIMED(h, K_GEMM_QKV, 1, st, gemm_tc(h->bf, h->bn_qkv, h->m_xn, h->m_wqkv, lora ? &h->m_tq : nullptr,
-                                           lora ? &h->m_lqb : nullptr, ga, ep, st));
+        TIMED(h, K_GEMM_QKV, 1, st, gemm_tc(h->bf, h->bn_qkv, h->m_xn, h->m_wqkv[li], nullptr, nullptr, ga, ep, st));
         at.q = h->qkv;
         at.ldq = h->nqkv;
         at.q_hstride = c.head_dim;
@@ -793,16 +817,10 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
     at.flags = h->flags;
     TIMED(h, K_ATTENTION, 1, st, attention(h->bf, at, st));
 
-    if (lora) {
-        const void* A = static_cast<const char*>(h->loa) + static_cast<size_t>(li) * c.lora_rank * h->nq * h->esz;
-        TIMED(h, K_LORA_DOWN, 1, st, lora_down(h->bf, h->o, h->owidth, N, h->owidth, A, c.lora_rank, h->to, st));
-    }
     GemmArgs go{};
     go.M = N;
     go.N = d;
     go.kb_main = static_cast<int>(h->owidth * h->esz / 128);
-    go.kb_ext = lora ? 1 : 0;
-    go.b2_row0 = li * d;
     go.pair = h->pair_o;
     go.flags = h->flags;
     EpiParams eo{};
@@ -818,8 +836,7 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         eo.out = a_out;
         eo.ldo = d;
     }
-    TIMED(h, K_GEMM_O, 1, st, gemm_tc(h->bf, h->bn_o, h->m_o, h->m_wo, lora ? &h->m_to : nullptr,
-                                      lora ? &h->m_lob : nullptr, go, eo, st));
+    TIMED(h, K_GEMM_O, 1, st, gemm_tc(h->bf, h->bn_o, h->m_o, h->m_wo[li], nullptr, nullptr, go, eo, st));
     return RDT_OK;
 }
 
@@ -1039,7 +1056,7 @@ void drop_graph(rdt_handle* h) {
 // and launches the graph, later ones only launch it. Tracing or profiling runs eagerly.
 rdt_status run_loop(rdt_handle* h, const void* h0, const void* e, int T, float* out, cudaStream_t st,
                     bool act = false, int32_t* n_loops = nullptr) {
-    const bool graphable = !h->prof_on && !h->tr_idx && !h->tr_w && !h->tr_h;
+    const bool graphable = (!h->prof_on || h->prof_graph) && !h->tr_idx && !h->tr_w && !h->tr_h;
     if (!graphable) return loop_impl(h, h0, e, T, out, act, n_loops, st);
     rdt_handle::GraphKey key;
     key.h0 = h0;
@@ -1051,6 +1068,7 @@ rdt_status run_loop(rdt_handle* h, const void* h0, const void* e, int T, float* 
     if (h->gexec && h->gkey == key) {
         RDT_CUDA_TRY(cudaGraphLaunch(h->gexec, st));
         h->launches += h->g_launches;
+        h->graph_ran = true;
         return RDT_OK;
     }
     if (!(h->seen_key == key)) {
@@ -1063,8 +1081,11 @@ rdt_status run_loop(rdt_handle* h, const void* h0, const void* e, int T, float* 
     }
     if (!h->cap_stream) RDT_CUDA_TRY(cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking));
     const int64_t l0 = h->launches;
+    h->graph_pending.clear();
     RDT_CUDA_TRY(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal));
+    h->capturing = true;
     const rdt_status s = loop_impl(h, h0, e, T, out, act, n_loops, h->cap_stream);
+    h->capturing = false;
     cudaGraph_t g = nullptr;
     const cudaError_t ce = cudaStreamEndCapture(h->cap_stream, &g);
     if (s != RDT_OK) {
@@ -1088,6 +1109,7 @@ rdt_status run_loop(rdt_handle* h, const void* h0, const void* e, int T, float* 
     h->gkey = key;
     RDT_CUDA_TRY(cudaGraphLaunch(h->gexec, st));
     h->launches += h->g_launches;
+    h->graph_ran = true;
     return RDT_OK;
 }
 
@@ -1417,15 +1439,23 @@ rdt_status rdt_profile(rdt_handle* h, int enable) {
         set_error("handle is NULL");
         return RDT_ERR_INVALID_ARG;
     }
+    if (enable < 0 || enable > 2) {
+        set_error("enable must be 0, 1 or 2");
+        return RDT_ERR_INVALID_ARG;
+    }
     if (enable) {
         RDT_CUDA_TRY(cudaStreamSynchronize(h->last_stream));
         h->pending.clear();
         h->ev_used = 0;
+        h->graph_ran = false;
         std::fill(h->prof_ms.begin(), h->prof_ms.end(), 0.0);
         std::fill(h->prof_n.begin(), h->prof_n.end(), 0);
+        if (h->prof_on && h->prof_graph == (enable == 2)) return RDT_OK;   // statistics restarted
     }
     h->prof_on = enable != 0;
+    h->prof_graph = enable == 2;
     drop_graph(h);
+    h->graph_pending.clear();
     return RDT_OK;
 }
 
@@ -1466,6 +1496,7 @@ void rdt_destroy(rdt_handle* h) {
     if (!h) return;
     cudaDeviceSynchronize();
     for (cudaEvent_t ev : h->ev_pool) cudaEventDestroy(ev);
+    for (cudaEvent_t ev : h->graph_events) cudaEventDestroy(ev);
     if (h->gexec) cudaGraphExecDestroy(h->gexec);
     if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
     for (void* p : h->allocs) cudaFree(p);

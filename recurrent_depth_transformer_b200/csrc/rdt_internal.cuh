@@ -484,9 +484,6 @@ struct Norm1Args {
     const float* gamma;
     void* xn;          // [N, dim] cfg dtype
     int ntok, dim; float eps;
-    const void* lora_a;   // [r, dim] adapter down-projection or NULL
-    int lora_r;
-    void* lora_t;         // [N, 64] cfg dtype, columns [0, r) written
     int* zero_counts; int n_zero;   // counts to clear (next MoE), or NULL
     // loop mode: also write the fp32 block input x into y0 and A (.) h + Be into hn0, which
     // the O projection then completes with its output a (NULL: not written)
@@ -536,8 +533,6 @@ rdt_status moe_copy(bool bf16_elems, void* xperm, const int* slot_row, int ntok,
 rdt_status moe_combine(const float* rows, const int* slot_row, int ntok, int top_k, int n_shared, int cap,
                        float* dst, int dim, cudaStream_t st);
 
-rdt_status lora_down(bool bf16_elems, const void* x, int ldx, int ntok, int width,
-                     const void* lora_a, int r, void* t_out, cudaStream_t st);
 
 rdt_status hoist(bool bf16_elems, const void* h0, const void* e, const float* Bdiag, float* h,
                  float* Be, size_t n, int dim, cudaStream_t st);
@@ -569,10 +564,12 @@ struct ActArgs {
 };
 rdt_status act_step(const ActArgs& a, cudaStream_t st);
 
-// Weight preparation: C[m, n] = sum_k A(m, k) B(k, n) with A(m, k) = A[m*sam + k*sak] and
-// B(k, n) = B[k*sbk + n*sbn] (element type of the configuration), fp32 sums.
+// Weight preparation: C[m, n] = add[m, n] + sum_k A(m, k) B(k, n) with A(m, k) = A[m*sam + k*sak]
+// and B(k, n) = B[k*sbk + n*sbn] (element type of the configuration; add [M, ld_add] or NULL),
+// fp32 sums rounded once.
 rdt_status prep_matmul(bool bf16_elems, const void* A, long sam, long sak, const void* B, long sbk,
-                       long sbn, void* C, int ldc, int M, int N, int K, cudaStream_t st);
+                       long sbn, void* C, int ldc, int M, int N, int K, cudaStream_t st,
+                       const void* add = nullptr, int ld_add = 0);
 rdt_status check_finite(const float* x, size_t n, int* flags, cudaStream_t st);
 
 }  // namespace rdt

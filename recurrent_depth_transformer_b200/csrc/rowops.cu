@@ -1,14 +1,14 @@
 // Memory-bound row kernels of the recurrent block (one warp per token row, 16-byte
 // vectorised, coalesced across the warp):
 //   hoist          h <- h0 (fp32 state), Be <- B (.) e      (once per call)
-//   norm1          x = h + e, xn = RMSNorm1(x), optional LoRA-down t = xn A_t^T
+//   norm1          x = h + e, xn = RMSNorm1(x); in the loop also y <- x, h_next <- A h + B e
 //   norm2_router   yn = RMSNorm2(y) (fp32 in registers, stored in the element type for the
 //                  experts), router logits yn W_r^T in fp32, top-k of logits + bias with
 //                  ties to the lower expert index, softmax over the k chosen logits,
 //                  per-expert histogram
 //   moe_copy       the copy of each token's normalised row into the expert rows its
 //                  router claimed (capacity layout), for routers that do not write them
-//   lora_down      t = x A^T for the O-projection adapter
+//   moe_combine    deterministic mode: a token's expert-row outputs added in a fixed order
 //   mla_latent_norm  RMSNorm of c_q and c_kv, RoPE of the decoupled key
 //   act_step       ACT halting after a loop: halting probability of the new state,
 //                  the halting decision, the weighted output sum, frozen halted states
@@ -144,23 +144,6 @@ __global__ void __launch_bounds__(kRowThreads, NV <= 8 ? 2 : 1) norm1_kernel(con
 #pragma unroll
         for (int j = 0; j < 4; ++j) x[i][j] = to_f(from_f<T>(x[i][j] * inv * gi[j]));
         store4(xn + col, x[i]);
-    }
-    if (a.lora_a) {
-        const T* A = static_cast<const T*>(a.lora_a);
-        T* t = static_cast<T*>(a.lora_t) + static_cast<size_t>(row) * (128 / sizeof(T));
-#pragma unroll 1
-        for (int r = 0; r < a.lora_r; ++r) {
-            float p = 0.0f;
-#pragma unroll
-            for (int i = 0; i < NV; ++i) {
-                float w[4];
-                load4(A + static_cast<size_t>(r) * a.dim + i * 128 + lane * 4, w);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) p = fmaf(x[i][j], w[j], p);
-            }
-            p = warp_sum(p);
-            if (lane == 0) store_t(t + r, p);
-        }
     }
 }
 
@@ -404,36 +387,6 @@ __global__ void __launch_bounds__(kRowThreads) moe_combine_kernel(const float* r
     for (int i = 0; i < NV; ++i) store4(d + i * 128 + lane * 4, acc[i]);
 }
 
-// ----------------------------------------------------------------------------- LoRA down
-
-template <typename T, int NV>
-__global__ void __launch_bounds__(kRowThreads) lora_down_kernel(const T* x, int ldx, int ntok,
-                                                                const T* A, int r, T* t) {
-    pdl_trigger();
-    pdl_wait();
-    const int row = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= ntok) return;
-    const int width = NV * 128;
-    float v[NV][4];
-#pragma unroll
-    for (int i = 0; i < NV; ++i) load4(x + static_cast<size_t>(row) * ldx + i * 128 + lane * 4, v[i]);
-    T* out = t + static_cast<size_t>(row) * (128 / sizeof(T));
-#pragma unroll 1
-    for (int j = 0; j < r; ++j) {
-        float p = 0.0f;
-#pragma unroll
-        for (int i = 0; i < NV; ++i) {
-            float w[4];
-            load4(A + static_cast<size_t>(j) * width + i * 128 + lane * 4, w);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) p = fmaf(v[i][q], w[q], p);
-        }
-        p = warp_sum(p);
-        if (lane == 0) store_t(out + j, p);
-    }
-}
-
 // ----------------------------------------------------------------------------- MLA latents
 
 template <typename T>
@@ -475,11 +428,11 @@ __global__ void __launch_bounds__(kRowThreads) mla_latent_norm_kernel(const MlaN
 
 template <typename T>
 __global__ void prep_matmul_kernel(const T* A, long sam, long sak, const T* B, long sbk, long sbn,
-                                   T* C, int ldc, int M, int N, int K) {
+                                   T* C, int ldc, int M, int N, int K, const T* add, int ld_add) {
     const int m = blockIdx.y * blockDim.y + threadIdx.y;
     const int n = blockIdx.x * blockDim.x + threadIdx.x;
     if (m >= M || n >= N) return;
-    float acc = 0.0f;
+    float acc = add ? to_f(add[static_cast<size_t>(m) * ld_add + n]) : 0.0f;
     for (int k = 0; k < K; ++k) acc = fmaf(to_f(A[m * sam + k * sak]), to_f(B[k * sbk + n * sbn]), acc);
     C[static_cast<size_t>(m) * ldc + n] = from_f<T>(acc);
 }
@@ -571,14 +524,6 @@ struct Norm1L {
     }
 };
 template <typename T, int NV>
-struct LoraL {
-    static void run(dim3 g, cudaStream_t st, const void* x, int ldx, int ntok, const void* A,
-                    int r, void* t) {
-        launch_pdl(lora_down_kernel<T, NV>, g, dim3(kRowThreads), 0, st, static_cast<const T*>(x), ldx,
-                   ntok, static_cast<const T*>(A), r, static_cast<T*>(t));
-    }
-};
-template <typename T, int NV>
 struct ActL {
     static void run(dim3 g, cudaStream_t st, ActArgs a) {
         launch_pdl(act_step_kernel<NV>, g, dim3(kRowThreads), 0, st, a);
@@ -643,13 +588,6 @@ rdt_status norm1(bool bf, const Norm1Args& a, cudaStream_t st) {
               : launch_rows<float, Norm1L>(nv, a.ntok, st, a);
 }
 
-rdt_status lora_down(bool bf, const void* x, int ldx, int ntok, int width, const void* A, int r,
-                     void* t, cudaStream_t st) {
-    const int nv = width / 128;
-    return bf ? launch_rows<bf16, LoraL>(nv, ntok, st, x, ldx, ntok, A, r, t)
-              : launch_rows<float, LoraL>(nv, ntok, st, x, ldx, ntok, A, r, t);
-}
-
 rdt_status norm2_split(bool bf, const Norm2Args& a, cudaStream_t st) {
     const int nv = a.dim / 128;
     return bf ? launch_rows<bf16, Norm2L>(nv, a.ntok, st, a)
@@ -692,16 +630,19 @@ rdt_status moe_combine(const float* rows, const int* slot_row, int ntok, int top
 }
 
 rdt_status prep_matmul(bool bf, const void* A, long sam, long sak, const void* B, long sbk,
-                       long sbn, void* C, int ldc, int M, int N, int K, cudaStream_t st) {
+                       long sbn, void* C, int ldc, int M, int N, int K, cudaStream_t st, const void* add,
+                       int ld_add) {
     const dim3 blk(32, 8), grid((N + 31) / 32, (M + 7) / 8);
     if (bf)
         prep_matmul_kernel<bf16><<<grid, blk, 0, st>>>(static_cast<const bf16*>(A), sam, sak,
                                                        static_cast<const bf16*>(B), sbk, sbn,
-                                                       static_cast<bf16*>(C), ldc, M, N, K);
+                                                       static_cast<bf16*>(C), ldc, M, N, K,
+                                                       static_cast<const bf16*>(add), ld_add);
     else
         prep_matmul_kernel<float><<<grid, blk, 0, st>>>(static_cast<const float*>(A), sam, sak,
                                                         static_cast<const float*>(B), sbk, sbn,
-                                                        static_cast<float*>(C), ldc, M, N, K);
+                                                        static_cast<float*>(C), ldc, M, N, K,
+                                                        static_cast<const float*>(add), ld_add);
     RDT_CUDA_TRY(cudaGetLastError());
     return RDT_OK;
 }

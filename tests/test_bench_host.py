@@ -15,14 +15,51 @@ from workloads import WORKLOADS, by_name
 
 def test_algorithmic_flops_of_the_bench_workload():
     wl = by_name(bench.WORKLOAD)
-    assert wl is WORKLOADS[1]
+    assert wl is WORKLOADS[4] and bench.LOOPS == 16     # the largest configuration is the headline
     per_loop = bench.step_flops(wl, 1)
-    # 2N d (Hq+2Hkv) dh + 2N Hq dh d + 4 B Hq dh S(S+1)/2 + 2N d E + 6 d hid N k
-    N, d = 2048, 1024
-    want = (2 * N * d * 1536 + 2 * N * 1024 * d + 4 * 4 * 16 * 64 * 512 * 513 / 2
-            + 2 * N * d * 16 + 6 * d * 1024 * N * 2)
+    # 2N d (Hq+2Hkv) dh + 2N Hq dh d + LoRA 2N r (d + Hq dh) x 2 + 4 B Hq dh S(S+1)/2
+    #   + 2N d E + 6 d hid N k
+    N, d, S = 8192, 2048, 8192
+    want = (2 * N * d * 3072 + 2 * N * 2048 * d + 2 * 2 * N * 16 * (d + 2048) + 4 * 32 * 64 * S * (S + 1) / 2
+            + 2 * N * d * 64 + 6 * d * 512 * N * 8)
     assert per_loop == pytest.approx(want)
-    assert per_loop == pytest.approx(38.7e9, rel=0.01)
+    assert per_loop == pytest.approx(863.3e9, rel=0.001)
+    # the GQA configuration: 38.7 GFLOP per loop
+    assert bench.step_flops(WORKLOADS[1], 1) == pytest.approx(38.7e9, rel=0.01)
+    # absorbed MLA: latent 2N d (ql + kvl + r), q~ 2N ql H (kvl + r), attention 2 H (2 kvl + r) pairs,
+    # O 2N H kvl d, experts as GQA, router
+    m = WORKLOADS[2]
+    N, d = 2048, 1024
+    pairs = 4 * 512 * 513 / 2
+    want = (2 * N * d * 544 + 2 * N * 384 * 16 * 160 + 2 * 16 * 288 * pairs + 2 * N * 2048 * d
+            + 6 * d * 1024 * N * 2 + 2 * N * d * 16)
+    assert bench.step_flops(m, 1) == pytest.approx(want)
+
+
+def test_replica_plan_gives_each_rank_its_own_inputs():
+    wl = WORKLOADS[4]
+    seeds = [bench.replica_plan(wl, r, 4)[0] for r in range(4)]
+    assert len(set(seeds)) == 4 and seeds[0] == wl.seed
+    assert all(bench.replica_plan(wl, r, 4)[1] == wl.batch * wl.seq for r in range(4))
+    with pytest.raises(ValueError):
+        bench.replica_plan(wl, 4, 4)
+
+
+def test_launch_ranks_runs_torchrun_with_one_process_per_gpu(monkeypatch):
+    seen = {}
+    monkeypatch.setattr(bench.subprocess, "call", lambda cmd: seen.setdefault("cmd", cmd) and 0)
+    bench.launch_ranks(["--gpus", "4", "--steps", "3"], 4)
+    cmd = seen["cmd"]
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--master-addr=127.0.0.1" in cmd
+    assert cmd[-3:] == ["--gpus", "4", "--steps", "3"][-3:]
+
+
+def test_oracle_sample_is_bounded():
+    # the long configuration: one loop of the whole sequence fits the CPU budget's estimate
+    # only for the baseline sample; the reference arm's per-step sample is a prefix
+    assert bench.oracle_sample_plan(WORKLOADS[1]) == 512
+    assert bench.oracle_sample_plan(WORKLOADS[4], budget_s=4.0) < 8192
 
 
 def test_parse_clocks():
@@ -57,12 +94,14 @@ def _free_port():
 def _rank_main(rank, world, port, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
-    dist.init_process_group("gloo", rank=rank, world_size=world)
-    assert bench.dist_env() == (rank, rank, world)
+    assert bench.init_ranks(backend="gloo", timeout_s=60) == (rank, rank, world)
+    assert dist.get_world_size() == world
+    wl = WORKLOADS[1]
+    seed, tokens = bench.replica_plan(wl, rank, world)
     m = bench.reduce_max(1.5 + rank, device="cpu")
-    v, ms = bench.aggregate([m], 1000, 4, world)
-    q.put((rank, m, v))
-    dist.barrier()
+    v, ms = bench.aggregate([m], tokens, 4, world)
+    q.put((rank, m, v, seed))
+    bench.barrier()
     dist.destroy_process_group()
 
 
@@ -77,8 +116,9 @@ def test_two_ranks_take_the_max_over_ranks():
         p.join(120)
         assert p.exitcode == 0
     res = sorted(q.get(timeout=10) for _ in range(2))
-    assert [r[1] for r in res] == [2.5, 2.5]
-    assert res[0][2] == pytest.approx(2 * 1000 * 4 / 0.0025)
+    assert [r[1] for r in res] == [2.5, 2.5]                       # the slowest rank's time
+    assert res[0][2] == pytest.approx(2 * 2048 * 4 / 0.0025)        # both ranks' tokens
+    assert res[0][3] != res[1][3]                                   # each rank its own inputs
 
 
 def test_reference_arm_prints_one_json_line(capsys):
@@ -93,11 +133,13 @@ def test_reference_arm_prints_one_json_line(capsys):
 def test_measured_traffic_only_for_unchanged_sources(monkeypatch):
     files = bench.KERNEL_SOURCES["gemm_up"]
     fp = bench.source_fingerprint(files)
-    monkeypatch.setitem(bench.MEASURED_TRAFFIC, "gemm_up", (123.0, fp))
-    assert bench.measured_traffic("gemm_up") == 123.0
-    monkeypatch.setitem(bench.MEASURED_TRAFFIC, "gemm_up", (123.0, "0" * 16))
-    assert bench.measured_traffic("gemm_up") is None          # sources changed since the capture
-    assert bench.measured_traffic("attention") is None        # never captured
+    key = (bench.WORKLOAD, "gemm_up")
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, key, (123.0, fp))
+    assert bench.measured_traffic(bench.WORKLOAD, "gemm_up") == 123.0
+    assert bench.measured_traffic("other-workload", "gemm_up") is None   # captured on another workload
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, key, (123.0, "0" * 16))
+    assert bench.measured_traffic(bench.WORKLOAD, "gemm_up") is None     # sources changed since
+    assert bench.measured_traffic(bench.WORKLOAD, "norm1") is None       # never captured
 
 
 def test_fingerprint_ignores_comments_not_code(tmp_path):
@@ -117,31 +159,22 @@ def test_fingerprint_ignores_comments_not_code(tmp_path):
 
 
 
-def test_act_line_reports_halting_histogram(capsys):
-    """The --act leg's JSON line, from a stand-in handle (no GPU): the workload, the
-    halting histogram, the mean loops and the kernel shares."""
-    import argparse
+def test_act_summary_reports_the_halting_histogram():
+    nl = [[1, 2, 2, 8], [8, 8, 3, 1]]
+    a = bench.act_summary(nl, 8)
+    assert a["hist"] == [2, 2, 1, 0, 0, 0, 0, 3]
+    assert a["mean_loops"] == pytest.approx(33 / 8)
+    assert a["loops_run_fraction"] == pytest.approx(33 / 64)
 
-    class FakeHandle:
-        closed = False
 
-        def diagnostics(self):
-            return {"nonfinite": 0, "timeout": 0}
-
-        def close(self):
-            self.closed = True
-
+def test_roofline_of_a_tensor_and_an_hbm_kernel():
     wl = by_name(bench.WORKLOAD)
-    nl = torch.tensor([[1, 2, 2, 8], [8, 8, 3, 1]], dtype=torch.int32)
-    args = argparse.Namespace(steps=10, warmup=3)
-    stats = {"gemm_up": (80, 3.0), "act_halting": (80, 1.0)}
-    h = FakeHandle()
-    assert bench.act_line(args, h, wl, nl, 2.0e7, 0.82, 1, 0, stats, 1234, None) == 0
-    line = json.loads(capsys.readouterr().out.strip())
-    assert h.closed
-    assert line["impl"] == "ours+act" and line["config"]["workload"].endswith("+act")
-    assert line["act"]["hist"] == [2, 2, 1, 0, 0, 0, 0, 3]
-    assert line["act"]["mean_loops"] == pytest.approx(33 / 8)
-    assert line["act"]["loops_run_fraction"] == pytest.approx(33 / 64)
-    assert line["kernels"]["gemm_up"]["share"] == pytest.approx(0.75)
-    assert line["gpu_launches"] == 1234 and line["finite"] is True
+    work = bench.kernel_work(wl)
+    peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}
+    r = bench.roofline_of("attention", 16, 16 * 0.5, work, peaks, "measured", bench.WORKLOAD)
+    assert r["bound"] == "tensor" and r["avg_launch_us"] == pytest.approx(500.0)
+    assert r["achieved"] == pytest.approx(274.9e9 / 500e-6 / 1e12, rel=1e-3)
+    assert r["frac"] == pytest.approx(r["achieved"] / 1000.0)
+    r = bench.roofline_of("norm1", 2, 0.1, work, peaks, "measured", bench.WORKLOAD)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(8192 * 2048 * 20 / 50e-6 / 1e9)
