@@ -94,6 +94,11 @@ typedef struct {
                                      * atomics. Costs N * top_k * dim * 8 bytes of extra
                                      * traffic per loop. 0: reductions by fp32 atomics,
                                      * whose order (and so the last bits) may vary.      */
+    int32_t max_decode;             /* > 0: a per-loop KV cache of seq + max_decode positions
+                                     * per sequence for rdt_decode_prefill / _step (bf16
+                                     * only): max_loops * batch * (seq + max_decode) rows of
+                                     * 2 n_kv_heads head_dim (GQA) or kv_lora_rank +
+                                     * qk_rope_dim (MLA) elements. 0: no cache.         */
 } rdt_config;
 
 /* Weights, all DEVICE pointers, row-major [out, in]; element type = cfg.dtype
@@ -186,6 +191,28 @@ rdt_status rdt_loop_forward(rdt_handle* h, const void* h0, const void* e, int T,
  * host memory gives asynchronous copies; pageable memory also works. */
 rdt_status rdt_loop_forward_host(rdt_handle* h, const void* h0_host, const void* e_host, int T,
                                  float* out_host, void* stream);
+
+/* Decode with a per-loop KV cache (getting-started page "Introducao ao OpenMythos", Passo 4:
+ * the prompt is run once, then one token per call; troubleshooting item 1: every loop keeps
+ * the keys and values of all tokens; Passo 5: MLA caches its compressed latent and rebuilds
+ * K and V from it). Loop t of a new token attends over the keys and values that loop t
+ * produced for the earlier positions and for itself. GQA caches its rotated keys and its
+ * values; MLA its normalised latent and rotated shared key. Needs cfg.max_decode > 0.
+ *
+ * rdt_decode_prefill runs the loop over the prompt (h0, e: device [batch, seq, dim] in
+ * cfg.dtype; out: device fp32 [batch, seq, dim] = h_T) exactly as rdt_loop_forward and fills
+ * the cache of loops 0 .. T - 1 with positions 0 .. seq - 1 (a new prefill starts over).
+ * rdt_decode_step runs T loops (T must be the prefill's) for one new token per sequence at
+ * the next position (h0, e: device [batch, dim] in cfg.dtype; out: device fp32 [batch, dim]
+ * = h_T of the new tokens) and appends it to every loop's cache. INVALID_ARG without a
+ * prefill, for another T or when the cache is full (seq + max_decode positions). The
+ * position advances on the device, so a step's launch sequence replays as one CUDA graph.
+ * A trace set by rdt_set_trace records a step's loops in its first batch rows: loop t's
+ * routing at offset t * batch * seq * top_k, its states packed as [T + 1, batch, dim]. */
+rdt_status rdt_decode_prefill(rdt_handle* h, const void* h0, const void* e, int T, float* out,
+                              void* stream);
+rdt_status rdt_decode_step(rdt_handle* h, const void* h0, const void* e, int T, float* out,
+                           void* stream);
 
 /* ACT halting ("Dynamic Adaptive Computation Time" halting, techbriefly article on
  * the OpenMythos project; act_threshold = 0.99, getting-started page

@@ -602,7 +602,7 @@ def attention_cached(x, W, cfg, t: int, cache: LoopKVCache) -> np.ndarray:
     return out_proj(o, W, cfg, t)
 
 
-def _loop_cached(h0, e, T: int, W, cfg, cache: LoopKVCache) -> np.ndarray:
+def _loop_cached(h0, e, T: int, W, cfg, cache: LoopKVCache, follow=None, stats=None) -> np.ndarray:
     A = _f(W["A"])
     e = _f(e)
     Be = input_injection(e, W["B"])
@@ -611,21 +611,27 @@ def _loop_cached(h0, e, T: int, W, cfg, cache: LoopKVCache) -> np.ndarray:
         x = h + e if cfg.inject_e else h
         a = attention_cached(x, W, cfg, t, cache)
         y = x + a
-        f, _, _ = moe_sublayer(y, W, cfg)
+        f, _, st = moe_sublayer(y, W, cfg, None if follow is None else follow[t])
+        if stats is not None:
+            for k in st:
+                stats[k] = stats.get(k, 0) + st[k]
         h = A * h + Be + a + f
     cache.length += h.shape[1]
     return h
 
 
-def loop_prefill(h0, e, T: int, W, cfg) -> Tuple[np.ndarray, LoopKVCache]:
+def loop_prefill(h0, e, T: int, W, cfg, follow=None, stats=None) -> Tuple[np.ndarray, LoopKVCache]:
     """The loop over a whole prompt [B, S, d] ([GS] Passo 4, first call): h_T and the
-    cache of every loop's keys and values for positions 0..S-1."""
+    cache of every loop's keys and values for positions 0..S-1. ``follow[t]`` ([B*S, k])
+    is another implementation's routing, adopted on near-ties as in :func:`moe_sublayer`;
+    ``stats`` (a dict) collects the counts."""
     cache = LoopKVCache()
-    h = _loop_cached(h0, e, T, W, cfg, cache)
+    h = _loop_cached(h0, e, T, W, cfg, cache, follow, stats)
     return h, cache
 
 
-def loop_decode(h0, e, T: int, W, cfg, cache: LoopKVCache) -> np.ndarray:
+def loop_decode(h0, e, T: int, W, cfg, cache: LoopKVCache, follow=None, stats=None) -> np.ndarray:
     """T loops for new tokens h0, e [B, Sn, d] (Sn = 1 in a decode step) at positions
-    cache.length .., each loop t attending over loop t's cache; extends the cache."""
-    return _loop_cached(h0, e, T, W, cfg, cache)
+    cache.length .., each loop t attending over loop t's cache; extends the cache.
+    ``follow`` and ``stats`` as in :func:`loop_prefill`."""
+    return _loop_cached(h0, e, T, W, cfg, cache, follow, stats)

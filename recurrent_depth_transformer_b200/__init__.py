@@ -37,7 +37,8 @@ EXPORTED = ("rdt_create", "rdt_attn_forward", "rdt_moe_forward", "rdt_loop_forwa
             "rdt_loop_forward_host", "rdt_set_trace", "rdt_get_diagnostics", "rdt_memory_bytes",
             "rdt_status_string", "rdt_last_error", "rdt_destroy", "rdt_matmul", "rdt_attention",
             "rdt_profile", "rdt_profile_read", "rdt_moe_route_noalloc", "rdt_moe_route_noalloc_status",
-            "rdt_set_act", "rdt_loop_forward_act", "rdt_wait_probe")
+            "rdt_set_act", "rdt_loop_forward_act", "rdt_wait_probe", "rdt_decode_prefill",
+            "rdt_decode_step")
 
 
 class RdtError(RuntimeError):
@@ -53,7 +54,7 @@ class RdtConfig(ctypes.Structure):
         ("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float)] + [
         (n, ctypes.c_int32) for n in ("n_experts", "top_k", "n_shared", "expert_hidden",
                                       "lora_rank", "n_lora", "b_kind", "inject_e", "max_loops",
-                                      "gemm_tiles", "deterministic")]
+                                      "gemm_tiles", "deterministic", "max_decode")]
 
 
 WEIGHT_FIELDS = ("A", "B", "norm1", "norm2", "wq", "wk", "wv", "wo", "w_dq", "q_norm", "w_uq",
@@ -110,6 +111,8 @@ def load_library() -> ctypes.CDLL:
                                           vp, vp, vp, vp]
     lib.rdt_moe_route_noalloc_status.argtypes = [vp]
     lib.rdt_wait_probe.argtypes = [ctypes.c_int64, vp]
+    lib.rdt_decode_prefill.argtypes = [vp, vp, vp, i32, vp, vp]
+    lib.rdt_decode_step.argtypes = [vp, vp, vp, i32, vp, vp]
     lib.rdt_profile.argtypes = [vp, i32]
     lib.rdt_profile_read.argtypes = [vp, ctypes.POINTER(RdtKernelStat), i32, ctypes.POINTER(i32),
                                      ctypes.POINTER(ctypes.c_int64)]
@@ -118,7 +121,8 @@ def load_library() -> ctypes.CDLL:
     for f in ("rdt_create", "rdt_attn_forward", "rdt_moe_forward", "rdt_loop_forward",
               "rdt_loop_forward_host", "rdt_set_trace", "rdt_get_diagnostics", "rdt_memory_bytes",
               "rdt_matmul", "rdt_attention", "rdt_profile", "rdt_profile_read", "rdt_moe_route_noalloc",
-              "rdt_set_act", "rdt_loop_forward_act", "rdt_moe_route_noalloc_status", "rdt_wait_probe"):
+              "rdt_set_act", "rdt_loop_forward_act", "rdt_moe_route_noalloc_status", "rdt_wait_probe",
+              "rdt_decode_prefill", "rdt_decode_step"):
         getattr(lib, f).restype = i32
     _LIB = lib
     return lib
@@ -131,7 +135,7 @@ def _check(status: int) -> None:
 
 
 def make_config(wl, max_loops: int = 16, batch: Optional[int] = None, seq: Optional[int] = None,
-                gemm_tiles: int = 0, deterministic: bool = False) -> RdtConfig:
+                gemm_tiles: int = 0, deterministic: bool = False, max_decode: int = 0) -> RdtConfig:
     """Fill the C config from any object with the block's hyper-parameters as attributes."""
     c = RdtConfig()
     c.dtype = RDT_BF16 if wl.dtype == "bf16" else RDT_F32
@@ -160,6 +164,7 @@ def make_config(wl, max_loops: int = 16, batch: Optional[int] = None, seq: Optio
     c.max_loops = max_loops
     c.gemm_tiles = gemm_tiles
     c.deterministic = 1 if deterministic else 0
+    c.max_decode = max_decode
     return c
 
 
@@ -247,6 +252,22 @@ class RDT:
         if out is None:
             out = torch.empty(e.shape, dtype=torch.float32, device=e.device)
         _check(self._lib.rdt_loop_forward(self._h, _ptr(h0), _ptr(e), T, _ptr(out), _stream(stream)))
+        return out
+
+    def decode_prefill(self, h0, e, T: int, out=None, stream=None):
+        """The loop over the prompt [batch, seq, dim], filling every loop's KV cache."""
+        import torch
+        if out is None:
+            out = torch.empty(e.shape, dtype=torch.float32, device=e.device)
+        _check(self._lib.rdt_decode_prefill(self._h, _ptr(h0), _ptr(e), T, _ptr(out), _stream(stream)))
+        return out
+
+    def decode_step(self, h0, e, T: int, out=None, stream=None):
+        """T loops for one new token per sequence (h0, e [batch, dim]); appends to the caches."""
+        import torch
+        if out is None:
+            out = torch.empty(e.shape, dtype=torch.float32, device=e.device)
+        _check(self._lib.rdt_decode_step(self._h, _ptr(h0), _ptr(e), T, _ptr(out), _stream(stream)))
         return out
 
     def set_act(self, w_halt, b_halt: float, threshold: float = 0.99, stream=None):

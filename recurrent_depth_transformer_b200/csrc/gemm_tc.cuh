@@ -271,12 +271,12 @@ __device__ __forceinline__ void epilogue_pre(const EpiParams& p, int lane, int n
     if constexpr (KIND == EPI_ROPE) {
         // The angle tables are [rot/2][seq]: for a fixed frequency the lanes (consecutive
         // positions) read consecutive floats.
-        const int pos = (row0 + lane) % p.seq;
+        const int pos = (row0 + lane) % p.seq + (p.pos_dev ? *p.pos_dev : 0);
         const int half = p.rot_dim / 2;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            pre.cs[i] = i < half ? p.rope_cos[static_cast<size_t>(i) * p.seq + pos] : 0.0f;
-            pre.sn[i] = i < half ? p.rope_sin[static_cast<size_t>(i) * p.seq + pos] : 0.0f;
+            pre.cs[i] = i < half ? p.rope_cos[static_cast<size_t>(i) * p.rope_ld + pos] : 0.0f;
+            pre.sn[i] = i < half ? p.rope_sin[static_cast<size_t>(i) * p.rope_ld + pos] : 0.0f;
         }
     } else if constexpr (KIND == EPI_SCATTER) {
         // Row r of the tile is expert output for token row_token[r] with gate weight row_w[r]

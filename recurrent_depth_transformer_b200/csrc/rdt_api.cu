@@ -78,6 +78,16 @@ struct rdt_handle {
     int max_tiles_pair = 0;        // ... and on 256-row tiles
     int* flags = nullptr;
     float* det_rows = nullptr;     // deterministic mode: [cap * (S + E), dim] expert row outputs
+    // decode with a per-loop KV cache (cfg.max_decode > 0): [max_loops][batch][s_cap][cache_w]
+    int s_cap = 0;                 // positions a sequence may reach (seq + max_decode); RoPE rows
+    int cache_w = 0;               // GQA: [K | V] = 2 n_kv_heads head_dim; MLA: kv_lat + rope
+    void* kv_cache = nullptr;
+    int* dec_len = nullptr;        // device: cached positions (the new token's position in a step)
+    float* dec_part = nullptr;     // split decode attention partials
+    int dec_T = 0;                 // loops of the prefill (decode steps run the same number)
+    int dec_len_host = 0;          // the same length, tracked on the host for validation
+    int mode = 0;                  // 0 plain loop, 1 prefill (fills the cache), 2 decode step
+    int cur_ntok = 0;              // tokens of the current call (batch in a decode step)
     void *stage_h0 = nullptr, *stage_e = nullptr;
     float* stage_out = nullptr;
 
@@ -114,8 +124,10 @@ struct rdt_handle {
         int T = 0;
         bool act = false;
         const int32_t* n_loops = nullptr;
+        int mode = 0;
         bool operator==(const GraphKey& o) const {
-            return h0 == o.h0 && e == o.e && out == o.out && T == o.T && act == o.act && n_loops == o.n_loops;
+            return h0 == o.h0 && e == o.e && out == o.out && T == o.T && act == o.act && n_loops == o.n_loops &&
+                   mode == o.mode;
         }
     };
     cudaStream_t cap_stream = nullptr;
@@ -138,11 +150,12 @@ constexpr int kFillerRows = 256;
 // kernel classes reported by rdt_profile_read
 enum Kind { K_HOIST, K_NORM1, K_GEMM_QKV, K_GEMM_LAT, K_MLA_NORM, K_GEMM_Q, K_ATTENTION,
             K_GEMM_O, K_NORM2, K_ROUTER, K_DISPATCH, K_GEMM_UP, K_GEMM_DOWN, K_CHECK, K_DENSE_B, K_ACT,
-            K_COMBINE, K_COUNT };
+            K_COMBINE, K_CACHE, K_DEC_ATTN, K_COUNT };
 const char* const kKindName[K_COUNT] = {"hoist", "norm1", "gemm_qkv", "gemm_latent", "mla_latent_norm",
                                          "gemm_q_absorbed", "attention", "gemm_o",
                                          "norm2", "router_topk", "moe_dispatch", "gemm_up", "gemm_down",
-                                         "check_finite", "dense_injection", "act_halting", "moe_combine"};
+                                         "check_finite", "dense_injection", "act_halting", "moe_combine", "kv_cache_append",
+                                         "decode_attention"};
 
 // During graph capture the events become event-record nodes of the graph (external
 // records), so that every replay records them again; they are then kept apart from the
@@ -260,6 +273,9 @@ rdt_status validate_config(const rdt_config* c) {
     if (c->max_loops < 1 || c->max_loops > 64) return bad("max_loops must be in [1, 64]");
     if (c->gemm_tiles < 0 || c->gemm_tiles > 2) return bad("gemm_tiles must be 0, 1 or 2");
     if (c->deterministic != 0 && c->deterministic != 1) return bad("deterministic must be 0 or 1");
+    if (c->max_decode < 0 || c->max_decode > (1 << 20)) return bad("max_decode");
+    if (c->max_decode > 0 && c->dtype != RDT_BF16) return uns("decode with a KV cache is provided in bf16");
+    if (static_cast<long long>(c->seq) + c->max_decode > (1 << 24)) return uns("seq + max_decode too large");
     if (c->b_kind != RDT_B_DIAG && c->b_kind != RDT_B_DENSE) return bad("b_kind");
     if (!(c->norm_eps >= 0.0f) || !(c->rope_base > 1.0f)) return bad("norm_eps / rope_base");
     if (c->lora_rank < 0 || c->n_lora < 0) return bad("lora");
@@ -402,6 +418,7 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
     h->bf = c.dtype == RDT_BF16;
     h->esz = h->bf ? 2 : 4;
     h->ntok = c.batch * c.seq;
+    h->cur_ntok = h->ntok;
     h->G = c.n_experts + c.n_shared;
     h->prof_ms.assign(K_COUNT, 0.0);
     h->prof_n.assign(K_COUNT, 0);
@@ -604,16 +621,18 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         }
     }
 
-    // RoPE tables [rot/2][seq] (frequency-major, so that consecutive positions are adjacent)
-    // from double-precision angles
+    // RoPE tables [rot/2][s_cap] (frequency-major, so that consecutive positions are adjacent)
+    // from double-precision angles, for every position a sequence may reach
+    h->s_cap = c.seq + c.max_decode;
     {
         const int half = h->rot / 2;
-        std::vector<float> cs(static_cast<size_t>(c.seq) * half), sn(cs.size());
+        const int P = h->s_cap;
+        std::vector<float> cs(static_cast<size_t>(P) * half), sn(cs.size());
         for (int i = 0; i < half; ++i)
-            for (int p = 0; p < c.seq; ++p) {
+            for (int p = 0; p < P; ++p) {
                 const double ang = p * std::pow(static_cast<double>(c.rope_base), -2.0 * i / h->rot);
-                cs[static_cast<size_t>(i) * c.seq + p] = static_cast<float>(std::cos(ang));
-                sn[static_cast<size_t>(i) * c.seq + p] = static_cast<float>(std::sin(ang));
+                cs[static_cast<size_t>(i) * P + p] = static_cast<float>(std::cos(ang));
+                sn[static_cast<size_t>(i) * P + p] = static_cast<float>(std::sin(ang));
             }
         RDT_TRY(dev_alloc(h, &h->rope_cos, cs.size() * 4));
         RDT_TRY(dev_alloc(h, &h->rope_sin, sn.size() * 4));
@@ -675,6 +694,15 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
     RDT_TRY(dev_alloc(h, &h->flags, FLAG_COUNT * 4, true));
     if (c.deterministic)
         RDT_TRY(dev_alloc(h, &h->det_rows, static_cast<size_t>(h->cap) * (S + E) * d * 4));
+    if (c.max_decode > 0) {
+        h->cache_w = c.attn_type == RDT_GQA ? 2 * c.n_kv_heads * c.head_dim : c.kv_lora_rank + c.qk_rope_dim;
+        RDT_TRY(dev_alloc(h, &h->kv_cache,
+                          static_cast<size_t>(c.max_loops) * c.batch * h->s_cap * h->cache_w * es));
+        RDT_TRY(dev_alloc(h, &h->dec_len, 16, true));
+        const int dv = c.attn_type == RDT_GQA ? c.head_dim : c.kv_lora_rank;
+        RDT_TRY(dev_alloc(h, &h->dec_part, static_cast<size_t>(c.batch) * c.n_heads * decode_chunks(h->s_cap) *
+                                               (dv + 2) * 4));
+    }
     RDT_TRY(dev_alloc(h, &h->stage_h0, nd * es));
     RDT_TRY(dev_alloc(h, &h->stage_e, nd * es));
     RDT_TRY(dev_alloc(h, &h->stage_out, nd * 4));
@@ -690,9 +718,16 @@ int lora_index(const rdt_handle* h, int t) { return std::min(t, h->cfg.n_lora - 
 rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t, bool loop_mode,
                            float* a_out, float* h_next, cudaStream_t st) {
     const rdt_config& c = h->cfg;
-    const int N = h->ntok, d = c.dim;
+    const int N = h->cur_ntok, d = c.dim;
     const bool lora = c.n_lora > 0;
     const int li = lora ? lora_index(h, t) : 0;
+    const bool step = h->mode == 2;
+    // positions: a prompt row r sits at r % seq; a decode step's row b at the cached length
+    const int pos_seq = step ? 1 : c.seq;
+    const int* pos_dev = step ? h->dec_len : nullptr;
+    void* cache_t = h->mode ? static_cast<char*>(h->kv_cache) +
+                                  static_cast<size_t>(t) * c.batch * h->s_cap * h->cache_w * h->esz
+                            : nullptr;
 
     Norm1Args n1{};
     n1.h = hin;
@@ -735,12 +770,17 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         ep.ncols_valid = h->nqkv;
         ep.rope_cos = h->rope_cos;
         ep.rope_sin = h->rope_sin;
-        ep.seq = c.seq;
+        ep.seq = pos_seq;
+        ep.pos_dev = pos_dev;
+        ep.rope_ld = h->s_cap;
         ep.head_w = c.head_dim;
         ep.rot_off = 0;
         ep.rot_dim = c.head_dim;
         ep.rope_limit = h->nq + h->nkv;
         TIMED(h, K_GEMM_QKV, 1, st, gemm_tc(h->bf, h->bn_qkv, h->m_xn, h->m_wqkv[li], nullptr, nullptr, ga, ep, st));
+        if (cache_t)   // loop t's rotated keys and values of these positions: [K | V] per row
+            TIMED(h, K_CACHE, 1, st, cache_append(h->qkv, h->nqkv, h->nq, h->cache_w, cache_t, h->s_cap, pos_seq,
+                                                  pos_dev, N, st));
         at.q = h->qkv;
         at.ldq = h->nqkv;
         at.q_hstride = c.head_dim;
@@ -774,12 +814,17 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         mn.rope_cos = h->rope_cos;
         mn.rope_sin = h->rope_sin;
         mn.ntok = N;
-        mn.seq = c.seq;
+        mn.seq = pos_seq;
+        mn.pos_dev = pos_dev;
+        mn.rope_ld = h->s_cap;
         mn.q_lat = ql;
         mn.kv_lat = kvl;
         mn.rope = rp;
         mn.eps = c.norm_eps;
         TIMED(h, K_MLA_NORM, 1, st, mla_latent_norm(h->bf, mn, st));
+        if (cache_t)   // loop t's normalised latent and rotated shared key: [c_kv | k_rope] per row
+            TIMED(h, K_CACHE, 1, st, cache_append(h->kvlat, kvl + rp, 0, h->cache_w, cache_t, h->s_cap, pos_seq,
+                                                  pos_dev, N, st));
         // absorbed query projection with RoPE on the last rope columns of each head
         GemmArgs gq{};
         gq.M = N;
@@ -794,7 +839,9 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         eq.ncols_valid = h->qt_w;
         eq.rope_cos = h->rope_cos;
         eq.rope_sin = h->rope_sin;
-        eq.seq = c.seq;
+        eq.seq = pos_seq;
+        eq.pos_dev = pos_dev;
+        eq.rope_ld = h->s_cap;
         eq.head_w = kvl + rp;
         eq.rot_off = kvl;
         eq.rot_dim = rp;
@@ -815,7 +862,41 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         at.scale = 1.0f / std::sqrt(static_cast<float>(c.qk_nope_dim + rp));
     }
     at.flags = h->flags;
-    TIMED(h, K_ATTENTION, 1, st, attention(h->bf, at, st));
+    if (step) {
+        // one new query per sequence against loop t's cache (positions 0 .. length)
+        DecodeAttnArgs da{};
+        da.q = at.q;
+        da.q_ld = at.ldq;
+        da.q_hstride = at.q_hstride;
+        da.cache = cache_t;
+        da.cache_ld = h->cache_w;
+        da.s_cap = h->s_cap;
+        if (c.attn_type == RDT_GQA) {
+            da.k_col0 = 0;
+            da.k_hstride = c.head_dim;
+            da.v_col0 = h->nkv;
+            da.v_hstride = c.head_dim;
+        } else {          // the shared latent: keys the whole row, values its first kv_lat columns
+            da.k_col0 = 0;
+            da.k_hstride = 0;
+            da.v_col0 = 0;
+            da.v_hstride = 0;
+        }
+        da.batch = c.batch;
+        da.hq = c.n_heads;
+        da.hkv = at.hkv;
+        da.dqk = at.dqk;
+        da.dv = at.dv;
+        da.len_dev = h->dec_len;
+        da.scale = at.scale;
+        da.part = h->dec_part;
+        da.o = h->o;
+        da.ldo = h->owidth;
+        da.dv_out = at.dv;
+        TIMED(h, K_DEC_ATTN, 2, st, decode_attention(da, st));
+    } else {
+        TIMED(h, K_ATTENTION, 1, st, attention(h->bf, at, st));
+    }
 
     GemmArgs go{};
     go.M = N;
@@ -846,7 +927,8 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
 rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_out, float* w_out,
                      int32_t* tr_idx, float* tr_w, const int* halted, cudaStream_t st) {
     const rdt_config& c = h->cfg;
-    const int N = h->ntok, d = c.dim, hid = c.expert_hidden;
+    // N: tokens of this call; NL: the capacity layout's row base (expert rows start after it)
+    const int N = h->cur_ntok, NL = h->ntok, d = c.dim, hid = c.expert_hidden;
     int32_t* idx = idx_out ? idx_out : h->idx;
     float* wts = w_out ? w_out : h->wts;
     bool copies_written = false;
@@ -873,7 +955,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
         ra.row_w = h->row_w;
         ra.cap = h->cap;
         ra.xperm = h->xperm;
-        ra.a_routed_base = N;
+        ra.a_routed_base = NL;
         ra.store_yn = c.n_shared > 0;          // shared experts read yn itself
         if (h->det_rows) ra.slot_row = h->slot_row;   // the combine finds each slot's row
         ra.weights_static = 1;                 // the library's own copy, written at create
@@ -948,7 +1030,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
         TIMED(h, K_ROUTER, 1, st, gemm_tc(h->bf, h->bn_router, h->m_xperm, h->m_wr, &h->m_ynlo, &h->m_wr, gr, er, st));
     }
     if (!copies_written)
-        TIMED(h, K_DISPATCH, 1, st, moe_copy(h->bf, h->xperm, h->slot_row, N, c.top_k, d, N, st));
+        TIMED(h, K_DISPATCH, 1, st, moe_copy(h->bf, h->xperm, h->slot_row, N, c.top_k, d, NL, st));
 
     GemmArgs gu{};
     gu.M = N;
@@ -958,7 +1040,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     gu.n_routed = c.n_experts;
     gu.n_shared = c.n_shared;
     gu.cap = h->cap;
-    gu.a_routed_base = N;
+    gu.a_routed_base = NL;
     gu.pair = h->pair_up;
     gu.max_tiles = h->pair_up ? h->max_tiles_pair : h->max_tiles;
     gu.flags = h->flags;
@@ -978,7 +1060,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
     gd.n_routed = c.n_experts;
     gd.n_shared = c.n_shared;
     gd.cap = h->cap;
-    gd.a_routed_base = N;
+    gd.a_routed_base = NL;
     gd.pair = h->pair_down;
     gd.split_k = h->split_down;
     gd.max_tiles = h->pair_down ? h->max_tiles_pair : h->max_tiles;
@@ -1006,7 +1088,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
 rdt_status loop_impl(rdt_handle* h, const void* h0, const void* e, int T, float* out, bool act,
                      int32_t* n_loops, cudaStream_t st) {
     const rdt_config& c = h->cfg;
-    const int N = h->ntok, d = c.dim;
+    const int N = h->cur_ntok, d = c.dim;
     const size_t nd = static_cast<size_t>(N) * d;
     TIMED(h, K_HOIST, 1, st, hoist(h->bf, h0, e, c.b_kind == RDT_B_DIAG ? h->Bw : nullptr, h->hbuf[0], h->Be, nd, d, st));
     if (c.b_kind == RDT_B_DENSE) TIMED(h, K_DENSE_B, 1, st, matmul_nt_simt(h->bf, e, h->Bw, h->Be, N, d, d, st));
@@ -1016,7 +1098,7 @@ rdt_status loop_impl(rdt_handle* h, const void* h0, const void* e, int T, float*
         float* hcur = h->hbuf[t & 1];
         float* hnext = (t == T - 1 && !act) ? out : h->hbuf[(t + 1) & 1];
         RDT_TRY(attention_block(h, hcur, c.inject_e ? e : nullptr, t, true, nullptr, hnext, st));
-        const size_t tk = static_cast<size_t>(t) * N * c.top_k;
+        const size_t tk = static_cast<size_t>(t) * h->ntok * c.top_k;   // trace layout [loops, batch * seq, k]
         RDT_TRY(moe_block(h, h->y, hnext, nullptr, nullptr, h->tr_idx ? h->tr_idx + tk : nullptr,
                           h->tr_w ? h->tr_w + tk : nullptr, act && t > 0 ? h->act_loops : nullptr, st));
         if (act) {
@@ -1041,6 +1123,12 @@ rdt_status loop_impl(rdt_handle* h, const void* h0, const void* e, int T, float*
     if (act && n_loops)
         RDT_CUDA_TRY(cudaMemcpyAsync(n_loops, h->act_loops, static_cast<size_t>(N) * 4, cudaMemcpyDeviceToDevice, st));
     TIMED(h, K_CHECK, 1, st, check_finite(out, nd, h->flags, st));
+    if (h->mode == 1) {            // the cache now holds the prompt's positions
+        RDT_CUDA_TRY(cudaMemsetAsync(h->dec_len, 0, 4, st));
+        RDT_TRY(len_advance(h->dec_len, c.seq, st));
+    } else if (h->mode == 2) {     // and one more after a step
+        RDT_TRY(len_advance(h->dec_len, 1, st));
+    }
     return RDT_OK;
 }
 
@@ -1065,6 +1153,7 @@ rdt_status run_loop(rdt_handle* h, const void* h0, const void* e, int T, float* 
     key.T = T;
     key.act = act;
     key.n_loops = n_loops;
+    key.mode = h->mode;
     if (h->gexec && h->gkey == key) {
         RDT_CUDA_TRY(cudaGraphLaunch(h->gexec, st));
         h->launches += h->g_launches;
@@ -1184,11 +1273,19 @@ static rdt_status check_ptr(const void* p, const char* name) {
     return RDT_OK;
 }
 
+// Every entry point names the tokens its call processes: all batch * seq positions, or one
+// new position per sequence in a decode step.
+static void set_mode(rdt_handle* h, int mode) {
+    h->mode = mode;
+    h->cur_ntok = mode == 2 ? h->cfg.batch : h->ntok;
+}
+
 rdt_status rdt_attn_forward(rdt_handle* h, const void* x, int loop, float* a_out, void* stream) {
     if (!h) {
         set_error("handle is NULL");
         return RDT_ERR_INVALID_ARG;
     }
+    set_mode(h, 0);
     RDT_TRY(check_ptr(x, "x"));
     RDT_TRY(check_ptr(a_out, "a_out"));
     if (loop < 0) {
@@ -1212,6 +1309,7 @@ rdt_status rdt_moe_forward(rdt_handle* h, const float* y, float* f_out, int32_t*
     RDT_TRY(check_ptr(f_out, "f_out"));
     if (topk_idx) RDT_TRY(check_ptr(topk_idx, "topk_idx"));
     if (topk_w) RDT_TRY(check_ptr(topk_w, "topk_w"));
+    set_mode(h, 0);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     h->last_stream = st;
     const size_t nd = static_cast<size_t>(h->ntok) * h->cfg.dim;
@@ -1236,9 +1334,76 @@ rdt_status rdt_loop_forward(rdt_handle* h, const void* h0, const void* e, int T,
         set_error("out must not alias e (e is read in every loop)");
         return RDT_ERR_INVALID_ARG;
     }
+    set_mode(h, 0);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     h->last_stream = st;
     return run_loop(h, h0, e, T, out, st);
+}
+
+rdt_status rdt_decode_prefill(rdt_handle* h, const void* h0, const void* e, int T, float* out, void* stream) {
+    if (!h) {
+        set_error("handle is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (!h->kv_cache) {
+        set_error("the handle has no KV cache: create it with max_decode > 0");
+        return RDT_ERR_INVALID_ARG;
+    }
+    RDT_TRY(check_ptr(h0, "h0"));
+    RDT_TRY(check_ptr(e, "e"));
+    RDT_TRY(check_ptr(out, "out"));
+    if (T < 1 || T > h->cfg.max_loops) {
+        set_error("T must be in [1, max_loops]");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (out == e) {
+        set_error("out must not alias e (e is read in every loop)");
+        return RDT_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    h->last_stream = st;
+    h->dec_T = 0;
+    set_mode(h, 1);
+    const rdt_status s = run_loop(h, h0, e, T, out, st);
+    set_mode(h, 0);
+    if (s == RDT_OK) {
+        h->dec_T = T;
+        h->dec_len_host = h->cfg.seq;
+    }
+    return s;
+}
+
+rdt_status rdt_decode_step(rdt_handle* h, const void* h0, const void* e, int T, float* out, void* stream) {
+    if (!h) {
+        set_error("handle is NULL");
+        return RDT_ERR_INVALID_ARG;
+    }
+    RDT_TRY(check_ptr(h0, "h0"));
+    RDT_TRY(check_ptr(e, "e"));
+    RDT_TRY(check_ptr(out, "out"));
+    if (h->dec_T == 0) {
+        set_error("no prefill: call rdt_decode_prefill first");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (T != h->dec_T) {
+        set_error("a decode step runs the prefill's number of loops (every loop needs its cache)");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (h->dec_len_host >= h->s_cap) {
+        set_error("the KV cache is full (seq + max_decode positions)");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (out == e) {
+        set_error("out must not alias e (e is read in every loop)");
+        return RDT_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    h->last_stream = st;
+    set_mode(h, 2);
+    const rdt_status s = run_loop(h, h0, e, T, out, st);
+    set_mode(h, 0);
+    if (s == RDT_OK) h->dec_len_host += 1;
+    return s;
 }
 
 rdt_status rdt_loop_forward_host(rdt_handle* h, const void* h0_host, const void* e_host, int T, float* out_host,
@@ -1264,6 +1429,7 @@ rdt_status rdt_loop_forward_host(rdt_handle* h, const void* h0_host, const void*
         RDT_CUDA_TRY(cudaMemcpyAsync(h->stage_h0, h0_host, nd * h->esz, cudaMemcpyHostToDevice, st));
         h0d = h->stage_h0;
     }
+    set_mode(h, 0);
     RDT_TRY(run_loop(h, h0d, h->stage_e, T, h->stage_out, st));
     RDT_CUDA_TRY(cudaMemcpyAsync(out_host, h->stage_out, nd * 4, cudaMemcpyDeviceToHost, st));
     RDT_CUDA_TRY(cudaStreamSynchronize(st));
@@ -1329,6 +1495,7 @@ rdt_status rdt_loop_forward_act(rdt_handle* h, const void* h0, const void* e, in
         set_error("out must not alias e (e is read in every loop)");
         return RDT_ERR_INVALID_ARG;
     }
+    set_mode(h, 0);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     h->last_stream = st;
     return run_loop(h, h0, e, T, out, st, true, n_loops);

@@ -397,7 +397,9 @@ struct EpiParams {
     // RoPE
     const float* rope_cos; // [seq, rot/2]
     const float* rope_sin;
-    int seq;
+    int seq;               // positions per sequence: row r sits at r % seq (+ *pos_dev)
+    const int* pos_dev;    // decode: the device-resident position of every row, or NULL
+    int rope_ld;           // row stride of the angle tables ([rot/2][rope_ld])
     int head_w;            // width of one head's columns (64 or 160)
     int rot_off;           // rotary part starts at this column inside a head
     int rot_dim;           // rotary width
@@ -546,6 +548,8 @@ struct MlaNormArgs {
     void* kv;   // [N, kv_lat + rope]
     const float* rope_cos; const float* rope_sin;
     int ntok, seq, q_lat, kv_lat, rope; float eps;
+    const int* pos_dev;    // decode: added to every row's position (NULL: 0)
+    int rope_ld;           // row stride of the angle tables
 };
 rdt_status mla_latent_norm(bool bf16_elems, const MlaNormArgs& a, cudaStream_t st);
 
@@ -571,5 +575,30 @@ rdt_status prep_matmul(bool bf16_elems, const void* A, long sam, long sak, const
                        long sbn, void* C, int ldc, int M, int N, int K, cudaStream_t st,
                        const void* add = nullptr, int ld_add = 0);
 rdt_status check_finite(const float* x, size_t n, int* flags, cudaStream_t st);
+
+// ---- decode with a per-loop KV cache (decode.cu). Caches hold bf16 rows; the current length
+// (the new token's position during a step) lives in device memory.
+
+// Copy columns [src_col0, src_col0 + width) of ntok rows into a loop's cache: row r belongs to
+// sequence r / rows_per_seq at position r % rows_per_seq (+ *pos_dev), cache row
+// (sequence * s_cap + position), width elements per cache row.
+rdt_status cache_append(const void* src, int src_ld, int src_col0, int width, void* cache, int s_cap,
+                        int rows_per_seq, const int* pos_dev, int ntok, cudaStream_t st);
+
+struct DecodeAttnArgs {
+    const void* q; int q_ld, q_hstride;      // new queries: row b, head h at column h * q_hstride
+    const void* cache; int cache_ld, s_cap;  // loop t's cache, row (b * s_cap + position)
+    int k_col0, k_hstride, v_col0, v_hstride;// key / value columns of KV head g in a cache row
+    int batch, hq, hkv, dqk, dv;
+    const int* len_dev;                      // keys 0 .. *len_dev
+    float scale;
+    float* part;                             // [batch, hq, decode_chunks(s_cap), dv + 2] scratch
+    void* o; int ldo, dv_out;                // o [batch, ldo] bf16, head h at column h * dv_out
+};
+// softmax(q k^T * scale) v over the cached keys 0 .. length of each sequence, split over
+// chunks of keys, then merged (two launches).
+rdt_status decode_attention(const DecodeAttnArgs& a, cudaStream_t st);
+int decode_chunks(int s_cap);
+rdt_status len_advance(int* len, int by, cudaStream_t st);
 
 }  // namespace rdt

@@ -415,9 +415,9 @@ __global__ void __launch_bounds__(kRowThreads) mla_latent_norm_kernel(const MlaN
     // decoupled RoPE key
     const float* R = C + a.kv_lat;
     const int half = a.rope / 2;
-    const int pos = row % a.seq;
+    const int pos = row % a.seq + (a.pos_dev ? *a.pos_dev : 0);
     for (int i = lane; i < half; i += 32) {
-        const float c = a.rope_cos[i * a.seq + pos], s = a.rope_sin[i * a.seq + pos];
+        const float c = a.rope_cos[i * a.rope_ld + pos], s = a.rope_sin[i * a.rope_ld + pos];
         const float x1 = R[i], x2 = R[i + half];
         store_t(kv + a.kv_lat + i, x1 * c - x2 * s);
         store_t(kv + a.kv_lat + half + i, x2 * c + x1 * s);
