@@ -6,4 +6,5 @@ from .rdt_oracle import (rmsnorm, rope_angles, apply_rope, silu, swiglu_ffn, cau
                          spectral_radius, mla_attention_explicit, mla_attention_absorbed,
                          LoopTrace, Routing, NEAR_TIE, NEAR_HALT, halting_probability,
                          loop_forward_act, ActResult, apply_rope_at, LoopKVCache,
-                         attention_cached, loop_prefill, loop_decode)
+                         attention_cached, loop_prefill, loop_decode,
+                         depth_rope_angles, apply_depth_rope, depth_attention_sublayer, DepthKV)

@@ -27,6 +27,10 @@ Sources (pages about the OpenMythos recurrent-depth transformer):
         DeepSeek-V3) vs GQA (Llama 3) section; spectral-radius section.
 * [CB]  hamidun article "OpenMythos: criando transformadores avancados com MLA
         e GQA no Colab": Sparse MoE section (router picks a few experts).
+* [DR]  gist.science summary of "Dreamer" (depth-recurrent attention mixtures):
+        depth attention, attention over a token's earlier depths with depth as the
+        sequence and tokens as the batch, RoPE over depth with a reversed half, applied
+        before sequence attention and the experts (DA -> SA -> EA).
 
 Readings where the pages are silent (each is listed with its reason in the
 design notes of the repository):
@@ -56,12 +60,19 @@ design notes of the repository):
   threshold (or at the last loop), taking the remainder 1 - (sum before) as
   that loop's weight; the output is the weighted sum of its states; a halted
   position keeps its state and still serves as a key, and is routed to no
-  expert.
+  expert;
+* depth attention (an optional sublayer, ``da_heads`` > 0): before the sequence
+  attention, x' = x + DA(RMSNorm_da(x)), where a token's query at loop t attends over
+  its own keys and values of loops 0 .. t (computed from its block inputs at those
+  loops); RoPE over the loop index, the first half of the rotation pairs at t, the
+  second half at T - 1 - t; the sequence attention then takes x', and the block's
+  increment is d + a + f.
 
 Parity status: every function below is pinned (closed forms, library special cases,
 hand-computed fixtures, identities, brute force): the block and the loop by
 ``tests/test_oracle_pins.py``, ACT halting by ``tests/test_oracle_act_pins.py``, the
-cached decode by ``tests/test_oracle_decode_pins.py``.
+cached decode by ``tests/test_oracle_decode_pins.py``, depth attention by
+``tests/test_oracle_depth_pins.py``.
 """
 from __future__ import annotations
 
@@ -337,6 +348,64 @@ def moe_sublayer(y, W, cfg, follow_idx=None, tie_band: float = NEAR_TIE) -> Tupl
 
 
 # --------------------------------------------------------------------------------------
+# Depth attention (attention over a token's earlier loop states)
+# --------------------------------------------------------------------------------------
+
+def depth_rope_angles(depth: int, n_depths: int, rot_dim: int, base: float) -> Tuple[np.ndarray, np.ndarray]:
+    """cos/sin [rot/2] of the rotation at loop `depth` of `n_depths` ([DR] Dreamer summary,
+    depth attention: RoPE over depth, with half of it reversed towards the last depth): pairs
+    i < rot/4 turn by depth * theta_i, pairs i >= rot/4 by (n_depths - 1 - depth) * theta_i,
+    theta_i = base^(-2i/rot)."""
+    i = np.arange(rot_dim // 2, dtype=F)
+    theta = np.power(F(base), -2.0 * i / rot_dim)
+    pos = np.where(i < rot_dim // 4, F(depth), F(n_depths - 1 - depth))
+    ang = pos * theta
+    return np.cos(ang), np.sin(ang)
+
+
+def apply_depth_rope(x, depth: int, n_depths: int, base: float) -> np.ndarray:
+    """Rotate-half RoPE of x [..., r] at loop `depth` (see :func:`depth_rope_angles`)."""
+    x = _f(x)
+    r = x.shape[-1]
+    cos, sin = depth_rope_angles(depth, n_depths, r, base)
+    x1, x2 = x[..., : r // 2], x[..., r // 2:]
+    return np.concatenate([x1 * cos - x2 * sin, x2 * cos + x1 * sin], axis=-1)
+
+
+@dataclass
+class DepthKV:
+    """Keys and values of the depth attention at every loop so far, per token:
+    ``k[s]``, ``v[s]`` [B, S, Hkv, dh] for loops s = 0 .. t."""
+    k: List[np.ndarray] = field(default_factory=list)
+    v: List[np.ndarray] = field(default_factory=list)
+
+
+def depth_attention_sublayer(x, W, cfg, t: int, n_depths: int, kv: DepthKV) -> np.ndarray:
+    """d = DA(RMSNorm_da(x)) at loop t ([DR] depth attention: the sequence dimension is the
+    batch and the depth is the sequence): every token's query attends over its own keys of
+    loops 0 .. t (causal over depth), heads grouped as in GQA, scale 1/sqrt(head_dim);
+    appends loop t's keys and values to ``kv``. Returns d [B, S, dim]."""
+    x = _f(x)
+    Bn, S, _ = x.shape
+    hq, hkv, dh = cfg.da_heads, cfg.da_kv_heads, cfg.head_dim
+    xn = rmsnorm(x, W["norm_da"], cfg.norm_eps)
+    q = apply_depth_rope((xn @ _f(W["wq_d"]).T).reshape(Bn, S, hq, dh), t, n_depths, cfg.rope_base)
+    kv.k.append(apply_depth_rope((xn @ _f(W["wk_d"]).T).reshape(Bn, S, hkv, dh), t, n_depths, cfg.rope_base))
+    kv.v.append((xn @ _f(W["wv_d"]).T).reshape(Bn, S, hkv, dh))
+    K = np.stack(kv.k, axis=2)                      # [B, S, t + 1, hkv, dh]
+    V = np.stack(kv.v, axis=2)
+    o = np.empty((Bn, S, hq, dh), dtype=F)
+    for h in range(hq):
+        g = (h * hkv) // hq
+        s = np.einsum("bnd,bnkd->bnk", q[:, :, h], K[:, :, :, g]) / np.sqrt(dh)   # keys: loops 0 .. t
+        s = s - s.max(axis=-1, keepdims=True)
+        p = np.exp(s)
+        p /= p.sum(axis=-1, keepdims=True)
+        o[:, :, h] = np.einsum("bnk,bnkd->bnd", p, V[:, :, :, g])
+    return o.reshape(Bn, S, hq * dh) @ _f(W["wo_d"]).T
+
+
+# --------------------------------------------------------------------------------------
 # The loop
 # --------------------------------------------------------------------------------------
 
@@ -368,21 +437,27 @@ def loop_forward(h0, e, T: int, W, cfg, follow: Optional[Sequence[np.ndarray]] =
     [GS] Passo 3: the same block repeated n_loops times).
 
     Transformer(h, e) = a + f with x = h + e (or x = h), a = Attn(RMSNorm1(x)),
-    y = x + a, f = MoE(RMSNorm2(y)). ``follow[t]`` is an optional [N, k] selection to
+    y = x + a, f = MoE(RMSNorm2(y)); with depth attention (``cfg.da_heads`` > 0) first
+    d = DA(x) at loop t of T, x <- x + d, and Transformer(h, e) = d + a + f. ``follow[t]`` is an optional [N, k] selection to
     adopt on near-ties at loop t, those within ``tie_band`` (see :func:`moe_sublayer`).
     """
     A = _f(W["A"])
     e = _f(e)
     Be = input_injection(e, W["B"])
     h = _f(h0)
+    depth = DepthKV() if getattr(cfg, "da_heads", 0) else None
     if trace is not None:
         trace.h.append(h.copy())
     for t in range(T):
         x = h + e if cfg.inject_e else h
+        d = 0.0
+        if depth is not None:
+            d = depth_attention_sublayer(x, W, cfg, t, T, depth)
+            x = x + d
         a = attention_sublayer(x, W, cfg, t, mla_form)
         y = x + a
         f, r, st = moe_sublayer(y, W, cfg, None if follow is None else follow[t], tie_band)
-        delta = a + f
+        delta = d + a + f
         h = A * h + Be + delta
         if trace is not None:
             trace.h.append(h.copy())

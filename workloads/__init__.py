@@ -44,6 +44,7 @@ import numpy as np
 __all__ = [
     "Workload", "WORKLOADS", "by_name", "generate", "round_bf16", "bf16_bits",
     "WEIGHT_ORDER_GQA", "WEIGHT_ORDER_MLA", "weight_shapes", "act_head", "ACT_THRESHOLD",
+    "DEPTH_WORKLOAD", "depth_weights",
 ]
 
 # u range that makes A = exp(-exp(u)) <= 0.95 exactly at the upper end.
@@ -82,6 +83,8 @@ class Workload:
     seed: int = 0
     inject_e: bool = True
     weight_std: float = 0.02
+    da_heads: int = 0          # depth attention: query heads (0: no depth attention)
+    da_kv_heads: int = 0       # depth attention: KV heads (head width = head_dim)
 
     @property
     def tokens(self) -> int:
@@ -122,9 +125,16 @@ WORKLOADS: Tuple[Workload, ...] = (
              b_kind="diag", u_low=U_LOW_RHO_095, loops=(16,), seed=4),
 )
 
+# The GQA configuration with a depth-attention sublayer (16 query / 4 KV heads of 64) before
+# the sequence attention: the fifth item of the work list beyond the benchmark set.
+DEPTH_WORKLOAD = Workload(name="gqa-da-bf16-b4s512-d1024-h16x4-e16k2-da16x4", dtype="bf16", batch=4, seq=512,
+                          dim=1024, attn="gqa", n_heads=16, n_kv_heads=4, head_dim=64,
+                          n_experts=16, top_k=2, expert_hidden=1024, b_kind="diag", u_low=-3.0,
+                          loops=(8,), seed=5, da_heads=16, da_kv_heads=4)
+
 
 def by_name(name: str) -> Workload:
-    for w in WORKLOADS:
+    for w in WORKLOADS + (DEPTH_WORKLOAD,):
         if w.name == name:
             return w
     raise KeyError(name)
@@ -243,6 +253,8 @@ def generate(wl: Workload, *, seed: Optional[int] = None, h0_independent: bool =
         out["q_norm"] = np.ones(wl.q_lora_rank, dtype=np.float32)
         out["kv_norm"] = np.ones(wl.kv_lora_rank, dtype=np.float32)
     out["router_bias"] = np.zeros(wl.n_experts, dtype=np.float32)
+    if wl.da_heads:
+        out.update(depth_weights(wl, seed=seed, zero=zero_block))
     if h0_independent:
         h0 = _normal(rng, (wl.batch, wl.seq, wl.dim), 0.0, 1.0)
         out["h0"] = round_bf16(h0) if bf else h0
@@ -257,6 +269,24 @@ def prefix(inputs: Dict[str, np.ndarray], n_tok: int) -> Dict[str, np.ndarray]:
     d["e"] = np.ascontiguousarray(inputs["e"][:, :n_tok])
     d["h0"] = np.ascontiguousarray(inputs["h0"][:, :n_tok])
     return d
+
+
+def depth_weights(wl: Workload, *, seed: Optional[int] = None, zero: bool = False) -> Dict[str, np.ndarray]:
+    """Depth-attention weights, from the PCG64 stream keyed by (seed, 2) so that the draws of
+    :func:`generate` stay as they are: ``norm_da`` = 1, ``wq_d`` [da_heads * head_dim, dim],
+    ``wk_d``, ``wv_d`` [da_kv_heads * head_dim, dim], ``wo_d`` [dim, da_heads * head_dim],
+    each ~ N(0, weight_std), rounded like the other matrices."""
+    rng = np.random.Generator(np.random.PCG64([wl.seed if seed is None else seed, 2]))
+    bf = wl.dtype == "bf16"
+    dh, d = wl.head_dim, wl.dim
+    out = {"norm_da": np.ones(d, dtype=np.float32)}
+    for k, shp in (("wq_d", (wl.da_heads * dh, d)), ("wk_d", (wl.da_kv_heads * dh, d)),
+                   ("wv_d", (wl.da_kv_heads * dh, d)), ("wo_d", (d, wl.da_heads * dh))):
+        w = _normal(rng, shp, 0.0, wl.weight_std)
+        if zero:
+            w[...] = 0.0
+        out[k] = round_bf16(w) if bf else w
+    return out
 
 
 ACT_THRESHOLD = 0.99
