@@ -11,6 +11,11 @@ step is reported.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--workload NAME] [--loops T] [--act] [--all]
+                    [--decode] [--kernel attention]
+
+--decode times rdt_decode_step (one new token per sequence, T loops, over a prompt of the
+workload's length) instead. `--kernel attention` times rdt_attention alone on the workload's
+sequence-attention shape (the command the attention kernel's ncu captures run).
 
 --gpus N > 1 runs one process per GPU (re-launched under torch.distributed.run when not
 started by it): every rank runs a replica of the workload on inputs of its own (no
@@ -60,7 +65,11 @@ KERNEL_SOURCES = {
                 "recurrent_depth_transformer_b200/csrc/rdt_api.cu"),
 }
 # (workload, kernel) -> (bytes per launch, source fingerprint)
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum on the default command:
+    # 50.38 MB read + 2.04 MB written (o stays in L2 when the kernel ends)
+    ("long-bf16-b1s8192-d2048-h32x8-e64k8-lora16", "attention"): (50376704.0 + 2036736.0, "4fca9a59cb512285"),
+}
 
 
 def code_text(src: str) -> str:
@@ -148,6 +157,18 @@ def kernel_work(wl):
         ow = H * kvl
         w["gemm_o"] = dict(flops=2.0 * N * ow * d, bytes=b2 * (N * ow + d * ow) + 4 * 2 * N * d, bound="tensor")
         w["mla_latent_norm"] = dict(flops=0.0, bytes=N * (4 * lat + b2 * (ql + kvl + rp)), bound="hbm")
+    if getattr(wl, "da_heads", 0):
+        # depth attention: projections of every token, each query over its T loops' keys
+        # (the mean over loops t = 0 .. T-1 of t + 1 keys is counted per launch by the caller)
+        hqd, hkvd, dh = wl.da_heads, wl.da_kv_heads, wl.head_dim
+        nqd, nqkvd = hqd * dh, (hqd + 2 * hkvd) * dh
+        w["gemm_qkv_depth"] = dict(flops=2.0 * N * d * nqkvd, bytes=b2 * (N * d + nqkvd * d + N * nqkvd), bound="tensor")
+        T = max(wl.loops)
+        keys = (T + 1) / 2.0
+        w["depth_attention"] = dict(flops=4.0 * N * hqd * dh * keys,
+                                    bytes=b2 * N * (nqd + 2 * hkvd * dh * keys + nqd), bound="hbm")
+        w["gemm_o_depth"] = dict(flops=2.0 * N * nqd * d, bytes=b2 * (N * nqd + d * nqd) + 4 * 2 * N * d,
+                                 bound="tensor")
     w["gemm_up"] = dict(flops=2.0 * rows * d * 2 * hid, bytes=b2 * (rows * d + (E + S) * 2 * hid * d + rows * hid),
                         bound="tensor")
     w["gemm_down"] = dict(flops=2.0 * rows * hid * d, bytes=b2 * (rows * hid + (E + S) * d * hid) + 4 * N * d * 2,
@@ -168,7 +189,8 @@ def kernel_work(wl):
     return w
 
 
-PATH_KERNELS = ("gemm_qkv", "gemm_latent", "gemm_q_absorbed", "attention", "gemm_o", "gemm_up", "gemm_down")
+PATH_KERNELS = ("gemm_qkv", "gemm_latent", "gemm_q_absorbed", "attention", "gemm_o", "gemm_up", "gemm_down",
+                "gemm_qkv_depth", "depth_attention", "gemm_o_depth")
 
 
 def step_flops(wl, T):
@@ -601,6 +623,140 @@ ALL_RUNS = (("tiny-f32-b1s64-d128-gqa4x2-e4k2", 4), ("gqa-bf16-b4s512-d1024-h16x
             ("long-bf16-b1s8192-d2048-h32x8-e64k8-lora16", 16))
 
 
+def decode_bytes(wl, length, experts_used):
+    """Algorithmic bytes of one decode step's loop: every projection and router weight once,
+    the weights of the experts the step's tokens chose, the cache read up to the new position
+    and the new row written, the state and activation rows."""
+    d, b2, B = wl.dim, 2, wl.batch
+    if wl.attn == "gqa":
+        nq, nkv = wl.n_heads * wl.head_dim, wl.n_kv_heads * wl.head_dim
+        proj = (nq + 2 * nkv) * d + d * nq
+        cache_row = 2 * nkv
+    else:
+        H, ql, kvl, rp = wl.n_heads, wl.q_lora_rank, wl.kv_lora_rank, wl.qk_rope_dim
+        proj = (ql + kvl + rp) * d + ql * H * (kvl + rp) + d * H * kvl
+        cache_row = kvl + rp
+    experts = (experts_used + wl.n_shared) * 3 * wl.expert_hidden * d
+    return b2 * (proj + wl.n_experts * d + experts + B * (length + 1) * cache_row + B * cache_row) + B * d * 4 * 6
+
+
+def bench_decode(args, dev, rank, world):
+    """Decode steps of one token per sequence after a prompt of the workload's length."""
+    import numpy as np
+    import torch
+
+    import recurrent_depth_transformer_b200 as R
+    from workloads import by_name, generate, round_bf16
+
+    wl = by_name(args.workload)
+    T = args.loops
+    inputs = generate(wl)
+    steps = args.warmup + args.steps
+    weights = R.device_weights(inputs, True, device=dev)
+    h = R.RDT(R.make_config(wl, max_loops=T, max_decode=steps), weights)
+    del weights
+    e = torch.from_numpy(inputs["e"]).to(torch.bfloat16).to(dev)
+    h.decode_prefill(e, e, T)
+    rng = np.random.default_rng(wl.seed + 7)
+    new = torch.from_numpy(round_bf16(rng.standard_normal((steps, wl.batch, wl.dim)).astype(np.float32)))
+    new = new.to(torch.bfloat16).to(dev)
+    out = torch.empty((wl.batch, wl.dim), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    xs = [new[i].contiguous() for i in range(steps)]
+    buf = torch.empty_like(xs[0])
+    for i in range(args.warmup):             # eager, capture, replays (same pointers every step)
+        buf.copy_(xs[i])
+        h.decode_step(buf, buf, T, out=out)
+    torch.cuda.synchronize()
+    barrier()
+    launches0 = h.launch_count()
+    evs = []
+    for i in range(args.warmup, steps):
+        buf.copy_(xs[i])
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        h.decode_step(buf, buf, T, out=out)
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    launches = (h.launch_count() - launches0) / args.steps
+    ms = reduce_max(statistics.median(a.elapsed_time(b) for a, b in evs), dev)
+    diag = h.diagnostics()
+    used = sum(1 for c in diag["expert_counts"][:wl.n_experts] if c > 0)
+    length = wl.seq + steps - 1
+    nbytes = decode_bytes(wl, length, used) * T
+    peaks, src = load_peaks()
+    h.close()
+    if rank != 0:
+        return None
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {
+        "impl": "ours-decode", "metric": "decode tokens/s (one token per sequence per step, T loops)",
+        "value": world * wl.batch / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": wl.batch, "prompt": wl.seq, "dim": wl.dim, "loops": T,
+                   "cache_positions": wl.seq + steps, "parallelism": f"replicas x{world}"},
+        "roofline": {"kernel": "decode step (whole)", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": f"{src} HBM copy", "algorithmic_per_step": nbytes,
+                     "experts_read_last_step": used},
+        "gpu_launches": int(round(launches)),
+    }
+
+
+def bench_attention(args, dev, rank, world):
+    """rdt_attention alone on the workload's sequence-attention shape (GQA heads; bf16 q, k, v
+    drawn from a seeded normal), event-timed per launch: the kernel-level line that the
+    attention ncu captures run."""
+    import torch
+
+    import recurrent_depth_transformer_b200 as R
+    from workloads import by_name
+
+    wl = by_name(args.workload)
+    if wl.attn != "gqa" or wl.dtype != "bf16":
+        raise SystemExit("--kernel attention times bf16 GQA workloads")
+    B, S, Hq, Hkv, D = wl.batch, wl.seq, wl.n_heads, wl.n_kv_heads, wl.head_dim
+    g = torch.Generator(device=dev).manual_seed(wl.seed)
+    q = torch.randn(B * S, Hq * D, device=dev, generator=g).to(torch.bfloat16)
+    k = torch.randn(B * S, Hkv * D, device=dev, generator=g).to(torch.bfloat16)
+    v = torch.randn(B * S, Hkv * D, device=dev, generator=g).to(torch.bfloat16)
+    o = torch.empty(B * S, Hq * D, device=dev, dtype=torch.bfloat16)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        R.attention(q, k, v, B, S, Hq, Hkv, D, D, D ** -0.5, o=o)
+    torch.cuda.synchronize()
+    barrier()
+    evs = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        R.attention(q, k, v, B, S, Hq, Hkv, D, D, D ** -0.5, o=o)
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    ms = reduce_max(statistics.median(a.elapsed_time(b) for a, b in evs), dev)
+    if rank != 0:
+        return None
+    peaks, src = load_peaks()
+    flops = 4.0 * B * Hq * D * S * (S + 1) / 2
+    tf = flops / (ms / 1e3) / 1e12
+    return {
+        "impl": "ours-kernel", "metric": "causal attention TFLOP/s (one launch)", "value": world * tf,
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": B, "seq": S, "heads": Hq, "kv_heads": Hkv, "head_dim": D,
+                   "l2": "flushed between launches", "parallelism": f"replicas x{world}"},
+        "roofline": {"kernel": "attention", "bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"], "traffic": None,
+                     "peak_source": f"{src} cuBLAS bf16 burst"},
+        "gpu_launches": 1,
+    }
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -609,6 +765,14 @@ def run_gpu(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     init_ranks(dev)
+    if args.decode or args.kernel:
+        line = (bench_attention if args.kernel else bench_decode)(args, dev, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        barrier()
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
     runs = ALL_RUNS if args.all else ((args.workload, args.loops),)
     for name, T in runs:
         line = bench_one(args, name, T, dev, rank, world, with_cpu=not args.all or name == args.workload)
@@ -633,6 +797,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=WORKLOAD, help="workload name (default: the headline one)")
     ap.add_argument("--loops", type=int, default=LOOPS, help="loops T per step")
     ap.add_argument("--all", action="store_true", help="one line per configuration and loop count")
+    ap.add_argument("--decode", action="store_true", help="time decode steps with the per-loop KV cache")
+    ap.add_argument("--kernel", choices=("attention",), help="time one kernel alone on the workload's shape")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -99,6 +99,9 @@ typedef struct {
                                      * only): max_loops * batch * (seq + max_decode) rows of
                                      * 2 n_kv_heads head_dim (GQA) or kv_lora_rank +
                                      * qk_rope_dim (MLA) elements. 0: no cache.         */
+    int32_t da_heads;               /* depth attention: query heads (0: none); GQA, bf16,
+                                     * head width head_dim = 64                          */
+    int32_t da_kv_heads;            /* depth attention: KV heads (divides da_heads)     */
 } rdt_config;
 
 /* Weights, all DEVICE pointers, row-major [out, in]; element type = cfg.dtype
@@ -138,6 +141,16 @@ typedef struct {
     const void* lq_b;          /* [n_lora, n_heads * head_dim, lora_rank]                */
     const void* lo_a;          /* [n_lora, lora_rank, n_heads * head_dim]                */
     const void* lo_b;          /* [n_lora, dim, lora_rank]                               */
+    /* depth attention (cfg.da_heads > 0): before the sequence attention of loop t of T,
+     * x' = x + DA(RMSNorm_da(x)); a token's query attends over its own keys and values of
+     * loops 0 .. t (RoPE over the loop index: rotation pairs i < head_dim/4 at t, the rest
+     * at T - 1 - t); the sequence attention takes x' and the increment is d + a + f
+     * (gist.science summary of "Dreamer", depth attention) */
+    const float* norm_da;      /* [dim] fp32 RMSNorm gain of the depth attention        */
+    const void* wq_d;          /* [da_heads * head_dim, dim]                             */
+    const void* wk_d;          /* [da_kv_heads * head_dim, dim]                          */
+    const void* wv_d;          /* [da_kv_heads * head_dim, dim]                          */
+    const void* wo_d;          /* [dim, da_heads * head_dim]                             */
 } rdt_weights;
 
 typedef struct rdt_handle rdt_handle;

@@ -54,13 +54,15 @@ class RdtConfig(ctypes.Structure):
         ("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float)] + [
         (n, ctypes.c_int32) for n in ("n_experts", "top_k", "n_shared", "expert_hidden",
                                       "lora_rank", "n_lora", "b_kind", "inject_e", "max_loops",
-                                      "gemm_tiles", "deterministic", "max_decode")]
+                                      "gemm_tiles", "deterministic", "max_decode", "da_heads",
+                                      "da_kv_heads")]
 
 
 WEIGHT_FIELDS = ("A", "B", "norm1", "norm2", "wq", "wk", "wv", "wo", "w_dq", "q_norm", "w_uq",
                  "w_dkv", "kv_norm", "w_kr", "w_uk", "w_uv", "w_router", "router_bias", "w1",
-                 "w3", "w2", "ws1", "ws3", "ws2", "lq_a", "lq_b", "lo_a", "lo_b")
-FP32_FIELDS = ("A", "B", "norm1", "norm2", "q_norm", "kv_norm", "router_bias")
+                 "w3", "w2", "ws1", "ws3", "ws2", "lq_a", "lq_b", "lo_a", "lo_b", "norm_da", "wq_d",
+                 "wk_d", "wv_d", "wo_d")
+FP32_FIELDS = ("A", "B", "norm1", "norm2", "q_norm", "kv_norm", "router_bias", "norm_da")
 
 
 class RdtWeights(ctypes.Structure):
@@ -165,6 +167,8 @@ def make_config(wl, max_loops: int = 16, batch: Optional[int] = None, seq: Optio
     c.gemm_tiles = gemm_tiles
     c.deterministic = 1 if deterministic else 0
     c.max_decode = max_decode
+    c.da_heads = getattr(wl, "da_heads", 0)
+    c.da_kv_heads = getattr(wl, "da_kv_heads", 0)
     return c
 
 

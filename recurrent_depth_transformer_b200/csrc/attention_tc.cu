@@ -497,6 +497,8 @@ rdt_status launch_choose(const AttnArgs& a, cudaStream_t st) {
 rdt_status attention_tc(const AttnArgs& a, cudaStream_t st) {
     if (a.dqk == 64 && a.dv == 64) return launch_choose<64, 64, false>(a, st);
     if (a.dqk == 160 && a.dv == 128 && a.v == a.k) return launch_choose<160, 128, true>(a, st);
+    // 160-wide keys with values of their own: one tile per CTA (two would not fit in shared memory)
+    if (a.dqk == 160 && a.dv == 128) return launch_tc<160, 128, false, 1>(a, st);
     set_error("tensor-core attention: unsupported head dimensions");
     return RDT_ERR_UNSUPPORTED;
 }

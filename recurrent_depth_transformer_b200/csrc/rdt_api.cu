@@ -87,6 +87,14 @@ struct rdt_handle {
     int dec_T = 0;                 // loops of the prefill (decode steps run the same number)
     int dec_len_host = 0;          // the same length, tracked on the host for validation
     int mode = 0;                  // 0 plain loop, 1 prefill (fills the cache), 2 decode step
+    // depth attention (cfg.da_heads > 0)
+    int nq_d = 0, nkv_d = 0, nqkv_d = 0;
+    float* g_da = nullptr;
+    void *wqkv_d = nullptr, *wo_d = nullptr, *qkv_d = nullptr, *o_d = nullptr, *depth_cache = nullptr;
+    float *dtab_cos = nullptr, *dtab_sin = nullptr;   // [max_loops * max_loops][head_dim / 2]
+    int* didx = nullptr;           // device [max_loops]: 0, 1, .. (loop t's depth-cache row)
+    CUtensorMap m_wqkv_d, m_od, m_wo_d;
+    int cur_T = 0;                 // loops of the current call (the depth rotation's last depth)
     int cur_ntok = 0;              // tokens of the current call (batch in a decode step)
     void *stage_h0 = nullptr, *stage_e = nullptr;
     float* stage_out = nullptr;
@@ -150,12 +158,13 @@ constexpr int kFillerRows = 256;
 // kernel classes reported by rdt_profile_read
 enum Kind { K_HOIST, K_NORM1, K_GEMM_QKV, K_GEMM_LAT, K_MLA_NORM, K_GEMM_Q, K_ATTENTION,
             K_GEMM_O, K_NORM2, K_ROUTER, K_DISPATCH, K_GEMM_UP, K_GEMM_DOWN, K_CHECK, K_DENSE_B, K_ACT,
-            K_COMBINE, K_CACHE, K_DEC_ATTN, K_COUNT };
+            K_COMBINE, K_CACHE, K_DEC_ATTN, K_DA_QKV, K_DA_ATTN, K_DA_O, K_COUNT };
 const char* const kKindName[K_COUNT] = {"hoist", "norm1", "gemm_qkv", "gemm_latent", "mla_latent_norm",
                                          "gemm_q_absorbed", "attention", "gemm_o",
                                          "norm2", "router_topk", "moe_dispatch", "gemm_up", "gemm_down",
                                          "check_finite", "dense_injection", "act_halting", "moe_combine", "kv_cache_append",
-                                         "decode_attention"};
+                                         "decode_attention", "gemm_qkv_depth", "depth_attention",
+                                         "gemm_o_depth"};
 
 // During graph capture the events become event-record nodes of the graph (external
 // records), so that every replay records them again; they are then kept apart from the
@@ -276,6 +285,14 @@ rdt_status validate_config(const rdt_config* c) {
     if (c->max_decode < 0 || c->max_decode > (1 << 20)) return bad("max_decode");
     if (c->max_decode > 0 && c->dtype != RDT_BF16) return uns("decode with a KV cache is provided in bf16");
     if (static_cast<long long>(c->seq) + c->max_decode > (1 << 24)) return uns("seq + max_decode too large");
+    if (c->da_heads < 0 || c->da_kv_heads < 0) return bad("da_heads / da_kv_heads");
+    if (c->da_heads > 0) {
+        if (c->attn_type != RDT_GQA || c->dtype != RDT_BF16 || c->head_dim != 64)
+            return uns("depth attention is provided for bf16 GQA with head_dim 64");
+        if (c->da_kv_heads < 1 || c->da_heads % c->da_kv_heads) return bad("da_heads % da_kv_heads");
+        if ((c->da_heads * 64) % 128 || ((c->da_heads + 2 * c->da_kv_heads) * 64) % 128)
+            return uns("depth attention widths must be multiples of 128");
+    }
     if (c->b_kind != RDT_B_DIAG && c->b_kind != RDT_B_DENSE) return bad("b_kind");
     if (!(c->norm_eps >= 0.0f) || !(c->rope_base > 1.0f)) return bad("norm_eps / rope_base");
     if (c->lora_rank < 0 || c->n_lora < 0) return bad("lora");
@@ -408,6 +425,11 @@ rdt_status build_maps(rdt_handle* h) {
     RDT_TRY(make_tmap_2d(&h->m_U, h->U, bf, hid, urows, hid * es, kbox, 128));
     RDT_TRY(make_tmap_2d(&h->m_w2, h->w2, bf, hid, static_cast<uint64_t>(E + S) * d, hid * es, kbox, h->bn_down >> h->pair_down));
     RDT_TRY(make_tmap_2d(&h->m_ynlo, h->yn_lo, bf, d, N, d * es, kbox, 128));
+    if (c.da_heads) {
+        RDT_TRY(make_tmap_2d(&h->m_wqkv_d, h->wqkv_d, bf, d, h->nqkv_d, d * es, kbox, 128));
+        RDT_TRY(make_tmap_2d(&h->m_od, h->o_d, bf, h->nq_d, N, h->nq_d * es, kbox, 128));
+        RDT_TRY(make_tmap_2d(&h->m_wo_d, h->wo_d, bf, h->nq_d, d, h->nq_d * es, kbox, 128));
+    }
     RDT_TRY(make_tmap_2d(&h->m_wr, h->wr, bf, d, E, d * es, kbox, h->bn_router));
     return RDT_OK;
 }
@@ -456,6 +478,13 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         RDT_TRY(need(w->w_uk, "w_uk"));
         RDT_TRY(need(w->w_uv, "w_uv"));
         RDT_TRY(need(w->wo, "wo"));
+    }
+    if (c.da_heads) {
+        RDT_TRY(need(w->norm_da, "norm_da"));
+        RDT_TRY(need(w->wq_d, "wq_d"));
+        RDT_TRY(need(w->wk_d, "wk_d"));
+        RDT_TRY(need(w->wv_d, "wv_d"));
+        RDT_TRY(need(w->wo_d, "wo_d"));
     }
     if (c.n_lora) {
         RDT_TRY(need(w->lq_a, "lq_a"));
@@ -694,6 +723,44 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
     RDT_TRY(dev_alloc(h, &h->flags, FLAG_COUNT * 4, true));
     if (c.deterministic)
         RDT_TRY(dev_alloc(h, &h->det_rows, static_cast<size_t>(h->cap) * (S + E) * d * 4));
+    if (c.da_heads) {
+        h->nq_d = c.da_heads * c.head_dim;
+        h->nkv_d = c.da_kv_heads * c.head_dim;
+        h->nqkv_d = h->nq_d + 2 * h->nkv_d;
+        RDT_TRY(dev_alloc(h, &h->g_da, d * 4));
+        RDT_TRY(copy_d2d(h->g_da, w->norm_da, d * 4, st));
+        RDT_TRY(dev_alloc(h, &h->wqkv_d, static_cast<size_t>(h->nqkv_d) * d * es));
+        char* q = static_cast<char*>(h->wqkv_d);
+        RDT_TRY(copy_d2d(q, w->wq_d, static_cast<size_t>(h->nq_d) * d * es, st));
+        RDT_TRY(copy_d2d(q + static_cast<size_t>(h->nq_d) * d * es, w->wk_d, static_cast<size_t>(h->nkv_d) * d * es, st));
+        RDT_TRY(copy_d2d(q + static_cast<size_t>(h->nq_d + h->nkv_d) * d * es, w->wv_d,
+                         static_cast<size_t>(h->nkv_d) * d * es, st));
+        RDT_TRY(dev_alloc(h, &h->wo_d, static_cast<size_t>(d) * h->nq_d * es));
+        RDT_TRY(copy_d2d(h->wo_d, w->wo_d, static_cast<size_t>(d) * h->nq_d * es, st));
+        RDT_TRY(dev_alloc(h, &h->qkv_d, static_cast<size_t>(N) * h->nqkv_d * es));
+        RDT_TRY(dev_alloc(h, &h->o_d, static_cast<size_t>(N) * h->nq_d * es));
+        RDT_TRY(dev_alloc(h, &h->depth_cache, static_cast<size_t>(N) * c.max_loops * 2 * h->nkv_d * es));
+        // rotation of loop t of T: pairs i < head_dim/4 at t, the others at T - 1 - t
+        const int half = c.head_dim / 2, L = c.max_loops;
+        std::vector<float> dc(static_cast<size_t>(L) * L * half, 0.0f), ds(dc.size(), 0.0f);
+        for (int T = 1; T <= L; ++T)
+            for (int t = 0; t < T; ++t)
+                for (int i = 0; i < half; ++i) {
+                    const double pos = i < c.head_dim / 4 ? t : T - 1 - t;
+                    const double ang = pos * std::pow(static_cast<double>(c.rope_base), -2.0 * i / c.head_dim);
+                    const size_t o = (static_cast<size_t>(T - 1) * L + t) * half + i;
+                    dc[o] = static_cast<float>(std::cos(ang));
+                    ds[o] = static_cast<float>(std::sin(ang));
+                }
+        RDT_TRY(dev_alloc(h, &h->dtab_cos, dc.size() * 4));
+        RDT_TRY(dev_alloc(h, &h->dtab_sin, ds.size() * 4));
+        RDT_CUDA_TRY(cudaMemcpy(h->dtab_cos, dc.data(), dc.size() * 4, cudaMemcpyHostToDevice));
+        RDT_CUDA_TRY(cudaMemcpy(h->dtab_sin, ds.data(), ds.size() * 4, cudaMemcpyHostToDevice));
+        std::vector<int> idx(L);
+        for (int t = 0; t < L; ++t) idx[t] = t;
+        RDT_TRY(dev_alloc(h, &h->didx, L * 4));
+        RDT_CUDA_TRY(cudaMemcpy(h->didx, idx.data(), L * 4, cudaMemcpyHostToDevice));
+    }
     if (c.max_decode > 0) {
         h->cache_w = c.attn_type == RDT_GQA ? 2 * c.n_kv_heads * c.head_dim : c.kv_lora_rank + c.qk_rope_dim;
         RDT_TRY(dev_alloc(h, &h->kv_cache,
@@ -714,6 +781,84 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
 
 int lora_index(const rdt_handle* h, int t) { return std::min(t, h->cfg.n_lora - 1); }
 
+// ---- depth attention of loop t: RMSNorm_da(x) -> [q; k; v] with the depth rotation -> loop
+// t's keys and values into the token's depth cache -> attention over loops 0 .. t -> output
+// projection adding d into y (= x, written by the same RMSNorm) and h_next (A h + B e)
+rdt_status depth_block(rdt_handle* h, const float* hin, const void* e, int t, float* h_next, cudaStream_t st) {
+    const rdt_config& c = h->cfg;
+    const int N = h->cur_ntok, d = c.dim;
+    Norm1Args n1{};
+    n1.h = hin;
+    n1.e = e;
+    n1.gamma = h->g_da;
+    n1.xn = h->xn;
+    n1.ntok = N;
+    n1.dim = d;
+    n1.eps = c.norm_eps;
+    n1.zero_counts = h->counts;
+    n1.n_zero = h->G;
+    n1.y0 = h->y;
+    n1.hn0 = h_next;
+    n1.Be = h->Be;
+    n1.Adiag = h->A;
+    TIMED(h, K_NORM1, 1, st, norm1(h->bf, n1, st));
+
+    GemmArgs ga{};
+    ga.M = N;
+    ga.N = h->nqkv_d;
+    ga.kb_main = static_cast<int>(d * h->esz / 128);
+    ga.flags = h->flags;
+    EpiParams ep{};
+    ep.flags = h->flags;
+    ep.kind = EPI_ROPE;
+    ep.out = h->qkv_d;
+    ep.ldo = h->nqkv_d;
+    ep.ncols_valid = h->nqkv_d;
+    const size_t tab = (static_cast<size_t>(h->cur_T - 1) * c.max_loops + t) * (c.head_dim / 2);
+    ep.rope_cos = h->dtab_cos + tab;   // one row: every token of loop t at the same depth
+    ep.rope_sin = h->dtab_sin + tab;
+    ep.seq = 1;
+    ep.rope_ld = 1;
+    ep.head_w = c.head_dim;
+    ep.rot_off = 0;
+    ep.rot_dim = c.head_dim;
+    ep.rope_limit = h->nq_d + h->nkv_d;
+    TIMED(h, K_DA_QKV, 1, st, gemm_tc(h->bf, 128, h->m_xn, h->m_wqkv_d, nullptr, nullptr, ga, ep, st));
+    // loop t's keys and values: row (token, t) of the depth cache
+    TIMED(h, K_CACHE, 1, st, cache_append(h->qkv_d, h->nqkv_d, h->nq_d, 2 * h->nkv_d, h->depth_cache, c.max_loops,
+                                          1, h->didx + t, N, st));
+    DepthAttnArgs da{};
+    da.q = static_cast<const bf16*>(h->qkv_d);
+    da.q_ld = h->nqkv_d;
+    da.cache = static_cast<const bf16*>(h->depth_cache);
+    da.cache_w = 2 * h->nkv_d;
+    da.max_depth = c.max_loops;
+    da.v_col0 = h->nkv_d;
+    da.t = t;
+    da.ntok = N;
+    da.hq = c.da_heads;
+    da.hkv = c.da_kv_heads;
+    da.scale_log2 = 1.4426950408889634f / std::sqrt(static_cast<float>(c.head_dim));
+    da.o = static_cast<bf16*>(h->o_d);
+    da.o_ld = h->nq_d;
+    TIMED(h, K_DA_ATTN, 1, st, depth_attention(da, st));
+
+    GemmArgs go{};
+    go.M = N;
+    go.N = d;
+    go.kb_main = static_cast<int>(h->nq_d * h->esz / 128);
+    go.flags = h->flags;
+    EpiParams eo{};
+    eo.flags = h->flags;
+    eo.kind = EPI_OPROJ_LOOP;
+    eo.ncols_valid = d;
+    eo.y = h->y;
+    eo.h_next = h_next;
+    eo.ld = d;
+    TIMED(h, K_DA_O, 1, st, gemm_tc(h->bf, 128, h->m_od, h->m_wo_d, nullptr, nullptr, go, eo, st));
+    return RDT_OK;
+}
+
 // ---- the attention sublayer: norm1 -> projections -> attention -> O projection
 rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t, bool loop_mode,
                            float* a_out, float* h_next, cudaStream_t st) {
@@ -729,19 +874,19 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
                                   static_cast<size_t>(t) * c.batch * h->s_cap * h->cache_w * h->esz
                             : nullptr;
 
+    const bool depth = c.da_heads > 0 && loop_mode;
+    if (depth) RDT_TRY(depth_block(h, hin, e, t, h_next, st));
     Norm1Args n1{};
-    n1.h = hin;
-    n1.e = e;
+    n1.h = depth ? h->y : hin;          // with depth attention: x' = x + d, complete in y
+    n1.e = depth ? nullptr : e;
     n1.gamma = h->g1;
     n1.xn = h->xn;
     n1.ntok = N;
     n1.dim = d;
     n1.eps = c.norm_eps;
-    if (loop_mode) {
+    if (loop_mode && !depth) {          // (the depth block's RMSNorm did this)
         n1.zero_counts = h->counts;
         n1.n_zero = h->G;
-    }
-    if (loop_mode) {
         n1.y0 = h->y;
         n1.hn0 = h_next;
         n1.Be = h->Be;
@@ -1090,6 +1235,7 @@ rdt_status loop_impl(rdt_handle* h, const void* h0, const void* e, int T, float*
     const rdt_config& c = h->cfg;
     const int N = h->cur_ntok, d = c.dim;
     const size_t nd = static_cast<size_t>(N) * d;
+    h->cur_T = T;
     TIMED(h, K_HOIST, 1, st, hoist(h->bf, h0, e, c.b_kind == RDT_B_DIAG ? h->Bw : nullptr, h->hbuf[0], h->Be, nd, d, st));
     if (c.b_kind == RDT_B_DENSE) TIMED(h, K_DENSE_B, 1, st, matmul_nt_simt(h->bf, e, h->Bw, h->Be, N, d, d, st));
     if (h->tr_h) RDT_CUDA_TRY(cudaMemcpyAsync(h->tr_h, h->hbuf[0], nd * 4, cudaMemcpyDeviceToDevice, st));

@@ -601,4 +601,15 @@ rdt_status decode_attention(const DecodeAttnArgs& a, cudaStream_t st);
 int decode_chunks(int s_cap);
 rdt_status len_advance(int* len, int by, cudaStream_t st);
 
+// ---- depth attention (depth.cu): a token's query at loop t against its own keys and values
+// of loops 0 .. t, kept in a per-token depth cache [ntok][max_depth][cache_w] (bf16).
+struct DepthAttnArgs {
+    const bf16* q; int q_ld;               // queries: row n, head h at column h * 64
+    const bf16* cache; int cache_w, max_depth, v_col0;   // keys at column g * 64, values at v_col0 + g * 64
+    int t, ntok, hq, hkv;
+    float scale_log2;
+    bf16* o; int o_ld;                     // o: row n, head h at column h * 64
+};
+rdt_status depth_attention(const DepthAttnArgs& a, cudaStream_t st);
+
 }  // namespace rdt
