@@ -13,10 +13,11 @@
 //   warp 1      allocates the TMEM accumulator; one thread issues tcgen05.mma (M = 128,
 //               N = BN, K = 16 bf16 / 8 tf32 per instruction) and frees each stage with
 //               tcgen05.commit when its MMAs have read it;
-//   warps 2-5   the epilogue: each warp reads its 32-lane quadrant of TMEM (one output row
-//               per thread, 32 columns at a time), transposes the 32 x 32 chunk through a
-//               private shared-memory buffer so that each global access of the warp covers
-//               four whole row segments, and applies one of the fused epilogues below.
+//   warps 2-9   the epilogue (warps 2-5 for the router's top-k): each warp reads its 32-lane
+//               quadrant of TMEM (one output row per thread, 32 columns at a time; two warps
+//               per quadrant take alternate column chunks), transposes the 32 x 32 chunk
+//               through a private shared-memory buffer so that each global access of the warp
+//               covers four whole row segments, and applies one of the fused epilogues below.
 //
 // The fused epilogues are where the block's element-wise work lives:
 //   EPI_ROPE        Q/K/V projection + rotary embedding on the rotated heads;
@@ -43,16 +44,25 @@ namespace rdt {
 namespace {
 
 constexpr int BM = 128;
-constexpr int kThreads = 192;
 
-template <int BN, int CG>
+// Epilogue warps per TMEM lane quadrant: two for the epilogues that work chunk by chunk
+// (each warp takes every other 32-column chunk of the tile, so that one warp's TMEM loads,
+// transposes and stores or reductions overlap the other's), one for the router's top-k (a
+// warp needs its rows' whole logits).
+template <int KIND>
+__host__ __device__ constexpr int epi_split() { return KIND == EPI_TOPK ? 1 : 2; }
+// warp 0: TMA, warp 1: MMA, then 4 x epi_split epilogue warps
+template <int KIND>
+__host__ __device__ constexpr int gemm_threads() { return 64 + 128 * epi_split<KIND>(); }
+
+template <int BN, int CG, int ES>
 struct TcCfg {
     static constexpr int B_ROWS = BN / CG;               // B rows this CTA loads per stage
     static constexpr int A_BYTES = BM * 128;
     static constexpr int B_BYTES = B_ROWS * 128;
     static constexpr int BAR_BYTES = 192;
     static constexpr int GROUP_BYTES = 2064;
-    static constexpr int STG_BYTES = 4 * 32 * 32 * 4;     // one 32 x 32 fp32 chunk per epilogue warp
+    static constexpr int STG_BYTES = 4 * ES * 32 * 32 * 4;   // one 32 x 32 fp32 chunk per epilogue warp
     // As many stages as keep the block (plus the 1 KB reserved per CTA) within the 196 KB
     // shared-memory carveout, at most 8: beyond it the driver takes the 228 KB carveout and
     // L1 shrinks from 60 to 28 KB, which measurably slows the epilogues' global traffic.
@@ -297,16 +307,18 @@ __device__ __forceinline__ void epilogue_pre(const EpiParams& p, int lane, int n
 }
 
 // One epilogue warp's share of a tile: rows row0 .. row0 + 31 of C (lane l owns row
-// row0 + l in TMEM, the first nvalid of them are real), columns n0 .. n0 + BN - 1.
+// row0 + l in TMEM, the first nvalid of them are real), columns n0 .. n0 + BN - 1, the
+// 32-column chunks ch0, ch0 + chs, ... of them (RoPE: of its heads).
 template <typename T, int BN, int KIND>
 __device__ __forceinline__ void epilogue(const EpiParams& p, const EpiPre& pre, uint32_t taddr, float* stg,
-                                         int lane, int nvalid, int row0, int n0, int split = 1, int mtile = 0) {
+                                         int lane, int nvalid, int row0, int n0, int ch0, int chs, int split = 1,
+                                         int mtile = 0) {
     const int cc = (lane & 7) * 4;                 // this lane's columns after the transpose
     if constexpr (KIND == EPI_STORE || KIND == EPI_STORE_F32 || KIND == EPI_OPROJ_PLAIN) {
         using OutT = std::conditional_t<KIND == EPI_STORE, T, float>;
         OutT* out = static_cast<OutT*>(p.out) + static_cast<size_t>(row0) * p.ldo;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = ch0; c < BN / 32; c += chs) {
             float v[32];
             ld_chunk(taddr, c, v);
             const int col = n0 + c * 32;
@@ -323,7 +335,7 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, const EpiPre& pre, 
         const float* sn = pre.sn;
         T* out = static_cast<T*>(p.out) + static_cast<size_t>(row0) * p.ldo;
 #pragma unroll 1
-        for (int hc = 0; hc < BN / 32; hc += hw_chunks) {
+        for (int hc = ch0 * hw_chunks; hc < BN / 32; hc += chs * hw_chunks) {
             const int head_col0 = n0 + hc * 32;
             const bool rotate = head_col0 < p.rope_limit;
 #pragma unroll 1
@@ -369,7 +381,7 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, const EpiPre& pre, 
         // completes both: y = x + a, h_next = A (.) h + B.e + a. Vector atomics need no reads
         // here, so the epilogue never waits on memory.
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = ch0; c < BN / 32; c += chs) {
             float v[32];
             ld_chunk(taddr, c, v);
             const int col = n0 + c * 32;
@@ -391,7 +403,7 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, const EpiPre& pre, 
         // Tile columns [0, BN/2) are gate rows (W1), [BN/2, BN) the matching up rows (W3).
         T* out = static_cast<T*>(p.out) + static_cast<size_t>(row0) * p.ldo + n0 / 2;
 #pragma unroll 1
-        for (int c = 0; c < BN / 64; ++c) {
+        for (int c = ch0; c < BN / 64; c += chs) {
             float g[32], u[32];
             ld_chunk(taddr, c, g);
             ld_chunk(taddr, c + BN / 64, u);
@@ -416,7 +428,7 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, const EpiPre& pre, 
             wt[it] = __shfl_sync(0xffffffffu, w, it * 4 + (lane >> 3));
         }
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = ch0; c < BN / 32; c += chs) {
             float v[32];
             ld_chunk(taddr, c, v);
             const int col = n0 + c * 32;
@@ -542,15 +554,16 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& args, const Grou
 //   empty[s]  each CTA: the leader's commit arrives on both CTAs' barriers when the MMAs
 //             that read stage s (in both CTAs) are done.
 //   tfull[b]  each CTA: the leader's commit arrives on both when accumulator b is complete.
-//   tempty[b] leader only: eight arrivals, the epilogue warps of both CTAs.
+//   tempty[b] leader only: one arrival per epilogue warp of both CTAs.
 // Every wait is bounded; on a timeout the roles stop and the kernel still passes its
 // closing barriers.
 template <typename T, int BN, int KIND, int CG>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(gemm_threads<KIND>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
                    const __grid_constant__ CUtensorMap tA2, const __grid_constant__ CUtensorMap tB2,
                    const GemmArgs args, const EpiParams epi) {
-    using C = TcCfg<BN, CG>;
+    constexpr int ES = epi_split<KIND>();
+    using C = TcCfg<BN, CG, ES>;
     constexpr bool kBf16 = std::is_same<T, bf16>::value;
     constexpr int kElemsPerRow = 128 / static_cast<int>(sizeof(T));   // K elements per stage
     constexpr int kTileRows = BM * CG;
@@ -586,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4 * CG);    // one arrival per epilogue warp of the pair
+            mbar_init(&tempty[b], 4 * ES * CG);   // one arrival per epilogue warp of the pair
         }
         mbar_fence_init();
     }
@@ -734,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&tfull[b], use & 1, epi.flags)) break;
             tc_fence_after();
             epilogue<T, BN, KIND>(epi, pre, tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN, stg, lane,
-                                  nvalid, tc.c_row0 + row_off, tc.n0, split, tc.mt);
+                                  nvalid, tc.c_row0 + row_off, tc.n0, (warp - 2) >> 2, ES, split, tc.mt);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -757,7 +770,7 @@ template <typename T, int BN, int KIND, int CG>
 rdt_status launch(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap* tA2,
                   const CUtensorMap* tB2, const GemmArgs& args, const EpiParams& epi,
                   cudaStream_t st) {
-    using C = TcCfg<BN, CG>;
+    using C = TcCfg<BN, CG, epi_split<KIND>()>;
     auto kern = gemm_tc_kernel<T, BN, KIND, CG>;
     constexpr int kTileRows = BM * CG;
     static int dev_ready[64] = {};         // per device: attributes set, co-resident clusters
@@ -774,7 +787,7 @@ rdt_status launch(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMa
         if (CG > 1) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(2 * mc);
-            cfg.blockDim = dim3(kThreads);
+            cfg.blockDim = dim3(gemm_threads<KIND>());
             cfg.dynamicSmemBytes = C::SMEM;
             cudaLaunchAttribute attr[1];
             attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -799,7 +812,7 @@ rdt_status launch(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMa
     const long total = mt * n_ntiles * (args.split_k > 1 ? args.split_k : 1);
     if (total <= 0) return RDT_OK;
     const int clusters = static_cast<int>(std::min<long>(total, max_clusters[dev]));
-    RDT_CUDA_TRY(launch_pdl_cluster(kern, dim3(clusters * CG), dim3(kThreads), C::SMEM, st, CG, tA, tB,
+    RDT_CUDA_TRY(launch_pdl_cluster(kern, dim3(clusters * CG), dim3(gemm_threads<KIND>()), C::SMEM, st, CG, tA, tB,
                                     tA2 ? *tA2 : tA, tB2 ? *tB2 : tB, args, epi));
     return RDT_OK;
 }

@@ -546,11 +546,13 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         TileChoice t = choose_tiles(grows, E + S, 2 * hid, kb_d, hid % 128 == 0, false, hid % 64 == 0, 1, mode);
         h->bn_up = t.bn;
         h->pair_up = t.pair;
-        // the down-projection's epilogue reduces every output into h_next; on pairs a CTA's
-        // share of it doubles and measured slower (24.3 vs 23.7 us), so it runs on pairs only
-        // when they are forced
+        // the down-projection's epilogue reduces every output into h_next. CTA pairs load a
+        // third less per SM (their B rows are split) and measured faster with many routed
+        // rows (65536 rows: 191 -> 179 us; 36864: 116 -> 113 us), not with few (4096 rows:
+        // the same), so pairs are allowed from 16384 rows on.
         // deterministic mode: no K split (its partial sums would meet in atomics)
-        t = choose_tiles(grows, E + S, d, kb_h, true, false, mode == 2, c.deterministic ? 1 : 4, mode);
+        t = choose_tiles(grows, E + S, d, kb_h, true, false, mode == 2 || (mode == 0 && grows >= 16384),
+                         c.deterministic ? 1 : 4, mode);
         h->bn_down = t.bn;
         h->pair_down = t.pair;
         h->split_down = t.split;
