@@ -102,6 +102,14 @@ typedef struct {
     int32_t da_heads;               /* depth attention: query heads (0: none); GQA, bf16,
                                      * head width head_dim = 64                          */
     int32_t da_kv_heads;            /* depth attention: KV heads (divides da_heads)     */
+    int32_t cp_size;                /* context parallelism: ranks (GPUs) one sequence is
+                                     * split over, 0 or 1: none, <= 8. Rank r holds
+                                     * positions [r * seq, (r + 1) * seq) of sequences of
+                                     * cp_size * seq positions (seq, batch as above: this
+                                     * rank's share). GQA, bf16, head_dim 64, seq % 128 ==
+                                     * 0, no decode cache, no ACT; rdt_cp_connect before the
+                                     * first rdt_loop_forward.                             */
+    int32_t cp_rank;                /* this rank, 0 .. cp_size - 1                       */
 } rdt_config;
 
 /* Weights, all DEVICE pointers, row-major [out, in]; element type = cfg.dtype
@@ -360,6 +368,33 @@ rdt_status rdt_profile_read(rdt_handle* h, rdt_kernel_stat* out, int max_entries
  * returns. Synchronises `stream`. Returns RDT_ERR_DEVICE_TIMEOUT, the expected outcome
  * (the device context stays usable); INVALID_ARG for a limit out of range. */
 rdt_status rdt_wait_probe(int64_t limit_ns, void* stream);
+
+/* Context parallelism (cfg.cp_size > 1; the pages run several GPUs only through torchrun,
+ * "Introducao ao OpenMythos" Passo 8, so the split of one long sequence over GPUs is this
+ * library's own). Per loop the QKV projection of rank r writes its rotated keys and values
+ * into its own gather buffer and, over peer memory (NVLink), into those of ranks r + 1 ..
+ * cp_size - 1, which attend over them; ranks signal one another through flag words in each
+ * other's memory with bounded waits (a wait that gives up records a timeout in the
+ * diagnostics). Everything else in the block is token-local.
+ *
+ * rdt_cp_buffers: this handle's gather buffer ([batch][cp_size * seq][2 n_kv_heads head_dim]
+ * bf16) and flag words, both device memory owned by the handle, for the caller to share
+ * with the other ranks (rdt_ipc_get_handle). INVALID_ARG without cp_size > 1.
+ * rdt_cp_connect: peer_kv[q] and peer_flags[q] (q = 0 .. cp_size - 1) are rank q's two
+ * buffers as device pointers valid in this process (rdt_ipc_open_handle, or the buffers of
+ * another handle on the same device); entry cp_rank is ignored. The pointers must stay
+ * valid while the handle runs loops; every rank must connect before any rank's first
+ * rdt_loop_forward, and every rank must run the same loop counts in the same order (their
+ * calls wait for one another). */
+rdt_status rdt_cp_buffers(rdt_handle* h, void** kv, size_t* kv_bytes, void** flags, size_t* flag_bytes);
+rdt_status rdt_cp_connect(rdt_handle* h, void* const* peer_kv, void* const* peer_flags);
+
+/* CUDA inter-process handles of device memory for sharing the buffers above between
+ * processes (64 bytes, opaque). rdt_ipc_open_handle maps another process's allocation into
+ * this one (peer access enabled on demand); rdt_ipc_close_handle unmaps it. */
+rdt_status rdt_ipc_get_handle(const void* dev_ptr, void* handle64);
+rdt_status rdt_ipc_open_handle(const void* handle64, void** dev_ptr);
+rdt_status rdt_ipc_close_handle(void* dev_ptr);
 
 const char* rdt_status_string(rdt_status s);
 const char* rdt_last_error(void);

@@ -20,7 +20,7 @@ from typing import Dict, Optional
 import numpy as np
 
 __all__ = ["RDT", "RdtError", "library_path", "load_library", "make_config", "device_weights",
-           "EXPORTED"]
+           "EXPORTED", "ipc_get_handle", "ipc_open_handle", "ipc_close_handle", "cp_connect_ranks"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_PKG, "librdt.so")
@@ -38,7 +38,8 @@ EXPORTED = ("rdt_create", "rdt_attn_forward", "rdt_moe_forward", "rdt_loop_forwa
             "rdt_status_string", "rdt_last_error", "rdt_destroy", "rdt_matmul", "rdt_attention",
             "rdt_profile", "rdt_profile_read", "rdt_moe_route_noalloc", "rdt_moe_route_noalloc_status",
             "rdt_set_act", "rdt_loop_forward_act", "rdt_wait_probe", "rdt_decode_prefill",
-            "rdt_decode_step")
+            "rdt_decode_step", "rdt_cp_buffers", "rdt_cp_connect", "rdt_ipc_get_handle",
+            "rdt_ipc_open_handle", "rdt_ipc_close_handle")
 
 
 class RdtError(RuntimeError):
@@ -55,7 +56,7 @@ class RdtConfig(ctypes.Structure):
         (n, ctypes.c_int32) for n in ("n_experts", "top_k", "n_shared", "expert_hidden",
                                       "lora_rank", "n_lora", "b_kind", "inject_e", "max_loops",
                                       "gemm_tiles", "deterministic", "max_decode", "da_heads",
-                                      "da_kv_heads")]
+                                      "da_kv_heads", "cp_size", "cp_rank")]
 
 
 WEIGHT_FIELDS = ("A", "B", "norm1", "norm2", "wq", "wk", "wv", "wo", "w_dq", "q_norm", "w_uq",
@@ -120,11 +121,18 @@ def load_library() -> ctypes.CDLL:
                                      ctypes.POINTER(ctypes.c_int64)]
     lib.rdt_attention.argtypes = [i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                   ctypes.c_float, vp]
+    sz = ctypes.POINTER(ctypes.c_size_t)
+    lib.rdt_cp_buffers.argtypes = [vp, ctypes.POINTER(vp), sz, ctypes.POINTER(vp), sz]
+    lib.rdt_cp_connect.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp)]
+    lib.rdt_ipc_get_handle.argtypes = [vp, vp]
+    lib.rdt_ipc_open_handle.argtypes = [vp, ctypes.POINTER(vp)]
+    lib.rdt_ipc_close_handle.argtypes = [vp]
     for f in ("rdt_create", "rdt_attn_forward", "rdt_moe_forward", "rdt_loop_forward",
               "rdt_loop_forward_host", "rdt_set_trace", "rdt_get_diagnostics", "rdt_memory_bytes",
               "rdt_matmul", "rdt_attention", "rdt_profile", "rdt_profile_read", "rdt_moe_route_noalloc",
               "rdt_set_act", "rdt_loop_forward_act", "rdt_moe_route_noalloc_status", "rdt_wait_probe",
-              "rdt_decode_prefill", "rdt_decode_step"):
+              "rdt_decode_prefill", "rdt_decode_step", "rdt_cp_buffers", "rdt_cp_connect",
+              "rdt_ipc_get_handle", "rdt_ipc_open_handle", "rdt_ipc_close_handle"):
         getattr(lib, f).restype = i32
     _LIB = lib
     return lib
@@ -137,8 +145,10 @@ def _check(status: int) -> None:
 
 
 def make_config(wl, max_loops: int = 16, batch: Optional[int] = None, seq: Optional[int] = None,
-                gemm_tiles: int = 0, deterministic: bool = False, max_decode: int = 0) -> RdtConfig:
-    """Fill the C config from any object with the block's hyper-parameters as attributes."""
+                gemm_tiles: int = 0, deterministic: bool = False, max_decode: int = 0,
+                cp_size: int = 0, cp_rank: int = 0) -> RdtConfig:
+    """Fill the C config from any object with the block's hyper-parameters as attributes.
+    With cp_size > 1, seq is this rank's share of each sequence."""
     c = RdtConfig()
     c.dtype = RDT_BF16 if wl.dtype == "bf16" else RDT_F32
     c.batch = wl.batch if batch is None else batch
@@ -169,7 +179,58 @@ def make_config(wl, max_loops: int = 16, batch: Optional[int] = None, seq: Optio
     c.max_decode = max_decode
     c.da_heads = getattr(wl, "da_heads", 0)
     c.da_kv_heads = getattr(wl, "da_kv_heads", 0)
+    c.cp_size = cp_size
+    c.cp_rank = cp_rank
     return c
+
+
+def ipc_get_handle(dev_ptr: int) -> bytes:
+    """The 64-byte inter-process handle of a device allocation (rdt_ipc_get_handle)."""
+    lib = load_library()
+    buf = ctypes.create_string_buffer(64)
+    _check(lib.rdt_ipc_get_handle(ctypes.c_void_p(dev_ptr), buf))
+    return buf.raw
+
+
+def ipc_open_handle(handle: bytes) -> int:
+    """Map another process's allocation; returns its device address here."""
+    lib = load_library()
+    if len(handle) != 64:
+        raise ValueError("an IPC handle has 64 bytes")
+    ptr = ctypes.c_void_p()
+    _check(lib.rdt_ipc_open_handle(ctypes.create_string_buffer(handle, 64), ctypes.byref(ptr)))
+    return ptr.value
+
+
+def ipc_close_handle(dev_ptr: int) -> None:
+    _check(load_library().rdt_ipc_close_handle(ctypes.c_void_p(dev_ptr)))
+
+
+def cp_connect_ranks(handle, rank: int, size: int, all_gather, get_handle=ipc_get_handle,
+                     open_handle=ipc_open_handle):
+    """Connect the context-parallel ranks of one sequence, one process per GPU.
+
+    Every rank calls this collectively. all_gather(obj) returns the list of every rank's
+    obj (torch.distributed.all_gather_object, for example). Each rank publishes the
+    inter-process handles of its gather buffer and flag words, opens the other ranks',
+    and passes the mapped addresses to rdt_cp_connect. Returns the opened addresses (close
+    them with ipc_close_handle once the handle is destroyed)."""
+    kv, kv_bytes, flags, flag_bytes = handle.cp_buffers()
+    mine = (rank, get_handle(kv), get_handle(flags))
+    every = all_gather(mine)
+    if len(every) != size or sorted(r for r, _, _ in every) != list(range(size)):
+        raise RuntimeError(f"context parallelism: expected ranks 0 .. {size - 1}, got "
+                           f"{sorted(r for r, _, _ in every)}")
+    peer_kv, peer_flags, opened = [0] * size, [0] * size, []
+    for r, hkv, hfl in every:
+        if r == rank:
+            peer_kv[r], peer_flags[r] = kv, flags
+            continue
+        peer_kv[r] = open_handle(hkv)
+        peer_flags[r] = open_handle(hfl)
+        opened += [peer_kv[r], peer_flags[r]]
+    handle.cp_connect(peer_kv, peer_flags)
+    return opened
 
 
 def device_weights(arrays: Dict[str, np.ndarray], bf16: bool, device="cuda"):
@@ -326,6 +387,21 @@ class RDT:
         n = ctypes.c_size_t()
         _check(self._lib.rdt_memory_bytes(self._h, ctypes.byref(n)))
         return n.value
+
+    def cp_buffers(self):
+        """(gather buffer address, its bytes, flag words address, their bytes) of this rank."""
+        kv, fl = ctypes.c_void_p(), ctypes.c_void_p()
+        kvb, flb = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(self._lib.rdt_cp_buffers(self._h, ctypes.byref(kv), ctypes.byref(kvb), ctypes.byref(fl),
+                                        ctypes.byref(flb)))
+        return kv.value, kvb.value, fl.value, flb.value
+
+    def cp_connect(self, peer_kv, peer_flags):
+        """Every rank's gather buffer and flag words as device addresses in this process."""
+        n = len(peer_kv)
+        kv = (ctypes.c_void_p * n)(*[ctypes.c_void_p(p) for p in peer_kv])
+        fl = (ctypes.c_void_p * n)(*[ctypes.c_void_p(p) for p in peer_flags])
+        _check(self._lib.rdt_cp_connect(self._h, kv, fl))
 
     def close(self):
         if getattr(self, "_h", None):

@@ -63,6 +63,10 @@ rdt_status launch_f32(const AttnArgs& a, cudaStream_t st) {
 
 rdt_status attention(bool bf16_elems, const AttnArgs& a, cudaStream_t st) {
     if (bf16_elems) return attention_tc(a, st);
+    if (a.q_off != 0 || (a.kv_seq != 0 && a.kv_seq != a.seq)) {
+        set_error("attention: a query offset needs bf16");
+        return RDT_ERR_UNSUPPORTED;
+    }
     {
         if (a.dqk == 32 && a.dv == 32) return launch_f32<32, 32>(a, st);
         if (a.dqk == 64 && a.dv == 64) return launch_f32<64, 64>(a, st);

@@ -148,6 +148,7 @@ struct AttnCfg {
 
 struct AttnTcArgs {
     int seq, hq, hkv, q_hstride, k_hstride, v_hstride, ldo, dv_out;
+    int q_off, kv_seq;   // queries at positions q_off + 0 .. seq - 1 of kv_seq keys (attn96 only)
     int nqb, npairs, batch, sms;   // query blocks and CTA work items (of QT blocks) per sequence
     float scale_log2;
     void* o;
@@ -541,12 +542,14 @@ __global__ void __launch_bounds__(K96Cfg<QT>::THREADS, K96Cfg<QT>::BLOCKS_PER_SM
     const int h = (rank % per_p) % a.hq;
     const int b = (rank % per_p) / a.hq;
     const int g = (h * a.hkv) / a.hq;
-    const int row0 = b * a.seq;
+    const int row0 = b * a.seq;                 // first query row of this sequence
+    const int kvrow0 = b * a.kv_seq;            // first key / value row of this sequence
     const int qb0 = pr * QT;
-    // tile t (query block qb0 + t) sees the key blocks that start at or before its last row
-    const int nkv = (a.seq + BK - 1) / BK;
+    // tile t (query block qb0 + t, positions from q_off + 128 (qb0 + t)) sees the key blocks
+    // that start at or before its last position
+    const int nkv = (a.kv_seq + BK - 1) / BK;
     const auto nkb_of = [&](int t) {
-        return qb0 + t < a.nqb ? min(((qb0 + t + 1) * kBQ + BK - 1) / BK, nkv) : 0;
+        return qb0 + t < a.nqb ? min((a.q_off + (qb0 + t + 1) * kBQ + BK - 1) / BK, nkv) : 0;
     };
     int n_kb = 0;
 #pragma unroll
@@ -608,8 +611,8 @@ __global__ void __launch_bounds__(K96Cfg<QT>::THREADS, K96Cfg<QT>::BLOCKS_PER_SM
                         ok = mbar_wait(&empty[t * NS + s], ((j / NS) & 1) ^ 1, a.flags);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&full[s], 2 * C::KV_BYTES);
-                tma_load_2d(smem + C::OFF_K + s * C::KV_BYTES, &tk, &full[s], g * a.k_hstride, row0 + j * BK);
-                tma_load_2d(smem + C::OFF_V + s * C::KV_BYTES, &tv, &full[s], g * a.v_hstride, row0 + j * BK);
+                tma_load_2d(smem + C::OFF_K + s * C::KV_BYTES, &tk, &full[s], g * a.k_hstride, kvrow0 + j * BK);
+                tma_load_2d(smem + C::OFF_V + s * C::KV_BYTES, &tv, &full[s], g * a.v_hstride, kvrow0 + j * BK);
             }
         }
       } else if (warp <= QT) {
@@ -678,7 +681,7 @@ __global__ void __launch_bounds__(K96Cfg<QT>::THREADS, K96Cfg<QT>::BLOCKS_PER_SM
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
         const uint32_t o_col = C::O_COL + 64 * t;
         const float sl = a.scale_log2;
-        const int kmax_row = min(qpos, a.seq - 1);     // last key the row may see
+        const int kmax_row = min(a.q_off + qpos, a.kv_seq - 1);   // last key the row may see
         float m_ref = -INFINITY, l = 0.0f;
         bool ok = true;
 #pragma unroll 1
@@ -812,8 +815,10 @@ rdt_status launch_k96(const AttnArgs& a, cudaStream_t st) {
     const long rows = static_cast<long>(a.batch) * a.seq;
     CUtensorMap tq, tk, tv;
     RDT_TRY(make_tmap_2d(&tq, a.q, true, a.ldq, rows, static_cast<uint64_t>(a.ldq) * 2, 64, 128));
-    RDT_TRY(make_tmap_2d(&tk, a.k, true, a.ldk, rows, static_cast<uint64_t>(a.ldk) * 2, 64, C::BK));
-    RDT_TRY(make_tmap_2d(&tv, a.v, true, a.ldv, rows, static_cast<uint64_t>(a.ldv) * 2, 64, C::BK));
+    const int kv_seq = a.kv_seq > 0 ? a.kv_seq : a.seq;
+    const long kv_rows = static_cast<long>(a.batch) * kv_seq;
+    RDT_TRY(make_tmap_2d(&tk, a.k, true, a.ldk, kv_rows, static_cast<uint64_t>(a.ldk) * 2, 64, C::BK));
+    RDT_TRY(make_tmap_2d(&tv, a.v, true, a.ldv, kv_rows, static_cast<uint64_t>(a.ldv) * 2, 64, C::BK));
     AttnTcArgs ta{};
     ta.seq = a.seq;
     ta.hq = a.hq;
@@ -823,6 +828,8 @@ rdt_status launch_k96(const AttnArgs& a, cudaStream_t st) {
     ta.v_hstride = a.v_hstride;
     ta.ldo = a.ldo;
     ta.dv_out = a.dv;
+    ta.q_off = a.q_off;
+    ta.kv_seq = kv_seq;
     ta.scale_log2 = a.scale * 1.4426950408889634f;
     ta.o = a.o;
     ta.flags = a.flags;
@@ -908,6 +915,10 @@ rdt_status launch_choose(const AttnArgs& a, cudaStream_t st) {
 
 rdt_status attention_tc(const AttnArgs& a, cudaStream_t st) {
     if (a.dqk == 64 && a.dv == 64) return launch_k96_choose(a, st);
+    if (a.q_off != 0 || (a.kv_seq != 0 && a.kv_seq != a.seq)) {
+        set_error("tensor-core attention: a query offset needs head width 64");
+        return RDT_ERR_UNSUPPORTED;
+    }
     if (a.dqk == 160 && a.dv == 128 && a.v == a.k) return launch_choose<160, 128, true>(a, st);
     // 160-wide keys with values of their own: one tile per CTA (two would not fit in shared memory)
     if (a.dqk == 160 && a.dv == 128) return launch_tc<160, 128, false, 1>(a, st);

@@ -125,6 +125,34 @@ __device__ __forceinline__ void store_chunk(float* stg, int lane, const float (&
     }
 }
 
+// store_chunk for the QKV projection: the chunk goes to base as above and, when it holds key
+// or value columns (col >= cp_col0) and context parallelism is on, also to every rank's
+// gather buffer (this rank's and, over peer memory, its peers'), rows renumbered to the
+// sequence positions of this rank: local row r -> (r / seq) * cp_seq_tot + cp_row_off +
+// r % seq. One transpose serves all destinations.
+template <typename OutT>
+__device__ __forceinline__ void store_chunk_cp(const EpiParams& p, float* stg, int lane, const float (&v)[32],
+                                               OutT* base, int nvalid, int row0, int col) {
+    stage_put(stg, lane, v);
+    const int cc = (lane & 7) * 4;
+    const bool push = p.cp_n > 0 && col >= p.cp_col0;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+        const int rr = it * 4 + (lane >> 3);
+        float o[4];
+        stage_get(stg, lane, it, o);
+        if (rr >= nvalid) continue;
+        store4(base + static_cast<size_t>(rr) * p.ldo + cc, o);
+        if (push) {
+            const int r = row0 + rr;
+            const size_t grow = static_cast<size_t>(r / p.seq) * p.cp_seq_tot + p.cp_row_off + r % p.seq;
+            const size_t off = grow * p.cp_w + (col - p.cp_col0) + cc;
+#pragma unroll 1
+            for (int q = 0; q < p.cp_n; ++q) store4(static_cast<OutT*>(p.cp_dst[q]) + off, o);
+        }
+    }
+}
+
 // ----------------------------------------------------------------------------- epilogues
 
 // Router top-k: keep the KMAX best (score = logit + bias) in registers, visiting experts in
@@ -281,7 +309,7 @@ __device__ __forceinline__ void epilogue_pre(const EpiParams& p, int lane, int n
     if constexpr (KIND == EPI_ROPE) {
         // The angle tables are [rot/2][seq]: for a fixed frequency the lanes (consecutive
         // positions) read consecutive floats.
-        const int pos = (row0 + lane) % p.seq + (p.pos_dev ? *p.pos_dev : 0);
+        const int pos = (row0 + lane) % p.seq + p.pos_off + (p.pos_dev ? *p.pos_dev : 0);
         const int half = p.rot_dim / 2;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -354,8 +382,8 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, const EpiPre& pre, 
                             v1[i] = x2 * cs[i] + x1 * sn[i];
                         }
                         if (keep) {
-                            store_chunk(stg, lane, v0, out + col, p.ldo, nvalid);
-                            store_chunk(stg, lane, v1, out + col + 32, p.ldo, nvalid);
+                            store_chunk_cp(p, stg, lane, v0, out + col, nvalid, row0, col);
+                            store_chunk_cp(p, stg, lane, v1, out + col + 32, nvalid, row0, col + 32);
                         }
                         c += 1;
                     } else {
@@ -367,12 +395,12 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, const EpiPre& pre, 
                             v[i] = x1 * cs[i] - x2 * sn[i];
                             v[i + 16] = x2 * cs[i] + x1 * sn[i];
                         }
-                        if (keep) store_chunk(stg, lane, v, out + col, p.ldo, nvalid);
+                        if (keep) store_chunk_cp(p, stg, lane, v, out + col, nvalid, row0, col);
                     }
                 } else {
                     float v[32];
                     ld_chunk(taddr, hc + c, v);
-                    if (keep) store_chunk(stg, lane, v, out + col, p.ldo, nvalid);
+                    if (keep) store_chunk_cp(p, stg, lane, v, out + col, nvalid, row0, col);
                 }
             }
         }

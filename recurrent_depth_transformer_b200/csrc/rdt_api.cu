@@ -99,6 +99,16 @@ struct rdt_handle {
     void *stage_h0 = nullptr, *stage_e = nullptr;
     float* stage_out = nullptr;
 
+    // context parallelism (cfg.cp_size > 1): this rank's gather buffer of every rank's rotated
+    // keys and values ([batch][cp_size * seq][2 nkv]), its flag words, and the peers' (device
+    // pointers valid in this process; the rank's own entries point to its own buffers)
+    int cp_size = 1, cp_rank = 0;
+    void* cp_kv = nullptr;
+    unsigned* cp_flags = nullptr;
+    void* cp_peer_kv[kMaxCp] = {};
+    unsigned* cp_peer_flags[kMaxCp] = {};
+    bool cp_connected = false;
+
     // ACT halting (rdt_set_act): head, and per-token running sum / loops run
     bool act_set = false;
     float* act_w = nullptr;
@@ -158,13 +168,13 @@ constexpr int kFillerRows = 256;
 // kernel classes reported by rdt_profile_read
 enum Kind { K_HOIST, K_NORM1, K_GEMM_QKV, K_GEMM_LAT, K_MLA_NORM, K_GEMM_Q, K_ATTENTION,
             K_GEMM_O, K_NORM2, K_ROUTER, K_DISPATCH, K_GEMM_UP, K_GEMM_DOWN, K_CHECK, K_DENSE_B, K_ACT,
-            K_COMBINE, K_CACHE, K_DEC_ATTN, K_DA_QKV, K_DA_ATTN, K_DA_O, K_COUNT };
+            K_COMBINE, K_CACHE, K_DEC_ATTN, K_DA_QKV, K_DA_ATTN, K_DA_O, K_CP_SYNC, K_COUNT };
 const char* const kKindName[K_COUNT] = {"hoist", "norm1", "gemm_qkv", "gemm_latent", "mla_latent_norm",
                                          "gemm_q_absorbed", "attention", "gemm_o",
                                          "norm2", "router_topk", "moe_dispatch", "gemm_up", "gemm_down",
                                          "check_finite", "dense_injection", "act_halting", "moe_combine", "kv_cache_append",
                                          "decode_attention", "gemm_qkv_depth", "depth_attention",
-                                         "gemm_o_depth"};
+                                         "gemm_o_depth", "cp_sync"};
 
 // During graph capture the events become event-record nodes of the graph (external
 // records), so that every replay records them again; they are then kept apart from the
@@ -285,6 +295,17 @@ rdt_status validate_config(const rdt_config* c) {
     if (c->max_decode < 0 || c->max_decode > (1 << 20)) return bad("max_decode");
     if (c->max_decode > 0 && c->dtype != RDT_BF16) return uns("decode with a KV cache is provided in bf16");
     if (static_cast<long long>(c->seq) + c->max_decode > (1 << 24)) return uns("seq + max_decode too large");
+    if (c->cp_size < 0 || c->cp_size > kMaxCp) return bad("cp_size must be in [0, 8]");
+    if (c->cp_size > 1) {
+        if (c->cp_rank < 0 || c->cp_rank >= c->cp_size) return bad("cp_rank must be in [0, cp_size)");
+        if (c->attn_type != RDT_GQA || c->dtype != RDT_BF16 || c->head_dim != 64)
+            return uns("context parallelism is provided for bf16 GQA with head_dim 64");
+        if (c->seq % 128) return uns("context parallelism: seq (this rank's share) must be a multiple of 128");
+        if (c->max_decode > 0) return uns("context parallelism with a decode cache");
+        if (static_cast<long long>(c->seq) * c->cp_size > (1 << 24)) return uns("cp_size * seq too large");
+    } else if (c->cp_rank != 0) {
+        return bad("cp_rank without cp_size > 1");
+    }
     if (c->da_heads < 0 || c->da_kv_heads < 0) return bad("da_heads / da_kv_heads");
     if (c->da_heads > 0) {
         if (c->attn_type != RDT_GQA || c->dtype != RDT_BF16 || c->head_dim != 64)
@@ -654,7 +675,10 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
 
     // RoPE tables [rot/2][s_cap] (frequency-major, so that consecutive positions are adjacent)
     // from double-precision angles, for every position a sequence may reach
-    h->s_cap = c.seq + c.max_decode;
+    // (context parallelism: this rank's positions start at cp_rank * seq)
+    h->cp_size = c.cp_size > 1 ? c.cp_size : 1;
+    h->cp_rank = c.cp_size > 1 ? c.cp_rank : 0;
+    h->s_cap = c.seq * h->cp_size + c.max_decode;
     {
         const int half = h->rot / 2;
         const int P = h->s_cap;
@@ -771,6 +795,15 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         const int dv = c.attn_type == RDT_GQA ? c.head_dim : c.kv_lora_rank;
         RDT_TRY(dev_alloc(h, &h->dec_part, static_cast<size_t>(c.batch) * c.n_heads * decode_chunks(h->s_cap) *
                                                (dv + 2) * 4));
+    }
+    if (h->cp_size > 1) {
+        // zeroed: rows no rank writes here (later ranks' positions) meet P = 0 in the PV
+        // product, and 0 * garbage could be NaN
+        RDT_TRY(dev_alloc(h, &h->cp_kv, static_cast<size_t>(c.batch) * h->s_cap * 2 * c.n_kv_heads * c.head_dim * es,
+                          true));
+        RDT_TRY(dev_alloc(h, &h->cp_flags, 256, true));
+        h->cp_peer_kv[h->cp_rank] = h->cp_kv;
+        h->cp_peer_flags[h->cp_rank] = h->cp_flags;
     }
     RDT_TRY(dev_alloc(h, &h->stage_h0, nd * es));
     RDT_TRY(dev_alloc(h, &h->stage_e, nd * es));
@@ -924,7 +957,28 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         ep.rot_off = 0;
         ep.rot_dim = c.head_dim;
         ep.rope_limit = h->nq + h->nkv;
+        const bool cp = h->cp_size > 1;
+        CpSyncArgs cs{};
+        if (cp) {
+            // this rank's positions start at cp_rank * seq; its rotated keys and values also go
+            // to the gather buffers of this rank and the later ones (the causal mask gives rank
+            // q the keys of ranks 0 .. q), once those have finished with the previous loop's
+            cs.flags = h->cp_flags;
+            for (int q = 0; q < h->cp_size; ++q) cs.peer_flags[q] = h->cp_peer_flags[q];
+            cs.rank = h->cp_rank;
+            cs.size = h->cp_size;
+            cs.status = h->flags;
+            TIMED(h, K_CP_SYNC, 1, st, cp_wait_consumed(cs, st));
+            ep.pos_off = h->cp_rank * c.seq;
+            ep.cp_n = h->cp_size - h->cp_rank;
+            for (int q = h->cp_rank; q < h->cp_size; ++q) ep.cp_dst[q - h->cp_rank] = h->cp_peer_kv[q];
+            ep.cp_col0 = h->nq;
+            ep.cp_w = 2 * h->nkv;
+            ep.cp_seq_tot = h->cp_size * c.seq;
+            ep.cp_row_off = h->cp_rank * c.seq;
+        }
         TIMED(h, K_GEMM_QKV, 1, st, gemm_tc(h->bf, h->bn_qkv, h->m_xn, h->m_wqkv[li], nullptr, nullptr, ga, ep, st));
+        if (cp) TIMED(h, K_CP_SYNC, 1, st, cp_ready(cs, st));
         if (cache_t)   // loop t's rotated keys and values of these positions: [K | V] per row
             TIMED(h, K_CACHE, 1, st, cache_append(h->qkv, h->nqkv, h->nq, h->cache_w, cache_t, h->s_cap, pos_seq,
                                                   pos_dev, N, st));
@@ -941,6 +995,14 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         at.dqk = c.head_dim;
         at.dv = c.head_dim;
         at.scale = 1.0f / std::sqrt(static_cast<float>(c.head_dim));
+        if (cp) {   // every rank's keys and values up to this rank's positions, from the gather buffer
+            at.k = h->cp_kv;
+            at.ldk = 2 * h->nkv;
+            at.v = static_cast<const char*>(h->cp_kv) + static_cast<size_t>(h->nkv) * h->esz;
+            at.ldv = 2 * h->nkv;
+            at.q_off = h->cp_rank * c.seq;
+            at.kv_seq = h->cp_size * c.seq;
+        }
     } else {
         const int ql = c.q_lora_rank, kvl = c.kv_lora_rank, rp = c.qk_rope_dim;
         // latent projection -> fp32 [N, ql + kvl + rope]
@@ -1043,6 +1105,15 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         TIMED(h, K_DEC_ATTN, 2, st, decode_attention(da, st));
     } else {
         TIMED(h, K_ATTENTION, 1, st, attention(h->bf, at, st));
+        if (h->cp_size > 1) {
+            CpSyncArgs cs{};
+            cs.flags = h->cp_flags;
+            for (int q = 0; q < h->cp_size; ++q) cs.peer_flags[q] = h->cp_peer_flags[q];
+            cs.rank = h->cp_rank;
+            cs.size = h->cp_size;
+            cs.status = h->flags;
+            TIMED(h, K_CP_SYNC, 1, st, cp_consumed(cs, st));
+        }
     }
 
     GemmArgs go{};
@@ -1292,6 +1363,15 @@ void drop_graph(rdt_handle* h) {
 // and launches the graph, later ones only launch it. Tracing or profiling runs eagerly.
 rdt_status run_loop(rdt_handle* h, const void* h0, const void* e, int T, float* out, cudaStream_t st,
                     bool act = false, int32_t* n_loops = nullptr) {
+    if (h->cp_size > 1 && !h->cp_connected) {
+        set_error("context parallelism: rdt_cp_connect has not been called on this handle");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (h->cp_size > 1 && act) {
+        // ranks that stop at different loops would leave their peers waiting
+        set_error("context parallelism with ACT halting is not provided");
+        return RDT_ERR_UNSUPPORTED;
+    }
     const bool graphable = (!h->prof_on || h->prof_graph) && !h->tr_idx && !h->tr_w && !h->tr_h;
     if (!graphable) return loop_impl(h, h0, e, T, out, act, n_loops, st);
     rdt_handle::GraphKey key;
@@ -1432,6 +1512,10 @@ rdt_status rdt_attn_forward(rdt_handle* h, const void* x, int loop, float* a_out
     if (!h) {
         set_error("handle is NULL");
         return RDT_ERR_INVALID_ARG;
+    }
+    if (h->cp_size > 1) {
+        set_error("context parallelism runs through rdt_loop_forward only");
+        return RDT_ERR_UNSUPPORTED;
     }
     set_mode(h, 0);
     RDT_TRY(check_ptr(x, "x"));
@@ -1804,6 +1888,50 @@ rdt_status rdt_memory_bytes(const rdt_handle* h, size_t* bytes) {
         return RDT_ERR_INVALID_ARG;
     }
     *bytes = h->bytes;
+    return RDT_OK;
+}
+
+rdt_status rdt_cp_buffers(rdt_handle* h, void** kv, size_t* kv_bytes, void** flags, size_t* flag_bytes) {
+    if (!h || !kv || !kv_bytes || !flags || !flag_bytes) {
+        set_error("rdt_cp_buffers: NULL argument");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (h->cp_size < 2) {
+        set_error("rdt_cp_buffers: the handle was created without cp_size > 1");
+        return RDT_ERR_INVALID_ARG;
+    }
+    const rdt_config& c = h->cfg;
+    *kv = h->cp_kv;
+    *kv_bytes = static_cast<size_t>(c.batch) * h->s_cap * 2 * h->nkv * h->esz;
+    *flags = h->cp_flags;
+    *flag_bytes = 256;
+    return RDT_OK;
+}
+
+rdt_status rdt_cp_connect(rdt_handle* h, void* const* peer_kv, void* const* peer_flags) {
+    if (!h || !peer_kv || !peer_flags) {
+        set_error("rdt_cp_connect: NULL argument");
+        return RDT_ERR_INVALID_ARG;
+    }
+    if (h->cp_size < 2) {
+        set_error("rdt_cp_connect: the handle was created without cp_size > 1");
+        return RDT_ERR_INVALID_ARG;
+    }
+    for (int q = 0; q < h->cp_size; ++q) {
+        if (q == h->cp_rank) continue;
+        if (!peer_kv[q] || !peer_flags[q] || (reinterpret_cast<uintptr_t>(peer_kv[q]) & 15) ||
+            (reinterpret_cast<uintptr_t>(peer_flags[q]) & 15)) {
+            set_error("rdt_cp_connect: rank " + std::to_string(q) + "'s buffers are NULL or not 16-byte aligned");
+            return RDT_ERR_INVALID_ARG;
+        }
+    }
+    for (int q = 0; q < h->cp_size; ++q) {
+        if (q == h->cp_rank) continue;
+        h->cp_peer_kv[q] = peer_kv[q];
+        h->cp_peer_flags[q] = static_cast<unsigned*>(peer_flags[q]);
+    }
+    drop_graph(h);              // captured graphs hold the previous peers
+    h->cp_connected = true;
     return RDT_OK;
 }
 

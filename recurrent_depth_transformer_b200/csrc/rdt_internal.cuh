@@ -389,6 +389,8 @@ enum EpiKind {
     EPI_TOPK = 7        // router: top-k of the row's logits, gate weights, histogram
 };
 
+constexpr int kMaxCp = 8;   // context-parallel ranks at most
+
 struct EpiParams {
     int kind;
     void* out;             // EPI_STORE / ROPE / SWIGLU: output base; OPROJ_PLAIN: a_out
@@ -404,6 +406,12 @@ struct EpiParams {
     int rot_off;           // rotary part starts at this column inside a head
     int rot_dim;           // rotary width
     int rope_limit;        // columns >= rope_limit are not rotated (V heads)
+    int pos_off;           // context parallelism: position of this rank's first row of a sequence
+    // context parallelism: the rotated K and V columns [cp_col0, cp_col0 + cp_w) of every row
+    // are also stored into cp_n gather buffers (this rank's and its peers': [batch][cp_seq_tot]
+    // [cp_w]), row (r / seq) * cp_seq_tot + cp_row_off + r % seq
+    void* cp_dst[kMaxCp];
+    int cp_n, cp_col0, cp_w, cp_seq_tot, cp_row_off;
     // O-projection loop epilogue: y and h_next hold x and A (.) h + B.e (RMSNorm1 wrote them)
     float* y;              // += a   ->  x + a
     float* h_next;         // += a   ->  A*h + Be + a (the MoE adds its share later)
@@ -474,10 +482,31 @@ struct AttnArgs {
     int batch, seq, hq, hkv, dqk, dv;
     float scale;
     int* flags;
+    // context parallelism (head width 64 only): the queries are positions q_off .. q_off +
+    // seq - 1 of sequences whose keys and values have kv_seq rows each (0: kv_seq = seq,
+    // q_off = 0)
+    int q_off, kv_seq;
 };
 rdt_status attention(bool bf16_elems, const AttnArgs& a, cudaStream_t st);
 // tcgen05 kernel: (dqk, dv) = (64, 64), or (160, 128) with v == k (absorbed MLA)
 rdt_status attention_tc(const AttnArgs& a, cudaStream_t st);
+
+// Context-parallel synchronisation (cp.cu). flags: this rank's words [READY 0..7 | CONS
+// 0..7 | epoch]; peer_flags[q]: rank q's (this rank's own at q == rank). A loop's epoch is
+// the handle's epoch + 1.
+constexpr int kCpReady = 0, kCpCons = kMaxCp, kCpEpoch = 2 * kMaxCp, kCpFlagWords = 2 * kMaxCp + 1;
+struct CpSyncArgs {
+    unsigned* flags;
+    unsigned* peer_flags[kMaxCp];
+    int rank, size;
+    int* status;
+};
+// before the push of loop e: ranks q > rank have consumed loop e - 1's keys
+rdt_status cp_wait_consumed(const CpSyncArgs& a, cudaStream_t st);
+// after the push: tell ranks q > rank that loop e's keys are there, wait for ranks s < rank
+rdt_status cp_ready(const CpSyncArgs& a, cudaStream_t st);
+// after the attention: tell ranks s < rank that loop e's keys are consumed; epoch = e
+rdt_status cp_consumed(const CpSyncArgs& a, cudaStream_t st);
 
 // Row kernels (rowops.cu).
 struct Norm1Args {
