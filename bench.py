@@ -11,11 +11,12 @@ step is reported.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--workload NAME] [--loops T] [--act] [--all]
-                    [--decode] [--kernel attention]
+                    [--decode] [--kernel attention] [--cp]
 
 --decode times rdt_decode_step (one new token per sequence, T loops, over a prompt of the
 workload's length) instead. `--kernel attention` times rdt_attention alone on the workload's
-sequence-attention shape (the command the attention kernel's ncu captures run).
+sequence-attention shape (the command the attention kernel's ncu captures run). `--cp`
+splits one sequence of the workload over the N GPUs (context parallelism; strong scaling).
 
 --gpus N > 1 runs one process per GPU (re-launched under torch.distributed.run when not
 started by it): every rank runs a replica of the workload on inputs of its own (no
@@ -757,6 +758,89 @@ def bench_attention(args, dev, rank, world):
     }
 
 
+def bench_cp(args, dev, rank, world):
+    """Context parallelism: one sequence of the workload split over the ranks (rank r holds
+    positions [r S / N, (r + 1) S / N)); the keys of every loop travel over peer memory from
+    the QKV projection's epilogue. The whole job's tokens per step are the workload's, so the
+    scaling is strong."""
+    import torch
+    import torch.distributed as dist
+
+    import recurrent_depth_transformer_b200 as R
+    from workloads import by_name, generate
+
+    wl = by_name(args.workload)
+    T = args.loops
+    if wl.seq % world or (wl.seq // world) % 128:
+        raise SystemExit(f"--cp: {wl.seq} positions do not split into {world} shares of a multiple of 128")
+    S = wl.seq // world
+    inputs = generate(wl)
+    weights = R.device_weights(inputs, wl.dtype == "bf16", device=dev)
+    h = R.RDT(R.make_config(wl, max_loops=T, seq=S, cp_size=world if world > 1 else 0,
+                            cp_rank=rank if world > 1 else 0), weights)
+    del weights
+    opened = []
+    if world > 1:
+        def all_gather(obj):
+            out = [None] * world
+            dist.all_gather_object(out, obj)
+            return out
+        opened = R.cp_connect_ranks(h, rank, world, all_gather)
+    barrier()
+    e_all = torch.from_numpy(inputs["e"]).to(torch.bfloat16)
+    e = e_all[:, rank * S:(rank + 1) * S].contiguous().to(dev)
+    out = torch.empty(e.shape, dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):          # every rank makes the same calls: their loops wait for one another
+        flush.zero_()
+        h.loop_forward(e, e, T, out=out)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = h.launch_count()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_wall0 = time.time()
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        h.loop_forward(e, e, T, out=out)
+        b.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier()
+    launches = (h.launch_count() - launches0) / args.steps
+    clocks = sampler.stop((t_wall0, t_wall1)) if sampler else None
+    ms = reduce_max(statistics.median(a.elapsed_time(b) for a, b in evs), dev)
+    diag = h.diagnostics()
+    finite = bool(torch.isfinite(out).all().item()) and diag["nonfinite"] == 0 and diag["timeout"] == 0
+    barrier()                              # nobody touches a peer's buffers any more
+    for p_ in opened:
+        R.ipc_close_handle(p_)
+    barrier()
+    h.close()
+    if rank != 0:
+        return None
+    tokens = wl.batch * wl.seq
+    peaks, _ = load_peaks()
+    flops = step_flops(wl, T)
+    return {
+        "impl": "ours-cp", "metric": METRIC, "value": tokens * T / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": wl.batch, "seq": wl.seq, "dim": wl.dim, "loops": T,
+                   "tokens_per_step": tokens, "positions_per_rank": S, "parallelism": f"context parallel x{world}",
+                   "l2": "flushed before every timed step (256 MiB write)", "step_time": "median of the timed steps"},
+        "path_roofline": {"step_flops": flops, "achieved_tflops": flops / (ms / 1e3) / 1e12,
+                          "frac_of_bf16_peak_all_gpus": flops / (ms / 1e3) / 1e12 / (peaks["bf16_tflops"] * world)},
+        "e2e": None, "gpu_launches": int(round(launches)), "clocks": clocks, "finite": finite,
+    }
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -765,8 +849,8 @@ def run_gpu(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     init_ranks(dev)
-    if args.decode or args.kernel:
-        line = (bench_attention if args.kernel else bench_decode)(args, dev, rank, world)
+    if args.decode or args.kernel or args.cp:
+        line = (bench_attention if args.kernel else bench_cp if args.cp else bench_decode)(args, dev, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
         barrier()
@@ -799,6 +883,8 @@ def main(argv=None):
     ap.add_argument("--all", action="store_true", help="one line per configuration and loop count")
     ap.add_argument("--decode", action="store_true", help="time decode steps with the per-loop KV cache")
     ap.add_argument("--kernel", choices=("attention",), help="time one kernel alone on the workload's shape")
+    ap.add_argument("--cp", action="store_true",
+                    help="context parallelism: split the workload's sequence over the N GPUs (strong scaling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

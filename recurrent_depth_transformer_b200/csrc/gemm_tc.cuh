@@ -170,22 +170,42 @@ struct TopK {
             bi[j] = -1;
         }
     }
-    __device__ __forceinline__ void insert(float logit, float bias, int ex, int k) {
+    // Branch-free: the list stays sorted by score (entries past top_k are the runners-up).
+    __device__ __forceinline__ void insert(float logit, float bias, int ex) {
         float cs = logit + bias, cl = logit;
         int ci = ex;
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) {
-            if (j < k && cs > bs[j]) {
-                const float ts = bs[j], tl = bl[j];
-                const int ti = bi[j];
-                bs[j] = cs; bl[j] = cl; bi[j] = ci;
-                cs = ts; cl = tl; ci = ti;
-            }
+            const bool sw = cs > bs[j];
+            const float ts = bs[j], tl = bl[j];
+            const int ti = bi[j];
+            bs[j] = sw ? cs : ts;
+            bl[j] = sw ? cl : tl;
+            bi[j] = sw ? ci : ti;
+            cs = sw ? ts : cs;
+            cl = sw ? tl : cl;
+            ci = sw ? ti : ci;
         }
     }
-    __device__ __forceinline__ void write(const EpiParams& p, int row) const {
+    // four consecutive experts ex0 .. ex0 + 3, those from n on left out
+    __device__ __forceinline__ void insert4(const float (&x)[4], const float* bias, int ex0, int n) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const bool in = ex0 + u < n;
+            insert(in ? x[u] : -INFINITY, in && bias ? __ldg(bias + ex0 + u) : 0.0f, ex0 + u);
+        }
+    }
+    // Warp-collective (every lane calls it; `valid`: the lane's row is a real one). The
+    // rows claimed in each expert's capacity block are counted per warp in shared memory
+    // first (sc: 2 n_exp ints of the warp's own staging buffer) and then taken from the
+    // global counter with one atomic per expert the warp chose: a token's top-k claims,
+    // one atomic each on n_exp counters that share two cache lines, serialised at the L2
+    // and cost more than the router GEMM itself.
+    __device__ __forceinline__ void write(const EpiParams& p, int row, bool valid, int lane, int* sc) const {
         const size_t o = static_cast<size_t>(row) * p.top_k;
-        if (p.halted && p.halted[row]) {             // ACT: a halted token is routed nowhere
+        const bool halted = valid && p.halted && p.halted[row];
+        const bool route = valid && !halted;
+        if (halted) {                                // ACT: a halted token is routed nowhere
             for (int j = 0; j < p.top_k; ++j) {
                 p.idx_out[o + j] = -1;
                 p.w_out[o + j] = 0.0f;
@@ -193,7 +213,6 @@ struct TopK {
                 if (p.trace_w) p.trace_w[o + j] = 0.0f;
                 if (p.route_token) p.slot_row[o + j] = -1;
             }
-            return;
         }
         float mx = -INFINITY;
 #pragma unroll
@@ -205,23 +224,41 @@ struct TopK {
             ex[j] = (j < p.top_k && bi[j] >= 0) ? expf(bl[j] - mx) : 0.0f;
             den += ex[j];
         }
+        int* cnt = sc;
+        int* base = sc + p.n_exp;
+        for (int x = lane; x < p.n_exp; x += 32) cnt[x] = 0;
+        __syncwarp();
+        int pos[KMAX];
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) {
-            if (j >= p.top_k) break;
-            const int e = bi[j] < 0 ? 0 : bi[j];      // only when every score was NaN
-            const float w = den > 0.0f ? ex[j] / den : 0.0f;
-            p.idx_out[o + j] = e;
-            p.w_out[o + j] = w;
-            if (p.trace_idx) p.trace_idx[o + j] = e;
-            if (p.trace_w) p.trace_w[o + j] = w;
-            const int pos = atomicAdd(p.counts + e, 1);          // histogram and row claim
-            if (p.route_token) {
-                const int rr = e * p.cap + pos;
-                p.route_token[rr] = row;
-                p.route_w[rr] = w;
-                p.slot_row[o + j] = rr;
+            pos[j] = 0;
+            if (j < p.top_k && route) pos[j] = atomicAdd(cnt + (bi[j] < 0 ? 0 : bi[j]), 1);
+        }
+        __syncwarp();
+        for (int x = lane; x < p.n_exp; x += 32) {
+            const int c = cnt[x];
+            base[x] = c ? atomicAdd(p.counts + x, c) : 0;   // histogram and the warp's rows
+        }
+        __syncwarp();
+        if (route) {
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                if (j >= p.top_k) break;
+                const int e = bi[j] < 0 ? 0 : bi[j];      // only when every score was NaN
+                const float w = den > 0.0f ? ex[j] / den : 0.0f;
+                p.idx_out[o + j] = e;
+                p.w_out[o + j] = w;
+                if (p.trace_idx) p.trace_idx[o + j] = e;
+                if (p.trace_w) p.trace_w[o + j] = w;
+                if (p.route_token) {
+                    const int rr = e * p.cap + base[e] + pos[j];
+                    p.route_token[rr] = row;
+                    p.route_w[rr] = w;
+                    p.slot_row[o + j] = rr;
+                }
             }
         }
+        __syncwarp();                                // the staging buffer is free again
     }
 };
 
@@ -230,40 +267,58 @@ struct TopK {
 // that arrives last on their counter (threadfence-reduction order: adds, fence, count) reads
 // the complete rows back and selects.
 template <int BN, int KMAX>
-__device__ __forceinline__ void epilogue_topk(const EpiParams& p, uint32_t taddr, bool valid, int crow,
-                                              int split, int mtile) {
+__device__ __forceinline__ void epilogue_topk(const EpiParams& p, uint32_t taddr, float* stg, bool valid,
+                                              int crow, int split, int mtile) {
+    const int lane = threadIdx.x & 31;
+    int* sc = reinterpret_cast<int*>(stg);
+    // The selection runs as a short rolled loop (four logits per step): fully unrolled over
+    // the experts it was tens of kilobytes of straight-line code that one warp per SM
+    // sub-partition streamed through the instruction cache, ~60K cycles at 64 experts.
+    const float* bias = p.bias;
     if (split <= 1) {
         TopK<KMAX> tk;
+        uint32_t r[4];
+#pragma unroll 1
+        for (int ex = 0; ex < p.n_exp; ex += 4) {
+            tmem_ld4(taddr + static_cast<uint32_t>(ex), r);
+            tmem_wait_ld();
+            const float x[4] = {__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]),
+                                __uint_as_float(r[3])};
+            tk.insert4(x, bias, ex, p.n_exp);
+        }
+        tk.write(p, crow, valid, lane, sc);
+        return;
+    }
+    float* lrow = p.logits + static_cast<size_t>(crow) * p.n_exp;
+    // the partial logits, transposed through the warp's staging buffer so that each vector
+    // reduction of the warp covers four whole 128-byte row pieces (scalar atomics, one row
+    // per lane, cost ~30 us at 8192 rows and delayed every later L2 access of the router)
+    {
+        const int crow0 = crow - lane;              // the warp's first row
+        const int nrow = __reduce_add_sync(0xffffffffu, valid ? 1 : 0);
+        const int cc = (lane & 7) * 4;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
             float v[32];
             ld_chunk(taddr, c, v);
+            if (c * 32 >= p.n_exp) continue;
+            stage_put(stg, lane, v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int ex = c * 32 + i;
-                if (ex < p.n_exp) tk.insert(v[i], p.bias ? p.bias[ex] : 0.0f, ex, p.top_k);
+            for (int it = 0; it < 8; ++it) {
+                const int rr = it * 4 + (lane >> 3);
+                float o[4];
+                stage_get(stg, lane, it, o);
+                if (rr >= nrow || c * 32 + cc >= p.n_exp) continue;
+                atomicAdd(reinterpret_cast<float4*>(p.logits + static_cast<size_t>(crow0 + rr) * p.n_exp + c * 32 + cc),
+                          make_float4(o[0], o[1], o[2], o[3]));
             }
         }
-        if (valid) tk.write(p, crow);
-        return;
-    }
-    float* lrow = p.logits + static_cast<size_t>(crow) * p.n_exp;
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        ld_chunk(taddr, c, v);
-        if (!valid) continue;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int ex = c * 32 + i;
-            if (ex < p.n_exp) atomicAdd(lrow + ex, v[i]);
-        }
+        __syncwarp();                               // the staging buffer is free again
     }
     // Each warp elects alone, on the counter of its 32 rows (no barrier between warps, so a
     // warp that left on a timeout cannot stall the others): adds, fence, count.
     __threadfence();
     __syncwarp();
-    const int lane = threadIdx.x & 31;
     const int quad = (threadIdx.x >> 5) & 3;
     int last = 0;
     if (lane == 0) {
@@ -273,26 +328,23 @@ __device__ __forceinline__ void epilogue_topk(const EpiParams& p, uint32_t taddr
     }
     if (!__shfl_sync(0xffffffffu, last, 0)) return;
     __threadfence();
-    if (!valid) return;
-    // the complete row, 32 logits at a time: eight 16-byte L2 loads in flight per chunk
-    // (n_exp is a multiple of 8: rows are 32-byte aligned), then the insertions
+    // the complete row from L2, four logits per step, the next two loads in flight
+    // (n_exp is a multiple of 4: 16-byte pieces)
     TopK<KMAX> tk;
+    if (valid) {
+        const float4* row4 = reinterpret_cast<const float4*>(lrow);
+        const int n4 = p.n_exp / 4;
+        float4 a0 = __ldcg(row4);
+        float4 a1 = n4 > 1 ? __ldcg(row4 + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
-    for (int c0 = 0; c0 < p.n_exp; c0 += 32) {
-        float v[32];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const float4 x = c0 + 4 * q < p.n_exp ? __ldcg(reinterpret_cast<const float4*>(lrow + c0 + 4 * q))
-                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-            v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int ex = c0 + i;
-            if (ex < p.n_exp) tk.insert(v[i], p.bias ? p.bias[ex] : 0.0f, ex, p.top_k);
+        for (int q = 0; q < n4; ++q) {
+            const float x[4] = {a0.x, a0.y, a0.z, a0.w};
+            a0 = a1;
+            if (q + 2 < n4) a1 = __ldcg(row4 + q + 2);
+            tk.insert4(x, bias, 4 * q, p.n_exp);
         }
     }
-    tk.write(p, crow);
+    tk.write(p, crow, valid, lane, sc);
 }
 
 // Operands of an epilogue that do not depend on the accumulator: loaded before the epilogue
@@ -480,13 +532,13 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, const EpiPre& pre, 
         const bool valid = lane < nvalid;
         const int crow = row0 + lane;
         if (p.top_k <= 2)
-            epilogue_topk<BN, 2>(p, taddr, valid, crow, split, mtile);
+            epilogue_topk<BN, 2>(p, taddr, stg, valid, crow, split, mtile);
         else if (p.top_k <= 4)
-            epilogue_topk<BN, 4>(p, taddr, valid, crow, split, mtile);
+            epilogue_topk<BN, 4>(p, taddr, stg, valid, crow, split, mtile);
         else if (p.top_k <= 8)
-            epilogue_topk<BN, 8>(p, taddr, valid, crow, split, mtile);
+            epilogue_topk<BN, 8>(p, taddr, stg, valid, crow, split, mtile);
         else
-            epilogue_topk<BN, 16>(p, taddr, valid, crow, split, mtile);
+            epilogue_topk<BN, 16>(p, taddr, stg, valid, crow, split, mtile);
     }
 }
 
