@@ -51,92 +51,141 @@ struct DecAttnArgs {
     float* part;                                 // [B, hq, n_chunks, DV + 2]: o, max, sum
 };
 
-// One CTA per (chunk, head, sequence). Scores are in log2 units (q is scaled on load). Each
-// lane scores one key at a time against q held in shared memory; the warp then folds its 32
-// probabilities into its running (max, sum, o) with the lanes spread over o's columns.
-template <int DQK, int DV>
+// One CTA per (chunk, group of HG query heads, sequence); the HG heads share one KV head, so
+// a key or value row is read once for all of them. Scores are in log2 units (q is scaled on
+// load). Each lane scores one key at a time against the HG queries held in shared memory;
+// the warp then folds its 32 probabilities into the heads' running (max, sum, o) with the
+// lanes spread over o's columns (two adjacent columns per lane and pass: one coalesced
+// 4-byte load per value row), eight keys' value loads in flight at a time.
+template <int DQK, int DV, int HG>
 __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecAttnArgs a) {
     pdl_trigger();
     pdl_wait();
-    __shared__ float qs[DQK];
-    __shared__ float wm[4], wl[4];
-    __shared__ float wo[4][DV];
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    __shared__ float qs[HG][DQK];
+    __shared__ float wm[4][HG], wl[4][HG];
+    __shared__ float wo[4][HG][DV];
+    const int c = blockIdx.x, hg0 = blockIdx.y * HG, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = (h * a.hkv) / a.hq;
+    const int g = (hg0 * a.hkv) / a.hq;
     const int n_keys = *a.len_dev + 1;
-    const bf16* qrow = a.q + static_cast<size_t>(b) * a.q_ld + h * a.q_hstride;
-    for (int i = threadIdx.x; i < DQK; i += kDecThreads) qs[i] = __bfloat162float(qrow[i]) * a.scale_log2;
+    for (int i = threadIdx.x; i < HG * DQK; i += kDecThreads) {
+        const int hh = i / DQK, d = i % DQK;
+        qs[hh][d] = __bfloat162float(a.q[static_cast<size_t>(b) * a.q_ld + (hg0 + hh) * a.q_hstride + d]) * a.scale_log2;
+    }
     __syncthreads();
-    constexpr int VPL = DV / 32;                 // o columns per lane
-    float m = -INFINITY, l = 0.0f, o[VPL];
+    constexpr int VP = DV / 64;                  // column pairs per lane
+    float m[HG], l[HG], o[HG][VP][2];
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) o[i] = 0.0f;
+    for (int hh = 0; hh < HG; ++hh) {
+        m[hh] = -INFINITY;
+        l[hh] = 0.0f;
+#pragma unroll
+        for (int i = 0; i < VP; ++i) o[hh][i][0] = o[hh][i][1] = 0.0f;
+    }
     const bf16* base = a.cache + static_cast<size_t>(b) * a.s_cap * a.cache_ld;
     const int kbeg = c * kDecChunk + warp * (kDecChunk / 4);
 #pragma unroll 1
     for (int r = 0; r < kDecChunk / 4 / 32; ++r) {
-        const int key = kbeg + r * 32 + lane;
-        float s = -INFINITY;
+        const int kfirst = kbeg + r * 32;
+        if (kfirst >= n_keys) break;                 // warp-uniform
+        const int key = kfirst + lane;
+        float sc[HG];
+#pragma unroll
+        for (int hh = 0; hh < HG; ++hh) sc[hh] = -INFINITY;
         if (key < n_keys) {
             const bf16* krow = base + static_cast<size_t>(key) * a.cache_ld + a.k_col0 + g * a.k_hstride;
-            float acc = 0.0f;
+            float acc[HG];
+#pragma unroll
+            for (int hh = 0; hh < HG; ++hh) acc[hh] = 0.0f;
 #pragma unroll
             for (int d0 = 0; d0 < DQK; d0 += 8) {
                 const uint4 u = *reinterpret_cast<const uint4*>(krow + d0);
                 const bf16* kk = reinterpret_cast<const bf16*>(&u);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc = fmaf(qs[d0 + j], __bfloat162float(kk[j]), acc);
+                for (int j = 0; j < 8; ++j) {
+                    const float kv = __bfloat162float(kk[j]);
+#pragma unroll
+                    for (int hh = 0; hh < HG; ++hh) acc[hh] = fmaf(qs[hh][d0 + j], kv, acc[hh]);
+                }
             }
-            s = acc;
+#pragma unroll
+            for (int hh = 0; hh < HG; ++hh) sc[hh] = acc[hh];
         }
-        float mx = s;
+        float p[HG];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        if (mx == -INFINITY) continue;           // no key of this group (warp-uniform)
-        const float m_new = fmaxf(m, mx);
-        const float corr = exp2f(m - m_new);     // 0 at the first group (m = -inf)
-        const float p = exp2f(s - m_new);        // 0 for a key past the length
-        float ps = p;
+        for (int hh = 0; hh < HG; ++hh) {
+            float mx = sc[hh];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-        l = l * corr + ps;
+            for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            const float m_new = fmaxf(m[hh], mx);        // finite: the group has a key
+            const float corr = exp2f(m[hh] - m_new);     // 0 at the first group (m = -inf)
+            p[hh] = exp2f(sc[hh] - m_new);               // 0 for a key past the length
+            float ps = p[hh];
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) o[i] *= corr;
-        const int kfirst = kbeg + r * 32;
+            for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+            l[hh] = l[hh] * corr + ps;
+#pragma unroll
+            for (int i = 0; i < VP; ++i) {
+                o[hh][i][0] *= corr;
+                o[hh][i][1] *= corr;
+            }
+            m[hh] = m_new;
+        }
         const int nk = min(32, n_keys - kfirst);
+        const bf16* vbase = base + static_cast<size_t>(kfirst) * a.cache_ld + a.v_col0 + g * a.v_hstride + 2 * lane;
 #pragma unroll 1
-        for (int k = 0; k < nk; ++k) {
-            const float pk = __shfl_sync(0xffffffffu, p, k);
-            const bf16* vrow = base + static_cast<size_t>(kfirst + k) * a.cache_ld + a.v_col0 + g * a.v_hstride;
+        for (int k0 = 0; k0 < nk; k0 += 8) {
+            __nv_bfloat162 v[8][VP];
 #pragma unroll
-            for (int i = 0; i < VPL; ++i) o[i] = fmaf(pk, __bfloat162float(vrow[lane + 32 * i]), o[i]);
+            for (int u = 0; u < 8; ++u)
+#pragma unroll
+                for (int i = 0; i < VP; ++i)
+                    v[u][i] = k0 + u < nk ? *reinterpret_cast<const __nv_bfloat162*>(
+                                                vbase + static_cast<size_t>(k0 + u) * a.cache_ld + 64 * i)
+                                          : __floats2bfloat162_rn(0.0f, 0.0f);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+#pragma unroll
+                for (int hh = 0; hh < HG; ++hh) {
+                    const float pk = __shfl_sync(0xffffffffu, p[hh], (k0 + u) & 31);
+#pragma unroll
+                    for (int i = 0; i < VP; ++i) {
+                        const float2 vf = __bfloat1622float2(v[u][i]);
+                        o[hh][i][0] = fmaf(pk, vf.x, o[hh][i][0]);
+                        o[hh][i][1] = fmaf(pk, vf.y, o[hh][i][1]);
+                    }
+                }
+            }
         }
-        m = m_new;
     }
-    // the four warps' partials, then the chunk's
+    // the four warps' partials, then the chunk's (warp hh % 4 merges head hh)
     if (lane == 0) {
-        wm[warp] = m;
-        wl[warp] = l;
+#pragma unroll
+        for (int hh = 0; hh < HG; ++hh) {
+            wm[warp][hh] = m[hh];
+            wl[warp][hh] = l[hh];
+        }
     }
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) wo[warp][lane + 32 * i] = o[i];
+    for (int hh = 0; hh < HG; ++hh)
+#pragma unroll
+        for (int i = 0; i < VP; ++i) {
+            wo[warp][hh][64 * i + 2 * lane] = o[hh][i][0];
+            wo[warp][hh][64 * i + 2 * lane + 1] = o[hh][i][1];
+        }
     __syncthreads();
-    if (warp == 0) {
-        float mc = fmaxf(fmaxf(wm[0], wm[1]), fmaxf(wm[2], wm[3]));
-        float sc[4];
+    for (int hh = warp; hh < HG; hh += 4) {
+        const float mc = fmaxf(fmaxf(wm[0][hh], wm[1][hh]), fmaxf(wm[2][hh], wm[3][hh]));
+        float sw[4];
         float lc = 0.0f;
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-            sc[w] = mc == -INFINITY ? 0.0f : exp2f(wm[w] - mc);
-            lc += wl[w] * sc[w];
+            sw[w] = wm[w][hh] == -INFINITY ? 0.0f : exp2f(wm[w][hh] - mc);
+            lc += wl[w][hh] * sw[w];
         }
-        float* part = a.part + ((static_cast<size_t>(b) * a.hq + h) * a.n_chunks + c) * (DV + 2);
-#pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            const int col = lane + 32 * i;
-            part[col] = wo[0][col] * sc[0] + wo[1][col] * sc[1] + wo[2][col] * sc[2] + wo[3][col] * sc[3];
-        }
+        float* part = a.part + ((static_cast<size_t>(b) * a.hq + hg0 + hh) * a.n_chunks + c) * (DV + 2);
+        for (int col = lane; col < DV; col += 32)
+            part[col] = wo[0][hh][col] * sw[0] + wo[1][hh][col] * sw[1] + wo[2][hh][col] * sw[2] + wo[3][hh][col] * sw[3];
         if (lane == 0) {
             part[DV] = mc;
             part[DV + 1] = lc;
@@ -214,15 +263,22 @@ rdt_status decode_attention(const DecodeAttnArgs& d, cudaStream_t st) {
     a.len_dev = d.len_dev;
     a.scale_log2 = d.scale * 1.4426950408889634f;
     a.part = d.part;
-    const dim3 grid(a.n_chunks, d.hq, d.batch);
+    // query heads per CTA: up to four of those that share a KV head
+    const int G = d.hq / d.hkv;
+    const int HG = G % 4 == 0 ? 4 : G % 2 == 0 ? 2 : 1;
+    const dim3 grid(a.n_chunks, d.hq / HG, d.batch);
     const int nrows = d.batch * d.hq;
     if (d.dqk == 64 && d.dv == 64) {
-        RDT_CUDA_TRY(launch_pdl(decode_attn_kernel<64, 64>, grid, dim3(kDecThreads), 0, st, a));
+        if (HG == 4) RDT_CUDA_TRY(launch_pdl(decode_attn_kernel<64, 64, 4>, grid, dim3(kDecThreads), 0, st, a));
+        else if (HG == 2) RDT_CUDA_TRY(launch_pdl(decode_attn_kernel<64, 64, 2>, grid, dim3(kDecThreads), 0, st, a));
+        else RDT_CUDA_TRY(launch_pdl(decode_attn_kernel<64, 64, 1>, grid, dim3(kDecThreads), 0, st, a));
         RDT_CUDA_TRY(launch_pdl(decode_merge_kernel<64>, dim3((nrows + 7) / 8), dim3(256), 0, st,
                                 static_cast<const float*>(d.part), d.hq, a.n_chunks, d.len_dev,
                                 static_cast<bf16*>(d.o), d.ldo, d.dv_out, nrows));
     } else if (d.dqk == 160 && d.dv == 128) {
-        RDT_CUDA_TRY(launch_pdl(decode_attn_kernel<160, 128>, grid, dim3(kDecThreads), 0, st, a));
+        if (HG == 4) RDT_CUDA_TRY(launch_pdl(decode_attn_kernel<160, 128, 4>, grid, dim3(kDecThreads), 0, st, a));
+        else if (HG == 2) RDT_CUDA_TRY(launch_pdl(decode_attn_kernel<160, 128, 2>, grid, dim3(kDecThreads), 0, st, a));
+        else RDT_CUDA_TRY(launch_pdl(decode_attn_kernel<160, 128, 1>, grid, dim3(kDecThreads), 0, st, a));
         RDT_CUDA_TRY(launch_pdl(decode_merge_kernel<128>, dim3((nrows + 7) / 8), dim3(256), 0, st,
                                 static_cast<const float*>(d.part), d.hq, a.n_chunks, d.len_dev,
                                 static_cast<bf16*>(d.o), d.ldo, d.dv_out, nrows));

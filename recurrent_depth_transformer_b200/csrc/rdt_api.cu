@@ -62,6 +62,7 @@ struct rdt_handle {
     void *cq = nullptr, *kvlat = nullptr, *xperm = nullptr, *U = nullptr, *yn_lo = nullptr;
     int bn_router = 64;
     int router_split = 1;          // K split of the router GEMM over CTAs
+    int router_split_dec = 1;      // ... for a decode step's batch rows
     float* logits = nullptr;       // [N, E] partial-logit accumulator of the split router
     int* tile_count = nullptr;     // arrival counters of the split router, per 32 rows of a row tile
     // output tile widths of the projection and expert GEMMs (128, 192 on pairs, or 256), and
@@ -735,6 +736,12 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
         for (int sp = 1; sp <= kb && !c.deterministic && E % 4 == 0; ++sp)
             if (kb % sp == 0 && static_cast<long>(mt) * sp <= num_sms()) split = sp;
         h->router_split = split;
+        // a decode step routes batch rows: one row tile, so the K blocks spread over many CTAs
+        int split_dec = 1;
+        const int mt_dec = (c.batch + 127) / 128;
+        for (int sp = 1; sp <= kb && c.max_decode > 0 && !c.deterministic && E % 4 == 0; ++sp)
+            if (kb % sp == 0 && static_cast<long>(mt_dec) * sp <= num_sms()) split_dec = sp;
+        h->router_split_dec = split_dec;
         RDT_TRY(dev_alloc(h, &h->logits, static_cast<size_t>(N) * E * 4, true));
         RDT_TRY(dev_alloc(h, &h->tile_count, static_cast<size_t>(mt) * 4 * 4, true));   // per 32 rows
     }
@@ -1213,7 +1220,8 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
         n2.ntok = N;
         n2.dim = d;
         n2.eps = c.norm_eps;
-        if (h->router_split > 1) {
+        const int rsplit = h->mode == 2 ? h->router_split_dec : h->router_split;
+        if (rsplit > 1) {
             n2.zero_rows = h->logits;
             n2.zero_width = c.n_experts;
         }
@@ -1225,7 +1233,7 @@ rdt_status moe_block(rdt_handle* h, const float* yin, float* dst, int32_t* idx_o
         gr.kb_main = static_cast<int>(d * h->esz / 128);
         gr.kb_ext = gr.kb_main;
         gr.b2_row0 = 0;
-        gr.split_k = h->router_split;
+        gr.split_k = rsplit;
         gr.flags = h->flags;
         EpiParams er{};
         er.kind = EPI_TOPK;
