@@ -176,12 +176,20 @@ def kernel_work(wl):
                           bound="tensor")
     # RMSNorm1 reads h, e, B e and writes xn, y = x and h_next = A h + B e
     w["norm1"] = dict(flops=0.0, bytes=N * d * (4 + b2 + 4 + b2 + 4 + 4), bound="hbm")
-    # the router: y in, W_r once, per (token, slot) the routing words and the yn copy in the
-    # expert's rows; yn itself where shared experts read it
-    w["router_topk"] = dict(flops=2.0 * N * d * E,
-                            bytes=N * d * 4 + (N * d * b2 if S else 0) + E * d * b2 + N * k * (d * b2 + 16),
-                            bound="hbm")
-    w["norm2"] = dict(flops=0.0, bytes=N * d * (4 + b2), bound="hbm")
+    if E * d * b2 <= 65536 or wl.dtype != "bf16":
+        # the fused router (W_r in shared memory; fp32: FMA): y in, W_r once, per (token,
+        # slot) the routing words and the yn copy in the expert's rows; yn itself where
+        # shared experts read it
+        w["router_topk"] = dict(flops=2.0 * N * d * E,
+                                bytes=N * d * 4 + (N * d * b2 if S else 0) + E * d * b2 + N * k * (d * b2 + 16),
+                                bound="hbm")
+    else:
+        # the tensor-core router: yn and its bf16 residual in, W_r once (both halves), per
+        # (token, slot) the routing words (index, weight, claimed row, token of the row)
+        w["router_topk"] = dict(flops=2.0 * N * 2 * d * E, bytes=N * d * b2 * 2 + 2 * E * d * b2 + N * k * 16,
+                                bound="hbm")
+    # RMSNorm2 for the tensor-core router: y in, yn and its bf16 residual out
+    w["norm2"] = dict(flops=0.0, bytes=N * d * (4 + 2 * b2), bound="hbm")
     w["moe_dispatch"] = dict(flops=0.0, bytes=N * k * (d * b2 * 2 + 4), bound="hbm")
     w["moe_combine"] = dict(flops=0.0, bytes=N * d * 4 * (2 + k + S), bound="hbm")
     w["hoist"] = dict(flops=0.0, bytes=N * d * (b2 + b2 + 4 + 4), bound="hbm")
