@@ -16,7 +16,8 @@
 //
 // attn96_kernel (head width 64, the GQA shapes): blocks of 96 keys, two score buffers per
 // tile so that S_t(j + 1) is computed while the softmax works on S_t(j), one MMA-issuing
-// thread per tile, part of the exponentials on the FMA pipe.
+// thread per tile, two softmax warps per query row (48 keys of every block each; they agree
+// on the row maximum through shared memory), part of the exponentials on the FMA pipe.
 //
 // attn_tc_kernel (the 160-wide absorbed MLA keys, values of 128): blocks of 128 keys, one
 // score buffer per tile, one MMA thread. Absorbed MLA attends over the shared latent key
@@ -476,30 +477,57 @@ __global__ void __launch_bounds__(AttnCfg<DQK, DV, SHARE_KV, QT>::THREADS,
 constexpr int kPolyOf8 = 2;
 
 
+// Softmax warps per query row: 2 splits every block's 96 keys between two warps of the same
+// TMEM lane quadrant (they exchange their row maxima through shared memory)
+// (measured at 8192 positions: 381 us with one warp per row, 373 with two)
+constexpr int kRowWarps = 2;
+
 template <int QT>
 struct K96Cfg {
     static constexpr int BK = 96;                       // keys per block
+    static constexpr int RW = kRowWarps;                // softmax warps per query row
+    static constexpr int NV = BK / RW;                  // scores per softmax thread and block
     static constexpr int KV_BYTES = BK * 128;           // 96 keys x 64 bf16
     static constexpr int STAGES = QT == 2 ? 4 : 3;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + QT * kAtom;
     static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
     static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
-    static constexpr int SMEM = OFF_BAR + 256 + 1024;   // + alignment slack
+    static constexpr int OFF_X = OFF_BAR + 256;         // float [2 slots][QT][RW][128] row maxima, then [QT][RW][128] sums
+    static constexpr int SMEM = OFF_X + 3 * QT * RW * 128 * 4 + 1024;   // + alignment slack
     static constexpr int O_COL = 2 * BK * QT;           // S buffers first, then O_t
     static constexpr int COLS_USED = O_COL + 64 * QT;
     static constexpr int TMEM_COLS = COLS_USED <= 256 ? 256 : 512;
-    static constexpr int THREADS = 128 + 128 * QT;
+    static constexpr int THREADS = 128 + 128 * QT * RW;
     static constexpr int BLOCKS_PER_SM = QT == 1 ? 2 : 1;
     static constexpr int REGS_LAUNCH = (65536 / (THREADS * BLOCKS_PER_SM)) / 8 * 8;
-    static constexpr int REGS_CONTROL = 56;
-    static constexpr int REGS_SOFTMAX = ((REGS_LAUNCH * THREADS - 128 * REGS_CONTROL) / (128 * QT)) / 8 * 8;
-    static_assert(128 * REGS_CONTROL + 128 * QT * REGS_SOFTMAX <= REGS_LAUNCH * THREADS, "register split");
+    static constexpr int REGS_CONTROL = RW == 2 ? 48 : 56;
+    static constexpr int REGS_SOFTMAX = ((REGS_LAUNCH * THREADS - 128 * REGS_CONTROL) / (128 * QT * RW)) / 8 * 8;
+    static_assert(RW == 1 || RW == 2, "one or two softmax warps per row");
+    static_assert(128 * REGS_CONTROL + 128 * QT * RW * REGS_SOFTMAX <= REGS_LAUNCH * THREADS, "register split");
     static_assert(REGS_SOFTMAX <= 256, "setmaxnreg limit");
     static_assert(COLS_USED <= TMEM_COLS && TMEM_COLS * BLOCKS_PER_SM <= 512, "TMEM budget");
     static_assert(SMEM * BLOCKS_PER_SM <= 228 * 1024, "shared-memory budget");
 };
 
+// Warp-collective: lane i reads TMEM lane (base lane + i), 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+// Warp-collective: lane i writes TMEM lane (base lane + i), 8 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 // Warp-collective: lane i writes TMEM lane (base lane + i), 16 consecutive 32-bit columns.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
     asm volatile(
@@ -564,7 +592,7 @@ __global__ void __launch_bounds__(K96Cfg<QT>::THREADS, K96Cfg<QT>::BLOCKS_PER_SM
         for (int t = 0; t < QT; ++t) {
             for (int u = 0; u < 2; ++u) {
                 mbar_init(&sfull[2 * t + u], 1);
-                mbar_init(&pfull[2 * t + u], 4);
+                mbar_init(&pfull[2 * t + u], 4 * C::RW);
             }
             mbar_init(&oready[t], 1);
             mbar_init(&odone[t], 1);
@@ -672,8 +700,12 @@ __global__ void __launch_bounds__(K96Cfg<QT>::THREADS, K96Cfg<QT>::BLOCKS_PER_SM
       }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_SOFTMAX));
-        // softmax warpgroup 1 + t (warps 4 + 4 t .. 7 + 4 t): TMEM lane quadrant warp & 3
-        const int t = (warp - 4) >> 2;
+        // softmax warps 4 + 4 RW t + 4 hf + quad: tile t, half hf of every block's keys (RW = 2),
+        // TMEM lane quadrant quad, one query row per thread
+        constexpr int RW = C::RW, NV = C::NV;
+        const int sw = warp - 4;
+        const int t = sw / (4 * RW);
+        const int hf = RW == 2 ? (sw >> 2) & 1 : 0;
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
         const int qpos = (qb0 + t) * kBQ + r;
@@ -682,6 +714,8 @@ __global__ void __launch_bounds__(K96Cfg<QT>::THREADS, K96Cfg<QT>::BLOCKS_PER_SM
         const uint32_t o_col = C::O_COL + 64 * t;
         const float sl = a.scale_log2;
         const int kmax_row = min(a.q_off + qpos, a.kv_seq - 1);   // last key the row may see
+        float* xmax = reinterpret_cast<float*>(smem + C::OFF_X);   // [2][QT][RW][128]
+        float* xsum = xmax + 2 * QT * RW * 128;                   // [QT][RW][128]
         float m_ref = -INFINITY, l = 0.0f;
         bool ok = true;
 #pragma unroll 1
@@ -690,25 +724,41 @@ __global__ void __launch_bounds__(K96Cfg<QT>::THREADS, K96Cfg<QT>::BLOCKS_PER_SM
             if (ok && !mbar_wait(&sfull[2 * t + u], (j >> 1) & 1, a.flags)) ok = false;
             tc_fence_after();
             const uint32_t s_col = 2 * BK * t + BK * u;
-            uint32_t v[96];
-            tmem_ld32(lane_base + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(v + 0));
-            tmem_ld32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-            tmem_ld32(lane_base + s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
+            uint32_t v[NV];
+            if constexpr (RW == 1) {
+                tmem_ld32(lane_base + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(v + 0));
+                tmem_ld32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                tmem_ld32(lane_base + s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
+            } else {
+                tmem_ld32(lane_base + s_col + NV * hf, *reinterpret_cast<uint32_t(*)[32]>(v + 0));
+                tmem_ld16(lane_base + s_col + NV * hf + 32, v + 32);
+            }
             tmem_wait_ld();
-            const int kmax = kmax_row - j * BK;
-            if (kmax < BK - 1) {
+            const int kmax = kmax_row - j * BK - NV * hf;
+            if (kmax < NV - 1) {
 #pragma unroll
-                for (int i = 0; i < 96; ++i)
+                for (int i = 0; i < NV; ++i)
                     if (i > kmax) v[i] = __float_as_uint(-INFINITY);
             }
             float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int i = 0; i < 96; i += 8) {
+            for (int i = 0; i < NV; i += 8) {
 #pragma unroll
                 for (int w = 0; w < 4; ++w)
                     m4[w] = fmax3(m4[w], __uint_as_float(v[i + 2 * w]), __uint_as_float(v[i + 2 * w + 1]));
             }
-            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl;
+            float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl;
+            if constexpr (RW == 2) {
+                // the two halves of the row agree on the maximum (so on m_ref): each writes its
+                // own into this block's slot and reads the other's after the pair's barrier (the
+                // slot alternates with the block, so a half a block ahead never overwrites a
+                // value its partner has yet to read). The barrier also orders the partner's
+                // score loads before this half's P overwrites its columns.
+                float* slot = xmax + (u * QT + t) * RW * 128;
+                slot[hf * 128 + r] = mx;
+                named_barrier(1 + t * 4 + quad, 64);
+                mx = fmaxf(mx, slot[(hf ^ 1) * 128 + r]);
+            }
             float corr = 1.0f;
             if (mx > m_ref + kRescaleThreshold) {
                 corr = exp2_ftz(m_ref - mx);
@@ -720,9 +770,9 @@ __global__ void __launch_bounds__(K96Cfg<QT>::THREADS, K96Cfg<QT>::BLOCKS_PER_SM
             const float2 slv = make_float2(sl, sl);
             const float2 mneg = make_float2(-mr, -mr);
             float2 rs2 = make_float2(0.0f, 0.0f);
-            uint32_t pk[48];
+            uint32_t pk[NV / 2];
 #pragma unroll
-            for (int c = 0; c < 48; ++c) {
+            for (int c = 0; c < NV / 2; ++c) {
                 const float2 x = __ffma2_rn(make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])),
                                             slv, mneg);
                 // kPolyOf8 pairs in every 8 on the FMA pipe, the rest on the MUFU
@@ -736,25 +786,32 @@ __global__ void __launch_bounds__(K96Cfg<QT>::THREADS, K96Cfg<QT>::BLOCKS_PER_SM
                 pk[c] = pack_bf16(pp.x, pp.y);
             }
             l += rs2.x + rs2.y;
-            tmem_st32(lane_base + s_col, *reinterpret_cast<uint32_t(*)[32]>(pk));
-            tmem_st16(lane_base + s_col + 32, pk + 32);
+            // P over the first 48 score columns (keys 2c, 2c + 1 in column c)
+            if constexpr (RW == 1) {
+                tmem_st32(lane_base + s_col, *reinterpret_cast<uint32_t(*)[32]>(pk));
+                tmem_st16(lane_base + s_col + 32, pk + 32);
+            } else {
+                tmem_st16(lane_base + s_col + (NV / 2) * hf, pk);
+                tmem_st8(lane_base + s_col + (NV / 2) * hf + 16, pk + 16);
+            }
             if (corr != 1.0f && j > 0) {
                 // O_t holds blocks 0 .. j - 1 once PV_t(j - 1) has completed: S_t(j + 1) was
                 // issued after it (its completion implies PV_t(j - 1)'s), and for the last
                 // block the MMA thread commits oready after PV_t(j - 1). PV_t(j) waits for this
-                // rescale (pfull).
+                // rescale (pfull). With two halves each rescales 32 of the 64 columns.
                 const bool w = j + 1 < nkb ? mbar_wait(&sfull[2 * t + (u ^ 1)], ((j + 1) >> 1) & 1, a.flags)
                                            : mbar_wait(&oready[t], 0, a.flags);
                 if (ok && !w) ok = false;
                 tc_fence_after();
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
+                for (int c = 0; c < 2 / RW; ++c) {
                     uint32_t ov[32];
-                    tmem_ld32(lane_base + o_col + c * 32, ov);
+                    const uint32_t oc = o_col + (RW == 2 ? 32 * hf : 32 * c);
+                    tmem_ld32(lane_base + oc, ov);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
-                    tmem_st32(lane_base + o_col + c * 32, ov);
+                    tmem_st32(lane_base + oc, ov);
                 }
             }
             tmem_wait_st();
@@ -763,14 +820,20 @@ __global__ void __launch_bounds__(K96Cfg<QT>::THREADS, K96Cfg<QT>::BLOCKS_PER_SM
             if (lane == 0) mbar_arrive(&pfull[2 * t + u]);
         }
         if (nkb > 0) {
+            if constexpr (RW == 2) {             // the row sum is the two halves' (same m_ref)
+                xsum[(t * RW + hf) * 128 + r] = l;
+                named_barrier(1 + t * 4 + quad, 64);
+                l += xsum[(t * RW + (hf ^ 1)) * 128 + r];
+            }
             if (ok) ok = mbar_wait(&odone[t], 0, a.flags);   // the tile's last PV
             tc_fence_after();
             const float inv = ok ? 1.0f / l : 0.0f;
             bf16* out = static_cast<bf16*>(a.o) + static_cast<size_t>(row0 + qpos) * a.ldo + h * a.dv_out;
 #pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < 2 / RW; ++c) {
+                const int oc = RW == 2 ? 32 * hf : 32 * c;
                 uint32_t ov[32];
-                tmem_ld32(lane_base + o_col + c * 32, ov);
+                tmem_ld32(lane_base + o_col + oc, ov);
                 tmem_wait_ld();
                 if (!ok || qpos >= a.seq) continue;
 #pragma unroll
@@ -780,7 +843,7 @@ __global__ void __launch_bounds__(K96Cfg<QT>::THREADS, K96Cfg<QT>::BLOCKS_PER_SM
                     for (int w = 0; w < 4; ++w)
                         w4[w] = pack_bf16(__uint_as_float(ov[8 * q + 2 * w]) * inv,
                                           __uint_as_float(ov[8 * q + 2 * w + 1]) * inv);
-                    *reinterpret_cast<uint4*>(out + c * 32 + 8 * q) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    *reinterpret_cast<uint4*>(out + oc + 8 * q) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
             }
         }
