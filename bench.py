@@ -137,6 +137,13 @@ def kernel_work(wl):
     b2 = 2 if wl.dtype == "bf16" else 4
     pairs = wl.batch * wl.seq * (wl.seq + 1) / 2
     w = {}
+    # the O projection that forms y = x + a and h_next = A h + B e + a reads h (and e, or the
+    # hoisted B e) and stores both once; after depth attention it adds a into them instead
+    e_in = b2 if wl.inject_e else 0
+    be_in = 4 if (wl.b_kind == "dense" or not wl.inject_e) else 0
+    resid = N * d * (4 + e_in + be_in + 4 + 4)
+    depth = bool(getattr(wl, "da_heads", 0))
+    o_out = 4 * 2 * N * d if depth else resid
     if wl.attn == "gqa":
         hq, hkv, dh = wl.n_heads, wl.n_kv_heads, wl.head_dim
         nq, nqkv = hq * dh, (hq + 2 * hkv) * dh
@@ -146,7 +153,7 @@ def kernel_work(wl):
         w["attention"] = dict(flops=4.0 * hq * dh * pairs, bytes=b2 * N * (nqkv + nq), bound="tensor")
         ow = nq
         w["gemm_o"] = dict(flops=2.0 * N * nq * d + 2.0 * N * r * (nq + d),
-                           bytes=b2 * (N * nq + d * nq) + 4 * 2 * N * d, bound="tensor")
+                           bytes=b2 * (N * nq + d * nq) + o_out, bound="tensor")
     else:
         H, ql, kvl, rp = wl.n_heads, wl.q_lora_rank, wl.kv_lora_rank, wl.qk_rope_dim
         lat = ql + kvl + rp
@@ -157,7 +164,7 @@ def kernel_work(wl):
         w["attention"] = dict(flops=2.0 * H * (kvl + rp + kvl) * pairs,
                               bytes=b2 * N * (H * (kvl + rp) + kvl + rp + H * kvl), bound="tensor")
         ow = H * kvl
-        w["gemm_o"] = dict(flops=2.0 * N * ow * d, bytes=b2 * (N * ow + d * ow) + 4 * 2 * N * d, bound="tensor")
+        w["gemm_o"] = dict(flops=2.0 * N * ow * d, bytes=b2 * (N * ow + d * ow) + o_out, bound="tensor")
         w["mla_latent_norm"] = dict(flops=0.0, bytes=N * (4 * lat + b2 * (ql + kvl + rp)), bound="hbm")
     if getattr(wl, "da_heads", 0):
         # depth attention: projections of every token, each query over its T loops' keys
@@ -169,14 +176,14 @@ def kernel_work(wl):
         keys = (T + 1) / 2.0
         w["depth_attention"] = dict(flops=4.0 * N * hqd * dh * keys,
                                     bytes=b2 * N * (nqd + 2 * hkvd * dh * keys + nqd), bound="hbm")
-        w["gemm_o_depth"] = dict(flops=2.0 * N * nqd * d, bytes=b2 * (N * nqd + d * nqd) + 4 * 2 * N * d,
+        w["gemm_o_depth"] = dict(flops=2.0 * N * nqd * d, bytes=b2 * (N * nqd + d * nqd) + resid,
                                  bound="tensor")
     w["gemm_up"] = dict(flops=2.0 * rows * d * 2 * hid, bytes=b2 * (rows * d + (E + S) * 2 * hid * d + rows * hid),
                         bound="tensor")
     w["gemm_down"] = dict(flops=2.0 * rows * hid * d, bytes=b2 * (rows * hid + (E + S) * d * hid) + 4 * N * d * 2,
                           bound="tensor")
-    # RMSNorm1 reads h, e, B e and writes xn, y = x and h_next = A h + B e
-    w["norm1"] = dict(flops=0.0, bytes=N * d * (4 + b2 + 4 + b2 + 4 + 4), bound="hbm")
+    # RMSNorm1 reads h and e and writes xn (after depth attention: reads y, writes xn)
+    w["norm1"] = dict(flops=0.0, bytes=N * d * (4 + e_in + b2), bound="hbm")
     if E * d * b2 <= 65536 or wl.dtype != "bf16":
         # the fused router (W_r in shared memory; fp32: FMA): y in, W_r once, per (token,
         # slot) the routing words and the yn copy in the expert's rows; yn itself where
@@ -193,7 +200,9 @@ def kernel_work(wl):
     w["norm2"] = dict(flops=0.0, bytes=N * d * (4 + 2 * b2), bound="hbm")
     w["moe_dispatch"] = dict(flops=0.0, bytes=N * k * (d * b2 * 2 + 4), bound="hbm")
     w["moe_combine"] = dict(flops=0.0, bytes=N * d * 4 * (2 + k + S), bound="hbm")
-    w["hoist"] = dict(flops=0.0, bytes=N * d * (b2 + b2 + 4 + 4), bound="hbm")
+    # h <- h0; B e only where the O projection does not form it (dense B: a separate matmul)
+    keep_be = wl.b_kind == "diag" and not wl.inject_e
+    w["hoist"] = dict(flops=0.0, bytes=N * d * (b2 + 4 + ((b2 + 4) if keep_be else 0)), bound="hbm")
     w["check_finite"] = dict(flops=0.0, bytes=N * d * 4, bound="hbm")
     w["act_halting"] = dict(flops=0.0, bytes=N * d * 12, bound="hbm")
     return w

@@ -24,6 +24,10 @@ rdt_status gemm_tc(bool bf16_elems, int bn, const CUtensorMap& tA, const CUtenso
         set_error("gemm_tc: a K split needs an epilogue that reduces into its output");
         return RDT_ERR_INVALID_ARG;
     }
+    if (args.split_k > 1 && epi.kind == EPI_OPROJ_LOOP && epi.h_in) {
+        set_error("gemm_tc: the O projection's stores of y and h_next need the whole K");
+        return RDT_ERR_INVALID_ARG;
+    }
     if (epi.kind == EPI_TOPK) {
         if (bf16_elems) {
             if (bn == 64) return dispatch_router<bf16, 64>(tA, tB, tA2, tB2, args, epi, st);

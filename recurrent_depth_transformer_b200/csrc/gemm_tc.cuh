@@ -21,9 +21,10 @@
 //
 // The fused epilogues are where the block's element-wise work lives:
 //   EPI_ROPE        Q/K/V projection + rotary embedding on the rotated heads;
-//   EPI_OPROJ_LOOP  output projection completing the residual y = x + a and the recurrent
-//                   update h_next = A (.) h + B.e + a (RMSNorm1 wrote x and A h + B.e; the
-//                   MoE adds f later);
+//   EPI_OPROJ_LOOP  output projection forming the residual y = x + a and the recurrent
+//                   update h_next = A (.) h + B.e + a from h and e (after depth attention:
+//                   adding a into the y and h_next its O projection formed; the MoE adds f
+//                   later);
 //   EPI_SWIGLU      expert up-projection (gate and up rows interleaved per tile) -> silu(g)*u;
 //   EPI_SCATTER     expert down-projection, gate weight, and reduction into h_next
 //                   (h_{t+1} = A h + B e + a + sum_j w_j E_j(yn));
@@ -47,8 +48,8 @@ constexpr int BM = 128;
 
 // Epilogue warps per TMEM lane quadrant: two for the epilogues that work chunk by chunk
 // (each warp takes every other 32-column chunk of the tile, so that one warp's TMEM loads,
-// transposes and stores or reductions overlap the other's), one for the router's top-k (a
-// warp needs its rows' whole logits).
+// transposes and stores or reductions overlap the other's; four made the expert
+// down-projection slower), one for the router's top-k (a warp needs its rows' whole logits).
 template <int KIND>
 __host__ __device__ constexpr int epi_split() { return KIND == EPI_TOPK ? 1 : 2; }
 // warp 0: TMA, warp 1: MMA, then 4 x epi_split epilogue warps
@@ -457,9 +458,70 @@ __device__ __forceinline__ void epilogue(const EpiParams& p, const EpiPre& pre, 
             }
         }
     } else if constexpr (KIND == EPI_OPROJ_LOOP) {
-        // y (= x) and h_next (= A (.) h + B.e) were written by RMSNorm1; the attention output
-        // completes both: y = x + a, h_next = A (.) h + B.e + a. Vector atomics need no reads
-        // here, so the epilogue never waits on memory.
+        if (p.h_in) {
+            // y = x + a and h_next = A (.) h + B.e + a, x = h (+ e), from h and e read here
+            // (issued before the chunk's accumulator load); every output is stored once
+            const T* e = static_cast<const T*>(p.e_in);
+            const bool fuse_b = p.b_diag && e;
+#pragma unroll 1
+            for (int c = ch0; c < BN / 32; c += chs) {
+                const int col = n0 + c * 32;
+                if (col >= p.ncols_valid) continue;
+                float hv[8][4], ev[8][4];
+#pragma unroll
+                for (int it = 0; it < 8; ++it) {
+                    const int rr = it * 4 + (lane >> 3);
+                    if (rr >= nvalid) continue;
+                    const size_t off = static_cast<size_t>(row0 + rr) * p.ld + col + cc;
+                    load4(p.h_in + off, hv[it]);
+                    if (e) load4(e + off, ev[it]);
+                    if (!fuse_b) {   // ev holds B.e itself; x = h + e then needs e as well
+                        if (e) {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) hv[it][j] += ev[it][j];   // x
+                        }
+                        load4(p.be + off, ev[it]);
+                    }
+                }
+                float v[32], ad[4], bd[4];
+                ld_chunk(taddr, c, v);
+                stage_put(stg, lane, v);
+                load4(p.a_diag + col + cc, ad);
+                if (fuse_b) load4(p.b_diag + col + cc, bd);
+#pragma unroll
+                for (int it = 0; it < 8; ++it) {
+                    const int rr = it * 4 + (lane >> 3);
+                    float o[4];
+                    stage_get(stg, lane, it, o);
+                    if (rr >= nvalid) continue;
+                    const size_t off = static_cast<size_t>(row0 + rr) * p.ld + col + cc;
+                    float y[4], hn[4];
+                    if (fuse_b) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float h = hv[it][j];
+                            hn[j] = fmaf(ad[j], h, ev[it][j] * bd[j]) + o[j];
+                            y[j] = (h + ev[it][j]) + o[j];
+                        }
+                    } else {
+                        // hv holds x; A (.) h takes h, read again (the line is in L1)
+                        float h[4];
+                        load4(p.h_in + off, h);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            hn[j] = fmaf(ad[j], h[j], ev[it][j]) + o[j];
+                            y[j] = hv[it][j] + o[j];
+                        }
+                    }
+                    store4(p.y + off, y);
+                    store4(p.h_next + off, hn);
+                }
+            }
+            return;
+        }
+        // y and h_next were formed by an earlier O projection (depth attention's: x + d and
+        // A (.) h + B.e + d); a is added into both. Vector atomics need no reads here, so the
+        // epilogue never waits on memory.
 #pragma unroll 1
         for (int c = ch0; c < BN / 32; c += chs) {
             float v[32];

@@ -5,7 +5,7 @@
 //   h_{t+1} = A (.) h_t + B.e + a_t + f_t       (techbriefly article, update equation)
 //
 // per loop t:  norm1 -> QKV(+RoPE, +LoRA) -> attention -> [LoRA-down] -> O-proj fused with
-//              y = x + a and h_next = A h + Be + a -> norm2 + router top-k -> dispatch ->
+//              y = x + a and h_next = A h + B.e + a -> norm2 + router top-k -> dispatch ->
 //              expert up (SwiGLU) -> expert down fused with gate weight and h_next += w E(yn).
 #include <algorithm>
 #include <cmath>
@@ -823,9 +823,20 @@ rdt_status create_impl(const rdt_config* cfg, const rdt_weights* w, cudaStream_t
 
 int lora_index(const rdt_handle* h, int t) { return std::min(t, h->cfg.n_lora - 1); }
 
+// The O-projection epilogue's inputs for y = x + acc and h_next = A (.) h + B.e + acc, x = h
+// (+ e when the block input includes it): a diagonal B is applied to e there, a dense B's
+// product (or B.e when the block input leaves e out) comes from the hoisted Be.
+void set_residual(const rdt_handle* h, const float* hin, const void* e, EpiParams& eo) {
+    eo.h_in = hin;
+    eo.e_in = e;
+    eo.a_diag = h->A;
+    eo.b_diag = h->cfg.b_kind == RDT_B_DIAG && e ? h->Bw : nullptr;
+    eo.be = h->Be;
+}
+
 // ---- depth attention of loop t: RMSNorm_da(x) -> [q; k; v] with the depth rotation -> loop
 // t's keys and values into the token's depth cache -> attention over loops 0 .. t -> output
-// projection adding d into y (= x, written by the same RMSNorm) and h_next (A h + B e)
+// projection forming y = x + d and h_next = A h + B e + d
 rdt_status depth_block(rdt_handle* h, const float* hin, const void* e, int t, float* h_next, cudaStream_t st) {
     const rdt_config& c = h->cfg;
     const int N = h->cur_ntok, d = c.dim;
@@ -839,10 +850,6 @@ rdt_status depth_block(rdt_handle* h, const float* hin, const void* e, int t, fl
     n1.eps = c.norm_eps;
     n1.zero_counts = h->counts;
     n1.n_zero = h->G;
-    n1.y0 = h->y;
-    n1.hn0 = h_next;
-    n1.Be = h->Be;
-    n1.Adiag = h->A;
     TIMED(h, K_NORM1, 1, st, norm1(h->bf, n1, st));
 
     GemmArgs ga{};
@@ -897,6 +904,7 @@ rdt_status depth_block(rdt_handle* h, const float* hin, const void* e, int t, fl
     eo.y = h->y;
     eo.h_next = h_next;
     eo.ld = d;
+    set_residual(h, hin, e, eo);   // y = x + d, h_next = A h + B.e + d
     TIMED(h, K_DA_O, 1, st, gemm_tc(h->bf, 128, h->m_od, h->m_wo_d, nullptr, nullptr, go, eo, st));
     return RDT_OK;
 }
@@ -929,10 +937,6 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
     if (loop_mode && !depth) {          // (the depth block's RMSNorm did this)
         n1.zero_counts = h->counts;
         n1.n_zero = h->G;
-        n1.y0 = h->y;
-        n1.hn0 = h_next;
-        n1.Be = h->Be;
-        n1.Adiag = h->A;
     }
     TIMED(h, K_NORM1, 1, st, norm1(h->bf, n1, st));
 
@@ -1137,6 +1141,9 @@ rdt_status attention_block(rdt_handle* h, const float* hin, const void* e, int t
         eo.y = h->y;
         eo.h_next = h_next;
         eo.ld = d;
+        // without depth attention the O projection forms y and h_next from h and e; after
+        // it, both already hold x + d and A h + B.e + d, and a is added in
+        if (!depth) set_residual(h, hin, e, eo);
     } else {
         eo.kind = EPI_OPROJ_PLAIN;
         eo.out = a_out;
@@ -1317,7 +1324,10 @@ rdt_status loop_impl(rdt_handle* h, const void* h0, const void* e, int T, float*
     const int N = h->cur_ntok, d = c.dim;
     const size_t nd = static_cast<size_t>(N) * d;
     h->cur_T = T;
-    TIMED(h, K_HOIST, 1, st, hoist(h->bf, h0, e, c.b_kind == RDT_B_DIAG ? h->Bw : nullptr, h->hbuf[0], h->Be, nd, d, st));
+    // B.e is only kept for dense B or when the block input leaves e out (the O projection
+    // forms a diagonal B's product from the e it reads)
+    const bool keep_be = c.b_kind == RDT_B_DIAG && !c.inject_e;
+    TIMED(h, K_HOIST, 1, st, hoist(h->bf, h0, e, keep_be ? h->Bw : nullptr, h->hbuf[0], h->Be, nd, d, st));
     if (c.b_kind == RDT_B_DENSE) TIMED(h, K_DENSE_B, 1, st, matmul_nt_simt(h->bf, e, h->Bw, h->Be, N, d, d, st));
     if (h->tr_h) RDT_CUDA_TRY(cudaMemcpyAsync(h->tr_h, h->hbuf[0], nd * 4, cudaMemcpyDeviceToDevice, st));
     for (int t = 0; t < T; ++t) {

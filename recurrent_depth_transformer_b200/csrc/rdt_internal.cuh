@@ -387,7 +387,8 @@ rdt_status make_tmap_2d(CUtensorMap* map, const void* base, bool bf16_elems, uin
 enum EpiKind {
     EPI_STORE = 0,      // C[row, col] = acc                     (OutT)
     EPI_ROPE = 1,       // C = acc with RoPE on the rotary part of rotated heads (OutT)
-    EPI_OPROJ_LOOP = 2, // y += acc, h_next += acc (fp32 vector atomics; both preset by RMSNorm1)
+    EPI_OPROJ_LOOP = 2, // y += acc, h_next += acc (fp32 vector atomics; both preset by RMSNorm1),
+                        // or, given h_in: y = x + acc, h_next = A h + B.e + acc (stores)
     EPI_OPROJ_PLAIN = 3,// a_out = acc                             (fp32)
     EPI_SWIGLU = 4,     // U[row, j] = silu(acc_gate) * acc_up    (OutT)
     EPI_SCATTER = 5,    // dst[token, col] += w * acc             (fp32, vector atomics)
@@ -418,10 +419,17 @@ struct EpiParams {
     // [cp_w]), row (r / seq) * cp_seq_tot + cp_row_off + r % seq
     void* cp_dst[kMaxCp];
     int cp_n, cp_col0, cp_w, cp_seq_tot, cp_row_off;
-    // O-projection loop epilogue: y and h_next hold x and A (.) h + B.e (RMSNorm1 wrote them)
+    // O-projection loop epilogue. Without h_in: y and h_next hold x and A (.) h + B.e
+    // (RMSNorm1 wrote them) and a is added into both. With h_in (no K split): the epilogue
+    // reads h (and e) itself and stores y = x + a, h_next = A (.) h + B.e + a.
     float* y;              // += a   ->  x + a
     float* h_next;         // += a   ->  A*h + Be + a (the MoE adds its share later)
     int ld;                // row stride of y and h_next (= dim)
+    const float* h_in;     // h_t [rows, ld] fp32, or NULL
+    const void* e_in;      // e [rows, ld] (element type) when the block input is h + e, else NULL
+    const float* a_diag;   // A [ld]
+    const float* b_diag;   // diagonal B [ld] (B.e formed from e_in), or NULL: be is read
+    const float* be;       // B.e [rows, ld] fp32 (dense B, or no e in the block input)
     // scatter
     const int* row_token;  // routed rows: token of each output row
     const float* row_w;    // routed rows: gate weight
@@ -522,9 +530,6 @@ struct Norm1Args {
     void* xn;          // [N, dim] cfg dtype
     int ntok, dim; float eps;
     int* zero_counts; int n_zero;   // counts to clear (next MoE), or NULL
-    // loop mode: also write the fp32 block input x into y0 and A (.) h + Be into hn0, which
-    // the O projection then completes with its output a (NULL: not written)
-    float* y0; float* hn0; const float* Be; const float* Adiag;
 };
 rdt_status norm1(bool bf16_elems, const Norm1Args& a, cudaStream_t st);
 

@@ -1,7 +1,7 @@
 // Memory-bound row kernels of the recurrent block (one warp per token row, 16-byte
 // vectorised, coalesced across the warp):
 //   hoist          h <- h0 (fp32 state), Be <- B (.) e      (once per call)
-//   norm1          x = h + e, xn = RMSNorm1(x); in the loop also y <- x, h_next <- A h + B e
+//   norm1          x = h + e, xn = RMSNorm1(x)
 //   norm2_router   yn = RMSNorm2(y) (fp32 in registers, stored in the element type for the
 //                  experts), router logits yn W_r^T in fp32, top-k of logits + bias with
 //                  ties to the lower expert index, softmax over the k chosen logits,
@@ -90,45 +90,29 @@ __global__ void __launch_bounds__(kRowThreads, NV <= 8 ? 2 : 1) norm1_kernel(con
 #pragma unroll
         for (int i = 0; i < NV; ++i) load4(a.gamma + i * 128 + lane * 4, g[i]);
     }
-    // Groups of up to 4 vectors: every load of a group is issued before its stores (which
-    // could alias the loads as far as the compiler knows, and would serialise them).
-    constexpr int GV = NV < 4 ? NV : 4;
 #pragma unroll
-    for (int i0 = 0; i0 < NV; i0 += GV) {
-        float ev[GV][4], be[GV][4], ad[GV][4];
+    for (int i = 0; i < NV; ++i) {
+        const int col = i * 128 + lane * 4;
+        if (a.h) {
+            load4(a.h + base + col, x[i]);
+        } else {
 #pragma unroll
-        for (int i = 0; i < GV; ++i) {
-            const int col = (i0 + i) * 128 + lane * 4;
-            if (a.h) {
-                load4(a.h + base + col, x[i0 + i]);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) x[i0 + i][j] = 0.0f;
-            }
-            if (e) load4(e + base + col, ev[i]);
-            if (a.hn0) {
-                load4(a.Be + base + col, be[i]);
-                load4(a.Adiag + col, ad[i]);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < GV; ++i) {
-            const int col = (i0 + i) * 128 + lane * 4;
-            if (a.hn0) {   // A (.) h + B.e, the part of h_next the O projection and the MoE complete
-                float hn[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) hn[j] = fmaf(ad[i][j], x[i0 + i][j], be[i][j]);
-                store4(a.hn0 + base + col, hn);
-            }
-            if (e) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) x[i0 + i][j] += ev[i][j];
-            }
-            if (a.y0) store4(a.y0 + base + col, x[i0 + i]);   // the block input x, completed to x + a
-#pragma unroll
-            for (int j = 0; j < 4; ++j) ss = fmaf(x[i0 + i][j], x[i0 + i][j], ss);
+            for (int j = 0; j < 4; ++j) x[i][j] = 0.0f;
         }
     }
+    if (e) {
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            float ev[4];
+            load4(e + base + i * 128 + lane * 4, ev);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) x[i][j] += ev[j];
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ss = fmaf(x[i][j], x[i][j], ss);
     ss = warp_sum(ss);
     const float inv = rsqrtf(ss / a.dim + a.eps);
     T* xn = static_cast<T*>(a.xn) + base;
