@@ -177,4 +177,5 @@ def test_roofline_of_a_tensor_and_an_hbm_kernel():
     assert r["frac"] == pytest.approx(r["achieved"] / 1000.0)
     r = bench.roofline_of("norm1", 2, 0.1, work, peaks, "measured", bench.WORKLOAD)
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
-    assert r["achieved"] == pytest.approx(8192 * 2048 * 20 / 50e-6 / 1e9)
+    # RMSNorm1: h (fp32) and e (bf16) in, xn (bf16) out: 8 bytes per element
+    assert r["achieved"] == pytest.approx(8192 * 2048 * 8 / 50e-6 / 1e9)
