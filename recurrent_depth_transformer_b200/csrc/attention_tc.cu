@@ -472,9 +472,11 @@ __global__ void __launch_bounds__(AttnCfg<DQK, DV, SHARE_KV, QT>::THREADS,
 // the buffer that PV_t(j) has just read (the MMAs of one thread execute in issue order).
 // The K and V of a block share one shared-memory stage, released after the block's last PV.
 
-// Pairs of probabilities, out of every 8, whose exponentials run on the FMA pipe instead of
-// the MUFU (measured at 8192 positions: 0 -> 413 us, 2 -> 371 us, 3 -> 369 us, 4 -> 379 us).
-constexpr int kPolyOf8 = 2;
+// Pairs of probabilities, out of the NV / 2 = 24 of a softmax thread's block, whose
+// exponentials run on the FMA pipe instead of the MUFU (measured at 8192 positions with two
+// softmax warps per row: 0 -> 369 us, 1 -> 360, 2 -> 358, 3 -> 361, 4 -> 363, 6 -> 374;
+// with one warp per row, 24 of 96: 371 us against 413 with none).
+constexpr int kPolyPairs = 2;
 
 
 // Softmax warps per query row: 2 splits every block's 96 keys between two warps of the same
@@ -775,9 +777,9 @@ __global__ void __launch_bounds__(K96Cfg<QT>::THREADS, K96Cfg<QT>::BLOCKS_PER_SM
             for (int c = 0; c < NV / 2; ++c) {
                 const float2 x = __ffma2_rn(make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])),
                                             slv, mneg);
-                // kPolyOf8 pairs in every 8 on the FMA pipe, the rest on the MUFU
+                // kPolyPairs of the NV / 2 pairs on the FMA pipe, evenly spaced; the rest on the MUFU
                 float2 pp;
-                if ((c * kPolyOf8) / 8 != ((c + 1) * kPolyOf8) / 8) {
+                if ((c * kPolyPairs) / (NV / 2) != ((c + 1) * kPolyPairs) / (NV / 2)) {
                     pp = exp2_poly2(x);
                 } else {
                     pp = make_float2(exp2_ftz(x.x), exp2_ftz(x.y));
