@@ -72,59 +72,86 @@ __global__ void matmul_nt_kernel(const T* A, const float* B, float* C, int M, in
 
 // ----------------------------------------------------------------------------- norm1
 
+// Wide rows are split over WR warps (each lane then holds PV = NV / WR vectors of 4): a row
+// of 2048 elements held by one warp took 138 registers a thread, one block per SM, and the
+// norms ran at a quarter of the HBM bandwidth. Warp w of a row takes the vectors
+// (i WR + w) 128 + 4 lane, so each warp-wide access still covers one contiguous segment; the
+// row's sum of squares is the WR warps' partial sums added in warp order.
+template <int NV>
+struct RowSplit {
+    static constexpr int WR = NV >= 8 ? NV / 4 : 1;        // warps per row
+    static constexpr int PV = NV / WR;                      // vectors of 4 per lane
+    static constexpr int ROWS = (kRowThreads / 32) / WR;    // rows per block
+    static_assert(WR * PV == NV && ROWS >= 1, "row split");
+};
+
+// Sum over the WR warps of a row (every thread of the block must call it: it synchronises
+// the block when WR > 1).
+template <int WR>
+__device__ __forceinline__ float row_sum(float v, float* part) {
+    v = warp_sum(v);
+    if constexpr (WR > 1) {
+        const int warp = threadIdx.x >> 5;
+        if ((threadIdx.x & 31) == 0) part[warp] = v;
+        __syncthreads();
+        const int w0 = warp / WR * WR;
+        v = 0.0f;
+#pragma unroll
+        for (int w = 0; w < WR; ++w) v += part[w0 + w];
+    }
+    return v;
+}
+
 template <typename T, int NV>
-__global__ void __launch_bounds__(kRowThreads, NV <= 8 ? 2 : 1) norm1_kernel(const Norm1Args a) {
+__global__ void __launch_bounds__(kRowThreads) norm1_kernel(const Norm1Args a) {
+    using RS = RowSplit<NV>;
+    constexpr int PV = RS::PV;
+    __shared__ float part[kRowThreads / 32];
     pdl_trigger();
     pdl_wait();
     if (blockIdx.x == 0 && a.zero_counts)
         for (int i = threadIdx.x; i < a.n_zero; i += blockDim.x) a.zero_counts[i] = 0;
-    const int row = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+    const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    if (row >= a.ntok) return;
-    const size_t base = static_cast<size_t>(row) * a.dim;
+    const int row = blockIdx.x * RS::ROWS + warp / RS::WR;
+    const int wr = warp % RS::WR;
+    const bool live = row < a.ntok;
+    const size_t base = static_cast<size_t>(live ? row : 0) * a.dim;
     const T* e = static_cast<const T*>(a.e);
-    constexpr bool kHoistG = NV <= 8;          // gamma in flight with the row, registers allowing
-    float x[NV][4], g[kHoistG ? NV : 1][4];
+    float x[PV][4];
     float ss = 0.0f;
-    if constexpr (kHoistG) {
 #pragma unroll
-        for (int i = 0; i < NV; ++i) load4(a.gamma + i * 128 + lane * 4, g[i]);
-    }
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        const int col = i * 128 + lane * 4;
-        if (a.h) {
+    for (int i = 0; i < PV; ++i) {
+        const int col = (i * RS::WR + wr) * 128 + lane * 4;
+        if (a.h && live) {
             load4(a.h + base + col, x[i]);
         } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j) x[i][j] = 0.0f;
         }
     }
-    if (e) {
+    if (e && live) {
 #pragma unroll
-        for (int i = 0; i < NV; ++i) {
+        for (int i = 0; i < PV; ++i) {
             float ev[4];
-            load4(e + base + i * 128 + lane * 4, ev);
+            load4(e + base + (i * RS::WR + wr) * 128 + lane * 4, ev);
 #pragma unroll
             for (int j = 0; j < 4; ++j) x[i][j] += ev[j];
         }
     }
 #pragma unroll
-    for (int i = 0; i < NV; ++i)
+    for (int i = 0; i < PV; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) ss = fmaf(x[i][j], x[i][j], ss);
-    ss = warp_sum(ss);
+    ss = row_sum<RS::WR>(ss, part);
+    if (!live) return;
     const float inv = rsqrtf(ss / a.dim + a.eps);
     T* xn = static_cast<T*>(a.xn) + base;
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        const int col = i * 128 + lane * 4;
+    for (int i = 0; i < PV; ++i) {
+        const int col = (i * RS::WR + wr) * 128 + lane * 4;
         float gi[4];
-        if constexpr (kHoistG) {
-            gi[0] = g[i][0]; gi[1] = g[i][1]; gi[2] = g[i][2]; gi[3] = g[i][3];
-        } else {
-            load4(a.gamma + col, gi);
-        }
+        load4(a.gamma + col, gi);
 #pragma unroll
         for (int j = 0; j < 4; ++j) x[i][j] = to_f(from_f<T>(x[i][j] * inv * gi[j]));
         store4(xn + col, x[i]);
@@ -275,29 +302,41 @@ __device__ __forceinline__ void split_hi_lo(float v, float& hi, float& lo) {
 
 template <typename T, int NV>
 __global__ void __launch_bounds__(kRowThreads) norm2_split_kernel(const Norm2Args a) {
+    using RS = RowSplit<NV>;
+    constexpr int PV = RS::PV;
+    __shared__ float part[kRowThreads / 32];
     pdl_trigger();
     pdl_wait();
-    const int row = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+    const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    if (row >= a.ntok) return;
-    const size_t base = static_cast<size_t>(row) * a.dim;
-    float y[NV][4];
+    const int row = blockIdx.x * RS::ROWS + warp / RS::WR;
+    const int wr = warp % RS::WR;
+    const bool live = row < a.ntok;
+    const size_t base = static_cast<size_t>(live ? row : 0) * a.dim;
+    float y[PV][4];
     float ss = 0.0f;
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        load4(a.y + base + i * 128 + lane * 4, y[i]);
+    for (int i = 0; i < PV; ++i) {
+        if (live) {
+            load4(a.y + base + (i * RS::WR + wr) * 128 + lane * 4, y[i]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) y[i][j] = 0.0f;
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j) ss = fmaf(y[i][j], y[i][j], ss);
     }
-    ss = warp_sum(ss);
+    ss = row_sum<RS::WR>(ss, part);
+    if (!live) return;
     const float inv = rsqrtf(ss / a.dim + a.eps);
     if (a.zero_rows)
-        for (int i = lane; i < a.zero_width; i += 32) a.zero_rows[static_cast<size_t>(row) * a.zero_width + i] = 0.0f;
+        for (int i = wr * 32 + lane; i < a.zero_width; i += RS::WR * 32)
+            a.zero_rows[static_cast<size_t>(row) * a.zero_width + i] = 0.0f;
     T* yn = static_cast<T*>(a.yn) + base;
     T* lo = static_cast<T*>(a.yn_lo) + base;
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        const int col = i * 128 + lane * 4;
+    for (int i = 0; i < PV; ++i) {
+        const int col = (i * RS::WR + wr) * 128 + lane * 4;
         float g[4], hv[4], lv[4];
         load4(a.gamma + col, g);
 #pragma unroll
@@ -314,32 +353,33 @@ __global__ void __launch_bounds__(kRowThreads) norm2_split_kernel(const Norm2Arg
 
 // ----------------------------------------------------------------------------- MoE dispatch copy
 
-// One warp per (token, slot): copy the normalised row yn[token] into the row the router
-// claimed for it (capacity layout).
+// One warp per token: the normalised row yn[token] is read once (eight 16-byte vectors of the
+// lane in flight) and stored into each row the router claimed for it (capacity layout). A
+// warp per (token, slot) re-read the row k times from L2 and ran at ~4.6 TB/s of stores.
 template <typename T>
 __global__ void __launch_bounds__(kRowThreads) moe_copy_kernel(T* xperm, const int* slot_row, int ntok,
                                                                int top_k, int dim, int a_routed_base) {
     pdl_trigger();
     pdl_wait();
-    const int ws = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+    const int n = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (ws >= ntok * top_k) return;
-    const int n = ws / top_k;
-    if (slot_row[ws] < 0) return;                 // halted token: no row claimed
-    const int r = a_routed_base + slot_row[ws];
+    if (n >= ntok) return;
     const uint4* src = reinterpret_cast<const uint4*>(xperm + static_cast<size_t>(n) * dim);
-    uint4* dst = reinterpret_cast<uint4*>(xperm + static_cast<size_t>(r) * dim);
     const int nvec = dim * static_cast<int>(sizeof(T)) / 16;
-    // eight 16-byte loads of the lane in flight before its stores (one at a time left the
-    // copy at ~4 TB/s, bound by the loads' L2 latency)
     for (int i0 = lane; i0 < nvec; i0 += 8 * 32) {
         uint4 t[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u)
             if (i0 + 32 * u < nvec) t[u] = src[i0 + 32 * u];
+#pragma unroll 1
+        for (int s = 0; s < top_k; ++s) {
+            const int sr = slot_row[static_cast<size_t>(n) * top_k + s];
+            if (sr < 0) continue;                 // halted token: no row claimed
+            uint4* dst = reinterpret_cast<uint4*>(xperm + static_cast<size_t>(a_routed_base + sr) * dim);
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-            if (i0 + 32 * u < nvec) dst[i0 + 32 * u] = t[u];
+            for (int u = 0; u < 8; ++u)
+                if (i0 + 32 * u < nvec) dst[i0 + 32 * u] = t[u];
+        }
     }
 }
 
@@ -513,7 +553,8 @@ rdt_status launch_rows(int nv, int rows, cudaStream_t st, Args... args) {
 
 template <typename T, int NV>
 struct Norm1L {
-    static void run(dim3 g, cudaStream_t st, Norm1Args a) {
+    static void run(dim3, cudaStream_t st, Norm1Args a) {
+        const dim3 g((a.ntok + RowSplit<NV>::ROWS - 1) / RowSplit<NV>::ROWS);
         launch_pdl(norm1_kernel<T, NV>, g, dim3(kRowThreads), 0, st, a);
     }
 };
@@ -533,7 +574,8 @@ struct CombineL {
 };
 template <typename T, int NV>
 struct Norm2L {
-    static void run(dim3 g, cudaStream_t st, Norm2Args a) {
+    static void run(dim3, cudaStream_t st, Norm2Args a) {
+        const dim3 g((a.ntok + RowSplit<NV>::ROWS - 1) / RowSplit<NV>::ROWS);
         launch_pdl(norm2_split_kernel<T, NV>, g, dim3(kRowThreads), 0, st, a);
     }
 };
@@ -596,8 +638,7 @@ rdt_status norm2_router(bool bf, const RouterArgs& a, cudaStream_t st) {
 
 rdt_status moe_copy(bool bf, void* xperm, const int* slot_row, int ntok, int top_k, int dim,
                     int a_routed_base, cudaStream_t st) {
-    const int warps = ntok * top_k;
-    const dim3 grid((warps + kRowThreads / 32 - 1) / (kRowThreads / 32));
+    const dim3 grid((ntok + kRowThreads / 32 - 1) / (kRowThreads / 32));
     if (bf)
         RDT_CUDA_TRY(launch_pdl(moe_copy_kernel<bf16>, grid, dim3(kRowThreads), 0, st, static_cast<bf16*>(xperm),
                                 slot_row, ntok, top_k, dim, a_routed_base));
