@@ -16,10 +16,10 @@ def torch_mod():
     return torch
 
 
-def handle(wl: Workload, inputs, max_loops: int = 16, gemm_tiles: int = 0):
+def handle(wl: Workload, inputs, max_loops: int = 16, gemm_tiles: int = 0, deterministic: bool = False):
     import recurrent_depth_transformer_b200 as R
     w = R.device_weights(inputs, wl.dtype == "bf16")
-    return R.RDT(R.make_config(wl, max_loops=max_loops, gemm_tiles=gemm_tiles), w)
+    return R.RDT(R.make_config(wl, max_loops=max_loops, gemm_tiles=gemm_tiles, deterministic=deterministic), w)
 
 
 def act(wl: Workload, arr):

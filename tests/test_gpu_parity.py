@@ -209,17 +209,19 @@ def test_causality_and_batch_independence():
 
 
 def test_host_entry_matches_device_entry():
+    # deterministic mode: the host entry runs the same kernels on the same data, so the two
+    # results agree bit for bit (in the default mode the fp32 atomics' order moves the last
+    # bits, ~1e-3 after three loops)
     torch = torch_mod()
     wl = C1.replace(batch=1, seq=128)
     inputs = generate(wl)
-    with handle(wl, inputs) as h:
+    with handle(wl, inputs, deterministic=True) as h:
         e = act(wl, inputs["e"])
         dev = h.loop_forward(e, e, 3).cpu()
         eh = e.cpu().pin_memory()
         out = torch.empty(dev.shape, dtype=torch.float32).pin_memory()
         h.loop_forward_host(eh, eh, 3, out)
-    ma, _ = errors(out.numpy(), dev.numpy())
-    assert ma < 1e-3
+    assert np.array_equal(out.numpy(), dev.numpy())
 
 
 def sampled_rows(wl, seed, per_batch_min=8, total_min=32):
