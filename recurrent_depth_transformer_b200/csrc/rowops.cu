@@ -28,10 +28,12 @@ __device__ __forceinline__ void store_t(T* p, float v) { *p = from_f<T>(v); }
 // ----------------------------------------------------------------------------- hoist
 
 template <typename T>
-__global__ void hoist_kernel(const T* h0, const T* e, const float* Bd, float* h, float* Be,
-                             size_t n4, int dim) {
+__global__ void hoist_kernel(const T* __restrict__ h0, const T* __restrict__ e, const float* __restrict__ Bd,
+                             float* __restrict__ h, float* __restrict__ Be, size_t n4, int dim) {
     pdl_trigger();
     pdl_wait();
+    // (restrict: the unrolled iterations' loads may be issued before the earlier stores)
+#pragma unroll 4
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
          i += static_cast<size_t>(gridDim.x) * blockDim.x) {
         const size_t off = i * 4;
@@ -525,13 +527,26 @@ __global__ void __launch_bounds__(kRowThreads) act_step_kernel(const ActArgs a) 
     }
 }
 
-__global__ void check_finite_kernel(const float* x, size_t n, int* flags) {
+// 16-byte loads, four of a thread in flight (one 4-byte load at a time left it at a third of
+// the HBM bandwidth); scalar loads for a misaligned start and the tail.
+__global__ void check_finite_kernel(const float* __restrict__ x, size_t n, int* flags) {
     pdl_trigger();
     pdl_wait();
     bool bad = false;
-    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
-         i += static_cast<size_t>(gridDim.x) * blockDim.x)
-        bad |= !isfinite(x[i]);
+    const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+    const size_t tid = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+    size_t tail = 0;
+    if ((reinterpret_cast<uintptr_t>(x) & 15) == 0) {
+        const float4* x4 = reinterpret_cast<const float4*>(x);
+        const size_t n4 = n / 4;
+#pragma unroll 4
+        for (size_t i = tid; i < n4; i += stride) {
+            const float4 v = x4[i];
+            bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
+        }
+        tail = n4 * 4;
+    }
+    for (size_t i = tail + tid; i < n; i += stride) bad |= !isfinite(x[i]);
     if (__syncthreads_or(bad) && threadIdx.x == 0) atomicExch(flags + FLAG_NONFINITE, 1);
 }
 
