@@ -172,21 +172,24 @@ struct TopK {
         }
     }
     // Branch-free: the list stays sorted by score (entries past top_k are the runners-up).
+    // The candidate goes to the first slot whose score it beats (strictly: of equal scores
+    // the earlier expert stays ahead) and the slots after it shift down by one. Every slot's
+    // new entry follows from the old list and the comparisons alone, so the slots update in
+    // parallel rather than as a chain through the list.
     __device__ __forceinline__ void insert(float logit, float bias, int ex) {
-        float cs = logit + bias, cl = logit;
-        int ci = ex;
+        const float cs = logit + bias;
+        bool c[KMAX];
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            const bool sw = cs > bs[j];
-            const float ts = bs[j], tl = bl[j];
-            const int ti = bi[j];
-            bs[j] = sw ? cs : ts;
-            bl[j] = sw ? cl : tl;
-            bi[j] = sw ? ci : ti;
-            cs = sw ? ts : cs;
-            cl = sw ? tl : cl;
-            ci = sw ? ti : ci;
+        for (int j = 0; j < KMAX; ++j) c[j] = cs > bs[j];
+#pragma unroll
+        for (int j = KMAX - 1; j > 0; --j) {         // downwards: slot j - 1 is still the old one
+            bs[j] = c[j] ? (c[j - 1] ? bs[j - 1] : cs) : bs[j];
+            bl[j] = c[j] ? (c[j - 1] ? bl[j - 1] : logit) : bl[j];
+            bi[j] = c[j] ? (c[j - 1] ? bi[j - 1] : ex) : bi[j];
         }
+        bs[0] = c[0] ? cs : bs[0];
+        bl[0] = c[0] ? logit : bl[0];
+        bi[0] = c[0] ? ex : bi[0];
     }
     // four consecutive experts ex0 .. ex0 + 3, those from n on left out
     __device__ __forceinline__ void insert4(const float (&x)[4], const float* bias, int ex0, int n) {
@@ -330,7 +333,8 @@ __device__ __forceinline__ void epilogue_topk(const EpiParams& p, uint32_t taddr
     if (!__shfl_sync(0xffffffffu, last, 0)) return;
     __threadfence();
     // the complete row from L2, four logits per step, the next two loads in flight
-    // (n_exp is a multiple of 4: 16-byte pieces)
+    // (n_exp is a multiple of 4: 16-byte pieces; a loop over eight loads at a time, unrolled,
+    // measured slower: its code no longer stays in the instruction cache)
     TopK<KMAX> tk;
     if (valid) {
         const float4* row4 = reinterpret_cast<const float4*>(lrow);
