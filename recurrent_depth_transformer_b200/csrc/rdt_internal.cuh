@@ -387,8 +387,9 @@ rdt_status make_tmap_2d(CUtensorMap* map, const void* base, bool bf16_elems, uin
 enum EpiKind {
     EPI_STORE = 0,      // C[row, col] = acc                     (OutT)
     EPI_ROPE = 1,       // C = acc with RoPE on the rotary part of rotated heads (OutT)
-    EPI_OPROJ_LOOP = 2, // y += acc, h_next += acc (fp32 vector atomics; both preset by RMSNorm1),
-                        // or, given h_in: y = x + acc, h_next = A h + B.e + acc (stores)
+    EPI_OPROJ_LOOP = 2, // given h_in: y = x + acc, h_next = A h + B.e + acc (stores); without:
+                        // y += acc, h_next += acc (fp32 vector atomics, into an earlier O
+                        // projection's y and h_next: after depth attention)
     EPI_OPROJ_PLAIN = 3,// a_out = acc                             (fp32)
     EPI_SWIGLU = 4,     // U[row, j] = silu(acc_gate) * acc_up    (OutT)
     EPI_SCATTER = 5,    // dst[token, col] += w * acc             (fp32, vector atomics)
@@ -419,9 +420,10 @@ struct EpiParams {
     // [cp_w]), row (r / seq) * cp_seq_tot + cp_row_off + r % seq
     void* cp_dst[kMaxCp];
     int cp_n, cp_col0, cp_w, cp_seq_tot, cp_row_off;
-    // O-projection loop epilogue. Without h_in: y and h_next hold x and A (.) h + B.e
-    // (RMSNorm1 wrote them) and a is added into both. With h_in (no K split): the epilogue
-    // reads h (and e) itself and stores y = x + a, h_next = A (.) h + B.e + a.
+    // O-projection loop epilogue. With h_in (no K split): the epilogue reads h (and e) itself
+    // and stores y = x + a, h_next = A (.) h + B.e + a. Without h_in: y and h_next already
+    // hold x + d and A (.) h + B.e + d (the depth-attention O projection formed them) and a
+    // is added into both.
     float* y;              // += a   ->  x + a
     float* h_next;         // += a   ->  A*h + Be + a (the MoE adds its share later)
     int ld;                // row stride of y and h_next (= dim)
