@@ -424,8 +424,8 @@ struct EpiParams {
     // and stores y = x + a, h_next = A (.) h + B.e + a. Without h_in: y and h_next already
     // hold x + d and A (.) h + B.e + d (the depth-attention O projection formed them) and a
     // is added into both.
-    float* y;              // += a   ->  x + a
-    float* h_next;         // += a   ->  A*h + Be + a (the MoE adds its share later)
+    float* y;              // x + a (stored, or += a)
+    float* h_next;         // A*h + Be + a (stored, or += a); the MoE adds its share later
     int ld;                // row stride of y and h_next (= dim)
     const float* h_in;     // h_t [rows, ld] fp32, or NULL
     const void* e_in;      // e [rows, ld] (element type) when the block input is h + e, else NULL
