@@ -44,6 +44,22 @@ def test_loop_matches_oracle_small(name):
     assert_close(got, want, what=name)
 
 
+@pytest.mark.parametrize("name", ["gqa-s200", "tiny-f32", "long-lora-s320"])
+def test_block_input_without_e_matches_oracle(name):
+    """inject_e = 0: the block input is h alone (x = h) while B.e still enters the update.
+    RMSNorm1 reads no e; the O projection's epilogue takes B.e from the hoist (a diagonal B
+    is not applied to e there) or, for the dense B of the fp32 configuration, from the
+    once-per-call product."""
+    wl = SMALL[name].replace(inject_e=False)
+    inputs = generate(wl)
+    T = _loops(name)
+    got, idx, _, _, diag = run_loop(wl, inputs, T)
+    assert diag["nonfinite"] == 0 and diag["timeout"] == 0
+    want, mism, _, _ = oracle_follow(wl, inputs, T, idx)
+    assert mism == 0, f"{mism} routing differences outside near-ties"
+    assert_close(got, want, what=f"{name} without e in the block input")
+
+
 @pytest.mark.parametrize("tiles", [1, 2])
 @pytest.mark.parametrize("name", ["gqa-s200", "mla-s136", "widemoe-s192", "long-lora-s320"])
 def test_gemm_tile_modes_match_oracle(name, tiles):
