@@ -179,3 +179,27 @@ def test_roofline_of_a_tensor_and_an_hbm_kernel():
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
     # RMSNorm1: h (fp32) and e (bf16) in, xn (bf16) out: 8 bytes per element
     assert r["achieved"] == pytest.approx(8192 * 2048 * 8 / 50e-6 / 1e9)
+
+
+def test_state_traffic_of_the_o_projection_and_the_hoist():
+    """The O projection forms y and h_next from h and e (reads h 4 B and e 2 B, stores 2 x 4 B
+    per element); after depth attention it adds into them instead (2 x 4 B of reductions).
+    The hoist stores B.e only where the O projection cannot form it (no e in the block
+    input); with a dense B the product comes from a separate matmul."""
+    from workloads import DEPTH_WORKLOAD
+    wl = WORKLOADS[4]                                     # long: diagonal B, e injected
+    N, d = wl.batch * wl.seq, wl.dim
+    nq = wl.n_heads * wl.head_dim
+    w = bench.kernel_work(wl)
+    assert w["gemm_o"]["bytes"] == 2 * (N * nq + d * nq) + N * d * (4 + 2 + 4 + 4)
+    assert w["norm1"]["bytes"] == N * d * (4 + 2 + 2)
+    assert w["hoist"]["bytes"] == N * d * (2 + 4)
+    w0 = bench.kernel_work(wl.replace(inject_e=False))   # B.e kept by the hoist, read by O
+    assert w0["gemm_o"]["bytes"] == 2 * (N * nq + d * nq) + N * d * (4 + 4 + 4 + 4)
+    assert w0["hoist"]["bytes"] == N * d * (2 + 4 + 2 + 4)
+    wd = bench.kernel_work(DEPTH_WORKLOAD)
+    Nd, dd = DEPTH_WORKLOAD.batch * DEPTH_WORKLOAD.seq, DEPTH_WORKLOAD.dim
+    nqd = DEPTH_WORKLOAD.n_heads * DEPTH_WORKLOAD.head_dim
+    assert wd["gemm_o"]["bytes"] == 2 * (Nd * nqd + dd * nqd) + 4 * 2 * Nd * dd
+    nqd_da = DEPTH_WORKLOAD.da_heads * DEPTH_WORKLOAD.head_dim
+    assert wd["gemm_o_depth"]["bytes"] == 2 * (Nd * nqd_da + dd * nqd_da) + Nd * dd * (4 + 2 + 4 + 4)
